@@ -1,0 +1,367 @@
+"""Float64 CPU oracle for reduced-KV softmax decode attention.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path imports, calls or runs this
+module; only the tests, the smoke check and the benchmark's CPU-baseline leg do.
+It shares no code with the CUDA path: it is plain NumPy in float64, written step by
+step from the pages, with no blocking, fusion or reordering beyond what each
+definition states.
+
+Sources (page title, then section / equation):
+  [COBS]  "COBS: Cumulant Order Block Sparse Attention" -- block masses and block
+          probabilities (Equation 1 and the text around it), the per-KV-head GQA
+          score (Equation 5 and the normaliser Z^(g,h) of (5)), the first-order
+          mean-pool score (affine score (18): phi_b = mean key, a_b = ln L), OSA
+          exact-mass ranking (the OSA paragraph).
+  [OA]    "OpenAttention reads 1% of the KV cache -- Count-aware tail proxy",
+          section "Skipping reviews without losing the verdict" (the proxy token)
+          and section "A worked example with named numbers".
+  [WC]    "WildCat: Near-Linear Attention in Theory and Practice", abstract
+          (attention over a small weighted coreset).
+
+Readings where the pages are silent or garbled (each is also listed in the design
+notes of the repository):
+  R1  The GQA group score is the sum over the group's query heads of per-head
+      block softmax probabilities, normalised over all valid blocks (forced ones
+      included).
+  R2  The count term is the natural log of the block's actual token count n_b
+      (ln L for full blocks).
+  R3  Logits are sigma * q.k with sigma passed in (1/sqrt(D), or 1 when q is
+      already scaled).
+  R4  Query head g reads KV head floor(g / G).
+  R5  Forced blocks (first and/or last) do not compete and do not count toward k.
+  R6  Ties are broken by lowest block index.
+  R7  The proxy logit is sigma * q . (mean tail key) + ln n_T, which equals the
+      mean tail logit plus ln n_T by linearity; with an empty tail there is no
+      proxy.
+  R8  Weighted mode: logit + ln w_i, no proxy; w_i = 0 excludes the token.
+  R9  An empty softmax (no token, no proxy) gives out = 0 and lse = -inf.
+  R10 Near tie: (S_(k) - S_(k+1)) / S_(k) < 1e-3 between the k-th and (k+1)-th
+      candidate scores.
+"""
+from __future__ import annotations
+
+import math
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+NEAR_TIE_REL = 1e-3
+
+
+# --------------------------------------------------------------------------- blocks
+def blocks_of(n: int, L: int) -> List[Tuple[int, int]]:
+    """Contiguous blocks of L tokens over [0, n); the last one may be short."""
+    return [(s, min(s + L, n)) for s in range(0, n, L)]
+
+
+def block_summaries_one(K: np.ndarray, V: np.ndarray, n: int, L: int, NBcap: int):
+    """Per-block key sum, value sum and token count for one (sequence, KV head),
+    plus whole-sequence totals. The mean key k_sum/n_b is the mean-pool summary
+    [COBS, affine score (18)]; the sums feed the tail proxy [OA].
+
+    K, V: [Ncap][D] float64. Returns k_sum, v_sum [NBcap][D], counts [NBcap],
+    k_tot, v_tot [D]. Blocks at or beyond ceil(n/L) are zero with count 0.
+    """
+    D = K.shape[1]
+    k_sum = np.zeros((NBcap, D))
+    v_sum = np.zeros((NBcap, D))
+    counts = np.zeros(NBcap, dtype=np.int64)
+    for b, (s, e) in enumerate(blocks_of(n, L)):
+        k_sum[b] = K[s:e].sum(axis=0)
+        v_sum[b] = V[s:e].sum(axis=0)
+        counts[b] = e - s
+    return k_sum, v_sum, counts, K[:n].sum(axis=0), V[:n].sum(axis=0)
+
+
+def build_block_summaries(K, V, seq_lens, L):
+    """Batched block summaries. K, V: [B][Hkv][Ncap][D] float64."""
+    B, Hkv, Ncap, D = K.shape
+    NBcap = (Ncap + L - 1) // L
+    k_sum = np.zeros((B, Hkv, NBcap, D))
+    v_sum = np.zeros((B, Hkv, NBcap, D))
+    counts = np.zeros((B, NBcap), dtype=np.int64)
+    k_tot = np.zeros((B, Hkv, D))
+    v_tot = np.zeros((B, Hkv, D))
+    for b in range(B):
+        for h in range(Hkv):
+            ks, vs, c, kt, vt = block_summaries_one(K[b, h], V[b, h], int(seq_lens[b]), L, NBcap)
+            k_sum[b, h], v_sum[b, h], k_tot[b, h], v_tot[b, h] = ks, vs, kt, vt
+            counts[b] = c
+    return k_sum, v_sum, counts, k_tot, v_tot
+
+
+# --------------------------------------------------------------------------- scores
+def logsumexp(x: np.ndarray) -> float:
+    """ln sum exp(x) with a max shift; -inf for an empty or all -inf input."""
+    x = np.asarray(x, dtype=np.float64)
+    if x.size == 0:
+        return -math.inf
+    m = np.max(x)
+    if m == -math.inf:
+        return -math.inf
+    return float(m + math.log(np.sum(np.exp(x - m))))
+
+
+def summary_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, sigma: float):
+    """First-order mean-pool estimate of the block log-mass [COBS, text after
+    Equation (8): the first-order term is a mean-pool; affine score (18) with
+    phi_b = mean key, a_b = ln L; reading R2 uses ln n_b]:
+
+        s_hat[g, b] = sigma * q_g . (k_sum_b / n_b) + ln n_b
+
+    qg: [G][D]; k_sum: [NB][D]; counts: [NB]. Blocks with n_b = 0 get -inf.
+    """
+    G = qg.shape[0]
+    NB = k_sum.shape[0]
+    out = np.full((G, NB), -math.inf)
+    for b in range(NB):
+        nb = int(counts[b])
+        if nb <= 0:
+            continue
+        mean_key = k_sum[b] / nb
+        out[:, b] = sigma * (qg @ mean_key) + math.log(nb)
+    return out
+
+
+def exact_log_mass(qg: np.ndarray, K: np.ndarray, n: int, L: int, NB: int, sigma: float):
+    """Exact block log-mass ln m_b = ln sum_{r in b} exp(sigma q.k_r), the quantity
+    OSA ranks by [COBS, OSA paragraph; block mass m_b of Equation 1].
+
+    qg: [G][D]; K: [Ncap][D]. Returns [G][NB] with -inf for empty blocks.
+    """
+    G = qg.shape[0]
+    out = np.full((G, NB), -math.inf)
+    for b, (s, e) in enumerate(blocks_of(n, L)):
+        logits = sigma * (K[s:e] @ qg.T)          # [e-s][G]
+        for g in range(G):
+            out[g, b] = logsumexp(logits[:, g])
+    return out
+
+
+def group_score(shat: np.ndarray) -> np.ndarray:
+    """GQA-normalised group score [COBS, Equation (5) and its normaliser Z^(g,h);
+    reading R1]: S_b = sum_g exp(s_hat[g,b] - ln sum_b' exp(s_hat[g,b'])), i.e. the
+    sum of the group's per-head block softmax probabilities.
+    """
+    G, NB = shat.shape
+    S = np.zeros(NB)
+    for g in range(G):
+        lse = logsumexp(shat[g])
+        if lse == -math.inf:
+            continue
+        S += np.exp(shat[g] - lse)
+    return S
+
+
+def select_blocks(S: np.ndarray, valid_nb: int, k: int, force_first: bool,
+                  force_last: bool) -> Dict:
+    """Top-k block choice per KV head [COBS: "maximized by the top-k blocks under"
+    (5); readings R5, R6, R10].
+
+    Forced blocks (first = 0, last = valid_nb - 1) are kept and do not compete.
+    The others are ordered by (S descending, block index ascending) and the first
+    min(k, |C|) are kept. Returns kept (ascending), the candidate order, and the
+    near-tie flag at the k / k+1 boundary.
+    """
+    forced = set()
+    if valid_nb > 0:
+        if force_first:
+            forced.add(0)
+        if force_last:
+            forced.add(valid_nb - 1)
+    cand = [b for b in range(valid_nb) if b not in forced]
+    order = sorted(cand, key=lambda b: (-S[b], b))
+    chosen = order[:min(k, len(order))]
+    near_tie = False
+    if 0 < k < len(order):
+        sk, sk1 = S[order[k - 1]], S[order[k]]
+        near_tie = bool(sk <= 0 or (sk - sk1) / sk < NEAR_TIE_REL)
+    kept = sorted(forced | set(chosen))
+    return {"kept": kept, "order": order, "near_tie": near_tie, "forced": sorted(forced)}
+
+
+# --------------------------------------------------------------------------- attention
+def softmax_attend(logits: np.ndarray, values: np.ndarray):
+    """out = sum_i softmax(logits)_i values_i and lse = ln sum_i exp(logits_i),
+    with a max shift. logits: [T]; values: [T][D]. Entries with logit -inf do not
+    contribute. Empty or all -inf -> (zeros, -inf) (reading R9)."""
+    D = values.shape[1] if values.ndim == 2 else 0
+    logits = np.asarray(logits, dtype=np.float64)
+    if logits.size == 0 or np.max(logits) == -math.inf:
+        return np.zeros(D), -math.inf
+    m = np.max(logits)
+    p = np.exp(logits - m)
+    z = p.sum()
+    out = (p[:, None] * values).sum(axis=0) / z
+    return out, float(m + math.log(z))
+
+
+def tail_proxy(qg: np.ndarray, K: np.ndarray, V: np.ndarray, n: int, L: int,
+               kept: Sequence[int], sigma: float):
+    """Count-aware tail proxy [OA, "Skipping reviews without losing the verdict";
+    reading R7]: one virtual token whose value is the mean of the unread values and
+    whose logit is the mean unread logit plus ln(count), computed here directly
+    from the tail tokens.
+
+    Returns (logits [G], value [D], n_T) or None when the tail is empty.
+    """
+    mask = np.ones(n, dtype=bool)
+    for b in kept:
+        mask[b * L:min(n, (b + 1) * L)] = False
+    nT = int(mask.sum())
+    if nT == 0:
+        return None
+    tail_logits = sigma * (K[:n][mask] @ qg.T)    # [nT][G]
+    mean_logit = tail_logits.mean(axis=0)          # [G]
+    value = V[:n][mask].mean(axis=0)
+    return mean_logit + math.log(nT), value, nT
+
+
+def sparse_attend_one(qg, K, V, n, L, kept, sigma, use_proxy=True):
+    """Exact attention over the kept blocks' tokens plus, when use_proxy, the tail
+    proxy as one more softmax entry [OA: the proxy "enters the softmax next to the
+    exact tokens"]. Without the proxy this is top-k discard: the kept tokens are
+    renormalised among themselves [COBS, text after Equation 1].
+
+    qg: [G][D]; K, V: [Ncap][D]. Returns out [G][D], lse [G], proxy info.
+    """
+    G = qg.shape[0]
+    D = V.shape[1]
+    rows = []
+    for b in sorted(kept):
+        rows.extend(range(b * L, min(n, (b + 1) * L)))
+    rows = np.asarray(rows, dtype=np.int64)
+    proxy = tail_proxy(qg, K, V, n, L, kept, sigma) if use_proxy else None
+    out = np.zeros((G, D))
+    lse = np.full(G, -math.inf)
+    for g in range(G):
+        logits = sigma * (K[rows] @ qg[g]) if rows.size else np.zeros(0)
+        vals = V[rows] if rows.size else np.zeros((0, D))
+        if proxy is not None:
+            logits = np.concatenate([logits, [proxy[0][g]]])
+            vals = np.concatenate([vals, proxy[1][None, :]], axis=0)
+        out[g], lse[g] = softmax_attend(logits, vals)
+    return out, lse, proxy
+
+
+def weighted_attend_one(qg, K, V, n, tok_idx, w, sigma):
+    """Attention over an explicitly weighted coreset [WC, abstract]: token i enters
+    the softmax with logit sigma q.k_i + ln w_i (reading R8). Tokens with w_i = 0
+    or an index outside [0, n) are excluded."""
+    G = qg.shape[0]
+    D = V.shape[1]
+    out = np.zeros((G, D))
+    lse = np.full(G, -math.inf)
+    idx = np.asarray(tok_idx, dtype=np.int64)
+    w = np.asarray(w, dtype=np.float64)
+    keep = (w > 0) & (idx >= 0) & (idx < n)
+    idx, w = idx[keep], w[keep]
+    for g in range(G):
+        logits = sigma * (K[idx] @ qg[g]) + np.log(w)
+        out[g], lse[g] = softmax_attend(logits, V[idx])
+    return out, lse
+
+
+def dense_attend_one(qg, K, V, n, sigma):
+    """Exact softmax attention over all n tokens [COBS: "Dense reads the whole KV
+    cache"]."""
+    G = qg.shape[0]
+    D = V.shape[1]
+    out = np.zeros((G, D))
+    lse = np.full(G, -math.inf)
+    for g in range(G):
+        out[g], lse[g] = softmax_attend(sigma * (K[:n] @ qg[g]), V[:n])
+    return out, lse
+
+
+# --------------------------------------------------------------------------- batched
+def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
+                 k_sum=None, counts=None, bh=None):
+    """Block choice for every (sequence, KV head), or for the listed ones.
+
+    q: [B][Hq][D]; K: [B][Hkv][Ncap][D] float64 (needed for exact-mass mode and to
+    build summaries when k_sum is not given). Returns a dict keyed by (b, h) with
+    kept, near_tie, S and s_hat.
+    """
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    Ncap = K.shape[2]
+    G = Hq // Hkv
+    NBcap = (Ncap + L - 1) // L
+    res = {}
+    pairs = bh if bh is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for (b, h) in pairs:
+        n = int(seq_lens[b])
+        nb = (n + L - 1) // L
+        qg = q[b, h * G:(h + 1) * G]
+        if mode == "summary":
+            if k_sum is None:
+                ks, _, c, _, _ = block_summaries_one(K[b, h], K[b, h], n, L, NBcap)
+            else:
+                ks, c = k_sum[b, h], counts[b]
+            shat = summary_logits(qg, ks[:nb], c[:nb], sigma)
+        elif mode == "exact_mass":
+            shat = exact_log_mass(qg, K[b, h], n, L, nb, sigma)
+        else:
+            raise ValueError(mode)
+        S = group_score(shat)
+        sel = select_blocks(S, nb, k, force_first, force_last)
+        sel["S"] = S
+        sel["s_hat"] = shat
+        res[(b, h)] = sel
+    return res
+
+
+def sparse_batch(q, K, V, seq_lens, L, sigma, kept: Dict, use_proxy=True, bh=None):
+    """out [B][Hq][D], lse [B][Hq] for the given kept-block lists (dict keyed by
+    (b, h)); rows not listed in bh stay NaN."""
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    out = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    pairs = bh if bh is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for (b, h) in pairs:
+        o, l, _ = sparse_attend_one(q[b, h * G:(h + 1) * G], K[b, h], V[b, h],
+                                    int(seq_lens[b]), L, kept[(b, h)], sigma, use_proxy)
+        out[b, h * G:(h + 1) * G], lse[b, h * G:(h + 1) * G] = o, l
+    return out, lse
+
+
+def weighted_batch(q, K, V, seq_lens, tok_idx, w, sigma, bh=None):
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    out = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    pairs = bh if bh is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for (b, h) in pairs:
+        o, l = weighted_attend_one(q[b, h * G:(h + 1) * G], K[b, h], V[b, h],
+                                   int(seq_lens[b]), tok_idx[b, h], w[b, h], sigma)
+        out[b, h * G:(h + 1) * G], lse[b, h * G:(h + 1) * G] = o, l
+    return out, lse
+
+
+def dense_batch(q, K, V, seq_lens, sigma, bh=None):
+    B, Hq, D = q.shape
+    Hkv = K.shape[1]
+    G = Hq // Hkv
+    out = np.full((B, Hq, D), np.nan)
+    lse = np.full((B, Hq), np.nan)
+    pairs = bh if bh is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    for (b, h) in pairs:
+        o, l = dense_attend_one(q[b, h * G:(h + 1) * G], K[b, h], V[b, h],
+                                int(seq_lens[b]), sigma)
+        out[b, h * G:(h + 1) * G], lse[b, h * G:(h + 1) * G] = o, l
+    return out, lse
+
+
+def decode_step(q, K, V, seq_lens, L, sigma, k, force_first, force_last,
+                score_mode="summary", use_proxy=True, bh=None):
+    """One decode step of one layer for every sequence: block choice per KV head,
+    then attention over the kept blocks plus the tail proxy."""
+    sel = select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last,
+                       score_mode, bh=bh)
+    kept = {key: v["kept"] for key, v in sel.items()}
+    out, lse = sparse_batch(q, K, V, seq_lens, L, sigma, kept, use_proxy, bh=bh)
+    return sel, out, lse

@@ -1,0 +1,378 @@
+"""Pins for the float64 oracle: each function checks the oracle against something
+other than itself -- a brute-force loop in plain Python floats, a closed form, an
+invariant the pages state, or the numbers of the pages' worked example -- and raises
+AssertionError on a mismatch. The tests call them as they are, and the planted-mistake
+test calls them against deliberately broken copies of oracle functions.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+from oracle import oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+TOL = 1e-12
+
+
+def _close(a, b, tol=TOL, what=""):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    scale = max(1.0, float(np.max(np.abs(b))) if b.size else 1.0)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} > {tol:.1e} * {scale:.3g}"
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------- brute force helpers
+def _py_dense(qg, K, V, n, sigma):
+    """Softmax attention written as nested Python loops over floats."""
+    G, D = len(qg), len(qg[0])
+    outs, lses = [], []
+    for g in range(G):
+        logits = []
+        for r in range(n):
+            s = 0.0
+            for d in range(D):
+                s += float(qg[g][d]) * float(K[r][d])
+            logits.append(sigma * s)
+        m = max(logits)
+        ws = [math.exp(x - m) for x in logits]
+        z = sum(ws)
+        o = [sum(ws[r] * float(V[r][d]) for r in range(n)) / z for d in range(D)]
+        outs.append(o)
+        lses.append(m + math.log(z))
+    return outs, lses
+
+
+# ----------------------------------------------------------------------------- pins
+def pin_dense_bruteforce(seed=0):
+    r = _rng(seed)
+    G, D, n = 3, 5, 23
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n + 4, D)), r.normal(size=(n + 4, D))
+    o, l = O.dense_attend_one(qg, K, V, n, 0.7)
+    po, pl = _py_dense(qg.tolist(), K.tolist(), V.tolist(), n, 0.7)
+    _close(o, po, what="dense out")
+    _close(l, pl, what="dense lse")
+
+
+def pin_summaries_closed_form(seed=1):
+    r = _rng(seed)
+    D, Ncap, L = 4, 37, 8
+    for n in (0, 1, 8, 29, 37):
+        K, V = r.normal(size=(Ncap, D)), r.normal(size=(Ncap, D))
+        NBcap = (Ncap + L - 1) // L
+        ks, vs, c, kt, vt = O.block_summaries_one(K, V, n, L, NBcap)
+        for b in range(NBcap):
+            cnt = 0
+            sk = [0.0] * D
+            sv = [0.0] * D
+            for t in range(b * L, (b + 1) * L):
+                if t < n:
+                    cnt += 1
+                    for d in range(D):
+                        sk[d] += float(K[t][d])
+                        sv[d] += float(V[t][d])
+            assert int(c[b]) == cnt, f"count of block {b} at n={n}"
+            _close(ks[b], sk, what="k_sum")
+            _close(vs[b], sv, what="v_sum")
+        _close(kt, [sum(float(K[t][d]) for t in range(n)) for d in range(D)], what="k_tot")
+        _close(vt, [sum(float(V[t][d]) for t in range(n)) for d in range(D)], what="v_tot")
+
+
+def pin_exact_mass_bruteforce(seed=2):
+    r = _rng(seed)
+    G, D, n, L = 2, 3, 21, 6
+    qg, K = r.normal(size=(G, D)), r.normal(size=(n, D))
+    nb = (n + L - 1) // L
+    lm = O.exact_log_mass(qg, K, n, L, nb, 0.9)
+    for g in range(G):
+        for b in range(nb):
+            tot = 0.0
+            for t in range(b * L, min(n, (b + 1) * L)):
+                tot += math.exp(0.9 * sum(float(qg[g][d]) * float(K[t][d]) for d in range(D)))
+            _close(lm[g, b], math.log(tot), what="ln m_b")
+
+
+def pin_block_decomposition(seed=3):
+    """COBS, text around Equation 1: the dense output is the P_b-weighted mixture of
+    the block centroids v^c_b, with P_b = m_b / Z."""
+    r = _rng(seed)
+    G, D, n, L = 2, 4, 45, 8
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    o, _ = O.dense_attend_one(qg, K, V, n, 1.0)
+    for g in range(G):
+        masses, cents = [], []
+        for (s, e) in O.blocks_of(n, L):
+            ws = [math.exp(float(qg[g] @ K[t])) for t in range(s, e)]
+            m = sum(ws)
+            masses.append(m)
+            cents.append([sum(ws[i] * float(V[s + i][d]) for i in range(e - s)) / m
+                          for d in range(D)])
+        Z = sum(masses)
+        mix = [sum(masses[b] / Z * cents[b][d] for b in range(len(masses))) for d in range(D)]
+        _close(o[g], mix, what="block decomposition")
+
+
+def pin_discard_error_identity(seed=4):
+    """COBS, text after Equation 1: o - o_S = (1/(1 - tau)) sum_{b not in S} P_b
+    (v^c_b - o), tau the dropped mass. o_S is the oracle's discard-mode output."""
+    r = _rng(seed)
+    G, D, n, L = 1, 3, 40, 5
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    kept = [0, 3, 6]
+    o, _ = O.dense_attend_one(qg, K, V, n, 1.0)
+    oS, _, _ = O.sparse_attend_one(qg, K, V, n, L, kept, 1.0, use_proxy=False)
+    ws = [math.exp(float(qg[0] @ K[t])) for t in range(n)]
+    Z = sum(ws)
+    tau = 0.0
+    rhs = [0.0] * D
+    for b, (s, e) in enumerate(O.blocks_of(n, L)):
+        if b in kept:
+            continue
+        m = sum(ws[s:e])
+        P = m / Z
+        tau += P
+        cent = [sum(ws[t] * float(V[t][d]) for t in range(s, e)) / m for d in range(D)]
+        for d in range(D):
+            rhs[d] += P * (cent[d] - float(o[0][d]))
+    rhs = [x / (1.0 - tau) for x in rhs]
+    _close(o[0] - oS[0], rhs, what="discard error identity")
+
+
+def pin_all_kept_equals_dense(seed=5):
+    r = _rng(seed)
+    G, D, n, L = 2, 6, 61, 8
+    q = r.normal(size=(1, G, D))
+    K, V = r.normal(size=(1, 1, n, D)), r.normal(size=(1, 1, n, D))
+    nb = (n + L - 1) // L
+    sel, out, lse = O.decode_step(q, K, V, [n], L, 0.5, nb, False, False)
+    assert sel[(0, 0)]["kept"] == list(range(nb))
+    do, dl = O.dense_batch(q, K, V, [n], 0.5)
+    _close(out, do, what="all kept out")
+    _close(lse, dl, what="all kept lse")
+
+
+def pin_proxy_exact_equal_tail(seed=6):
+    """OA: the proxy represents the tail exactly when every tail token has the same
+    logit. Tail keys differ from each other but share their projection on q."""
+    r = _rng(seed)
+    D, n, L = 5, 50, 10
+    q = r.normal(size=(1, D))
+    qhat = q[0] / np.linalg.norm(q[0])
+    K = r.normal(size=(n, D))
+    V = r.normal(size=(n, D))
+    kept = [1, 3]
+    for t in range(n):
+        if t // L not in kept:
+            u = K[t] - (K[t] @ qhat) * qhat          # component orthogonal to q
+            K[t] = 0.3 * qhat + u                    # every tail logit = 0.3 |q| sigma
+    o, l, proxy = O.sparse_attend_one(q, K, V, n, L, kept, 0.8, use_proxy=True)
+    do, dl = O.dense_attend_one(q, K, V, n, 0.8)
+    _close(o, do, what="proxy exact out")
+    _close(l, dl, what="proxy exact lse")
+
+
+def pin_proxy_logit_is_mean_plus_log_count(seed=7):
+    """OA: proxy logit = mean tail logit + ln(count), so its weight is count times
+    the weight of a mean-logit token; its value is the mean of the tail values."""
+    r = _rng(seed)
+    G, D, n, L = 2, 4, 33, 4
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    kept = [0, 5]
+    logit, value, nT = O.tail_proxy(qg, K, V, n, L, kept, 0.6)
+    tail = [t for t in range(n) if t // L not in kept]
+    assert nT == len(tail)
+    for g in range(G):
+        ls = [0.6 * sum(float(qg[g][d]) * float(K[t][d]) for d in range(D)) for t in tail]
+        mean_l = sum(ls) / len(ls)
+        _close(logit[g], mean_l + math.log(len(tail)), what="proxy logit")
+        _close(math.exp(logit[g]), len(tail) * math.exp(mean_l), what="proxy weight")
+    _close(value, [sum(float(V[t][d]) for t in tail) / len(tail) for d in range(D)],
+           what="proxy value")
+
+
+def pin_jensen(seed=8):
+    """Proxy weight <= true tail mass (equality iff equal tail logits, OA), and the
+    mean-pool score <= exact log-mass (COBS: mean pooling matches only the zeroth
+    and first cumulant terms)."""
+    r = _rng(seed)
+    G, D, n, L = 3, 6, 90, 9
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    kept = [2, 7]
+    logit, _, _ = O.tail_proxy(qg, K, V, n, L, kept, 1.0)
+    tail = [t for t in range(n) if t // L not in kept]
+    for g in range(G):
+        mass = sum(math.exp(float(qg[g] @ K[t])) for t in tail)
+        assert math.exp(logit[g]) <= mass * (1 + 1e-12)
+        assert math.exp(logit[g]) < mass * (1 - 1e-6), "random tail should be strict"
+    nb = (n + L - 1) // L
+    ks, _, c, _, _ = O.block_summaries_one(K, V, n, L, nb)
+    sh = O.summary_logits(qg, ks, c, 1.0)
+    lm = O.exact_log_mass(qg, K, n, L, nb, 1.0)
+    assert np.all(sh <= lm + 1e-12), "summary score above exact log-mass"
+    assert np.all(sh < lm - 1e-9), "random blocks should be strict"
+
+
+def pin_integer_weights_duplication(seed=9):
+    """WC form: exp(s + ln w) = w exp(s), so integer w equals w-fold duplication."""
+    r = _rng(seed)
+    G, D, n = 2, 5, 40
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    idx = r.choice(n, size=12, replace=False)
+    w = r.integers(1, 5, size=12).astype(np.float64)
+    o, l = O.weighted_attend_one(qg, K, V, n, idx, w, 0.9)
+    rows = [int(i) for i, c in zip(idx, w) for _ in range(int(c))]
+    Kd, Vd = K[rows], V[rows]
+    po, pl = _py_dense(qg.tolist(), Kd.tolist(), Vd.tolist(), len(rows), 0.9)
+    _close(o, po, what="weighted == duplicated out")
+    _close(l, pl, what="weighted == duplicated lse")
+
+
+def pin_zero_weight_excluded(seed=10):
+    r = _rng(seed)
+    G, D, n = 1, 3, 20
+    qg, K, V = r.normal(size=(G, D)), r.normal(size=(n, D)), r.normal(size=(n, D))
+    idx = np.array([1, 4, 7, 9])
+    w = np.array([2.0, 0.0, 1.0, 3.0])
+    o, l = O.weighted_attend_one(qg, K, V, n, idx, w, 1.0)
+    o2, l2 = O.weighted_attend_one(qg, K, V, n, idx[[0, 2, 3]], w[[0, 2, 3]], 1.0)
+    _close(o, o2, what="zero weight")
+    _close(l, l2, what="zero weight lse")
+
+
+def pin_summary_equals_exact_for_constant_blocks(seed=13):
+    """When every key of a block is the same vector k, m_b = n_b exp(sigma q.k)
+    exactly, so the mean-pool score must equal the exact log-mass (the Jensen
+    equality case); ragged last block included."""
+    r = _rng(seed)
+    G, D, n, L = 3, 4, 27, 8
+    qg = r.normal(size=(G, D))
+    K = np.zeros((n, D))
+    for b, (s, e) in enumerate(O.blocks_of(n, L)):
+        K[s:e] = r.normal(size=D)
+    nb = (n + L - 1) // L
+    ks, _, c, _, _ = O.block_summaries_one(K, K, n, L, nb)
+    sh = O.summary_logits(qg, ks, c, 0.7)
+    for g in range(G):
+        for b, (s, e) in enumerate(O.blocks_of(n, L)):
+            want = math.log((e - s) * math.exp(0.7 * float(qg[g] @ K[s])))
+            _close(sh[g, b], want, what="constant-block summary score")
+
+
+def pin_group_score_invariants(seed=11):
+    """Each head's block probabilities sum to one, so sum_b S_b = G; for G = 1 the
+    ranking equals the ranking by s_hat (COBS: for G = 1, keeping the top-k by m_b,
+    equivalently by ln m_b)."""
+    r = _rng(seed)
+    for G in (1, 4, 7):
+        sh = r.normal(size=(G, 30)) * 3
+        S = O.group_score(sh)
+        _close(S.sum(), G, what="sum of S")
+        assert np.all(S >= 0) and np.all(S <= G)
+        # brute-force probabilities for one head
+        z = sum(math.exp(x) for x in sh[0])
+        if G == 1:
+            _close(S, [math.exp(x) / z for x in sh[0]], what="G=1 probabilities")
+            a = O.select_blocks(S, 30, 7, False, False)["order"]
+            b = sorted(range(30), key=lambda i: (-sh[0][i], i))
+            assert a == b, "G=1 order differs from s_hat order"
+
+
+def pin_topk_bruteforce(seed=12):
+    """The kept set maximises the summed score over all k-subsets of the competing
+    blocks; among equal sums the lexicographically smallest index set wins."""
+    r = _rng(seed)
+    for trial in range(6):
+        nb = 9
+        S = np.round(r.random(nb) * 4) / 4 if trial % 2 else r.random(nb)
+        for ff, fl in ((False, False), (True, True), (True, False)):
+            forced = set([0] if ff else []) | set([nb - 1] if fl else [])
+            cand = [b for b in range(nb) if b not in forced]
+            for k in (1, 3, 5, len(cand), len(cand) + 2):
+                best = None
+                for sub in itertools.combinations(cand, min(k, len(cand))):
+                    # ties in the sum are broken by the per-element (score, index) order
+                    key = (sorted([(-S[b], b) for b in sub]),)
+                    if best is None or key < best[0]:
+                        best = (key, sub)
+                want = sorted(forced | set(best[1]))
+                got = O.select_blocks(S, nb, k, ff, fl)["kept"]
+                assert got == want, f"top-k {got} != brute force {want}"
+                assert sum(S[b] for b in got if b not in forced) >= \
+                    max(sum(S[b] for b in sub) for sub in
+                        itertools.combinations(cand, min(k, len(cand)))) - 1e-15
+
+
+def pin_near_tie_flag():
+    S = np.array([0.5, 0.30, 0.2999, 0.1])
+    assert O.select_blocks(S, 4, 2, False, False)["near_tie"]
+    assert not O.select_blocks(S, 4, 1, False, False)["near_tie"]
+    assert not O.select_blocks(S, 4, 4, False, False)["near_tie"]
+
+
+def pin_worked_example():
+    """OA, "A worked example with named numbers": 10,000 tokens; 100 exact tokens
+    hold 60%; a 9,900-token tail with equal logits holds 40%."""
+    with open(os.path.join(GOLDEN, "openattention_worked_example.json")) as f:
+        ex = json.load(f)
+    n, n_ex, n_tail = ex["context_tokens"], ex["exact_tokens"], ex["tail_tokens"]
+    assert n_ex + n_tail == n
+    # one channel: logit = key value; exact tokens share logit a, the tail logit 0
+    a = math.log(ex["exact_mass"] / ex["tail_mass"] * n_tail / n_ex)
+    K = np.zeros((n, 1))
+    K[:n_ex, 0] = a
+    V = np.zeros((n, 2))
+    V[:n_ex, 0] = 1.0            # channel 0 reads the exact tokens' share
+    V[n_ex:, 1] = 1.0            # channel 1 reads the tail's share
+    q = np.ones((1, 1))
+    L = n_ex
+    dense, _ = O.dense_attend_one(q, K, V, n, 1.0)
+    _close(dense[0], [ex["exact_mass"], ex["tail_mass"]], what="toy masses")
+    disc, _, _ = O.sparse_attend_one(q, K, V, n, L, [0], 1.0, use_proxy=False)
+    infl = disc[0][0] / dense[0][0]
+    assert abs(infl - 1 / 0.6) < 1e-12 and round(infl, 2) == ex["discard_inflation_about"]
+    prox, _, p = O.sparse_attend_one(q, K, V, n, L, [0], 1.0, use_proxy=True)
+    _close(prox[0], [ex["exact_mass"], ex["proxy_tail_mass_kept"]], what="proxy keeps 40%")
+    assert p[2] == n_tail
+    # scaled-up sample through the weighted mode: 50 tail tokens with weight 198
+    s = ex["sample_tokens"]
+    scale = n_tail / s
+    assert scale == ex["sample_scale_up"]
+    hit = s / n_tail
+    assert round(hit, 3) == ex["sample_hit_probability_about"]
+    assert round(1 - hit, 3) == ex["sample_miss_fraction_about"]
+    idx = np.concatenate([np.arange(n_ex), n_ex + np.arange(s) * 7])
+    w = np.concatenate([np.ones(n_ex), np.full(s, scale)])
+    wo, _ = O.weighted_attend_one(q, K, V, n, idx, w, 1.0)
+    _close(wo[0], [ex["exact_mass"], ex["tail_mass"]], what="scaled sample mass")
+
+
+def pin_empty_inputs():
+    D = 3
+    K = np.zeros((8, D))
+    o, l = O.dense_attend_one(np.ones((2, D)), K, K, 0, 1.0)
+    assert np.all(o == 0) and np.all(l == -math.inf)
+    o, l = O.weighted_attend_one(np.ones((1, D)), K, K, 8, [1, 2], [0.0, 0.0], 1.0)
+    assert np.all(o == 0) and l[0] == -math.inf
+    sel = O.select_blocks(np.zeros(0), 0, 3, True, True)
+    assert sel["kept"] == []
+    sel = O.select_blocks(np.array([0.7]), 1, 3, True, True)
+    assert sel["kept"] == [0]
+
+
+ALL_PINS = [
+    pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
+    pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
+    pin_proxy_exact_equal_tail, pin_proxy_logit_is_mean_plus_log_count, pin_jensen,
+    pin_integer_weights_duplication, pin_zero_weight_excluded, pin_group_score_invariants,
+    pin_topk_bruteforce, pin_near_tie_flag, pin_worked_example, pin_empty_inputs,
+    pin_summary_equals_exact_for_constant_blocks,
+]

@@ -1,0 +1,123 @@
+"""Planted mistakes: each mutant breaks one oracle function in a plausible way
+(a dropped term, a wrong sign or index, a wrong reduction) and at least one pin
+must fail on it. This checks that the pins can see such mistakes."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle_pins as P
+from oracle import oracle as O
+
+
+def _mut_proxy_no_log_count(orig):
+    def f(qg, K, V, n, L, kept, sigma):
+        r = orig(qg, K, V, n, L, kept, sigma)
+        return None if r is None else (r[0] - math.log(r[2]), r[1], r[2])
+    return f
+
+
+def _mut_proxy_sum_value(orig):
+    def f(qg, K, V, n, L, kept, sigma):
+        r = orig(qg, K, V, n, L, kept, sigma)
+        return None if r is None else (r[0], r[1] * r[2], r[2])
+    return f
+
+
+def _mut_summary_no_log(orig):
+    def f(qg, k_sum, counts, sigma):
+        out = orig(qg, k_sum, counts, sigma)
+        c = np.asarray(counts, dtype=np.float64)
+        return np.where(c > 0, out - np.log(np.maximum(c, 1)), out)
+    return f
+
+
+def _mut_summary_sum_not_mean(orig):
+    def f(qg, k_sum, counts, sigma):
+        return orig(qg, k_sum * np.maximum(np.asarray(counts)[:, None], 1), counts, sigma)
+    return f
+
+
+def _mut_group_score_logits(orig):
+    def f(shat):
+        return np.where(np.isfinite(shat), shat, 0.0).sum(axis=0)
+    return f
+
+
+def _mut_select_high_index(orig):
+    def f(S, valid_nb, k, ff, fl):
+        r = orig(-np.asarray(S)[::-1] * -1 if False else S, valid_nb, k, ff, fl)
+        forced = set(r["forced"])
+        cand = [b for b in range(valid_nb) if b not in forced]
+        order = sorted(cand, key=lambda b: (-S[b], -b))
+        r["order"] = order
+        r["kept"] = sorted(forced | set(order[:min(k, len(order))]))
+        return r
+    return f
+
+
+def _mut_exact_mass_max(orig):
+    def f(qg, K, n, L, NB, sigma):
+        out = np.full((qg.shape[0], NB), -math.inf)
+        for b, (s, e) in enumerate(O.blocks_of(n, L)):
+            out[:, b] = (sigma * (K[s:e] @ qg.T)).max(axis=0)
+        return out
+    return f
+
+
+def _mut_weighted_no_log(orig):
+    def f(qg, K, V, n, idx, w, sigma):
+        w = np.asarray(w, dtype=np.float64)
+        return orig(qg, K, V, n, idx, np.where(w > 0, 1.0, 0.0), sigma)
+    return f
+
+
+def _mut_summaries_count(orig):
+    def f(K, V, n, L, NBcap):
+        ks, vs, c, kt, vt = orig(K, V, n, L, NBcap)
+        c = c.copy()
+        c[c > 0] = L
+        return ks, vs, c, kt, vt
+    return f
+
+
+def _mut_softmax_no_norm(orig):
+    def f(logits, values):
+        o, l = orig(logits, values)
+        return o * 1.01, l
+    return f
+
+
+def _mut_logsumexp_shift(orig):
+    def f(x):
+        v = orig(x)
+        return v if v == -math.inf else v + 1e-3
+    return f
+
+
+MUTANTS = {
+    "tail_proxy/no ln count": ("tail_proxy", _mut_proxy_no_log_count),
+    "tail_proxy/sum not mean": ("tail_proxy", _mut_proxy_sum_value),
+    "summary_logits/no ln n_b": ("summary_logits", _mut_summary_no_log),
+    "summary_logits/sum not mean": ("summary_logits", _mut_summary_sum_not_mean),
+    "group_score/sums logits": ("group_score", _mut_group_score_logits),
+    "select_blocks/high-index ties": ("select_blocks", _mut_select_high_index),
+    "exact_log_mass/max not lse": ("exact_log_mass", _mut_exact_mass_max),
+    "weighted/no ln w": ("weighted_attend_one", _mut_weighted_no_log),
+    "summaries/count": ("block_summaries_one", _mut_summaries_count),
+    "softmax/unnormalised": ("softmax_attend", _mut_softmax_no_norm),
+    "logsumexp/offset": ("logsumexp", _mut_logsumexp_shift),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_some_pin_fails_on_mutant(name, monkeypatch):
+    attr, make = MUTANTS[name]
+    monkeypatch.setattr(O, attr, make(getattr(O, attr)))
+    failed = []
+    for pin in P.ALL_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin caught mutant {name}"
