@@ -1,0 +1,537 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of reduced-KV softmax attention on B200.
+
+One step = one decode step of one layer for the whole batch: block selection per
+KV head (kv_select_blocks, summary mode) and attention over the kept blocks plus
+the tail proxy (kv_sparse_decode_attn). The block summaries are built once before
+timing (they belong to prefill). Default workload: Llama-3.1-8B-shaped GQA decode
+(32 query heads, 8 KV heads, head dim 128), batch 32, 32K context, block 64, 1%
+read budget (top-5 + first + last block + proxy), synthetic bf16 cache.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 launch with torch.distributed.run: every rank runs its own batch on its
+GPU (weak scaling, no collective on the data path); value = queries of all ranks /
+max-over-ranks time. `--impl reference` times the float64 CPU oracle on the host
+cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import multiprocessing as mp
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode queries/s and achieved HBM GB/s (% of 8 TB/s) at B=32, 32K ctx"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 512 << 20
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_coreset"])
+    ap.add_argument("--budget", type=float, default=0.01)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------- distributed
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        import torch.distributed as dist
+        if self.world > 1 and not dist.is_initialized():
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=180))
+            self.pg = True
+
+    def barrier(self, device=None):
+        if self.pg:
+            import torch.distributed as dist
+            if device is not None and device.type == "cuda":
+                dist.barrier(device_ids=[device.index])
+            else:
+                dist.barrier()
+
+    def max(self, x: float, device) -> float:
+        if not self.pg:
+            return x
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+def shard_seed_offset(rank: int) -> int:
+    """Each rank draws its own batch: seeds shift by 1000 per rank."""
+    return 1000 * rank
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, period_ms: int = 20):
+        self.idx = gpu_index
+        self.period = period_ms
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 f"-lms", str(self.period)], stdout=self.fh, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self, t0: float, t1: float):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(2 * self.period / 1000.0)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[5], parts[6:10]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05]
+        use = inside if inside else sorted(rows, key=lambda r: abs(r[0] - (t0 + t1) / 2))[:3]
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[4]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
+
+def measured_peak_hbm():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- byte model
+def attention_bytes(wl, n_kept, seq_lens):
+    """Algorithmic bytes of one kv_sparse_decode_attn launch (block mode + proxy):
+    the kept blocks' K and V rows, the kept blocks' key/value sums and counts, the
+    totals, the index lists, q in and out/lse out."""
+    import numpy as np
+    L, D, G = wl.block_size, wl.D, wl.G
+    es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    nk = n_kept.cpu().numpy()
+    total = 0
+    for b in range(wl.B):
+        n = seq_lens[b]
+        for h in range(wl.Hkv):
+            k = int(nk[b, h])
+            # all kept blocks are full except possibly the last block of the sequence
+            toks = min(k * L, n) if k else 0
+            total += toks * D * es * 2                  # K and V rows
+            total += k * (D * 4 * 2 + 4 + 4)            # kept k_sum, v_sum rows, counts, indices
+            total += 2 * D * 4 + 4 + 4                  # totals, n_kept, seq_len
+            total += G * D * es + G * D * 4 + G * 4     # q in, out and lse out
+    return total
+
+
+def select_bytes(wl, seq_lens):
+    """Algorithmic bytes of one kv_select_blocks launch (summary mode): every valid
+    block's fp32 key sum and count, q, and the kept indices written."""
+    L, D, G = wl.block_size, wl.D, wl.G
+    es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    total = 0
+    for b in range(wl.B):
+        nbv = (seq_lens[b] + L - 1) // L
+        total += wl.Hkv * (nbv * (D * 4 + 4) + G * D * es + wl.kmax * 4 + 4)
+    return total
+
+
+def osa_select_bytes(wl, seq_lens):
+    es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
+
+
+def weighted_bytes(wl):
+    es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    return wl.B * wl.Hkv * (wl.m * (wl.D * es * 2 + 8) + wl.G * wl.D * (es + 4) + wl.G * 4)
+
+
+# ----------------------------------------------------------------- CPU oracle
+def _oracle_task(args):
+    """One (sequence, KV head) decode step with the float64 oracle."""
+    import numpy as np
+    from oracle import oracle as O
+    kind, q16, K16, V16, n, L, scale, k_top, ff, fl, extra = args
+
+    def f64(a):
+        if a.dtype == np.uint16:
+            return (a.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        return a.astype(np.float64)
+
+    q, K, V = f64(q16)[None], f64(K16)[None, None], f64(V16)[None, None]
+    if kind == "weighted":
+        O.weighted_batch(q, K, V, [n], extra[0][None, None], extra[1][None, None], scale)
+    elif kind == "dense":
+        O.dense_batch(q, K, V, [n], scale)
+    else:
+        O.decode_step(q, K, V, [n], L, scale, k_top, ff, fl, score_mode=kind, use_proxy=True)
+    return 1
+
+
+def _pool_init():
+    os.environ.setdefault("OMP_NUM_THREADS", "1")
+    os.environ.setdefault("OPENBLAS_NUM_THREADS", "1")
+    os.environ.setdefault("MKL_NUM_THREADS", "1")
+
+
+def oracle_tasks(wl, pairs):
+    import numpy as np
+    import torch
+    tasks = []
+    kind = {"summary": "summary", "exact_mass": "exact_mass"}[wl.score_mode]
+    if wl.attn_mode == "weighted":
+        kind = "weighted"
+    for (b, h) in pairs:
+        def raw(t):
+            t = t.detach().cpu()
+            return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+        q = raw(wl.q[b, h * wl.G:(h + 1) * wl.G])
+        K = raw(wl.K[b, h])
+        V = raw(wl.V[b, h])
+        extra = None
+        if kind == "weighted":
+            extra = (wl.tok_idx[b, h].cpu().numpy(), wl.w[b, h].cpu().numpy().astype(np.float64))
+        tasks.append((kind, q, K, V, wl.seq_lens[b], wl.block_size, wl.scale, wl.k_top,
+                      bool(wl.force_first), bool(wl.force_last), extra))
+    return tasks
+
+
+def time_oracle(wl, n_pairs_target, workers, warm_pairs=1):
+    """Wall time of the oracle over n pairs (sequence, KV head) on a spawn pool."""
+    pairs_all = [(b, h) for b in range(wl.B) for h in range(wl.Hkv)]
+    n = max(1, n_pairs_target)
+    pairs = [pairs_all[i % len(pairs_all)] for i in range(n)]
+    uniq = sorted(set(pairs))
+    tmap = dict(zip(uniq, oracle_tasks(wl, uniq)))
+    tasks = [tmap[p] for p in pairs]
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(workers, initializer=_pool_init) as pool:
+        pool.map(_oracle_task, tasks[:max(1, min(warm_pairs, len(tasks)))] * 1)
+        t0 = time.perf_counter()
+        pool.map(_oracle_task, tasks, chunksize=1)
+        dt = time.perf_counter() - t0
+    return dt, n
+
+
+def cpu_baseline(wl, seconds, label_sample):
+    """Oracle throughput on the host cores over a bounded sample of the workload."""
+    workers = max(1, min(os.cpu_count() or 1, 32))
+    # calibrate with one pair in-process, single-threaded BLAS
+    _pool_init()
+    t0 = time.perf_counter()
+    _oracle_task(oracle_tasks(wl, [(0, 0)])[0])
+    t1 = time.perf_counter() - t0
+    n = int(max(1, min(wl.B * wl.Hkv * 4, seconds * workers / max(t1, 1e-3))))
+    n = max(workers, n) if n >= workers else n
+    dt, n = time_oracle(wl, n, workers)
+    queries = n / wl.Hkv
+    return {"value": queries / dt, "unit": "queries/s", "cores": workers, "kind": "oracle",
+            "sample": f"{n} (sequence, KV head) decode steps = {queries:g} queries of {label_sample}; "
+                      f"float64 NumPy oracle (select + attend), {workers} spawn workers, 1 BLAS thread each",
+            "seconds": dt}
+
+
+# ----------------------------------------------------------------- our arm
+def workload_label(wl, budget):
+    names = {
+        "llama": "Llama-3.1-8B-shaped GQA decode",
+        "qwen_long": "Qwen2.5-7B-shaped long-context GQA decode",
+        "llama_osa": "Llama-3.1-8B-shaped GQA decode, OSA exact-mass selection",
+        "llama_coreset": "Llama-3.1-8B-shaped GQA decode, weighted coreset m=2048",
+    }
+    return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, "
+            f"ctx={wl.Ncap}, block={wl.block_size}, read budget {budget:g} "
+            f"(top-{wl.k_top} + first + last + tail proxy)" if wl.attn_mode != "weighted" else
+            f"{names[wl.name]}: B={wl.B}, ctx={wl.Ncap}, m={wl.m} weighted tokens per KV head")
+
+
+def run_ours(args, dist):
+    import torch
+    import weighted_coreset_softmax_b200 as kv
+    from weighted_coreset_softmax_b200 import workloads as W
+
+    dev = torch.device("cuda", dist.local_rank if torch.cuda.device_count() > dist.local_rank else 0)
+    torch.cuda.set_device(dev)
+    dist.init("nccl")
+    kv.lib()
+
+    name = args.workload
+    wl = W.make(name, dev, budget=args.budget,
+                seed=(None if dist.rank == 0 else (100 if name == "llama" else 3) + shard_seed_offset(dist.rank)))
+    sl = wl.seq_lens_tensor(dev)
+    B = wl.B
+    summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
+    shape = kv.make_shape(wl.q, wl.K, sl, wl.block_size)
+    ws = kv.Workspace(shape, dev)
+    mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
+    kmax = wl.kmax
+    idx = torch.zeros(B, wl.Hkv, kmax, dtype=torch.int32, device=dev)
+    nk = torch.zeros(B, wl.Hkv, dtype=torch.int32, device=dev)
+    out = torch.empty(B, wl.Hq, wl.D, dtype=torch.float32, device=dev)
+    lse = torch.empty(B, wl.Hq, dtype=torch.float32, device=dev)
+    weighted = wl.attn_mode == "weighted"
+
+    def select():
+        if not weighted:
+            kv.kv_select_blocks(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["counts"], wl.k_top,
+                                wl.force_first, wl.force_last, mode=mode, k_sum=summ["k_sum"], kmax=kmax,
+                                block_idx=idx, n_kept=nk)
+
+    def attend():
+        if weighted:
+            kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws, tok_idx=wl.tok_idx,
+                                     w=wl.w, out=out, lse=lse)
+        else:
+            kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws, block_idx=idx,
+                                     n_kept=nk, summaries=summ, use_tail_proxy=True, out=out, lse=lse)
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        select()
+        attend()
+    torch.cuda.synchronize(dev)
+    if kv.kv_workspace_status(ws.tensor) != 0:
+        raise RuntimeError("device checks failed during warm-up")
+
+    K_steps = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K_steps)]
+    clocks = ClockSampler(dev.index)
+    clocks.start()
+    time.sleep(0.1)
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    w0 = time.time()
+    for i in range(K_steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        select()
+        ev[i][1].record(stream)
+        attend()
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(dev)
+    w1 = time.time()
+    dist.barrier(dev)
+    clk = clocks.stop(w0, w1)
+    sel_ms = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K_steps)]
+    att_ms = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K_steps)]
+    step_ms_local = statistics.fmean(a + b for a, b in zip(sel_ms, att_ms))
+    step_ms = dist.max(step_ms_local, dev)
+    sel_avg, att_avg = statistics.fmean(sel_ms), statistics.fmean(att_ms)
+
+    # end to end through the public API: q from pinned host memory in, out/lse back
+    q_host = wl.q.detach().cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+    q_dev = wl.q
+    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
+    dist.barrier(dev)
+    torch.cuda.synchronize(dev)
+    for i in range(K_steps):
+        flush.zero_()
+        e2e_ev[i][0].record(stream)
+        q_dev.copy_(q_host, non_blocking=True)
+        select()
+        attend()
+        out_host.copy_(out, non_blocking=True)
+        lse_host.copy_(lse, non_blocking=True)
+        e2e_ev[i][1].record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier(dev)
+    e2e_ms = dist.max(statistics.fmean(e[0].elapsed_time(e[1]) for e in e2e_ev), dev)
+
+    # the dense baseline on the identical cache
+    dense = None
+    if not args.no_dense and not weighted:
+        dws = ws
+        dout = torch.empty_like(out)
+        dl = torch.empty_like(lse)
+        for _ in range(2):
+            kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, dws, out=dout, lse=dl)
+        dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(10)]
+        for i in range(10):
+            flush.zero_()
+            dev_ev[i][0].record(stream)
+            kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, dws, out=dout, lse=dl)
+            dev_ev[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        d_ms = statistics.fmean(e[0].elapsed_time(e[1]) for e in dev_ev)
+        dbytes = sum(wl.Hkv * wl.seq_lens[b] * wl.D * 2 * 2 for b in range(B))
+        dense = {"ms": d_ms, "GB_s": dbytes / (d_ms * 1e-3) / 1e9, "bytes": dbytes,
+                 "speedup_attn_kernel": d_ms / att_avg, "speedup_step": d_ms / step_ms_local}
+
+    torch.cuda.synchronize(dev)
+    if kv.kv_workspace_status(ws.tensor) != 0:
+        raise RuntimeError("device checks failed during timing")
+
+    # algorithmic bytes and the roofline of the dominant kernel
+    if weighted:
+        a_bytes, s_bytes = weighted_bytes(wl), 0
+    else:
+        a_bytes = attention_bytes(wl, nk, wl.seq_lens)
+        s_bytes = select_bytes(wl, wl.seq_lens) if mode == kv.KV_SCORE_SUMMARY else osa_select_bytes(wl, wl.seq_lens)
+    peak, peak_kind = measured_peak_hbm()
+    if att_avg >= sel_avg or weighted:
+        dom, dom_bytes, dom_ms = "kv_sparse_decode_attn", a_bytes, att_avg
+    else:
+        dom, dom_bytes, dom_ms = "kv_select_blocks", s_bytes, sel_avg
+    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    step_gbs = (a_bytes + s_bytes) / (step_ms_local * 1e-3) / 1e9
+
+    queries = B * dist.world
+    res = {
+        "metric": METRIC,
+        "value": queries / (step_ms * 1e-3),
+        "unit": "queries/s",
+        "n_gpus": dist.world,
+        "steps": K_steps,
+        "warmup": args.warmup,
+        "ms_per_step": step_ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded bf16 caches shaped like the pages' workloads)",
+        "config": {
+            "workload": workload_label(wl, args.budget),
+            "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "ctx": wl.Ncap,
+            "block": wl.block_size, "k_top": wl.k_top, "kmax": kmax, "kv_dtype": "bf16",
+            "parallelism": f"replicas: batch-sharded, {dist.world} rank(s), no collective",
+            "l2": "flushed before every step (512 MiB write), outside the timed events",
+            "step": "kv_select_blocks + kv_sparse_decode_attn" if not weighted else "kv_sparse_decode_attn",
+        },
+        "achieved_step_GB_s": step_gbs,
+        "achieved_step_pct_of_8TBs": 100.0 * step_gbs / NOMINAL_HBM_GBS,
+        "kernels_ms": {"kv_select_blocks": sel_avg, "kv_sparse_decode_attn": att_avg},
+        "bytes_per_launch": {"kv_select_blocks": s_bytes, "kv_sparse_decode_attn": a_bytes},
+        "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "pct_of_8TBs": 100.0 * achieved / NOMINAL_HBM_GBS},
+        "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
+                "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * 4 + lse_host.numel() * 4, "ms_per_step": e2e_ms},
+        "gpu_launches": (1 if weighted else 2) * K_steps,
+        "clocks": clk,
+        "dense": dense,
+    }
+    if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, workload_label(wl, args.budget))
+    dist.close()
+    return res
+
+
+# ----------------------------------------------------------------- reference arm
+def run_reference(args, dist):
+    """The float64 oracle on the host cores, rank 0 only; same metric and config."""
+    if dist.rank != 0:
+        return None
+    import torch
+    from weighted_coreset_softmax_b200 import workloads as W
+    _pool_init()
+    name = args.workload
+    # a bounded sample of the same workload: the first sequences of the batch
+    nseq = 4
+    wl = W.make(name, "cpu", budget=args.budget, B=nseq)
+    workers = max(1, min(os.cpu_count() or 1, 32))
+    steps = args.steps
+    # one step = one (sequence, KV head) decode step; capped so the run stays short
+    t_one = time.perf_counter()
+    _oracle_task(oracle_tasks(wl, [(0, 0)])[0])
+    t_one = time.perf_counter() - t_one
+    cap = int(max(workers, 90.0 * workers / max(t_one, 1e-3)))
+    n = min(steps, cap)
+    if args.warmup:
+        time_oracle(wl, min(args.warmup, workers), workers)
+    dt, n = time_oracle(wl, n, workers)
+    queries = n / wl.Hkv
+    value = queries / dt
+    sample = (f"{n} (sequence, KV head) decode steps = {queries:g} queries from the first {nseq} sequences "
+              f"of the workload; float64 NumPy oracle, {workers} spawn workers, 1 BLAS thread each")
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": dist.world,
+        "steps": n, "warmup": args.warmup, "ms_per_step": dt / n * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_label(wl, args.budget) + f" (sample of {nseq} sequences)",
+                   "parallelism": "host CPU pool"},
+        "cpu_baseline": {"value": value, "unit": "queries/s", "cores": workers, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    dist = Dist()
+    if args.impl == "reference":
+        res = run_reference(args, dist)
+    else:
+        res = run_ours(args, dist)
+    if res is not None and dist.rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,216 @@
+/*
+ * kvsparse.h -- C ABI of the reduced-KV softmax decode-attention library
+ * (libkvsparse.so, CUDA kernels for sm_100a).
+ *
+ * The method, per decode step of one layer:
+ *   1. Once after prefill, every block of L cached tokens is summarised by its
+ *      key sum, value sum and token count (kv_build_block_summaries).
+ *   2. Each KV head scores its blocks for the current query group and keeps the
+ *      top-k by the GQA-normalised group score (kv_select_blocks).
+ *   3. Attention runs exactly over the kept blocks' tokens plus one count-aware
+ *      proxy token standing for the unread tail (kv_sparse_decode_attn), or over
+ *      an explicitly weighted coreset; kv_dense_decode_attn is exact attention
+ *      over every token, the baseline.
+ *
+ * Conventions shared by every entry point
+ *   - Pointers named K, V, q, k_sum, ... are DEVICE pointers unless stated.
+ *     The library never allocates device memory; the caller owns every buffer.
+ *   - Layouts are dense row-major, C order:
+ *       q        [B][Hq][D]         dtype of the shape
+ *       K, V     [B][Hkv][Ncap][D]  dtype of the shape
+ *       out      [B][Hq][D]         fp32
+ *       lse      [B][Hq]            fp32, natural log of the softmax normaliser
+ *     Query head g reads KV head g / G, G = Hq / Hkv.
+ *   - Every call is asynchronous on `stream` and returns before the kernels run.
+ *     Argument errors are reported BEFORE anything is launched.
+ *   - Sizes: D in {64, 128}; 1 <= G <= 8; L (block_size) in {16, 32, 64, 128};
+ *     dtype bf16 or fp32; NBcap = ceil(Ncap / L) <= 4096. Other shapes return
+ *     KV_ERR_UNSUPPORTED. Every device pointer must be 16-byte aligned.
+ *   - Values that live on the device (seq_lens, block indices, token indices)
+ *     cannot be checked by the host. The kernels check them and never read out
+ *     of bounds: a bad entry is skipped and a bit is set in the workspace status
+ *     word (kv_workspace_status), after which results are unspecified.
+ *   - Thread safety: calls are re-entrant. The last error message is kept per
+ *     host thread (kv_last_error). Calls that share one workspace must be
+ *     ordered on the device (same stream, or events); overlapping ones race.
+ */
+#ifndef KVSPARSE_H
+#define KVSPARSE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* kv_stream_t;
+
+typedef enum {
+  KV_OK = 0,
+  KV_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size; nothing launched  */
+  KV_ERR_UNSUPPORTED = 2,   /* valid but not built: D, G, L, dtype or NBcap         */
+  KV_ERR_CUDA = 3,          /* a CUDA call or launch failed (see kv_last_error)      */
+  KV_ERR_DEVICE_CHECK = 4   /* kv_workspace_status found a device-side check failed  */
+} kv_status;
+
+typedef enum { KV_BF16 = 0, KV_F32 = 1 } kv_dtype;
+
+typedef enum {
+  KV_SCORE_SUMMARY = 0,     /* first-order mean-pool score from the block sums       */
+  KV_SCORE_EXACT_MASS = 1   /* exact block log-mass from all block keys (OSA)        */
+} kv_score_mode;
+
+/* Device-status bits written into the workspace by the attention kernels. */
+#define KV_DEV_BAD_BLOCK_INDEX  0x1u  /* block index out of range or not ascending   */
+#define KV_DEV_BAD_TOKEN_INDEX  0x2u  /* coreset token index outside [0, seq_len)    */
+#define KV_DEV_BAD_SEQ_LEN      0x4u  /* seq_len outside [0, Ncap]                   */
+#define KV_DEV_BAD_N_KEPT       0x8u  /* n_kept outside [0, kmax]                    */
+#define KV_DEV_WAIT_TIMEOUT     0x10u /* a bounded wait on a copy gave up            */
+
+typedef struct {
+  int B;                    /* sequences in the batch, >= 0                          */
+  int Hq;                   /* query heads                                           */
+  int Hkv;                  /* KV heads; Hq % Hkv == 0                               */
+  int D;                    /* head dimension                                        */
+  int Ncap;                 /* allocated tokens per (sequence, KV head), >= 1        */
+  int block_size;           /* L, tokens per block                                   */
+  kv_dtype dtype;           /* element type of q, K and V                            */
+  const int32_t* seq_lens;  /* device [B]: tokens actually cached, 0..Ncap           */
+} kv_shape;
+
+/*
+ * kv_build_block_summaries -- per-block key sum, value sum and token count.
+ *
+ * Source: "COBS: Cumulant Order Block Sparse Attention", the affine score (18)
+ * (mean-pool summary: phi_b = block mean key, a_b = ln L) and the paragraph that
+ * stores the mean key per block; "OpenAttention reads 1% of the KV cache --
+ * Count-aware tail proxy" (the proxy needs the unread tail's mean key and value,
+ * obtained from the totals minus the kept blocks' sums).
+ *
+ * Writes, for every (b, h, block) with block < NBcap:
+ *   k_sum, v_sum [B][Hkv][NBcap][D] fp32  sums over the block's tokens < seq_len
+ *   counts       [B][NBcap] int32         min(L, seq_len - block*L) clamped at 0
+ *   k_tot, v_tot [B][Hkv][D] fp32         sums over all tokens < seq_len
+ * Blocks at or past ceil(seq_len / L) get zero sums and count 0. Accumulation is
+ * fp32; the totals are summed from the block sums in a fixed order, so results
+ * are bit-reproducible. Run once after prefill (and again if the cache changes).
+ */
+kv_status kv_build_block_summaries(const kv_shape* shape, const void* K, const void* V,
+                                   float* k_sum, float* v_sum, int32_t* counts,
+                                   float* k_tot, float* v_tot, kv_stream_t stream);
+
+/*
+ * kv_select_blocks -- per-KV-head block choice for one decode step.
+ *
+ * Source: "COBS: Cumulant Order Block Sparse Attention" -- Equation (5), the
+ * GQA-normalised group score (a sum over the group's query heads of per-head
+ * block softmax probabilities, normaliser Z^(g,h) of (5)); the first-order
+ * mean-pool estimate of ln m_b (text after Equation (8), affine score (18)); the
+ * OSA paragraph for KV_SCORE_EXACT_MASS.
+ *
+ *   summary mode:  s[g,b] = scale * q_g . (k_sum_b / n_b) + ln n_b
+ *   exact mode:    s[g,b] = ln sum_{r in b} exp(scale * q_g . k_r)   (reads all K)
+ *   S[b] = sum_{g in group} exp(s[g,b] - ln sum_b' exp(s[g,b']))      over valid b'
+ *
+ * Forced blocks (block 0 if force_first, block ceil(n/L)-1 if force_last) are
+ * always kept and do not compete. The other valid blocks are ranked by
+ * (S descending, block index ascending) and the first min(k_top, candidates)
+ * are kept.
+ *
+ *   q          device [B][Hq][D], dtype of the shape
+ *   scale      softmax scale applied to q.k (e.g. 1/sqrt(D))
+ *   k_sum      device, from kv_build_block_summaries (summary mode; may be NULL
+ *              in exact mode)
+ *   counts     device [B][NBcap] from kv_build_block_summaries (both modes)
+ *   K          device cache (exact mode only; may be NULL in summary mode)
+ *   kmax       row stride of block_idx; must be >= min(NBcap, k_top + forced)
+ *   block_idx  device out [B][Hkv][kmax] int32: kept block indices, ascending;
+ *              entries past n_kept are left unchanged
+ *   n_kept     device out [B][Hkv] int32
+ *   scores     device out [B][Hkv][NBcap] fp32 S[b] (0 for invalid blocks), or NULL
+ */
+kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale,
+                           kv_score_mode mode, const float* k_sum, const int32_t* counts,
+                           const void* K, int k_top, int force_first, int force_last,
+                           int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                           kv_stream_t stream);
+
+/*
+ * kv_sparse_decode_attn -- softmax attention over a reduced KV cache.
+ *
+ * Block mode (tok_idx == NULL). Source: "OpenAttention reads 1% of the KV cache
+ * -- Count-aware tail proxy", section "Skipping reviews without losing the
+ * verdict": exact attention over the kept blocks' tokens plus, if use_tail_proxy,
+ * one virtual token for the n_T unread tokens whose value is their mean value and
+ * whose logit is scale * q . (their mean key) + ln n_T (their mean logit plus the
+ * log of their count). The tail means come from the block sums:
+ * (k_tot - sum of kept k_sum) / n_T. With use_tail_proxy = 0 the tail is dropped
+ * and the kept tokens are renormalised (top-k discard).
+ *   block_idx [B][Hkv][kmax], n_kept [B][Hkv]: kept blocks, strictly ascending,
+ *   each < ceil(seq_len / L) (kv_select_blocks output, or the caller's own).
+ *   k_sum, v_sum, counts, k_tot, v_tot: kv_build_block_summaries output; needed
+ *   only when use_tail_proxy != 0 (else may be NULL).
+ *
+ * Weighted-coreset mode (tok_idx != NULL). Source: "WildCat: Near-Linear
+ * Attention in Theory and Practice", abstract: attention over a small weighted
+ * coreset, token i entering the softmax with logit scale * q . k_i + ln w_i.
+ *   tok_idx [B][Hkv][m] int32 token positions (< seq_len), w [B][Hkv][m] fp32
+ *   weights (>= 0; 0 excludes the token). No proxy; block arguments ignored.
+ *
+ *   out [B][Hq][D] fp32; lse [B][Hq] fp32 or NULL. A head with no token and no
+ *   proxy gets out = 0 and lse = -inf.
+ *   workspace: device, >= kv_workspace_bytes(shape) bytes, zeroed once before
+ *   its first use (kv_workspace_init); every call leaves it ready for the next.
+ */
+kv_status kv_sparse_decode_attn(const kv_shape* shape, const void* q, float scale,
+                                const void* K, const void* V,
+                                const int32_t* block_idx, const int32_t* n_kept, int kmax,
+                                const float* k_sum, const float* v_sum, const int32_t* counts,
+                                const float* k_tot, const float* v_tot, int use_tail_proxy,
+                                const int32_t* tok_idx, const float* w, int m,
+                                float* out, float* lse, void* workspace, size_t ws_bytes,
+                                kv_stream_t stream);
+
+/*
+ * kv_dense_decode_attn -- exact softmax attention over every cached token, the
+ * baseline the reduced path is measured against. Source: "COBS: Cumulant Order
+ * Block Sparse Attention", the read-traffic accounting ("Dense reads the whole
+ * KV cache"); "OpenAttention reads 1% of the KV cache", section "The news" (the
+ * decode-attention speed comparison against dense attention).
+ * Arguments as in kv_sparse_decode_attn.
+ */
+kv_status kv_dense_decode_attn(const kv_shape* shape, const void* q, float scale,
+                               const void* K, const void* V, float* out, float* lse,
+                               void* workspace, size_t ws_bytes, kv_stream_t stream);
+
+/*
+ * kv_workspace_bytes -- device workspace the attention entry points need for
+ * this shape (split partial results, arrival counters, a status word). The size
+ * depends only on B, Hkv, G and D. Returns 0 for an invalid shape pointer.
+ */
+size_t kv_workspace_bytes(const kv_shape* shape);
+
+/*
+ * kv_workspace_init -- zeroes the counters and the status word of a workspace
+ * (an async memset on `stream`). Needed once after allocation; calls leave the
+ * counters at zero, and the status word keeps its bits until the next init.
+ */
+kv_status kv_workspace_init(void* workspace, size_t ws_bytes, kv_stream_t stream);
+
+/*
+ * kv_workspace_status -- synchronises `stream`, then copies the workspace status
+ * word (KV_DEV_* bits) to *status_out (host pointer). Returns KV_ERR_DEVICE_CHECK
+ * if any bit is set, KV_OK otherwise.
+ */
+kv_status kv_workspace_status(const void* workspace, uint32_t* status_out, kv_stream_t stream);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* kv_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVSPARSE_H */

@@ -21,3 +21,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session", autouse=True)
+def _built_library():
+    """Builds libkvsparse.so in-tree when it is missing or older than its sources
+    (nvcc cross-compiles for sm_100a without a GPU)."""
+    from weighted_coreset_softmax_b200 import build
+    build.build()
+    yield

@@ -1,0 +1,353 @@
+"""GPU parity: every kernel against the float64 oracle on the same seeded inputs.
+
+Small cases compare every output element and span several chunks, several CTAs
+per head and ragged tails; the full-size cases (the benchmark's launch
+configuration) compare sampled heads the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import weighted_coreset_softmax_b200 as kv
+from weighted_coreset_softmax_b200 import workloads as W
+from oracle import oracle as O
+from gpu_helpers import (OUT_TOL, all_pairs, check_out, kept_tensor, oracle_inputs, row_rel_err,
+                         run_pipeline, selection_matches, to64)
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+# ------------------------------------------------------------------ summaries
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", {}),
+    ("llama", dict(B=3, Ncap=4160, seq_lens=[4160, 3001, 1])),
+    ("qwen_long", dict(B=2, Ncap=2048 + 100, seq_lens=[2148, 700])),
+])
+def test_block_summaries(name, kw):
+    wl = W.make(name, DEV, **kw)
+    sl = wl.seq_lens_tensor(DEV)
+    s = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
+    torch.cuda.synchronize()
+    q, K, V = oracle_inputs(wl)
+    ks, vs, c, kt, vt = O.build_block_summaries(K, V, wl.seq_lens, wl.block_size)
+    assert np.array_equal(s["counts"].cpu().numpy(), c)
+    for got, ref, nm in ((s["k_sum"], ks, "k_sum"), (s["v_sum"], vs, "v_sum"),
+                         (s["k_tot"], kt, "k_tot"), (s["v_tot"], vt, "v_tot")):
+        g = got.cpu().numpy().astype(np.float64)
+        scale = np.maximum(1.0, np.abs(ref).max(axis=-1, keepdims=True))
+        err = float(np.max(np.abs(g - ref) / scale))
+        assert err < 2e-5, f"{nm} err {err:.3e}"
+
+
+# ------------------------------------------------------------- tiny workload
+def test_tiny_pipeline():
+    """Single head, d=64, n=1024 in 64 blocks of 16, fp32: top-8 + proxy."""
+    wl = W.make("tiny", DEV)
+    r = run_pipeline(wl)
+    q, K, V = oracle_inputs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, wl.block_size, wl.scale, wl.k_top, False, False, "summary")
+    selection_matches(r["idx"], r["nk"], sel, all_pairs(wl), "tiny select")
+    S = r["scores"].cpu().numpy()[0, 0].astype(np.float64)
+    assert np.max(np.abs(S - sel[(0, 0)]["S"])) < 1e-4
+    kept = {k: v["kept"] for k, v in sel.items()}
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, kept, True)
+    check_out(r["out"], r["lse"], ro, rl, what="tiny proxy")
+
+
+def test_tiny_all_kept_equals_dense():
+    wl = W.make("tiny", DEV, k_top=64)
+    r = run_pipeline(wl)
+    assert int(r["nk"][0, 0]) == 64
+    q, K, V = oracle_inputs(wl)
+    do, dl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
+    check_out(r["out"], r["lse"], do, dl, what="all kept vs oracle dense")
+    go, gl = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, r["sl"], wl.block_size, wl.scale, r["ws"])
+    check_out(go, gl, do, dl, what="gpu dense")
+
+
+def test_tiny_equal_tail_proxy_exact():
+    """Tail keys set equal: the proxy must reproduce dense attention."""
+    wl = W.make("tiny", DEV)
+    q, K, V = oracle_inputs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, wl.block_size, wl.scale, wl.k_top, False, False, "summary")
+    kept = [[sel[(0, 0)]["kept"]]]
+    W.equalize_tail(wl, kept)
+    q, K, V = oracle_inputs(wl)
+    sl = wl.seq_lens_tensor(DEV)
+    summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
+    idx, nk = kept_tensor({(0, 0): sel[(0, 0)]}, 1, 1, 8, DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        block_idx=idx, n_kept=nk, summaries=summ)
+    do, dl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, {(0, 0): kept[0][0]}, True)
+    assert np.max(np.abs(ro - do)) < 1e-12  # oracle: proxy exact
+    check_out(out, lse, do, dl, what="equal tail vs dense")
+
+
+# -------------------------------------------------- small multi-head workloads
+SMALL = [
+    ("llama", dict(B=3, Ncap=4160, seq_lens=[4160, 3001, 70], budget=0.05)),
+    ("llama", dict(B=2, Ncap=2048, seq_lens=[2048, 1], k_top=3)),
+    ("qwen_long", dict(B=2, Ncap=4096 + 128 + 5, seq_lens=[4229, 2000], k_top=4)),
+]
+
+
+@pytest.mark.parametrize("name,kw", SMALL)
+@pytest.mark.parametrize("use_proxy", [True, False])
+def test_small_pipeline(name, kw, use_proxy):
+    wl = W.make(name, DEV, **kw)
+    r = run_pipeline(wl, use_proxy=use_proxy)
+    q, K, V = oracle_inputs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, wl.block_size, wl.scale, wl.k_top, True, True, "summary")
+    selection_matches(r["idx"], r["nk"], sel, all_pairs(wl), f"{name} select")
+    # attention parity on the GPU's own kept sets (index parity checked above)
+    gi, gn = r["idx"].cpu().numpy(), r["nk"].cpu().numpy()
+    kept = {(b, h): [int(x) for x in gi[b, h, :gn[b, h]]] for (b, h) in all_pairs(wl)}
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, kept, use_proxy)
+    check_out(r["out"], r["lse"], ro, rl, what=f"{name} attention proxy={use_proxy}")
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("llama", dict(B=2, Ncap=3000, seq_lens=[3000, 1234])),
+    ("qwen_long", dict(B=2, Ncap=1500, seq_lens=[1500, 3])),
+    ("tiny", dict(B=1)),
+])
+def test_dense(name, kw):
+    wl = W.make(name, DEV, **kw)
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws)
+    q, K, V = oracle_inputs(wl)
+    do, dl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
+    check_out(out, lse, do, dl, what=f"dense {name}")
+
+
+@pytest.mark.parametrize("m", [1, 37, 300])
+def test_weighted(m):
+    wl = W.make("llama_coreset", DEV, B=2, Ncap=2500, seq_lens=[2500, 900], m=m)
+    wl.w[0, 0, ::5] = 0.0  # some zero weights: excluded tokens
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        tok_idx=wl.tok_idx, w=wl.w)
+    torch.cuda.synchronize()
+    assert kv.kv_workspace_status(ws.tensor) == 0
+    q, K, V = oracle_inputs(wl)
+    ro, rl = O.weighted_batch(q, K, V, wl.seq_lens, wl.tok_idx.cpu().numpy(),
+                              wl.w.cpu().numpy().astype(np.float64), wl.scale)
+    check_out(out, lse, ro, rl, what=f"weighted m={m}")
+
+
+def test_weighted_integer_weights_duplication():
+    """Integer weights equal attention over a cache with w-fold duplicated tokens."""
+    wl = W.make("llama_coreset", DEV, B=1, Ncap=512, m=64)
+    g = torch.Generator(device="cpu").manual_seed(5)
+    # one weight pattern for every head, so all heads' duplicated caches are equally long
+    wint = torch.randint(1, 5, (1, 1, 64), generator=g).to(torch.float32).expand(1, wl.Hkv, 64).contiguous()
+    wl.w = wint.to(DEV)
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        tok_idx=wl.tok_idx, w=wl.w)
+    # duplicated cache, dense GPU attention over it
+    idx = wl.tok_idx.cpu()
+    reps = wint.to(torch.int64)
+    n_dup = int(reps.sum(dim=-1).max())
+    Kd = torch.zeros(1, wl.Hkv, n_dup, wl.D, dtype=wl.dtype)
+    Vd = torch.zeros_like(Kd)
+    lens = []
+    for h in range(wl.Hkv):
+        rows = torch.repeat_interleave(idx[0, h].to(torch.int64), reps[0, h])
+        Kd[0, h, :len(rows)] = wl.K[0, h].cpu()[rows]
+        Vd[0, h, :len(rows)] = wl.V[0, h].cpu()[rows]
+        lens.append(len(rows))
+    assert len(set(lens)) == 1
+    sl2 = torch.tensor(lens[:1], dtype=torch.int32, device=DEV)
+    Kd, Vd = Kd.to(DEV), Vd.to(DEV)
+    ws2 = kv.Workspace(kv.make_shape(wl.q, Kd, sl2, 64), DEV)
+    do, dl = kv.kv_dense_decode_attn(wl.q, Kd, Vd, sl2, 64, wl.scale, ws2)
+    torch.cuda.synchronize()
+    err = float((out - do).abs().max() / do.abs().max())
+    assert err < 2e-5, err
+    assert float((lse - dl).abs().max()) < 1e-4
+
+
+@pytest.mark.parametrize("G,D,dtype", [(2, 64, torch.bfloat16), (4, 128, torch.float32),
+                                       (1, 128, torch.bfloat16), (8, 64, torch.float32),
+                                       (3, 128, torch.bfloat16), (5, 64, torch.bfloat16)])
+def test_shape_coverage(G, D, dtype):
+    """Head dims, group sizes and dtypes beyond the named workloads."""
+    B, Hkv, N, L = 2, 2, 1000, 32
+    g = torch.Generator(device=DEV).manual_seed(G * 100 + D)
+    q = torch.randn(B, Hkv * G, D, generator=g, device=DEV).to(dtype)
+    K = torch.randn(B, Hkv, N, D, generator=g, device=DEV).to(dtype)
+    V = torch.randn(B, Hkv, N, D, generator=g, device=DEV).to(dtype)
+    lens = [1000, 517]
+    sl = torch.tensor(lens, dtype=torch.int32, device=DEV)
+    scale = 1 / math.sqrt(D)
+    summ = kv.kv_build_block_summaries(K, V, sl, L)
+    idx, nk, _ = kv.kv_select_blocks(q, K, sl, L, scale, summ["counts"], 4, True, True, k_sum=summ["k_sum"])
+    ws = kv.Workspace(kv.make_shape(q, K, sl, L), DEV)
+    out, lse = kv.kv_sparse_decode_attn(q, K, V, sl, L, scale, ws, block_idx=idx, n_kept=nk, summaries=summ)
+    dout, dlse = kv.kv_dense_decode_attn(q, K, V, sl, L, scale, ws)
+    torch.cuda.synchronize()
+    q64, K64, V64 = to64(q), to64(K), to64(V)
+    sel = O.select_batch(q64, K64, lens, L, scale, 4, True, True, "summary")
+    pairs = [(b, h) for b in range(B) for h in range(Hkv)]
+    selection_matches(idx, nk, sel, pairs, "coverage select")
+    gi, gn = idx.cpu().numpy(), nk.cpu().numpy()
+    kept = {p: [int(x) for x in gi[p[0], p[1], :gn[p]]] for p in pairs}
+    ro, rl = O.sparse_batch(q64, K64, V64, lens, L, scale, kept, True)
+    check_out(out, lse, ro, rl, what=f"coverage sparse G={G} D={D} {dtype}")
+    do, dl = O.dense_batch(q64, K64, V64, lens, scale)
+    check_out(dout, dlse, do, dl, what=f"coverage dense G={G} D={D} {dtype}")
+
+
+def test_exact_mass_small():
+    wl = W.make("llama_osa", DEV, B=2, Ncap=3000, seq_lens=[3000, 1100])
+    r = run_pipeline(wl)
+    q, K, V = oracle_inputs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, wl.block_size, wl.scale, wl.k_top, True, True, "exact_mass")
+    selection_matches(r["idx"], r["nk"], sel, all_pairs(wl), "exact-mass select")
+    S = r["scores"].cpu().numpy().astype(np.float64)
+    for (b, h) in all_pairs(wl):
+        nb = len(sel[(b, h)]["S"])
+        assert np.max(np.abs(S[b, h, :nb] - sel[(b, h)]["S"])) < 1e-4
+
+
+# ------------------------------------------------------------------ edge cases
+def test_edge_cases():
+    """Empty sequence, one token, k = 0 (proxy only), n_kept below kmax."""
+    wl = W.make("llama", DEV, B=4, Ncap=640, seq_lens=[0, 1, 640, 200], k_top=0)
+    r = run_pipeline(wl, kmax=5)
+    nk = r["nk"].cpu().numpy()
+    assert list(nk[0]) == [0] * wl.Hkv and list(nk[1]) == [1] * wl.Hkv
+    q, K, V = oracle_inputs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, wl.block_size, wl.scale, 0, True, True, "summary")
+    selection_matches(r["idx"], r["nk"], sel, all_pairs(wl), "edge select")
+    kept = {k: v["kept"] for k, v in sel.items()}
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, kept, True)
+    out = r["out"].cpu().numpy()
+    assert np.all(out[0] == 0) and np.all(np.isneginf(r["lse"].cpu().numpy()[0]))
+    check_out(r["out"], r["lse"], ro, rl, what="edge cases")
+
+
+def test_weighted_all_zero_and_m_zero():
+    wl = W.make("llama_coreset", DEV, B=1, Ncap=256, m=16)
+    wl.w.zero_()
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        tok_idx=wl.tok_idx, w=wl.w)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+    e = torch.zeros(1, wl.Hkv, 0, dtype=torch.int32, device=DEV)
+    ew = torch.zeros(1, wl.Hkv, 0, dtype=torch.float32, device=DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        tok_idx=e, w=ew)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+
+
+def test_device_checks_flag_bad_indices():
+    """Out-of-range block and token indices are skipped and flagged, not read."""
+    wl = W.make("llama", DEV, B=1, Ncap=640, k_top=2)
+    sl = wl.seq_lens_tensor(DEV)
+    summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, 64)
+    idx = torch.tensor([[[0, 3, 10_000, 9]] * wl.Hkv], dtype=torch.int32, device=DEV)
+    nk = torch.full((1, wl.Hkv), 4, dtype=torch.int32, device=DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, 64), DEV)
+    kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, 64, wl.scale, ws, block_idx=idx, n_kept=nk,
+                             summaries=summ)
+    st = kv.kv_workspace_status(ws.tensor)
+    assert st & 0x1, hex(st)
+    kv.kv_workspace_init(ws.tensor)
+    tok = torch.tensor([[[5, 700, -3, 2]] * wl.Hkv], dtype=torch.int32, device=DEV)
+    w = torch.ones(1, wl.Hkv, 4, dtype=torch.float32, device=DEV)
+    kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, 64, wl.scale, ws, tok_idx=tok, w=w)
+    st = kv.kv_workspace_status(ws.tensor)
+    assert st & 0x2, hex(st)
+
+
+def test_deterministic_repeat():
+    wl = W.make("llama", DEV, B=2, Ncap=4096)
+    a = run_pipeline(wl)
+    b = run_pipeline(wl)
+    assert torch.equal(a["idx"], b["idx"]) and torch.equal(a["out"], b["out"])
+    assert torch.equal(a["summ"]["k_tot"], b["summ"]["k_tot"])
+
+
+# ------------------------------------------------------ full-size, sampled
+FULL = [
+    ("llama", dict(budget=0.01)),
+    ("llama", dict(budget=0.05)),
+    ("qwen_long", dict(budget=0.01)),
+    ("llama_osa", dict()),
+]
+
+
+@pytest.mark.parametrize("name,kw", FULL)
+def test_full_size_sampled(name, kw):
+    wl = W.make(name, DEV, **kw)
+    r = run_pipeline(wl)
+    gen = np.random.default_rng(7)
+    pairs = sorted({(int(gen.integers(wl.B)), int(gen.integers(wl.Hkv))) for _ in range(3)}
+                   | {(0, 0), (wl.B - 1, wl.Hkv - 1)})
+    q = to64(wl.q)
+    K = {}
+    res_sel, res_out = {}, {}
+    for (b, h) in pairs:
+        Kb = to64(wl.K[b:b + 1, h:h + 1])
+        Vb = to64(wl.V[b:b + 1, h:h + 1])
+        qb = q[b:b + 1, h * wl.G:(h + 1) * wl.G]
+        sel = O.select_batch(qb, Kb, [wl.seq_lens[b]], wl.block_size, wl.scale, wl.k_top,
+                             True, True, wl.score_mode)
+        res_sel[(b, h)] = sel[(0, 0)]
+        gi = r["idx"][b, h, :int(r["nk"][b, h])].cpu().tolist()
+        o, l, _ = O.sparse_attend_one(qb[0], Kb[0, 0], Vb[0, 0], wl.seq_lens[b], wl.block_size,
+                                      gi, wl.scale, True)
+        res_out[(b, h)] = (o, l)
+    selection_matches(r["idx"], r["nk"], res_sel, pairs, f"full {name} select")
+    go = r["out"].cpu().numpy().astype(np.float64)
+    gl = r["lse"].cpu().numpy().astype(np.float64)
+    for (b, h), (o, l) in res_out.items():
+        sl_ = slice(h * wl.G, (h + 1) * wl.G)
+        err = row_rel_err(go[b, sl_], o)
+        assert err <= OUT_TOL, f"full {name} {(b, h)}: {err:.3e}"
+        assert np.max(np.abs(gl[b, sl_] - l)) <= OUT_TOL * max(1.0, float(np.max(np.abs(l))))
+
+
+def test_full_size_weighted_sampled():
+    wl = W.make("llama_coreset", DEV)
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
+                                        tok_idx=wl.tok_idx, w=wl.w)
+    torch.cuda.synchronize()
+    assert kv.kv_workspace_status(ws.tensor) == 0
+    q = to64(wl.q)
+    for (b, h) in [(0, 0), (13, 5), (31, 7)]:
+        qb = q[b, h * wl.G:(h + 1) * wl.G]
+        o, l = O.weighted_attend_one(qb, to64(wl.K[b, h]), to64(wl.V[b, h]), wl.seq_lens[b],
+                                     wl.tok_idx[b, h].cpu().numpy(),
+                                     wl.w[b, h].cpu().numpy().astype(np.float64), wl.scale)
+        err = row_rel_err(out[b, h * wl.G:(h + 1) * wl.G].cpu().numpy().astype(np.float64), o)
+        assert err <= OUT_TOL, err
+
+
+def test_full_size_dense_sampled():
+    wl = W.make("llama", DEV)
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws)
+    torch.cuda.synchronize()
+    q = to64(wl.q)
+    for (b, h) in [(0, 0), (17, 3), (31, 7)]:
+        qb = q[b, h * wl.G:(h + 1) * wl.G]
+        o, l = O.dense_attend_one(qb, to64(wl.K[b, h]), to64(wl.V[b, h]), wl.seq_lens[b], wl.scale)
+        err = row_rel_err(out[b, h * wl.G:(h + 1) * wl.G].cpu().numpy().astype(np.float64), o)
+        assert err <= OUT_TOL, err

@@ -1,0 +1,304 @@
+"""Reduced-KV softmax decode attention for B200 (sm_100a).
+
+Thin Python binding of libkvsparse.so (C ABI declared in include/kvsparse.h).
+The functions keep the C names; they only marshal torch tensors into pointers,
+sizes and the current CUDA stream. Every step of the computation runs in the
+library's CUDA kernels; there is no fallback: if the library is missing or no GPU
+is present the calls raise.
+
+Method (see include/kvsparse.h for the per-call sources):
+  kv_build_block_summaries  once after prefill: per-block key/value sums, counts
+  kv_select_blocks          per step: GQA-normalised block score, top-k per KV head
+  kv_sparse_decode_attn     per step: attention over kept blocks + tail proxy, or
+                            over a weighted coreset
+  kv_dense_decode_attn      exact attention over every token (baseline)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "KV_OK", "KV_ERR_INVALID_ARG", "KV_ERR_UNSUPPORTED", "KV_ERR_CUDA", "KV_ERR_DEVICE_CHECK",
+    "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KVShape", "KVError",
+    "lib", "library_path", "header_path", "make_shape", "kv_build_block_summaries",
+    "kv_select_blocks", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_workspace_bytes",
+    "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace",
+]
+
+KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
+KV_BF16, KV_F32 = 0, 1
+KV_SCORE_SUMMARY, KV_SCORE_EXACT_MASS = 0, 1
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+_ROOT = os.path.dirname(_PKG)
+
+
+def library_path() -> str:
+    return os.path.join(_PKG, "libkvsparse.so")
+
+
+def header_path() -> str:
+    return os.path.join(_ROOT, "include", "kvsparse.h")
+
+
+class KVShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("D", ctypes.c_int), ("Ncap", ctypes.c_int), ("block_size", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("seq_lens", ctypes.c_void_p)]
+
+
+class KVError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"kvsparse status {status}: {message}")
+        self.status = status
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_S = ctypes.c_size_t
+_SHP = ctypes.POINTER(KVShape)
+
+
+def lib():
+    """Loads libkvsparse.so (once). Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing; build it with "
+                           "`python -m weighted_coreset_softmax_b200.build`")
+    L = ctypes.CDLL(path)
+    sigs = {
+        "kv_build_block_summaries": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P],
+        "kv_select_blocks": [_SHP, _P, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
+        "kv_sparse_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
+                                  _P, _P, _I, _P, _P, _P, _S, _P],
+        "kv_dense_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _P, _S, _P],
+        "kv_workspace_init": [_P, _S, _P],
+        "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
+    }
+    for name, args in sigs.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = _I
+    L.kv_workspace_bytes.argtypes = [_SHP]
+    L.kv_workspace_bytes.restype = _S
+    L.kv_last_error.argtypes = []
+    L.kv_last_error.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def header_functions():
+    """Names of the functions include/kvsparse.h declares."""
+    with open(header_path()) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kv_[a-z_]+)\s*\(", text)))
+
+
+def kv_last_error() -> str:
+    return lib().kv_last_error().decode()
+
+
+def _check(status: int):
+    if status != KV_OK:
+        raise KVError(status, kv_last_error())
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(dt: torch.dtype) -> int:
+    if dt == torch.bfloat16:
+        return KV_BF16
+    if dt == torch.float32:
+        return KV_F32
+    raise TypeError(f"unsupported cache dtype {dt}")
+
+
+def _need(t: torch.Tensor, name: str, dtype=None, cuda=True):
+    if t is None:
+        raise ValueError(f"{name} is required")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t
+
+
+def make_shape(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int) -> KVShape:
+    """Shape descriptor from q [B][Hq][D], K [B][Hkv][Ncap][D], seq_lens [B] int32."""
+    if q.dim() != 3 or K.dim() != 4:
+        raise ValueError("q must be [B][Hq][D] and K [B][Hkv][Ncap][D]")
+    B, Hq, D = q.shape
+    B2, Hkv, Ncap, D2 = K.shape
+    if B != B2 or D != D2:
+        raise ValueError(f"q {tuple(q.shape)} and K {tuple(K.shape)} disagree")
+    return KVShape(B, Hq, Hkv, D, Ncap, int(block_size), _dtype_code(K.dtype),
+                   seq_lens.data_ptr() if seq_lens is not None else None)
+
+
+def kv_workspace_bytes(shape: KVShape) -> int:
+    return int(lib().kv_workspace_bytes(ctypes.byref(shape)))
+
+
+class Workspace:
+    """A zero-initialised device workspace for the attention entry points."""
+
+    def __init__(self, shape: KVShape, device):
+        n = kv_workspace_bytes(shape)
+        self.tensor = torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+    @property
+    def nbytes(self) -> int:
+        return self.tensor.numel()
+
+    def ptr(self):
+        return ctypes.c_void_p(self.tensor.data_ptr())
+
+
+def kv_workspace_init(ws: torch.Tensor):
+    _check(lib().kv_workspace_init(_ptr(ws), ws.numel() * ws.element_size(), _stream(ws.device)))
+
+
+def kv_workspace_status(ws: torch.Tensor) -> int:
+    v = ctypes.c_uint32(0)
+    st = lib().kv_workspace_status(_ptr(ws), ctypes.byref(v), _stream(ws.device))
+    if st not in (KV_OK, KV_ERR_DEVICE_CHECK):
+        _check(st)
+    return int(v.value)
+
+
+def kv_build_block_summaries(K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                             out: Optional[dict] = None) -> dict:
+    """Block summaries of the cache; returns dict(k_sum, v_sum, counts, k_tot, v_tot)."""
+    _need(K, "K")
+    _need(V, "V", K.dtype)
+    _need(seq_lens, "seq_lens", torch.int32)
+    B, Hkv, Ncap, D = K.shape
+    NB = (Ncap + block_size - 1) // block_size
+    dev = K.device
+    if out is None:
+        out = {
+            "k_sum": torch.empty(B, Hkv, NB, D, dtype=torch.float32, device=dev),
+            "v_sum": torch.empty(B, Hkv, NB, D, dtype=torch.float32, device=dev),
+            "counts": torch.empty(B, NB, dtype=torch.int32, device=dev),
+            "k_tot": torch.empty(B, Hkv, D, dtype=torch.float32, device=dev),
+            "v_tot": torch.empty(B, Hkv, D, dtype=torch.float32, device=dev),
+        }
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, block_size, _dtype_code(K.dtype), seq_lens.data_ptr())
+    _check(lib().kv_build_block_summaries(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(out["k_sum"]),
+                                          _ptr(out["v_sum"]), _ptr(out["counts"]), _ptr(out["k_tot"]),
+                                          _ptr(out["v_tot"]), _stream(dev)))
+    return out
+
+
+def kv_select_blocks(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                     scale: float, counts: torch.Tensor, k_top: int, force_first: bool = False,
+                     force_last: bool = False, mode: int = KV_SCORE_SUMMARY,
+                     k_sum: Optional[torch.Tensor] = None, kmax: Optional[int] = None,
+                     block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                     scores: Optional[torch.Tensor] = None, want_scores: bool = False):
+    """Kept blocks per KV head. K is read only in exact-mass mode (its shape is
+    always used for the descriptor). Returns (block_idx [B][Hkv][kmax], n_kept
+    [B][Hkv], scores or None)."""
+    _need(q, "q", K.dtype)
+    _need(counts, "counts", torch.int32)
+    if mode == KV_SCORE_SUMMARY:
+        _need(k_sum, "k_sum", torch.float32)
+    else:
+        _need(K, "K")
+    shape = make_shape(q, K, seq_lens, block_size)
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    dev = q.device
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if scores is None and want_scores:
+        scores = torch.empty(shape.B, shape.Hkv, NB, dtype=torch.float32, device=dev)
+    _check(lib().kv_select_blocks(ctypes.byref(shape), _ptr(q), float(scale), int(mode), _ptr(k_sum),
+                                  _ptr(counts), _ptr(K) if mode == KV_SCORE_EXACT_MASS else None,
+                                  int(k_top), int(bool(force_first)), int(bool(force_last)), int(kmax),
+                                  _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
+    return block_idx, n_kept, scores
+
+
+def kv_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor,
+                          block_size: int, scale: float, workspace: Workspace, *,
+                          block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                          summaries: Optional[dict] = None, use_tail_proxy: bool = True,
+                          tok_idx: Optional[torch.Tensor] = None, w: Optional[torch.Tensor] = None,
+                          out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                          want_lse: bool = True):
+    """Block mode (block_idx, n_kept, summaries) or weighted-coreset mode
+    (tok_idx, w). Returns (out [B][Hq][D] fp32, lse [B][Hq] fp32 or None)."""
+    _need(q, "q", K.dtype)
+    _need(K, "K")
+    _need(V, "V", K.dtype)
+    shape = make_shape(q, K, seq_lens, block_size)
+    dev = q.device
+    if out is None:
+        out = torch.empty(shape.B, shape.Hq, shape.D, dtype=torch.float32, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty(shape.B, shape.Hq, dtype=torch.float32, device=dev)
+    kmax, m = 0, 0
+    s = summaries or {}
+    if tok_idx is not None:
+        _need(tok_idx, "tok_idx", torch.int32)
+        _need(w, "w", torch.float32)
+        m = tok_idx.shape[-1]
+        if m == 0:
+            # an empty tensor may have a NULL data pointer, which the C API reads as
+            # block mode; with m = 0 nothing is read, so any aligned pointer will do
+            tok_idx = w = workspace.tensor
+    else:
+        _need(block_idx, "block_idx", torch.int32)
+        _need(n_kept, "n_kept", torch.int32)
+        kmax = block_idx.shape[-1]
+    st = lib().kv_sparse_decode_attn(
+        ctypes.byref(shape), _ptr(q), float(scale), _ptr(K), _ptr(V), _ptr(block_idx), _ptr(n_kept),
+        int(kmax), _ptr(s.get("k_sum")), _ptr(s.get("v_sum")), _ptr(s.get("counts")), _ptr(s.get("k_tot")),
+        _ptr(s.get("v_tot")), int(bool(use_tail_proxy)) if tok_idx is None else 0, _ptr(tok_idx), _ptr(w),
+        int(m), _ptr(out), _ptr(lse), workspace.ptr(), workspace.nbytes, _stream(dev))
+    _check(st)
+    return out, lse
+
+
+def kv_dense_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor,
+                         block_size: int, scale: float, workspace: Workspace, *,
+                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                         want_lse: bool = True):
+    """Exact attention over every cached token. Returns (out, lse or None)."""
+    _need(q, "q", K.dtype)
+    _need(K, "K")
+    _need(V, "V", K.dtype)
+    shape = make_shape(q, K, seq_lens, block_size)
+    dev = q.device
+    if out is None:
+        out = torch.empty(shape.B, shape.Hq, shape.D, dtype=torch.float32, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty(shape.B, shape.Hq, dtype=torch.float32, device=dev)
+    _check(lib().kv_dense_decode_attn(ctypes.byref(shape), _ptr(q), float(scale), _ptr(K), _ptr(V),
+                                      _ptr(out), _ptr(lse), workspace.ptr(), workspace.nbytes,
+                                      _stream(dev)))
+    return out, lse

@@ -1,0 +1,355 @@
+// C ABI of libkvsparse: argument validation and kernel dispatch. Every check
+// runs on the host before anything is launched; kernels are enqueued on the
+// caller's stream and nothing here allocates device memory.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "attention.cuh"
+#include "kvsparse.h"
+#include "launch.h"
+#include "select.cuh"
+#include "summaries.cuh"
+
+namespace kvs {
+
+cudaError_t attn_launch_bf16_d64(int, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_bf16_d128(int, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_f32_d64(int, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_f32_d128(int, const AttnParams&, int, cudaStream_t);
+int attn_cps_bf16_d64(int);
+int attn_cps_bf16_d128(int);
+int attn_cps_f32_d64(int);
+int attn_cps_f32_d128(int);
+cudaError_t select_launch_bf16_d64(int, int, const SelParams&, int, cudaStream_t);
+cudaError_t select_launch_bf16_d128(int, int, const SelParams&, int, cudaStream_t);
+cudaError_t select_launch_f32_d64(int, int, const SelParams&, int, cudaStream_t);
+cudaError_t select_launch_f32_d128(int, int, const SelParams&, int, cudaStream_t);
+
+cudaError_t launch_attn(int dtype, int D, int G, const AttnParams& p, int grid, cudaStream_t st) {
+  if (dtype == KV_BF16) return D == 64 ? attn_launch_bf16_d64(G, p, grid, st) : attn_launch_bf16_d128(G, p, grid, st);
+  return D == 64 ? attn_launch_f32_d64(G, p, grid, st) : attn_launch_f32_d128(G, p, grid, st);
+}
+int attn_ctas_per_sm(int dtype, int D, int G) {
+  if (dtype == KV_BF16) return D == 64 ? attn_cps_bf16_d64(G) : attn_cps_bf16_d128(G);
+  return D == 64 ? attn_cps_f32_d64(G) : attn_cps_f32_d128(G);
+}
+cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st) {
+  if (dtype == KV_BF16)
+    return D == 64 ? select_launch_bf16_d64(G, mode, p, grid, st) : select_launch_bf16_d128(G, mode, p, grid, st);
+  return D == 64 ? select_launch_f32_d64(G, mode, p, grid, st) : select_launch_f32_d128(G, mode, p, grid, st);
+}
+
+template <typename T, int D>
+static cudaError_t sums_td(const void* K, const void* V, const int32_t* seq_lens, float* k_sum, float* v_sum,
+                           int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap, int L, int NBcap,
+                           cudaStream_t st) {
+  constexpr int LPR = D / (16 / static_cast<int>(sizeof(T)));
+  const int64_t total = 2LL * NBH * NBcap * LPR;
+  const int64_t blocks = (total + 255) / 256;
+  block_sums_kernel<T, D><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const T*>(K), static_cast<const T*>(V), seq_lens, k_sum, v_sum, counts, NBH, Hkv, Ncap, L, NBcap);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int64_t tot2 = 2LL * NBH * D;
+  block_totals_kernel<<<static_cast<unsigned>((tot2 + 255) / 256), 256, 0, st>>>(k_sum, v_sum, k_tot, v_tot, NBH,
+                                                                                  NBcap, D);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
+                        float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,
+                        int L, int NBcap, cudaStream_t st) {
+  if (dtype == KV_BF16) {
+    if (D == 64)
+      return sums_td<__nv_bfloat16, 64>(K, V, seq_lens, k_sum, v_sum, counts, k_tot, v_tot, NBH, Hkv, Ncap, L, NBcap,
+                                        st);
+    return sums_td<__nv_bfloat16, 128>(K, V, seq_lens, k_sum, v_sum, counts, k_tot, v_tot, NBH, Hkv, Ncap, L, NBcap,
+                                       st);
+  }
+  if (D == 64)
+    return sums_td<float, 64>(K, V, seq_lens, k_sum, v_sum, counts, k_tot, v_tot, NBH, Hkv, Ncap, L, NBcap, st);
+  return sums_td<float, 128>(K, V, seq_lens, k_sum, v_sum, counts, k_tot, v_tot, NBH, Hkv, Ncap, L, NBcap, st);
+}
+
+}  // namespace kvs
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kv_status fail(kv_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+kv_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(KV_ERR_CUDA, "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Shape checks shared by every entry point.
+kv_status check_shape(const kv_shape* s) {
+  if (!s) return fail(KV_ERR_INVALID_ARG, "shape is NULL");
+  if (s->B < 0) return fail(KV_ERR_INVALID_ARG, "B = %d < 0", s->B);
+  if (s->Hq < 1 || s->Hkv < 1 || s->Hq % s->Hkv != 0)
+    return fail(KV_ERR_INVALID_ARG, "Hq = %d must be a positive multiple of Hkv = %d", s->Hq, s->Hkv);
+  if (s->Ncap < 1) return fail(KV_ERR_INVALID_ARG, "Ncap = %d < 1", s->Ncap);
+  if (s->block_size < 1) return fail(KV_ERR_INVALID_ARG, "block_size = %d < 1", s->block_size);
+  if (s->dtype != KV_BF16 && s->dtype != KV_F32) return fail(KV_ERR_INVALID_ARG, "unknown dtype %d", (int)s->dtype);
+  const int G = s->Hq / s->Hkv;
+  if (G > 8) return fail(KV_ERR_UNSUPPORTED, "group size G = %d > 8", G);
+  if (s->D != 64 && s->D != 128) return fail(KV_ERR_UNSUPPORTED, "head dim D = %d (supported: 64, 128)", s->D);
+  const int L = s->block_size;
+  if (L != 16 && L != 32 && L != 64 && L != 128)
+    return fail(KV_ERR_UNSUPPORTED, "block_size = %d (supported: 16, 32, 64, 128)", L);
+  const long long nb = (static_cast<long long>(s->Ncap) + L - 1) / L;
+  if (nb > kvs::SEL_MAXNB) return fail(KV_ERR_UNSUPPORTED, "NBcap = %lld > %d", nb, kvs::SEL_MAXNB);
+  if (static_cast<long long>(s->B) * s->Hkv > (1LL << 24))
+    return fail(KV_ERR_UNSUPPORTED, "B * Hkv = %lld too large", static_cast<long long>(s->B) * s->Hkv);
+  if (s->B > 0 && !s->seq_lens) return fail(KV_ERR_INVALID_ARG, "seq_lens is NULL");
+  if (s->seq_lens && !aligned(s->seq_lens, 4)) return fail(KV_ERR_INVALID_ARG, "seq_lens not 4-byte aligned");
+  return KV_OK;
+}
+
+kv_status need(const void* p, const char* name, size_t align = 16) {
+  if (!p) return fail(KV_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(KV_ERR_INVALID_ARG, "%s is not %zu-byte aligned", name, align);
+  return KV_OK;
+}
+
+#define KV_TRY(expr)                 \
+  do {                               \
+    kv_status _st = (expr);          \
+    if (_st != KV_OK) return _st;    \
+  } while (0)
+
+int num_sms_current() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cache[64] = {0};
+  int& c = cache[dev & 63];
+  if (c == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    c = v;
+  }
+  return c;
+}
+
+kv_status run_attention(const kv_shape* s, const void* q, float scale, const void* K, const void* V,
+                        const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
+                        const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
+                        int use_proxy, const int32_t* tok_idx, const float* w, int m, int mode, float* out,
+                        float* lse, void* ws, size_t ws_bytes, kv_stream_t stream) {
+  const int G = s->Hq / s->Hkv;
+  const int NBH = s->B * s->Hkv;
+  const int NBcap = (s->Ncap + s->block_size - 1) / s->block_size;
+  if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
+  KV_TRY(need(q, "q"));
+  KV_TRY(need(K, "K"));
+  KV_TRY(need(V, "V"));
+  KV_TRY(need(out, "out"));
+  if (lse) KV_TRY(need(lse, "lse", 4));
+  KV_TRY(need(ws, "workspace", 256));
+  const size_t want = kv_workspace_bytes(s);
+  if (ws_bytes < want) return fail(KV_ERR_INVALID_ARG, "workspace has %zu bytes, needs %zu", ws_bytes, want);
+  int P = 0;
+  if (mode == kvs::ATTN_BLOCKS) {
+    if (kmax < 0) return fail(KV_ERR_INVALID_ARG, "kmax = %d < 0", kmax);
+    if (kmax > NBcap) return fail(KV_ERR_INVALID_ARG, "kmax = %d > NBcap = %d", kmax, NBcap);
+    KV_TRY(need(block_idx, "block_idx", 4));
+    KV_TRY(need(n_kept, "n_kept", 4));
+    if (use_proxy) {
+      KV_TRY(need(k_sum, "k_sum"));
+      KV_TRY(need(v_sum, "v_sum"));
+      KV_TRY(need(counts, "counts", 4));
+      KV_TRY(need(k_tot, "k_tot"));
+      KV_TRY(need(v_tot, "v_tot"));
+    }
+    P = (kmax > 0 ? kmax : 1) * s->block_size;
+  } else if (mode == kvs::ATTN_WEIGHTED) {
+    if (m < 0) return fail(KV_ERR_INVALID_ARG, "m = %d < 0", m);
+    KV_TRY(need(tok_idx, "tok_idx", 4));
+    KV_TRY(need(w, "w", 4));
+    P = m > 0 ? m : 1;
+    use_proxy = 0;
+  } else {
+    P = s->Ncap;
+    use_proxy = 0;
+  }
+  if (NBH == 0) return KV_OK;
+  const int sms = num_sms_current();
+  if (sms <= 0) return fail(KV_ERR_CUDA, "no CUDA device available");
+  kvs::AttnParams p{};
+  p.q = q;
+  p.K = K;
+  p.V = V;
+  p.seq_lens = s->seq_lens;
+  p.block_idx = block_idx;
+  p.n_kept = n_kept;
+  p.kmax = kmax;
+  p.k_sum = k_sum;
+  p.v_sum = v_sum;
+  p.counts = counts;
+  p.k_tot = k_tot;
+  p.v_tot = v_tot;
+  p.tok_idx = tok_idx;
+  p.w = w;
+  p.m = m;
+  p.out = out;
+  p.lse = lse;
+  unsigned char* wsb = static_cast<unsigned char*>(ws);
+  p.status = reinterpret_cast<uint32_t*>(wsb);
+  p.counters = reinterpret_cast<uint32_t*>(wsb + kvs::ws_counters_off());
+  p.recs = reinterpret_cast<float*>(wsb + kvs::ws_records_off(NBH));
+  p.proxy_recs = reinterpret_cast<float*>(wsb + kvs::ws_proxy_off(NBH, G, s->D));
+  p.B = s->B;
+  p.Hq = s->Hq;
+  p.Hkv = s->Hkv;
+  p.Ncap = s->Ncap;
+  p.L = s->block_size;
+  p.NBcap = NBcap;
+  p.mode = mode;
+  p.use_proxy = use_proxy ? 1 : 0;
+  p.qscale = scale * 1.4426950408889634f;
+  p.part = kvs::make_partition(NBH, P, sms, kvs::attn_ctas_per_sm(s->dtype, s->D, G));
+  cudaError_t e = kvs::launch_attn(s->dtype, s->D, G, p, p.part.C, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  return KV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kv_status kv_build_block_summaries(const kv_shape* shape, const void* K, const void* V, float* k_sum, float* v_sum,
+                                   int32_t* counts, float* k_tot, float* v_tot, kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  KV_TRY(need(K, "K"));
+  KV_TRY(need(V, "V"));
+  KV_TRY(need(k_sum, "k_sum"));
+  KV_TRY(need(v_sum, "v_sum"));
+  KV_TRY(need(counts, "counts", 4));
+  KV_TRY(need(k_tot, "k_tot"));
+  KV_TRY(need(v_tot, "v_tot"));
+  const int NBH = shape->B * shape->Hkv;
+  if (NBH == 0) return KV_OK;
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  cudaError_t e = kvs::launch_sums(shape->dtype, shape->D, K, V, shape->seq_lens, k_sum, v_sum, counts, k_tot, v_tot,
+                                   NBH, shape->Hkv, shape->Ncap, shape->block_size, NBcap,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "summary launch");
+  return KV_OK;
+}
+
+kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv_score_mode mode,
+                           const float* k_sum, const int32_t* counts, const void* K, int k_top, int force_first,
+                           int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                           kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  if (mode != KV_SCORE_SUMMARY && mode != KV_SCORE_EXACT_MASS)
+    return fail(KV_ERR_INVALID_ARG, "unknown score mode %d", (int)mode);
+  if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
+  KV_TRY(need(q, "q"));
+  KV_TRY(need(counts, "counts", 4));
+  if (mode == KV_SCORE_SUMMARY) KV_TRY(need(k_sum, "k_sum"));
+  if (mode == KV_SCORE_EXACT_MASS) KV_TRY(need(K, "K"));
+  KV_TRY(need(block_idx, "block_idx", 4));
+  KV_TRY(need(n_kept, "n_kept", 4));
+  if (scores) KV_TRY(need(scores, "scores", 4));
+  if (k_top < 0) return fail(KV_ERR_INVALID_ARG, "k_top = %d < 0", k_top);
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  const int forced = (force_first ? 1 : 0) + (force_last ? 1 : 0);
+  const long long need_k = std::min<long long>(NBcap, static_cast<long long>(k_top) + forced);
+  if (kmax < need_k)
+    return fail(KV_ERR_INVALID_ARG, "kmax = %d < min(NBcap, k_top + forced) = %lld", kmax, need_k);
+  const int NBH = shape->B * shape->Hkv;
+  if (NBH == 0) return KV_OK;
+  kvs::SelParams p{};
+  p.q = q;
+  p.k_sum = k_sum;
+  p.counts = counts;
+  p.K = K;
+  p.seq_lens = shape->seq_lens;
+  p.block_idx = block_idx;
+  p.n_kept = n_kept;
+  p.scores = scores;
+  p.B = shape->B;
+  p.Hq = shape->Hq;
+  p.Hkv = shape->Hkv;
+  p.Ncap = shape->Ncap;
+  p.L = shape->block_size;
+  p.NBcap = NBcap;
+  p.k_top = k_top;
+  p.force_first = force_first ? 1 : 0;
+  p.force_last = force_last ? 1 : 0;
+  p.kmax = kmax;
+  p.qscale = scale * 1.4426950408889634f;
+  const int G = shape->Hq / shape->Hkv;
+  cudaError_t e = kvs::launch_select(shape->dtype, shape->D, G, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY
+                                                                                        : kvs::SEL_EXACT,
+                                     p, NBH * kvs::SEL_CS, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "select launch");
+  return KV_OK;
+}
+
+kv_status kv_sparse_decode_attn(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                                const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
+                                const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
+                                int use_tail_proxy, const int32_t* tok_idx, const float* w, int m, float* out,
+                                float* lse, void* workspace, size_t ws_bytes, kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  const int mode = tok_idx ? kvs::ATTN_WEIGHTED : kvs::ATTN_BLOCKS;
+  return run_attention(shape, q, scale, K, V, block_idx, n_kept, kmax, k_sum, v_sum, counts, k_tot, v_tot,
+                       use_tail_proxy, tok_idx, w, m, mode, out, lse, workspace, ws_bytes, stream);
+}
+
+kv_status kv_dense_decode_attn(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                               float* out, float* lse, void* workspace, size_t ws_bytes, kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  return run_attention(shape, q, scale, K, V, nullptr, nullptr, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0,
+                       nullptr, nullptr, 0, kvs::ATTN_DENSE, out, lse, workspace, ws_bytes, stream);
+}
+
+size_t kv_workspace_bytes(const kv_shape* shape) {
+  if (!shape || shape->Hkv < 1 || shape->Hq < shape->Hkv || shape->B < 0 || shape->D < 1) return 0;
+  const int G = shape->Hq / shape->Hkv;
+  return kvs::ws_total(shape->B * shape->Hkv, G, shape->D);
+}
+
+kv_status kv_workspace_init(void* workspace, size_t ws_bytes, kv_stream_t stream) {
+  KV_TRY(need(workspace, "workspace", 256));
+  if (ws_bytes < 256) return fail(KV_ERR_INVALID_ARG, "workspace too small (%zu bytes)", ws_bytes);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "workspace memset");
+  return KV_OK;
+}
+
+kv_status kv_workspace_status(const void* workspace, uint32_t* status_out, kv_stream_t stream) {
+  KV_TRY(need(workspace, "workspace", 256));
+  if (!status_out) return fail(KV_ERR_INVALID_ARG, "status_out is NULL");
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, workspace, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status copy");
+  *status_out = v;
+  if (v != 0) return fail(KV_ERR_DEVICE_CHECK, "device checks failed: status 0x%x", v);
+  return KV_OK;
+}
+
+const char* kv_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

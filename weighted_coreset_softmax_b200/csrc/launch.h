@@ -1,0 +1,22 @@
+// Launchers of the kvsparse kernels. Each is instantiated in its own
+// translation unit per (element type, head dimension) so the build parallelises.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "partition.h"
+
+namespace kvs {
+
+struct AttnParams;
+struct SelParams;
+
+// dtype: 0 = bf16, 1 = fp32. Return cudaSuccess or the launch error.
+cudaError_t launch_attn(int dtype, int D, int G, const AttnParams& p, int grid, cudaStream_t st);
+int attn_ctas_per_sm(int dtype, int D, int G);
+cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
+cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
+                        float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,
+                        int L, int NBcap, cudaStream_t st);
+
+}  // namespace kvs

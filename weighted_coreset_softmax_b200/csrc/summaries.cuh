@@ -1,0 +1,107 @@
+// Block summaries built once after prefill: per-block key sum, value sum and
+// token count, and per-(sequence, KV head) totals.
+//
+// Sources: "COBS: Cumulant Order Block Sparse Attention" -- the mean-pool block
+// summary (affine score (18): phi_b = mean key, a_b = ln L) and the per-block
+// stored mean key; "OpenAttention reads 1% of the KV cache -- Count-aware tail
+// proxy" -- the unread tail's mean key and value, which the attention kernel
+// forms as (total - sum over kept blocks) / count.
+//
+// One thread owns one 16-byte channel chunk of one block and walks the block's
+// rows, so a warp reads whole 256-byte rows of two blocks per instruction and no
+// cross-thread reduction is needed. The totals are summed from the block sums by a
+// second kernel in a fixed order (bit-reproducible, no float atomics).
+#pragma once
+
+#include "common.cuh"
+
+namespace kvs {
+
+template <typename T, int D>
+__global__ void __launch_bounds__(256) block_sums_kernel(const T* __restrict__ K, const T* __restrict__ V,
+                                                         const int32_t* __restrict__ seq_lens,
+                                                         float* __restrict__ k_sum, float* __restrict__ v_sum,
+                                                         int32_t* __restrict__ counts, int NBH, int Hkv, int Ncap,
+                                                         int L, int NBcap) {
+  constexpr int CH = 16 / sizeof(T);
+  constexpr int LPR = D / CH;
+  constexpr int CH2 = CH / 2;
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = 2LL * NBH * NBcap * LPR;
+  if (gid >= total) return;
+  const int c = static_cast<int>(gid % LPR);
+  int64_t rest = gid / LPR;
+  const int blk = static_cast<int>(rest % NBcap);
+  rest /= NBcap;
+  const int bh = static_cast<int>(rest % NBH);
+  const int tensor = static_cast<int>(rest / NBH);
+  const int b = bh / Hkv;
+  const int n = max(0, min(seq_lens[b], Ncap));
+  const int start = blk * L;
+  const int cnt = max(0, min(L, n - start));
+  const T* src = (tensor ? V : K) + (static_cast<int64_t>(bh) * Ncap + start) * D + c * CH;
+  float2 acc[CH2];
+#pragma unroll
+  for (int e = 0; e < CH2; ++e) acc[e] = make_float2(0.f, 0.f);
+  int r = 0;
+  for (; r + 8 <= cnt; r += 8) {
+    uint4 raw[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r + u) * D));
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      float2 f[CH2];
+      Chunk<T>::unpack(raw[u], f);
+#pragma unroll
+      for (int e = 0; e < CH2; ++e) {
+        acc[e].x += f[e].x;
+        acc[e].y += f[e].y;
+      }
+    }
+  }
+  for (; r < cnt; ++r) {
+    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r) * D));
+    float2 f[CH2];
+    Chunk<T>::unpack(raw, f);
+#pragma unroll
+    for (int e = 0; e < CH2; ++e) {
+      acc[e].x += f[e].x;
+      acc[e].y += f[e].y;
+    }
+  }
+  float* dst = (tensor ? v_sum : k_sum) + (static_cast<int64_t>(bh) * NBcap + blk) * D + c * CH;
+#pragma unroll
+  for (int e = 0; e < CH2; e += 2) {
+    if (e + 1 < CH2)
+      *reinterpret_cast<float4*>(dst + 2 * e) = make_float4(acc[e].x, acc[e].y, acc[e + 1].x, acc[e + 1].y);
+    else
+      *reinterpret_cast<float2*>(dst + 2 * e) = acc[e];
+  }
+  if (tensor == 0 && (bh % Hkv) == 0 && c == 0) counts[static_cast<int64_t>(b) * NBcap + blk] = cnt;
+}
+
+// tot[bh][d] = sum over blocks of sums[bh][blk][d], four interleaved partial sums
+// combined in a fixed order.
+__global__ void __launch_bounds__(256) block_totals_kernel(const float* __restrict__ k_sum,
+                                                           const float* __restrict__ v_sum,
+                                                           float* __restrict__ k_tot, float* __restrict__ v_tot,
+                                                           int NBH, int NBcap, int D) {
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = 2LL * NBH * D;
+  if (gid >= total) return;
+  const int d = static_cast<int>(gid % D);
+  const int64_t rest = gid / D;
+  const int bh = static_cast<int>(rest % NBH);
+  const int tensor = static_cast<int>(rest / NBH);
+  const float* src = (tensor ? v_sum : k_sum) + static_cast<int64_t>(bh) * NBcap * D + d;
+  float a[4] = {0.f, 0.f, 0.f, 0.f};
+  int blk = 0;
+  for (; blk + 4 <= NBcap; blk += 4) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) a[u] += src[static_cast<int64_t>(blk + u) * D];
+  }
+  for (; blk < NBcap; ++blk) a[0] += src[static_cast<int64_t>(blk) * D];
+  (tensor ? v_tot : k_tot)[static_cast<int64_t>(bh) * D + d] = (a[0] + a[1]) + (a[2] + a[3]);
+}
+
+}  // namespace kvs
