@@ -14,7 +14,9 @@
  *
  * Conventions shared by every entry point
  *   - Pointers named K, V, q, k_sum, ... are DEVICE pointers unless stated.
- *     The library never allocates device memory; the caller owns every buffer.
+ *     The library calls no allocator; the caller owns every buffer (the one
+ *     exception, kv_sparse_decode_attn_noalloc, uses a fixed array inside the
+ *     library instead of a caller workspace).
  *   - Layouts are dense row-major, C order:
  *       q        [B][Hq][D]         dtype of the shape
  *       K, V     [B][Hkv][Ncap][D]  dtype of the shape
@@ -205,6 +207,31 @@ kv_status kv_workspace_init(void* workspace, size_t ws_bytes, kv_stream_t stream
  * if any bit is set, KV_OK otherwise.
  */
 kv_status kv_workspace_status(const void* workspace, uint32_t* status_out, kv_stream_t stream);
+
+/*
+ * kv_sparse_decode_attn_noalloc -- kv_sparse_decode_attn for callers that cannot
+ * allocate device memory (a plugin or operator that is handed only its inputs and
+ * outputs, or a process that forbids allocation once it is serving). The pages
+ * have no counterpart of this entry point: it only changes where the kernel's
+ * scratch lives.
+ *
+ * Same arguments and results as kv_sparse_decode_attn, without the workspace:
+ * the scratch comes from a fixed 16 MiB array inside the library (held on every
+ * GPU that loads it, until exit). Shapes whose kv_workspace_bytes exceeds 16 MiB
+ * are rejected with KV_ERR_INVALID_ARG. The first call on a device looks up the
+ * array's device address (make it before any stream capture). Each call clears
+ * the array's counters with an async memset on `stream`; calls share the array,
+ * so calls that overlap on the GPU race -- order them on one stream or with
+ * events. Nothing is allocated. Device-check status bits are not reported.
+ */
+kv_status kv_sparse_decode_attn_noalloc(const kv_shape* shape, const void* q, float scale,
+                                        const void* K, const void* V,
+                                        const int32_t* block_idx, const int32_t* n_kept, int kmax,
+                                        const float* k_sum, const float* v_sum,
+                                        const int32_t* counts, const float* k_tot,
+                                        const float* v_tot, int use_tail_proxy,
+                                        const int32_t* tok_idx, const float* w, int m,
+                                        float* out, float* lse, kv_stream_t stream);
 
 /* Message of the last failed call on this host thread ("" if none). */
 const char* kv_last_error(void);

@@ -353,3 +353,9 @@ kv_status kv_workspace_status(const void* workspace, uint32_t* status_out, kv_st
 const char* kv_last_error(void) { return g_last_error.c_str(); }
 
 }  // extern "C"
+
+namespace kvs {
+// Lets other translation units of the library report a message through
+// kv_last_error().
+void set_last_error(const char* msg) { g_last_error = msg; }
+}  // namespace kvs
