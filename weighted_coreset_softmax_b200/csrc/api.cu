@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <string>
 
@@ -18,26 +19,28 @@
 
 namespace kvs {
 
-cudaError_t attn_launch_bf16_d64(int, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_bf16_d128(int, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_f32_d64(int, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_f32_d128(int, const AttnParams&, int, cudaStream_t);
-int attn_cps_bf16_d64(int);
-int attn_cps_bf16_d128(int);
-int attn_cps_f32_d64(int);
-int attn_cps_f32_d128(int);
+cudaError_t attn_launch_bf16_d64(int, bool, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_bf16_d128(int, bool, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_f32_d64(int, bool, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_f32_d128(int, bool, const AttnParams&, int, cudaStream_t);
+int attn_prepare_bf16_d64(int, bool, int);
+int attn_prepare_bf16_d128(int, bool, int);
+int attn_prepare_f32_d64(int, bool, int);
+int attn_prepare_f32_d128(int, bool, int);
 cudaError_t select_launch_bf16_d64(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_bf16_d128(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_f32_d64(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_f32_d128(int, int, const SelParams&, int, cudaStream_t);
 
-cudaError_t launch_attn(int dtype, int D, int G, const AttnParams& p, int grid, cudaStream_t st) {
-  if (dtype == KV_BF16) return D == 64 ? attn_launch_bf16_d64(G, p, grid, st) : attn_launch_bf16_d128(G, p, grid, st);
-  return D == 64 ? attn_launch_f32_d64(G, p, grid, st) : attn_launch_f32_d128(G, p, grid, st);
+cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
+  if (dtype == KV_BF16)
+    return D == 64 ? attn_launch_bf16_d64(G, use_mma, p, grid, st) : attn_launch_bf16_d128(G, use_mma, p, grid, st);
+  return D == 64 ? attn_launch_f32_d64(G, false, p, grid, st) : attn_launch_f32_d128(G, false, p, grid, st);
 }
-int attn_ctas_per_sm(int dtype, int D, int G) {
-  if (dtype == KV_BF16) return D == 64 ? attn_cps_bf16_d64(G) : attn_cps_bf16_d128(G);
-  return D == 64 ? attn_cps_f32_d64(G) : attn_cps_f32_d128(G);
+int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev) {
+  if (dtype == KV_BF16)
+    return D == 64 ? attn_prepare_bf16_d64(G, use_mma, dev) : attn_prepare_bf16_d128(G, use_mma, dev);
+  return D == 64 ? attn_prepare_f32_d64(G, false, dev) : attn_prepare_f32_d128(G, false, dev);
 }
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st) {
   if (dtype == KV_BF16)
@@ -135,6 +138,16 @@ kv_status need(const void* p, const char* name, size_t align = 16) {
     if (_st != KV_OK) return _st;    \
   } while (0)
 
+// bf16 caches use the tensor-core attention consumer unless the environment
+// variable KVSPARSE_ATTN=fma selects the CUDA-core one (read once per process).
+bool attention_uses_tensor_cores() {
+  static const bool v = [] {
+    const char* e = std::getenv("KVSPARSE_ATTN");
+    return !(e && std::strcmp(e, "fma") == 0);
+  }();
+  return v;
+}
+
 int num_sms_current() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -192,6 +205,11 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   if (NBH == 0) return KV_OK;
   const int sms = num_sms_current();
   if (sms <= 0) return fail(KV_ERR_CUDA, "no CUDA device available");
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const bool use_mma = attention_uses_tensor_cores();
+  const int cps = kvs::attn_ctas_per_sm(s->dtype, s->D, G, use_mma, dev);
+  if (cps <= 0) return fail(KV_ERR_CUDA, "attention kernel does not fit on an SM");
   kvs::AttnParams p{};
   p.q = q;
   p.K = K;
@@ -220,12 +238,14 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   p.Hkv = s->Hkv;
   p.Ncap = s->Ncap;
   p.L = s->block_size;
+  p.log2L = 0;
+  while ((1 << p.log2L) < s->block_size) ++p.log2L;
   p.NBcap = NBcap;
   p.mode = mode;
   p.use_proxy = use_proxy ? 1 : 0;
   p.qscale = scale * 1.4426950408889634f;
-  p.part = kvs::make_partition(NBH, P, sms, kvs::attn_ctas_per_sm(s->dtype, s->D, G));
-  cudaError_t e = kvs::launch_attn(s->dtype, s->D, G, p, p.part.C, reinterpret_cast<cudaStream_t>(stream));
+  p.part = kvs::make_partition(NBH, P, sms, cps);
+  cudaError_t e = kvs::launch_attn(s->dtype, s->D, G, use_mma, p, p.part.C, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return KV_OK;
 }
@@ -300,7 +320,7 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv
   const int G = shape->Hq / shape->Hkv;
   cudaError_t e = kvs::launch_select(shape->dtype, shape->D, G, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY
                                                                                         : kvs::SEL_EXACT,
-                                     p, NBH * kvs::SEL_CS, reinterpret_cast<cudaStream_t>(stream));
+                                     p, NBH, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return KV_OK;
 }

@@ -6,7 +6,7 @@
 //  * "OpenAttention reads 1% of the KV cache -- Count-aware tail proxy", section
 //    "Skipping reviews without losing the verdict": the unread tail enters the
 //    softmax as one token whose value is the tail's mean value and whose logit is
-//    its mean logit plus ln(count); it is handled like an ordinary token, so here
+//    its mean logit plus ln(count); it has the form of an ordinary token, so here
 //    it is one more partial result merged with the others.
 //  * "WildCat: Near-Linear Attention in Theory and Practice", abstract: weighted
 //    coreset attention, logit + ln w_i.
@@ -14,20 +14,42 @@
 //    dense attention reads the whole cache.
 //
 // Design (sm_100a). All (sequence, KV head) pairs ("bh") lay their P token slots
-// end to end on one axis; the grid (about two CTAs per SM) splits that axis into
-// equal contiguous ranges, so every CTA streams the same number of bytes whatever
-// the per-head work. In each CTA one producer warp walks its range in chunks of
-// TR rows and moves the K and V rows of each chunk into a 4-stage shared-memory
-// ring with cp.async.bulk (one copy per contiguous run; one per row when rows are
-// gathered), completion tracked by mbarrier transaction counts. Four consumer
-// warps compute q.k for all G query heads of the group in fp32 (16-byte row
-// chunks per lane, packed f32x2 FMAs, a transpose reduction across the lanes of a
-// row), keep an online softmax per row group in the log2 domain, and accumulate
-// p * v. When the range leaves a bh (or ends) the consumers merge their states
-// into one partial record (m, l, acc) in the workspace and take an arrival ticket
-// for that bh; whichever CTA arrives last merges all of the bh's records (and the
-// proxy record) into the output. No CTA ever waits for another.
+// end to end on one axis; the grid cuts that axis into equal contiguous ranges,
+// one per CTA, so every SM streams the same bytes whatever the per-head work.
+// A CTA walks its range in chunks of TR rows that stay inside one bh (and, in
+// block mode, one kept block); warp w owns rows [16w, 16w + 16) of every chunk.
+// Each warp is an independent pipeline: it moves its rows' K and V (and, at the
+// start of a bh, the group's q) into its own two-slot shared-memory ring with
+// cp.async.bulk, tracked by its own mbarriers, and refills a slot as soon as it
+// has consumed it; the per-chunk indices are prefetched one chunk ahead.
+//  q.k: four lanes share a group of two tokens (each lane reads a quarter of
+//  each row); q is held once per warp in fp32, prescaled by scale*log2(e), split
+//  into two 16-byte planes per chunk; every lane visits its row chunks in a
+//  rotated order chosen so that the eight lanes of each quarter-warp (the unit
+//  in which 16-byte shared loads are served) hit eight different bank groups,
+//  for the K rows and for q alike; packed f32x2 FMAs; a 4-lane all-reduce
+//  finishes the dots and the first two lanes of each group then own one token's
+//  logits each.
+//  softmax: per warp, in the log2 domain; the running maximum is uniform across
+//  the warp, so partial states merge without rescaling.
+//  p.v: lanes own 16-byte channel chunks of V rows, packed f32x2 FMAs.
+// For bf16 caches a tensor-core consumer replaces the CUDA-core one (warp-chunks
+// of 32 rows, copied one row per lane into rows padded by 16 bytes so that the
+// 8x8 ldmatrix tiles are conflict-free): q.k is mma.sync m16n8k16 with the 16
+// tokens of a tile as M and the G <= 8 query heads as N (q^T fragments stay in
+// registers for the whole bh), so the bf16 products are exact and accumulate in
+// fp32; the softmax runs on the accumulator fragments; P is split into a bf16
+// high part and a bf16 remainder (about 16 significant bits together), moved
+// into B-operand layout with movmatrix, and p.v is two mma.sync per 16x16 tile of
+// V^T. The q.k and p.v of a kept token then cost a few instructions instead of
+// a few dozen, which leaves the kernel bound by HBM rather than by issue.
+// When a warp's chunk sequence leaves a bh it writes one partial record
+// (acc, m, l) to the workspace and takes an arrival ticket for that bh; the last
+// arriver merges all records of the bh (and the proxy record) into the output.
+// No warp ever waits for another.
 #pragma once
+
+#include <climits>
 
 #include "common.cuh"
 
@@ -57,137 +79,242 @@ struct AttnParams {
   uint32_t* counters;
   float* recs;
   float* proxy_recs;
-  int B, Hq, Hkv, Ncap, L, NBcap;
+  int B, Hq, Hkv, Ncap, L, log2L, NBcap;
   int mode;
   int use_proxy;
   float qscale;  // softmax scale * log2(e): logits are kept in the log2 domain
   Partition part;
 };
 
-template <typename T, int D, int G>
+// Shape constants of one instantiation. MMA selects the tensor-core consumer
+// (bf16 caches): 32 rows per warp-chunk in padded rows; otherwise the CUDA-core
+// consumer: 16 rows per warp-chunk in dense rows.
+template <typename T, int D, int G, bool MMA>
 struct AttnCfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int RB = D * ES;        // bytes per cached row
-  static constexpr int LPR = RB / 16;      // lanes per row (16 bytes each)
-  static constexpr int RPW = 32 / LPR;     // row groups per warp
-  static constexpr int CH = 16 / ES;       // elements per lane chunk
-  static constexpr int CH2 = CH / 2;       // float2 pairs per lane chunk
-  static constexpr int R = 4;              // rows per lane per chunk
-  static constexpr int NCW = 4;            // consumer warps
-  static constexpr int NTHREADS = (NCW + 1) * 32;
-  static constexpr int TR = NCW * RPW * R;  // rows per chunk (8 KB of K, 8 KB of V)
-  static constexpr int GP = pow2ceil(G);
-  static constexpr int NV = R * GP;        // partial dots per lane per chunk
-  // Up to G = 4 two CTAs share an SM; larger groups need more registers, so one
-  // CTA per SM runs with a deeper ring to keep as many bytes in flight.
-  static constexpr int CPS = G <= 4 ? 2 : 1;          // CTAs per SM
-  static constexpr int S = G <= 4 ? 4 : 8;            // pipeline stages
-  using HV = HeldValues<NV, LPR, GP>;
-  static constexpr int NH = HV::NH;
-  static constexpr int QBYTES = G * D * ES;
-  static constexpr int QB = (QBYTES + 15) & ~15;
-  static constexpr int PSTR = GP < 4 ? 4 : GP;  // floats per P row (16-byte rows)
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = TR * RB;
-  static constexpr int OFF_Q = 2 * TR * RB;
-  static constexpr int OFF_BIAS = OFF_Q + QB;
-  static constexpr int OFF_HDR = OFF_BIAS + TR * 4;
-  static constexpr int STAGE = (OFF_HDR + 16 + 127) & ~127;
-  static constexpr int OFF_BARS = S * STAGE;
-  static constexpr int OFF_P = OFF_BARS + 128;
-  static constexpr int PW_FLOATS = RPW * (R + 1) * PSTR;  // per consumer warp
-  static constexpr int OFF_MERGE = OFF_P + NCW * PW_FLOATS * 4;
-  static constexpr int MERGE_FLOATS = NCW * G * D + 2 * NCW * G;
-  static constexpr int SMEM = OFF_MERGE + MERGE_FLOATS * 4;
+  static constexpr int RB = D * ES;          // bytes per cached row
+  static constexpr int RS = MMA ? RB + 16 : RB;  // bytes per row in shared memory
+  static constexpr int CPR = RB / 16;        // 16-byte chunks per row
+  static constexpr int CH = 16 / ES;         // elements per chunk
+  static constexpr int CH2 = CH / 2;         // float2 pairs per chunk
+  static constexpr int LPT = 4;              // lanes per token group (CUDA-core q.k)
+  static constexpr int CPL = CPR / LPT;      // chunks per lane per row (CUDA-core q.k)
+  static constexpr int TPL = 2;              // tokens per token group (CUDA-core q.k)
+  static constexpr int TPW = MMA ? 32 : 8 * TPL;  // rows per warp per chunk
+  static constexpr int NW = ATTN_NW;         // warps per CTA
+  static constexpr int NTHREADS = NW * 32;
+  static constexpr int TR = NW * TPW;        // rows per chunk
+  static constexpr int S = 2;                // ring slots per warp
+  static constexpr int VR = 32 / CPR;        // V rows per p.v step (CUDA-core)
+  static constexpr int KS = D / 16;          // k-steps of q.k and d-tiles of p.v (MMA)
+  static constexpr int QPL = CH / 4;         // 16-byte planes of fp32 q per chunk
+  static constexpr int QPLANE = CPR * 16;    // bytes of one plane of one head
+  static constexpr int QHEAD = QPL * QPLANE; // bytes of one head of q (fp32)
+  static constexpr int QBYTES = G * RB;      // q of one KV head's group, input type
+  static constexpr int PSTR = G <= 4 ? 4 : 8;
+  // one ring slot: K rows | V rows | raw q | bias | header
+  static constexpr int SL_K = 0;
+  static constexpr int SL_V = TPW * RS;
+  static constexpr int SL_Q = 2 * TPW * RS;
+  static constexpr int SL_BIAS = SL_Q + QBYTES;
+  static constexpr int SL_HDR = SL_BIAS + TPW * 4;
+  static constexpr int SLOT = (SL_HDR + 16 + 127) & ~127;
+  // one warp: S slots | q fp32 | p | barriers (q fp32 and p: CUDA-core only)
+  static constexpr int W_Q = S * SLOT;
+  static constexpr int W_P = W_Q + (MMA ? 0 : G * QHEAD);
+  static constexpr int W_BAR = W_P + (MMA ? 0 : TPW * PSTR * 4);
+  static constexpr int W_BYTES = (W_BAR + S * 8 + 127) & ~127;
+  static constexpr int SMEM = NW * W_BYTES;
   static constexpr int RECF = (G * D + 2 * G + 3) & ~3;
-  static_assert(LPR >= 1 && LPR <= 32 && (32 % LPR) == 0, "row layout");
-  static_assert(TR <= 64, "producer covers at most 64 rows per chunk");
-  static_assert(2 * S * 8 <= 128, "barrier area");
+  static_assert(MMA || CPL == 2 || CPL == 4 || CPL == 8, "chunks per lane");
+  static_assert(MMA || (VR >= 1 && 32 % CPR == 0 && TPW % VR == 0), "p.v row layout");
+  static_assert(!MMA || (ES == 2 && G <= 8 && D % 16 == 0), "tensor-core consumer: bf16, G <= 8");
+  static_assert(TPW <= 32, "one row per lane when issuing copies");
+  static_assert((S & (S - 1)) == 0, "ring slots must be a power of two");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
+  // CUDA-core q.k: rotation of the chunk a lane reads at step st. Within a
+  // quarter-warp the lanes are (ts & 1) x pq; rows sit 128-byte aligned, so the
+  // bank group of chunk c is c mod 8 -- this choice gives the eight lanes eight
+  // different groups.
+  __device__ __forceinline__ static int chunk_at(int st, int ts, int pq) {
+    const int rot = CPL == 2 ? 0 : (CPL == 4 ? 2 * (pq >> 1) : 2 * pq);
+    return pq * CPL + ((st + (ts & 1) + rot) & (CPL - 1));
+  }
 };
+
+// ---- tensor-core helpers (warp-wide, bf16 operands, fp32 accumulate)
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ uint32_t movm_trans(uint32_t x) {
+  uint32_t y;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+// D += A(16x16, row) * B(16x8, col), bf16 inputs, fp32 accumulators
+__device__ __forceinline__ void mma_bf16(float& d0, float& d1, float& d2, float& d3, const uint32_t (&a)[4],
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d0), "+f"(d1), "+f"(d2), "+f"(d3)
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// two floats -> bf16x2 (lo in the low half), round to nearest
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 __device__ __forceinline__ float safe_max_ref(float m) { return m == -INFINITY ? 0.f : m; }
 
 // Walks [cur, end) of the token axis in chunks that stay inside one bh, hold at
-// most TR rows, and (block mode) stay inside one kept block.
+// most TR rows and, in block mode, stay inside one kept block. Incremental: no
+// division after init.
 struct ChunkIter {
   int64_t cur, end;
-  __device__ __forceinline__ bool next(int P, int L, int TR, int mode, int& bh, int& j0, int& rows) {
+  int bh, j0;
+  __device__ __forceinline__ void init(int64_t t0, int64_t t1, int P) {
+    cur = t0;
+    end = t1;
+    bh = static_cast<int>(t0 / P);
+    j0 = static_cast<int>(t0 - static_cast<int64_t>(bh) * P);
+  }
+  __device__ __forceinline__ bool next(int P, int L, int TR, int mode, int& obh, int& oj0, int& rows) {
     if (cur >= end) return false;
-    bh = static_cast<int>(cur / P);
-    j0 = static_cast<int>(cur - static_cast<int64_t>(bh) * P);
-    int64_t lim = min(end, static_cast<int64_t>(bh + 1) * P) - cur;
-    int r = static_cast<int>(min(lim, static_cast<int64_t>(TR)));
-    if (mode == ATTN_BLOCKS) r = min(r, L - (j0 % L));
+    int r = P - j0;
+    const int64_t left = end - cur;
+    if (left < r) r = static_cast<int>(left);
+    if (r > TR) r = TR;
+    if (mode == ATTN_BLOCKS) r = min(r, L - (j0 & (L - 1)));
+    obh = bh;
+    oj0 = j0;
     rows = r;
     cur += r;
+    j0 += r;
+    if (j0 == P) {
+      ++bh;
+      j0 = 0;
+    }
     return true;
   }
 };
 
-// Per-chunk metadata the producer loads one ring cycle ahead.
+// What a warp needs to issue one chunk's copies. Held one chunk per lane, a
+// batch of 32 chunks at a time.
 struct ChunkMeta {
   int has, bh, j0, rows, first;
-  int n, nk, blk;   // seq_len; block mode: n_kept and block index of the slot
-  int i0, i1;       // weighted mode: token index of rows lane, lane + 32
-  float w0, w1;
+  int n;       // seq_len of the sequence
+  int nk;      // block mode: n_kept of the bh
+  int blk;     // block mode: block index of the chunk's slot
 };
 
-__device__ __forceinline__ int expected_arrivals(const Partition& pt, int bh, int use_proxy) {
-  const int64_t a = static_cast<int64_t>(bh) * pt.P;
-  const int cf = part_cta_of(pt, a);
-  const int cl = part_cta_of(pt, a + pt.P - 1);
-  return cl - cf + 1 + (use_proxy ? 1 : 0);
+__device__ __forceinline__ int first_cta(const Partition& pt, int bh) {
+  return part_cta_of(pt, static_cast<int64_t>(bh) * pt.P);
+}
+__device__ __forceinline__ int last_cta(const Partition& pt, int bh) {
+  return part_cta_of(pt, static_cast<int64_t>(bh) * pt.P + pt.P - 1);
 }
 
-// Merges every partial record of one bh into out / lse. One warp.
+// Merges every partial record of one bh into out / lse. One warp. The records'
+// maxima and sums are read by one lane each (one round trip), the weights follow
+// from warp reductions, then every lane streams its channels of all records with
+// the loads of several records in flight.
 template <int D, int G>
 __device__ void finalize_bh(const AttnParams& p, int bh, int lane) {
   constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   constexpr int VEC = D / 32;
-  const int64_t a = static_cast<int64_t>(bh) * p.part.P;
-  const int cf = part_cta_of(p.part, a);
-  const int cl = part_cta_of(p.part, a + p.part.P - 1);
-  const int nrec = cl - cf + 1 + (p.use_proxy ? 1 : 0);
-  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const int cf = first_cta(p.part, bh), cl = last_cta(p.part, bh);
+  const int nattn = (cl - cf + 1) * ATTN_NW;
+  const int nrec = nattn + (p.use_proxy ? 1 : 0);
+  const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
+  const float* base = p.recs + static_cast<size_t>(cf + bh) * ATTN_NW * RECF;
   auto rec_ptr = [&](int j) -> const float* {
-    return (j <= cl - cf) ? p.recs + static_cast<size_t>(cf + j + bh) * RECF
-                          : p.proxy_recs + static_cast<size_t>(bh) * RECF;
+    return j < nattn ? base + static_cast<size_t>(j) * RECF : p.proxy_recs + static_cast<size_t>(bh) * RECF;
   };
-#pragma unroll 1
+  float* o = p.out + (static_cast<size_t>(b) * p.Hq + h * G) * D + lane * VEC;
+  // weights of up to 32 records at a time; more records are folded in passes
+  float Mg[G], Lg[G], acc[G][VEC];
+#pragma unroll
   for (int g = 0; g < G; ++g) {
-    float M = -INFINITY;
-    for (int j = 0; j < nrec; ++j) M = fmaxf(M, __ldcg(rec_ptr(j) + G * D + g));
-    const float Ms = safe_max_ref(M);
-    float Lsum = 0.f;
-    float acc[VEC];
+    Mg[g] = -INFINITY;
+    Lg[g] = 0.f;
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) acc[v] = 0.f;
-    for (int j = 0; j < nrec; ++j) {
-      const float* r = rec_ptr(j);
-      const float mj = __ldcg(r + G * D + g);
-      const float wj = exp2f(mj - Ms);
-      Lsum = fmaf(wj, __ldcg(r + G * D + G + g), Lsum);
+    for (int v = 0; v < VEC; ++v) acc[g][v] = 0.f;
+  }
+  for (int j0 = 0; j0 < nrec; j0 += 32) {
+    const int j = j0 + lane;
+    float mj[G], lj[G];
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wj, __ldcg(r + g * D + lane * VEC + v), acc[v]);
+    for (int g = 0; g < G; ++g) {
+      mj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + g) : -INFINITY;
+      lj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + G + g) : 0.f;
     }
-    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
-    float* o = p.out + (static_cast<size_t>(b) * p.Hq + h * G + g) * D + lane * VEC;
+    float wj[G];
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) o[v] = acc[v] * inv;
+    for (int g = 0; g < G; ++g) {
+      const float Mn = fmaxf(Mg[g], warp_max(mj[g]));
+      const float Ms = safe_max_ref(Mn);
+      const float rescale = fast_exp2(Mg[g] - Ms);
+      wj[g] = fast_exp2(mj[g] - Ms);
+      Lg[g] = Lg[g] * rescale + warp_sum(wj[g] * lj[g]);
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[g][v] *= rescale;
+      Mg[g] = Mn;
+    }
+    const int cnt = min(32, nrec - j0);
+#pragma unroll 4
+    for (int k = 0; k < cnt; ++k) {
+      const float* r = rec_ptr(j0 + k) + lane * VEC;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float wk = __shfl_sync(FULL_MASK, wj[g], k);
+        if (VEC == 4) {
+          const float4 x = __ldcg(reinterpret_cast<const float4*>(r + g * D));
+          acc[g][0] = fmaf(wk, x.x, acc[g][0]);
+          acc[g][1] = fmaf(wk, x.y, acc[g][1]);
+          acc[g][2] = fmaf(wk, x.z, acc[g][2]);
+          acc[g][3] = fmaf(wk, x.w, acc[g][3]);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wk, __ldcg(r + g * D + v), acc[g][v]);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    const float inv = Lg[g] > 0.f ? 1.f / Lg[g] : 0.f;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) o[g * D + v] = acc[g][v] * inv;
     if (p.lse && lane == 0)
-      p.lse[static_cast<size_t>(b) * p.Hq + h * G + g] =
-          Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
+      p.lse[static_cast<size_t>(b) * p.Hq + h * G + g] = Lg[g] > 0.f ? (Mg[g] + log2f(Lg[g])) * LN2 : -INFINITY;
   }
 }
 
 // Arrival ticket for bh; the last arriver merges. Called by one whole warp after
-// its writes are complete and fenced.
+// its record writes are complete and fenced.
 template <int D, int G>
 __device__ __forceinline__ void arrive_bh(const AttnParams& p, int bh, int lane) {
   int last = 0;
   if (lane == 0) {
-    const int E = expected_arrivals(p.part, bh, p.use_proxy);
+    const int E = (last_cta(p.part, bh) - first_cta(p.part, bh) + 1) * ATTN_NW + (p.use_proxy ? 1 : 0);
     const uint32_t old = atomicAdd(p.counters + bh, 1u);
     last = (old + 1 == static_cast<uint32_t>(E));
     if (last) p.counters[bh] = 0u;  // ready for the next launch
@@ -200,73 +327,119 @@ __device__ __forceinline__ void arrive_bh(const AttnParams& p, int bh, int lane)
 }
 
 // The tail proxy of one bh as a partial record (m = its log2 logit, l = 1,
-// acc = its value). One warp.
+// acc = its value). One warp. All kept block indices are read in one round trip
+// and the key/value sums of the kept blocks are then requested together, so the
+// proxy costs two dependent memory round trips (up to 32 kept blocks).
 template <typename T, int D, int G>
 __device__ void build_proxy(const AttnParams& p, int bh, int lane) {
   constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   constexpr int VEC = D / 32;
-  const int b = bh / p.Hkv, h = bh % p.Hkv;
+  constexpr int UNR = 8;  // kept blocks whose sums are in flight together
+  const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
+  // independent first loads: length, count, indices, q, totals
   int n = p.seq_lens[b];
+  int nk = p.n_kept[bh];
+  const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D;
+  float qv[G][VEC];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) qv[g][v] = load_as_float(qrow + g * D + lane * VEC + v);
+  float kt[VEC], vt[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    kt[v] = p.k_tot[static_cast<size_t>(bh) * D + lane * VEC + v];
+    vt[v] = p.v_tot[static_cast<size_t>(bh) * D + lane * VEC + v];
+  }
   if (n < 0 || n > p.Ncap) {
     if (lane == 0) atomicOr(p.status, KV_DEV_BAD_SEQ_LEN);
     n = max(0, min(n, p.Ncap));
   }
-  const int nbv = (n + p.L - 1) / p.L;
-  int nk = p.n_kept[bh];
   if (nk < 0 || nk > p.kmax) {
     if (lane == 0) atomicOr(p.status, KV_DEV_BAD_N_KEPT);
     nk = max(0, min(nk, p.kmax));
   }
+  const int nbv = (n + p.L - 1) >> p.log2L;
   float ks[VEC], vs[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) ks[v] = vs[v] = 0.f;
-  int cnt = 0, prev = -1;
+  int cnt = 0;
+  int prev_last = -1;  // last block index of the previous group of 32
+  // the first 32 index slots are read before n_kept is known (they are in bounds)
+  const int first32 = lane < p.kmax ? p.block_idx[static_cast<size_t>(bh) * p.kmax + lane] : INT_MAX;
   for (int s0 = 0; s0 < nk; s0 += 32) {
-    const int mine = (s0 + lane < nk) ? p.block_idx[static_cast<size_t>(bh) * p.kmax + s0 + lane] : -1;
+    int mine = s0 == 0 ? first32 : ((s0 + lane < nk) ? p.block_idx[static_cast<size_t>(bh) * p.kmax + s0 + lane] : INT_MAX);
+    if (s0 + lane >= nk) mine = INT_MAX;
+    // a kept index must lie in [0, nbv) and exceed the one before it
+    int before = __shfl_up_sync(FULL_MASK, mine, 1);
+    if (lane == 0) before = prev_last;
+    const bool in_list = s0 + lane < nk;
+    const bool ok = in_list && mine >= 0 && mine < nbv && mine > before;
+    if (__any_sync(FULL_MASK, in_list && !ok) && lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
+    const unsigned okmask = __ballot_sync(FULL_MASK, ok);
+    prev_last = __shfl_sync(FULL_MASK, mine, 31);
+    // the counts of this group of kept blocks, one per lane
+    int c = ok ? p.counts[static_cast<size_t>(b) * p.NBcap + mine] : 0;
+    c = __reduce_add_sync(FULL_MASK, c);
+    cnt += c;
     const int lim = min(32, nk - s0);
-    for (int jj = 0; jj < lim; ++jj) {
-      const int blk = __shfl_sync(FULL_MASK, mine, jj);
-      if (blk <= prev || blk >= nbv) {
-        if (lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
-        continue;
-      }
-      prev = blk;
-      const size_t row = (static_cast<size_t>(bh) * p.NBcap + blk) * D + lane * VEC;
+    for (int j0 = 0; j0 < lim; j0 += UNR) {
+      float kr[UNR][VEC], vr[UNR][VEC];
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) {
-        ks[v] += p.k_sum[row + v];
-        vs[v] += p.v_sum[row + v];
+      for (int u = 0; u < UNR; ++u) {
+        const int j = j0 + u;
+        const int blk = __shfl_sync(FULL_MASK, mine, j & 31);
+        const bool use = j < lim && ((okmask >> (j & 31)) & 1u);
+        const size_t row = (static_cast<size_t>(bh) * p.NBcap + (use ? blk : 0)) * D + lane * VEC;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          kr[u][v] = use ? p.k_sum[row + v] : 0.f;
+          vr[u][v] = use ? p.v_sum[row + v] : 0.f;
+        }
       }
-      cnt += p.counts[static_cast<size_t>(b) * p.NBcap + blk];
+#pragma unroll
+      for (int u = 0; u < UNR; ++u)
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          ks[v] += kr[u][v];
+          vs[v] += vr[u][v];
+        }
     }
   }
   const int nT = n - cnt;
   float* rec = p.proxy_recs + static_cast<size_t>(bh) * RECF;
-  const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D;
   if (nT > 0) {
     const float inv = 1.f / static_cast<float>(nT);
     float kb[VEC], vb[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) {
-      kb[v] = (p.k_tot[static_cast<size_t>(bh) * D + lane * VEC + v] - ks[v]) * inv;
-      vb[v] = (p.v_tot[static_cast<size_t>(bh) * D + lane * VEC + v] - vs[v]) * inv;
+      kb[v] = (kt[v] - ks[v]) * inv;
+      vb[v] = (vt[v] - vs[v]) * inv;
     }
     const float lc = log2f(static_cast<float>(nT));
-#pragma unroll 1
-    for (int g = 0; g < G; ++g) {
-      float dot = 0.f;
+    float dot[G];
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) dot = fmaf(load_as_float(qrow + g * D + lane * VEC + v), kb[v], dot);
-      dot = warp_sum(dot);
+    for (int g = 0; g < G; ++g) {
+      float d = 0.f;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) d = fmaf(qv[g][v], kb[v], d);
+      dot[g] = d;
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+      for (int g = 0; g < G; ++g) dot[g] += __shfl_xor_sync(FULL_MASK, dot[g], m);
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int v = 0; v < VEC; ++v) rec[g * D + lane * VEC + v] = vb[v];
       if (lane == 0) {
-        rec[G * D + g] = dot * p.qscale + lc;
+        rec[G * D + g] = dot[g] * p.qscale + lc;
         rec[G * D + G + g] = 1.f;
       }
     }
   } else {
-#pragma unroll 1
+#pragma unroll
     for (int g = 0; g < G; ++g) {
 #pragma unroll
       for (int v = 0; v < VEC; ++v) rec[g * D + lane * VEC + v] = 0.f;
@@ -281,394 +454,551 @@ __device__ void build_proxy(const AttnParams& p, int bh, int lane) {
   arrive_bh<D, G>(p, bh, lane);
 }
 
-template <typename T, int D, int G>
-__global__ void __launch_bounds__(AttnCfg<T, D, G>::NTHREADS, AttnCfg<T, D, G>::CPS)
-    attn_kernel(const AttnParams p) {
-  using C = AttnCfg<T, D, G>;
+template <typename T, int D, int G, bool MMA>
+__global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(const AttnParams p) {
+  using C = AttnCfg<T, D, G, MMA>;
   extern __shared__ __align__(128) unsigned char smem[];
-  const int tid = threadIdx.x;
-  const int warp = tid >> 5;
-  const int lane = tid & 31;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
   const int cta = blockIdx.x;
   const int64_t t0 = part_t0(p.part, cta);
   const int64_t t1 = part_t0(p.part, cta + 1);
   const int P = p.part.P;
+  unsigned char* wb = smem + warp * C::W_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wb + C::W_BAR);
+  float* q32 = reinterpret_cast<float*>(wb + C::W_Q);
+  float* pbuf = reinterpret_cast<float*>(wb + C::W_P);
 
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BARS);
-  uint64_t* empty = full + C::S;
-  if (tid == 0) {
+  if (lane == 0) {
 #pragma unroll
-    for (int s = 0; s < C::S; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, C::NCW);
-    }
+    for (int s = 0; s < C::S; ++s) mbar_init(bars + s, 1);
     fence_mbar_init();
   }
-  // Rows a chunk does not fill keep stale (finite) data; zero the K/V buffers
-  // once so that no uninitialised pattern can ever be multiplied by p = 0.
-  for (int s = 0; s < C::S; ++s) {
-    uint4* b4 = reinterpret_cast<uint4*>(smem + s * C::STAGE);
-    for (int i = tid; i < 2 * C::TR * C::RB / 16; i += C::NTHREADS) b4[i] = make_uint4(0, 0, 0, 0);
-  }
+  // Rows a chunk does not fill keep stale (finite) data; zero the ring once so
+  // that no uninitialised pattern is ever multiplied by p = 0.
+  for (int i = lane; i < C::S * C::SLOT / 16; i += 32) reinterpret_cast<uint4*>(wb)[i] = make_uint4(0, 0, 0, 0);
   fence_proxy_async_smem();
-  __syncthreads();
+  __syncwarp();
 
-  if (warp == C::NCW) {
-    // ------------------------------------------------------------ producer
-    const uint64_t pol = l2_evict_first_policy();
-    const unsigned char* Kb = static_cast<const unsigned char*>(p.K);
-    const unsigned char* Vb = static_cast<const unsigned char*>(p.V);
-    const unsigned char* Qb = static_cast<const unsigned char*>(p.q);
-    ChunkIter ahead{t0, t1};
-    int prev_bh = -1;
-    auto fetch = [&](ChunkMeta& mt) {
-      int bh, j0, rows;
-      mt.has = ahead.next(P, p.L, C::TR, p.mode, bh, j0, rows);
-      if (!mt.has) return;
-      mt.bh = bh;
-      mt.j0 = j0;
-      mt.rows = rows;
-      mt.first = (bh != prev_bh);
-      prev_bh = bh;
-      const int b = bh / p.Hkv;
-      mt.n = p.seq_lens[b];
-      if (p.mode == ATTN_BLOCKS) {
-        // with kmax = 0 the axis still has one (empty) slot per bh: read nothing
-        const int slot = j0 / p.L;
-        mt.nk = p.n_kept[bh];
-        mt.blk = slot < p.kmax ? p.block_idx[static_cast<size_t>(bh) * p.kmax + slot] : -1;
-      } else if (p.mode == ATTN_WEIGHTED) {
-        // rows past m (m = 0 leaves one empty row per bh) are never read
-        const size_t base = static_cast<size_t>(bh) * p.m + j0;
-        const bool r0 = lane < rows && j0 + lane < p.m, r1 = lane + 32 < rows && j0 + lane + 32 < p.m;
-        mt.i0 = r0 ? p.tok_idx[base + lane] : -1;
-        mt.w0 = r0 ? p.w[base + lane] : 0.f;
-        mt.i1 = r1 ? p.tok_idx[base + lane + 32] : -1;
-        mt.w1 = r1 ? p.w[base + lane + 32] : 0.f;
-      }
-    };
-    ChunkMeta ring[C::S];
-    bool gave_up = false;  // after one timed-out wait, wait no more
-#pragma unroll
-    for (int s = 0; s < C::S; ++s) fetch(ring[s]);
-    for (int base = 0;; base += C::S) {
-      bool done = false;
-#pragma unroll
-      for (int s = 0; s < C::S; ++s) {
-        ChunkMeta& mt = ring[s];
-        if (!done && !mt.has) done = true;
-        if (done) continue;
-        const uint32_t phase = static_cast<uint32_t>(base / C::S) & 1u;
-        if (base > 0 && !gave_up && !mbar_wait(empty + s, phase ^ 1u, p.status)) gave_up = true;
-        unsigned char* stg = smem + s * C::STAGE;
-        float* bias = reinterpret_cast<float*>(stg + C::OFF_BIAS);
-        int* hdr = reinterpret_cast<int*>(stg + C::OFF_HDR);
-        const int b = mt.bh / p.Hkv, h = mt.bh % p.Hkv;
-        int n = mt.n;
-        if (n < 0 || n > p.Ncap) {
-          if (lane == 0) atomicOr(p.status, KV_DEV_BAD_SEQ_LEN);
-          n = max(0, min(n, p.Ncap));
-        }
-        int nvalid = 0;
-        int64_t tok0 = 0;
-        bool v0 = false, v1 = false;
-        if (p.mode == ATTN_WEIGHTED) {
-          const bool in0 = mt.i0 >= 0 && mt.i0 < n, in1 = mt.i1 >= 0 && mt.i1 < n;
-          v0 = lane < mt.rows && in0 && mt.w0 > 0.f;
-          v1 = lane + 32 < mt.rows && in1 && mt.w1 > 0.f;
-          if ((lane < mt.rows && mt.w0 > 0.f && !in0) || (lane + 32 < mt.rows && mt.w1 > 0.f && !in1))
-            atomicOr(p.status, KV_DEV_BAD_TOKEN_INDEX);
-          nvalid = __popc(__ballot_sync(FULL_MASK, v0)) + __popc(__ballot_sync(FULL_MASK, v1));
-          if (lane < C::TR) bias[lane] = v0 ? log2f(mt.w0) : -INFINITY;
-          if (lane + 32 < C::TR) bias[lane + 32] = v1 ? log2f(mt.w1) : -INFINITY;
-        } else {
-          if (p.mode == ATTN_BLOCKS) {
-            const int nbv = (n + p.L - 1) / p.L;
-            const int slot = mt.j0 / p.L;
-            const int nk = mt.nk;
-            if ((nk < 0 || nk > p.kmax) && lane == 0) atomicOr(p.status, KV_DEV_BAD_N_KEPT);
-            const bool ok = slot < max(0, min(nk, p.kmax));
-            if (ok && (mt.blk < 0 || mt.blk >= nbv) && lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
-            if (ok && mt.blk >= 0 && mt.blk < nbv) {
-              tok0 = static_cast<int64_t>(mt.blk) * p.L + (mt.j0 % p.L);
-              nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(mt.rows), n - tok0)));
-            }
-          } else {
-            tok0 = mt.j0;
-            nvalid = max(0, min(mt.rows, n - mt.j0));
-          }
-          if (lane < C::TR) bias[lane] = lane < nvalid ? 0.f : -INFINITY;
-          if (lane + 32 < C::TR) bias[lane + 32] = lane + 32 < nvalid ? 0.f : -INFINITY;
-        }
-        if (lane == 0) hdr[0] = nvalid;
-        const uint32_t tx = (mt.first ? C::QBYTES : 0) + 2u * nvalid * C::RB;
-        __syncwarp();
-        if (lane == 0) mbar_arrive_expect_tx(full + s, tx);
-        __syncwarp();
-        if (mt.first && lane == 0)
-          bulk_g2s(stg + C::OFF_Q, Qb + (static_cast<size_t>(b) * p.Hq + h * G) * C::RB, C::QBYTES, full + s,
-                   pol);
-        if (p.mode == ATTN_WEIGHTED) {
-          const size_t hb = static_cast<size_t>(mt.bh) * p.Ncap;
-          if (v0) {
-            bulk_g2s(stg + C::OFF_K + lane * C::RB, Kb + (hb + mt.i0) * C::RB, C::RB, full + s, pol);
-            bulk_g2s(stg + C::OFF_V + lane * C::RB, Vb + (hb + mt.i0) * C::RB, C::RB, full + s, pol);
-          }
-          if (v1) {
-            bulk_g2s(stg + C::OFF_K + (lane + 32) * C::RB, Kb + (hb + mt.i1) * C::RB, C::RB, full + s, pol);
-            bulk_g2s(stg + C::OFF_V + (lane + 32) * C::RB, Vb + (hb + mt.i1) * C::RB, C::RB, full + s, pol);
-          }
-        } else if (nvalid > 0) {
-          const size_t off = (static_cast<size_t>(mt.bh) * p.Ncap + tok0) * C::RB;
-          if (lane == 1) bulk_g2s(stg + C::OFF_K, Kb + off, nvalid * C::RB, full + s, pol);
-          if (lane == 2) bulk_g2s(stg + C::OFF_V, Vb + off, nvalid * C::RB, full + s, pol);
-        }
-        fetch(mt);
-      }
-      if (done) break;
+  const uint64_t pol = l2_evict_first_policy();
+  const unsigned char* Kg = static_cast<const unsigned char*>(p.K);
+  const unsigned char* Vg = static_cast<const unsigned char*>(p.V);
+  const unsigned char* Qg = static_cast<const unsigned char*>(p.q);
+  const int r0 = warp * C::TPW;  // first row of this warp in every chunk
+
+  // ---- chunk metadata, 32 chunks per batch (lane j holds chunk j) ---------
+  // Every lane walks the chunk sequence to its own chunk and loads that chunk's
+  // sequence length, kept count and block index, so one memory round trip covers
+  // the next 32 copies; the following batch is loaded while this one is used.
+  ChunkIter bstart;
+  bstart.init(t0, t1, P);
+  int batch_prev_bh = -1;
+  auto load_batch = [&](ChunkMeta& lc) {
+    ChunkIter c = bstart;
+    int bh = -1, j0 = 0, rows = 0;
+    bool has = false;
+    for (int k = 0; k <= lane; ++k) {
+      has = c.next(P, p.L, C::TR, p.mode, bh, j0, rows);
+      if (!has) break;
     }
-    return;
+    lc.has = has;
+    lc.bh = has ? bh : -1;
+    lc.j0 = j0;
+    lc.rows = rows;
+    int prev = __shfl_up_sync(FULL_MASK, lc.bh, 1);
+    if (lane == 0) prev = batch_prev_bh;
+    lc.first = has && lc.bh != prev;
+    // the next batch starts where lane 31 stopped
+    bstart.cur = __shfl_sync(FULL_MASK, c.cur, 31);
+    bstart.bh = __shfl_sync(FULL_MASK, c.bh, 31);
+    bstart.j0 = __shfl_sync(FULL_MASK, c.j0, 31);
+    batch_prev_bh = __shfl_sync(FULL_MASK, lc.bh, 31);
+    lc.n = has ? p.seq_lens[lc.bh / p.Hkv] : 0;
+    lc.nk = 0;
+    lc.blk = -1;
+    if (has && p.mode == ATTN_BLOCKS) {
+      const int slot = j0 >> p.log2L;
+      lc.nk = p.n_kept[lc.bh];
+      lc.blk = slot < p.kmax ? p.block_idx[static_cast<size_t>(lc.bh) * p.kmax + slot] : -1;
+    }
+  };
+  // weighted mode: this lane's row (token index, weight) of one chunk
+  auto load_rows = [&](int bh, int j0, int rows, int& idx, float& w) {
+    const int row = j0 + r0 + lane;
+    const bool in = bh >= 0 && lane < C::TPW && r0 + lane < rows && row < p.m;
+    const size_t at = static_cast<size_t>(in ? bh : 0) * p.m + (in ? row : 0);
+    idx = in ? p.tok_idx[at] : -1;
+    w = in ? p.w[at] : 0.f;
+  };
+  ChunkMeta bcur, bnext;
+  load_batch(bcur);
+  load_batch(bnext);
+  int widx = -1, widx_n = -1;
+  float ww = 0.f, ww_n = 0.f;
+  if (p.mode == ATTN_WEIGHTED) {
+    load_rows(__shfl_sync(FULL_MASK, bcur.bh, 0), __shfl_sync(FULL_MASK, bcur.j0, 0),
+              __shfl_sync(FULL_MASK, bcur.rows, 0), widx, ww);
+    load_rows(__shfl_sync(FULL_MASK, bcur.bh, 1), __shfl_sync(FULL_MASK, bcur.j0, 1),
+              __shfl_sync(FULL_MASK, bcur.rows, 1), widx_n, ww_n);
   }
 
-  // -------------------------------------------------------------- consumers
-  const int w = warp;
-  const int rg = lane / C::LPR;
-  const int c = lane % C::LPR;
-  using HV = typename C::HV;
+  // issue the copies of chunk c (its metadata sits in lane c & 31 of bcur)
+  auto issue = [&](int c, int s) {
+    const int src = c & 31;
+    const int mbh = __shfl_sync(FULL_MASK, bcur.bh, src);
+    const int mj0 = __shfl_sync(FULL_MASK, bcur.j0, src);
+    const int mrows = __shfl_sync(FULL_MASK, bcur.rows, src);
+    const int mfirst = __shfl_sync(FULL_MASK, bcur.first, src);
+    int n = __shfl_sync(FULL_MASK, bcur.n, src);
+    const int mnk = __shfl_sync(FULL_MASK, bcur.nk, src);
+    const int mblk = __shfl_sync(FULL_MASK, bcur.blk, src);
+    unsigned char* sl = wb + s * C::SLOT;
+    float* bias = reinterpret_cast<float*>(sl + C::SL_BIAS);
+    if (n < 0 || n > p.Ncap) {
+      if (lane == 0) atomicOr(p.status, KV_DEV_BAD_SEQ_LEN);
+      n = max(0, min(n, p.Ncap));
+    }
+    const int nr = max(0, min(C::TPW, mrows - r0));  // rows of this chunk owned by this warp
+    bool vrow = false;
+    int64_t tok = 0;
+    float bz = -INFINITY;
+    int nvalid = 0;
+    if (p.mode == ATTN_WEIGHTED) {
+      const bool inb = widx >= 0 && widx < n;
+      vrow = lane < nr && ww > 0.f && inb;
+      if (lane < nr && ww > 0.f && !inb) atomicOr(p.status, KV_DEV_BAD_TOKEN_INDEX);
+      tok = widx;
+      if (vrow) bz = log2f(ww);
+      nvalid = __popc(__ballot_sync(FULL_MASK, vrow));
+    } else {
+      int64_t tok0 = 0;
+      if (p.mode == ATTN_BLOCKS) {
+        const int nbv = (n + p.L - 1) >> p.log2L;
+        const int slot = mj0 >> p.log2L;
+        if ((mnk < 0 || mnk > p.kmax) && lane == 0) atomicOr(p.status, KV_DEV_BAD_N_KEPT);
+        const bool kept = slot < max(0, min(mnk, p.kmax));
+        if (kept && (mblk < 0 || mblk >= nbv) && lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
+        if (kept && mblk >= 0 && mblk < nbv) {
+          tok0 = (static_cast<int64_t>(mblk) << p.log2L) + (mj0 & (p.L - 1)) + r0;
+          nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(nr), n - tok0)));
+        }
+      } else {
+        tok0 = mj0 + r0;
+        nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(nr), n - tok0)));
+      }
+      vrow = lane < nvalid;
+      tok = tok0 + lane;
+      if (vrow) bz = 0.f;
+    }
+    if (lane < C::TPW) bias[lane] = bz;
+    if (lane == 0) *reinterpret_cast<int*>(sl + C::SL_HDR) = nvalid;
+    const uint32_t tx = (mfirst ? C::QBYTES : 0u) + 2u * nvalid * C::RB;
+    __syncwarp();
+    if (lane == 0) mbar_arrive_expect_tx(bars + s, tx);
+    __syncwarp();
+    const int b = mbh / p.Hkv, h = mbh - b * p.Hkv;
+    if (mfirst && lane == 0)
+      bulk_g2s(sl + C::SL_Q, Qg + (static_cast<size_t>(b) * p.Hq + h * G) * C::RB, C::QBYTES, bars + s, pol);
+    if (MMA || p.mode == ATTN_WEIGHTED) {
+      // one copy per row (rows land in padded slots for the tensor-core reads)
+      if (vrow) {
+        const size_t off = (static_cast<size_t>(mbh) * p.Ncap + tok) * C::RB;
+        bulk_g2s(sl + C::SL_K + lane * C::RS, Kg + off, C::RB, bars + s, pol);
+        bulk_g2s(sl + C::SL_V + lane * C::RS, Vg + off, C::RB, bars + s, pol);
+      }
+    } else if (nvalid > 0) {
+      const size_t off = (static_cast<size_t>(mbh) * p.Ncap + (tok - lane)) * C::RB;
+      if (lane == 1) bulk_g2s(sl + C::SL_K, Kg + off, nvalid * C::RB, bars + s, pol);
+      if (lane == 2) bulk_g2s(sl + C::SL_V, Vg + off, nvalid * C::RB, bars + s, pol);
+    }
+  };
+  // advance the issue cursor past chunk c: roll batches, prefetch weighted rows
+  auto issued_one = [&](int c) {
+    const int nc = c + 1;
+    if ((nc & 31) == 0) {
+      bcur = bnext;
+      load_batch(bnext);
+    }
+    if (p.mode == ATTN_WEIGHTED) {
+      widx = widx_n;
+      ww = ww_n;
+      // rows of chunk nc + 1 (it lies in bcur, or at lane 0 of bnext)
+      const int c2 = nc + 1;
+      const bool in_cur = (c2 >> 5) == (nc >> 5);
+      const int src = c2 & 31;
+      const int rbh = in_cur ? __shfl_sync(FULL_MASK, bcur.bh, src) : __shfl_sync(FULL_MASK, bnext.bh, src);
+      const int rj0 = in_cur ? __shfl_sync(FULL_MASK, bcur.j0, src) : __shfl_sync(FULL_MASK, bnext.j0, src);
+      const int rrows = in_cur ? __shfl_sync(FULL_MASK, bcur.rows, src) : __shfl_sync(FULL_MASK, bnext.rows, src);
+      load_rows(rbh, rj0, rrows, widx_n, ww_n);
+    }
+  };
 
-  if (p.mode == ATTN_BLOCKS && p.use_proxy) {
-    const int64_t bh_lo = (t0 + P - 1) / P;
-    const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), (t1 + P - 1) / P);
-    for (int64_t bh = bh_lo + w; bh < bh_hi; bh += C::NCW) build_proxy<T, D, G>(p, static_cast<int>(bh), lane);
-  }
-
-  float* Pw = reinterpret_cast<float*>(smem + C::OFF_P) + w * C::PW_FLOATS + rg * (C::R + 1) * C::PSTR;
-  float* MA = reinterpret_cast<float*>(smem + C::OFF_MERGE);  // [NCW][G][D]
-  float* MM = MA + C::NCW * G * D;                             // [NCW][G]
-  float* ML = MM + C::NCW * G;                                 // [NCW][G]
-
-  float2 qf[G][C::CH2];
-  float2 acc[G][C::CH2];
-  float mrun[G], lrun[G];
+  // ---- per-warp softmax state --------------------------------------------
+  // CUDA-core: mrun/lrun per head (warp-uniform max), acc[g] = channel chunk vc
+  //   of rows owned in p.v.
+  // Tensor core: this lane's heads are h0 = 2 (lane & 3) and h0 + 1; o[i] is the
+  //   fragment of O^T rows 16 i + lane / 4 (+ 8) for those two heads.
+  constexpr int NA = MMA ? 2 : G;                 // heads tracked per lane
+  constexpr int ACC = MMA ? C::KS * 4 : G * C::CH;  // accumulator floats per lane
+  float mrun[NA], lrun[NA];
+  float acc[ACC];
+  uint32_t qb[MMA ? C::KS * 2 : 1];               // q^T fragments (tensor core)
   auto reset_state = [&]() {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int g = 0; g < NA; ++g) {
       mrun[g] = -INFINITY;
       lrun[g] = 0.f;
-#pragma unroll
-      for (int e = 0; e < C::CH2; ++e) acc[g][e] = make_float2(0.f, 0.f);
     }
+#pragma unroll
+    for (int e = 0; e < ACC; ++e) acc[e] = 0.f;
   };
 
   auto flush = [&](int bh) {
-    // 1) merge the row groups of this warp (lanes with the same channel chunk)
+    float* rec = p.recs + (static_cast<size_t>(cta + bh) * C::NW + warp) * C::RECF;
+    if constexpr (MMA) {
+      const int h0 = 2 * (lane & 3);
+      float lt[2];
 #pragma unroll
-    for (int mask = C::LPR; mask < 32; mask <<= 1) {
+      for (int u = 0; u < 2; ++u) {
+        float v = lrun[u];
+        v += __shfl_xor_sync(FULL_MASK, v, 4);
+        v += __shfl_xor_sync(FULL_MASK, v, 8);
+        v += __shfl_xor_sync(FULL_MASK, v, 16);
+        lt[u] = v;
+      }
+      const int dr = lane >> 2;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const float mo = __shfl_xor_sync(FULL_MASK, mrun[g], mask);
-        const float lo = __shfl_xor_sync(FULL_MASK, lrun[g], mask);
-        const float M = fmaxf(mrun[g], mo);
-        const float Ms = safe_max_ref(M);
-        const float a = exp2f(mrun[g] - Ms), bw = exp2f(mo - Ms);
-        lrun[g] = lrun[g] * a + lo * bw;
-#pragma unroll
-        for (int e = 0; e < C::CH2; ++e) {
-          const float ox = __shfl_xor_sync(FULL_MASK, acc[g][e].x, mask);
-          const float oy = __shfl_xor_sync(FULL_MASK, acc[g][e].y, mask);
-          acc[g][e].x = acc[g][e].x * a + ox * bw;
-          acc[g][e].y = acc[g][e].y * a + oy * bw;
+      for (int i = 0; i < C::KS; ++i) {
+        if (h0 < G) {
+          rec[h0 * D + 16 * i + dr] = acc[4 * i + 0];
+          rec[h0 * D + 16 * i + dr + 8] = acc[4 * i + 2];
         }
-        mrun[g] = M;
+        if (h0 + 1 < G) {
+          rec[(h0 + 1) * D + 16 * i + dr] = acc[4 * i + 1];
+          rec[(h0 + 1) * D + 16 * i + dr + 8] = acc[4 * i + 3];
+        }
       }
-    }
-    // 2) one row group per warp publishes its state
-    if (rg == 0) {
+      if (lane < 4) {
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float2* dst = reinterpret_cast<float2*>(MA + (w * G + g) * D + c * C::CH);
-#pragma unroll
-        for (int e = 0; e < C::CH2; ++e) dst[e] = acc[g][e];
+        for (int u = 0; u < 2; ++u)
+          if (h0 + u < G) {
+            rec[G * D + h0 + u] = mrun[u];
+            rec[G * D + G + h0 + u] = lt[u];
+          }
       }
-      if (lane == 0) {
+    } else {
+      const int vc = lane % C::CPR;
+      // the row groups of p.v hold disjoint rows with the same (warp-uniform) max
+#pragma unroll
+      for (int mask = C::CPR; mask < 32; mask <<= 1)
+#pragma unroll
+        for (int e = 0; e < ACC; ++e) acc[e] += __shfl_xor_sync(FULL_MASK, acc[e], mask);
+      if (lane < C::CPR) {
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          MM[w * G + g] = mrun[g];
-          ML[w * G + g] = lrun[g];
+          float* dst = rec + g * D + vc * C::CH;
+#pragma unroll
+          for (int e = 0; e < C::CH; e += 4)
+            *reinterpret_cast<float4*>(dst + e) =
+                make_float4(acc[g * C::CH + e], acc[g * C::CH + e + 1], acc[g * C::CH + e + 2], acc[g * C::CH + e + 3]);
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        const float lt = warp_sum(lrun[g]);
+        if (lane == 0) {
+          rec[G * D + g] = mrun[g];
+          rec[G * D + G + g] = lt;
         }
       }
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(C::NCW * 32) : "memory");
-    // 3) the four warp states -> one partial record
-    float* rec = p.recs + static_cast<size_t>(cta + bh) * C::RECF;
-    const int ctid = w * 32 + lane;
-    for (int it = ctid; it < G * D / 4; it += C::NCW * 32) {
-      const int g = it / (D / 4), d4 = it % (D / 4);
-      float M = -INFINITY;
-#pragma unroll
-      for (int ww = 0; ww < C::NCW; ++ww) M = fmaxf(M, MM[ww * G + g]);
-      const float Ms = safe_max_ref(M);
-      float4 r = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int ww = 0; ww < C::NCW; ++ww) {
-        const float a = exp2f(MM[ww * G + g] - Ms);
-        const float4 x = *reinterpret_cast<const float4*>(MA + (ww * G + g) * D + d4 * 4);
-        r.x = fmaf(a, x.x, r.x);
-        r.y = fmaf(a, x.y, r.y);
-        r.z = fmaf(a, x.z, r.z);
-        r.w = fmaf(a, x.w, r.w);
-      }
-      *reinterpret_cast<float4*>(rec + g * D + d4 * 4) = r;
-    }
-    if (ctid < G) {
-      const int g = ctid;
-      float M = -INFINITY;
-#pragma unroll
-      for (int ww = 0; ww < C::NCW; ++ww) M = fmaxf(M, MM[ww * G + g]);
-      const float Ms = safe_max_ref(M);
-      float Ls = 0.f;
-#pragma unroll
-      for (int ww = 0; ww < C::NCW; ++ww) Ls = fmaf(exp2f(MM[ww * G + g] - Ms), ML[ww * G + g], Ls);
-      rec[G * D + g] = M;
-      rec[G * D + G + g] = Ls;
-    }
     __threadfence();
-    asm volatile("bar.sync 1, %0;" ::"n"(C::NCW * 32) : "memory");
-    if (w == 0) arrive_bh<D, G>(p, bh, lane);
+    __syncwarp();
+    arrive_bh<D, G>(p, bh, lane);
   };
 
-  ChunkIter it{t0, t1};
+  ChunkIter it;
+  it.init(t0, t1, P);
   int cur_bh = -1;
   bool timed_out = false;
-  int bh, j0, rows;
-  int i = 0;
+  bool proxies_done = false;
+  int i = 0;       // chunks consumed
+  int issued = 0;  // chunks whose copies were issued
   reset_state();
 #pragma unroll 1
-  while (it.next(P, p.L, C::TR, p.mode, bh, j0, rows)) {
-    const int s = i % C::S;
+  while (true) {
+    // keep the ring full: the only copy-issue site (the first S rounds only issue)
+    if (issued - i < C::S && __shfl_sync(FULL_MASK, bcur.has, issued & 31)) {
+      issue(issued, issued & (C::S - 1));
+      issued_one(issued);
+      ++issued;
+      continue;
+    }
+    if (!proxies_done) {
+      // tail proxies of the bh whose first token lies in this CTA's range, built
+      // while the first copies are in flight
+      proxies_done = true;
+      if (p.mode == ATTN_BLOCKS && p.use_proxy) {
+        const int64_t bh_lo = (t0 + P - 1) / P;
+        const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), (t1 + P - 1) / P);
+        for (int64_t pbh = bh_lo + warp; pbh < bh_hi; pbh += C::NW)
+          build_proxy<T, D, G>(p, static_cast<int>(pbh), lane);
+      }
+    }
+    int bh, j0, rows;
+    const bool more = it.next(P, p.L, C::TR, p.mode, bh, j0, rows);
+    const bool first = more && bh != cur_bh;
+    if ((first || !more) && cur_bh >= 0) flush(cur_bh);  // the only flush site
+    if (!more) break;
+    const int s = i & (C::S - 1);
     const uint32_t phase = static_cast<uint32_t>(i / C::S) & 1u;
-    const bool first = (bh != cur_bh);
     if (first) {
-      if (cur_bh >= 0) flush(cur_bh);
       cur_bh = bh;
       reset_state();
     }
-    if (!timed_out && !mbar_wait(full + s, phase, p.status)) timed_out = true;
-    const unsigned char* stg = smem + s * C::STAGE;
-    if (first) {
+    if (!timed_out && !mbar_wait(bars + s, phase, p.status)) timed_out = true;
+    const unsigned char* sl = wb + s * C::SLOT;
+    const int nvalid = *reinterpret_cast<const int*>(sl + C::SL_HDR);
+    const float* bias = reinterpret_cast<const float*>(sl + C::SL_BIAS);
+    if constexpr (MMA) {
+      // ====================================================== tensor cores
+      if (first) {
+        // q^T as the B operand of q.k: b0 = q[h][16k + 2(l&3) .. +1], b1 = +8
+        const int hq = lane >> 2;
+        const unsigned char* qrow = sl + C::SL_Q + hq * C::RB;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        const uint4 raw = lds128(stg + C::OFF_Q + g * C::RB + c * 16);
-        float2 f[C::CH2];
-        Chunk<T>::unpack(raw, f);
-#pragma unroll
-        for (int e = 0; e < C::CH2; ++e) qf[g][e] = make_float2(f[e].x * p.qscale, f[e].y * p.qscale);
+        for (int k = 0; k < C::KS; ++k) {
+          const int d0 = 16 * k + 2 * (lane & 3);
+          qb[2 * k] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + d0 * 2) : 0u;
+          qb[2 * k + 1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2) : 0u;
+        }
       }
-    }
-    const int nvalid = *reinterpret_cast<const int*>(stg + C::OFF_HDR);
-    if (nvalid > 0) {
-      const float* bias = reinterpret_cast<const float*>(stg + C::OFF_BIAS);
-      // q . k for R rows x G heads, finished by a transpose reduction
-      float part[C::NV];
+      if (nvalid > 0) {
+        const uint32_t kbase = smem_u32(sl + C::SL_K);
+        const uint32_t vbase = smem_u32(sl + C::SL_V);
+        // ---- S^T = K q^T for two 16-token tiles: rows t = 16mt + l/4 (+8), heads h0, h0+1
+        float sc4[2][4];
 #pragma unroll
-      for (int r = 0; r < C::R; ++r) {
-        const int row = w * (C::RPW * C::R) + r * C::RPW + rg;
-        const uint4 raw = lds128(stg + C::OFF_K + row * C::RB + c * 16);
-        float2 kf[C::CH2];
-        Chunk<T>::unpack(raw, kf);
+        for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-        for (int g = 0; g < C::GP; ++g) {
-          if (g < G) {
-            float2 a2 = make_float2(0.f, 0.f);
+          for (int e = 0; e < 4; ++e) sc4[mt][e] = 0.f;
+          const int row = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+          const uint32_t a0 = kbase + row * C::RS + (lane >> 4) * 16;
 #pragma unroll
-            for (int e = 0; e < C::CH2; ++e) a2 = ffma2(qf[g][e], kf[e], a2);
-            part[r * C::GP + g] = a2.x + a2.y;
-          } else {
-            part[r * C::GP + g] = 0.f;
+          for (int k = 0; k < C::KS; ++k) {
+            uint32_t a[4];
+            ldsm_x4(a0 + k * 32, a);
+            mma_bf16(sc4[mt][0], sc4[mt][1], sc4[mt][2], sc4[mt][3], a, qb[2 * k], qb[2 * k + 1]);
+          }
+        }
+        // ---- logits (log2 domain) and the chunk maximum of each head
+        const int tr = lane >> 2;
+        float x[2][4];
+        float cm0 = -INFINITY, cm1 = -INFINITY;
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const float ba = bias[16 * mt + tr], bb = bias[16 * mt + tr + 8];
+          x[mt][0] = fmaf(sc4[mt][0], p.qscale, ba);
+          x[mt][1] = fmaf(sc4[mt][1], p.qscale, ba);
+          x[mt][2] = fmaf(sc4[mt][2], p.qscale, bb);
+          x[mt][3] = fmaf(sc4[mt][3], p.qscale, bb);
+          cm0 = fmaxf(cm0, fmaxf(x[mt][0], x[mt][2]));
+          cm1 = fmaxf(cm1, fmaxf(x[mt][1], x[mt][3]));
+        }
+#pragma unroll
+        for (int m = 4; m < 32; m <<= 1) {
+          cm0 = fmaxf(cm0, __shfl_xor_sync(FULL_MASK, cm0, m));
+          cm1 = fmaxf(cm1, __shfl_xor_sync(FULL_MASK, cm1, m));
+        }
+        const float mn0 = fmaxf(mrun[0], cm0), mn1 = fmaxf(mrun[1], cm1);
+        const float ms0 = safe_max_ref(mn0), ms1 = safe_max_ref(mn1);
+        const float sc0 = fast_exp2(mrun[0] - ms0), sc1 = fast_exp2(mrun[1] - ms1);
+        const bool same = __all_sync(FULL_MASK, mn0 == mrun[0] && mn1 == mrun[1]);
+        mrun[0] = mn0;
+        mrun[1] = mn1;
+        if (!same) {
+#pragma unroll
+          for (int k = 0; k < C::KS; ++k) {
+            acc[4 * k] *= sc0;
+            acc[4 * k + 1] *= sc1;
+            acc[4 * k + 2] *= sc0;
+            acc[4 * k + 3] *= sc1;
+          }
+        }
+        float ls0 = 0.f, ls1 = 0.f;
+        // ---- P as the B operand of p.v (hi + lo bf16 parts), per token tile
+        uint32_t bh_[2][2], bl_[2][2];
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const float p0 = fast_exp2(x[mt][0] - ms0), p1 = fast_exp2(x[mt][1] - ms1);
+          const float p2 = fast_exp2(x[mt][2] - ms0), p3 = fast_exp2(x[mt][3] - ms1);
+          ls0 += p0 + p2;
+          ls1 += p1 + p3;
+          const uint32_t h01 = pack_bf16(p0, p1), h23 = pack_bf16(p2, p3);
+          const uint32_t l01 = pack_bf16(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
+          const uint32_t l23 = pack_bf16(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
+          bh_[mt][0] = movm_trans(h01);
+          bh_[mt][1] = movm_trans(h23);
+          bl_[mt][0] = movm_trans(l01);
+          bl_[mt][1] = movm_trans(l23);
+        }
+        lrun[0] = lrun[0] * sc0 + ls0;
+        lrun[1] = lrun[1] * sc1 + ls1;
+        // ---- O^T += V^T P over the two token tiles
+#pragma unroll
+        for (int mt = 0; mt < 2; ++mt) {
+          const int row = 16 * mt + (lane & 7) + (lane >> 4) * 8;
+          const uint32_t v0 = vbase + row * C::RS + ((lane >> 3) & 1) * 16;
+#pragma unroll
+          for (int k = 0; k < C::KS; ++k) {
+            uint32_t a[4];
+            ldsm_x4_trans(v0 + k * 32, a);
+            mma_bf16(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3], a, bh_[mt][0], bh_[mt][1]);
+            mma_bf16(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3], a, bl_[mt][0], bl_[mt][1]);
           }
         }
       }
-      transpose_reduce<C::NV, C::LPR / 2>(part, lane);
-      // held values -> logits, chunk maxima, probabilities
+    } else {
+      // ====================================================== CUDA cores
+      const int ts = lane >> 2;  // token group: rows ts + 8j, j < TPL
+      const int pq = lane & 3;   // quarter of each row; lanes pq < TPL own row ts + 8 pq
+      const bool owner = pq < C::TPL;
+      const int vr = lane / C::CPR, vc = lane % C::CPR;
+      if (first) {
+        // q of the new group: input type -> fp32 * scale * log2(e), two planes
+        constexpr int NQC = G * C::CPR;
+        constexpr int PER = (NQC + 31) / 32;
 #pragma unroll
-      for (int j = 0; j < C::NH; ++j) {
-        const int vi = HV::index(c, j);
-        const int ri = vi / C::GP, g = vi % C::GP;
-        const int row = w * (C::RPW * C::R) + ri * C::RPW + rg;
-        float sj = g < G ? part[j] + bias[row] : -INFINITY;
-        float cm = sj;
+        for (int k = 0; k < PER; ++k) {
+          const int qc = lane + 32 * k;
+          if (qc < NQC) {
+            const int g = qc / C::CPR, c = qc - g * C::CPR;
+            float2 f[C::CH2];
+            Chunk<T>::unpack(lds128(sl + C::SL_Q + qc * 16), f);
 #pragma unroll
-        for (int mask = HV::ROW_MASK_LO; mask < C::LPR; mask <<= 1)
-          cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, mask));
-        float mold = mrun[0];
-#pragma unroll
-        for (int gg = 1; gg < G; ++gg)
-          if (g == gg) mold = mrun[gg];
-        const float mnew = fmaxf(mold, cm);
-        const float pj = exp2f(sj - safe_max_ref(mnew));
-        if (g < G) {
-          Pw[ri * C::PSTR + g] = pj;
-          Pw[C::R * C::PSTR + g] = mnew;
+            for (int pl = 0; pl < C::QPL; ++pl)
+              *reinterpret_cast<float4*>(q32 + (g * C::QHEAD + pl * C::QPLANE + c * 16) / 4) =
+                  make_float4(f[2 * pl].x * p.qscale, f[2 * pl].y * p.qscale, f[2 * pl + 1].x * p.qscale,
+                              f[2 * pl + 1].y * p.qscale);
+          }
         }
+        __syncwarp();
       }
-      __syncwarp();
-      // rescale, then accumulate p * v
-      float sc[G];
-      {
-        float mn[C::PSTR];
+      if (nvalid > 0) {
+        float2 d[C::TPL][G];
 #pragma unroll
-        for (int g4 = 0; g4 < C::PSTR; g4 += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(Pw + C::R * C::PSTR + g4);
-          mn[g4] = x.x;
-          mn[g4 + 1] = x.y;
-          mn[g4 + 2] = x.z;
-          mn[g4 + 3] = x.w;
+        for (int j = 0; j < C::TPL; ++j)
+#pragma unroll
+          for (int g = 0; g < G; ++g) d[j][g] = make_float2(0.f, 0.f);
+        const unsigned char* krow = sl + C::SL_K + ts * C::RB;
+#pragma unroll
+        for (int st = 0; st < C::CPL; ++st) {
+          const int c = C::chunk_at(st, ts, pq);
+          float2 kf[C::TPL][C::CH2];
+#pragma unroll
+          for (int j = 0; j < C::TPL; ++j) Chunk<T>::unpack(lds128(krow + j * 8 * C::RB + c * 16), kf[j]);
+          const float* qc = q32 + c * 4;
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+#pragma unroll
+            for (int pl = 0; pl < C::QPL; ++pl) {
+              const float4 qv = *reinterpret_cast<const float4*>(qc + (g * C::QHEAD + pl * C::QPLANE) / 4);
+              const float2 q0 = make_float2(qv.x, qv.y), q1 = make_float2(qv.z, qv.w);
+#pragma unroll
+              for (int j = 0; j < C::TPL; ++j) {
+                d[j][g] = ffma2(q0, kf[j][2 * pl], d[j][g]);
+                d[j][g] = ffma2(q1, kf[j][2 * pl + 1], d[j][g]);
+              }
+            }
+          }
         }
+        float sv[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          sc[g] = exp2f(mrun[g] - safe_max_ref(mn[g]));
-          mrun[g] = mn[g];
-          lrun[g] *= sc[g];
+          float v[C::TPL];
 #pragma unroll
-          for (int e = 0; e < C::CH2; ++e) acc[g][e] = fmul2(acc[g][e], make_float2(sc[g], sc[g]));
+          for (int j = 0; j < C::TPL; ++j) {
+            v[j] = d[j][g].x + d[j][g].y;
+            v[j] += __shfl_xor_sync(FULL_MASK, v[j], 1);
+            v[j] += __shfl_xor_sync(FULL_MASK, v[j], 2);
+          }
+          float mine = v[0];
+#pragma unroll
+          for (int j = 1; j < C::TPL; ++j)
+            if (pq == j) mine = v[j];
+          sv[g] = mine;
         }
-      }
-#pragma unroll
-      for (int r = 0; r < C::R; ++r) {
-        const int row = w * (C::RPW * C::R) + r * C::RPW + rg;
-        const uint4 raw = lds128(stg + C::OFF_V + row * C::RB + c * 16);
-        float2 vf[C::CH2];
-        Chunk<T>::unpack(raw, vf);
-        float pr[C::PSTR];
-#pragma unroll
-        for (int g4 = 0; g4 < C::PSTR; g4 += 4) {
-          const float4 x = *reinterpret_cast<const float4*>(Pw + r * C::PSTR + g4);
-          pr[g4] = x.x;
-          pr[g4 + 1] = x.y;
-          pr[g4 + 2] = x.z;
-          pr[g4 + 3] = x.w;
-        }
+        const int myrow = ts + 8 * pq;
+        const float bz = owner ? bias[myrow] : -INFINITY;
+        float sc[G];
+        bool all_one = true;
+        float pv[G];
 #pragma unroll
         for (int g = 0; g < G; ++g) {
-          lrun[g] += pr[g];
-          const float2 pp = make_float2(pr[g], pr[g]);
+          const float xg = sv[g] + bz;
+          const float cm = warp_max(xg);
+          const float mn = fmaxf(mrun[g], cm);
+          const float ms = safe_max_ref(mn);
+          sc[g] = fast_exp2(mrun[g] - ms);
+          all_one = all_one && (mn == mrun[g]);
+          mrun[g] = mn;
+          pv[g] = fast_exp2(xg - ms);
+          lrun[g] = lrun[g] * sc[g] + pv[g];
+        }
+        if (owner) {
+          float* prow = pbuf + myrow * C::PSTR;
 #pragma unroll
-          for (int e = 0; e < C::CH2; ++e) acc[g][e] = ffma2(pp, vf[e], acc[g][e]);
+          for (int g4 = 0; g4 < G; g4 += 4) {
+            float a4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) a4[u] = g4 + u < G ? pv[g4 + u] : 0.f;
+            *reinterpret_cast<float4*>(prow + g4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
+          }
+        }
+        if (!all_one) {
+#pragma unroll
+          for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int e = 0; e < C::CH; ++e) acc[g * C::CH + e] *= sc[g];
+        }
+        __syncwarp();
+#pragma unroll 4
+        for (int r = vr; r < C::TPW; r += C::VR) {
+          float2 vf[C::CH2];
+          Chunk<T>::unpack(lds128(sl + C::SL_V + r * C::RB + vc * 16), vf);
+          float pr[C::PSTR];
+#pragma unroll
+          for (int g4 = 0; g4 < C::PSTR; g4 += 4) {
+            const float4 xx = *reinterpret_cast<const float4*>(pbuf + r * C::PSTR + g4);
+            pr[g4] = xx.x;
+            pr[g4 + 1] = xx.y;
+            pr[g4 + 2] = xx.z;
+            pr[g4 + 3] = xx.w;
+          }
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            const float2 pp = make_float2(pr[g], pr[g]);
+#pragma unroll
+            for (int e = 0; e < C::CH2; ++e) {
+              float2 a2 = make_float2(acc[g * C::CH + 2 * e], acc[g * C::CH + 2 * e + 1]);
+              a2 = ffma2(pp, vf[e], a2);
+              acc[g * C::CH + 2 * e] = a2.x;
+              acc[g * C::CH + 2 * e + 1] = a2.y;
+            }
+          }
         }
       }
     }
+    // the slot is free again: order these reads before the next copy into it
     __syncwarp();
-    if (lane == 0) mbar_arrive(empty + s);
+    fence_proxy_async_smem();
     ++i;
   }
-  if (cur_bh >= 0) flush(cur_bh);
   if (timed_out) {
-    // Give copies that may still be in flight a last bounded chance to land
-    // before this CTA's shared memory is released.
-    for (int s = 0; s < C::S; ++s) {
-      const int last_use = (i - 1 - s) >= 0 ? (i - 1 - s) / C::S : -1;
-      if (last_use >= 0) mbar_wait(full + ((i - 1 - s) % C::S), static_cast<uint32_t>(last_use) & 1u, nullptr);
-    }
+    // give copies that may still be in flight a last bounded chance to land
+    // before this CTA's shared memory is released
+    for (int k = max(0, i - C::S); k < issued; ++k)
+      mbar_wait(bars + (k & (C::S - 1)), static_cast<uint32_t>(k / C::S) & 1u, nullptr);
   }
 }
 

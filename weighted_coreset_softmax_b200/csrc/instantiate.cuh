@@ -12,59 +12,92 @@
 
 namespace kvs {
 
-template <typename T, int D, int G>
+// Raises the kernel's dynamic shared-memory limit once per device and returns how
+// many CTAs fit on one SM.
+template <typename T, int D, int G, bool MMA>
+int attn_prepare(int dev) {
+  using C = AttnCfg<T, D, G, MMA>;
+  static std::atomic<int> blocks_per_sm[64];
+  int v = blocks_per_sm[dev & 63].load();
+  if (v > 0) return v;
+  if (cudaFuncSetAttribute(attn_kernel<T, D, G, MMA>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+      cudaSuccess)
+    return 0;
+  int n = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<T, D, G, MMA>, C::NTHREADS, C::SMEM) !=
+      cudaSuccess)
+    return 0;
+  blocks_per_sm[dev & 63].store(n);
+  return n;
+}
+
+template <typename T, int D, int G, bool MMA>
 cudaError_t attn_launch_one(const AttnParams& p, int grid, cudaStream_t st) {
-  using C = AttnCfg<T, D, G>;
-  static std::atomic<int> configured_mask{0};  // one bit per device: smem limit raised
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (!(configured_mask & (1 << (dev & 31)))) {
-    cudaError_t e = cudaFuncSetAttribute(attn_kernel<T, D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    configured_mask.fetch_or(1 << (dev & 31));
-  }
-  attn_kernel<T, D, G><<<grid, C::NTHREADS, C::SMEM, st>>>(p);
+  using C = AttnCfg<T, D, G, MMA>;
+  attn_kernel<T, D, G, MMA><<<grid, C::NTHREADS, C::SMEM, st>>>(p);
   return cudaGetLastError();
 }
 
-template <typename T, int D>
-cudaError_t attn_launch_td(int G, const AttnParams& p, int grid, cudaStream_t st) {
-  switch (G) {
-    case 1: return attn_launch_one<T, D, 1>(p, grid, st);
-    case 2: return attn_launch_one<T, D, 2>(p, grid, st);
-    case 3: return attn_launch_one<T, D, 3>(p, grid, st);
-    case 4: return attn_launch_one<T, D, 4>(p, grid, st);
-    case 5: return attn_launch_one<T, D, 5>(p, grid, st);
-    case 6: return attn_launch_one<T, D, 6>(p, grid, st);
-    case 7: return attn_launch_one<T, D, 7>(p, grid, st);
-    case 8: return attn_launch_one<T, D, 8>(p, grid, st);
-    default: return cudaErrorInvalidValue;
-  }
+// Tensor-core consumer for bf16 caches, CUDA-core consumer for fp32 (and for
+// bf16 when the caller asks for it).
+template <typename T>
+constexpr bool has_mma() {
+  return sizeof(T) == 2;
 }
 
-// CTAs per SM the attention kernel is built for (its launch bound).
-template <typename T, int D>
-int attn_cps_td(int G) {
-  switch (G) {
-    case 1: return AttnCfg<T, D, 1>::CPS;
-    case 2: return AttnCfg<T, D, 2>::CPS;
-    case 3: return AttnCfg<T, D, 3>::CPS;
-    case 4: return AttnCfg<T, D, 4>::CPS;
-    case 5: return AttnCfg<T, D, 5>::CPS;
-    case 6: return AttnCfg<T, D, 6>::CPS;
-    case 7: return AttnCfg<T, D, 7>::CPS;
-    case 8: return AttnCfg<T, D, 8>::CPS;
-    default: return 1;
+#define KVS_ATTN_SWITCH(FN, ...)                                       \
+  switch (G) {                                                         \
+    case 1: return use_mma ? FN<T, D, 1, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 1, false>(__VA_ARGS__);          \
+    case 2: return use_mma ? FN<T, D, 2, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 2, false>(__VA_ARGS__);          \
+    case 3: return use_mma ? FN<T, D, 3, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 3, false>(__VA_ARGS__);          \
+    case 4: return use_mma ? FN<T, D, 4, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 4, false>(__VA_ARGS__);          \
+    case 5: return use_mma ? FN<T, D, 5, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 5, false>(__VA_ARGS__);          \
+    case 6: return use_mma ? FN<T, D, 6, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 6, false>(__VA_ARGS__);          \
+    case 7: return use_mma ? FN<T, D, 7, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 7, false>(__VA_ARGS__);          \
+    case 8: return use_mma ? FN<T, D, 8, has_mma<T>()>(__VA_ARGS__)     \
+                           : FN<T, D, 8, false>(__VA_ARGS__);          \
+    default: break;                                                    \
   }
+
+template <typename T, int D>
+cudaError_t attn_launch_td(int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
+  KVS_ATTN_SWITCH(attn_launch_one, p, grid, st)
+  return cudaErrorInvalidValue;
+}
+
+template <typename T, int D>
+int attn_prepare_td(int G, bool use_mma, int dev) {
+  KVS_ATTN_SWITCH(attn_prepare, dev)
+  return 0;
+}
+
+template <typename T, int D, int G, int MODE>
+cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
+  static std::atomic<int> configured{0};  // one bit per device: smem limit raised
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const size_t smem = sel_smem_bytes(G, p.NBcap);
+  if (!(configured.load() & (1 << (dev & 31)))) {
+    cudaError_t e = cudaFuncSetAttribute(select_kernel<T, D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sel_smem_bytes(G, SEL_MAXNB)));
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(1 << (dev & 31));
+  }
+  select_kernel<T, D, G, MODE><<<grid, SEL_THREADS, smem, st>>>(p);
+  return cudaGetLastError();
 }
 
 template <typename T, int D, int G>
 cudaError_t select_launch_one(int mode, const SelParams& p, int grid, cudaStream_t st) {
-  if (mode == SEL_SUMMARY)
-    select_kernel<T, D, G, SEL_SUMMARY><<<grid, SEL_THREADS, 0, st>>>(p);
-  else
-    select_kernel<T, D, G, SEL_EXACT><<<grid, SEL_THREADS, 0, st>>>(p);
-  return cudaGetLastError();
+  return mode == SEL_SUMMARY ? select_launch_mode<T, D, G, SEL_SUMMARY>(p, grid, st)
+                             : select_launch_mode<T, D, G, SEL_EXACT>(p, grid, st);
 }
 
 template <typename T, int D>
@@ -89,10 +122,12 @@ cudaError_t select_launch_td(int G, int mode, const SelParams& p, int grid, cuda
 
 // Exported (internal) entry points of this unit.
 namespace kvs {
-cudaError_t KVS_CAT(attn_launch_, KVS_SUFFIX)(int G, const AttnParams& p, int grid, cudaStream_t st) {
-  return attn_launch_td<KVS_T, KVS_D>(G, p, grid, st);
+cudaError_t KVS_CAT(attn_launch_, KVS_SUFFIX)(int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
+  return attn_launch_td<KVS_T, KVS_D>(G, use_mma, p, grid, st);
 }
-int KVS_CAT(attn_cps_, KVS_SUFFIX)(int G) { return attn_cps_td<KVS_T, KVS_D>(G); }
+int KVS_CAT(attn_prepare_, KVS_SUFFIX)(int G, bool use_mma, int dev) {
+  return attn_prepare_td<KVS_T, KVS_D>(G, use_mma, dev);
+}
 cudaError_t KVS_CAT(select_launch_, KVS_SUFFIX)(int G, int mode, const SelParams& p, int grid, cudaStream_t st) {
   return select_launch_td<KVS_T, KVS_D>(G, mode, p, grid, st);
 }

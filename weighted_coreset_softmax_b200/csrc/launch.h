@@ -12,8 +12,10 @@ struct AttnParams;
 struct SelParams;
 
 // dtype: 0 = bf16, 1 = fp32. Return cudaSuccess or the launch error.
-cudaError_t launch_attn(int dtype, int D, int G, const AttnParams& p, int grid, cudaStream_t st);
-int attn_ctas_per_sm(int dtype, int D, int G);
+// use_mma: tensor-core consumer (bf16 only; ignored for fp32).
+cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st);
+// CTAs of the attention kernel that fit on one SM (0 on error).
+int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,

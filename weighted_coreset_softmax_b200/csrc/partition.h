@@ -17,6 +17,7 @@
 namespace kvs {
 
 constexpr int MAX_CTAS = 1024;          // upper bound on attention CTAs per launch
+constexpr int ATTN_NW = 2;              // warps per attention CTA (one partial record each)
 constexpr int MIN_TOKENS_PER_CTA = 64;  // below this a CTA is not worth launching
 constexpr int RANGE_ALIGN = 8;          // CTA token ranges start on multiples of 8
 
@@ -60,15 +61,16 @@ KVS_HD Partition make_partition(int NBH, int P, int num_sms, int ctas_per_sm) {
 }
 
 // ------------------------------------------------------- workspace layout
-// [status word | counters[NBH] | records[MAX_CTAS + NBH] | proxy records[NBH]]
-// A record holds acc[G][D], m[G] (log2 domain), l[G] as fp32, padded to 16 bytes.
+// [status word | counters[NBH] | records[(MAX_CTAS + NBH) * ATTN_NW] | proxy records[NBH]]
+// A record holds acc[G][D], m[G] (log2 domain), l[G] as fp32, padded to 16 bytes;
+// warp w of CTA c writes its record for pair bh at index (c + bh) * ATTN_NW + w.
 KVS_HD int record_floats(int G, int D) { return ((G * D + 2 * G) + 3) & ~3; }
 KVS_HD size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 KVS_HD size_t ws_counters_off() { return 256; }
 KVS_HD size_t ws_records_off(int NBH) { return ws_counters_off() + align256(sizeof(uint32_t) * NBH); }
 KVS_HD size_t ws_proxy_off(int NBH, int G, int D) {
   return ws_records_off(NBH) +
-         align256(sizeof(float) * static_cast<size_t>(record_floats(G, D)) * (MAX_CTAS + NBH));
+         align256(sizeof(float) * static_cast<size_t>(record_floats(G, D)) * (MAX_CTAS + NBH) * ATTN_NW);
 }
 KVS_HD size_t ws_total(int NBH, int G, int D) {
   return ws_proxy_off(NBH, G, D) +

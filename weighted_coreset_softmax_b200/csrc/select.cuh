@@ -7,31 +7,29 @@
 // Equation (8) and the affine score (18)); OSA computes the exact masses from all
 // block keys instead (the OSA paragraph).
 //
-// Design (sm_100a). One thread-block cluster of SEL_CS CTAs per (sequence, KV
-// head). Each CTA scores a contiguous slice of the blocks into shared memory
-// (summary mode: a GEMV over the fp32 key sums, 16-byte loads, transpose
-// reduction; exact mode: all block keys, an online log-sum-exp per block), then
-// the cluster exchanges per-head (max, sum) pairs through distributed shared
-// memory to form the normalisers, each CTA ranks its candidates locally, and the
-// global rank of a candidate is its local rank plus a binary search in every other
-// CTA's sorted candidate list. Selected blocks are written in ascending order.
-// Nothing goes through global scratch memory and no CTA spins on another:
-// cluster barriers are hardware barriers of co-scheduled CTAs.
+// Design (sm_100a). One 256-thread CTA per (sequence, KV head), two per SM.
+//  scoring: summary mode is a GEMV over the fp32 block key sums -- each warp
+//  streams rows with 16-byte loads, several rows in flight per lane, and finishes
+//  the G dot products of a row batch with a transpose reduction; exact mode
+//  streams every key of a block and keeps an online log-sum-exp per head. The
+//  block logits (log2 domain) stay in shared memory.
+//  normalisers: one warp per query head reduces max and sum over the blocks.
+//  ranking: each block gets a 64-bit key (score bits, then the inverted block
+//  index, so larger keys win and ties go to the lower index); a most-significant-
+//  digit-first radix select over those keys, with warp-aggregated shared-memory
+//  histograms, finds the k-th largest key and stops as soon as the remaining
+//  digit bucket is taken whole.
+//  output: a CTA-wide prefix sum over the selected flags writes the kept blocks in
+//  ascending order.
 #pragma once
-
-#include <cooperative_groups.h>
 
 #include "common.cuh"
 
 namespace kvs {
 
-namespace cg = cooperative_groups;
-
-constexpr int SEL_CS = 8;          // CTAs per cluster (one cluster per bh)
-constexpr int SEL_THREADS = 256;   // 8 warps
+constexpr int SEL_THREADS = 256;
 constexpr int SEL_NW = SEL_THREADS / 32;
-constexpr int SEL_MAXNB = 4096;    // NBcap limit
-constexpr int SEL_MAXLOCAL = SEL_MAXNB / SEL_CS;
+constexpr int SEL_MAXNB = 4096;  // NBcap limit
 
 enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1 };
 
@@ -49,21 +47,24 @@ struct SelParams {
   float qscale;  // softmax scale * log2(e)
 };
 
-template <int G>
-struct SelShared {
-  float lg[G][SEL_MAXLOCAL];               // block log2-mass estimates
-  unsigned long long key[SEL_MAXLOCAL];    // ranking keys (0 = not competing)
-  unsigned long long cand[SEL_MAXLOCAL];   // local candidates, descending
-  float2 part[G];                          // per-head (max, sum) over the slice
-  float lse[G];
-  int flag[SEL_MAXLOCAL];
+// Shared memory beyond the dynamic arrays.
+struct SelMisc {
+  float lse[8];
+  unsigned hist[256];
+  unsigned long long prefix, mask;
+  int krem, digit, above, bucket;
   int wsum[SEL_NW];
-  int ncand;
-  int nsel;
 };
 
+// Dynamic shared memory: lg[G][NBP] floats | key[NBP] u64 | misc.
+__host__ __device__ inline int sel_nbp(int NBcap) { return (NBcap + 31) & ~31; }
+__host__ __device__ inline size_t sel_smem_bytes(int G, int NBcap) {
+  const int nbp = sel_nbp(NBcap);
+  return static_cast<size_t>(G) * nbp * 4 + static_cast<size_t>(nbp) * 8 + sizeof(SelMisc);
+}
+
 // Sum of one int per thread over the CTA; every thread gets the result.
-__device__ __forceinline__ int block_sum(int v, int* wsum) {
+__device__ __forceinline__ int sel_block_sum(int v, int* wsum) {
   v = __reduce_add_sync(FULL_MASK, v);
   if ((threadIdx.x & 31) == 0) wsum[threadIdx.x >> 5] = v;
   __syncthreads();
@@ -74,28 +75,16 @@ __device__ __forceinline__ int block_sum(int v, int* wsum) {
   return s;
 }
 
-__device__ __forceinline__ int count_greater(const unsigned long long* arr, int n, unsigned long long x) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (arr[mid] > x)
-      lo = mid + 1;
-    else
-      hi = mid;
-  }
-  return lo;
-}
-
-// Summary mode: s2[g][i] = (q_g * qscale) . k_sum_b / n_b + log2 n_b for the
-// slice [lo, lo + nl) of blocks.
+// Summary mode: lg[g][b] = (q_g * qscale) . k_sum_b / n_b + log2 n_b.
 template <typename T, int D, int G>
-__device__ void score_summary(const SelParams& p, SelShared<G>& sh, int bh, int lo, int nl) {
+__device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv) {
   constexpr int LPR = D / 4;  // fp32 rows, float4 per lane
   constexpr int RPW = 32 / LPR;
   constexpr int GP = pow2ceil(G);
   constexpr int RS0 = LPR / GP;
   constexpr int RS = RS0 < 1 ? 1 : (RS0 > 8 ? 8 : RS0);  // rows per lane per batch
   constexpr int NV = RS * GP;
+  constexpr int BATCH = RPW * RS;                         // rows per warp per batch
   using HV = HeldValues<NV, LPR, GP>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rg = lane / LPR, c = lane % LPR;
@@ -106,53 +95,61 @@ __device__ void score_summary(const SelParams& p, SelShared<G>& sh, int bh, int 
   for (int g = 0; g < G; ++g)
     qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
                         load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
-  const float* ks = p.k_sum + (static_cast<size_t>(bh) * p.NBcap + lo) * D + c * 4;
-  const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap + lo;
-  constexpr int BATCH = RPW * RS;
-  for (int rb = warp * BATCH; rb < nl; rb += SEL_NW * BATCH) {
-    float part[NV];
-    int cnt[RS];
+  const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
+  const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
+  // two batches in flight per warp
+  for (int rb = warp * 2 * BATCH; rb < nbv; rb += SEL_NW * 2 * BATCH) {
+    float4 k4[2][RS];
+    int cnt[2][RS];
 #pragma unroll
-    for (int i = 0; i < RS; ++i) {
-      const int row = rb + i * RPW + rg;
-      float4 k4 = make_float4(0.f, 0.f, 0.f, 0.f);
-      cnt[i] = 0;
-      if (row < nl) {
-        k4 = __ldg(reinterpret_cast<const float4*>(ks + static_cast<size_t>(row) * D));
-        cnt[i] = __ldg(cn + row);
-      }
+    for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        if (g < G) {
-          float d = qf[g].x * k4.x;
-          d = fmaf(qf[g].y, k4.y, d);
-          d = fmaf(qf[g].z, k4.z, d);
-          d = fmaf(qf[g].w, k4.w, d);
-          part[i * GP + g] = d;
-        } else {
-          part[i * GP + g] = 0.f;
+      for (int i = 0; i < RS; ++i) {
+        const int row = rb + u * BATCH + i * RPW + rg;
+        k4[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        cnt[u][i] = 0;
+        if (row < nbv) {
+          k4[u][i] = __ldg(reinterpret_cast<const float4*>(ks + static_cast<size_t>(row) * D));
+          cnt[u][i] = __ldg(cn + row);
         }
       }
-    }
-    transpose_reduce<NV, LPR / 2>(part, lane);
 #pragma unroll
-    for (int j = 0; j < HV::NH; ++j) {
-      const int vi = HV::index(c, j);
-      const int ri = vi / GP, g = vi % GP;
-      const int row = rb + ri * RPW + rg;
-      int nb = cnt[0];
+    for (int u = 0; u < 2; ++u) {
+      float part[NV];
 #pragma unroll
-      for (int i = 1; i < RS; ++i)
-        if (ri == i) nb = cnt[i];
-      if (g < G && row < nl)
-        sh.lg[g][row] = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+      for (int i = 0; i < RS; ++i)
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          if (g < G) {
+            float d = qf[g].x * k4[u][i].x;
+            d = fmaf(qf[g].y, k4[u][i].y, d);
+            d = fmaf(qf[g].z, k4[u][i].z, d);
+            d = fmaf(qf[g].w, k4[u][i].w, d);
+            part[i * GP + g] = d;
+          } else {
+            part[i * GP + g] = 0.f;
+          }
+        }
+      transpose_reduce<NV, LPR / 2>(part, lane);
+#pragma unroll
+      for (int j = 0; j < HV::NH; ++j) {
+        const int vi = HV::index(c, j);
+        const int ri = vi / GP, g = vi % GP;
+        const int row = rb + u * BATCH + ri * RPW + rg;
+        int nb = cnt[u][0];
+#pragma unroll
+        for (int i = 1; i < RS; ++i)
+          if (ri == i) nb = cnt[u][i];
+        if (g < G && row < nbv)
+          lg[g * nbp + row] = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+      }
     }
   }
 }
 
-// Exact mode: s2[g][i] = log2 sum_{r in block} exp2((q_g * qscale) . k_r).
+// Exact mode: lg[g][b] = log2 sum_{r in block} exp2((q_g * qscale) . k_r).
 template <typename T, int D, int G>
-__device__ void score_exact(const SelParams& p, SelShared<G>& sh, int bh, int lo, int nl, int n) {
+__device__ void score_exact(const SelParams& p, float* lg, int nbp, int bh, int nbv, int n) {
   constexpr int ES = sizeof(T);
   constexpr int RB = D * ES;
   constexpr int LPR = RB / 16;
@@ -161,6 +158,7 @@ __device__ void score_exact(const SelParams& p, SelShared<G>& sh, int bh, int lo
   constexpr int R = 4;
   constexpr int GP = pow2ceil(G);
   constexpr int NV = R * GP;
+  constexpr int BATCH = RPW * R;
   using HV = HeldValues<NV, LPR, GP>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int rg = lane / LPR, c = lane % LPR;
@@ -177,10 +175,8 @@ __device__ void score_exact(const SelParams& p, SelShared<G>& sh, int bh, int lo
     for (int e = 0; e < CH2; ++e) qf[g][e] = make_float2(f[e].x * p.qscale, f[e].y * p.qscale);
   }
   const unsigned char* Kb = static_cast<const unsigned char*>(p.K) + static_cast<size_t>(bh) * p.Ncap * RB + c * 16;
-  constexpr int BATCH = RPW * R;
-  for (int i = warp; i < nl; i += SEL_NW) {
-    const int blk = lo + i;
-    const int t0 = blk * p.L;
+  for (int i = warp; i < nbv; i += SEL_NW) {
+    const int t0 = i * p.L;
     const int cnt = min(p.L, n - t0);
     float M[HV::NH], S[HV::NH];
 #pragma unroll
@@ -188,172 +184,220 @@ __device__ void score_exact(const SelParams& p, SelShared<G>& sh, int bh, int lo
       M[j] = -INFINITY;
       S[j] = 0.f;
     }
-    for (int rb = 0; rb < cnt; rb += BATCH) {
-      float part[NV];
+    for (int rb = 0; rb < cnt; rb += 2 * BATCH) {
+      uint4 raw[2][R];
 #pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const int row = rb + r * RPW + rg;
-        uint4 raw = make_uint4(0, 0, 0, 0);
-        if (row < cnt) raw = __ldcs(reinterpret_cast<const uint4*>(Kb + static_cast<size_t>(t0 + row) * RB));
-        float2 kf[CH2];
-        Chunk<T>::unpack(raw, kf);
+      for (int u = 0; u < 2; ++u)
 #pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          if (g < G) {
-            float2 a2 = make_float2(0.f, 0.f);
+        for (int r = 0; r < R; ++r) {
+          const int row = rb + u * BATCH + r * RPW + rg;
+          raw[u][r] = row < cnt ? __ldcs(reinterpret_cast<const uint4*>(Kb + static_cast<size_t>(t0 + row) * RB))
+                                : make_uint4(0, 0, 0, 0);
+        }
 #pragma unroll
-            for (int e = 0; e < CH2; ++e) a2 = ffma2(qf[g][e], kf[e], a2);
-            part[r * GP + g] = a2.x + a2.y;
-          } else {
-            part[r * GP + g] = 0.f;
+      for (int u = 0; u < 2; ++u) {
+        if (rb + u * BATCH >= cnt) break;  // warp-uniform
+        float part[NV];
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+          float2 kf[CH2];
+          Chunk<T>::unpack(raw[u][r], kf);
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            if (g < G) {
+              float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+              for (int e = 0; e < CH2; ++e) a2 = ffma2(qf[g][e], kf[e], a2);
+              part[r * GP + g] = a2.x + a2.y;
+            } else {
+              part[r * GP + g] = 0.f;
+            }
           }
         }
-      }
-      transpose_reduce<NV, LPR / 2>(part, lane);
+        transpose_reduce<NV, LPR / 2>(part, lane);
 #pragma unroll
-      for (int j = 0; j < HV::NH; ++j) {
-        const int vi = HV::index(c, j);
-        const int ri = vi / GP;
-        const int row = rb + ri * RPW + rg;
-        const float s = row < cnt ? part[j] : -INFINITY;
-        // reduce over every lane bit that changes the row: the row bits inside a
-        // row group and the row-group bits above them
-        float cm = s;
+        for (int j = 0; j < HV::NH; ++j) {
+          const int vi = HV::index(c, j);
+          const int ri = vi / GP;
+          const int row = rb + u * BATCH + ri * RPW + rg;
+          const float sv = row < cnt ? part[j] : -INFINITY;
+          // reduce over every lane bit that changes the row: the row bits inside
+          // a row group and the row-group bits above them
+          float cm = sv;
 #pragma unroll
-        for (int mask = HV::ROW_MASK_LO; mask < 32; mask <<= 1) cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, mask));
-        const float Mn = fmaxf(M[j], cm);  // finite: row rb of the batch is valid
-        float e = exp2f(s - Mn);
+          for (int mask = HV::ROW_MASK_LO; mask < 32; mask <<= 1)
+            cm = fmaxf(cm, __shfl_xor_sync(FULL_MASK, cm, mask));
+          const float Mn = fmaxf(M[j], cm);  // finite: the batch's first row is valid
+          float e = exp2f(sv - Mn);
 #pragma unroll
-        for (int mask = HV::ROW_MASK_LO; mask < 32; mask <<= 1) e += __shfl_xor_sync(FULL_MASK, e, mask);
-        S[j] = S[j] * exp2f(M[j] - Mn) + e;
-        M[j] = Mn;
+          for (int mask = HV::ROW_MASK_LO; mask < 32; mask <<= 1) e += __shfl_xor_sync(FULL_MASK, e, mask);
+          S[j] = S[j] * exp2f(M[j] - Mn) + e;
+          M[j] = Mn;
+        }
       }
     }
 #pragma unroll
     for (int j = 0; j < HV::NH; ++j) {
       const int g = HV::index(c, j) % GP;
-      if (g < G) sh.lg[g][i] = cnt > 0 ? M[j] + log2f(S[j]) : -INFINITY;
+      if (g < G) lg[g * nbp + i] = cnt > 0 ? M[j] + log2f(S[j]) : -INFINITY;
     }
   }
 }
 
 template <typename T, int D, int G, int MODE>
-__global__ void __cluster_dims__(SEL_CS, 1, 1) __launch_bounds__(SEL_THREADS)
-    select_kernel(const SelParams p) {
-  __shared__ SelShared<G> sh;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int rank = static_cast<int>(cluster.block_rank());
-  const int bh = blockIdx.x / SEL_CS;
+__global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams p) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
+  const int nbp = sel_nbp(p.NBcap);
+  float* lg = reinterpret_cast<float*>(sel_smem);
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(sel_smem + static_cast<size_t>(G) * nbp * 4);
+  SelMisc& ms = *reinterpret_cast<SelMisc*>(sel_smem + static_cast<size_t>(G) * nbp * 4 + static_cast<size_t>(nbp) * 8);
+  const int bh = blockIdx.x;
   const int b = bh / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
-  const int per = (nbv + SEL_CS - 1) / SEL_CS;
-  const int lo = min(nbv, rank * per);
-  const int nl = min(nbv, lo + per) - lo;
 
   if (MODE == SEL_SUMMARY)
-    score_summary<T, D, G>(p, sh, bh, lo, nl);
+    score_summary<T, D, G>(p, lg, nbp, bh, nbv);
   else
-    score_exact<T, D, G>(p, sh, bh, lo, nl, n);
+    score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
   __syncthreads();
 
-  // per-head (max, sum of 2^(s - max)) over this slice
+  // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain)
   if (warp < G) {
     float M = -INFINITY;
-    for (int i = lane; i < nl; i += 32) M = fmaxf(M, sh.lg[warp][i]);
+    for (int i = lane; i < nbv; i += 32) M = fmaxf(M, lg[warp * nbp + i]);
     M = warp_max(M);
     float S = 0.f;
     if (M != -INFINITY)
-      for (int i = lane; i < nl; i += 32) S += exp2f(sh.lg[warp][i] - M);
+      for (int i = lane; i < nbv; i += 32) S += exp2f(lg[warp * nbp + i] - M);
     S = warp_sum(S);
-    if (lane == 0) sh.part[warp] = make_float2(M, S);
-  }
-  cluster.sync();
-  if (tid < G) {
-    float M = -INFINITY;
-    for (int r = 0; r < SEL_CS; ++r) M = fmaxf(M, cluster.map_shared_rank(&sh.part[tid], r)->x);
-    float S = 0.f;
-    if (M != -INFINITY)
-      for (int r = 0; r < SEL_CS; ++r) {
-        const float2 pr = *cluster.map_shared_rank(&sh.part[tid], r);
-        S += pr.y * exp2f(pr.x - M);
-      }
-    sh.lse[tid] = (M == -INFINITY || S <= 0.f) ? -INFINITY : M + log2f(S);
+    if (lane == 0) ms.lse[warp] = (M == -INFINITY || S <= 0.f) ? -INFINITY : M + log2f(S);
   }
   __syncthreads();
 
-  // group score (Equation 5) and ranking keys
-  for (int i = tid; i < nl; i += SEL_THREADS) {
+  // group score and ranking keys
+  int ncand = 0;
+  for (int i = tid; i < nbv; i += SEL_THREADS) {
     float Sg = 0.f;
 #pragma unroll
     for (int g = 0; g < G; ++g)
-      if (sh.lse[g] != -INFINITY) Sg += exp2f(sh.lg[g][i] - sh.lse[g]);
-    const int blk = lo + i;
-    if (p.scores) p.scores[static_cast<size_t>(bh) * p.NBcap + blk] = Sg;
-    const bool forced = (p.force_first && blk == 0) || (p.force_last && blk == nbv - 1);
-    sh.key[i] = forced ? 0ull
-                       : ((static_cast<unsigned long long>(__float_as_uint(Sg)) << 32) |
-                          static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(blk)));
-    sh.flag[i] = forced ? 1 : 0;
+      if (ms.lse[g] != -INFINITY) Sg += exp2f(lg[g * nbp + i] - ms.lse[g]);
+    if (p.scores) p.scores[static_cast<size_t>(bh) * p.NBcap + i] = Sg;
+    const bool forced = (p.force_first && i == 0) || (p.force_last && i == nbv - 1);
+    key[i] = forced ? 0ull
+                    : ((static_cast<unsigned long long>(__float_as_uint(Sg)) << 32) |
+                       static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(i)));
+    ncand += !forced;
   }
-  if (p.scores) {
-    // blocks past the sequence: score 0, split over the cluster
-    const int tail = p.NBcap - nbv;
-    const int tper = (tail + SEL_CS - 1) / SEL_CS;
-    const int a0 = nbv + rank * tper, a1 = min(p.NBcap, a0 + tper);
-    for (int blk = a0 + tid; blk < a1; blk += SEL_THREADS) p.scores[static_cast<size_t>(bh) * p.NBcap + blk] = 0.f;
-  }
-  __syncthreads();
+  if (p.scores)
+    for (int i = nbv + tid; i < p.NBcap; i += SEL_THREADS) p.scores[static_cast<size_t>(bh) * p.NBcap + i] = 0.f;
+  ncand = sel_block_sum(ncand, ms.wsum);  // also orders the key writes
 
-  // local ranks; the best min(k, candidates) go to cand[] in descending order
+  // threshold: select keys with (key & mask) >= prefix
+  unsigned long long prefix = 1ull, mask = ~0ull;  // default: every candidate
+  if (p.k_top <= 0) {
+    prefix = ~0ull;  // nothing competes successfully
+  } else if (p.k_top < ncand) {
+    if (tid == 0) {
+      ms.prefix = 0ull;
+      ms.mask = 0ull;
+      ms.krem = p.k_top;
+    }
+    for (int shift = 56; shift >= 0; shift -= 8) {
+      if (tid < 256) ms.hist[tid] = 0u;
+      __syncthreads();
+      const unsigned long long pf = ms.prefix, mk = ms.mask;
+      for (int i0 = 0; i0 < nbv; i0 += SEL_THREADS) {
+        const int i = i0 + tid;
+        int d = -1;
+        if (i < nbv) {
+          const unsigned long long x = key[i];
+          if (x != 0ull && (x & mk) == pf) d = static_cast<int>((x >> shift) & 0xffull);
+        }
+        // warp-aggregated histogram update
+        const unsigned peers = __match_any_sync(FULL_MASK, d);
+        if (d >= 0 && (__ffs(peers) - 1) == lane) atomicAdd(&ms.hist[d], static_cast<unsigned>(__popc(peers)));
+      }
+      __syncthreads();
+      if (warp == 0) {
+        // lane l covers digits 255-8l .. 248-8l (descending)
+        unsigned h8[8];
+        unsigned tot = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          h8[j] = ms.hist[255 - 8 * lane - j];
+          tot += h8[j];
+        }
+        unsigned incl = tot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned v = __shfl_up_sync(FULL_MASK, incl, o);
+          if (lane >= o) incl += v;
+        }
+        const unsigned before = incl - tot;  // keys in higher digits than this lane's
+        const unsigned krem = static_cast<unsigned>(ms.krem);
+        if (before < krem && krem <= incl) {
+          unsigned run = before;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (run < krem && krem <= run + h8[j]) {
+              ms.digit = 255 - 8 * lane - j;
+              ms.above = static_cast<int>(run);
+              ms.bucket = static_cast<int>(h8[j]);
+            }
+            run += h8[j];
+          }
+        }
+      }
+      __syncthreads();
+      if (tid == 0) {
+        ms.krem -= ms.above;
+        ms.prefix |= static_cast<unsigned long long>(ms.digit) << shift;
+        ms.mask |= 0xffull << shift;
+      }
+      __syncthreads();
+      if (ms.bucket == ms.krem) break;  // the whole bucket is taken: done (uniform)
+    }
+    prefix = ms.prefix;
+    mask = ms.mask;
+  }
+
+  // ascending compaction of the selected blocks (forced ones included)
+  const int per = (nbv + SEL_THREADS - 1) / SEL_THREADS;
+  const int a0 = min(nbv, tid * per), a1 = min(nbv, a0 + per);
   int mine = 0;
-  for (int i = tid; i < nl; i += SEL_THREADS) {
-    const unsigned long long x = sh.key[i];
-    if (x == 0ull) continue;
-    ++mine;
-    int r = 0;
-    for (int j = 0; j < nl; ++j) r += sh.key[j] > x;
-    if (r < p.k_top) sh.cand[r] = x;
+  for (int i = a0; i < a1; ++i) {
+    const unsigned long long x = key[i];
+    const bool forced = (p.force_first && i == 0) || (p.force_last && i == nbv - 1);
+    mine += forced || (x != 0ull && (x & mask) >= prefix);
   }
-  mine = block_sum(mine, sh.wsum);
-  if (tid == 0) sh.ncand = min(mine, p.k_top);
-  cluster.sync();
-
-  // global rank = local rank + candidates of other CTAs that beat it
-  for (int r = tid; r < sh.ncand; r += SEL_THREADS) {
-    const unsigned long long x = sh.cand[r];
-    int grank = r;
-    for (int q = 0; q < SEL_CS; ++q) {
-      if (q == rank) continue;
-      const SelShared<G>* other = cluster.map_shared_rank(&sh, q);
-      grank += count_greater(other->cand, other->ncand, x);
-    }
-    if (grank < p.k_top) {
-      const int blk = static_cast<int>(0xffffffffu - static_cast<uint32_t>(x & 0xffffffffull));
-      sh.flag[blk - lo] = 1;
-    }
+  // exclusive scan over the CTA
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(FULL_MASK, incl, o);
+    if (lane >= o) incl += v;
   }
+  if (lane == 31) ms.wsum[warp] = incl;
   __syncthreads();
-  int nflag = 0;
-  for (int i = tid; i < nl; i += SEL_THREADS) nflag += sh.flag[i];
-  nflag = block_sum(nflag, sh.wsum);
-  if (tid == 0) sh.nsel = nflag;
-  cluster.sync();
-  int offset = 0, total = 0;
-  for (int q = 0; q < SEL_CS; ++q) {
-    const int v = cluster.map_shared_rank(&sh, q)->nsel;
-    if (q < rank) offset += v;
+  int wbase = 0, total = 0;
+#pragma unroll
+  for (int w = 0; w < SEL_NW; ++w) {
+    const int v = ms.wsum[w];
+    if (w < warp) wbase += v;
     total += v;
   }
-  for (int i = tid; i < nl; i += SEL_THREADS) {
-    if (!sh.flag[i]) continue;
-    int pos = offset;
-    for (int j = 0; j < i; ++j) pos += sh.flag[j];
-    if (pos < p.kmax) p.block_idx[static_cast<size_t>(bh) * p.kmax + pos] = lo + i;
+  int pos = wbase + incl - mine;
+  for (int i = a0; i < a1; ++i) {
+    const unsigned long long x = key[i];
+    const bool forced = (p.force_first && i == 0) || (p.force_last && i == nbv - 1);
+    if (forced || (x != 0ull && (x & mask) >= prefix)) {
+      if (pos < p.kmax) p.block_idx[static_cast<size_t>(bh) * p.kmax + pos] = i;
+      ++pos;
+    }
   }
-  if (rank == 0 && tid == 0) p.n_kept[bh] = min(total, p.kmax);
-  cluster.sync();
+  if (tid == 0) p.n_kept[bh] = min(total, p.kmax);
 }
 
 }  // namespace kvs
