@@ -1,0 +1,42 @@
+"""The CUDA-core attention consumer on bf16 caches (selected by KVSPARSE_ATTN=fma,
+read once per process) against the float64 oracle, run in a child process."""
+import os
+import subprocess
+import sys
+
+import pytest
+
+pytestmark = pytest.mark.gpu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+SCRIPT = r"""
+import sys
+sys.path.insert(0, {root!r}); sys.path.insert(0, {tests!r})
+import numpy as np, torch
+import weighted_coreset_softmax_b200 as kv
+from weighted_coreset_softmax_b200 import workloads as W
+from oracle import oracle as O
+from gpu_helpers import all_pairs, check_out, oracle_inputs, run_pipeline, selection_matches
+for name, kw in (("llama", dict(B=2, Ncap=3100, seq_lens=[3100, 777], budget=0.05)),
+                 ("qwen_long", dict(B=1, Ncap=2100, k_top=3))):
+    wl = W.make(name, "cuda", **kw)
+    r = run_pipeline(wl)
+    q, K, V = oracle_inputs(wl)
+    gi, gn = r["idx"].cpu().numpy(), r["nk"].cpu().numpy()
+    kept = {{(b, h): [int(x) for x in gi[b, h, :gn[b, h]]] for (b, h) in all_pairs(wl)}}
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, kept, True)
+    check_out(r["out"], r["lse"], ro, rl, what=name + " cuda-core consumer")
+    sl = wl.seq_lens_tensor("cuda")
+    out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, r["ws"])
+    do, dl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
+    check_out(out, lse, do, dl, what=name + " cuda-core dense")
+print("ok")
+"""
+
+
+def test_cuda_core_consumer_on_bf16():
+    env = dict(os.environ, KVSPARSE_ATTN="fma")
+    code = SCRIPT.format(root=ROOT, tests=os.path.join(ROOT, "tests"))
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "ok" in r.stdout, r.stdout[-3000:] + r.stderr[-3000:]

@@ -1,6 +1,7 @@
 // C ABI of libkvsparse: argument validation and kernel dispatch. Every check
 // runs on the host before anything is launched; kernels are enqueued on the
 // caller's stream and nothing here allocates device memory.
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -9,6 +10,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <string>
 
 #include "attention.cuh"
@@ -19,10 +21,14 @@
 
 namespace kvs {
 
-cudaError_t attn_launch_bf16_d64(int, bool, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_bf16_d128(int, bool, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_f32_d64(int, bool, const AttnParams&, int, cudaStream_t);
-cudaError_t attn_launch_f32_d128(int, bool, const AttnParams&, int, cudaStream_t);
+cudaError_t attn_launch_bf16_d64(int, bool, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int,
+                                  cudaStream_t);
+cudaError_t attn_launch_bf16_d128(int, bool, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int,
+                                  cudaStream_t);
+cudaError_t attn_launch_f32_d64(int, bool, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int,
+                                  cudaStream_t);
+cudaError_t attn_launch_f32_d128(int, bool, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int,
+                                  cudaStream_t);
 int attn_prepare_bf16_d64(int, bool, int);
 int attn_prepare_bf16_d128(int, bool, int);
 int attn_prepare_f32_d64(int, bool, int);
@@ -32,10 +38,12 @@ cudaError_t select_launch_bf16_d128(int, int, const SelParams&, int, cudaStream_
 cudaError_t select_launch_f32_d64(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_f32_d128(int, int, const SelParams&, int, cudaStream_t);
 
-cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
+cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int grid, cudaStream_t st) {
   if (dtype == KV_BF16)
-    return D == 64 ? attn_launch_bf16_d64(G, use_mma, p, grid, st) : attn_launch_bf16_d128(G, use_mma, p, grid, st);
-  return D == 64 ? attn_launch_f32_d64(G, false, p, grid, st) : attn_launch_f32_d128(G, false, p, grid, st);
+    return D == 64 ? attn_launch_bf16_d64(G, use_mma, p, tk, tv, grid, st)
+                   : attn_launch_bf16_d128(G, use_mma, p, tk, tv, grid, st);
+  return D == 64 ? attn_launch_f32_d64(G, false, p, tk, tv, grid, st) : attn_launch_f32_d128(G, false, p, tk, tv, grid, st);
 }
 int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev) {
   if (dtype == KV_BF16)
@@ -148,6 +156,52 @@ bool attention_uses_tensor_cores() {
   return v;
 }
 
+// Tiled 2-D tensor map over a [rows][D] bf16 cache: boxes of 32 rows x 64
+// elements (128 bytes), 128-byte swizzle, zero fill past the last row. Encoded
+// through the driver entry point (no link against the driver library); the last
+// few maps are cached, keyed by address and extent.
+kv_status encode_kv_map(const void* base, uint64_t rows, int D, CUtensorMap* out) {
+  using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                              const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                              CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static Encode encode = nullptr;
+  static std::mutex mu;
+  struct Entry {
+    const void* base;
+    uint64_t rows;
+    int D;
+    CUtensorMap map;
+  };
+  static Entry cache[16];
+  static int next_slot = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Entry& e : cache)
+    if (e.base == base && e.rows == rows && e.D == D) {
+      *out = e.map;
+      return KV_OK;
+    }
+  if (!encode) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess || !fn)
+      return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    encode = reinterpret_cast<Encode>(fn);
+  }
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t estr[2] = {1, 1};
+  CUtensorMap m;
+  const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KV_ERR_CUDA, "tensor map encoding failed (CUresult %d)", static_cast<int>(r));
+  cache[next_slot] = Entry{base, rows, D, m};
+  next_slot = (next_slot + 1) % 16;
+  *out = m;
+  return KV_OK;
+}
+
 int num_sms_current() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -207,7 +261,9 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   if (sms <= 0) return fail(KV_ERR_CUDA, "no CUDA device available");
   int dev = 0;
   cudaGetDevice(&dev);
-  const bool use_mma = attention_uses_tensor_cores();
+  // tensor cores: bf16 caches, block and dense modes (gathered coreset rows use
+  // the CUDA-core consumer)
+  const bool use_mma = attention_uses_tensor_cores() && s->dtype == KV_BF16 && mode != kvs::ATTN_WEIGHTED;
   const int cps = kvs::attn_ctas_per_sm(s->dtype, s->D, G, use_mma, dev);
   if (cps <= 0) return fail(KV_ERR_CUDA, "attention kernel does not fit on an SM");
   kvs::AttnParams p{};
@@ -244,8 +300,19 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   p.mode = mode;
   p.use_proxy = use_proxy ? 1 : 0;
   p.qscale = scale * 1.4426950408889634f;
-  p.part = kvs::make_partition(NBH, P, sms, cps);
-  cudaError_t e = kvs::launch_attn(s->dtype, s->D, G, use_mma, p, p.part.C, reinterpret_cast<cudaStream_t>(stream));
+  p.part = kvs::make_partition(NBH, P, static_cast<int64_t>(sms) * cps * kvs::ATTN_NW);
+  CUtensorMap tk, tv;
+  std::memset(&tk, 0, sizeof(tk));
+  std::memset(&tv, 0, sizeof(tv));
+  if (use_mma) {
+    const uint64_t rows = static_cast<uint64_t>(NBH) * s->Ncap;
+    if (rows > 0x7fffffffull) return fail(KV_ERR_UNSUPPORTED, "B * Hkv * Ncap = %llu rows is too many", (unsigned long long)rows);
+    KV_TRY(encode_kv_map(K, rows, s->D, &tk));
+    KV_TRY(encode_kv_map(V, rows, s->D, &tv));
+  }
+  cudaError_t e =
+      kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),
+                       reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "attention launch");
   return KV_OK;
 }

@@ -14,14 +14,14 @@
 //    dense attention reads the whole cache.
 //
 // Design (sm_100a). All (sequence, KV head) pairs ("bh") lay their P token slots
-// end to end on one axis; the grid cuts that axis into equal contiguous ranges,
-// one per CTA, so every SM streams the same bytes whatever the per-head work.
-// A CTA walks its range in chunks of TR rows that stay inside one bh (and, in
-// block mode, one kept block); warp w owns rows [16w, 16w + 16) of every chunk.
-// Each warp is an independent pipeline: it moves its rows' K and V (and, at the
-// start of a bh, the group's q) into its own two-slot shared-memory ring with
-// cp.async.bulk, tracked by its own mbarriers, and refills a slot as soon as it
-// has consumed it; the per-chunk indices are prefetched one chunk ahead.
+// end to end on one axis; the launch cuts that axis into equal contiguous ranges,
+// one per warp ("worker"), so every SM streams the same bytes whatever the
+// per-head work. A worker walks its range in chunks of TR rows that stay inside
+// one bh (and, in block mode, one kept block). Each worker is an independent
+// pipeline: it moves its chunks' K and V (and, at the start of a bh, the group's
+// q) into its own two-slot shared-memory ring with bulk copies, tracked by its
+// own mbarriers, and refills a slot as soon as it has consumed it; the per-chunk
+// indices are loaded 32 chunks at a time, one batch ahead.
 //  q.k: four lanes share a group of two tokens (each lane reads a quarter of
 //  each row); q is held once per warp in fp32, prescaled by scale*log2(e), split
 //  into two 16-byte planes per chunk; every lane visits its row chunks in a
@@ -33,9 +33,10 @@
 //  softmax: per warp, in the log2 domain; the running maximum is uniform across
 //  the warp, so partial states merge without rescaling.
 //  p.v: lanes own 16-byte channel chunks of V rows, packed f32x2 FMAs.
-// For bf16 caches a tensor-core consumer replaces the CUDA-core one (warp-chunks
-// of 32 rows, copied one row per lane into rows padded by 16 bytes so that the
-// 8x8 ldmatrix tiles are conflict-free): q.k is mma.sync m16n8k16 with the 16
+// For bf16 caches in block and dense modes a tensor-core consumer replaces the
+// CUDA-core one: warp-chunks of 32 rows move with tiled tensor copies (two boxes
+// of 32 rows x 128 bytes per tensor for d = 128) into 128-byte-swizzled tiles, so
+// the 8x8 ldmatrix reads are conflict-free; q.k is mma.sync m16n8k16 with the 16
 // tokens of a tile as M and the G <= 8 query heads as N (q^T fragments stay in
 // registers for the whole bh), so the bf16 products are exact and accumulate in
 // fp32; the softmax runs on the accumulator fragments; P is split into a bf16
@@ -48,6 +49,8 @@
 // arriver merges all records of the bh (and the proxy record) into the output.
 // No warp ever waits for another.
 #pragma once
+
+#include <cuda.h>
 
 #include <climits>
 
@@ -87,13 +90,13 @@ struct AttnParams {
 };
 
 // Shape constants of one instantiation. MMA selects the tensor-core consumer
-// (bf16 caches): 32 rows per warp-chunk in padded rows; otherwise the CUDA-core
+// (bf16 caches, block and dense modes): 32 rows per warp-chunk, K and V moved by
+// tiled tensor copies into 128-byte-swizzled tiles; otherwise the CUDA-core
 // consumer: 16 rows per warp-chunk in dense rows.
 template <typename T, int D, int G, bool MMA>
 struct AttnCfg {
   static constexpr int ES = sizeof(T);
   static constexpr int RB = D * ES;          // bytes per cached row
-  static constexpr int RS = MMA ? RB + 16 : RB;  // bytes per row in shared memory
   static constexpr int CPR = RB / 16;        // 16-byte chunks per row
   static constexpr int CH = 16 / ES;         // elements per chunk
   static constexpr int CH2 = CH / 2;         // float2 pairs per chunk
@@ -103,32 +106,36 @@ struct AttnCfg {
   static constexpr int TPW = MMA ? 32 : 8 * TPL;  // rows per warp per chunk
   static constexpr int NW = ATTN_NW;         // warps per CTA
   static constexpr int NTHREADS = NW * 32;
-  static constexpr int TR = NW * TPW;        // rows per chunk
+  static constexpr int TR = TPW;             // rows per chunk (one worker)
   static constexpr int S = 2;                // ring slots per warp
   static constexpr int VR = 32 / CPR;        // V rows per p.v step (CUDA-core)
   static constexpr int KS = D / 16;          // k-steps of q.k and d-tiles of p.v (MMA)
+  static constexpr int KH = MMA ? RB / 128 : 1;   // 128-byte column boxes per row (MMA)
+  static constexpr int BOX = TPW * 128;      // bytes of one swizzled box (MMA)
   static constexpr int QPL = CH / 4;         // 16-byte planes of fp32 q per chunk
   static constexpr int QPLANE = CPR * 16;    // bytes of one plane of one head
   static constexpr int QHEAD = QPL * QPLANE; // bytes of one head of q (fp32)
   static constexpr int QBYTES = G * RB;      // q of one KV head's group, input type
   static constexpr int PSTR = G <= 4 ? 4 : 8;
-  // one ring slot: K rows | V rows | raw q | bias | header
+  // one ring slot: K rows | V rows | raw q | bias | header (1024-byte aligned
+  // for the swizzled tiles)
   static constexpr int SL_K = 0;
-  static constexpr int SL_V = TPW * RS;
-  static constexpr int SL_Q = 2 * TPW * RS;
+  static constexpr int SL_V = TPW * RB;
+  static constexpr int SL_Q = 2 * TPW * RB;
   static constexpr int SL_BIAS = SL_Q + QBYTES;
   static constexpr int SL_HDR = SL_BIAS + TPW * 4;
-  static constexpr int SLOT = (SL_HDR + 16 + 127) & ~127;
+  static constexpr int SLOT = MMA ? (SL_HDR + 16 + 1023) & ~1023 : (SL_HDR + 16 + 127) & ~127;
   // one warp: S slots | q fp32 | p | barriers (q fp32 and p: CUDA-core only)
   static constexpr int W_Q = S * SLOT;
   static constexpr int W_P = W_Q + (MMA ? 0 : G * QHEAD);
   static constexpr int W_BAR = W_P + (MMA ? 0 : TPW * PSTR * 4);
-  static constexpr int W_BYTES = (W_BAR + S * 8 + 127) & ~127;
-  static constexpr int SMEM = NW * W_BYTES;
+  static constexpr int W_BYTES = MMA ? (W_BAR + S * 8 + 1023) & ~1023 : (W_BAR + S * 8 + 127) & ~127;
+  static constexpr int ALIGN_SLACK = MMA ? 1024 : 0;
+  static constexpr int SMEM = NW * W_BYTES + ALIGN_SLACK;
   static constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   static_assert(MMA || CPL == 2 || CPL == 4 || CPL == 8, "chunks per lane");
   static_assert(MMA || (VR >= 1 && 32 % CPR == 0 && TPW % VR == 0), "p.v row layout");
-  static_assert(!MMA || (ES == 2 && G <= 8 && D % 16 == 0), "tensor-core consumer: bf16, G <= 8");
+  static_assert(!MMA || (ES == 2 && G <= 8 && RB % 128 == 0), "tensor-core consumer: bf16, G <= 8");
   static_assert(TPW <= 32, "one row per lane when issuing copies");
   static_assert((S & (S - 1)) == 0, "ring slots must be a power of two");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
@@ -139,6 +146,11 @@ struct AttnCfg {
   __device__ __forceinline__ static int chunk_at(int st, int ts, int pq) {
     const int rot = CPL == 2 ? 0 : (CPL == 4 ? 2 * (pq >> 1) : 2 * pq);
     return pq * CPL + ((st + (ts & 1) + rot) & (CPL - 1));
+  }
+  // Tensor core: byte offset of 16-byte chunk c of row r in a slot's K or V
+  // tiles (128-byte swizzle: chunk c of a 128-byte line sits at c ^ (r mod 8)).
+  __device__ __forceinline__ static int swz(int r, int c) {
+    return (c >> 3) * BOX + r * 128 + (((c & 7) ^ (r & 7)) << 4);
   }
 };
 
@@ -225,11 +237,11 @@ struct ChunkMeta {
   int blk;     // block mode: block index of the chunk's slot
 };
 
-__device__ __forceinline__ int first_cta(const Partition& pt, int bh) {
-  return part_cta_of(pt, static_cast<int64_t>(bh) * pt.P);
+__device__ __forceinline__ int first_worker(const Partition& pt, int bh) {
+  return part_worker_of(pt, static_cast<int64_t>(bh) * pt.P);
 }
-__device__ __forceinline__ int last_cta(const Partition& pt, int bh) {
-  return part_cta_of(pt, static_cast<int64_t>(bh) * pt.P + pt.P - 1);
+__device__ __forceinline__ int last_worker(const Partition& pt, int bh) {
+  return part_worker_of(pt, static_cast<int64_t>(bh) * pt.P + pt.P - 1);
 }
 
 // Merges every partial record of one bh into out / lse. One warp. The records'
@@ -240,11 +252,11 @@ template <int D, int G>
 __device__ void finalize_bh(const AttnParams& p, int bh, int lane) {
   constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   constexpr int VEC = D / 32;
-  const int cf = first_cta(p.part, bh), cl = last_cta(p.part, bh);
-  const int nattn = (cl - cf + 1) * ATTN_NW;
+  const int cf = first_worker(p.part, bh), cl = last_worker(p.part, bh);
+  const int nattn = cl - cf + 1;
   const int nrec = nattn + (p.use_proxy ? 1 : 0);
   const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
-  const float* base = p.recs + static_cast<size_t>(cf + bh) * ATTN_NW * RECF;
+  const float* base = p.recs + static_cast<size_t>(cf + bh) * RECF;
   auto rec_ptr = [&](int j) -> const float* {
     return j < nattn ? base + static_cast<size_t>(j) * RECF : p.proxy_recs + static_cast<size_t>(bh) * RECF;
   };
@@ -314,7 +326,7 @@ template <int D, int G>
 __device__ __forceinline__ void arrive_bh(const AttnParams& p, int bh, int lane) {
   int last = 0;
   if (lane == 0) {
-    const int E = (last_cta(p.part, bh) - first_cta(p.part, bh) + 1) * ATTN_NW + (p.use_proxy ? 1 : 0);
+    const int E = (last_worker(p.part, bh) - first_worker(p.part, bh) + 1) + (p.use_proxy ? 1 : 0);
     const uint32_t old = atomicAdd(p.counters + bh, 1u);
     last = (old + 1 == static_cast<uint32_t>(E));
     if (last) p.counters[bh] = 0u;  // ready for the next launch
@@ -455,14 +467,17 @@ __device__ void build_proxy(const AttnParams& p, int bh, int lane) {
 }
 
 template <typename T, int D, int G, bool MMA>
-__global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
+    attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using C = AttnCfg<T, D, G, MMA>;
-  extern __shared__ __align__(128) unsigned char smem[];
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  // swizzled tiles need 1024-byte alignment
+  unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u) * (MMA ? 1 : 0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int cta = blockIdx.x;
-  const int64_t t0 = part_t0(p.part, cta);
-  const int64_t t1 = part_t0(p.part, cta + 1);
+  const int wk = blockIdx.x * C::NW + warp;  // this worker
+  const int64_t t0 = part_t0(p.part, wk);
+  const int64_t t1 = part_t0(p.part, wk + 1);
   const int P = p.part.P;
   unsigned char* wb = smem + warp * C::W_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wb + C::W_BAR);
@@ -474,17 +489,19 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
     for (int s = 0; s < C::S; ++s) mbar_init(bars + s, 1);
     fence_mbar_init();
   }
-  // Rows a chunk does not fill keep stale (finite) data; zero the ring once so
-  // that no uninitialised pattern is ever multiplied by p = 0.
-  for (int i = lane; i < C::S * C::SLOT / 16; i += 32) reinterpret_cast<uint4*>(wb)[i] = make_uint4(0, 0, 0, 0);
-  fence_proxy_async_smem();
+  if constexpr (!MMA) {
+    // Rows a chunk does not fill keep stale (finite) data; zero the ring once so
+    // that no uninitialised pattern is ever multiplied by p = 0. (The tiled
+    // copies of the tensor-core consumer always fill whole boxes.)
+    for (int i = lane; i < C::S * C::SLOT / 16; i += 32) reinterpret_cast<uint4*>(wb)[i] = make_uint4(0, 0, 0, 0);
+    fence_proxy_async_smem();
+  }
   __syncwarp();
 
   const uint64_t pol = l2_evict_first_policy();
   const unsigned char* Kg = static_cast<const unsigned char*>(p.K);
   const unsigned char* Vg = static_cast<const unsigned char*>(p.V);
   const unsigned char* Qg = static_cast<const unsigned char*>(p.q);
-  const int r0 = warp * C::TPW;  // first row of this warp in every chunk
 
   // ---- chunk metadata, 32 chunks per batch (lane j holds chunk j) ---------
   // Every lane walks the chunk sequence to its own chunk and loads that chunk's
@@ -524,8 +541,8 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
   };
   // weighted mode: this lane's row (token index, weight) of one chunk
   auto load_rows = [&](int bh, int j0, int rows, int& idx, float& w) {
-    const int row = j0 + r0 + lane;
-    const bool in = bh >= 0 && lane < C::TPW && r0 + lane < rows && row < p.m;
+    const int row = j0 + lane;
+    const bool in = bh >= 0 && lane < C::TPW && lane < rows && row < p.m;
     const size_t at = static_cast<size_t>(in ? bh : 0) * p.m + (in ? row : 0);
     idx = in ? p.tok_idx[at] : -1;
     w = in ? p.w[at] : 0.f;
@@ -558,7 +575,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
       if (lane == 0) atomicOr(p.status, KV_DEV_BAD_SEQ_LEN);
       n = max(0, min(n, p.Ncap));
     }
-    const int nr = max(0, min(C::TPW, mrows - r0));  // rows of this chunk owned by this warp
+    const int nr = min(C::TPW, mrows);  // rows of this chunk
     bool vrow = false;
     int64_t tok = 0;
     float bz = -INFINITY;
@@ -579,11 +596,11 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
         const bool kept = slot < max(0, min(mnk, p.kmax));
         if (kept && (mblk < 0 || mblk >= nbv) && lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
         if (kept && mblk >= 0 && mblk < nbv) {
-          tok0 = (static_cast<int64_t>(mblk) << p.log2L) + (mj0 & (p.L - 1)) + r0;
+          tok0 = (static_cast<int64_t>(mblk) << p.log2L) + (mj0 & (p.L - 1));
           nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(nr), n - tok0)));
         }
       } else {
-        tok0 = mj0 + r0;
+        tok0 = mj0;
         nvalid = static_cast<int>(max(static_cast<int64_t>(0), min(static_cast<int64_t>(nr), n - tok0)));
       }
       vrow = lane < nvalid;
@@ -592,19 +609,30 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
     }
     if (lane < C::TPW) bias[lane] = bz;
     if (lane == 0) *reinterpret_cast<int*>(sl + C::SL_HDR) = nvalid;
-    const uint32_t tx = (mfirst ? C::QBYTES : 0u) + 2u * nvalid * C::RB;
+    const uint32_t tx = (mfirst ? C::QBYTES : 0u) + (MMA ? (nvalid > 0 ? 2u * C::KH * C::BOX : 0u) : 2u * nvalid * C::RB);
     __syncwarp();
     if (lane == 0) mbar_arrive_expect_tx(bars + s, tx);
     __syncwarp();
     const int b = mbh / p.Hkv, h = mbh - b * p.Hkv;
     if (mfirst && lane == 0)
       bulk_g2s(sl + C::SL_Q, Qg + (static_cast<size_t>(b) * p.Hq + h * G) * C::RB, C::QBYTES, bars + s, pol);
-    if (MMA || p.mode == ATTN_WEIGHTED) {
-      // one copy per row (rows land in padded slots for the tensor-core reads)
+    if constexpr (MMA) {
+      // two tiled tensor copies (K, V) per 128-byte column box, 32 rows each; rows
+      // past the valid ones are read but masked by their bias
+      if (nvalid > 0 && lane == 0) {
+        const int y = static_cast<int>(static_cast<int64_t>(mbh) * p.Ncap + (tok - lane));
+#pragma unroll
+        for (int hx = 0; hx < C::KH; ++hx) {
+          tma_load_2d(sl + C::SL_K + hx * C::BOX, &tmK, hx * 64, y, bars + s, pol);
+          tma_load_2d(sl + C::SL_V + hx * C::BOX, &tmV, hx * 64, y, bars + s, pol);
+        }
+      }
+    } else if (p.mode == ATTN_WEIGHTED) {
+      // one copy per gathered row
       if (vrow) {
         const size_t off = (static_cast<size_t>(mbh) * p.Ncap + tok) * C::RB;
-        bulk_g2s(sl + C::SL_K + lane * C::RS, Kg + off, C::RB, bars + s, pol);
-        bulk_g2s(sl + C::SL_V + lane * C::RS, Vg + off, C::RB, bars + s, pol);
+        bulk_g2s(sl + C::SL_K + lane * C::RB, Kg + off, C::RB, bars + s, pol);
+        bulk_g2s(sl + C::SL_V + lane * C::RB, Vg + off, C::RB, bars + s, pol);
       }
     } else if (nvalid > 0) {
       const size_t off = (static_cast<size_t>(mbh) * p.Ncap + (tok - lane)) * C::RB;
@@ -654,7 +682,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
   };
 
   auto flush = [&](int bh) {
-    float* rec = p.recs + (static_cast<size_t>(cta + bh) * C::NW + warp) * C::RECF;
+    float* rec = p.recs + static_cast<size_t>(wk + bh) * C::RECF;
     if constexpr (MMA) {
       const int h0 = 2 * (lane & 3);
       float lt[2];
@@ -735,13 +763,13 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
       continue;
     }
     if (!proxies_done) {
-      // tail proxies of the bh whose first token lies in this CTA's range, built
-      // while the first copies are in flight
+      // tail proxies of the bh whose first token lies in this worker's range,
+      // built while the first copies are in flight
       proxies_done = true;
       if (p.mode == ATTN_BLOCKS && p.use_proxy) {
         const int64_t bh_lo = (t0 + P - 1) / P;
         const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), (t1 + P - 1) / P);
-        for (int64_t pbh = bh_lo + warp; pbh < bh_hi; pbh += C::NW)
+        for (int64_t pbh = bh_lo; pbh < bh_hi; ++pbh)
           build_proxy<T, D, G>(p, static_cast<int>(pbh), lane);
       }
     }
@@ -773,6 +801,20 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
           qb[2 * k + 1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2) : 0u;
         }
       }
+      if (nvalid > 0 && nvalid < C::TPW) {
+        // The box brought rows past the valid ones (the next block, or cache
+        // rows past the sequence); their logits are masked below, and their V
+        // rows are zeroed so that a non-finite pattern there cannot reach p.v
+        // as 0 * inf.
+        unsigned char* vz = wb + s * C::SLOT + C::SL_V;
+        const int per_box = (C::TPW - nvalid) * 8;  // 16-byte chunks past the valid rows
+        for (int e = lane; e < per_box * C::KH; e += 32) {
+          const int hx = e / per_box, r = e - hx * per_box;
+          *reinterpret_cast<uint4*>(vz + hx * C::BOX + nvalid * 128 + r * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();  // the slot is refilled by the async proxy later
+        __syncwarp();
+      }
       if (nvalid > 0) {
         const uint32_t kbase = smem_u32(sl + C::SL_K);
         const uint32_t vbase = smem_u32(sl + C::SL_V);
@@ -783,11 +825,10 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
 #pragma unroll
           for (int e = 0; e < 4; ++e) sc4[mt][e] = 0.f;
           const int row = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
-          const uint32_t a0 = kbase + row * C::RS + (lane >> 4) * 16;
 #pragma unroll
           for (int k = 0; k < C::KS; ++k) {
             uint32_t a[4];
-            ldsm_x4(a0 + k * 32, a);
+            ldsm_x4(kbase + C::swz(row, 2 * k + (lane >> 4)), a);
             mma_bf16(sc4[mt][0], sc4[mt][1], sc4[mt][2], sc4[mt][3], a, qb[2 * k], qb[2 * k + 1]);
           }
         }
@@ -797,11 +838,12 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
         float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
+          // masked rows get -inf whatever their (possibly non-finite) dot
           const float ba = bias[16 * mt + tr], bb = bias[16 * mt + tr + 8];
-          x[mt][0] = fmaf(sc4[mt][0], p.qscale, ba);
-          x[mt][1] = fmaf(sc4[mt][1], p.qscale, ba);
-          x[mt][2] = fmaf(sc4[mt][2], p.qscale, bb);
-          x[mt][3] = fmaf(sc4[mt][3], p.qscale, bb);
+          x[mt][0] = ba == -INFINITY ? -INFINITY : fmaf(sc4[mt][0], p.qscale, ba);
+          x[mt][1] = ba == -INFINITY ? -INFINITY : fmaf(sc4[mt][1], p.qscale, ba);
+          x[mt][2] = bb == -INFINITY ? -INFINITY : fmaf(sc4[mt][2], p.qscale, bb);
+          x[mt][3] = bb == -INFINITY ? -INFINITY : fmaf(sc4[mt][3], p.qscale, bb);
           cm0 = fmaxf(cm0, fmaxf(x[mt][0], x[mt][2]));
           cm1 = fmaxf(cm1, fmaxf(x[mt][1], x[mt][3]));
         }
@@ -848,11 +890,10 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS) attn_kernel(c
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
           const int row = 16 * mt + (lane & 7) + (lane >> 4) * 8;
-          const uint32_t v0 = vbase + row * C::RS + ((lane >> 3) & 1) * 16;
 #pragma unroll
           for (int k = 0; k < C::KS; ++k) {
             uint32_t a[4];
-            ldsm_x4_trans(v0 + k * 32, a);
+            ldsm_x4_trans(vbase + C::swz(row, 2 * k + ((lane >> 3) & 1)), a);
             mma_bf16(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3], a, bh_[mt][0], bh_[mt][1]);
             mma_bf16(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3], a, bl_[mt][0], bl_[mt][1]);
           }

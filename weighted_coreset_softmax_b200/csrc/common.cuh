@@ -97,6 +97,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Tiled tensor copy of one box (2-D tensor map) into this CTA's shared memory.
+// The box shape, swizzle and fill come from the tensor map; x (innermost) must
+// be a multiple of 16 bytes.
+__device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, int y, uint64_t* bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y), "r"(smem_u32(bar)), "l"(policy)
+      : "memory");
+}
+
 // ------------------------------------------------------------ arithmetic
 // Two fp32 FMAs in one packed instruction: (a.x*b.x + c.x, a.y*b.y + c.y).
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {

@@ -32,9 +32,10 @@ int attn_prepare(int dev) {
 }
 
 template <typename T, int D, int G, bool MMA>
-cudaError_t attn_launch_one(const AttnParams& p, int grid, cudaStream_t st) {
+cudaError_t attn_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                            cudaStream_t st) {
   using C = AttnCfg<T, D, G, MMA>;
-  attn_kernel<T, D, G, MMA><<<grid, C::NTHREADS, C::SMEM, st>>>(p);
+  attn_kernel<T, D, G, MMA><<<grid, C::NTHREADS, C::SMEM, st>>>(p, tk, tv);
   return cudaGetLastError();
 }
 
@@ -67,8 +68,9 @@ constexpr bool has_mma() {
   }
 
 template <typename T, int D>
-cudaError_t attn_launch_td(int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
-  KVS_ATTN_SWITCH(attn_launch_one, p, grid, st)
+cudaError_t attn_launch_td(int G, bool use_mma, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                           int grid, cudaStream_t st) {
+  KVS_ATTN_SWITCH(attn_launch_one, p, tk, tv, grid, st)
   return cudaErrorInvalidValue;
 }
 
@@ -122,8 +124,9 @@ cudaError_t select_launch_td(int G, int mode, const SelParams& p, int grid, cuda
 
 // Exported (internal) entry points of this unit.
 namespace kvs {
-cudaError_t KVS_CAT(attn_launch_, KVS_SUFFIX)(int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st) {
-  return attn_launch_td<KVS_T, KVS_D>(G, use_mma, p, grid, st);
+cudaError_t KVS_CAT(attn_launch_, KVS_SUFFIX)(int G, bool use_mma, const AttnParams& p, const CUtensorMap& tk,
+                                               const CUtensorMap& tv, int grid, cudaStream_t st) {
+  return attn_launch_td<KVS_T, KVS_D>(G, use_mma, p, tk, tv, grid, st);
 }
 int KVS_CAT(attn_prepare_, KVS_SUFFIX)(int G, bool use_mma, int dev) {
   return attn_prepare_td<KVS_T, KVS_D>(G, use_mma, dev);

@@ -2,6 +2,7 @@
 // translation unit per (element type, head dimension) so the build parallelises.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "partition.h"
@@ -13,7 +14,8 @@ struct SelParams;
 
 // dtype: 0 = bf16, 1 = fp32. Return cudaSuccess or the launch error.
 // use_mma: tensor-core consumer (bf16 only; ignored for fp32).
-cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, int grid, cudaStream_t st);
+cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams& p, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int grid, cudaStream_t st);
 // CTAs of the attention kernel that fit on one SM (0 on error).
 int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
