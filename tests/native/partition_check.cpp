@@ -5,6 +5,7 @@
 // first violation.
 #include <cstdio>
 #include <cstdlib>
+#include <algorithm>
 #include <set>
 
 #include "partition.h"
@@ -45,6 +46,18 @@ static int check(int NBH, int P, long long cap) {
     if (meet != cl - cf + 1) return fail("arrival count", NBH, P, cap, meet, cl - cf + 1);
   }
   if (part_grid(pt) * ATTN_NW < pt.C) return fail("grid", NBH, P, cap, part_grid(pt), pt.C);
+  // bh-aligned splits: with enough room, every bh boundary is a worker boundary
+  // (P a multiple of the range alignment), so no worker straddles two bhs
+  const long long cap1 = cap < MAX_WORKERS ? cap : MAX_WORKERS;
+  const long long lim = (pt.TT + MIN_TOKENS_PER_WORKER - 1) / MIN_TOKENS_PER_WORKER;
+  const long long splits = NBH <= cap1 && NBH <= lim ? std::min(cap1 / NBH, lim / NBH) : 0;
+  if (splits > 0 && P % RANGE_ALIGN == 0 && pt.TT / (NBH * splits) <= ALIGN_MAX_TOKENS) {
+    if (pt.C % NBH) return fail("splits", NBH, P, cap, pt.C, NBH);
+    for (int bh = 1; bh < NBH; ++bh) {
+      const int u = part_worker_of(pt, static_cast<long long>(bh) * pt.P);
+      if (part_t0(pt, u) != static_cast<long long>(bh) * pt.P) return fail("bh boundary", NBH, P, cap, bh, u);
+    }
+  }
   return 0;
 }
 

@@ -111,6 +111,52 @@ def test_small_pipeline(name, kw, use_proxy):
     check_out(r["out"], r["lse"], ro, rl, what=f"{name} attention proxy={use_proxy}")
 
 
+# Batches of 256 (sequence, KV head) pairs split each pair's tokens across the
+# two workers of one CTA, so every partial result is merged inside the CTA
+# (shared memory, no workspace round trip); smaller batches take the workspace
+# path above. Every output row is compared, with the tail proxy, without it,
+# for ragged lengths, and for the dense and weighted modes.
+LOCAL = [
+    ("llama", dict(B=32, Ncap=1024, k_top=2)),
+    ("llama", dict(B=32, Ncap=1024 + 37, seq_lens=[1061 - 13 * i for i in range(32)], k_top=3)),
+]
+
+
+@pytest.mark.parametrize("name,kw", LOCAL)
+@pytest.mark.parametrize("use_proxy", [True, False])
+def test_cta_local_merge_all_rows(name, kw, use_proxy):
+    wl = W.make(name, DEV, **kw)
+    r = run_pipeline(wl, use_proxy=use_proxy)
+    q, K, V = oracle_inputs(wl)
+    gi, gn = r["idx"].cpu().numpy(), r["nk"].cpu().numpy()
+    kept = {(b, h): [int(x) for x in gi[b, h, :gn[b, h]]] for (b, h) in all_pairs(wl)}
+    ro, rl = O.sparse_batch(q, K, V, wl.seq_lens, wl.block_size, wl.scale, kept, use_proxy)
+    check_out(r["out"], r["lse"], ro, rl, what=f"local merge proxy={use_proxy}")
+
+
+def test_cta_local_merge_dense_and_weighted():
+    wl = W.make("llama", DEV, B=32, Ncap=704, seq_lens=[704 - 17 * i for i in range(32)])
+    sl = wl.seq_lens_tensor(DEV)
+    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
+    out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws)
+    torch.cuda.synchronize()
+    assert kv.kv_workspace_status(ws.tensor) == 0
+    q, K, V = oracle_inputs(wl)
+    ro, rl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
+    check_out(out, lse, ro, rl, what="local merge dense")
+    wc = W.make("llama_coreset", DEV, B=32, Ncap=600, m=128)
+    slc = wc.seq_lens_tensor(DEV)
+    wsc = kv.Workspace(kv.make_shape(wc.q, wc.K, slc, wc.block_size), DEV)
+    out, lse = kv.kv_sparse_decode_attn(wc.q, wc.K, wc.V, slc, wc.block_size, wc.scale, wsc,
+                                        tok_idx=wc.tok_idx, w=wc.w)
+    torch.cuda.synchronize()
+    assert kv.kv_workspace_status(wsc.tensor) == 0
+    qc, Kc, Vc = oracle_inputs(wc)
+    ro, rl = O.weighted_batch(qc, Kc, Vc, wc.seq_lens, wc.tok_idx.cpu().numpy(),
+                              wc.w.cpu().numpy().astype(np.float64), wc.scale)
+    check_out(out, lse, ro, rl, what="local merge weighted")
+
+
 @pytest.mark.parametrize("name,kw", [
     ("llama", dict(B=2, Ncap=3000, seq_lens=[3000, 1234])),
     ("qwen_long", dict(B=2, Ncap=1500, seq_lens=[1500, 3])),

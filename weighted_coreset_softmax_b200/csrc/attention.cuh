@@ -104,10 +104,9 @@ struct AttnCfg {
   static constexpr int CPL = CPR / LPT;      // chunks per lane per row (CUDA-core q.k)
   static constexpr int TPL = 2;              // tokens per token group (CUDA-core q.k)
   static constexpr int TPW = MMA ? 32 : 8 * TPL;  // rows per warp per chunk
-  static constexpr int NW = ATTN_NW;         // warps per CTA
-  static constexpr int NTHREADS = NW * 32;
+  static constexpr int NW = ATTN_NW;         // worker warps per CTA
+  static constexpr int NTHREADS = (NW + 1) * 32;  // + one helper warp (tail proxies)
   static constexpr int TR = TPW;             // rows per chunk (one worker)
-  static constexpr int S = 2;                // ring slots per warp
   static constexpr int VR = 32 / CPR;        // V rows per p.v step (CUDA-core)
   static constexpr int KS = D / 16;          // k-steps of q.k and d-tiles of p.v (MMA)
   static constexpr int KH = MMA ? RB / 128 : 1;   // 128-byte column boxes per row (MMA)
@@ -125,19 +124,22 @@ struct AttnCfg {
   static constexpr int SL_BIAS = SL_Q + QBYTES;
   static constexpr int SL_HDR = SL_BIAS + TPW * 4;
   static constexpr int SLOT = MMA ? (SL_HDR + 16 + 1023) & ~1023 : (SL_HDR + 16 + 127) & ~127;
+  // ring slots per worker: three where two CTAs of three-slot workers still fit
+  // in an SM's 228 KB (1 KB of it reserved per CTA), else two
+  static constexpr int S = (MMA && 2 * (NW * (3 * SLOT + 1024) + 1024 + 1024) <= 228 * 1024) ? 3 : 2;
   // one warp: S slots | q fp32 | p | barriers (q fp32 and p: CUDA-core only)
   static constexpr int W_Q = S * SLOT;
   static constexpr int W_P = W_Q + (MMA ? 0 : G * QHEAD);
   static constexpr int W_BAR = W_P + (MMA ? 0 : TPW * PSTR * 4);
   static constexpr int W_BYTES = MMA ? (W_BAR + S * 8 + 1023) & ~1023 : (W_BAR + S * 8 + 127) & ~127;
   static constexpr int ALIGN_SLACK = MMA ? 1024 : 0;
-  static constexpr int SMEM = NW * W_BYTES + ALIGN_SLACK;
+  static constexpr int CTA_EXTRA = 64;      // per-CTA: the workers' record-ready barriers
+  static constexpr int SMEM = NW * W_BYTES + CTA_EXTRA + ALIGN_SLACK;
   static constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   static_assert(MMA || CPL == 2 || CPL == 4 || CPL == 8, "chunks per lane");
   static_assert(MMA || (VR >= 1 && 32 % CPR == 0 && TPW % VR == 0), "p.v row layout");
   static_assert(!MMA || (ES == 2 && G <= 8 && RB % 128 == 0), "tensor-core consumer: bf16, G <= 8");
   static_assert(TPW <= 32, "one row per lane when issuing copies");
-  static_assert((S & (S - 1)) == 0, "ring slots must be a power of two");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // CUDA-core q.k: rotation of the chunk a lane reads at step st. Within a
   // quarter-warp the lanes are (ts & 1) x pq; rows sit 128-byte aligned, so the
@@ -205,7 +207,8 @@ struct ChunkIter {
   __device__ __forceinline__ void init(int64_t t0, int64_t t1, int P) {
     cur = t0;
     end = t1;
-    bh = static_cast<int>(t0 / P);
+    bh = t0 <= 0x7fffffff ? static_cast<int>(static_cast<unsigned>(t0) / static_cast<unsigned>(P))
+                          : static_cast<int>(t0 / P);
     j0 = static_cast<int>(t0 - static_cast<int64_t>(bh) * P);
   }
   __device__ __forceinline__ bool next(int P, int L, int TR, int mode, int& obh, int& oj0, int& rows) {
@@ -244,14 +247,16 @@ __device__ __forceinline__ int last_worker(const Partition& pt, int bh) {
   return part_worker_of(pt, static_cast<int64_t>(bh) * pt.P + pt.P - 1);
 }
 
-// Merges every partial record of one bh into out / lse. One warp. The records'
-// maxima and sums are read by one lane each (one round trip), the weights follow
-// from warp reductions, then every lane streams its channels of all records with
-// the loads of several records in flight.
+// Merges every partial record of one bh into out / lse. One warp. With at most
+// R records (the usual case: a bh spans a few workers, plus the proxy) each
+// lane requests its channels of all of them together with the records' maxima
+// and sums, so the merge costs one memory round trip; more records are folded
+// 32 at a time (maxima and sums by one lane each, then the channels streamed).
 template <int D, int G>
 __device__ void finalize_bh(const AttnParams& p, int bh, int lane) {
   constexpr int RECF = (G * D + 2 * G + 3) & ~3;
   constexpr int VEC = D / 32;
+  constexpr int R = G <= 4 ? 4 : 2;
   const int cf = first_worker(p.part, bh), cl = last_worker(p.part, bh);
   const int nattn = cl - cf + 1;
   const int nrec = nattn + (p.use_proxy ? 1 : 0);
@@ -260,8 +265,19 @@ __device__ void finalize_bh(const AttnParams& p, int bh, int lane) {
   auto rec_ptr = [&](int j) -> const float* {
     return j < nattn ? base + static_cast<size_t>(j) * RECF : p.proxy_recs + static_cast<size_t>(bh) * RECF;
   };
+  auto load_vec = [&](const float* r, float (&x)[VEC]) {
+    if constexpr (VEC == 4) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(r));
+      x[0] = f.x;
+      x[1] = f.y;
+      x[2] = f.z;
+      x[3] = f.w;
+    } else {
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) x[v] = __ldcg(r + v);
+    }
+  };
   float* o = p.out + (static_cast<size_t>(b) * p.Hq + h * G) * D + lane * VEC;
-  // weights of up to 32 records at a time; more records are folded in passes
   float Mg[G], Lg[G], acc[G][VEC];
 #pragma unroll
   for (int g = 0; g < G; ++g) {
@@ -270,42 +286,69 @@ __device__ void finalize_bh(const AttnParams& p, int bh, int lane) {
 #pragma unroll
     for (int v = 0; v < VEC; ++v) acc[g][v] = 0.f;
   }
-  for (int j0 = 0; j0 < nrec; j0 += 32) {
-    const int j = j0 + lane;
+  if (nrec <= R) {
+    float x[R][G][VEC];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (r < nrec) {
+          load_vec(rec_ptr(r) + g * D + lane * VEC, x[r][g]);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) x[r][g][v] = 0.f;
+        }
+      }
     float mj[G], lj[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      mj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + g) : -INFINITY;
-      lj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + G + g) : 0.f;
+      mj[g] = lane < nrec ? __ldcg(rec_ptr(lane) + G * D + g) : -INFINITY;
+      lj[g] = lane < nrec ? __ldcg(rec_ptr(lane) + G * D + G + g) : 0.f;
     }
-    float wj[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
-      const float Mn = fmaxf(Mg[g], warp_max(mj[g]));
-      const float Ms = safe_max_ref(Mn);
-      const float rescale = fast_exp2(Mg[g] - Ms);
-      wj[g] = fast_exp2(mj[g] - Ms);
-      Lg[g] = Lg[g] * rescale + warp_sum(wj[g] * lj[g]);
+      Mg[g] = warp_max(mj[g]);
+      const float wj = fast_exp2(mj[g] - safe_max_ref(Mg[g]));
+      Lg[g] = warp_sum(wj * lj[g]);
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) acc[g][v] *= rescale;
-      Mg[g] = Mn;
+      for (int r = 0; r < R; ++r) {
+        const float wr = __shfl_sync(FULL_MASK, wj, r);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wr, x[r][g][v], acc[g][v]);
+      }
     }
-    const int cnt = min(32, nrec - j0);
-#pragma unroll 4
-    for (int k = 0; k < cnt; ++k) {
-      const float* r = rec_ptr(j0 + k) + lane * VEC;
+  } else {
+    for (int j0 = 0; j0 < nrec; j0 += 32) {
+      const int j = j0 + lane;
+      float mj[G], lj[G];
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        const float wk = __shfl_sync(FULL_MASK, wj[g], k);
-        if (VEC == 4) {
-          const float4 x = __ldcg(reinterpret_cast<const float4*>(r + g * D));
-          acc[g][0] = fmaf(wk, x.x, acc[g][0]);
-          acc[g][1] = fmaf(wk, x.y, acc[g][1]);
-          acc[g][2] = fmaf(wk, x.z, acc[g][2]);
-          acc[g][3] = fmaf(wk, x.w, acc[g][3]);
-        } else {
+        mj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + g) : -INFINITY;
+        lj[g] = j < nrec ? __ldcg(rec_ptr(j) + G * D + G + g) : 0.f;
+      }
+      float wj[G];
 #pragma unroll
-          for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wk, __ldcg(r + g * D + v), acc[g][v]);
+      for (int g = 0; g < G; ++g) {
+        const float Mn = fmaxf(Mg[g], warp_max(mj[g]));
+        const float Ms = safe_max_ref(Mn);
+        const float rescale = fast_exp2(Mg[g] - Ms);
+        wj[g] = fast_exp2(mj[g] - Ms);
+        Lg[g] = Lg[g] * rescale + warp_sum(wj[g] * lj[g]);
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) acc[g][v] *= rescale;
+        Mg[g] = Mn;
+      }
+      const int cnt = min(32, nrec - j0);
+#pragma unroll 4
+      for (int k = 0; k < cnt; ++k) {
+        const float* r = rec_ptr(j0 + k) + lane * VEC;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          const float wk = __shfl_sync(FULL_MASK, wj[g], k);
+          float x[VEC];
+          load_vec(r + g * D, x);
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) acc[g][v] = fmaf(wk, x[v], acc[g][v]);
         }
       }
     }
@@ -338,13 +381,14 @@ __device__ __forceinline__ void arrive_bh(const AttnParams& p, int bh, int lane)
   }
 }
 
-// The tail proxy of one bh as a partial record (m = its log2 logit, l = 1,
-// acc = its value). One warp. All kept block indices are read in one round trip
-// and the key/value sums of the kept blocks are then requested together, so the
-// proxy costs two dependent memory round trips (up to 32 kept blocks).
+// The tail proxy of one bh: this lane's VEC channels of its value (the mean
+// unread value) and the G log2 logits (q_g . mean unread key * scale*log2(e) +
+// log2 of the unread count; -inf with no unread token). One warp. All kept
+// block indices are read in one round trip and the key/value sums of the kept
+// blocks are then requested together, so the proxy costs two dependent memory
+// round trips (up to 32 kept blocks).
 template <typename T, int D, int G>
-__device__ void build_proxy(const AttnParams& p, int bh, int lane) {
-  constexpr int RECF = (G * D + 2 * G + 3) & ~3;
+__device__ void proxy_values(const AttnParams& p, int bh, int lane, float (&vb)[D / 32], float (&pm)[G]) {
   constexpr int VEC = D / 32;
   constexpr int UNR = 8;  // kept blocks whose sums are in flight together
   const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
@@ -419,51 +463,91 @@ __device__ void build_proxy(const AttnParams& p, int bh, int lane) {
     }
   }
   const int nT = n - cnt;
-  float* rec = p.proxy_recs + static_cast<size_t>(bh) * RECF;
   if (nT > 0) {
     const float inv = 1.f / static_cast<float>(nT);
-    float kb[VEC], vb[VEC];
+    float kb[VEC];
 #pragma unroll
     for (int v = 0; v < VEC; ++v) {
       kb[v] = (kt[v] - ks[v]) * inv;
       vb[v] = (vt[v] - vs[v]) * inv;
     }
     const float lc = log2f(static_cast<float>(nT));
-    float dot[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       float d = 0.f;
 #pragma unroll
       for (int v = 0; v < VEC; ++v) d = fmaf(qv[g][v], kb[v], d);
-      dot[g] = d;
+      pm[g] = d;
     }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1)
 #pragma unroll
-      for (int g = 0; g < G; ++g) dot[g] += __shfl_xor_sync(FULL_MASK, dot[g], m);
+      for (int g = 0; g < G; ++g) pm[g] += __shfl_xor_sync(FULL_MASK, pm[g], m);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-#pragma unroll
-      for (int v = 0; v < VEC; ++v) rec[g * D + lane * VEC + v] = vb[v];
-      if (lane == 0) {
-        rec[G * D + g] = dot[g] * p.qscale + lc;
-        rec[G * D + G + g] = 1.f;
-      }
-    }
+    for (int g = 0; g < G; ++g) pm[g] = pm[g] * p.qscale + lc;
   } else {
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
+    for (int v = 0; v < VEC; ++v) vb[v] = 0.f;
 #pragma unroll
-      for (int v = 0; v < VEC; ++v) rec[g * D + lane * VEC + v] = 0.f;
-      if (lane == 0) {
-        rec[G * D + g] = -INFINITY;
-        rec[G * D + G + g] = 0.f;
-      }
+    for (int g = 0; g < G; ++g) pm[g] = -INFINITY;
+  }
+}
+
+// The tail proxy as one more partial record of the bh (m = its logit, l = 1,
+// acc = its value) in the workspace, followed by its arrival ticket.
+template <typename T, int D, int G>
+__device__ void build_proxy(const AttnParams& p, int bh, int lane) {
+  constexpr int RECF = (G * D + 2 * G + 3) & ~3;
+  constexpr int VEC = D / 32;
+  float vb[VEC], pm[G];
+  proxy_values<T, D, G>(p, bh, lane, vb, pm);
+  float* rec = p.proxy_recs + static_cast<size_t>(bh) * RECF;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) rec[g * D + lane * VEC + v] = pm[g] == -INFINITY ? 0.f : vb[v];
+    if (lane == 0) {
+      rec[G * D + g] = pm[g];
+      rec[G * D + G + g] = pm[g] == -INFINITY ? 0.f : 1.f;
     }
   }
   __threadfence();
   __syncwarp();
   arrive_bh<D, G>(p, bh, lane);
+}
+
+// Merge of one bh whose partial records all live in this CTA: nw records in
+// shared memory (written by the workers, layout as in the workspace) and the
+// proxy held in registers (pm = -inf: none). One warp.
+template <int D, int G>
+__device__ void merge_local(const AttnParams& p, int bh, int lane, const float* const* recs, int nw,
+                            const float (&vb)[D / 32], const float (&pm)[G]) {
+  constexpr int VEC = D / 32;
+  const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
+  float* o = p.out + (static_cast<size_t>(b) * p.Hq + h * G) * D + lane * VEC;
+#pragma unroll
+  for (int g = 0; g < G; ++g) {
+    float M = pm[g];
+    for (int j = 0; j < nw; ++j) M = fmaxf(M, recs[j][G * D + g]);
+    const float Ms = safe_max_ref(M);
+    const float wp = fast_exp2(pm[g] - Ms);
+    float Lsum = pm[g] == -INFINITY ? 0.f : wp;
+    float acc[VEC];
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) acc[v] = pm[g] == -INFINITY ? 0.f : wp * vb[v];
+    for (int j = 0; j < nw; ++j) {
+      const float wj = fast_exp2(recs[j][G * D + g] - Ms);
+      Lsum = fmaf(wj, recs[j][G * D + G + g], Lsum);
+      const float* r = recs[j] + g * D + lane * VEC;
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[v] = fmaf(wj, r[v], acc[v]);
+    }
+    const float inv = Lsum > 0.f ? 1.f / Lsum : 0.f;
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) o[g * D + v] = acc[v] * inv;
+    if (p.lse && lane == 0)
+      p.lse[static_cast<size_t>(b) * p.Hq + h * G + g] = Lsum > 0.f ? (M + log2f(Lsum)) * LN2 : -INFINITY;
+  }
 }
 
 template <typename T, int D, int G, bool MMA>
@@ -475,16 +559,77 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
   unsigned char* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u) * (MMA ? 1 : 0);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int wk = blockIdx.x * C::NW + warp;  // this worker
-  const int64_t t0 = part_t0(p.part, wk);
-  const int64_t t1 = part_t0(p.part, wk + 1);
   const int P = p.part.P;
+  constexpr int VEC = D / 32;
+  // Worker ranges of this CTA. When the CTA's range starts and ends on bh
+  // boundaries and each worker's range lies inside one bh ("local" CTA), every
+  // partial record of those bh is produced here: the workers leave their
+  // records in shared memory and the helper warp merges them with the proxy,
+  // with no workspace round trip, fence or ticket.
+  int64_t wa[C::NW + 1];
+#pragma unroll
+  for (int w = 0; w <= C::NW; ++w) wa[w] = part_t0(p.part, blockIdx.x * C::NW + w);
+  auto bh_of = [&](int64_t x) -> int64_t {
+    return p.part.TT <= 0x7fffffff ? static_cast<int64_t>(static_cast<unsigned>(x) / static_cast<unsigned>(P)) : x / P;
+  };
+  bool local = bh_of(wa[0]) * P == wa[0] && bh_of(wa[C::NW]) * P == wa[C::NW];
+#pragma unroll
+  for (int w = 0; w < C::NW; ++w)
+    if (wa[w] < wa[w + 1] && bh_of(wa[w]) != bh_of(wa[w + 1] - 1)) local = false;
+  uint64_t* ready = reinterpret_cast<uint64_t*>(smem + C::NW * C::W_BYTES);
+  if (threadIdx.x == 0) {
+#pragma unroll
+    for (int w = 0; w < C::NW; ++w) mbar_init(ready + w, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == C::NW) {
+    // helper warp: the tail proxies of the bh whose first token lies in this
+    // CTA's range, built while the workers stream (its memory round trips stay
+    // off their critical path); in a local CTA also the final merges
+    grid_dep_wait();
+    const int64_t bh_lo = bh_of(wa[0] + P - 1);
+    const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), bh_of(wa[C::NW] + P - 1));
+    const bool proxy = p.mode == ATTN_BLOCKS && p.use_proxy;
+    if (local) {
+      for (int64_t pbh = bh_lo; pbh < bh_hi; ++pbh) {
+        float vb[VEC], pm[G];
+        if (proxy) {
+          proxy_values<T, D, G>(p, static_cast<int>(pbh), lane, vb, pm);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) vb[v] = 0.f;
+#pragma unroll
+          for (int g = 0; g < G; ++g) pm[g] = -INFINITY;
+        }
+        const float* recs[C::NW];
+        int nw = 0;
+#pragma unroll
+        for (int w = 0; w < C::NW; ++w)
+          if (wa[w] < wa[w + 1] && bh_of(wa[w]) == pbh) {
+            mbar_wait(ready + w, 0u, p.status);
+            recs[nw++] = reinterpret_cast<const float*>(smem + w * C::W_BYTES);
+          }
+        merge_local<D, G>(p, static_cast<int>(pbh), lane, recs, nw, vb, pm);
+      }
+    } else if (proxy) {
+      for (int64_t pbh = bh_lo; pbh < bh_hi; ++pbh) build_proxy<T, D, G>(p, static_cast<int>(pbh), lane);
+    }
+    return;
+  }
+  const int wk = blockIdx.x * C::NW + warp;  // this worker
+  const int64_t t0 = wa[warp];
+  const int64_t t1 = wa[warp + 1];
   unsigned char* wb = smem + warp * C::W_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wb + C::W_BAR);
   float* q32 = reinterpret_cast<float*>(wb + C::W_Q);
   float* pbuf = reinterpret_cast<float*>(wb + C::W_P);
 
   if (lane == 0) {
+    if constexpr (MMA) {
+      prefetch_tensor_map(&tmK);
+      prefetch_tensor_map(&tmV);
+    }
 #pragma unroll
     for (int s = 0; s < C::S; ++s) mbar_init(bars + s, 1);
     fence_mbar_init();
@@ -504,19 +649,42 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
   const unsigned char* Qg = static_cast<const unsigned char*>(p.q);
 
   // ---- chunk metadata, 32 chunks per batch (lane j holds chunk j) ---------
-  // Every lane walks the chunk sequence to its own chunk and loads that chunk's
-  // sequence length, kept count and block index, so one memory round trip covers
-  // the next 32 copies; the following batch is loaded while this one is used.
+  // Each lane finds its own chunk and loads that chunk's sequence length, kept
+  // count and block index, so one memory round trip covers the next 32 copies.
+  // When every chunk has the same TE rows (P a multiple of TE; ranges start on
+  // multiples of 32) chunk j starts at the batch start + j TE, one division per
+  // lane; otherwise each lane walks the chunk sequence up to its chunk.
+  const int TE = (p.mode == ATTN_BLOCKS && p.L < C::TR) ? p.L : C::TR;
+  const bool uniform = (P % TE) == 0;
   ChunkIter bstart;
   bstart.init(t0, t1, P);
   int batch_prev_bh = -1;
   auto load_batch = [&](ChunkMeta& lc) {
-    ChunkIter c = bstart;
     int bh = -1, j0 = 0, rows = 0;
     bool has = false;
-    for (int k = 0; k <= lane; ++k) {
-      has = c.next(P, p.L, C::TR, p.mode, bh, j0, rows);
-      if (!has) break;
+    if (uniform) {
+      const int64_t cs = bstart.cur + static_cast<int64_t>(lane) * TE;
+      has = cs < bstart.end;
+      const int off = bstart.j0 + lane * TE;  // < P + 32 TE
+      const int qd = static_cast<int>(static_cast<unsigned>(off) / static_cast<unsigned>(P));
+      bh = bstart.bh + qd;
+      j0 = off - qd * P;
+      rows = static_cast<int>(min(static_cast<int64_t>(TE), bstart.end - cs));
+      bstart.cur += 32 * TE;
+      const int nj = bstart.j0 + 32 * TE;
+      const int nq = static_cast<int>(static_cast<unsigned>(nj) / static_cast<unsigned>(P));
+      bstart.bh += nq;
+      bstart.j0 = nj - nq * P;
+    } else {
+      ChunkIter c = bstart;
+      for (int k = 0; k <= lane; ++k) {
+        has = c.next(P, p.L, C::TR, p.mode, bh, j0, rows);
+        if (!has) break;
+      }
+      // the next batch starts where lane 31 stopped
+      bstart.cur = __shfl_sync(FULL_MASK, c.cur, 31);
+      bstart.bh = __shfl_sync(FULL_MASK, c.bh, 31);
+      bstart.j0 = __shfl_sync(FULL_MASK, c.j0, 31);
     }
     lc.has = has;
     lc.bh = has ? bh : -1;
@@ -525,10 +693,6 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     int prev = __shfl_up_sync(FULL_MASK, lc.bh, 1);
     if (lane == 0) prev = batch_prev_bh;
     lc.first = has && lc.bh != prev;
-    // the next batch starts where lane 31 stopped
-    bstart.cur = __shfl_sync(FULL_MASK, c.cur, 31);
-    bstart.bh = __shfl_sync(FULL_MASK, c.bh, 31);
-    bstart.j0 = __shfl_sync(FULL_MASK, c.j0, 31);
     batch_prev_bh = __shfl_sync(FULL_MASK, lc.bh, 31);
     lc.n = has ? p.seq_lens[lc.bh / p.Hkv] : 0;
     lc.nk = 0;
@@ -547,17 +711,11 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     idx = in ? p.tok_idx[at] : -1;
     w = in ? p.w[at] : 0.f;
   };
+  // bcur is loaded after the warm-up pass below, bnext once the ring is full
   ChunkMeta bcur, bnext;
-  load_batch(bcur);
-  load_batch(bnext);
+  bcur.has = 0;
   int widx = -1, widx_n = -1;
   float ww = 0.f, ww_n = 0.f;
-  if (p.mode == ATTN_WEIGHTED) {
-    load_rows(__shfl_sync(FULL_MASK, bcur.bh, 0), __shfl_sync(FULL_MASK, bcur.j0, 0),
-              __shfl_sync(FULL_MASK, bcur.rows, 0), widx, ww);
-    load_rows(__shfl_sync(FULL_MASK, bcur.bh, 1), __shfl_sync(FULL_MASK, bcur.j0, 1),
-              __shfl_sync(FULL_MASK, bcur.rows, 1), widx_n, ww_n);
-  }
 
   // issue the copies of chunk c (its metadata sits in lane c & 31 of bcur)
   auto issue = [&](int c, int s) {
@@ -682,7 +840,9 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
   };
 
   auto flush = [&](int bh) {
-    float* rec = p.recs + static_cast<size_t>(wk + bh) * C::RECF;
+    // local CTA: the record goes to ring slot 0 (this is the worker's last bh and
+    // every copy it issued has been consumed); otherwise to the workspace
+    float* rec = local ? reinterpret_cast<float*>(wb) : p.recs + static_cast<size_t>(wk + bh) * C::RECF;
     if constexpr (MMA) {
       const int h0 = 2 * (lane & 3);
       float lt[2];
@@ -740,51 +900,68 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
         }
       }
     }
-    __threadfence();
-    __syncwarp();
-    arrive_bh<D, G>(p, bh, lane);
+    if (local) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(ready + warp);
+    } else {
+      __threadfence();
+      __syncwarp();
+      arrive_bh<D, G>(p, bh, lane);
+    }
   };
 
   ChunkIter it;
   it.init(t0, t1, P);
   int cur_bh = -1;
   bool timed_out = false;
-  bool proxies_done = false;
+  bool next_loaded = false;
   int i = 0;       // chunks consumed
   int issued = 0;  // chunks whose copies were issued
   reset_state();
+  // The first pass of the loop below runs the consumer over slot 0 holding
+  // zeros with every row masked (it changes no state) before any global memory
+  // is touched -- while the previous kernel in the stream may still run: the
+  // consumer's instructions are then fetched before the copies load the memory
+  // system, where each instruction-cache miss would wait behind them.
+  {
+    unsigned char* s0 = wb;
+    if constexpr (MMA)
+      for (int e = lane; e < C::SL_BIAS / 16; e += 32) reinterpret_cast<uint4*>(s0)[e] = make_uint4(0, 0, 0, 0);
+    if (lane < C::TPW) reinterpret_cast<float*>(s0 + C::SL_BIAS)[lane] = -INFINITY;
+    if (lane == 0) *reinterpret_cast<int*>(s0 + C::SL_HDR) = C::TPW;
+    __syncwarp();
+  }
+  bool warm = true;
 #pragma unroll 1
   while (true) {
     // keep the ring full: the only copy-issue site (the first S rounds only issue)
-    if (issued - i < C::S && __shfl_sync(FULL_MASK, bcur.has, issued & 31)) {
-      issue(issued, issued & (C::S - 1));
+    if (!warm && issued - i < C::S && __shfl_sync(FULL_MASK, bcur.has, issued & 31)) {
+      issue(issued, issued % C::S);
       issued_one(issued);
       ++issued;
       continue;
     }
-    if (!proxies_done) {
-      // tail proxies of the bh whose first token lies in this worker's range,
-      // built while the first copies are in flight
-      proxies_done = true;
-      if (p.mode == ATTN_BLOCKS && p.use_proxy) {
-        const int64_t bh_lo = (t0 + P - 1) / P;
-        const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), (t1 + P - 1) / P);
-        for (int64_t pbh = bh_lo; pbh < bh_hi; ++pbh)
-          build_proxy<T, D, G>(p, static_cast<int>(pbh), lane);
+    if (!warm && !next_loaded) {
+      // the ring is full: fetch the next batch of chunk metadata
+      next_loaded = true;
+      load_batch(bnext);
+    }
+    int s = 0;
+    bool first = true;
+    if (!warm) {
+      int bh, j0, rows;
+      const bool more = it.next(P, p.L, C::TR, p.mode, bh, j0, rows);
+      first = more && bh != cur_bh;
+      if ((first || !more) && cur_bh >= 0) flush(cur_bh);  // the only flush site
+      if (!more) break;
+      s = i % C::S;
+      const uint32_t phase = static_cast<uint32_t>(i / C::S) & 1u;
+      if (first) {
+        cur_bh = bh;
+        reset_state();
       }
+      if (!timed_out && !mbar_wait(bars + s, phase, p.status)) timed_out = true;
     }
-    int bh, j0, rows;
-    const bool more = it.next(P, p.L, C::TR, p.mode, bh, j0, rows);
-    const bool first = more && bh != cur_bh;
-    if ((first || !more) && cur_bh >= 0) flush(cur_bh);  // the only flush site
-    if (!more) break;
-    const int s = i & (C::S - 1);
-    const uint32_t phase = static_cast<uint32_t>(i / C::S) & 1u;
-    if (first) {
-      cur_bh = bh;
-      reset_state();
-    }
-    if (!timed_out && !mbar_wait(bars + s, phase, p.status)) timed_out = true;
     const unsigned char* sl = wb + s * C::SLOT;
     const int nvalid = *reinterpret_cast<const int*>(sl + C::SL_HDR);
     const float* bias = reinterpret_cast<const float*>(sl + C::SL_BIAS);
@@ -819,18 +996,24 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
         const uint32_t kbase = smem_u32(sl + C::SL_K);
         const uint32_t vbase = smem_u32(sl + C::SL_V);
         // ---- S^T = K q^T for two 16-token tiles: rows t = 16mt + l/4 (+8), heads h0, h0+1
-        float sc4[2][4];
+        // (even and odd k-steps accumulate separately: two shorter mma chains)
+        float sc4[2][4], sc4o[2][4];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) sc4[mt][e] = 0.f;
+          for (int e = 0; e < 4; ++e) sc4[mt][e] = sc4o[mt][e] = 0.f;
           const int row = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
           for (int k = 0; k < C::KS; ++k) {
             uint32_t a[4];
             ldsm_x4(kbase + C::swz(row, 2 * k + (lane >> 4)), a);
-            mma_bf16(sc4[mt][0], sc4[mt][1], sc4[mt][2], sc4[mt][3], a, qb[2 * k], qb[2 * k + 1]);
+            if (k & 1)
+              mma_bf16(sc4o[mt][0], sc4o[mt][1], sc4o[mt][2], sc4o[mt][3], a, qb[2 * k], qb[2 * k + 1]);
+            else
+              mma_bf16(sc4[mt][0], sc4[mt][1], sc4[mt][2], sc4[mt][3], a, qb[2 * k], qb[2 * k + 1]);
           }
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sc4[mt][e] += sc4o[mt][e];
         }
         // ---- logits (log2 domain) and the chunk maximum of each head
         const int tr = lane >> 2;
@@ -1033,13 +1216,27 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     // the slot is free again: order these reads before the next copy into it
     __syncwarp();
     fence_proxy_async_smem();
-    ++i;
+    if (warm) {
+      warm = false;
+      reset_state();
+      // global memory from here on: the inputs may come from the kernel before
+      grid_dep_wait();
+      load_batch(bcur);
+      if (p.mode == ATTN_WEIGHTED) {
+        load_rows(__shfl_sync(FULL_MASK, bcur.bh, 0), __shfl_sync(FULL_MASK, bcur.j0, 0),
+                  __shfl_sync(FULL_MASK, bcur.rows, 0), widx, ww);
+        load_rows(__shfl_sync(FULL_MASK, bcur.bh, 1), __shfl_sync(FULL_MASK, bcur.j0, 1),
+                  __shfl_sync(FULL_MASK, bcur.rows, 1), widx_n, ww_n);
+      }
+    } else {
+      ++i;
+    }
   }
   if (timed_out) {
     // give copies that may still be in flight a last bounded chance to land
     // before this CTA's shared memory is released
     for (int k = max(0, i - C::S); k < issued; ++k)
-      mbar_wait(bars + (k & (C::S - 1)), static_cast<uint32_t>(k / C::S) & 1u, nullptr);
+      mbar_wait(bars + (k % C::S), static_cast<uint32_t>(k / C::S) & 1u, nullptr);
   }
 }
 

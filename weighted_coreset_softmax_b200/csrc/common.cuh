@@ -3,6 +3,8 @@
 // reduction" that finishes many short dot products at once.
 #pragma once
 
+#include <cuda.h>
+
 #include <cuda_bf16.h>
 #include <cstdint>
 
@@ -80,6 +82,16 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32
   return false;
 }
 
+// ------------------------------------------------ programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start while the
+// kernel before it in the stream is still running. Everything it does before
+// grid_dep_wait() must touch no global memory that a preceding kernel writes or
+// reads; grid_dep_wait() returns once the preceding grids have completed and
+// their writes are visible (at once when nothing precedes). grid_dep_launch()
+// lets the next kernel in the stream be scheduled early.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ------------------------------------------------------------- bulk copies
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
@@ -95,6 +107,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst)),
       "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
+}
+
+// Brings a tensor map (a __grid_constant__ kernel parameter) into the
+// descriptor cache ahead of its first tiled copy.
+__device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* m) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
 // Tiled tensor copy of one box (2-D tensor map) into this CTA's shared memory.

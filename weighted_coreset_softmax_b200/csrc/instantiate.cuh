@@ -5,12 +5,32 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <utility>
 
 #include "attention.cuh"
 #include "launch.h"
 #include "select.cuh"
 
 namespace kvs {
+
+// Launch with programmatic stream serialization: the kernel may be scheduled
+// while the previous kernel in the stream finishes; it calls grid_dep_wait()
+// before touching global memory.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Raises the kernel's dynamic shared-memory limit once per device and returns how
 // many CTAs fit on one SM.
@@ -35,8 +55,7 @@ template <typename T, int D, int G, bool MMA>
 cudaError_t attn_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                             cudaStream_t st) {
   using C = AttnCfg<T, D, G, MMA>;
-  attn_kernel<T, D, G, MMA><<<grid, C::NTHREADS, C::SMEM, st>>>(p, tk, tv);
-  return cudaGetLastError();
+  return launch_pdl(attn_kernel<T, D, G, MMA>, grid, C::NTHREADS, C::SMEM, st, p, tk, tv);
 }
 
 // Tensor-core consumer for bf16 caches, CUDA-core consumer for fp32 (and for
@@ -92,7 +111,8 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     configured.fetch_or(1 << (dev & 31));
   }
-  select_kernel<T, D, G, MODE><<<grid, SEL_THREADS, smem, st>>>(p);
+  const cudaError_t le = launch_pdl(select_kernel<T, D, G, MODE>, grid, SEL_THREADS, smem, st, p);
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 

@@ -20,6 +20,7 @@ constexpr int ATTN_NW = 2;                 // warps per attention CTA
 constexpr int MAX_WORKERS = 2048;          // upper bound on attention warps per launch
 constexpr int MIN_TOKENS_PER_WORKER = 64;  // below this a warp is not worth starting
 constexpr int RANGE_ALIGN = 32;            // worker ranges start on multiples of 32 (one copy box)
+constexpr int64_t ALIGN_MAX_TOKENS = 4096; // bh-aligned ranges only up to this many tokens a worker
 
 // Every (sequence, KV head) pair "bh" owns P consecutive slots of a global token
 // axis of length TT = NBH * P: the kept blocks' tokens (P = kmax * L), the coreset
@@ -32,37 +33,67 @@ struct Partition {
   int P;
   int NBH;
   int C;
+  int64_t tq;  // TT / C
+  int tr;      // TT % C
 };
 
+// floor(u TT / C) rounded down to RANGE_ALIGN, as u tq + floor(u tr / C): one
+// 32-bit division (u, tr < C <= MAX_WORKERS).
 KVS_HD int64_t part_t0(const Partition& p, int u) {
   if (u >= p.C) return p.TT;
-  const int64_t t = (static_cast<int64_t>(u) * p.TT) / p.C;
-  return t - (t % RANGE_ALIGN);
+  const int64_t t = static_cast<int64_t>(u) * p.tq + static_cast<int64_t>(static_cast<unsigned>(u * p.tr) / static_cast<unsigned>(p.C));
+  return t & ~static_cast<int64_t>(RANGE_ALIGN - 1);
 }
 
-// Worker whose range contains token x (0 <= x < TT). Ranges are never empty
-// below C (consecutive starts differ by at least MIN_TOKENS_PER_WORKER before
-// rounding down to RANGE_ALIGN <= MIN_TOKENS_PER_WORKER / 2).
+// Worker whose range contains token x (0 <= x < TT): a floating-point estimate,
+// corrected against the exact range starts. Ranges are never empty below C
+// (consecutive starts differ by at least MIN_TOKENS_PER_WORKER before rounding
+// down to RANGE_ALIGN <= MIN_TOKENS_PER_WORKER / 2).
 KVS_HD int part_worker_of(const Partition& p, int64_t x) {
-  int u = static_cast<int>((x * p.C) / (p.TT > 0 ? p.TT : 1));
+  int u = static_cast<int>(static_cast<double>(x) * p.C / static_cast<double>(p.TT > 0 ? p.TT : 1));
   if (u >= p.C) u = p.C - 1;
+  if (u < 0) u = 0;
   while (u + 1 < p.C && part_t0(p, u + 1) <= x) ++u;
   while (u > 0 && part_t0(p, u) > x) --u;
   return u;
 }
 
-// max_workers: resident warps the device can hold for this kernel
+// max_workers: resident warps the device can hold for this kernel. For short
+// ranges (up to ALIGN_MAX_TOKENS a worker) worker boundaries fall on bh
+// boundaries where the counts allow it -- each bh split into the same number of
+// ranges, or each worker holding whole bhs -- so that a worker finishes (writes
+// its record and takes its ticket) only once, at the end of its range, instead
+// of stalling on that round trip in mid-stream. Long ranges use every resident
+// warp with equal ranges: there the balance across SMs matters more than a
+// round trip or two.
 KVS_HD Partition make_partition(int NBH, int P, int64_t max_workers) {
   Partition p;
   p.NBH = NBH;
   p.P = P > 0 ? P : 1;
   p.TT = static_cast<int64_t>(NBH) * p.P;
-  int64_t want = (p.TT + MIN_TOKENS_PER_WORKER - 1) / MIN_TOKENS_PER_WORKER;
   int64_t cap = max_workers;
   if (cap > MAX_WORKERS) cap = MAX_WORKERS;
+  if (cap < 1) cap = 1;
+  int64_t lim = (p.TT + MIN_TOKENS_PER_WORKER - 1) / MIN_TOKENS_PER_WORKER;  // >= 64 tokens a worker
+  if (lim < 1) lim = 1;
+  int64_t want;
+  if (NBH <= cap && NBH <= lim) {
+    int64_t splits = cap / NBH;
+    if (splits > lim / NBH) splits = lim / NBH;
+    want = static_cast<int64_t>(NBH) * splits;
+  } else if (NBH > cap) {
+    const int64_t per = (NBH + cap - 1) / cap;  // whole bhs per worker
+    want = (NBH + per - 1) / per;
+  } else {
+    want = lim;
+  }
   if (want > cap) want = cap;
+  if (want > lim) want = lim;
   if (want < 1) want = 1;
+  if (p.TT / want > ALIGN_MAX_TOKENS) want = cap < lim ? cap : lim;
   p.C = static_cast<int>(want);
+  p.tq = p.TT / p.C;
+  p.tr = static_cast<int>(p.TT % p.C);
   return p;
 }
 

@@ -254,6 +254,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int bh = blockIdx.x;
   const int b = bh / p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dep_wait();    // inputs may come from the kernel before this one
+  grid_dep_launch();  // every CTA of this grid is resident: the next kernel may be scheduled
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
