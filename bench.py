@@ -152,6 +152,13 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
 
 
+# DRAM bytes per launch from the committed ncu capture
+# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.409 MB read, 0 written at B=8,
+# scaled x4 by sequences to the B=32 launch). Keyed by (kernel, workload, budget, B);
+# to be re-taken whenever the kernel changes.
+NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_409_408}
+
+
 def measured_peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -483,7 +490,8 @@ def run_ours(args, dist):
         "kernels_ms": {"kv_select_blocks": sel_avg, "kv_sparse_decode_attn": att_avg},
         "bytes_per_launch": {"kv_select_blocks": s_bytes, "kv_sparse_decode_attn": a_bytes},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": NCU_TRAFFIC.get((dom, args.workload, args.budget, B)),
                      "pct_of_8TBs": 100.0 * achieved / NOMINAL_HBM_GBS},
         "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
                 "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
