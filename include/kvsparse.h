@@ -188,6 +188,39 @@ kv_status kv_dense_decode_attn(const kv_shape* shape, const void* q, float scale
                                void* workspace, size_t ws_bytes, kv_stream_t stream);
 
 /*
+ * kv_decode_step -- one decode step of the reduced path: kv_select_blocks in
+ * summary mode followed by kv_sparse_decode_attn in block mode, with the same
+ * results. Sources: as for those two calls ("COBS: Cumulant Order Block Sparse
+ * Attention", Equation (5) and the mean-pool score after Equation (8);
+ * "OpenAttention reads 1% of the KV cache", "Skipping reviews without losing the
+ * verdict" for the tail proxy).
+ *   Arguments: those of kv_select_blocks (k_sum, counts, k_top, force_first,
+ *   force_last, kmax, block_idx and n_kept as outputs, scores optional) and of
+ *   kv_sparse_decode_attn in block mode (v_sum, k_tot, v_tot, use_tail_proxy,
+ *   out, lse, workspace). block_idx / n_kept are written and then read by the
+ *   attention, so they must not be read by another stream until the call's work
+ *   completes.
+ *   how: KV_STEP_TWO_KERNELS (also KV_STEP_AUTO) launches the selector and the
+ *   attention kernel back to back (the attention grid is scheduled while the
+ *   selector finishes). KV_STEP_FUSED runs one kernel in which each CTA selects
+ *   the blocks of one (sequence, KV head) and then attends to them (no cross-CTA
+ *   dependency); it applies to bf16 caches on the tensor-core path when the
+ *   per-CTA layout fits (three ring slots: G <= 4 at D = 128; block logits of the
+ *   pair in one 18 KB slot) and kmax * block_size is a multiple of 32, and falls
+ *   back to two kernels otherwise. On B200 the two-kernel form is the faster one
+ *   at the shapes measured, so it is the default.
+ *   Errors: the union of the two calls' argument errors, reported before any
+ *   launch; KV_ERR_INVALID_ARG for an unknown `how`.
+ */
+typedef enum { KV_STEP_AUTO = 0, KV_STEP_TWO_KERNELS = 1, KV_STEP_FUSED = 2 } kv_step_how;
+
+kv_status kv_decode_step(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                         const float* k_sum, const float* v_sum, const int32_t* counts, const float* k_tot,
+                         const float* v_tot, int k_top, int force_first, int force_last, int kmax,
+                         int use_tail_proxy, int32_t* block_idx, int32_t* n_kept, float* scores, float* out,
+                         float* lse, void* workspace, size_t ws_bytes, kv_step_how how, kv_stream_t stream);
+
+/*
  * kv_workspace_bytes -- device workspace the attention entry points need for
  * this shape (split partial results, arrival counters, a status word). The size
  * depends only on B, Hkv, G and D. Returns 0 for an invalid shape pointer.

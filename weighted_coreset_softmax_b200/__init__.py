@@ -24,15 +24,17 @@ import torch
 
 __all__ = [
     "KV_OK", "KV_ERR_INVALID_ARG", "KV_ERR_UNSUPPORTED", "KV_ERR_CUDA", "KV_ERR_DEVICE_CHECK",
-    "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KVShape", "KVError",
+    "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KV_STEP_AUTO", "KV_STEP_TWO_KERNELS",
+    "KV_STEP_FUSED", "KVShape", "KVError",
     "lib", "library_path", "header_path", "make_shape", "kv_build_block_summaries",
-    "kv_select_blocks", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_workspace_bytes",
+    "kv_select_blocks", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
 KV_BF16, KV_F32 = 0, 1
 KV_SCORE_SUMMARY, KV_SCORE_EXACT_MASS = 0, 1
+KV_STEP_AUTO, KV_STEP_TWO_KERNELS, KV_STEP_FUSED = 0, 1, 2
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 _ROOT = os.path.dirname(_PKG)
@@ -82,6 +84,8 @@ def lib():
         "kv_sparse_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                   _P, _P, _I, _P, _P, _P, _S, _P],
         "kv_dense_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _P, _S, _P],
+        "kv_decode_step": [_SHP, _P, _F, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P,
+                           _P, _S, _I, _P],
         "kv_workspace_init": [_P, _S, _P],
         "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
     }
@@ -282,6 +286,41 @@ def kv_sparse_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq
         int(m), _ptr(out), _ptr(lse), workspace.ptr(), workspace.nbytes, _stream(dev))
     _check(st)
     return out, lse
+
+
+def kv_decode_step(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                   scale: float, workspace: Workspace, summaries: dict, k_top: int, force_first: bool = False,
+                   force_last: bool = False, *, kmax: Optional[int] = None, use_tail_proxy: bool = True,
+                   block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                   scores: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                   lse: Optional[torch.Tensor] = None, want_lse: bool = True, how: int = KV_STEP_AUTO):
+    """Selection (summary mode) and attention over the kept blocks in one call;
+    how = KV_STEP_FUSED asks for the single-kernel form. Returns (out, lse or None,
+    block_idx, n_kept)."""
+    _need(q, "q", K.dtype)
+    _need(K, "K")
+    _need(V, "V", K.dtype)
+    shape = make_shape(q, K, seq_lens, block_size)
+    dev = q.device
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if out is None:
+        out = torch.empty(shape.B, shape.Hq, shape.D, dtype=torch.float32, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty(shape.B, shape.Hq, dtype=torch.float32, device=dev)
+    s = summaries
+    _check(lib().kv_decode_step(
+        ctypes.byref(shape), _ptr(q), float(scale), _ptr(K), _ptr(V), _ptr(s["k_sum"]), _ptr(s["v_sum"]),
+        _ptr(s["counts"]), _ptr(s["k_tot"]), _ptr(s["v_tot"]), int(k_top), int(bool(force_first)),
+        int(bool(force_last)), int(kmax), int(bool(use_tail_proxy)), _ptr(block_idx), _ptr(n_kept), _ptr(scores),
+        _ptr(out), _ptr(lse), workspace.ptr(), workspace.nbytes, int(how), _stream(dev)))
+    return out, lse, block_idx, n_kept
 
 
 def kv_dense_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor,

@@ -33,6 +33,10 @@ int attn_prepare_bf16_d64(int, bool, int);
 int attn_prepare_bf16_d128(int, bool, int);
 int attn_prepare_f32_d64(int, bool, int);
 int attn_prepare_f32_d128(int, bool, int);
+bool fused_fits_bf16_d64(int, int);
+bool fused_fits_bf16_d128(int, int);
+cudaError_t fused_launch_bf16_d64(int, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int, cudaStream_t);
+cudaError_t fused_launch_bf16_d128(int, const AttnParams&, const CUtensorMap&, const CUtensorMap&, int, cudaStream_t);
 cudaError_t select_launch_bf16_d64(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_bf16_d128(int, int, const SelParams&, int, cudaStream_t);
 cudaError_t select_launch_f32_d64(int, int, const SelParams&, int, cudaStream_t);
@@ -49,6 +53,15 @@ int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev) {
   if (dtype == KV_BF16)
     return D == 64 ? attn_prepare_bf16_d64(G, use_mma, dev) : attn_prepare_bf16_d128(G, use_mma, dev);
   return D == 64 ? attn_prepare_f32_d64(G, false, dev) : attn_prepare_f32_d128(G, false, dev);
+}
+bool fused_fits(int dtype, int D, int G, int NBcap) {
+  if (dtype != KV_BF16) return false;
+  return D == 64 ? fused_fits_bf16_d64(G, NBcap) : fused_fits_bf16_d128(G, NBcap);
+}
+cudaError_t launch_fused(int dtype, int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                         int grid, cudaStream_t st) {
+  if (dtype != KV_BF16) return cudaErrorInvalidValue;
+  return D == 64 ? fused_launch_bf16_d64(G, p, tk, tv, grid, st) : fused_launch_bf16_d128(G, p, tk, tv, grid, st);
 }
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st) {
   if (dtype == KV_BF16)
@@ -215,11 +228,28 @@ int num_sms_current() {
   return c;
 }
 
+// Selection done inside the attention kernel (fused decode step).
+struct FusedSel {
+  int k_top, force_first, force_last;
+  int32_t* block_idx;
+  int32_t* n_kept;
+  float* scores;
+};
+
+// Can the fused decode step run this shape? (bf16 caches, tensor cores, the
+// per-CTA layout fits, pair boundaries on 32-token range boundaries.)
+bool fused_applies(const kv_shape* s, int kmax) {
+  if (!attention_uses_tensor_cores() || s->dtype != KV_BF16) return false;
+  const int NBcap = (s->Ncap + s->block_size - 1) / s->block_size;
+  if (kmax <= 0 || (static_cast<long long>(kmax) * s->block_size) % kvs::RANGE_ALIGN != 0) return false;
+  return kvs::fused_fits(s->dtype, s->D, s->Hq / s->Hkv, NBcap);
+}
+
 kv_status run_attention(const kv_shape* s, const void* q, float scale, const void* K, const void* V,
                         const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
                         const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
                         int use_proxy, const int32_t* tok_idx, const float* w, int m, int mode, float* out,
-                        float* lse, void* ws, size_t ws_bytes, kv_stream_t stream) {
+                        float* lse, void* ws, size_t ws_bytes, kv_stream_t stream, const FusedSel* fs = nullptr) {
   const int G = s->Hq / s->Hkv;
   const int NBH = s->B * s->Hkv;
   const int NBcap = (s->Ncap + s->block_size - 1) / s->block_size;
@@ -264,6 +294,7 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   // tensor cores: bf16 caches, block and dense modes (gathered coreset rows use
   // the CUDA-core consumer)
   const bool use_mma = attention_uses_tensor_cores() && s->dtype == KV_BF16 && mode != kvs::ATTN_WEIGHTED;
+  if (fs && !use_mma) return fail(KV_ERR_UNSUPPORTED, "the fused decode step needs the tensor-core path");
   const int cps = kvs::attn_ctas_per_sm(s->dtype, s->D, G, use_mma, dev);
   if (cps <= 0) return fail(KV_ERR_CUDA, "attention kernel does not fit on an SM");
   kvs::AttnParams p{};
@@ -300,7 +331,23 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   p.mode = mode;
   p.use_proxy = use_proxy ? 1 : 0;
   p.qscale = scale * 1.4426950408889634f;
-  p.part = kvs::make_partition(NBH, P, static_cast<int64_t>(sms) * cps * kvs::ATTN_NW);
+  if (fs) {
+    // one CTA per pair: its two workers split the pair's kept tokens
+    p.part.NBH = NBH;
+    p.part.P = P;
+    p.part.TT = static_cast<int64_t>(NBH) * P;
+    p.part.C = NBH * kvs::ATTN_NW;
+    p.part.tq = p.part.TT / p.part.C;
+    p.part.tr = static_cast<int>(p.part.TT % p.part.C);
+    p.k_top = fs->k_top;
+    p.force_first = fs->force_first ? 1 : 0;
+    p.force_last = fs->force_last ? 1 : 0;
+    p.sel_block_idx = fs->block_idx;
+    p.sel_n_kept = fs->n_kept;
+    p.sel_scores = fs->scores;
+  } else {
+    p.part = kvs::make_partition(NBH, P, static_cast<int64_t>(sms) * cps * kvs::ATTN_NW);
+  }
   CUtensorMap tk, tv;
   std::memset(&tk, 0, sizeof(tk));
   std::memset(&tv, 0, sizeof(tv));
@@ -310,10 +357,10 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
     KV_TRY(encode_kv_map(K, rows, s->D, &tk));
     KV_TRY(encode_kv_map(V, rows, s->D, &tv));
   }
-  cudaError_t e =
-      kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),
-                       reinterpret_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "attention launch");
+  cudaError_t e = fs ? kvs::launch_fused(s->dtype, s->D, G, p, tk, tv, NBH, reinterpret_cast<cudaStream_t>(stream))
+                     : kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),
+                                        reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, fs ? "fused decode step launch" : "attention launch");
   return KV_OK;
 }
 
@@ -408,6 +455,39 @@ kv_status kv_dense_decode_attn(const kv_shape* shape, const void* q, float scale
   KV_TRY(check_shape(shape));
   return run_attention(shape, q, scale, K, V, nullptr, nullptr, 0, nullptr, nullptr, nullptr, nullptr, nullptr, 0,
                        nullptr, nullptr, 0, kvs::ATTN_DENSE, out, lse, workspace, ws_bytes, stream);
+}
+
+kv_status kv_decode_step(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                         const float* k_sum, const float* v_sum, const int32_t* counts, const float* k_tot,
+                         const float* v_tot, int k_top, int force_first, int force_last, int kmax, int use_tail_proxy,
+                         int32_t* block_idx, int32_t* n_kept, float* scores, float* out, float* lse, void* workspace,
+                         size_t ws_bytes, kv_step_how how, kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  if (how != KV_STEP_AUTO && how != KV_STEP_TWO_KERNELS && how != KV_STEP_FUSED)
+    return fail(KV_ERR_INVALID_ARG, "unknown decode-step form %d", static_cast<int>(how));
+  if (how != KV_STEP_FUSED || !fused_applies(shape, kmax)) {
+    KV_TRY(kv_select_blocks(shape, q, scale, KV_SCORE_SUMMARY, k_sum, counts, nullptr, k_top, force_first, force_last,
+                            kmax, block_idx, n_kept, scores, stream));
+    return kv_sparse_decode_attn(shape, q, scale, K, V, block_idx, n_kept, kmax, k_sum, v_sum, counts, k_tot, v_tot,
+                                 use_tail_proxy, nullptr, nullptr, 0, out, lse, workspace, ws_bytes, stream);
+  }
+  // the selection's argument checks (the attention's follow in run_attention)
+  if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
+  KV_TRY(need(k_sum, "k_sum"));
+  KV_TRY(need(counts, "counts", 4));
+  KV_TRY(need(block_idx, "block_idx", 4));
+  KV_TRY(need(n_kept, "n_kept", 4));
+  if (scores) KV_TRY(need(scores, "scores", 4));
+  if (k_top < 0) return fail(KV_ERR_INVALID_ARG, "k_top = %d < 0", k_top);
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  const int forced = (force_first ? 1 : 0) + (force_last ? 1 : 0);
+  const long long need_k = std::min<long long>(NBcap, static_cast<long long>(k_top) + forced);
+  if (kmax < need_k)
+    return fail(KV_ERR_INVALID_ARG, "kmax = %d < min(NBcap, k_top + forced) = %lld", kmax, need_k);
+  const FusedSel fs{k_top, force_first, force_last, block_idx, n_kept, scores};
+  return run_attention(shape, q, scale, K, V, block_idx, n_kept, kmax, k_sum, v_sum, counts, k_tot, v_tot,
+                       use_tail_proxy, nullptr, nullptr, 0, kvs::ATTN_BLOCKS, out, lse, workspace, ws_bytes, stream,
+                       &fs);
 }
 
 size_t kv_workspace_bytes(const kv_shape* shape) {

@@ -55,6 +55,7 @@
 #include <climits>
 
 #include "common.cuh"
+#include "rank.cuh"
 
 namespace kvs {
 
@@ -87,6 +88,11 @@ struct AttnParams {
   int use_proxy;
   float qscale;  // softmax scale * log2(e): logits are kept in the log2 domain
   Partition part;
+  // fused decode step only: block selection inside the CTA (summary scoring)
+  int k_top, force_first, force_last;
+  int32_t* sel_block_idx;  // the selection's outputs (block_idx / n_kept above alias them)
+  int32_t* sel_n_kept;
+  float* sel_scores;       // optional [B][Hkv][NBcap]
 };
 
 // Shape constants of one instantiation. MMA selects the tensor-core consumer
@@ -550,7 +556,135 @@ __device__ void merge_local(const AttnParams& p, int bh, int lane, const float* 
   }
 }
 
-template <typename T, int D, int G, bool MMA>
+// Selection phase of the fused decode step: one CTA holds one bh (its two
+// workers split the bh's kept tokens later). Summary scoring of every block
+// ("COBS: Cumulant Order Block Sparse Attention", text after Equation (8): the
+// mean-pool estimate s = q . k_mean + ln n_b), then the Eq. 5 ranking. The
+// workers stream the bh's fp32 key-sum rows through ring slots 0 and 1 (32 rows a
+// slot, bulk copies, chunks interleaved between the workers) and write the block
+// logits into worker 0's slot 2; the helper loads the block counts; keys, counts
+// and the ranking's scratch live in worker 1's slot 2. Every warp of the CTA calls
+// this once (same barrier sequence); afterwards block_idx / n_kept of the bh are
+// in global memory, visible to the whole CTA, and the workers' ring barriers are
+// fresh.
+template <typename T, int D, int G, typename C>
+__device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, int warp, int lane, uint64_t pol) {
+  constexpr int LPR = D / 4;            // lanes per fp32 row (float4 each)
+  constexpr int RPW = 32 / LPR;         // rows one warp load covers
+  constexpr int GR = 8;                 // rows per reduction group
+  constexpr int RS = GR / RPW;          // rows per lane per group
+  constexpr int GP = pow2ceil(G);
+  constexpr int NV = RS * GP;
+  constexpr int ROWB = D * 4;
+  constexpr int CROWS = 2 * C::TPW * C::RB / ROWB;  // rows in a slot's K+V region (32)
+  using HV = HeldValues<NV, LPR, GP>;
+  static_assert(CROWS % GR == 0, "fused selection layout");
+  if constexpr (C::S < 3) {
+    return;  // layout needs three ring slots; such shapes never launch the fused kernel
+  } else {
+  const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
+  const int n = max(0, min(p.seq_lens[b], p.Ncap));
+  const int nbv = (n + p.L - 1) >> p.log2L;
+  const int nbp = (p.NBcap + 31) & ~31;
+  float* lg = reinterpret_cast<float*>(smem + 2 * C::SLOT);  // worker 0, slot 2
+  unsigned char* x1 = smem + C::W_BYTES + 2 * C::SLOT;       // worker 1, slot 2
+  unsigned long long* key = reinterpret_cast<unsigned long long*>(x1);
+  int* cnt = reinterpret_cast<int*>(x1 + static_cast<size_t>(nbp) * 8);
+  RankMisc<C::NTHREADS>& ms = *reinterpret_cast<RankMisc<C::NTHREADS>*>(x1 + ((static_cast<size_t>(nbp) * 12 + 15) & ~15));
+  const int nch = (nbv + CROWS - 1) / CROWS;
+  unsigned char* wb = smem + warp * C::W_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(wb + C::W_BAR);
+  const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D;
+  auto issue = [&](int c, int s) {  // chunk c into slot s (lane 0)
+    const int rows = min(CROWS, nbv - c * CROWS);
+    const uint32_t bytes = static_cast<uint32_t>(rows * ROWB);
+    mbar_arrive_expect_tx(bars + s, bytes);
+    bulk_g2s(wb + s * C::SLOT, ks + static_cast<size_t>(c) * CROWS * D, bytes, bars + s, pol);
+  };
+  const int rg = lane / LPR, c4 = lane % LPR;
+  float4 qf[G];
+  if (warp == C::NW) {
+    const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
+    for (int i = lane; i < nbv; i += 32) cnt[i] = cn[i];
+  } else {
+    if (lane == 0) {
+      if (warp < nch) issue(warp, 0);
+      if (warp + C::NW < nch) issue(warp + C::NW, 1);
+    }
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c4 * 4;
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
+                          load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
+  }
+  __syncthreads();  // counts
+  if (warp < C::NW) {
+    bool ok = true;
+    int j = 0;
+    for (int c = warp; c < nch; c += C::NW, ++j) {
+      const int s = j & 1;
+      if (ok && !mbar_wait(bars + s, static_cast<uint32_t>(j >> 1) & 1u, p.status)) ok = false;
+      const float* chunk = reinterpret_cast<const float*>(wb + s * C::SLOT);
+#pragma unroll 1
+      for (int g0 = 0; g0 < CROWS; g0 += GR) {
+        float part[NV];
+#pragma unroll
+        for (int i = 0; i < RS; ++i) {
+          const int lr = g0 + i * RPW + rg;
+          const float4 k4 = c * CROWS + lr < nbv ? *reinterpret_cast<const float4*>(chunk + lr * D + c4 * 4)
+                                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            if (g < G) {
+              float d = qf[g].x * k4.x;
+              d = fmaf(qf[g].y, k4.y, d);
+              d = fmaf(qf[g].z, k4.z, d);
+              d = fmaf(qf[g].w, k4.w, d);
+              part[i * GP + g] = d;
+            } else {
+              part[i * GP + g] = 0.f;
+            }
+          }
+        }
+        transpose_reduce<NV, LPR / 2>(part, lane);
+#pragma unroll
+        for (int jj = 0; jj < HV::NH; ++jj) {
+          const int vi = HV::index(c4, jj);
+          const int ri = vi / GP, g = vi % GP;
+          const int row = c * CROWS + g0 + ri * RPW + rg;
+          const bool holder = NV >= LPR || (c4 % (LPR / NV)) == 0;
+          if (holder && g < G && row < nbv) {
+            const int nb = cnt[row];
+            lg[g * nbp + row] =
+                nb > 0 ? part[jj] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+          }
+        }
+      }
+      __syncwarp();
+      fence_proxy_async_smem();  // the slot is refilled by the async proxy
+      if (lane == 0 && ok && c + 2 * C::NW < nch) issue(c + 2 * C::NW, s);
+    }
+    // fresh ring barriers for the attention phase (every copy above was consumed)
+    __syncwarp();
+    if (lane == 0) {
+#pragma unroll
+      for (int s = 0; s < C::S; ++s) {
+        mbar_inval(bars + s);
+        mbar_init(bars + s, 1);
+      }
+      fence_mbar_init();
+    }
+    __syncwarp();
+  }
+  __syncthreads();  // every block logit is in lg
+  rank_in_cta<G, C::NTHREADS>(lg, nbp, nbv, p.NBcap, p.k_top, p.force_first != 0, p.force_last != 0, p.kmax,
+                              p.sel_scores ? p.sel_scores + static_cast<size_t>(bh) * p.NBcap : nullptr,
+                              p.sel_block_idx + static_cast<size_t>(bh) * p.kmax, p.sel_n_kept + bh, key, ms);
+  __syncthreads();  // the kept list is written (visible to this CTA) and the scratch is free
+  }
+}
+
+template <typename T, int D, int G, bool MMA, bool FUSED>
 __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV) {
   using C = AttnCfg<T, D, G, MMA>;
@@ -588,6 +722,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     // CTA's range, built while the workers stream (its memory round trips stay
     // off their critical path); in a local CTA also the final merges
     grid_dep_wait();
+    if constexpr (FUSED) fused_select<T, D, G, C>(p, smem, static_cast<int>(bh_of(wa[0])), warp, lane, 0ull);
     const int64_t bh_lo = bh_of(wa[0] + P - 1);
     const int64_t bh_hi = min(static_cast<int64_t>(p.part.NBH), bh_of(wa[C::NW] + P - 1));
     const bool proxy = p.mode == ATTN_BLOCKS && p.use_proxy;
@@ -1221,6 +1356,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
       reset_state();
       // global memory from here on: the inputs may come from the kernel before
       grid_dep_wait();
+      if constexpr (FUSED) fused_select<T, D, G, C>(p, smem, static_cast<int>(bh_of(wa[0])), warp, lane, pol);
       load_batch(bcur);
       if (p.mode == ATTN_WEIGHTED) {
         load_rows(__shfl_sync(FULL_MASK, bcur.bh, 0), __shfl_sync(FULL_MASK, bcur.j0, 0),

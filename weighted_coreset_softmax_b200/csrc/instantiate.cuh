@@ -40,11 +40,11 @@ int attn_prepare(int dev) {
   static std::atomic<int> blocks_per_sm[64];
   int v = blocks_per_sm[dev & 63].load();
   if (v > 0) return v;
-  if (cudaFuncSetAttribute(attn_kernel<T, D, G, MMA>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+  if (cudaFuncSetAttribute(attn_kernel<T, D, G, MMA, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
       cudaSuccess)
     return 0;
   int n = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<T, D, G, MMA>, C::NTHREADS, C::SMEM) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, attn_kernel<T, D, G, MMA, false>, C::NTHREADS, C::SMEM) !=
       cudaSuccess)
     return 0;
   blocks_per_sm[dev & 63].store(n);
@@ -55,7 +55,7 @@ template <typename T, int D, int G, bool MMA>
 cudaError_t attn_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                             cudaStream_t st) {
   using C = AttnCfg<T, D, G, MMA>;
-  return launch_pdl(attn_kernel<T, D, G, MMA>, grid, C::NTHREADS, C::SMEM, st, p, tk, tv);
+  return launch_pdl(attn_kernel<T, D, G, MMA, false>, grid, C::NTHREADS, C::SMEM, st, p, tk, tv);
 }
 
 // Tensor-core consumer for bf16 caches, CUDA-core consumer for fp32 (and for
@@ -64,6 +64,57 @@ template <typename T>
 constexpr bool has_mma() {
   return sizeof(T) == 2;
 }
+
+// Fused decode step (bf16, tensor-core consumer, one CTA per bh): does this
+// shape fit the in-CTA selection's shared-memory layout (three ring slots; the
+// block logits in one slot, keys, counts and scratch in another)?
+template <typename T, int D, int G>
+bool fused_fits(int NBcap) {
+  if constexpr (!has_mma<T>()) {
+    return false;
+  } else {
+    using C = AttnCfg<T, D, G, true>;
+    const size_t nbp = static_cast<size_t>((NBcap + 31) & ~31);
+    return C::S >= 3 && G * nbp * 4 <= static_cast<size_t>(C::SLOT) &&
+           ((nbp * 12 + 15) & ~static_cast<size_t>(15)) + sizeof(RankMisc<C::NTHREADS>) <= static_cast<size_t>(C::SLOT);
+  }
+}
+
+template <typename T, int D, int G>
+cudaError_t fused_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                             cudaStream_t st) {
+  if constexpr (!has_mma<T>()) {
+    return cudaErrorInvalidValue;
+  } else if constexpr (AttnCfg<T, D, G, true>::S < 3) {
+    return cudaErrorInvalidValue;  // fused_fits() is false for this shape
+  } else {
+    using C = AttnCfg<T, D, G, true>;
+    static std::atomic<int> configured{0};  // one bit per device: smem limit raised
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (!(configured.load() & (1 << (dev & 31)))) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(attn_kernel<T, D, G, true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+      if (e != cudaSuccess) return e;
+      configured.fetch_or(1 << (dev & 31));
+    }
+    return launch_pdl(attn_kernel<T, D, G, true, true>, grid, C::NTHREADS, C::SMEM, st, p, tk, tv);
+  }
+}
+
+#define KVS_G_SWITCH(FN, ...)                      \
+  switch (G) {                                      \
+    case 1: return FN<T, D, 1>(__VA_ARGS__);        \
+    case 2: return FN<T, D, 2>(__VA_ARGS__);        \
+    case 3: return FN<T, D, 3>(__VA_ARGS__);        \
+    case 4: return FN<T, D, 4>(__VA_ARGS__);        \
+    case 5: return FN<T, D, 5>(__VA_ARGS__);        \
+    case 6: return FN<T, D, 6>(__VA_ARGS__);        \
+    case 7: return FN<T, D, 7>(__VA_ARGS__);        \
+    case 8: return FN<T, D, 8>(__VA_ARGS__);        \
+    default: break;                                 \
+  }
+
 
 #define KVS_ATTN_SWITCH(FN, ...)                                       \
   switch (G) {                                                         \
@@ -144,6 +195,19 @@ cudaError_t select_launch_td(int G, int mode, const SelParams& p, int grid, cuda
 
 // Exported (internal) entry points of this unit.
 namespace kvs {
+bool KVS_CAT(fused_fits_, KVS_SUFFIX)(int G, int NBcap) {
+  using T = KVS_T;
+  constexpr int D = KVS_D;
+  KVS_G_SWITCH(fused_fits, NBcap)
+  return false;
+}
+cudaError_t KVS_CAT(fused_launch_, KVS_SUFFIX)(int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                                                int grid, cudaStream_t st) {
+  using T = KVS_T;
+  constexpr int D = KVS_D;
+  KVS_G_SWITCH(fused_launch_one, p, tk, tv, grid, st)
+  return cudaErrorInvalidValue;
+}
 cudaError_t KVS_CAT(attn_launch_, KVS_SUFFIX)(int G, bool use_mma, const AttnParams& p, const CUtensorMap& tk,
                                                const CUtensorMap& tv, int grid, cudaStream_t st) {
   return attn_launch_td<KVS_T, KVS_D>(G, use_mma, p, tk, tv, grid, st);

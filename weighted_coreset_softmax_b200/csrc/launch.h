@@ -18,6 +18,10 @@ cudaError_t launch_attn(int dtype, int D, int G, bool use_mma, const AttnParams&
                         const CUtensorMap& tv, int grid, cudaStream_t st);
 // CTAs of the attention kernel that fit on one SM (0 on error).
 int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev);
+// Fused decode step (selection + attention in one kernel, one CTA per bh).
+bool fused_fits(int dtype, int D, int G, int NBcap);
+cudaError_t launch_fused(int dtype, int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                         int grid, cudaStream_t st);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,
