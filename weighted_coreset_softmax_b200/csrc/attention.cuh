@@ -111,7 +111,7 @@ struct AttnCfg {
   static constexpr int TPL = 2;              // tokens per token group (CUDA-core q.k)
   static constexpr int TPW = MMA ? 32 : 8 * TPL;  // rows per warp per chunk
   static constexpr int NW = ATTN_NW;         // worker warps per CTA
-  static constexpr int NTHREADS = (NW + 1) * 32;  // + one helper warp (tail proxies)
+  static constexpr int NTHREADS = (NW + 1) * 32;  // + one helper warp (tail proxies, merges)
   static constexpr int TR = TPW;             // rows per chunk (one worker)
   static constexpr int VR = 32 / CPR;        // V rows per p.v step (CUDA-core)
   static constexpr int KS = D / 16;          // k-steps of q.k and d-tiles of p.v (MMA)
@@ -556,17 +556,17 @@ __device__ void merge_local(const AttnParams& p, int bh, int lane, const float* 
   }
 }
 
-// Selection phase of the fused decode step: one CTA holds one bh (its two
-// workers split the bh's kept tokens later). Summary scoring of every block
-// ("COBS: Cumulant Order Block Sparse Attention", text after Equation (8): the
-// mean-pool estimate s = q . k_mean + ln n_b), then the Eq. 5 ranking. The
-// workers stream the bh's fp32 key-sum rows through ring slots 0 and 1 (32 rows a
-// slot, bulk copies, chunks interleaved between the workers) and write the block
-// logits into worker 0's slot 2; the helper loads the block counts; keys, counts
-// and the ranking's scratch live in worker 1's slot 2. Every warp of the CTA calls
-// this once (same barrier sequence); afterwards block_idx / n_kept of the bh are
-// in global memory, visible to the whole CTA, and the workers' ring barriers are
-// fresh.
+// Selection phase of the fused decode step: one CTA holds one bh (its workers
+// split the bh's kept tokens later). Summary scoring of every block ("COBS:
+// Cumulant Order Block Sparse Attention", text after Equation (8): the mean-pool
+// estimate s = q . k_mean + ln n_b), then the Eq. 5 ranking. The workers stream
+// the bh's fp32 key-sum rows through their ring slots (32 rows a slot, bulk
+// copies, chunks interleaved between the workers) and write the block logits
+// into worker 0's last slot; the helper loads the block counts; keys, counts and
+// the ranking's scratch live in worker 1's last slot (those two slots do not
+// stream). Every warp of the CTA calls this once (same barrier sequence);
+// afterwards block_idx / n_kept of the bh are in global memory, visible to the
+// whole CTA, and the workers' ring barriers are fresh.
 template <typename T, int D, int G, typename C>
 __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, int warp, int lane, uint64_t pol) {
   constexpr int LPR = D / 4;            // lanes per fp32 row (float4 each)
@@ -578,16 +578,14 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
   constexpr int ROWB = D * 4;
   constexpr int CROWS = 2 * C::TPW * C::RB / ROWB;  // rows in a slot's K+V region (32)
   using HV = HeldValues<NV, LPR, GP>;
-  static_assert(CROWS % GR == 0, "fused selection layout");
-  if constexpr (C::S < 3) {
-    return;  // layout needs three ring slots; such shapes never launch the fused kernel
-  } else {
+  static_assert(CROWS % GR == 0 && C::NW >= 2, "fused selection layout");
+  {
   const int b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) >> p.log2L;
   const int nbp = (p.NBcap + 31) & ~31;
-  float* lg = reinterpret_cast<float*>(smem + 2 * C::SLOT);  // worker 0, slot 2
-  unsigned char* x1 = smem + C::W_BYTES + 2 * C::SLOT;       // worker 1, slot 2
+  float* lg = reinterpret_cast<float*>(smem + (C::S - 1) * C::SLOT);  // worker 0, last slot
+  unsigned char* x1 = smem + C::W_BYTES + (C::S - 1) * C::SLOT;       // worker 1, last slot
   unsigned long long* key = reinterpret_cast<unsigned long long*>(x1);
   int* cnt = reinterpret_cast<int*>(x1 + static_cast<size_t>(nbp) * 8);
   RankMisc<C::NTHREADS>& ms = *reinterpret_cast<RankMisc<C::NTHREADS>*>(x1 + ((static_cast<size_t>(nbp) * 12 + 15) & ~15));
@@ -595,6 +593,7 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
   unsigned char* wb = smem + warp * C::W_BYTES;
   uint64_t* bars = reinterpret_cast<uint64_t*>(wb + C::W_BAR);
   const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D;
+  const int nslots = warp < 2 ? C::S - 1 : C::S;  // streaming slots of this worker
   auto issue = [&](int c, int s) {  // chunk c into slot s (lane 0)
     const int rows = min(CROWS, nbv - c * CROWS);
     const uint32_t bytes = static_cast<uint32_t>(rows * ROWB);
@@ -607,10 +606,8 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
     const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
     for (int i = lane; i < nbv; i += 32) cnt[i] = cn[i];
   } else {
-    if (lane == 0) {
-      if (warp < nch) issue(warp, 0);
-      if (warp + C::NW < nch) issue(warp + C::NW, 1);
-    }
+    if (lane == 0)
+      for (int j = 0; j < nslots && warp + j * C::NW < nch; ++j) issue(warp + j * C::NW, j);
     const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c4 * 4;
 #pragma unroll
     for (int g = 0; g < G; ++g)
@@ -622,8 +619,8 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
     bool ok = true;
     int j = 0;
     for (int c = warp; c < nch; c += C::NW, ++j) {
-      const int s = j & 1;
-      if (ok && !mbar_wait(bars + s, static_cast<uint32_t>(j >> 1) & 1u, p.status)) ok = false;
+      const int s = j % nslots;
+      if (ok && !mbar_wait(bars + s, static_cast<uint32_t>(j / nslots) & 1u, p.status)) ok = false;
       const float* chunk = reinterpret_cast<const float*>(wb + s * C::SLOT);
 #pragma unroll 1
       for (int g0 = 0; g0 < CROWS; g0 += GR) {
@@ -652,7 +649,7 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
           const int vi = HV::index(c4, jj);
           const int ri = vi / GP, g = vi % GP;
           const int row = c * CROWS + g0 + ri * RPW + rg;
-          const bool holder = NV >= LPR || (c4 % (LPR / NV)) == 0;
+          const bool holder = NV >= LPR || (c4 % (NV >= LPR ? 1 : LPR / NV)) == 0;
           if (holder && g < G && row < nbv) {
             const int nb = cnt[row];
             lg[g * nbp + row] =
@@ -662,7 +659,7 @@ __device__ void fused_select(const AttnParams& p, unsigned char* smem, int bh, i
       }
       __syncwarp();
       fence_proxy_async_smem();  // the slot is refilled by the async proxy
-      if (lane == 0 && ok && c + 2 * C::NW < nch) issue(c + 2 * C::NW, s);
+      if (lane == 0 && ok && c + nslots * C::NW < nch) issue(c + nslots * C::NW, s);
     }
     // fresh ring barriers for the attention phase (every copy above was consumed)
     __syncwarp();

@@ -66,8 +66,8 @@ constexpr bool has_mma() {
 }
 
 // Fused decode step (bf16, tensor-core consumer, one CTA per bh): does this
-// shape fit the in-CTA selection's shared-memory layout (three ring slots; the
-// block logits in one slot, keys, counts and scratch in another)?
+// shape fit the in-CTA selection's shared-memory layout (the block logits in one
+// ring slot, keys, counts and scratch in another)?
 template <typename T, int D, int G>
 bool fused_fits(int NBcap) {
   if constexpr (!has_mma<T>()) {
@@ -75,7 +75,7 @@ bool fused_fits(int NBcap) {
   } else {
     using C = AttnCfg<T, D, G, true>;
     const size_t nbp = static_cast<size_t>((NBcap + 31) & ~31);
-    return C::S >= 3 && G * nbp * 4 <= static_cast<size_t>(C::SLOT) &&
+    return C::NW >= 2 && G * nbp * 4 <= static_cast<size_t>(C::SLOT) &&
            ((nbp * 12 + 15) & ~static_cast<size_t>(15)) + sizeof(RankMisc<C::NTHREADS>) <= static_cast<size_t>(C::SLOT);
   }
 }
@@ -85,8 +85,6 @@ cudaError_t fused_launch_one(const AttnParams& p, const CUtensorMap& tk, const C
                              cudaStream_t st) {
   if constexpr (!has_mma<T>()) {
     return cudaErrorInvalidValue;
-  } else if constexpr (AttnCfg<T, D, G, true>::S < 3) {
-    return cudaErrorInvalidValue;  // fused_fits() is false for this shape
   } else {
     using C = AttnCfg<T, D, G, true>;
     static std::atomic<int> configured{0};  // one bit per device: smem limit raised

@@ -16,7 +16,7 @@
 
 namespace kvs {
 
-constexpr int ATTN_NW = 2;                 // warps per attention CTA
+constexpr int ATTN_NW = 3;                 // worker warps per attention CTA
 constexpr int MAX_WORKERS = 2048;          // upper bound on attention warps per launch
 constexpr int MIN_TOKENS_PER_WORKER = 64;  // below this a warp is not worth starting
 constexpr int RANGE_ALIGN = 32;            // worker ranges start on multiples of 32 (one copy box)
@@ -46,9 +46,9 @@ KVS_HD int64_t part_t0(const Partition& p, int u) {
 }
 
 // Worker whose range contains token x (0 <= x < TT): a floating-point estimate,
-// corrected against the exact range starts. Ranges are never empty below C
-// (consecutive starts differ by at least MIN_TOKENS_PER_WORKER before rounding
-// down to RANGE_ALIGN <= MIN_TOKENS_PER_WORKER / 2).
+// corrected against the exact range starts. Ranges are never empty below C:
+// make_partition keeps consecutive starts at least RANGE_ALIGN apart before they
+// are rounded down to a multiple of RANGE_ALIGN.
 KVS_HD int part_worker_of(const Partition& p, int64_t x) {
   int u = static_cast<int>(static_cast<double>(x) * p.C / static_cast<double>(p.TT > 0 ? p.TT : 1));
   if (u >= p.C) u = p.C - 1;
@@ -60,10 +60,10 @@ KVS_HD int part_worker_of(const Partition& p, int64_t x) {
 
 // max_workers: resident warps the device can hold for this kernel. For short
 // ranges (up to ALIGN_MAX_TOKENS a worker) worker boundaries fall on bh
-// boundaries where the counts allow it -- each bh split into the same number of
-// ranges, or each worker holding whole bhs -- so that a worker finishes (writes
-// its record and takes its ticket) only once, at the end of its range, instead
-// of stalling on that round trip in mid-stream. Long ranges use every resident
+// boundaries where the counts allow it -- each bh split into ATTN_NW ranges (one
+// CTA a bh) or one range a bh, or each worker holding whole bhs -- so that a
+// worker finishes only once, at the end of its range, and a CTA holds whole bhs
+// (its partial results merge in shared memory). Long ranges use every resident
 // warp with equal ranges: there the balance across SMs matters more than a
 // round trip or two.
 KVS_HD Partition make_partition(int NBH, int P, int64_t max_workers) {
@@ -78,9 +78,12 @@ KVS_HD Partition make_partition(int NBH, int P, int64_t max_workers) {
   if (lim < 1) lim = 1;
   int64_t want;
   if (NBH <= cap && NBH <= lim) {
-    int64_t splits = cap / NBH;
-    if (splits > lim / NBH) splits = lim / NBH;
-    want = static_cast<int64_t>(NBH) * splits;
+    // ATTN_NW ranges a bh (one CTA per bh, each range at least one 32-token box)
+    // or one range a bh (ATTN_NW bhs a CTA): every CTA then holds whole bhs and
+    // merges them in shared memory
+    const bool per_cta = static_cast<int64_t>(NBH) * ATTN_NW <= cap && p.P >= ATTN_NW * RANGE_ALIGN;
+    want = static_cast<int64_t>(NBH) * (per_cta ? ATTN_NW : 1);
+    if (per_cta) lim = want;  // ranges of >= 32 tokens are fine here
   } else if (NBH > cap) {
     const int64_t per = (NBH + cap - 1) / cap;  // whole bhs per worker
     want = (NBH + per - 1) / per;
