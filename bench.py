@@ -50,6 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (three batches in memory)")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the workload's own batch; smaller for profiler captures)")
     return ap.parse_args(argv)
@@ -404,26 +405,112 @@ def run_ours(args, dist):
     sel_avg = statistics.fmean(e[0].elapsed_time(e[1]) for e in kev) if not weighted else 0.0
     att_avg = statistics.fmean(e[2].elapsed_time(e[3]) for e in kev)
 
-    # end to end through the public API: q from pinned host memory in, out/lse back
-    q_host = wl.q.detach().cpu().pin_memory()
-    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
-    lse_host = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
-    q_dev = wl.q
-    e2e_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
-    dist.barrier(dev)
-    torch.cuda.synchronize(dev)
-    for i in range(K_steps):
-        flush.zero_()
-        e2e_ev[i][0].record(stream)
-        q_dev.copy_(q_host, non_blocking=True)
-        select()
-        attend()
-        out_host.copy_(out, non_blocking=True)
-        lse_host.copy_(lse, non_blocking=True)
-        e2e_ev[i][1].record(stream)
-    torch.cuda.synchronize(dev)
-    dist.barrier(dev)
-    e2e_ms = dist.max(statistics.fmean(e[0].elapsed_time(e[1]) for e in e2e_ev), dev)
+    # End to end through the public API: every step's q comes in from pinned host
+    # memory and its out/lse go back, inside the timed region. The step's copies
+    # run on two copy streams and overlap the neighbouring steps' kernels, as a
+    # serving loop would; three independent batches (own caches, summaries and
+    # queries) rotate, so a step never finds its inputs in L2 (no flush needed).
+    e2e_ms = None
+    h2d_bytes = wl.q.numel() * wl.q.element_size()
+    d2h_bytes = out.numel() * 4 + lse.numel() * 4
+    if not args.no_e2e:
+        sets = [dict(wl=wl, sl=sl, summ=summ, idx=idx, nk=nk, out=out, lse=lse, ws=ws)]
+        for j in (1, 2):
+            wj = W.make(name, dev, budget=args.budget, B=args.batch,
+                        seed=(100 if name == "llama" else 3) + shard_seed_offset(dist.rank) + 50000 * j)
+            slj = wj.seq_lens_tensor(dev)
+            sets.append(dict(wl=wj, sl=slj, summ=kv.kv_build_block_summaries(wj.K, wj.V, slj, wj.block_size),
+                             idx=torch.zeros_like(idx), nk=torch.zeros_like(nk), out=torch.empty_like(out),
+                             lse=torch.empty_like(lse), ws=kv.Workspace(kv.make_shape(wj.q, wj.K, slj, wj.block_size), dev)))
+        for st_ in sets:
+            st_["q_dev"] = torch.empty_like(st_["wl"].q)
+            st_["q_host"] = st_["wl"].q.detach().cpu().pin_memory()
+            st_["out_host"] = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+            st_["lse_host"] = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+            for e in ("ev_in", "ev_comp", "ev_out"):
+                st_[e] = torch.cuda.Event()
+
+        def step_on(st_):
+            w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
+            if weighted:
+                kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
+                                         tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
+            else:
+                kv.kv_select_blocks(st_["q_dev"], w_.K, sl_, w_.block_size, w_.scale, su_["counts"], w_.k_top,
+                                    w_.force_first, w_.force_last, mode=mode, k_sum=su_["k_sum"], kmax=kmax,
+                                    block_idx=st_["idx"], n_kept=st_["nk"])
+                kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
+                                         block_idx=st_["idx"], n_kept=st_["nk"], summaries=su_,
+                                         use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
+
+        s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+        def enqueue(n):
+            # n steps over the rotating batches; a wait only on events recorded here
+            seen = set()
+            for i in range(n):
+                st_ = sets[i % 3]
+                key = i % 3
+                with torch.cuda.stream(s_in):
+                    if (key, "comp") in seen:
+                        s_in.wait_event(st_["ev_comp"])  # the step before on this batch has read q_dev
+                    st_["q_dev"].copy_(st_["q_host"], non_blocking=True)
+                    st_["ev_in"].record(s_in)
+                with torch.cuda.stream(s_comp):
+                    s_comp.wait_event(st_["ev_in"])
+                    if (key, "out") in seen:
+                        s_comp.wait_event(st_["ev_out"])  # out of the step before on this batch is back
+                    step_on(st_)
+                    st_["ev_comp"].record(s_comp)
+                with torch.cuda.stream(s_out):
+                    s_out.wait_event(st_["ev_comp"])
+                    st_["out_host"].copy_(st_["out"], non_blocking=True)
+                    st_["lse_host"].copy_(st_["lse"], non_blocking=True)
+                    st_["ev_out"].record(s_out)
+                seen.update({(key, "comp"), (key, "out")})
+
+        # the steps are captured once in a CUDA graph (24 steps, three streams forked
+        # from the capture stream and joined at its end) and replayed: the host
+        # issues one launch per 24 steps instead of a dozen calls per step
+        NG = 24
+        cap = torch.cuda.Stream(dev)
+        for _ in range(2):  # eager warm-up on the same streams
+            cap.wait_stream(torch.cuda.current_stream(dev))
+            for s_ in (s_in, s_comp, s_out):
+                s_.wait_stream(cap)
+            enqueue(3)
+            for s_ in (s_in, s_comp, s_out):
+                cap.wait_stream(s_)
+            torch.cuda.current_stream(dev).wait_stream(cap)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cap):
+            for s_ in (s_in, s_comp, s_out):
+                s_.wait_stream(cap)
+            enqueue(NG)
+            for s_ in (s_in, s_comp, s_out):
+                cap.wait_stream(s_)
+        torch.cuda.synchronize(dev)
+        reps = max(1, -(-K_steps // NG))
+        graph.replay()
+        torch.cuda.synchronize(dev)
+        dist.barrier(dev)
+        torch.cuda.synchronize(dev)
+        e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        rs = torch.cuda.current_stream(dev)
+        e_start.record(rs)
+        for _ in range(reps):
+            graph.replay()
+        e_end.record(rs)
+        torch.cuda.synchronize(dev)
+        dist.barrier(dev)
+        e2e_ms = dist.max(e_start.elapsed_time(e_end) / (reps * NG), dev)
+        del graph
+        for st_ in sets[1:]:
+            if kv.kv_workspace_status(st_["ws"].tensor) != 0:
+                raise RuntimeError("device checks failed in the end-to-end steps")
+        del sets
+        torch.cuda.empty_cache()
 
     # the dense baseline on the identical cache
     dense = None
@@ -493,9 +580,12 @@ def run_ours(args, dist):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": NCU_TRAFFIC.get((dom, args.workload, args.budget, B)),
                      "pct_of_8TBs": 100.0 * achieved / NOMINAL_HBM_GBS},
-        "e2e": {"value": queries / (e2e_ms * 1e-3), "unit": "queries/s",
-                "h2d_bytes_per_step": q_host.numel() * q_host.element_size(),
-                "d2h_bytes_per_step": out_host.numel() * 4 + lse_host.numel() * 4, "ms_per_step": e2e_ms},
+        "e2e": None if e2e_ms is None else {
+            "value": queries / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d_bytes,
+            "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms,
+            "how": "q in from pinned host memory and out/lse back every step, on two copy streams "
+                   "overlapping the neighbouring steps' kernels; three independent batches rotate "
+                   "(inputs never L2-resident); 24 steps per CUDA graph replay"},
         "gpu_launches": (1 if weighted else 2) * K_steps,  # our kernels in the timed steps
         "clocks": clk,
         "dense": dense,
