@@ -153,10 +153,11 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
   static std::atomic<int> configured{0};  // one bit per device: smem limit raised
   int dev = 0;
   cudaGetDevice(&dev);
-  const size_t smem = sel_smem_bytes(G, p.NBcap);
+  const size_t smem = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
   if (!(configured.load() & (1 << (dev & 31)))) {
+    const size_t most = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
     cudaError_t e = cudaFuncSetAttribute(select_kernel<T, D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sel_smem_bytes(G, SEL_MAXNB)));
+                                         static_cast<int>(most));
     if (e != cudaSuccess) return e;
     configured.fetch_or(1 << (dev & 31));
   }

@@ -56,7 +56,8 @@ struct SelMisc {
   int wsum[SEL_NW];
 };
 
-// Dynamic shared memory: lg[G][NBP] floats | key[NBP] u64 | misc.
+// Dynamic shared memory: lg[G][NBP] floats | key[NBP] u64 | misc; summary mode
+// adds cnt[NBP] i32 | the row ring (sel_ring_bytes, 16-byte aligned).
 __host__ __device__ inline int sel_nbp(int NBcap) { return (NBcap + 31) & ~31; }
 __host__ __device__ inline size_t sel_smem_bytes(int G, int NBcap) {
   const int nbp = sel_nbp(NBcap);
@@ -76,8 +77,37 @@ __device__ __forceinline__ int sel_block_sum(int v, int* wsum) {
 }
 
 // Summary mode: lg[g][b] = (q_g * qscale) . k_sum_b / n_b + log2 n_b.
+// Each warp takes 8-row batches (warp, warp + 8, ...); every lane moves its own
+// 16-byte pieces of a batch (one column chunk of RS rows) into a lane-private
+// three-stage ring with cp.async, so three batches per warp are in flight with
+// no register staging and no synchronisation between lanes.
+constexpr int SEL_STAGES = 3;
+__host__ __device__ inline size_t sel_ring_bytes(int G) {
+  const int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
+  const int RS = GP >= 4 ? 32 / GP : 8;  // rows per lane per batch (D = 128; D = 64 needs fewer)
+  return static_cast<size_t>(SEL_STAGES) * RS * SEL_THREADS * 16;
+}
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool pred) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %2, 0;\n\t"
+      "@p cp.async.cg.shared.global [%0], [%1], 16;\n\t}" ::"r"(smem_u32(dst)),
+      "l"(src), "r"(static_cast<int>(pred))
+      : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// Dynamic shared memory of a summary-mode selector CTA.
+__host__ __device__ inline size_t sel_summary_smem_bytes(int G, int NBcap) {
+  return ((sel_smem_bytes(G, NBcap) + static_cast<size_t>(sel_nbp(NBcap)) * 4 + 15) & ~static_cast<size_t>(15)) +
+         sel_ring_bytes(G);
+}
+
 template <typename T, int D, int G>
-__device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv) {
+__device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv, float4* ring, int* cnt) {
   constexpr int LPR = D / 4;  // fp32 rows, float4 per lane
   constexpr int RPW = 32 / LPR;
   constexpr int GP = pow2ceil(G);
@@ -86,65 +116,72 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
   constexpr int NV = RS * GP;
   constexpr int BATCH = RPW * RS;                         // rows per warp per batch
   using HV = HeldValues<NV, LPR, GP>;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = lane / LPR, c = lane % LPR;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
+  const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
+  const int nbt = (nbv + BATCH - 1) / BATCH;               // batches of the bh
+  const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;  // batches of this warp
+  // stage s, row i of this lane: ring[(s * RS + i) * SEL_THREADS + tid]
+  auto issue = [&](int m) {
+    const int st = m % SEL_STAGES;
+    const int rb = (warp + m * SEL_NW) * BATCH;
+#pragma unroll
+    for (int i = 0; i < RS; ++i) {
+      const int row = rb + i * RPW + rg;
+      cp_async16(ring + (st * RS + i) * SEL_THREADS + tid, ks + static_cast<size_t>(row < nbv ? row : 0) * D,
+                 m < nmine && row < nbv);
+    }
+    cp_async_commit();  // one group per batch slot, empty or not: the waits count groups
+  };
+#pragma unroll
+  for (int m = 0; m < SEL_STAGES; ++m) issue(m);
+  // counts and q while the first batches are in flight
+  const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
+  for (int i = tid; i < nbv; i += SEL_THREADS) cnt[i] = __ldg(cn + i);
   const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c * 4;
   float4 qf[G];
 #pragma unroll
   for (int g = 0; g < G; ++g)
     qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
                         load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
-  const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
-  const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
-  // two batches in flight per warp
-  for (int rb = warp * 2 * BATCH; rb < nbv; rb += SEL_NW * 2 * BATCH) {
-    float4 k4[2][RS];
-    int cnt[2][RS];
+  __syncthreads();  // cnt
+  for (int m = 0; m < nmine; ++m) {
+    cp_async_wait<SEL_STAGES - 1>();  // batch m has landed (this lane's pieces)
+    const int st = m % SEL_STAGES;
+    const int rb = (warp + m * SEL_NW) * BATCH;
+    float part[NV];
 #pragma unroll
-    for (int u = 0; u < 2; ++u)
+    for (int i = 0; i < RS; ++i) {
+      const int row = rb + i * RPW + rg;
+      const float4 k4 = row < nbv ? ring[(st * RS + i) * SEL_THREADS + tid] : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int i = 0; i < RS; ++i) {
-        const int row = rb + u * BATCH + i * RPW + rg;
-        k4[u][i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        cnt[u][i] = 0;
-        if (row < nbv) {
-          k4[u][i] = __ldg(reinterpret_cast<const float4*>(ks + static_cast<size_t>(row) * D));
-          cnt[u][i] = __ldg(cn + row);
+      for (int g = 0; g < GP; ++g) {
+        if (g < G) {
+          float d = qf[g].x * k4.x;
+          d = fmaf(qf[g].y, k4.y, d);
+          d = fmaf(qf[g].z, k4.z, d);
+          d = fmaf(qf[g].w, k4.w, d);
+          part[i * GP + g] = d;
+        } else {
+          part[i * GP + g] = 0.f;
         }
       }
+    }
+    issue(m + SEL_STAGES);  // refill this stage (its values are in registers now)
+    transpose_reduce<NV, LPR / 2>(part, lane);
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float part[NV];
-#pragma unroll
-      for (int i = 0; i < RS; ++i)
-#pragma unroll
-        for (int g = 0; g < GP; ++g) {
-          if (g < G) {
-            float d = qf[g].x * k4[u][i].x;
-            d = fmaf(qf[g].y, k4[u][i].y, d);
-            d = fmaf(qf[g].z, k4[u][i].z, d);
-            d = fmaf(qf[g].w, k4[u][i].w, d);
-            part[i * GP + g] = d;
-          } else {
-            part[i * GP + g] = 0.f;
-          }
-        }
-      transpose_reduce<NV, LPR / 2>(part, lane);
-#pragma unroll
-      for (int j = 0; j < HV::NH; ++j) {
-        const int vi = HV::index(c, j);
-        const int ri = vi / GP, g = vi % GP;
-        const int row = rb + u * BATCH + ri * RPW + rg;
-        int nb = cnt[u][0];
-#pragma unroll
-        for (int i = 1; i < RS; ++i)
-          if (ri == i) nb = cnt[u][i];
-        if (g < G && row < nbv)
-          lg[g * nbp + row] = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+    for (int j = 0; j < HV::NH; ++j) {
+      const int vi = HV::index(c, j);
+      const int ri = vi / GP, g = vi % GP;
+      const int row = rb + ri * RPW + rg;
+      if (g < G && row < nbv) {
+        const int nb = cnt[row];
+        lg[g * nbp + row] = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
       }
     }
   }
+  cp_async_wait<0>();  // nothing may still be writing the ring when the CTA moves on
 }
 
 // Exact mode: lg[g][b] = log2 sum_{r in block} exp2((q_g * qscale) . k_r).
@@ -259,8 +296,11 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
-  if (MODE == SEL_SUMMARY)
-    score_summary<T, D, G>(p, lg, nbp, bh, nbv);
+  if (MODE == SEL_SUMMARY) {
+    int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
+    float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
+    score_summary<T, D, G>(p, lg, nbp, bh, nbv, ring, cnt);
+  }
   else
     score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
   __syncthreads();
