@@ -51,11 +51,16 @@ static int check(int NBH, int P, long long cap) {
   const long long cap1 = cap < MAX_WORKERS ? cap : MAX_WORKERS;
   const long long lim = (pt.TT + MIN_TOKENS_PER_WORKER - 1) / MIN_TOKENS_PER_WORKER;
   long long splits = 0;
-  if (NBH <= cap1 && NBH <= lim)
-    splits = (static_cast<long long>(NBH) * ATTN_NW <= cap1 && P >= ATTN_NW * RANGE_ALIGN) ? ATTN_NW : 1;
+  if (NBH <= cap1 && NBH <= lim) {
+    const long long smax = std::min(cap1 / NBH, lim / NBH);
+    if (smax > ATTN_NW && static_cast<long long>(NBH) * ATTN_NW * 4 < cap1)
+      splits = smax;
+    else
+      splits = (static_cast<long long>(NBH) * ATTN_NW <= cap1 && P >= ATTN_NW * RANGE_ALIGN) ? ATTN_NW : 1;
+  }
   if (splits > 0 && P % RANGE_ALIGN == 0 && pt.TT / (NBH * splits) <= ALIGN_MAX_TOKENS) {
     if (pt.C % NBH) return fail("splits", NBH, P, cap, pt.C, NBH);
-    if (pt.C / NBH != 1 && pt.C / NBH != ATTN_NW) return fail("splits per bh", NBH, P, cap, pt.C, NBH);
+    if (pt.C / NBH != splits) return fail("splits per bh", NBH, P, cap, pt.C, NBH);
     for (int bh = 1; bh < NBH; ++bh) {
       const int u = part_worker_of(pt, static_cast<long long>(bh) * pt.P);
       if (part_t0(pt, u) != static_cast<long long>(bh) * pt.P) return fail("bh boundary", NBH, P, cap, bh, u);

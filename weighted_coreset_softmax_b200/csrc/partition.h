@@ -63,7 +63,9 @@ KVS_HD int part_worker_of(const Partition& p, int64_t x) {
 // boundaries where the counts allow it -- each bh split into ATTN_NW ranges (one
 // CTA a bh) or one range a bh, or each worker holding whole bhs -- so that a
 // worker finishes only once, at the end of its range, and a CTA holds whole bhs
-// (its partial results merge in shared memory). Long ranges use every resident
+// (its partial results merge in shared memory). With few bhs (one CTA each would
+// fill less than a quarter of the resident warps) each bh is cut into as many
+// ranges as fit instead, merged through the workspace. Long ranges use every resident
 // warp with equal ranges: there the balance across SMs matters more than a
 // round trip or two.
 KVS_HD Partition make_partition(int NBH, int P, int64_t max_workers) {
@@ -78,12 +80,21 @@ KVS_HD Partition make_partition(int NBH, int P, int64_t max_workers) {
   if (lim < 1) lim = 1;
   int64_t want;
   if (NBH <= cap && NBH <= lim) {
-    // ATTN_NW ranges a bh (one CTA per bh, each range at least one 32-token box)
-    // or one range a bh (ATTN_NW bhs a CTA): every CTA then holds whole bhs and
-    // merges them in shared memory
-    const bool per_cta = static_cast<int64_t>(NBH) * ATTN_NW <= cap && p.P >= ATTN_NW * RANGE_ALIGN;
-    want = static_cast<int64_t>(NBH) * (per_cta ? ATTN_NW : 1);
-    if (per_cta) lim = want;  // ranges of >= 32 tokens are fine here
+    int64_t smax = cap / NBH;
+    if (smax > lim / NBH) smax = lim / NBH;
+    const bool fills = static_cast<int64_t>(NBH) * ATTN_NW * 4 >= cap;  // a CTA per bh fills >= 1/4
+    if (smax > ATTN_NW && !fills) {
+      // few bhs: many ranges per bh fill the GPU; their partial results merge
+      // through the workspace
+      want = static_cast<int64_t>(NBH) * smax;
+    } else {
+      // ATTN_NW ranges a bh (one CTA per bh, each range at least one 32-token
+      // box) or one range a bh (ATTN_NW bhs a CTA): every CTA then holds whole
+      // bhs and merges them in shared memory
+      const bool per_cta = static_cast<int64_t>(NBH) * ATTN_NW <= cap && p.P >= ATTN_NW * RANGE_ALIGN;
+      want = static_cast<int64_t>(NBH) * (per_cta ? ATTN_NW : 1);
+      if (per_cta) lim = want;  // ranges of >= 32 tokens are fine here
+    }
   } else if (NBH > cap) {
     const int64_t per = (NBH + cap - 1) / cap;  // whole bhs per worker
     want = (NBH + per - 1) / per;
