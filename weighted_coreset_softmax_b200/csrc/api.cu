@@ -169,11 +169,12 @@ bool attention_uses_tensor_cores() {
   return v;
 }
 
-// Tiled 2-D tensor map over a [rows][D] bf16 cache: boxes of 32 rows x 64
-// elements (128 bytes), 128-byte swizzle, zero fill past the last row. Encoded
+// Tiled 2-D tensor map over a [rows][D] bf16 cache: boxes of box_rows rows x 64
+// elements (128 bytes; 32 rows for block copies, 1 row for gather4), 128-byte
+// swizzle, zero fill past the last row. Encoded
 // through the driver entry point (no link against the driver library); the last
 // few maps are cached, keyed by address and extent.
-kv_status encode_kv_map(const void* base, uint64_t rows, int D, CUtensorMap* out) {
+kv_status encode_kv_map(const void* base, uint64_t rows, int D, int box_rows, CUtensorMap* out) {
   using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -182,14 +183,14 @@ kv_status encode_kv_map(const void* base, uint64_t rows, int D, CUtensorMap* out
   struct Entry {
     const void* base;
     uint64_t rows;
-    int D;
+    int D, box_rows;
     CUtensorMap map;
   };
   static Entry cache[16];
   static int next_slot = 0;
   std::lock_guard<std::mutex> lock(mu);
   for (const Entry& e : cache)
-    if (e.base == base && e.rows == rows && e.D == D) {
+    if (e.base == base && e.rows == rows && e.D == D && e.box_rows == box_rows) {
       *out = e.map;
       return KV_OK;
     }
@@ -202,14 +203,14 @@ kv_status encode_kv_map(const void* base, uint64_t rows, int D, CUtensorMap* out
   }
   const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
   const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  const cuuint32_t box[2] = {64, 32};
+  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
   const cuuint32_t estr[2] = {1, 1};
   CUtensorMap m;
   const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KV_ERR_CUDA, "tensor map encoding failed (CUresult %d)", static_cast<int>(r));
-  cache[next_slot] = Entry{base, rows, D, m};
+  cache[next_slot] = Entry{base, rows, D, box_rows, m};
   next_slot = (next_slot + 1) % 16;
   *out = m;
   return KV_OK;
@@ -291,9 +292,9 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   if (sms <= 0) return fail(KV_ERR_CUDA, "no CUDA device available");
   int dev = 0;
   cudaGetDevice(&dev);
-  // tensor cores: bf16 caches, block and dense modes (gathered coreset rows use
-  // the CUDA-core consumer)
-  const bool use_mma = attention_uses_tensor_cores() && s->dtype == KV_BF16 && mode != kvs::ATTN_WEIGHTED;
+  // tensor cores for bf16 caches in every mode (gathered coreset rows arrive by
+  // gather4 tensor copies)
+  const bool use_mma = attention_uses_tensor_cores() && s->dtype == KV_BF16;
   if (fs && !use_mma) return fail(KV_ERR_UNSUPPORTED, "the fused decode step needs the tensor-core path");
   const int cps = kvs::attn_ctas_per_sm(s->dtype, s->D, G, use_mma, dev);
   if (cps <= 0) return fail(KV_ERR_CUDA, "attention kernel does not fit on an SM");
@@ -354,8 +355,9 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   if (use_mma) {
     const uint64_t rows = static_cast<uint64_t>(NBH) * s->Ncap;
     if (rows > 0x7fffffffull) return fail(KV_ERR_UNSUPPORTED, "B * Hkv * Ncap = %llu rows is too many", (unsigned long long)rows);
-    KV_TRY(encode_kv_map(K, rows, s->D, &tk));
-    KV_TRY(encode_kv_map(V, rows, s->D, &tv));
+    const int box_rows = mode == kvs::ATTN_WEIGHTED ? 1 : 32;  // gather4 needs a one-row box
+    KV_TRY(encode_kv_map(K, rows, s->D, box_rows, &tk));
+    KV_TRY(encode_kv_map(V, rows, s->D, box_rows, &tv));
   }
   cudaError_t e = fs ? kvs::launch_fused(s->dtype, s->D, G, p, tk, tv, NBH, reinterpret_cast<cudaStream_t>(stream))
                      : kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),

@@ -907,9 +907,26 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
     if (mfirst && lane == 0)
       bulk_g2s(sl + C::SL_Q, Qg + (static_cast<size_t>(b) * p.Hq + h * G) * C::RB, C::QBYTES, bars + s, pol);
     if constexpr (MMA) {
-      // two tiled tensor copies (K, V) per 128-byte column box, 32 rows each; rows
-      // past the valid ones are read but masked by their bias
-      if (nvalid > 0 && lane == 0) {
+      if (p.mode == ATTN_WEIGHTED) {
+        // gathered rows: gather4 tensor copies (the maps' box is one row high),
+        // four rows each, into the same swizzled tiles; a row that takes no part
+        // reads the bh's first token instead and is masked by its bias
+        if (nvalid > 0) {
+          const int yrow = static_cast<int>(static_cast<int64_t>(mbh) * p.Ncap + (vrow ? tok : 0));
+          const int g4 = (lane & 7) * 4;
+          const int y0 = __shfl_sync(FULL_MASK, yrow, g4), y1 = __shfl_sync(FULL_MASK, yrow, g4 + 1);
+          const int y2 = __shfl_sync(FULL_MASK, yrow, g4 + 2), y3 = __shfl_sync(FULL_MASK, yrow, g4 + 3);
+          if (lane < C::TPW / 4) {
+#pragma unroll
+            for (int hx = 0; hx < C::KH; ++hx) {
+              tma_gather4(sl + C::SL_K + hx * C::BOX + lane * 4 * 128, &tmK, hx * 64, y0, y1, y2, y3, bars + s);
+              tma_gather4(sl + C::SL_V + hx * C::BOX + lane * 4 * 128, &tmV, hx * 64, y0, y1, y2, y3, bars + s);
+            }
+          }
+        }
+      } else if (nvalid > 0 && lane == 0) {
+        // two tiled tensor copies (K, V) per 128-byte column box, 32 rows each; rows
+        // past the valid ones are read but masked by their bias
         const int y = static_cast<int>(static_cast<int64_t>(mbh) * p.Ncap + (tok - lane));
 #pragma unroll
         for (int hx = 0; hx < C::KH; ++hx) {
@@ -1110,7 +1127,7 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
           qb[2 * k + 1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2) : 0u;
         }
       }
-      if (nvalid > 0 && nvalid < C::TPW) {
+      if (p.mode != ATTN_WEIGHTED && nvalid > 0 && nvalid < C::TPW) {
         // The box brought rows past the valid ones (the next block, or cache
         // rows past the sequence); their logits are masked below, and their V
         // rows are zeroed so that a non-finite pattern there cannot reach p.v

@@ -112,6 +112,17 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
+// Four rows of a 2-D tensor at arbitrary row coordinates (the map's box is one
+// row high) into four consecutive box rows at dst, in the map's swizzle.
+__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* tmap, int x, int y0, int y1, int y2, int y3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // Brings a tensor map (a __grid_constant__ kernel parameter) into the
 // descriptor cache ahead of its first tiled copy.
 __device__ __forceinline__ void prefetch_tensor_map(const CUtensorMap* m) {
