@@ -251,6 +251,12 @@ def test_shape_coverage(G, D, dtype):
     check_out(out, lse, ro, rl, what=f"coverage sparse G={G} D={D} {dtype}")
     do, dl = O.dense_batch(q64, K64, V64, lens, scale)
     check_out(dout, dlse, do, dl, what=f"coverage dense G={G} D={D} {dtype}")
+    # exact-mass (OSA) selection at the same shape
+    xidx, xnk, _ = kv.kv_select_blocks(q, K, sl, L, scale, summ["counts"], 4, True, True,
+                                       mode=kv.KV_SCORE_EXACT_MASS)
+    torch.cuda.synchronize()
+    xsel = O.select_batch(q64, K64, lens, L, scale, 4, True, True, "exact_mass")
+    selection_matches(xidx, xnk, xsel, pairs, f"coverage exact-mass select G={G} D={D} {dtype}")
 
 
 def test_exact_mass_small():

@@ -155,12 +155,14 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
   cudaGetDevice(&dev);
   const size_t smem = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
   if (!(configured.load() & (1 << (dev & 31)))) {
-    const size_t most = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
+    size_t most = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
+    if (most > 227 * 1024) most = 227 * 1024;  // per-CTA limit; larger shapes are refused below
     cudaError_t e = cudaFuncSetAttribute(select_kernel<T, D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(most));
     if (e != cudaSuccess) return e;
     configured.fetch_or(1 << (dev & 31));
   }
+  if (smem > 227 * 1024) return cudaErrorInvalidConfiguration;
   const cudaError_t le = launch_pdl(select_kernel<T, D, G, MODE>, grid, SEL_THREADS, smem, st, p);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
