@@ -1,5 +1,6 @@
 """The CUDA-core attention consumer on bf16 caches (selected by KVSPARSE_ATTN=fma,
-read once per process) against the float64 oracle, run in a child process."""
+read once per process) against the float64 oracle in block, dense and weighted
+modes, run in a child process."""
 import os
 import subprocess
 import sys
@@ -31,6 +32,17 @@ for name, kw in (("llama", dict(B=2, Ncap=3100, seq_lens=[3100, 777], budget=0.0
     out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, r["ws"])
     do, dl = O.dense_batch(q, K, V, wl.seq_lens, wl.scale)
     check_out(out, lse, do, dl, what=name + " cuda-core dense")
+# weighted coreset rows, one copy per gathered row
+wc = W.make("llama_coreset", "cuda", B=2, Ncap=2500, seq_lens=[2500, 900], m=300)
+slc = wc.seq_lens_tensor("cuda")
+wsc = kv.Workspace(kv.make_shape(wc.q, wc.K, slc, wc.block_size), "cuda")
+out, lse = kv.kv_sparse_decode_attn(wc.q, wc.K, wc.V, slc, wc.block_size, wc.scale, wsc, tok_idx=wc.tok_idx, w=wc.w)
+torch.cuda.synchronize()
+assert kv.kv_workspace_status(wsc.tensor) == 0
+qc, Kc, Vc = oracle_inputs(wc)
+ro, rl = O.weighted_batch(qc, Kc, Vc, wc.seq_lens, wc.tok_idx.cpu().numpy(), wc.w.cpu().numpy().astype(np.float64),
+                          wc.scale)
+check_out(out, lse, ro, rl, what="cuda-core weighted")
 print("ok")
 """
 

@@ -112,7 +112,7 @@ def test_small_pipeline(name, kw, use_proxy):
 
 
 # Batches of 256 (sequence, KV head) pairs split each pair's tokens across the
-# two workers of one CTA, so every partial result is merged inside the CTA
+# workers of one CTA, so every partial result is merged inside the CTA
 # (shared memory, no workspace round trip); smaller batches take the workspace
 # path above. Every output row is compared, with the tail proxy, without it,
 # for ragged lengths, and for the dense and weighted modes.

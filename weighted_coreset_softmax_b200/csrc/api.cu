@@ -333,7 +333,7 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   p.use_proxy = use_proxy ? 1 : 0;
   p.qscale = scale * 1.4426950408889634f;
   if (fs) {
-    // one CTA per pair: its two workers split the pair's kept tokens
+    // one CTA per pair: its workers split the pair's kept tokens
     p.part.NBH = NBH;
     p.part.P = P;
     p.part.TT = static_cast<int64_t>(NBH) * P;
