@@ -50,6 +50,7 @@ struct SelParams {
 // Shared memory beyond the dynamic arrays.
 struct SelMisc {
   float lse[8];
+  float pm[SEL_NW][8], ps[SEL_NW][8];  // per-warp (max, sum) of the normalisers (summary mode)
   unsigned hist[256];
   unsigned long long prefix, mask;
   int krem, digit, above, bucket;
@@ -107,7 +108,8 @@ __host__ __device__ inline size_t sel_summary_smem_bytes(int G, int NBcap) {
 }
 
 template <typename T, int D, int G>
-__device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv, float4* ring, int* cnt) {
+__device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv, float4* ring, int* cnt,
+                              SelMisc& ms) {
   constexpr int LPR = D / 4;  // fp32 rows, float4 per lane
   constexpr int RPW = 32 / LPR;
   constexpr int GP = pow2ceil(G);
@@ -146,6 +148,14 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
                         load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
   __syncthreads();  // cnt
+  // running (max, sum of 2^(x - max)) of the logits this lane holds: the Eq. 5
+  // normalisers come out of the scoring pass
+  float om[HV::NH], os[HV::NH];
+#pragma unroll
+  for (int j = 0; j < HV::NH; ++j) {
+    om[j] = -INFINITY;
+    os[j] = 0.f;
+  }
   for (int m = 0; m < nmine; ++m) {
     cp_async_wait<SEL_STAGES - 1>();  // batch m has landed (this lane's pieces)
     const int st = m % SEL_STAGES;
@@ -177,11 +187,39 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
       const int row = rb + ri * RPW + rg;
       if (g < G && row < nbv) {
         const int nb = cnt[row];
-        lg[g * nbp + row] = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+        const float x = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+        lg[g * nbp + row] = x;
+        if (x != -INFINITY) {
+          if (x > om[j]) {
+            os[j] = os[j] * exp2f(om[j] - x) + 1.f;
+            om[j] = x;
+          } else {
+            os[j] += exp2f(x - om[j]);
+          }
+        }
       }
     }
   }
   cp_async_wait<0>();  // nothing may still be writing the ring when the CTA moves on
+  // merge the pairs of the lanes that hold the same head (every lane bit that
+  // changes the row), then one lane per head writes this warp's pair
+#pragma unroll
+  for (int j = 0; j < HV::NH; ++j) {
+#pragma unroll
+    for (int mask = HV::ROW_MASK_LO; mask < 32; mask <<= 1) {
+      const float m2 = __shfl_xor_sync(FULL_MASK, om[j], mask), s2 = __shfl_xor_sync(FULL_MASK, os[j], mask);
+      const float M = fmaxf(om[j], m2);
+      os[j] = (om[j] == -INFINITY ? 0.f : os[j] * exp2f(om[j] - M)) + (m2 == -INFINITY ? 0.f : s2 * exp2f(m2 - M));
+      om[j] = M;
+    }
+    const int vi = HV::index(c, j);
+    const int ri = vi / GP, g = vi % GP;
+    const bool holder = NV >= LPR || (c % (NV >= LPR ? 1 : LPR / NV)) == 0;
+    if (ri == 0 && rg == 0 && holder && g < G) {
+      ms.pm[warp][g] = om[j];
+      ms.ps[warp][g] = os[j];
+    }
+  }
 }
 
 // Exact mode: lg[g][b] = log2 sum_{r in block} exp2((q_g * qscale) . k_r).
@@ -299,14 +337,27 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   if (MODE == SEL_SUMMARY) {
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-    score_summary<T, D, G>(p, lg, nbp, bh, nbv, ring, cnt);
+    score_summary<T, D, G>(p, lg, nbp, bh, nbv, ring, cnt, ms);
   }
   else
     score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
   __syncthreads();
 
-  // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain)
-  if (warp < G) {
+  // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain): in summary
+  // mode from the warps' (max, sum) pairs of the scoring pass, else a pass over lg
+  if (MODE == SEL_SUMMARY) {
+    if (warp == 0 && lane < G) {
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < SEL_NW; ++w) M = fmaxf(M, ms.pm[w][lane]);
+      float S = 0.f;
+      if (M != -INFINITY)
+#pragma unroll
+        for (int w = 0; w < SEL_NW; ++w)
+          if (ms.pm[w][lane] != -INFINITY) S += ms.ps[w][lane] * exp2f(ms.pm[w][lane] - M);
+      ms.lse[lane] = (M == -INFINITY || S <= 0.f) ? -INFINITY : M + log2f(S);
+    }
+  } else if (warp < G) {
     float M = -INFINITY;
     for (int i = lane; i < nbv; i += 32) M = fmaxf(M, lg[warp * nbp + i]);
     M = warp_max(M);
