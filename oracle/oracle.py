@@ -11,7 +11,10 @@ Sources (page title, then section / equation):
           probabilities (Equation 1 and the text around it), the per-KV-head GQA
           score (Equation 5 and the normaliser Z^(g,h) of (5)), the first-order
           mean-pool score (affine score (18): phi_b = mean key, a_b = ln L), OSA
-          exact-mass ranking (the OSA paragraph).
+          exact-mass ranking (the OSA paragraph), and the Quest min/max score it
+          analyses (the paragraph on escaping the first-order ceiling: per block
+          the element-wise minimum and maximum of the keys, scored by the largest
+          inner product any point of that box can reach).
   [OA]    "OpenAttention reads 1% of the KV cache -- Count-aware tail proxy",
           section "Skipping reviews without losing the verdict" (the proxy token)
           and section "A worked example with named numbers".
@@ -37,6 +40,10 @@ notes of the repository):
   R9  An empty softmax (no token, no proxy) gives out = 0 and lse = -inf.
   R10 Near tie: (S_(k) - S_(k+1)) / S_(k) < 1e-3 between the k-th and (k+1)-th
       candidate scores.
+  R11 Quest scoring: the box bound sigma * sum_j max(q_j min_j, q_j max_j) takes
+      the place of the block log-mass estimate in the Equation 5 group score
+      (per-head block softmax probabilities summed over the group), with no count
+      term; forced blocks and ties as in R5 and R6.
 """
 from __future__ import annotations
 
@@ -88,6 +95,31 @@ def build_block_summaries(K, V, seq_lens, L):
             k_sum[b, h], v_sum[b, h], k_tot[b, h], v_tot[b, h] = ks, vs, kt, vt
             counts[b] = c
     return k_sum, v_sum, counts, k_tot, v_tot
+
+
+def block_bounds_one(K: np.ndarray, n: int, L: int, NBcap: int):
+    """Per-block, per-channel minimum and maximum of the keys of one (sequence, KV
+    head): the axis-aligned bounding box of each block's keys [COBS, the Quest
+    paragraph]. Blocks past the sequence stay 0."""
+    D = K.shape[1]
+    kmin = np.zeros((NBcap, D))
+    kmax = np.zeros((NBcap, D))
+    for b, (s, e) in enumerate(blocks_of(n, L)):
+        kmin[b] = K[s:e].min(axis=0)
+        kmax[b] = K[s:e].max(axis=0)
+    return kmin, kmax
+
+
+def quest_logits(qg: np.ndarray, kmin: np.ndarray, kmax: np.ndarray, sigma: float):
+    """s_hat[g][b] = sigma * the largest q_g . k over the box [kmin_b, kmax_b]: a
+    linear function is largest at the corner that takes, channel by channel, the
+    end whose product with q is larger [COBS, the Quest paragraph]."""
+    G = qg.shape[0]
+    NB = kmin.shape[0]
+    out = np.empty((G, NB))
+    for g in range(G):
+        out[g] = sigma * np.maximum(qg[g] * kmin, qg[g] * kmax).sum(axis=1)
+    return out
 
 
 # --------------------------------------------------------------------------- scores
@@ -302,6 +334,9 @@ def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
             shat = summary_logits(qg, ks[:nb], c[:nb], sigma)
         elif mode == "exact_mass":
             shat = exact_log_mass(qg, K[b, h], n, L, nb, sigma)
+        elif mode == "quest":
+            kmin, kmax = block_bounds_one(K[b, h], n, L, NBcap)
+            shat = quest_logits(qg, kmin[:nb], kmax[:nb], sigma)
         else:
             raise ValueError(mode)
         S = group_score(shat)

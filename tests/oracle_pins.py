@@ -368,11 +368,54 @@ def pin_empty_inputs():
     assert sel["kept"] == [0]
 
 
+def pin_quest_box_corners(seed=14):
+    """Quest bound = the largest q . corner over every corner of the block's
+    bounding box (brute force over 2^D corners), and the bounds are the
+    channel-wise min / max by loops."""
+    r = _rng(seed)
+    G, D, n, L = 2, 5, 23, 7
+    qg, K = r.normal(size=(G, D)), r.normal(size=(n, D))
+    NB = (n + L - 1) // L
+    kmin, kmax = O.block_bounds_one(K, n, L, NB)
+    for b in range(NB):
+        rows = range(b * L, min(n, (b + 1) * L))
+        for d in range(D):
+            _close(kmin[b, d], min(float(K[t][d]) for t in rows), what="min")
+            _close(kmax[b, d], max(float(K[t][d]) for t in rows), what="max")
+    sq = O.quest_logits(qg, kmin, kmax, 0.7)
+    for g in range(G):
+        for b in range(NB):
+            best = -math.inf
+            for mask in range(1 << D):
+                corner = [kmax[b, d] if (mask >> d) & 1 else kmin[b, d] for d in range(D)]
+                best = max(best, sum(float(qg[g][d]) * corner[d] for d in range(D)))
+            _close(sq[g, b], 0.7 * best, what="quest corner max")
+
+
+def pin_quest_upper_bound(seed=15):
+    """Every key of a block lies in its box, so the Quest score bounds each
+    token's logit from above; a one-key block's box is that key, so the bound is
+    that logit."""
+    r = _rng(seed)
+    G, D, n, L = 3, 8, 61, 8
+    qg, K = r.normal(size=(G, D)), r.normal(size=(n, D))
+    NB = (n + L - 1) // L
+    kmin, kmax = O.block_bounds_one(K, n, L, NB)
+    sq = O.quest_logits(qg, kmin, kmax, 0.5)
+    for b in range(NB):
+        lg = 0.5 * (K[b * L:min(n, (b + 1) * L)] @ qg.T)
+        assert np.all(sq[:, b] >= lg.max(axis=0) - 1e-12), "quest bound below a token logit"
+        assert np.all(sq[:, b] > lg.max(axis=0) + 1e-9), "quest bound equal to the max logit on a random block"
+    k1 = K[:1]
+    kmin1, kmax1 = O.block_bounds_one(k1, 1, L, 1)
+    _close(O.quest_logits(qg, kmin1, kmax1, 0.5)[:, 0], 0.5 * (k1 @ qg.T)[0], what="one-key block")
+
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
     pin_proxy_exact_equal_tail, pin_proxy_logit_is_mean_plus_log_count, pin_jensen,
     pin_integer_weights_duplication, pin_zero_weight_excluded, pin_group_score_invariants,
     pin_topk_bruteforce, pin_near_tie_flag, pin_worked_example, pin_empty_inputs,
-    pin_summary_equals_exact_for_constant_blocks,
+    pin_summary_equals_exact_for_constant_blocks, pin_quest_box_corners, pin_quest_upper_bound,
 ]

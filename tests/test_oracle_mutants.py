@@ -65,6 +65,19 @@ def _mut_exact_mass_max(orig):
     return f
 
 
+def _mut_quest_max_end_only(orig):
+    def f(qg, kmin, kmax, sigma):
+        return np.stack([sigma * (qg[g] * kmax).sum(axis=1) for g in range(qg.shape[0])])
+    return f
+
+
+def _mut_bounds_swapped(orig):
+    def f(K, n, L, NBcap):
+        a, b = orig(K, n, L, NBcap)
+        return b, a
+    return f
+
+
 def _mut_weighted_no_log(orig):
     def f(qg, K, V, n, idx, w, sigma):
         w = np.asarray(w, dtype=np.float64)
@@ -107,6 +120,8 @@ MUTANTS = {
     "summaries/count": ("block_summaries_one", _mut_summaries_count),
     "softmax/unnormalised": ("softmax_attend", _mut_softmax_no_norm),
     "logsumexp/offset": ("logsumexp", _mut_logsumexp_shift),
+    "quest/max end only": ("quest_logits", _mut_quest_max_end_only),
+    "quest/bounds swapped": ("block_bounds_one", _mut_bounds_swapped),
 }
 
 
