@@ -45,7 +45,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_coreset"])
+    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_quest", "llama_coreset"])
     ap.add_argument("--budget", type=float, default=0.01)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -205,6 +205,17 @@ def select_bytes(wl, seq_lens):
     return total
 
 
+def quest_select_bytes(wl, seq_lens):
+    """Algorithmic bytes of one kv_select_blocks_quest launch: every valid block's
+    bf16 (min, max) key bounds, q, and the kept indices written."""
+    L, D, G = wl.block_size, wl.D, wl.G
+    total = 0
+    for b in range(wl.B):
+        nbv = (seq_lens[b] + L - 1) // L
+        total += wl.Hkv * (nbv * D * 4 + G * D * 2 + wl.kmax * 4 + 4)
+    return total
+
+
 def osa_select_bytes(wl, seq_lens):
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
     return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
@@ -247,7 +258,7 @@ def oracle_tasks(wl, pairs):
     import numpy as np
     import torch
     tasks = []
-    kind = {"summary": "summary", "exact_mass": "exact_mass"}[wl.score_mode]
+    kind = {"summary": "summary", "exact_mass": "exact_mass", "quest": "quest"}[wl.score_mode]
     if wl.attn_mode == "weighted":
         kind = "weighted"
     for (b, h) in pairs:
@@ -306,6 +317,7 @@ def workload_label(wl, budget):
         "llama": "Llama-3.1-8B-shaped GQA decode",
         "qwen_long": "Qwen2.5-7B-shaped long-context GQA decode",
         "llama_osa": "Llama-3.1-8B-shaped GQA decode, OSA exact-mass selection",
+        "llama_quest": "Llama-3.1-8B-shaped GQA decode, Quest key-box selection",
         "llama_coreset": "Llama-3.1-8B-shaped GQA decode, weighted coreset m=2048",
     }
     return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, "
@@ -330,6 +342,9 @@ def run_ours(args, dist):
     sl = wl.seq_lens_tensor(dev)
     B = wl.B
     summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
+    quest = wl.score_mode == "quest"
+    if quest:
+        summ["k_bounds"] = kv.kv_build_block_bounds(wl.K, sl, wl.block_size)
     shape = kv.make_shape(wl.q, wl.K, sl, wl.block_size)
     ws = kv.Workspace(shape, dev)
     mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
@@ -340,11 +355,18 @@ def run_ours(args, dist):
     lse = torch.empty(B, wl.Hq, dtype=torch.float32, device=dev)
     weighted = wl.attn_mode == "weighted"
 
+    def select_on(q_, w_, sl_, su_, idx_, nk_):
+        if quest:
+            kv.kv_select_blocks_quest(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_bounds"], w_.k_top,
+                                      w_.force_first, w_.force_last, kmax=kmax, block_idx=idx_, n_kept=nk_)
+        else:
+            kv.kv_select_blocks(q_, w_.K, sl_, w_.block_size, w_.scale, su_["counts"], w_.k_top,
+                                w_.force_first, w_.force_last, mode=mode, k_sum=su_["k_sum"], kmax=kmax,
+                                block_idx=idx_, n_kept=nk_)
+
     def select():
         if not weighted:
-            kv.kv_select_blocks(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["counts"], wl.k_top,
-                                wl.force_first, wl.force_last, mode=mode, k_sum=summ["k_sum"], kmax=kmax,
-                                block_idx=idx, n_kept=nk)
+            select_on(wl.q, wl, sl, summ, idx, nk)
 
     def attend():
         if weighted:
@@ -419,7 +441,10 @@ def run_ours(args, dist):
             wj = W.make(name, dev, budget=args.budget, B=args.batch,
                         seed=(100 if name == "llama" else 3) + shard_seed_offset(dist.rank) + 50000 * j)
             slj = wj.seq_lens_tensor(dev)
-            sets.append(dict(wl=wj, sl=slj, summ=kv.kv_build_block_summaries(wj.K, wj.V, slj, wj.block_size),
+            suj = kv.kv_build_block_summaries(wj.K, wj.V, slj, wj.block_size)
+            if quest:
+                suj["k_bounds"] = kv.kv_build_block_bounds(wj.K, slj, wj.block_size)
+            sets.append(dict(wl=wj, sl=slj, summ=suj,
                              idx=torch.zeros_like(idx), nk=torch.zeros_like(nk), out=torch.empty_like(out),
                              lse=torch.empty_like(lse), ws=kv.Workspace(kv.make_shape(wj.q, wj.K, slj, wj.block_size), dev)))
         for st_ in sets:
@@ -436,9 +461,7 @@ def run_ours(args, dist):
                 kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
                                          tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
             else:
-                kv.kv_select_blocks(st_["q_dev"], w_.K, sl_, w_.block_size, w_.scale, su_["counts"], w_.k_top,
-                                    w_.force_first, w_.force_last, mode=mode, k_sum=su_["k_sum"], kmax=kmax,
-                                    block_idx=st_["idx"], n_kept=st_["nk"])
+                select_on(st_["q_dev"], w_, sl_, su_, st_["idx"], st_["nk"])
                 kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
                                          block_idx=st_["idx"], n_kept=st_["nk"], summaries=su_,
                                          use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
@@ -541,7 +564,8 @@ def run_ours(args, dist):
         a_bytes, s_bytes = weighted_bytes(wl), 0
     else:
         a_bytes = attention_bytes(wl, nk, wl.seq_lens)
-        s_bytes = select_bytes(wl, wl.seq_lens) if mode == kv.KV_SCORE_SUMMARY else osa_select_bytes(wl, wl.seq_lens)
+        s_bytes = (quest_select_bytes(wl, wl.seq_lens) if quest else
+                   select_bytes(wl, wl.seq_lens) if mode == kv.KV_SCORE_SUMMARY else osa_select_bytes(wl, wl.seq_lens))
     peak, peak_kind = measured_peak_hbm()
     if att_avg >= sel_avg or weighted:
         dom, dom_bytes, dom_ms = "kv_sparse_decode_attn", a_bytes, att_avg

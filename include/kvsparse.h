@@ -140,6 +140,40 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale,
                            kv_stream_t stream);
 
 /*
+ * kv_build_block_bounds -- per-block, per-channel key minimum and maximum (the
+ * axis-aligned bounding box of each block's keys). Source: "COBS: Cumulant Order
+ * Block Sparse Attention", the Quest paragraph (a block is scored by the largest
+ * inner product any point of its key box could reach).
+ *
+ *   K         device cache [B][Hkv][Ncap][D] bf16 (bf16 caches only)
+ *   k_bounds  device out [B][Hkv][NBcap][D][2] bf16: (min, max) of channel d over
+ *             the block's tokens < seq_len, as adjacent pairs; blocks at or past
+ *             ceil(seq_len / L) get zeros. Must be 16-byte aligned. The bounds
+ *             are exact (min and max of bf16 values are bf16 values).
+ * Returns KV_ERR_UNSUPPORTED for an fp32 cache. Run once after prefill.
+ */
+kv_status kv_build_block_bounds(const kv_shape* shape, const void* K, void* k_bounds,
+                                kv_stream_t stream);
+
+/*
+ * kv_select_blocks_quest -- kv_select_blocks with the Quest box bound as the
+ * per-head block logit. Source: "COBS: Cumulant Order Block Sparse Attention",
+ * the Quest paragraph and Equation (5):
+ *
+ *   s[g,b] = scale * sum_d max(q_g[d] * min_b[d], q_g[d] * max_b[d])
+ *   S[b]   = sum_{g in group} exp(s[g,b] - ln sum_b' exp(s[g,b']))  over valid b'
+ *
+ * The bound carries no ln n_b count term (the paragraph scores the box's largest
+ * inner product alone). Forcing, ranking, kmax, block_idx, n_kept and scores are
+ * as in kv_select_blocks. k_bounds: kv_build_block_bounds output. bf16 only
+ * (KV_ERR_UNSUPPORTED otherwise).
+ */
+kv_status kv_select_blocks_quest(const kv_shape* shape, const void* q, float scale,
+                                 const void* k_bounds, int k_top, int force_first,
+                                 int force_last, int kmax, int32_t* block_idx,
+                                 int32_t* n_kept, float* scores, kv_stream_t stream);
+
+/*
  * kv_sparse_decode_attn -- softmax attention over a reduced KV cache.
  *
  * Block mode (tok_idx == NULL). Source: "OpenAttention reads 1% of the KV cache

@@ -79,10 +79,16 @@ def run_pipeline(wl, *, want_scores=True, use_proxy=True, kmax=None):
     dev = wl.q.device
     sl = wl.seq_lens_tensor(dev)
     summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
-    mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
-    idx, nk, scores = kv.kv_select_blocks(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["counts"],
-                                          wl.k_top, wl.force_first, wl.force_last, mode=mode,
-                                          k_sum=summ["k_sum"], kmax=kmax, want_scores=want_scores)
+    if wl.score_mode == "quest":
+        summ["k_bounds"] = kv.kv_build_block_bounds(wl.K, sl, wl.block_size)
+        idx, nk, scores = kv.kv_select_blocks_quest(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_bounds"],
+                                                    wl.k_top, wl.force_first, wl.force_last, kmax=kmax,
+                                                    want_scores=want_scores)
+    else:
+        mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
+        idx, nk, scores = kv.kv_select_blocks(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["counts"],
+                                              wl.k_top, wl.force_first, wl.force_last, mode=mode,
+                                              k_sum=summ["k_sum"], kmax=kmax, want_scores=want_scores)
     shape = kv.make_shape(wl.q, wl.K, sl, wl.block_size)
     ws = kv.Workspace(shape, dev)
     out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,

@@ -27,7 +27,7 @@ __all__ = [
     "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KV_STEP_AUTO", "KV_STEP_TWO_KERNELS",
     "KV_STEP_FUSED", "KVShape", "KVError",
     "lib", "library_path", "header_path", "make_shape", "kv_build_block_summaries",
-    "kv_select_blocks", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
+    "kv_select_blocks", "kv_build_block_bounds", "kv_select_blocks_quest", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace",
 ]
 
@@ -81,6 +81,8 @@ def lib():
     sigs = {
         "kv_build_block_summaries": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P],
         "kv_select_blocks": [_SHP, _P, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
+        "kv_build_block_bounds": [_SHP, _P, _P, _P],
+        "kv_select_blocks_quest": [_SHP, _P, _F, _P, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_sparse_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                   _P, _P, _I, _P, _P, _P, _S, _P],
         "kv_dense_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _P, _S, _P],
@@ -244,6 +246,49 @@ def kv_select_blocks(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, b
                                   _ptr(counts), _ptr(K) if mode == KV_SCORE_EXACT_MASS else None,
                                   int(k_top), int(bool(force_first)), int(bool(force_last)), int(kmax),
                                   _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
+    return block_idx, n_kept, scores
+
+
+def kv_build_block_bounds(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                          out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-block key bounding boxes of a bf16 cache: [B][Hkv][NB][D][2] bf16, the
+    last axis (min, max)."""
+    _need(K, "K", torch.bfloat16)
+    _need(seq_lens, "seq_lens", torch.int32)
+    B, Hkv, Ncap, D = K.shape
+    NB = (Ncap + block_size - 1) // block_size
+    if out is None:
+        out = torch.empty(B, Hkv, NB, D, 2, dtype=torch.bfloat16, device=K.device)
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, block_size, KV_BF16, seq_lens.data_ptr())
+    _check(lib().kv_build_block_bounds(ctypes.byref(shape), _ptr(K), _ptr(out), _stream(K.device)))
+    return out
+
+
+def kv_select_blocks_quest(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                           scale: float, k_bounds: torch.Tensor, k_top: int, force_first: bool = False,
+                           force_last: bool = False, kmax: Optional[int] = None,
+                           block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                           scores: Optional[torch.Tensor] = None, want_scores: bool = False):
+    """Kept blocks per KV head, each query head scoring a block by its key box
+    bound. K is not read (its shape gives the descriptor). Returns (block_idx
+    [B][Hkv][kmax], n_kept [B][Hkv], scores or None)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_bounds, "k_bounds", torch.bfloat16)
+    shape = make_shape(q, K, seq_lens, block_size)
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    dev = q.device
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if scores is None and want_scores:
+        scores = torch.empty(shape.B, shape.Hkv, NB, dtype=torch.float32, device=dev)
+    _check(lib().kv_select_blocks_quest(ctypes.byref(shape), _ptr(q), float(scale), _ptr(k_bounds), int(k_top),
+                                        int(bool(force_first)), int(bool(force_last)), int(kmax),
+                                        _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
     return block_idx, n_kept, scores
 
 

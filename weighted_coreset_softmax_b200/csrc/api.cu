@@ -86,6 +86,19 @@ static cudaError_t sums_td(const void* K, const void* V, const int32_t* seq_lens
   return cudaGetLastError();
 }
 
+static cudaError_t launch_bounds(int D, const void* K, const int32_t* seq_lens, void* bounds, int NBH, int Hkv,
+                                 int Ncap, int L, int NBcap, cudaStream_t st) {
+  const int64_t total = static_cast<int64_t>(NBH) * NBcap * (D / 8);
+  const unsigned blocks = static_cast<unsigned>((total + 255) / 256);
+  const auto* k = static_cast<const __nv_bfloat16*>(K);
+  auto* out = static_cast<__nv_bfloat16*>(bounds);
+  if (D == 64)
+    block_bounds_kernel<64><<<blocks, 256, 0, st>>>(k, seq_lens, out, NBH, Hkv, Ncap, L, NBcap);
+  else
+    block_bounds_kernel<128><<<blocks, 256, 0, st>>>(k, seq_lens, out, NBH, Hkv, Ncap, L, NBcap);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,
                         int L, int NBcap, cudaStream_t st) {
@@ -390,18 +403,41 @@ kv_status kv_build_block_summaries(const kv_shape* shape, const void* K, const v
   return KV_OK;
 }
 
-kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv_score_mode mode,
-                           const float* k_sum, const int32_t* counts, const void* K, int k_top, int force_first,
-                           int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
-                           kv_stream_t stream) {
+kv_status kv_build_block_bounds(const kv_shape* shape, const void* K, void* k_bounds, kv_stream_t stream) {
   KV_TRY(check_shape(shape));
-  if (mode != KV_SCORE_SUMMARY && mode != KV_SCORE_EXACT_MASS)
-    return fail(KV_ERR_INVALID_ARG, "unknown score mode %d", (int)mode);
+  if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "block bounds are built for bf16 caches only");
+  KV_TRY(need(K, "K"));
+  KV_TRY(need(k_bounds, "k_bounds"));
+  const int NBH = shape->B * shape->Hkv;
+  if (NBH == 0) return KV_OK;
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  cudaError_t e = kvs::launch_bounds(shape->D, K, shape->seq_lens, k_bounds, NBH, shape->Hkv, shape->Ncap,
+                                     shape->block_size, NBcap, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "bounds launch");
+  return KV_OK;
+}
+
+}  // extern "C"
+
+namespace {
+// Shared by the summary, exact-mass and Quest selections: argument checks and the
+// launch. sel_mode is a kvs::SelMode.
+kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_mode, const float* k_sum,
+                     const void* k_bounds, const int32_t* counts, const void* K, int k_top, int force_first,
+                     int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                     kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
   if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
   KV_TRY(need(q, "q"));
-  KV_TRY(need(counts, "counts", 4));
-  if (mode == KV_SCORE_SUMMARY) KV_TRY(need(k_sum, "k_sum"));
-  if (mode == KV_SCORE_EXACT_MASS) KV_TRY(need(K, "K"));
+  if (sel_mode == kvs::SEL_SUMMARY) {
+    KV_TRY(need(k_sum, "k_sum"));
+    KV_TRY(need(counts, "counts", 4));
+  } else if (sel_mode == kvs::SEL_EXACT) {
+    KV_TRY(need(K, "K"));
+  } else {
+    if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "Quest scoring reads bf16 bounds (bf16 caches only)");
+    KV_TRY(need(k_bounds, "k_bounds"));
+  }
   KV_TRY(need(block_idx, "block_idx", 4));
   KV_TRY(need(n_kept, "n_kept", 4));
   if (scores) KV_TRY(need(scores, "scores", 4));
@@ -416,6 +452,7 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv
   kvs::SelParams p{};
   p.q = q;
   p.k_sum = k_sum;
+  p.k_bounds = k_bounds;
   p.counts = counts;
   p.K = K;
   p.seq_lens = shape->seq_lens;
@@ -434,11 +471,29 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv
   p.kmax = kmax;
   p.qscale = scale * 1.4426950408889634f;
   const int G = shape->Hq / shape->Hkv;
-  cudaError_t e = kvs::launch_select(shape->dtype, shape->D, G, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY
-                                                                                        : kvs::SEL_EXACT,
-                                     p, NBH, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = kvs::launch_select(shape->dtype, shape->D, G, sel_mode, p, NBH, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return KV_OK;
+}
+}  // namespace
+
+extern "C" {
+
+kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv_score_mode mode,
+                           const float* k_sum, const int32_t* counts, const void* K, int k_top, int force_first,
+                           int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                           kv_stream_t stream) {
+  if (mode != KV_SCORE_SUMMARY && mode != KV_SCORE_EXACT_MASS)
+    return fail(KV_ERR_INVALID_ARG, "unknown score mode %d", (int)mode);
+  return select_any(shape, q, scale, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY : kvs::SEL_EXACT, k_sum, nullptr,
+                    counts, K, k_top, force_first, force_last, kmax, block_idx, n_kept, scores, stream);
+}
+
+kv_status kv_select_blocks_quest(const kv_shape* shape, const void* q, float scale, const void* k_bounds, int k_top,
+                                 int force_first, int force_last, int kmax, int32_t* block_idx, int32_t* n_kept,
+                                 float* scores, kv_stream_t stream) {
+  return select_any(shape, q, scale, kvs::SEL_QUEST, nullptr, k_bounds, nullptr, nullptr, k_top, force_first,
+                    force_last, kmax, block_idx, n_kept, scores, stream);
 }
 
 kv_status kv_sparse_decode_attn(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,

@@ -153,9 +153,10 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
   static std::atomic<int> configured{0};  // one bit per device: smem limit raised
   int dev = 0;
   cudaGetDevice(&dev);
-  const size_t smem = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
+  if constexpr (MODE == SEL_QUEST && sizeof(T) != 2) return cudaErrorInvalidValue;  // bf16 bounds only
+  const size_t smem = MODE != SEL_EXACT ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
   if (!(configured.load() & (1 << (dev & 31)))) {
-    size_t most = MODE == SEL_SUMMARY ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
+    size_t most = MODE != SEL_EXACT ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
     if (most > 227 * 1024) most = 227 * 1024;  // per-CTA limit; larger shapes are refused below
     cudaError_t e = cudaFuncSetAttribute(select_kernel<T, D, G, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(most));
@@ -170,6 +171,10 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
 
 template <typename T, int D, int G>
 cudaError_t select_launch_one(int mode, const SelParams& p, int grid, cudaStream_t st) {
+  if (mode == SEL_QUEST) {
+    if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_QUEST>(p, grid, st);
+    return cudaErrorInvalidValue;
+  }
   return mode == SEL_SUMMARY ? select_launch_mode<T, D, G, SEL_SUMMARY>(p, grid, st)
                              : select_launch_mode<T, D, G, SEL_EXACT>(p, grid, st);
 }

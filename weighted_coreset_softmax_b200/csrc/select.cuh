@@ -31,11 +31,12 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_NW = SEL_THREADS / 32;
 constexpr int SEL_MAXNB = 4096;  // NBcap limit
 
-enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1 };
+enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2 };
 
 struct SelParams {
   const void* q;
   const float* k_sum;
+  const void* k_bounds;  // Quest mode: [B][Hkv][NBcap][D][2] bf16 (min, max)
   const int32_t* counts;
   const void* K;
   const int32_t* seq_lens;
@@ -107,7 +108,12 @@ __host__ __device__ inline size_t sel_summary_smem_bytes(int G, int NBcap) {
          sel_ring_bytes(G);
 }
 
-template <typename T, int D, int G>
+// QUEST: the rows are the Quest bounds -- per channel a (min, max) bf16 pair, also
+// four bytes per channel -- and a lane's logit part is sum_j max(q_j min_j,
+// q_j max_j) over its four channels, with no count term ("COBS: Cumulant Order
+// Block Sparse Attention", the Quest paragraph: the largest inner product any
+// point of the block's bounding box can reach).
+template <typename T, int D, int G, bool QUEST = false>
 __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv, float4* ring, int* cnt,
                               SelMisc& ms) {
   constexpr int LPR = D / 4;  // fp32 rows, float4 per lane
@@ -121,7 +127,8 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = lane / LPR, c = lane % LPR;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
-  const float* ks = p.k_sum + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
+  // four bytes per channel in either layout: fp32 sums, or (min, max) bf16 pairs
+  const float* ks = (QUEST ? static_cast<const float*>(p.k_bounds) : p.k_sum) + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
   const int nbt = (nbv + BATCH - 1) / BATCH;               // batches of the bh
   const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;  // batches of this warp
   // stage s, row i of this lane: ring[(s * RS + i) * SEL_THREADS + tid]
@@ -139,8 +146,10 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
 #pragma unroll
   for (int m = 0; m < SEL_STAGES; ++m) issue(m);
   // counts and q while the first batches are in flight
-  const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
-  for (int i = tid; i < nbv; i += SEL_THREADS) cnt[i] = __ldg(cn + i);
+  if constexpr (!QUEST) {
+    const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
+    for (int i = tid; i < nbv; i += SEL_THREADS) cnt[i] = __ldg(cn + i);
+  }
   const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c * 4;
   float4 qf[G];
 #pragma unroll
@@ -165,16 +174,39 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     for (int i = 0; i < RS; ++i) {
       const int row = rb + i * RPW + rg;
       const float4 k4 = row < nbv ? ring[(st * RS + i) * SEL_THREADS + tid] : make_float4(0.f, 0.f, 0.f, 0.f);
+      if constexpr (QUEST) {
+        // (min, max) pairs of channels 4c .. 4c + 3
+        const __nv_bfloat162* mm = reinterpret_cast<const __nv_bfloat162*>(&k4);
+        float lo[4], hi[4];
 #pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        if (g < G) {
-          float d = qf[g].x * k4.x;
-          d = fmaf(qf[g].y, k4.y, d);
-          d = fmaf(qf[g].z, k4.z, d);
-          d = fmaf(qf[g].w, k4.w, d);
-          part[i * GP + g] = d;
-        } else {
-          part[i * GP + g] = 0.f;
+        for (int e = 0; e < 4; ++e) {
+          lo[e] = __low2float(mm[e]);
+          hi[e] = __high2float(mm[e]);
+        }
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          if (g < G) {
+            const float qv[4] = {qf[g].x, qf[g].y, qf[g].z, qf[g].w};
+            float d = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d += fmaxf(qv[e] * lo[e], qv[e] * hi[e]);
+            part[i * GP + g] = d;
+          } else {
+            part[i * GP + g] = 0.f;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          if (g < G) {
+            float d = qf[g].x * k4.x;
+            d = fmaf(qf[g].y, k4.y, d);
+            d = fmaf(qf[g].z, k4.z, d);
+            d = fmaf(qf[g].w, k4.w, d);
+            part[i * GP + g] = d;
+          } else {
+            part[i * GP + g] = 0.f;
+          }
         }
       }
     }
@@ -186,8 +218,13 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
       const int ri = vi / GP, g = vi % GP;
       const int row = rb + ri * RPW + rg;
       if (g < G && row < nbv) {
-        const int nb = cnt[row];
-        const float x = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+        float x;
+        if constexpr (QUEST) {
+          x = part[j];  // the box bound, in the log2 domain through qscale
+        } else {
+          const int nb = cnt[row];
+          x = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
+        }
         lg[g * nbp + row] = x;
         if (x != -INFINITY) {
           if (x > om[j]) {
@@ -334,10 +371,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
-  if (MODE == SEL_SUMMARY) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST) {
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-    score_summary<T, D, G>(p, lg, nbp, bh, nbv, ring, cnt, ms);
+    score_summary<T, D, G, MODE == SEL_QUEST>(p, lg, nbp, bh, nbv, ring, cnt, ms);
   }
   else
     score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
@@ -345,7 +382,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
 
   // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain): in summary
   // mode from the warps' (max, sum) pairs of the scoring pass, else a pass over lg
-  if (MODE == SEL_SUMMARY) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST) {
     if (warp == 0 && lane < G) {
       float M = -INFINITY;
 #pragma unroll

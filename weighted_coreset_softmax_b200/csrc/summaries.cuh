@@ -80,6 +80,60 @@ __global__ void __launch_bounds__(256) block_sums_kernel(const T* __restrict__ K
   if (tensor == 0 && (bh % Hkv) == 0 && c == 0) counts[static_cast<int64_t>(b) * NBcap + blk] = cnt;
 }
 
+// Per-block key bounds for the Quest scorer ("COBS: Cumulant Order Block Sparse
+// Attention", the paragraph on escaping the first-order ceiling: per block the
+// element-wise minimum and maximum of its keys). bf16 caches; output
+// [B][Hkv][NBcap][D][2] bf16, (min, max) of each channel side by side, so a block
+// is one 4D-byte row like the fp32 key sums; blocks past the sequence get zeros.
+// One thread owns one 16-byte channel chunk of one block and walks its rows.
+template <int D>
+__global__ void __launch_bounds__(256) block_bounds_kernel(const __nv_bfloat16* __restrict__ K,
+                                                           const int32_t* __restrict__ seq_lens,
+                                                           __nv_bfloat16* __restrict__ bounds, int NBH, int Hkv,
+                                                           int Ncap, int L, int NBcap) {
+  constexpr int LPR = D / 8;  // 16-byte chunks (8 channels) per row
+  const int64_t gid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t total = static_cast<int64_t>(NBH) * NBcap * LPR;
+  if (gid >= total) return;
+  const int c = static_cast<int>(gid % LPR);
+  const int64_t rest = gid / LPR;
+  const int blk = static_cast<int>(rest % NBcap);
+  const int bh = static_cast<int>(rest / NBcap);
+  const int n = max(0, min(seq_lens[bh / Hkv], Ncap));
+  const int start = blk * L;
+  const int cnt = max(0, min(L, n - start));
+  const __nv_bfloat16* src = K + (static_cast<int64_t>(bh) * Ncap + start) * D + c * 8;
+  __nv_bfloat162 mn[4], mx[4];
+  if (cnt > 0) {
+    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(src));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) mn[e] = mx[e] = h[e];
+  } else {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) mn[e] = mx[e] = __floats2bfloat162_rn(0.f, 0.f);
+  }
+  for (int r = 1; r < cnt; ++r) {
+    const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(src + static_cast<int64_t>(r) * D));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      mn[e] = __hmin2(mn[e], h[e]);
+      mx[e] = __hmax2(mx[e], h[e]);
+    }
+  }
+  // channels 8c .. 8c + 7 as (min, max) pairs: 32 bytes
+  __nv_bfloat162 out[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    out[2 * e] = __halves2bfloat162(__low2bfloat16(mn[e]), __low2bfloat16(mx[e]));
+    out[2 * e + 1] = __halves2bfloat162(__high2bfloat16(mn[e]), __high2bfloat16(mx[e]));
+  }
+  uint4* dst = reinterpret_cast<uint4*>(bounds + ((static_cast<int64_t>(bh) * NBcap + blk) * D + c * 8) * 2);
+  dst[0] = *reinterpret_cast<const uint4*>(&out[0]);
+  dst[1] = *reinterpret_cast<const uint4*>(&out[4]);
+}
+
 // tot[bh][d] = sum over blocks of sums[bh][blk][d], four interleaved partial sums
 // combined in a fixed order.
 __global__ void __launch_bounds__(256) block_totals_kernel(const float* __restrict__ k_sum,
