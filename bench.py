@@ -337,59 +337,90 @@ def run_ours(args, dist):
     kv.lib()
 
     name = args.workload
-    wl = W.make(name, dev, budget=args.budget, B=args.batch,
-                seed=(None if dist.rank == 0 else (100 if name == "llama" else 3) + shard_seed_offset(dist.rank)))
-    sl = wl.seq_lens_tensor(dev)
+    base_seed = (100 if name == "llama" else 3) + shard_seed_offset(dist.rank)
+    L2_BYTES = 126 << 20
+
+    def make_set(j):
+        seed = (None if dist.rank == 0 else base_seed) if j == 0 else base_seed + 50000 * j
+        w_ = W.make(name, dev, budget=args.budget, B=args.batch, seed=seed)
+        sl_ = w_.seq_lens_tensor(dev)
+        su_ = kv.kv_build_block_summaries(w_.K, w_.V, sl_, w_.block_size)
+        if w_.score_mode == "quest":
+            su_["k_bounds"] = kv.kv_build_block_bounds(w_.K, sl_, w_.block_size)
+        return dict(wl=w_, sl=sl_, summ=su_,
+                    idx=torch.zeros(w_.B, w_.Hkv, w_.kmax, dtype=torch.int32, device=dev),
+                    nk=torch.zeros(w_.B, w_.Hkv, dtype=torch.int32, device=dev),
+                    out=torch.empty(w_.B, w_.Hq, w_.D, dtype=torch.float32, device=dev),
+                    lse=torch.empty(w_.B, w_.Hq, dtype=torch.float32, device=dev),
+                    ws=kv.Workspace(kv.make_shape(w_.q, w_.K, sl_, w_.block_size), dev))
+
+    # independent batches (own caches, summaries, queries) rotated through the timed
+    # steps: enough that twice the L2 capacity of other data passes between two uses
+    # of a batch
+    sets = [make_set(0)]
+    w0_ = sets[0]["wl"]
+    es = 2 if str(w0_.dtype).endswith("bfloat16") else 4
+    if w0_.attn_mode == "weighted":
+        step_est = weighted_bytes(w0_)
+    else:
+        step_est = (osa_select_bytes(w0_, w0_.seq_lens) if w0_.score_mode == "exact_mass" else
+                    select_bytes(w0_, w0_.seq_lens))
+        step_est += w0_.B * w0_.Hkv * w0_.kmax * w0_.block_size * w0_.D * es * 2
+    ROT = int(min(16, max(4, 1 + -(-2 * L2_BYTES // step_est))))
+    sets += [make_set(j) for j in range(1, ROT)]
+    s0 = sets[0]
+    wl, sl, summ, idx, nk, out, lse, ws = (s0[k] for k in ("wl", "sl", "summ", "idx", "nk", "out", "lse", "ws"))
     B = wl.B
-    summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
     quest = wl.score_mode == "quest"
-    if quest:
-        summ["k_bounds"] = kv.kv_build_block_bounds(wl.K, sl, wl.block_size)
-    shape = kv.make_shape(wl.q, wl.K, sl, wl.block_size)
-    ws = kv.Workspace(shape, dev)
     mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
     kmax = wl.kmax
-    idx = torch.zeros(B, wl.Hkv, kmax, dtype=torch.int32, device=dev)
-    nk = torch.zeros(B, wl.Hkv, dtype=torch.int32, device=dev)
-    out = torch.empty(B, wl.Hq, wl.D, dtype=torch.float32, device=dev)
-    lse = torch.empty(B, wl.Hq, dtype=torch.float32, device=dev)
     weighted = wl.attn_mode == "weighted"
 
-    def select_on(q_, w_, sl_, su_, idx_, nk_):
+    def select_on(st_, q_=None):
+        if weighted:
+            return
+        w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
+        q_ = w_.q if q_ is None else q_
         if quest:
             kv.kv_select_blocks_quest(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_bounds"], w_.k_top,
-                                      w_.force_first, w_.force_last, kmax=kmax, block_idx=idx_, n_kept=nk_)
+                                      w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
+                                      n_kept=st_["nk"])
         else:
             kv.kv_select_blocks(q_, w_.K, sl_, w_.block_size, w_.scale, su_["counts"], w_.k_top,
                                 w_.force_first, w_.force_last, mode=mode, k_sum=su_["k_sum"], kmax=kmax,
-                                block_idx=idx_, n_kept=nk_)
+                                block_idx=st_["idx"], n_kept=st_["nk"])
 
-    def select():
-        if not weighted:
-            select_on(wl.q, wl, sl, summ, idx, nk)
-
-    def attend():
+    def attend_on(st_, q_=None):
+        w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
+        q_ = w_.q if q_ is None else q_
         if weighted:
-            kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws, tok_idx=wl.tok_idx,
-                                     w=wl.w, out=out, lse=lse)
+            kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
+                                     tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
         else:
-            kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws, block_idx=idx,
-                                     n_kept=nk, summaries=summ, use_tail_proxy=True, out=out, lse=lse)
+            kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
+                                     block_idx=st_["idx"], n_kept=st_["nk"], summaries=su_,
+                                     use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        select()
-        attend()
+    def check_status(what):
+        for st_ in sets:
+            if kv.kv_workspace_status(st_["ws"].tensor) != 0:
+                raise RuntimeError(f"device checks failed {what}")
+
+    for i in range(max(3, args.warmup, ROT)):
+        select_on(sets[i % ROT])
+        attend_on(sets[i % ROT])
     torch.cuda.synchronize(dev)
-    if kv.kv_workspace_status(ws.tensor) != 0:
-        raise RuntimeError("device checks failed during warm-up")
+    check_status("during warm-up")
 
     K_steps = args.steps
-    # the step: select + attention back to back (the attention launch may overlap
-    # the end of the select kernel); events only at the step boundaries
+    # The step: select + attention back to back (the attention launch may overlap
+    # the end of the select kernel); events only at the step boundaries, so steps
+    # do not overlap one another. Step i works on batch i mod ROT: a batch's
+    # inputs were last touched ROT - 1 steps (at least twice the L2 capacity of
+    # other data) earlier, as in a decode loop over distinct layers.
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K_steps)]
     clocks = ClockSampler(dev.index)
     clocks.start()
@@ -399,54 +430,54 @@ def run_ours(args, dist):
     w0 = time.time()
     torch.cuda.nvtx.range_push("timed")  # lets a profiler restrict itself to the timed steps
     for i in range(K_steps):
-        flush.zero_()
+        st_ = sets[i % ROT]
         ev[i][0].record(stream)
-        select()
-        attend()
+        select_on(st_)
+        attend_on(st_)
         ev[i][1].record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
-    # each kernel alone, L2 flushed before it: the per-kernel durations of the roofline
+    # each kernel alone (an event pair around each launch, batches rotating): the
+    # per-kernel durations of the roofline
     k_steps = min(K_steps, 100)
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k_steps)]
     for i in range(k_steps):
-        flush.zero_()
+        st_ = sets[i % ROT]
         kev[i][0].record(stream)
-        select()
+        select_on(st_)
         kev[i][1].record(stream)
-        flush.zero_()
         kev[i][2].record(stream)
-        attend()
+        attend_on(st_)
         kev[i][3].record(stream)
+    torch.cuda.synchronize(dev)
+    # the same step on one batch with a 512 MiB write flushing L2 before each step
+    # (a stricter bound: it also evicts the kernels' code from L2)
+    fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(k_steps)]
+    for i in range(k_steps):
+        flush.zero_()
+        fev[i][0].record(stream)
+        select_on(s0)
+        attend_on(s0)
+        fev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     w1 = time.time()
     dist.barrier(dev)
     clk = clocks.stop(w0, w1)
     step_ms_local = statistics.fmean(e[0].elapsed_time(e[1]) for e in ev)
     step_ms = dist.max(step_ms_local, dev)
+    flushed_ms = dist.max(statistics.fmean(e[0].elapsed_time(e[1]) for e in fev), dev)
     sel_avg = statistics.fmean(e[0].elapsed_time(e[1]) for e in kev) if not weighted else 0.0
     att_avg = statistics.fmean(e[2].elapsed_time(e[3]) for e in kev)
 
     # End to end through the public API: every step's q comes in from pinned host
     # memory and its out/lse go back, inside the timed region. The step's copies
     # run on two copy streams and overlap the neighbouring steps' kernels, as a
-    # serving loop would; three independent batches (own caches, summaries and
-    # queries) rotate, so a step never finds its inputs in L2 (no flush needed).
+    # serving loop would; the ROT independent batches rotate, so a step never
+    # finds its inputs in L2 (no flush needed).
     e2e_ms = None
     h2d_bytes = wl.q.numel() * wl.q.element_size()
     d2h_bytes = out.numel() * 4 + lse.numel() * 4
     if not args.no_e2e:
-        sets = [dict(wl=wl, sl=sl, summ=summ, idx=idx, nk=nk, out=out, lse=lse, ws=ws)]
-        for j in (1, 2):
-            wj = W.make(name, dev, budget=args.budget, B=args.batch,
-                        seed=(100 if name == "llama" else 3) + shard_seed_offset(dist.rank) + 50000 * j)
-            slj = wj.seq_lens_tensor(dev)
-            suj = kv.kv_build_block_summaries(wj.K, wj.V, slj, wj.block_size)
-            if quest:
-                suj["k_bounds"] = kv.kv_build_block_bounds(wj.K, slj, wj.block_size)
-            sets.append(dict(wl=wj, sl=slj, summ=suj,
-                             idx=torch.zeros_like(idx), nk=torch.zeros_like(nk), out=torch.empty_like(out),
-                             lse=torch.empty_like(lse), ws=kv.Workspace(kv.make_shape(wj.q, wj.K, slj, wj.block_size), dev)))
         for st_ in sets:
             st_["q_dev"] = torch.empty_like(st_["wl"].q)
             st_["q_host"] = st_["wl"].q.detach().cpu().pin_memory()
@@ -456,15 +487,8 @@ def run_ours(args, dist):
                 st_[e] = torch.cuda.Event()
 
         def step_on(st_):
-            w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
-            if weighted:
-                kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
-                                         tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
-            else:
-                select_on(st_["q_dev"], w_, sl_, su_, st_["idx"], st_["nk"])
-                kv.kv_sparse_decode_attn(st_["q_dev"], w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
-                                         block_idx=st_["idx"], n_kept=st_["nk"], summaries=su_,
-                                         use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
+            select_on(st_, st_["q_dev"])
+            attend_on(st_, st_["q_dev"])
 
         s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
@@ -472,8 +496,8 @@ def run_ours(args, dist):
             # n steps over the rotating batches; a wait only on events recorded here
             seen = set()
             for i in range(n):
-                st_ = sets[i % 3]
-                key = i % 3
+                st_ = sets[i % ROT]
+                key = i % ROT
                 with torch.cuda.stream(s_in):
                     if (key, "comp") in seen:
                         s_in.wait_event(st_["ev_comp"])  # the step before on this batch has read q_dev
@@ -501,7 +525,7 @@ def run_ours(args, dist):
             cap.wait_stream(torch.cuda.current_stream(dev))
             for s_ in (s_in, s_comp, s_out):
                 s_.wait_stream(cap)
-            enqueue(3)
+            enqueue(ROT)
             for s_ in (s_in, s_comp, s_out):
                 cap.wait_stream(s_)
             torch.cuda.current_stream(dev).wait_stream(cap)
@@ -529,11 +553,7 @@ def run_ours(args, dist):
         dist.barrier(dev)
         e2e_ms = dist.max(e_start.elapsed_time(e_end) / (reps * NG), dev)
         del graph
-        for st_ in sets[1:]:
-            if kv.kv_workspace_status(st_["ws"].tensor) != 0:
-                raise RuntimeError("device checks failed in the end-to-end steps")
-        del sets
-        torch.cuda.empty_cache()
+        check_status("in the end-to-end steps")
 
     # the dense baseline on the identical cache
     dense = None
@@ -556,8 +576,7 @@ def run_ours(args, dist):
                  "speedup_attn_kernel": d_ms / att_avg, "speedup_step": d_ms / step_ms_local}
 
     torch.cuda.synchronize(dev)
-    if kv.kv_workspace_status(ws.tensor) != 0:
-        raise RuntimeError("device checks failed during timing")
+    check_status("during timing")
 
     # algorithmic bytes and the roofline of the dominant kernel
     if weighted:
@@ -583,6 +602,8 @@ def run_ours(args, dist):
         "steps": K_steps,
         "warmup": args.warmup,
         "ms_per_step": step_ms,
+        "ms_per_step_l2_flushed": flushed_ms,
+        "value_l2_flushed": queries / (flushed_ms * 1e-3),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -593,7 +614,10 @@ def run_ours(args, dist):
             "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "ctx": wl.Ncap,
             "block": wl.block_size, "k_top": wl.k_top, "kmax": kmax, "kv_dtype": "bf16",
             "parallelism": f"replicas: batch-sharded, {dist.world} rank(s), no collective",
-            "l2": "flushed before every step and before each kernel timed alone (512 MiB write), outside the timed events",
+            "l2": f"inputs larger than L2: {ROT} independent batches (own caches, summaries, queries) rotate, "
+                  f"so {ROT - 1} steps' data (about {(ROT - 1) * step_est / 1e6:.0f} MB) pass between two uses of "
+                  f"a batch; no flush. "
+                  f"ms_per_step_l2_flushed: the step on one batch after a 512 MiB L2-flushing write",
             "step": "kv_select_blocks + kv_sparse_decode_attn" if not weighted else "kv_sparse_decode_attn",
         },
         "achieved_step_GB_s": step_gbs,
@@ -608,7 +632,7 @@ def run_ours(args, dist):
             "value": queries / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d_bytes,
             "d2h_bytes_per_step": d2h_bytes, "ms_per_step": e2e_ms,
             "how": "q in from pinned host memory and out/lse back every step, on two copy streams "
-                   "overlapping the neighbouring steps' kernels; three independent batches rotate "
+                   f"overlapping the neighbouring steps' kernels; {ROT} independent batches rotate "
                    "(inputs never L2-resident); 24 steps per CUDA graph replay"},
         "gpu_launches": (1 if weighted else 2) * K_steps,  # our kernels in the timed steps
         "clocks": clk,
