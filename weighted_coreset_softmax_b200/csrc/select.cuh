@@ -24,6 +24,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "rank.cuh"
 
 namespace kvs {
 
@@ -49,10 +50,16 @@ struct SelParams {
 };
 
 // Shared memory beyond the dynamic arrays.
+// k_top up to this takes the per-warp top-k path, larger k the radix select
+constexpr int SEL_TOPK = 16;
+
 struct SelMisc {
   float lse[8];
   float pm[SEL_NW][8], ps[SEL_NW][8];  // per-warp (max, sum) of the normalisers (summary mode)
-  unsigned hist[256];
+  union {
+    unsigned hist[256];                          // radix select
+    unsigned long long wtop[SEL_NW * SEL_TOPK];  // per-warp largest keys (k <= SEL_TOPK)
+  };
   unsigned long long prefix, mask;
   int krem, digit, above, bucket;
   int wsum[SEL_NW];
@@ -156,6 +163,19 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
   for (int g = 0; g < G; ++g)
     qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
                         load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
+  // QUEST: max(q min, q max) = max(q, 0) max + min(q, 0) min (max >= min), two FMAs
+  float qa[QUEST ? G : 1][4], qb[QUEST ? G : 1][4];
+  if constexpr (QUEST) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      const float qv[4] = {qf[g].x, qf[g].y, qf[g].z, qf[g].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qa[g][e] = fmaxf(qv[e], 0.f);
+        qb[g][e] = fminf(qv[e], 0.f);
+      }
+    }
+  }
   __syncthreads();  // cnt
   // running (max, sum of 2^(x - max)) of the logits this lane holds: the Eq. 5
   // normalisers come out of the scoring pass
@@ -186,10 +206,9 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
 #pragma unroll
         for (int g = 0; g < GP; ++g) {
           if (g < G) {
-            const float qv[4] = {qf[g].x, qf[g].y, qf[g].z, qf[g].w};
             float d = 0.f;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) d += fmaxf(qv[e] * lo[e], qv[e] * hi[e]);
+            for (int e = 0; e < 4; ++e) d = fmaf(qa[g][e], hi[e], fmaf(qb[g][e], lo[e], d));
             part[i * GP + g] = d;
           } else {
             part[i * GP + g] = 0.f;
@@ -423,6 +442,64 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   if (p.scores)
     for (int i = nbv + tid; i < p.NBcap; i += SEL_THREADS) p.scores[static_cast<size_t>(bh) * p.NBcap + i] = 0.f;
   ncand = sel_block_sum(ncand, ms.wsum);  // also orders the key writes
+
+  if (p.k_top > 0 && p.k_top < ncand && p.k_top <= SEL_TOPK) {
+    // Small k: each warp extracts the k largest keys of its share of the blocks
+    // (k rounds of "largest key below the previous one"); warp 0 takes the k
+    // largest of those, adds the forced blocks and writes the kept list in
+    // ascending order. Keys of candidates are distinct and nonzero (the inverted
+    // index is in the low bits), and ncand > k >= 1 means nbv >= 2, so the two
+    // forced blocks are distinct.
+    const int per = (nbv + SEL_NW - 1) / SEL_NW;
+    const int lo = warp * per, hi = min(nbv, lo + per);
+    unsigned long long prev = ~0ull;
+    for (int r = 0; r < p.k_top; ++r) {
+      unsigned long long best = 0ull;
+      for (int i = lo + lane; i < hi; i += 32) {
+        const unsigned long long x = key[i];
+        if (x < prev && x > best) best = x;
+      }
+      best = warp_max_key(best);
+      if (lane == 0) ms.wtop[warp * SEL_TOPK + r] = best;  // 0: no more candidates here
+      prev = best;
+    }
+    __syncthreads();
+    if (warp == 0) {
+      unsigned long long cand[SEL_NW];
+#pragma unroll
+      for (int w = 0; w < SEL_NW; ++w) cand[w] = lane < p.k_top ? ms.wtop[w * SEL_TOPK + lane] : 0ull;
+      unsigned long long won = 0ull;  // lane r: the (r+1)-th largest key
+      prev = ~0ull;
+      for (int r = 0; r < p.k_top; ++r) {
+        unsigned long long best = 0ull;
+#pragma unroll
+        for (int w = 0; w < SEL_NW; ++w)
+          if (cand[w] < prev && cand[w] > best) best = cand[w];
+        best = warp_max_key(best);
+        if (lane == r) won = best;
+        prev = best;
+      }
+      int blk = lane < p.k_top ? static_cast<int>(0xffffffffu - static_cast<uint32_t>(won)) : -1;
+      int nsel = p.k_top;
+      if (p.force_first) {
+        if (lane == nsel) blk = 0;
+        ++nsel;
+      }
+      if (p.force_last) {
+        if (lane == nsel) blk = nbv - 1;
+        ++nsel;
+      }
+      int rank = 0;  // position in ascending order (indices are distinct)
+#pragma unroll 8
+      for (int j = 0; j < 32; ++j) {
+        const int o = __shfl_sync(FULL_MASK, blk, j);
+        rank += (o >= 0 && o < blk);
+      }
+      if (blk >= 0 && rank < p.kmax) p.block_idx[static_cast<size_t>(bh) * p.kmax + rank] = blk;
+      if (lane == 0) p.n_kept[bh] = min(nsel, p.kmax);
+    }
+    return;
+  }
 
   // threshold: select keys with (key & mask) >= prefix
   unsigned long long prefix = 1ull, mask = ~0ull;  // default: every candidate
