@@ -50,7 +50,10 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-dense", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg (three batches in memory)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--rot", type=int, default=None,
+                    help="independent batches rotated through the steps (default: enough to pass twice "
+                         "the L2 capacity between two uses of a batch; 1 for small profiling captures)")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the workload's own batch; smaller for profiler captures)")
     return ap.parse_args(argv)
@@ -154,10 +157,10 @@ class ClockSampler:
 
 
 # DRAM bytes per launch from the committed ncu capture
-# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.385 MB read, 0 written at B=8,
+# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.411 MB read, 0 written at B=8,
 # scaled x4 by sequences to the B=32 launch). Keyed by (kernel, workload, budget, B);
 # to be re-taken whenever the kernel changes.
-NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_384_832}
+NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_410_688}
 
 
 def measured_peak_hbm():
@@ -366,7 +369,7 @@ def run_ours(args, dist):
         step_est = (osa_select_bytes(w0_, w0_.seq_lens) if w0_.score_mode == "exact_mass" else
                     select_bytes(w0_, w0_.seq_lens))
         step_est += w0_.B * w0_.Hkv * w0_.kmax * w0_.block_size * w0_.D * es * 2
-    ROT = int(min(16, max(4, 1 + -(-2 * L2_BYTES // step_est))))
+    ROT = int(min(16, max(4, 1 + -(-2 * L2_BYTES // step_est)))) if args.rot is None else max(1, args.rot)
     sets += [make_set(j) for j in range(1, ROT)]
     s0 = sets[0]
     wl, sl, summ, idx, nk, out, lse, ws = (s0[k] for k in ("wl", "sl", "summ", "idx", "nk", "out", "lse", "ws"))
@@ -626,7 +629,8 @@ def run_ours(args, dist):
             "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "ctx": wl.Ncap,
             "block": wl.block_size, "k_top": wl.k_top, "kmax": kmax, "kv_dtype": "bf16",
             "parallelism": f"replicas: batch-sharded, {dist.world} rank(s), no collective",
-            "l2": f"inputs larger than L2: {ROT} independent batches (own caches, summaries, queries) rotate, "
+            "l2": "one batch and no flush (--rot 1, a profiling run: the timed steps may hit L2)" if ROT == 1 else
+                  f"inputs larger than L2: {ROT} independent batches (own caches, summaries, queries) rotate, "
                   f"so {ROT - 1} steps' data (about {(ROT - 1) * step_est / 1e6:.0f} MB) pass between two uses of "
                   f"a batch; no flush. "
                   f"ms_per_step: K steps back to back in one event pair; ms_per_step_isolated: an event "
