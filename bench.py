@@ -404,6 +404,10 @@ def run_ours(args, dist):
                                      block_idx=st_["idx"], n_kept=st_["nk"], summaries=su_,
                                      use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
 
+    def step_full(st_, q_=None):
+        select_on(st_, q_)
+        attend_on(st_, q_)
+
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -413,18 +417,28 @@ def run_ours(args, dist):
                 raise RuntimeError(f"device checks failed {what}")
 
     for i in range(max(3, args.warmup, ROT)):
-        select_on(sets[i % ROT])
-        attend_on(sets[i % ROT])
+        step_full(sets[i % ROT])
     torch.cuda.synchronize(dev)
     check_status("during warm-up")
 
     K_steps = args.steps
-    # The timed region: K steps back to back on one stream, one event pair around
-    # all of them. A step is select + attention (each kernel may be scheduled while
-    # the one before it finishes, and waits for it before touching memory). Step i
-    # works on batch i mod ROT: a batch's inputs were last touched ROT - 1 steps
-    # (at least twice the L2 capacity of other data) earlier, as in a decode loop
-    # over distinct layers.
+    # The timed region: K steps back to back on one stream, captured once in a
+    # CUDA graph (so the host's per-call cost cannot stretch the device time) and
+    # replayed between one event pair. A step is select + attention (each kernel
+    # may be scheduled while the one before it finishes, and waits for it before
+    # touching memory). Step i works on batch i mod ROT: a batch's inputs were last
+    # touched ROT - 1 steps (at least twice the L2 capacity of other data) earlier,
+    # as in a decode loop over distinct layers.
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    timed_graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(timed_graph, stream=cap):
+        for i in range(K_steps):
+            step_full(sets[i % ROT])
+    stream.wait_stream(cap)
+    timed_graph.replay()  # warm the graph
+    torch.cuda.synchronize(dev)
+    check_status("in the captured steps")
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(dev.index)
     clocks.start()
@@ -434,26 +448,30 @@ def run_ours(args, dist):
     w0 = time.time()
     torch.cuda.nvtx.range_push("timed")  # lets a profiler restrict itself to the timed steps
     t_start.record(stream)
-    for i in range(K_steps):
-        st_ = sets[i % ROT]
-        select_on(st_)
-        attend_on(st_)
+    timed_graph.replay()
     t_end.record(stream)
     torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize(dev)
+    del timed_graph
+
+    # The secondary loops are issued eagerly behind a GPU sleep long enough for the
+    # host to queue them all, so their events time the device, not the host.
+    def host_ahead(n_launch):
+        torch.cuda._sleep(int(min(4e9, 2.5e5 * n_launch)))  # about 125 us of SM clock per launch
+
     # each step alone: an event pair around every step, so steps do not overlap
     k_steps = min(K_steps, 100)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(k_steps)]
+    host_ahead(2 * k_steps)
     for i in range(k_steps):
-        st_ = sets[i % ROT]
         ev[i][0].record(stream)
-        select_on(st_)
-        attend_on(st_)
+        step_full(sets[i % ROT])
         ev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     # each kernel alone (an event pair around each launch, batches rotating): the
     # per-kernel durations of the roofline
     kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(k_steps)]
+    host_ahead(2 * k_steps)
     for i in range(k_steps):
         st_ = sets[i % ROT]
         kev[i][0].record(stream)
@@ -466,11 +484,11 @@ def run_ours(args, dist):
     # the same step on one batch with a 512 MiB write flushing L2 before each step
     # (a stricter bound: it also evicts the kernels' code from L2)
     fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(k_steps)]
+    host_ahead(3 * k_steps)
     for i in range(k_steps):
         flush.zero_()
         fev[i][0].record(stream)
-        select_on(s0)
-        attend_on(s0)
+        step_full(s0)
         fev[i][1].record(stream)
     torch.cuda.synchronize(dev)
     w1 = time.time()
@@ -501,8 +519,7 @@ def run_ours(args, dist):
                 st_[e] = torch.cuda.Event()
 
         def step_on(st_):
-            select_on(st_, st_["q_dev"])
-            attend_on(st_, st_["q_dev"])
+            step_full(st_, st_["q_dev"])
 
         s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
@@ -633,7 +650,7 @@ def run_ours(args, dist):
                   f"inputs larger than L2: {ROT} independent batches (own caches, summaries, queries) rotate, "
                   f"so {ROT - 1} steps' data (about {(ROT - 1) * step_est / 1e6:.0f} MB) pass between two uses of "
                   f"a batch; no flush. "
-                  f"ms_per_step: K steps back to back in one event pair; ms_per_step_isolated: an event "
+                  f"ms_per_step: K steps back to back (one CUDA graph) in one event pair; ms_per_step_isolated: an event "
                   f"pair around each step; ms_per_step_l2_flushed: the step on one batch after a 512 MiB "
                   f"L2-flushing write",
             "step": "kv_select_blocks + kv_sparse_decode_attn" if not weighted else "kv_sparse_decode_attn",
