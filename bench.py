@@ -369,7 +369,7 @@ def run_ours(args, dist):
         step_est = (osa_select_bytes(w0_, w0_.seq_lens) if w0_.score_mode == "exact_mass" else
                     select_bytes(w0_, w0_.seq_lens))
         step_est += w0_.B * w0_.Hkv * w0_.kmax * w0_.block_size * w0_.D * es * 2
-    ROT = int(min(16, max(4, 1 + -(-2 * L2_BYTES // step_est)))) if args.rot is None else max(1, args.rot)
+    ROT = int(min(16, max(8, 1 + -(-2 * L2_BYTES // step_est)))) if args.rot is None else max(1, args.rot)
     sets += [make_set(j) for j in range(1, ROT)]
     s0 = sets[0]
     wl, sl, summ, idx, nk, out, lse, ws = (s0[k] for k in ("wl", "sl", "summ", "idx", "nk", "out", "lse", "ws"))

@@ -14,7 +14,12 @@ Sources (page title, then section / equation):
           exact-mass ranking (the OSA paragraph), and the Quest min/max score it
           analyses (the paragraph on escaping the first-order ceiling: per block
           the element-wise minimum and maximum of the keys, scored by the largest
-          inner product any point of that box can reach).
+          inner product any point of that box can reach); the second-order
+          estimator (truncating the cumulant expansion (8) at second order: the
+          block log-mass as ln L plus the first two cumulants of sigma q.k over
+          the block's keys) with the covariance kept as its top r scaled
+          eigenvectors (the low-rank spectral decomposition (13): each
+          eigenvector times the square root of its eigenvalue).
   [OA]    "OpenAttention reads 1% of the KV cache -- Count-aware tail proxy",
           section "Skipping reviews without losing the verdict" (the proxy token)
           and section "A worked example with named numbers".
@@ -44,6 +49,12 @@ notes of the repository):
       the place of the block log-mass estimate in the Equation 5 group score
       (per-head block softmax probabilities summed over the group), with no count
       term; forced blocks and ties as in R5 and R6.
+  R12 Second-order scoring: the block's keys are the distribution whose
+      cumulants enter, so the covariance is the population one over the n_b keys
+      (divided by n_b) and ln L becomes ln n_b as in R2; the estimate
+      sigma q.mean + (sigma^2 / 2) q^T Sigma_r q + ln n_b, with Sigma_r = sum of the
+      top r xi_i xi_i^T, is the block logit in the Equation 5 group score. The
+      full-space factors are used (no query subspace, no FP4 quantisation).
 """
 from __future__ import annotations
 
@@ -119,6 +130,43 @@ def quest_logits(qg: np.ndarray, kmin: np.ndarray, kmax: np.ndarray, sigma: floa
     out = np.empty((G, NB))
     for g in range(G):
         out[g] = sigma * np.maximum(qg[g] * kmin, qg[g] * kmax).sum(axis=1)
+    return out
+
+
+def block_cov_factors_one(K: np.ndarray, n: int, L: int, NBcap: int, r: int):
+    """Per block, the top r scaled eigenvectors xi_i = sqrt(lambda_i) u_i of the
+    covariance of the block's keys (population covariance, divided by the count),
+    eigenvalues in descending order [COBS, the low-rank spectral decomposition
+    (13); reading R12]. Returns xi [NBcap][r][D] and the eigenvalues [NBcap][r];
+    blocks past the sequence, and directions past the covariance's rank, stay 0."""
+    D = K.shape[1]
+    xi = np.zeros((NBcap, r, D))
+    lam = np.zeros((NBcap, r))
+    for b, (s, e) in enumerate(blocks_of(n, L)):
+        X = K[s:e] - K[s:e].mean(axis=0)
+        cov = X.T @ X / (e - s)
+        w, U = np.linalg.eigh(cov)  # ascending
+        for i in range(min(r, D)):
+            li = max(float(w[D - 1 - i]), 0.0)
+            lam[b, i] = li
+            xi[b, i] = math.sqrt(li) * U[:, D - 1 - i]
+    return xi, lam
+
+
+def cobs_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, xi: np.ndarray, sigma: float):
+    """s_hat[g][b] = sigma q_g . mean_b + (sigma^2 / 2) sum_i (q_g . xi_bi)^2 + ln n_b:
+    the cumulant expansion of the block log-mass truncated at second order, with
+    the covariance in its rank-r form [COBS, text after Equation (8) and (13);
+    reading R12]."""
+    G = qg.shape[0]
+    NB = k_sum.shape[0]
+    out = np.empty((G, NB))
+    for b in range(NB):
+        nb = int(counts[b])
+        mean = k_sum[b] / nb
+        for g in range(G):
+            quad = float(np.sum((xi[b] @ qg[g]) ** 2))
+            out[g, b] = sigma * float(qg[g] @ mean) + 0.5 * sigma * sigma * quad + math.log(nb)
     return out
 
 
@@ -308,7 +356,7 @@ def dense_attend_one(qg, K, V, n, sigma):
 
 # --------------------------------------------------------------------------- batched
 def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
-                 k_sum=None, counts=None, bh=None):
+                 k_sum=None, counts=None, bh=None, rank=4):
     """Block choice for every (sequence, KV head), or for the listed ones.
 
     q: [B][Hq][D]; K: [B][Hkv][Ncap][D] float64 (needed for exact-mass mode and to
@@ -337,6 +385,10 @@ def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
         elif mode == "quest":
             kmin, kmax = block_bounds_one(K[b, h], n, L, NBcap)
             shat = quest_logits(qg, kmin[:nb], kmax[:nb], sigma)
+        elif mode == "cobs":
+            ks, _, c, _, _ = block_summaries_one(K[b, h], K[b, h], n, L, NBcap)
+            xi, _ = block_cov_factors_one(K[b, h], n, L, NBcap, rank)
+            shat = cobs_logits(qg, ks[:nb], c[:nb], xi[:nb], sigma)
         else:
             raise ValueError(mode)
         S = group_score(shat)

@@ -411,6 +411,123 @@ def pin_quest_upper_bound(seed=15):
     _close(O.quest_logits(qg, kmin1, kmax1, 0.5)[:, 0], 0.5 * (k1 @ qg.T)[0], what="one-key block")
 
 
+# ----------------------------------------------------------------- second-order (COBS) scorer
+def _py_cov_quadratic(K, s, e, q):
+    """q^T Sigma q of the keys K[s:e], Sigma the population covariance, by loops."""
+    n = e - s
+    D = len(q)
+    mean = [sum(float(K[r][j]) for r in range(s, e)) / n for j in range(D)]
+    tot = 0.0
+    for r in range(s, e):
+        d = sum(float(q[j]) * (float(K[r][j]) - mean[j]) for j in range(D))
+        tot += d * d
+    return tot / n, mean
+
+
+def pin_cobs_full_rank_is_exact_quadratic(seed=16):
+    # with r = D the stored factors carry the whole covariance: the logit equals
+    # sigma q.mean + (sigma^2 / 2) q^T Sigma q + ln n computed by loops
+    g = _rng(seed)
+    D, L, n = 6, 12, 30  # blocks of 12, 12 and 6 keys
+    K = g.normal(size=(n, D)) * g.uniform(0.3, 2.0, size=D)
+    qg = g.normal(size=(2, D))
+    NB = 3
+    ks, _, c, _, _ = O.block_summaries_one(K, K, n, L, NB)
+    xi, _ = O.block_cov_factors_one(K, n, L, NB, D)
+    sig = 0.8
+    sh = O.cobs_logits(qg, ks, c, xi, sig)
+    for b, (s, e) in enumerate(O.blocks_of(n, L)):
+        for gi in range(2):
+            quad, mean = _py_cov_quadratic(K, s, e, qg[gi])
+            ref = sig * sum(float(qg[gi][j]) * mean[j] for j in range(D)) + 0.5 * sig * sig * quad + math.log(e - s)
+            _close(sh[gi, b], ref, 1e-11, what="second-order logit, full rank")
+
+
+def pin_cobs_rank_one_block(seed=17):
+    # keys on a line through their mean: the covariance has rank 1, so r = 1
+    # already holds all of it, the first eigenvalue is var(t) |v|^2 and the rest 0
+    g = _rng(seed)
+    D, n = 5, 16
+    mu = g.normal(size=D)
+    v = g.normal(size=D)
+    t = g.normal(size=n)
+    K = mu[None, :] + t[:, None] * v[None, :]
+    xi1, lam = O.block_cov_factors_one(K, n, n, 1, 3)
+    var_t = float(np.mean((t - t.mean()) ** 2))
+    _close(lam[0, 0], var_t * float(v @ v), 1e-11, what="rank-one eigenvalue")
+    _close(lam[0, 1:], np.zeros(2), 1e-11, what="eigenvalues past the rank")
+    q = g.normal(size=D)
+    quad, _ = _py_cov_quadratic(K, 0, n, q)
+    _close(float((xi1[0, 0] @ q) ** 2), quad, 1e-11, what="rank-one quadratic form")
+
+
+def pin_cobs_two_point_closed_form(seed=18):
+    # keys mean +- v in equal numbers: the exact log-mass is ln n + x0 + ln cosh(x)
+    # with x0 = sigma q.mean, x = sigma q.v; the second-order estimate replaces
+    # ln cosh(x) by x^2 / 2
+    g = _rng(seed)
+    D, half = 4, 5
+    mu = g.normal(size=D)
+    v = 0.7 * g.normal(size=D)
+    K = np.concatenate([mu[None, :] + v[None, :]] * half + [mu[None, :] - v[None, :]] * half)
+    n = 2 * half
+    q = g.normal(size=(1, D))
+    sig = 0.9
+    ks, _, c, _, _ = O.block_summaries_one(K, K, n, n, 1)
+    xi, _ = O.block_cov_factors_one(K, n, n, 1, 2)
+    est = O.cobs_logits(q, ks, c, xi, sig)[0, 0]
+    exact = O.exact_log_mass(q, K, n, n, 1, sig)[0, 0]
+    x0 = sig * float(q[0] @ mu)
+    x = sig * float(q[0] @ v)
+    _close(exact, math.log(n) + x0 + math.log(math.cosh(x)), 1e-12, what="two-point exact mass")
+    _close(est - exact, 0.5 * x * x - math.log(math.cosh(x)), 1e-12, what="two-point second-order gap")
+
+
+def pin_cobs_error_order(seed=19):
+    # keys mean + eps z: the first-order (mean-pool) error shrinks like eps^2, the
+    # second-order one like eps^3 (the third cumulant is the first term dropped)
+    g = _rng(seed)
+    D, n = 6, 24
+    mu = g.normal(size=D)
+    Z = g.normal(size=(n, D))
+    q = g.normal(size=(1, D))
+    sig = 1.0
+
+    def errs(eps):
+        K = mu[None, :] + eps * Z
+        ks, _, c, _, _ = O.block_summaries_one(K, K, n, n, 1)
+        xi, _ = O.block_cov_factors_one(K, n, n, 1, D)
+        exact = O.exact_log_mass(q, K, n, n, 1, sig)[0, 0]
+        first = O.summary_logits(q, ks, c, sig)[0, 0]
+        second = O.cobs_logits(q, ks, c, xi, sig)[0, 0]
+        return abs(exact - first), abs(exact - second)
+
+    e1a, e2a = errs(0.02)
+    e1b, e2b = errs(0.01)
+    assert 3.6 < e1a / e1b < 4.4, f"first-order error ratio {e1a / e1b:.3f} (eps^2 expects 4)"
+    assert 6.5 < e2a / e2b < 9.5, f"second-order error ratio {e2a / e2b:.3f} (eps^3 expects 8)"
+    assert e2a < 0.1 * e1a, "the second-order estimate is not closer than the first-order one"
+
+
+def pin_cobs_eigen_structure(seed=20):
+    # scaled eigenvectors: mutually orthogonal, |xi_i|^2 = lambda_i descending, and
+    # with r = D their outer products sum to the covariance (by loops)
+    g = _rng(seed)
+    D, n = 5, 9
+    K = g.normal(size=(n, D)) * g.uniform(0.5, 2.0, size=D)
+    xi, lam = O.block_cov_factors_one(K, n, n, 1, D)
+    X = xi[0]
+    gram = X @ X.T
+    _close(gram - np.diag(np.diag(gram)), np.zeros((D, D)), 1e-11, what="orthogonal factors")
+    _close(np.diag(gram), lam[0], 1e-11, what="|xi|^2 = eigenvalue")
+    assert all(lam[0, i] >= lam[0, i + 1] - 1e-15 for i in range(D - 1)), "eigenvalues not descending"
+    for a in range(D):
+        for b2 in range(D):
+            ca = sum((float(K[r][a]) - float(np.mean(K[:, a]))) * (float(K[r][b2]) - float(np.mean(K[:, b2])))
+                     for r in range(n)) / n
+            _close(float(np.sum(X[:, a] * X[:, b2])), ca, 1e-11, what="sum of xi xi^T = covariance")
+
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -418,4 +535,6 @@ ALL_PINS = [
     pin_integer_weights_duplication, pin_zero_weight_excluded, pin_group_score_invariants,
     pin_topk_bruteforce, pin_near_tie_flag, pin_worked_example, pin_empty_inputs,
     pin_summary_equals_exact_for_constant_blocks, pin_quest_box_corners, pin_quest_upper_bound,
+    pin_cobs_full_rank_is_exact_quadratic, pin_cobs_rank_one_block, pin_cobs_two_point_closed_form,
+    pin_cobs_error_order, pin_cobs_eigen_structure,
 ]

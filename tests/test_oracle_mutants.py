@@ -65,6 +65,47 @@ def _mut_exact_mass_max(orig):
     return f
 
 
+def _mut_cobs_no_half(orig):
+    def f(qg, k_sum, counts, xi, sigma):
+        out = orig(qg, k_sum, counts, xi, sigma)
+        for b in range(k_sum.shape[0]):
+            for g in range(qg.shape[0]):
+                out[g, b] += 0.5 * sigma * sigma * float(np.sum((xi[b] @ qg[g]) ** 2))
+        return out
+    return f
+
+
+def _mut_cobs_unsquared(orig):
+    def f(qg, k_sum, counts, xi, sigma):
+        out = orig(qg, k_sum, counts, xi, sigma)
+        for b in range(k_sum.shape[0]):
+            for g in range(qg.shape[0]):
+                p = xi[b] @ qg[g]
+                out[g, b] += 0.5 * sigma * sigma * float(np.sum(p) - np.sum(p ** 2))
+        return out
+    return f
+
+
+def _mut_cov_sample(orig):
+    def f(K, n, L, NBcap, r):
+        xi, lam = orig(K, n, L, NBcap, r)
+        for b, (s, e) in enumerate(O.blocks_of(n, L)):
+            c = e - s
+            if c > 1:
+                xi[b] *= math.sqrt(c / (c - 1))
+                lam[b] *= c / (c - 1)
+        return xi, lam
+    return f
+
+
+def _mut_cov_smallest(orig):
+    def f(K, n, L, NBcap, r):
+        D = K.shape[1]
+        xi_all, lam_all = orig(K, n, L, NBcap, D)
+        return xi_all[:, ::-1][:, :r].copy(), lam_all[:, ::-1][:, :r].copy()
+    return f
+
+
 def _mut_quest_max_end_only(orig):
     def f(qg, kmin, kmax, sigma):
         return np.stack([sigma * (qg[g] * kmax).sum(axis=1) for g in range(qg.shape[0])])
@@ -122,6 +163,10 @@ MUTANTS = {
     "logsumexp/offset": ("logsumexp", _mut_logsumexp_shift),
     "quest/max end only": ("quest_logits", _mut_quest_max_end_only),
     "quest/bounds swapped": ("block_bounds_one", _mut_bounds_swapped),
+    "cobs/no one half": ("cobs_logits", _mut_cobs_no_half),
+    "cobs/projections not squared": ("cobs_logits", _mut_cobs_unsquared),
+    "cobs/sample covariance (n - 1)": ("block_cov_factors_one", _mut_cov_sample),
+    "cobs/smallest eigendirections": ("block_cov_factors_one", _mut_cov_smallest),
 }
 
 
