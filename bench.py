@@ -45,7 +45,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_quest", "llama_coreset"])
+    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_quest", "llama_cobs",
+                                                           "llama_coreset"])
     ap.add_argument("--budget", type=float, default=0.01)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -219,6 +220,17 @@ def quest_select_bytes(wl, seq_lens):
     return total
 
 
+def cobs_select_bytes(wl, seq_lens, rank=4):
+    """Algorithmic bytes of one kv_select_blocks_cobs launch: every valid block's
+    fp32 key sum, count and rank fp32 covariance factors, q, and the kept indices."""
+    L, D, G = wl.block_size, wl.D, wl.G
+    total = 0
+    for b in range(wl.B):
+        nbv = (seq_lens[b] + L - 1) // L
+        total += wl.Hkv * (nbv * (D * 4 + 4 + rank * D * 4) + G * D * 2 + wl.kmax * 4 + 4)
+    return total
+
+
 def osa_select_bytes(wl, seq_lens):
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
     return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
@@ -261,7 +273,7 @@ def oracle_tasks(wl, pairs):
     import numpy as np
     import torch
     tasks = []
-    kind = {"summary": "summary", "exact_mass": "exact_mass", "quest": "quest"}[wl.score_mode]
+    kind = {"summary": "summary", "exact_mass": "exact_mass", "quest": "quest", "cobs": "cobs"}[wl.score_mode]
     if wl.attn_mode == "weighted":
         kind = "weighted"
     for (b, h) in pairs:
@@ -321,6 +333,7 @@ def workload_label(wl, budget):
         "qwen_long": "Qwen2.5-7B-shaped long-context GQA decode",
         "llama_osa": "Llama-3.1-8B-shaped GQA decode, OSA exact-mass selection",
         "llama_quest": "Llama-3.1-8B-shaped GQA decode, Quest key-box selection",
+        "llama_cobs": "Llama-3.1-8B-shaped GQA decode, COBS second-order selection (rank-4 factors)",
         "llama_coreset": "Llama-3.1-8B-shaped GQA decode, weighted coreset m=2048",
     }
     return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, "
@@ -350,6 +363,8 @@ def run_ours(args, dist):
         su_ = kv.kv_build_block_summaries(w_.K, w_.V, sl_, w_.block_size)
         if w_.score_mode == "quest":
             su_["k_bounds"] = kv.kv_build_block_bounds(w_.K, sl_, w_.block_size)
+        if w_.score_mode == "cobs":
+            su_["k_xi"] = kv.kv_build_block_cov_factors(w_.K, sl_, w_.block_size, 4)
         return dict(wl=w_, sl=sl_, summ=su_,
                     idx=torch.zeros(w_.B, w_.Hkv, w_.kmax, dtype=torch.int32, device=dev),
                     nk=torch.zeros(w_.B, w_.Hkv, dtype=torch.int32, device=dev),
@@ -384,7 +399,11 @@ def run_ours(args, dist):
             return
         w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
         q_ = w_.q if q_ is None else q_
-        if quest:
+        if wl.score_mode == "cobs":
+            kv.kv_select_blocks_cobs(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_sum"], su_["counts"], su_["k_xi"],
+                                     w_.k_top, w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
+                                     n_kept=st_["nk"])
+        elif quest:
             kv.kv_select_blocks_quest(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_bounds"], w_.k_top,
                                       w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
                                       n_kept=st_["nk"])
@@ -410,6 +429,28 @@ def run_ours(args, dist):
 
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
+
+    # the once-after-prefill builds, timed on batch 0 (not part of the step)
+    def time_build(fn, reps=3):
+        fn()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        return e0.elapsed_time(e1) / reps
+
+    stream = torch.cuda.current_stream(dev)
+    builds = {"kv_build_block_summaries_ms": time_build(
+        lambda: kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size, out=summ))}
+    if quest:
+        builds["kv_build_block_bounds_ms"] = time_build(
+            lambda: kv.kv_build_block_bounds(wl.K, sl, wl.block_size, out=summ["k_bounds"]))
+    if wl.score_mode == "cobs":
+        builds["kv_build_block_cov_factors_ms"] = time_build(
+            lambda: kv.kv_build_block_cov_factors(wl.K, sl, wl.block_size, 4, out=summ["k_xi"]), reps=1)
 
     def check_status(what):
         for st_ in sets:
@@ -615,6 +656,7 @@ def run_ours(args, dist):
     else:
         a_bytes = attention_bytes(wl, nk, wl.seq_lens)
         s_bytes = (quest_select_bytes(wl, wl.seq_lens) if quest else
+                   cobs_select_bytes(wl, wl.seq_lens) if wl.score_mode == "cobs" else
                    select_bytes(wl, wl.seq_lens) if mode == kv.KV_SCORE_SUMMARY else osa_select_bytes(wl, wl.seq_lens))
     peak, peak_kind = measured_peak_hbm()
     if att_avg >= sel_avg or weighted:
@@ -672,6 +714,7 @@ def run_ours(args, dist):
         "gpu_launches": (1 if weighted else 2) * K_steps,  # our kernels in the timed steps
         "clocks": clk,
         "dense": dense,
+        "builds_once_after_prefill": builds,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, workload_label(wl, args.budget))

@@ -174,6 +174,45 @@ kv_status kv_select_blocks_quest(const kv_shape* shape, const void* q, float sca
                                  int32_t* n_kept, float* scores, kv_stream_t stream);
 
 /*
+ * kv_build_block_cov_factors -- per-block covariance factors for second-order
+ * block scoring. Source: "COBS: Cumulant Order Block Sparse Attention" -- the
+ * cumulant expansion (8) truncated at second order and the low-rank spectral
+ * decomposition (13) of the within-block key covariance.
+ *
+ *   K      device cache [B][Hkv][Ncap][D] (bf16 or fp32)
+ *   rank   r, 1..8: eigendirections kept per block
+ *   k_xi   device out [B][Hkv][NBcap][r][D] fp32, 16-byte aligned: xi_i =
+ *          sqrt(lambda_i) u_i for the r largest eigenvalues lambda_i (descending)
+ *          of the block's population covariance (sum over its n_b keys of
+ *          (k - mean)(k - mean)^T / n_b). The sign of each xi_i is arbitrary;
+ *          directions past the covariance's rank, blocks with fewer than two
+ *          keys and blocks at or past ceil(seq_len / L) are zero.
+ * block_size must be <= 64 (KV_ERR_UNSUPPORTED otherwise). Eigenvectors come from
+ * a float64 Jacobi diagonalisation of each block's Gram matrix. Run once after
+ * prefill (and again if the cache changes).
+ */
+kv_status kv_build_block_cov_factors(const kv_shape* shape, const void* K, int rank, float* k_xi,
+                                     kv_stream_t stream);
+
+/*
+ * kv_select_blocks_cobs -- kv_select_blocks with the second-order block logit.
+ * Source: "COBS: Cumulant Order Block Sparse Attention", text after Equation (8)
+ * (the second-order estimator), the low-rank form (13) and Equation (5):
+ *
+ *   s[g,b] = scale * q_g . (k_sum_b / n_b) + (scale^2 / 2) sum_i (q_g . xi_bi)^2
+ *            + ln n_b
+ *   S[b]   = sum_{g in group} exp(s[g,b] - ln sum_b' exp(s[g,b']))  over valid b'
+ *
+ * k_sum, counts: kv_build_block_summaries output; k_xi, rank: from
+ * kv_build_block_cov_factors. Forcing, ranking, kmax, block_idx, n_kept and
+ * scores are as in kv_select_blocks.
+ */
+kv_status kv_select_blocks_cobs(const kv_shape* shape, const void* q, float scale, const float* k_sum,
+                                const int32_t* counts, const float* k_xi, int rank, int k_top,
+                                int force_first, int force_last, int kmax, int32_t* block_idx,
+                                int32_t* n_kept, float* scores, kv_stream_t stream);
+
+/*
  * kv_sparse_decode_attn -- softmax attention over a reduced KV cache.
  *
  * Block mode (tok_idx == NULL). Source: "OpenAttention reads 1% of the KV cache

@@ -79,7 +79,12 @@ def run_pipeline(wl, *, want_scores=True, use_proxy=True, kmax=None):
     dev = wl.q.device
     sl = wl.seq_lens_tensor(dev)
     summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, wl.block_size)
-    if wl.score_mode == "quest":
+    if wl.score_mode == "cobs":
+        summ["k_xi"] = kv.kv_build_block_cov_factors(wl.K, sl, wl.block_size, 4)
+        idx, nk, scores = kv.kv_select_blocks_cobs(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_sum"],
+                                                   summ["counts"], summ["k_xi"], wl.k_top, wl.force_first,
+                                                   wl.force_last, kmax=kmax, want_scores=want_scores)
+    elif wl.score_mode == "quest":
         summ["k_bounds"] = kv.kv_build_block_bounds(wl.K, sl, wl.block_size)
         idx, nk, scores = kv.kv_select_blocks_quest(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_bounds"],
                                                     wl.k_top, wl.force_first, wl.force_last, kmax=kmax,

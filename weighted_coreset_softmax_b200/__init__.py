@@ -27,7 +27,8 @@ __all__ = [
     "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KV_STEP_AUTO", "KV_STEP_TWO_KERNELS",
     "KV_STEP_FUSED", "KVShape", "KVError",
     "lib", "library_path", "header_path", "make_shape", "kv_build_block_summaries",
-    "kv_select_blocks", "kv_build_block_bounds", "kv_select_blocks_quest", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
+    "kv_select_blocks", "kv_build_block_bounds", "kv_select_blocks_quest",
+    "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace",
 ]
 
@@ -83,6 +84,8 @@ def lib():
         "kv_select_blocks": [_SHP, _P, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_build_block_bounds": [_SHP, _P, _P, _P],
         "kv_select_blocks_quest": [_SHP, _P, _F, _P, _I, _I, _I, _I, _P, _P, _P, _P],
+        "kv_build_block_cov_factors": [_SHP, _P, _I, _P, _P],
+        "kv_select_blocks_cobs": [_SHP, _P, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_sparse_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _I, _P, _P, _P, _P, _P, _I,
                                   _P, _P, _I, _P, _P, _P, _S, _P],
         "kv_dense_decode_attn": [_SHP, _P, _F, _P, _P, _P, _P, _P, _S, _P],
@@ -289,6 +292,51 @@ def kv_select_blocks_quest(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Ten
     _check(lib().kv_select_blocks_quest(ctypes.byref(shape), _ptr(q), float(scale), _ptr(k_bounds), int(k_top),
                                         int(bool(force_first)), int(bool(force_last)), int(kmax),
                                         _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
+    return block_idx, n_kept, scores
+
+
+def kv_build_block_cov_factors(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int, rank: int = 4,
+                               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-block scaled covariance eigenvectors: [B][Hkv][NB][rank][D] fp32."""
+    _need(K, "K")
+    _need(seq_lens, "seq_lens", torch.int32)
+    B, Hkv, Ncap, D = K.shape
+    NB = (Ncap + block_size - 1) // block_size
+    if out is None:
+        out = torch.empty(B, Hkv, NB, rank, D, dtype=torch.float32, device=K.device)
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, block_size, _dtype_code(K.dtype), seq_lens.data_ptr())
+    _check(lib().kv_build_block_cov_factors(ctypes.byref(shape), _ptr(K), int(rank), _ptr(out), _stream(K.device)))
+    return out
+
+
+def kv_select_blocks_cobs(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                          scale: float, k_sum: torch.Tensor, counts: torch.Tensor, k_xi: torch.Tensor, k_top: int,
+                          force_first: bool = False, force_last: bool = False, kmax: Optional[int] = None,
+                          block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                          scores: Optional[torch.Tensor] = None, want_scores: bool = False):
+    """Kept blocks per KV head by the second-order block logit. K is not read (its
+    shape gives the descriptor); the rank is k_xi's fourth dimension. Returns
+    (block_idx [B][Hkv][kmax], n_kept [B][Hkv], scores or None)."""
+    _need(q, "q", K.dtype)
+    _need(k_sum, "k_sum", torch.float32)
+    _need(counts, "counts", torch.int32)
+    _need(k_xi, "k_xi", torch.float32)
+    shape = make_shape(q, K, seq_lens, block_size)
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    dev = q.device
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if scores is None and want_scores:
+        scores = torch.empty(shape.B, shape.Hkv, NB, dtype=torch.float32, device=dev)
+    _check(lib().kv_select_blocks_cobs(ctypes.byref(shape), _ptr(q), float(scale), _ptr(k_sum), _ptr(counts),
+                                       _ptr(k_xi), int(k_xi.shape[3]), int(k_top), int(bool(force_first)),
+                                       int(bool(force_last)), int(kmax), _ptr(block_idx), _ptr(n_kept),
+                                       _ptr(scores), _stream(dev)))
     return block_idx, n_kept, scores
 
 

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -14,6 +15,7 @@
 #include <string>
 
 #include "attention.cuh"
+#include "covariance.cuh"
 #include "kvsparse.h"
 #include "launch.h"
 #include "select.cuh"
@@ -97,6 +99,34 @@ static cudaError_t launch_bounds(int D, const void* K, const int32_t* seq_lens, 
   else
     block_bounds_kernel<128><<<blocks, 256, 0, st>>>(k, seq_lens, out, NBH, Hkv, Ncap, L, NBcap);
   return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t cov_td(const void* K, const int32_t* seq_lens, float* xi, int NBH, int Hkv, int Ncap, int L,
+                          int NBcap, int r, cudaStream_t st) {
+  const size_t smem = cov_smem_bytes(L, D);
+  static std::atomic<int> configured{0};  // one bit per device: smem limit raised
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured.load() & (1 << (dev & 31)))) {
+    const cudaError_t e = cudaFuncSetAttribute(cov_factors_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(cov_smem_bytes(COV_MAX_ROWS, D)));
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(1 << (dev & 31));
+  }
+  const long long grid = static_cast<long long>(NBH) * NBcap;
+  cov_factors_kernel<T, D><<<static_cast<unsigned>(grid), COV_THREADS, smem, st>>>(static_cast<const T*>(K), seq_lens, xi,
+                                                                                  Hkv, Ncap, L, NBcap, r);
+  return cudaGetLastError();
+}
+
+static cudaError_t launch_cov(int dtype, int D, const void* K, const int32_t* seq_lens, float* xi, int NBH, int Hkv,
+                              int Ncap, int L, int NBcap, int r, cudaStream_t st) {
+  if (dtype == KV_BF16)
+    return D == 64 ? cov_td<__nv_bfloat16, 64>(K, seq_lens, xi, NBH, Hkv, Ncap, L, NBcap, r, st)
+                   : cov_td<__nv_bfloat16, 128>(K, seq_lens, xi, NBH, Hkv, Ncap, L, NBcap, r, st);
+  return D == 64 ? cov_td<float, 64>(K, seq_lens, xi, NBH, Hkv, Ncap, L, NBcap, r, st)
+                 : cov_td<float, 128>(K, seq_lens, xi, NBH, Hkv, Ncap, L, NBcap, r, st);
 }
 
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
@@ -417,6 +447,25 @@ kv_status kv_build_block_bounds(const kv_shape* shape, const void* K, void* k_bo
   return KV_OK;
 }
 
+kv_status kv_build_block_cov_factors(const kv_shape* shape, const void* K, int rank, float* k_xi,
+                                     kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  if (rank < 1 || rank > kvs::COV_MAX_RANK) return fail(KV_ERR_INVALID_ARG, "rank = %d outside 1..%d", rank,
+                                                         kvs::COV_MAX_RANK);
+  if (shape->block_size > kvs::COV_MAX_ROWS)
+    return fail(KV_ERR_UNSUPPORTED, "covariance factors are built for block sizes up to %d", kvs::COV_MAX_ROWS);
+  KV_TRY(need(K, "K"));
+  KV_TRY(need(k_xi, "k_xi"));
+  const int NBH = shape->B * shape->Hkv;
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  if (NBH == 0 || NBcap == 0) return KV_OK;
+  if (static_cast<long long>(NBH) * NBcap > 0x7fffffffLL) return fail(KV_ERR_UNSUPPORTED, "too many blocks");
+  cudaError_t e = kvs::launch_cov(shape->dtype, shape->D, K, shape->seq_lens, k_xi, NBH, shape->Hkv, shape->Ncap,
+                                  shape->block_size, NBcap, rank, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "covariance factors launch");
+  return KV_OK;
+}
+
 }  // extern "C"
 
 namespace {
@@ -425,13 +474,18 @@ namespace {
 kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_mode, const float* k_sum,
                      const void* k_bounds, const int32_t* counts, const void* K, int k_top, int force_first,
                      int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
-                     kv_stream_t stream) {
+                     kv_stream_t stream, const float* k_xi = nullptr, int rank = 0) {
   KV_TRY(check_shape(shape));
   if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
   KV_TRY(need(q, "q"));
-  if (sel_mode == kvs::SEL_SUMMARY) {
+  if (sel_mode == kvs::SEL_SUMMARY || sel_mode == kvs::SEL_COBS) {
     KV_TRY(need(k_sum, "k_sum"));
     KV_TRY(need(counts, "counts", 4));
+    if (sel_mode == kvs::SEL_COBS) {
+      KV_TRY(need(k_xi, "k_xi"));
+      if (rank < 1 || rank > kvs::COV_MAX_RANK)
+        return fail(KV_ERR_INVALID_ARG, "rank = %d outside 1..%d", rank, kvs::COV_MAX_RANK);
+    }
   } else if (sel_mode == kvs::SEL_EXACT) {
     KV_TRY(need(K, "K"));
   } else {
@@ -453,6 +507,8 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
   p.q = q;
   p.k_sum = k_sum;
   p.k_bounds = k_bounds;
+  p.k_xi = k_xi;
+  p.cobs_r = rank;
   p.counts = counts;
   p.K = K;
   p.seq_lens = shape->seq_lens;
@@ -487,6 +543,14 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv
     return fail(KV_ERR_INVALID_ARG, "unknown score mode %d", (int)mode);
   return select_any(shape, q, scale, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY : kvs::SEL_EXACT, k_sum, nullptr,
                     counts, K, k_top, force_first, force_last, kmax, block_idx, n_kept, scores, stream);
+}
+
+kv_status kv_select_blocks_cobs(const kv_shape* shape, const void* q, float scale, const float* k_sum,
+                                const int32_t* counts, const float* k_xi, int rank, int k_top, int force_first,
+                                int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                                kv_stream_t stream) {
+  return select_any(shape, q, scale, kvs::SEL_COBS, k_sum, nullptr, counts, nullptr, k_top, force_first, force_last,
+                    kmax, block_idx, n_kept, scores, stream, k_xi, rank);
 }
 
 kv_status kv_select_blocks_quest(const kv_shape* shape, const void* q, float scale, const void* k_bounds, int k_top,

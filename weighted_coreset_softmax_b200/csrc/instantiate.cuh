@@ -175,6 +175,7 @@ cudaError_t select_launch_one(int mode, const SelParams& p, int grid, cudaStream
     if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_QUEST>(p, grid, st);
     return cudaErrorInvalidValue;
   }
+  if (mode == SEL_COBS) return select_launch_mode<T, D, G, SEL_COBS>(p, grid, st);
   return mode == SEL_SUMMARY ? select_launch_mode<T, D, G, SEL_SUMMARY>(p, grid, st)
                              : select_launch_mode<T, D, G, SEL_EXACT>(p, grid, st);
 }

@@ -32,12 +32,14 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_NW = SEL_THREADS / 32;
 constexpr int SEL_MAXNB = 4096;  // NBcap limit
 
-enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2 };
+enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2, SEL_COBS = 3 };
 
 struct SelParams {
   const void* q;
   const float* k_sum;
   const void* k_bounds;  // Quest mode: [B][Hkv][NBcap][D][2] bf16 (min, max)
+  const float* k_xi;     // second-order mode: [B][Hkv][NBcap][cobs_r][D] fp32 scaled eigenvectors
+  int cobs_r;
   const int32_t* counts;
   const void* K;
   const int32_t* seq_lens;
@@ -52,6 +54,7 @@ struct SelParams {
 // Shared memory beyond the dynamic arrays.
 // k_top up to this takes the per-warp top-k path, larger k the radix select
 constexpr int SEL_TOPK = 16;
+constexpr int COV_MAX_RANK_SEL = 8;  // largest rank of the second-order factors
 
 struct SelMisc {
   float lse[8];
@@ -375,6 +378,51 @@ __device__ void score_exact(const SelParams& p, float* lg, int nbp, int bh, int 
   }
 }
 
+// Second-order term ("COBS: Cumulant Order Block Sparse Attention", text after
+// Equation (8) and the low-rank form (13)): adds (sigma^2 / 2) sum_i (q . xi_i)^2
+// to the first-order block logits in lg. In the log2 domain, with qs = q sigma
+// log2(e), that is (ln 2 / 2) sum_i (qs . xi_i)^2. A warp takes RPW blocks at a
+// time (D / 4 lanes per row, a float4 each) and loads all of a block's factor
+// rows before reducing.
+template <int D, int G>
+__device__ void cobs_second_order(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float4 (&qf)[G]) {
+  constexpr int LPR = D / 4;
+  constexpr int RPW = 32 / LPR;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rg = lane / LPR;
+  const int r = p.cobs_r;
+  const float* base = p.k_xi + static_cast<size_t>(bh) * p.NBcap * r * D + (lane % LPR) * 4;
+  for (int b0 = warp * RPW; b0 < nbv; b0 += SEL_NW * RPW) {
+    const int b = b0 + rg;
+    const bool ok = b < nbv;
+    float4 x[COV_MAX_RANK_SEL];
+#pragma unroll
+    for (int i = 0; i < COV_MAX_RANK_SEL; ++i)
+      x[i] = (ok && i < r) ? __ldg(reinterpret_cast<const float4*>(base + (static_cast<size_t>(b) * r + i) * D))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+    float acc[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll
+    for (int i = 0; i < COV_MAX_RANK_SEL; ++i) {
+      if (i >= r) break;
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float d = qf[g].x * x[i].x;
+        d = fmaf(qf[g].y, x[i].y, d);
+        d = fmaf(qf[g].z, x[i].z, d);
+        d = fmaf(qf[g].w, x[i].w, d);
+#pragma unroll
+        for (int o = LPR / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL_MASK, d, o);
+        acc[g] = fmaf(d, d, acc[g]);
+      }
+    }
+    if (ok && (lane % LPR) == 0)
+#pragma unroll
+      for (int g = 0; g < G; ++g) lg[g * nbp + b] += 0.34657359027997264f * acc[g];  // ln 2 / 2
+  }
+}
+
 template <typename T, int D, int G, int MODE>
 __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams p) {
   extern __shared__ __align__(16) unsigned char sel_smem[];
@@ -390,7 +438,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
-  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS) {
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
     score_summary<T, D, G, MODE == SEL_QUEST>(p, lg, nbp, bh, nbv, ring, cnt, ms);
@@ -398,9 +446,22 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   else
     score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
   __syncthreads();
+  if constexpr (MODE == SEL_COBS) {
+    // the first-order logits are in lg; add the second-order term
+    const int h = bh - b * p.Hkv;
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + (lane % (D / 4)) * 4;
+    float4 qf[G];
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
+                          load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
+    cobs_second_order<D, G>(p, lg, nbp, bh, nbv, qf);
+    __syncthreads();
+  }
 
   // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain): in summary
-  // mode from the warps' (max, sum) pairs of the scoring pass, else a pass over lg
+  // and Quest modes from the warps' (max, sum) pairs of the scoring pass, else
+  // (exact and second-order modes) a pass over lg
   if (MODE == SEL_SUMMARY || MODE == SEL_QUEST) {
     if (warp == 0 && lane < G) {
       float M = -INFINITY;

@@ -46,7 +46,7 @@ class Workload:
     k_top: int                   # blocks chosen by score, forced blocks not counted
     force_first: int
     force_last: int
-    score_mode: str              # "summary", "exact_mass" or "quest"
+    score_mode: str              # "summary", "exact_mass", "quest" or "cobs"
     attn_mode: str               # "proxy", "discard", "weighted" or "dense"
     m: int = 0                   # coreset size per (sequence, KV head), weighted mode
     q: Optional[torch.Tensor] = None        # [B][Hq][D]
@@ -117,6 +117,7 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
     name: "tiny" (1 head, d=64, n=1024, L=16, fp32), "llama_b1" (batch 1, 32K),
     "llama" (batch 32, 32K, seeds 100..131), "qwen_long" (batch 8, 128K, G=7),
     "llama_osa" (exact-mass scoring), "llama_quest" (key-box bound scoring),
+    "llama_cobs" (second-order scoring, rank-4 covariance factors),
     "llama_coreset" (weighted coreset, m=2048).
     Keyword overrides shrink a workload for fast tests while keeping its head
     shapes and distributions.
@@ -146,6 +147,10 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=None, ff=1, fl=1, smode="quest", amode="proxy", planted=32,
                     seeds=[4], per_seq=False, plain=False)
+    elif name == "llama_cobs":
+        spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
+                    k_top=None, ff=1, fl=1, smode="cobs", amode="proxy", planted=32,
+                    seeds=[5], per_seq=False, plain=False)
     elif name == "llama_coreset":
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=0, ff=0, fl=0, smode="summary", amode="weighted", planted=32,
