@@ -142,3 +142,31 @@ def test_cobs_full_size_sampled():
         res[(b, h)] = O.select_batch(qb, Kb, [wl.seq_lens[b]], wl.block_size, wl.scale, wl.k_top, True, True,
                                      "cobs")[(0, 0)]
     selection_matches(r["idx"], r["nk"], res, pairs, "full cobs select")
+
+
+@pytest.mark.parametrize("name,rank,L", [
+    ("llama", 3, 64),       # ring, two blocks a batch (6 of 8 rows)
+    ("llama", 8, 64),       # ring, one block a batch
+    ("qwen_long", 4, 64),   # G = 7: ring of 4 rows a stage, one block a batch
+    ("qwen_long", 6, 32),   # G = 7, rank above the ring's rows: direct loads
+    ("tiny", 2, 16),        # D = 64, fp32, G = 1: direct loads
+])
+def test_cobs_rank_and_shape_paths(name, rank, L):
+    kw = dict(tiny=dict(), llama=dict(B=2, Ncap=2000, seq_lens=[2000, 900]),
+              qwen_long=dict(B=2, Ncap=2053, seq_lens=[2053, 700]))[name]
+    wl = W.make(name, DEV, **kw)
+    sl = wl.seq_lens_tensor(DEV)
+    k = 4
+    summ = kv.kv_build_block_summaries(wl.K, wl.V, sl, L)
+    xi = kv.kv_build_block_cov_factors(wl.K, sl, L, rank)
+    idx, nk, sc = kv.kv_select_blocks_cobs(wl.q, wl.K, sl, L, wl.scale, summ["k_sum"], summ["counts"], xi, k,
+                                           True, True, want_scores=True)
+    torch.cuda.synchronize()
+    q, K, _ = oracle_inputs(wl)
+    pairs = all_pairs(wl)
+    sel = O.select_batch(q, K, wl.seq_lens, L, wl.scale, k, True, True, "cobs", rank=rank)
+    selection_matches(idx, nk, sel, pairs, f"cobs {name} rank={rank} L={L}")
+    S = sc.cpu().numpy().astype(np.float64)
+    for (b, h) in pairs:
+        nb = len(sel[(b, h)]["S"])
+        assert np.max(np.abs(S[b, h, :nb] - sel[(b, h)]["S"])) < 1e-4, f"group score at {(b, h)}"

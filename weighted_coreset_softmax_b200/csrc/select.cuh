@@ -381,10 +381,11 @@ __device__ void score_exact(const SelParams& p, float* lg, int nbp, int bh, int 
 // Second-order term ("COBS: Cumulant Order Block Sparse Attention", text after
 // Equation (8) and the low-rank form (13)): adds (sigma^2 / 2) sum_i (q . xi_i)^2
 // to the first-order block logits in lg. In the log2 domain, with qs = q sigma
-// log2(e), that is (ln 2 / 2) sum_i (qs . xi_i)^2. A warp takes RPW blocks at a
-// time (D / 4 lanes per row, a float4 each) and loads all of a block's factor
-// rows before reducing.
-template <int D, int G>
+// log2(e), that is (ln 2 / 2) sum_i (qs . xi_i)^2. A warp takes NBW groups of RPW
+// blocks at a time (D / 4 lanes per row, a float4 each) and issues all their
+// factor-row loads (up to RMAX rows a block) before reducing, so NBW * RMAX loads
+// per lane are in flight.
+template <int D, int G, int NBW, int RMAX>
 __device__ void cobs_second_order(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float4 (&qf)[G]) {
   constexpr int LPR = D / 4;
   constexpr int RPW = 32 / LPR;
@@ -392,35 +393,106 @@ __device__ void cobs_second_order(const SelParams& p, float* lg, int nbp, int bh
   const int rg = lane / LPR;
   const int r = p.cobs_r;
   const float* base = p.k_xi + static_cast<size_t>(bh) * p.NBcap * r * D + (lane % LPR) * 4;
-  for (int b0 = warp * RPW; b0 < nbv; b0 += SEL_NW * RPW) {
-    const int b = b0 + rg;
-    const bool ok = b < nbv;
-    float4 x[COV_MAX_RANK_SEL];
+  for (int b0 = warp * RPW * NBW; b0 < nbv; b0 += SEL_NW * RPW * NBW) {
+    float4 x[NBW][RMAX];
 #pragma unroll
-    for (int i = 0; i < COV_MAX_RANK_SEL; ++i)
-      x[i] = (ok && i < r) ? __ldg(reinterpret_cast<const float4*>(base + (static_cast<size_t>(b) * r + i) * D))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-    float acc[G];
+    for (int j = 0; j < NBW; ++j) {
+      const int b = b0 + j * RPW + rg;
 #pragma unroll
-    for (int g = 0; g < G; ++g) acc[g] = 0.f;
-#pragma unroll
-    for (int i = 0; i < COV_MAX_RANK_SEL; ++i) {
-      if (i >= r) break;
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float d = qf[g].x * x[i].x;
-        d = fmaf(qf[g].y, x[i].y, d);
-        d = fmaf(qf[g].z, x[i].z, d);
-        d = fmaf(qf[g].w, x[i].w, d);
-#pragma unroll
-        for (int o = LPR / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL_MASK, d, o);
-        acc[g] = fmaf(d, d, acc[g]);
-      }
+      for (int i = 0; i < RMAX; ++i)
+        x[j][i] = (b < nbv && i < r)
+                      ? __ldg(reinterpret_cast<const float4*>(base + (static_cast<size_t>(b) * r + i) * D))
+                      : make_float4(0.f, 0.f, 0.f, 0.f);
     }
-    if (ok && (lane % LPR) == 0)
 #pragma unroll
-      for (int g = 0; g < G; ++g) lg[g * nbp + b] += 0.34657359027997264f * acc[g];  // ln 2 / 2
+    for (int j = 0; j < NBW; ++j) {
+      const int b = b0 + j * RPW + rg;
+      float acc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll
+      for (int i = 0; i < RMAX; ++i) {
+        if (i >= r) break;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float d = qf[g].x * x[j][i].x;
+          d = fmaf(qf[g].y, x[j][i].y, d);
+          d = fmaf(qf[g].z, x[j][i].z, d);
+          d = fmaf(qf[g].w, x[j][i].w, d);
+#pragma unroll
+          for (int o = LPR / 2; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL_MASK, d, o);
+          acc[g] = fmaf(d, d, acc[g]);
+        }
+      }
+      if (b < nbv && (lane % LPR) == 0)
+#pragma unroll
+        for (int g = 0; g < G; ++g) lg[g * nbp + b] += 0.34657359027997264f * acc[g];  // ln 2 / 2
+    }
   }
+}
+
+// The same second-order term for D = 128 streamed through the scorer's
+// lane-private cp.async ring (free once the first-order pass has drained it): a
+// batch is BPB = RSC / r whole blocks (RSC rows of 512 bytes a stage, a lane
+// holding its 16 bytes of each row), SEL_STAGES batches in flight per warp, the
+// warps taking batches in turn. Needs r <= RSC.
+template <int G, int RSC>
+__device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float4 (&qf)[G],
+                                       float4* ring) {
+  constexpr int D = 128;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = p.cobs_r;
+  const int bpb = RSC / r;
+  const int nbt = (nbv + bpb - 1) / bpb;
+  const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;
+  const float* base = p.k_xi + static_cast<size_t>(bh) * p.NBcap * r * D + lane * 4;
+  auto issue = [&](int m) {
+    const int st = m % SEL_STAGES;
+    const int b0 = (warp + m * SEL_NW) * bpb;
+#pragma unroll
+    for (int i = 0; i < RSC; ++i) {
+      const int blk = b0 + i / r, fac = i - (i / r) * r;
+      const bool ok = m < nmine && i < bpb * r && blk < nbv;
+      cp_async16(ring + (st * RSC + i) * SEL_THREADS + tid,
+                 base + (static_cast<size_t>(ok ? blk : 0) * r + (ok ? fac : 0)) * D, ok);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int m = 0; m < SEL_STAGES; ++m) issue(m);
+  for (int m = 0; m < nmine; ++m) {
+    cp_async_wait<SEL_STAGES - 1>();
+    const int st = m % SEL_STAGES;
+    const int b0 = (warp + m * SEL_NW) * bpb;
+    float4 xs[RSC];
+#pragma unroll
+    for (int i = 0; i < RSC; ++i) xs[i] = ring[(st * RSC + i) * SEL_THREADS + tid];
+    issue(m + SEL_STAGES);  // refill this stage (its values are in registers now)
+    for (int j = 0; j < bpb; ++j) {
+      float acc[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) acc[g] = 0.f;
+#pragma unroll
+      for (int i = 0; i < RSC; ++i) {
+        if (i < j * r || i >= (j + 1) * r) continue;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float d = qf[g].x * xs[i].x;
+          d = fmaf(qf[g].y, xs[i].y, d);
+          d = fmaf(qf[g].z, xs[i].z, d);
+          d = fmaf(qf[g].w, xs[i].w, d);
+#pragma unroll
+          for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL_MASK, d, o);
+          acc[g] = fmaf(d, d, acc[g]);
+        }
+      }
+      const int blk = b0 + j;
+      if (lane == 0 && blk < nbv)
+#pragma unroll
+        for (int g = 0; g < G; ++g) lg[g * nbp + blk] += 0.34657359027997264f * acc[g];  // ln 2 / 2
+    }
+  }
+  cp_async_wait<0>();
 }
 
 template <typename T, int D, int G, int MODE>
@@ -455,7 +527,20 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
     for (int g = 0; g < G; ++g)
       qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
                           load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
-    cobs_second_order<D, G>(p, lg, nbp, bh, nbv, qf);
+    constexpr int RSC = pow2ceil(G) >= 4 ? 32 / pow2ceil(G) : 8;  // ring rows a stage (sel_ring_bytes)
+    if constexpr (D == 128) {
+      if (p.cobs_r <= RSC) {
+        float4* ring = reinterpret_cast<float4*>(
+            sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
+        cobs_second_order_ring<G, RSC>(p, lg, nbp, bh, nbv, qf, ring);
+      } else {
+        cobs_second_order<D, G, 1, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qf);
+      }
+    } else if (p.cobs_r <= 4) {
+      cobs_second_order<D, G, 4, 4>(p, lg, nbp, bh, nbv, qf);
+    } else {
+      cobs_second_order<D, G, 1, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qf);
+    }
     __syncthreads();
   }
 
