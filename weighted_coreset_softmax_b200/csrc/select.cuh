@@ -468,29 +468,34 @@ __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, i
 #pragma unroll
     for (int i = 0; i < RSC; ++i) xs[i] = ring[(st * RSC + i) * SEL_THREADS + tid];
     issue(m + SEL_STAGES);  // refill this stage (its values are in registers now)
-    for (int j = 0; j < bpb; ++j) {
-      float acc[G];
+    // RSC rows x GP heads of partial dots, summed across the warp by halving
+    // exchanges (NV - 1 shuffles): lane c then holds value c / SPAN (row * GP + head)
+    constexpr int GP = pow2ceil(G);
+    constexpr int NV = RSC * GP;  // <= 32
+    constexpr int SPAN = 32 / NV;
+    float part[NV];
 #pragma unroll
-      for (int g = 0; g < G; ++g) acc[g] = 0.f;
+    for (int i = 0; i < RSC; ++i)
 #pragma unroll
-      for (int i = 0; i < RSC; ++i) {
-        if (i < j * r || i >= (j + 1) * r) continue;
-#pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float d = qf[g].x * xs[i].x;
+      for (int g = 0; g < GP; ++g) {
+        float d = 0.f;
+        if (g < G) {
+          d = qf[g].x * xs[i].x;
           d = fmaf(qf[g].y, xs[i].y, d);
           d = fmaf(qf[g].z, xs[i].z, d);
           d = fmaf(qf[g].w, xs[i].w, d);
-#pragma unroll
-          for (int o = 16; o >= 1; o >>= 1) d += __shfl_xor_sync(FULL_MASK, d, o);
-          acc[g] = fmaf(d, d, acc[g]);
         }
+        part[i * GP + g] = d;
       }
-      const int blk = b0 + j;
-      if (lane == 0 && blk < nbv)
-#pragma unroll
-        for (int g = 0; g < G; ++g) lg[g * nbp + blk] += 0.34657359027997264f * acc[g];  // ln 2 / 2
-    }
+    transpose_reduce<NV, 16>(part, lane);
+    const int vi = lane / SPAN;
+    const int row = vi / GP, g = vi - (vi / GP) * GP;
+    const float sq = part[0] * part[0];
+    float tot = sq;
+    for (int t = 1; t < r; ++t) tot += __shfl_down_sync(FULL_MASK, sq, t * GP * SPAN);  // the block's later rows
+    const int blk = b0 + row / r;
+    if ((lane % SPAN) == 0 && g < G && row % r == 0 && row < bpb * r && blk < nbv)
+      lg[g * nbp + blk] += 0.34657359027997264f * tot;  // ln 2 / 2
   }
   cp_async_wait<0>();
 }
