@@ -738,10 +738,16 @@ __global__ void __launch_bounds__(AttnCfg<T, D, G, MMA>::NTHREADS)
         int nw = 0;
 #pragma unroll
         for (int w = 0; w < C::NW; ++w)
-          if (wa[w] < wa[w + 1] && bh_of(wa[w]) == pbh) {
-            mbar_wait(ready + w, 0u, p.status);
-            recs[nw++] = reinterpret_cast<const float*>(smem + w * C::W_BYTES);
-          }
+          if (wa[w] < wa[w + 1] && bh_of(wa[w]) == pbh) recs[nw++] = reinterpret_cast<const float*>(smem + w * C::W_BYTES);
+        // a first pass of the merge over whatever the slots hold now, while the
+        // workers stream: it brings the merge's instructions into the SM's
+        // instruction cache off the critical path (the merge runs once a launch,
+        // so it would otherwise start cold); the merge after the waits rewrites
+        // every output this pass writes, in this thread
+        merge_local<D, G>(p, static_cast<int>(pbh), lane, recs, nw, vb, pm);
+#pragma unroll
+        for (int w = 0; w < C::NW; ++w)
+          if (wa[w] < wa[w + 1] && bh_of(wa[w]) == pbh) mbar_wait(ready + w, 0u, p.status);
         merge_local<D, G>(p, static_cast<int>(pbh), lane, recs, nw, vb, pm);
       }
     } else if (proxy) {
