@@ -52,6 +52,7 @@ struct SelParams {
 };
 
 // Shared memory beyond the dynamic arrays.
+constexpr int SEL_STAGES = 3;
 // k_top up to this takes the per-warp top-k path, larger k the radix select
 constexpr int SEL_TOPK = 16;
 constexpr int COV_MAX_RANK_SEL = 8;  // largest rank of the second-order factors
@@ -66,6 +67,7 @@ struct SelMisc {
   unsigned long long prefix, mask;
   int krem, digit, above, bucket;
   int wsum[SEL_NW];
+  unsigned long long rbar[SEL_NW][SEL_STAGES];  // scorer ring: one mbarrier per warp and stage
 };
 
 // Dynamic shared memory: lg[G][NBP] floats | key[NBP] u64 | misc; summary mode
@@ -93,7 +95,6 @@ __device__ __forceinline__ int sel_block_sum(int v, int* wsum) {
 // 16-byte pieces of a batch (one column chunk of RS rows) into a lane-private
 // three-stage ring with cp.async, so three batches per warp are in flight with
 // no register staging and no synchronisation between lanes.
-constexpr int SEL_STAGES = 3;
 __host__ __device__ inline size_t sel_ring_bytes(int G) {
   const int GP = G <= 1 ? 1 : (G <= 2 ? 2 : (G <= 4 ? 4 : 8));
   const int RS = GP >= 4 ? 32 / GP : 8;  // rows per lane per batch (D = 128; D = 64 needs fewer)
@@ -138,20 +139,31 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
   const int rg = lane / LPR, c = lane % LPR;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
   // four bytes per channel in either layout: fp32 sums, or (min, max) bf16 pairs
-  const float* ks = (QUEST ? static_cast<const float*>(p.k_bounds) : p.k_sum) + static_cast<size_t>(bh) * p.NBcap * D + c * 4;
+  const float* krows = (QUEST ? static_cast<const float*>(p.k_bounds) : p.k_sum) + static_cast<size_t>(bh) * p.NBcap * D;
   const int nbt = (nbv + BATCH - 1) / BATCH;               // batches of the bh
   const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;  // batches of this warp
-  // stage s, row i of this lane: ring[(s * RS + i) * SEL_THREADS + tid]
+  // The ring is filled by bulk copies with an L2 evict-first policy (the rows are
+  // read once a step; they should not push the next kernels' code and data out
+  // of L2). Stage s, slot i of a warp is 512 contiguous bytes -- rows
+  // rb + i * RPW .. + RPW - 1 -- at ring[(s * RS + i) * SEL_THREADS + warp * 32],
+  // so lane (rg, c) finds its 16 bytes where its own copy would have put them.
+  // Completion is counted in bytes on the warp's mbarrier of the stage.
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(ms.rbar[warp]);
+  const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int m) {
+    if (m >= nmine) return;  // warp-uniform
     const int st = m % SEL_STAGES;
     const int rb = (warp + m * SEL_NW) * BATCH;
-#pragma unroll
-    for (int i = 0; i < RS; ++i) {
-      const int row = rb + i * RPW + rg;
-      cp_async16(ring + (st * RS + i) * SEL_THREADS + tid, ks + static_cast<size_t>(row < nbv ? row : 0) * D,
-                 m < nmine && row < nbv);
+    const int nvalid = min(BATCH, nbv - rb);  // >= 1: batch rb starts below nbv
+    if (lane == 0) mbar_arrive_expect_tx(rbar + st, static_cast<uint32_t>(nvalid) * D * 4);
+    __syncwarp();
+    if (lane < RS) {
+      const int r0 = rb + lane * RPW;
+      const int nr = min(RPW, nbv - r0);
+      if (nr > 0)
+        bulk_g2s(ring + (st * RS + lane) * SEL_THREADS + warp * 32, krows + static_cast<size_t>(r0) * D,
+                 static_cast<uint32_t>(nr) * D * 4, rbar + st, pol);
     }
-    cp_async_commit();  // one group per batch slot, empty or not: the waits count groups
   };
 #pragma unroll
   for (int m = 0; m < SEL_STAGES; ++m) issue(m);
@@ -189,8 +201,10 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     os[j] = 0.f;
   }
   for (int m = 0; m < nmine; ++m) {
-    cp_async_wait<SEL_STAGES - 1>();  // batch m has landed (this lane's pieces)
     const int st = m % SEL_STAGES;
+    if (!mbar_wait(rbar + st, static_cast<uint32_t>((m / SEL_STAGES) & 1), nullptr))
+      mbar_wait(rbar + st, static_cast<uint32_t>((m / SEL_STAGES) & 1), nullptr);  // bounded: let a late copy land
+
     const int rb = (warp + m * SEL_NW) * BATCH;
     float part[NV];
 #pragma unroll
@@ -232,7 +246,11 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
         }
       }
     }
-    issue(m + SEL_STAGES);  // refill this stage (its values are in registers now)
+    // refill this stage: its values are in registers now; order those reads before
+    // the copies that overwrite the slots
+    __syncwarp();
+    fence_proxy_async_smem();
+    issue(m + SEL_STAGES);
     transpose_reduce<NV, LPR / 2>(part, lane);
 #pragma unroll
     for (int j = 0; j < HV::NH; ++j) {
@@ -259,7 +277,7 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
       }
     }
   }
-  cp_async_wait<0>();  // nothing may still be writing the ring when the CTA moves on
+  // every copy issued was waited for above (batches m >= nmine issue none)
   // merge the pairs of the lanes that hold the same head (every lane bit that
   // changes the row), then one lane per head writes this warp's pair
 #pragma unroll
@@ -516,6 +534,15 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int nbv = (n + p.L - 1) / p.L;
 
   if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS) {
+    // the scorer ring's mbarriers (one per warp and stage)
+    if (tid == 0) {
+#pragma unroll
+      for (int w = 0; w < SEL_NW; ++w)
+#pragma unroll
+        for (int st = 0; st < SEL_STAGES; ++st) mbar_init(reinterpret_cast<uint64_t*>(&ms.rbar[w][st]), 1);
+      fence_mbar_init();
+    }
+    __syncthreads();
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
     score_summary<T, D, G, MODE == SEL_QUEST>(p, lg, nbp, bh, nbv, ring, cnt, ms);
