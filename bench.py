@@ -158,10 +158,10 @@ class ClockSampler:
 
 
 # DRAM bytes per launch from the committed ncu capture
-# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.417 MB read, 0 written at B=8,
+# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.416 MB read, 0 written at B=8,
 # scaled x4 by sequences to the B=32 launch). Keyed by (kernel, workload, budget, B);
 # to be re-taken whenever the kernel changes.
-NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_417_344}
+NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_415_808}
 
 
 def measured_peak_hbm():
