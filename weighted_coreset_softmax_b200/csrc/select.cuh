@@ -449,43 +449,49 @@ __device__ void cobs_second_order(const SelParams& p, float* lg, int nbp, int bh
   }
 }
 
-// The same second-order term for D = 128 streamed through the scorer's
-// lane-private cp.async ring (free once the first-order pass has drained it): a
-// batch is BPB = RSC / r whole blocks (RSC rows of 512 bytes a stage, a lane
-// holding its 16 bytes of each row), SEL_STAGES batches in flight per warp, the
-// warps taking batches in turn. Needs r <= RSC.
+// The same second-order term for D = 128 streamed through the scorer's ring (free
+// once the first-order pass has drained it), filled the same way: one 512-byte
+// bulk copy per slot with an L2 evict-first policy, completion counted on the
+// warp's mbarrier of the stage (re-initialised after the first pass). A batch is
+// BPB = RSC / r whole blocks (RSC rows a stage, consecutive in memory), SEL_STAGES
+// batches in flight per warp, the warps taking batches in turn. Needs r <= RSC.
 template <int G, int RSC>
 __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float4 (&qf)[G],
-                                       float4* ring) {
+                                       float4* ring, uint64_t* rbar) {
   constexpr int D = 128;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int r = p.cobs_r;
   const int bpb = RSC / r;
   const int nbt = (nbv + bpb - 1) / bpb;
   const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;
-  const float* base = p.k_xi + static_cast<size_t>(bh) * p.NBcap * r * D + lane * 4;
+  const float* base = p.k_xi + static_cast<size_t>(bh) * p.NBcap * r * D;
+  const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int m) {
+    if (m >= nmine) return;  // warp-uniform
     const int st = m % SEL_STAGES;
     const int b0 = (warp + m * SEL_NW) * bpb;
-#pragma unroll
-    for (int i = 0; i < RSC; ++i) {
-      const int blk = b0 + i / r, fac = i - (i / r) * r;
-      const bool ok = m < nmine && i < bpb * r && blk < nbv;
-      cp_async16(ring + (st * RSC + i) * SEL_THREADS + tid,
-                 base + (static_cast<size_t>(ok ? blk : 0) * r + (ok ? fac : 0)) * D, ok);
-    }
-    cp_async_commit();
+    const int nrows = min(bpb, nbv - b0) * r;  // >= r: batch b0 starts below nbv
+    if (lane == 0) mbar_arrive_expect_tx(rbar + st, static_cast<uint32_t>(nrows) * D * 4);
+    __syncwarp();
+    if (lane < nrows)  // row `lane` of the batch: factor lane % r of block b0 + lane / r
+      bulk_g2s(ring + (st * RSC + lane) * SEL_THREADS + warp * 32, base + (static_cast<size_t>(b0) * r + lane) * D,
+               D * 4, rbar + st, pol);
   };
 #pragma unroll
   for (int m = 0; m < SEL_STAGES; ++m) issue(m);
   for (int m = 0; m < nmine; ++m) {
-    cp_async_wait<SEL_STAGES - 1>();
     const int st = m % SEL_STAGES;
+    if (!mbar_wait(rbar + st, static_cast<uint32_t>((m / SEL_STAGES) & 1), nullptr))
+      mbar_wait(rbar + st, static_cast<uint32_t>((m / SEL_STAGES) & 1), nullptr);  // bounded: let a late copy land
     const int b0 = (warp + m * SEL_NW) * bpb;
     float4 xs[RSC];
 #pragma unroll
     for (int i = 0; i < RSC; ++i) xs[i] = ring[(st * RSC + i) * SEL_THREADS + tid];
-    issue(m + SEL_STAGES);  // refill this stage (its values are in registers now)
+    // refill this stage: its values are in registers now; order those reads before
+    // the copies that overwrite the slots
+    __syncwarp();
+    fence_proxy_async_smem();
+    issue(m + SEL_STAGES);
     // RSC rows x GP heads of partial dots, summed across the warp by halving
     // exchanges (NV - 1 shuffles): lane c then holds value c / SPAN (row * GP + head)
     constexpr int GP = pow2ceil(G);
@@ -515,7 +521,7 @@ __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, i
     if ((lane % SPAN) == 0 && g < G && row % r == 0 && row < bpb * r && blk < nbv)
       lg[g * nbp + blk] += 0.34657359027997264f * tot;  // ln 2 / 2
   }
-  cp_async_wait<0>();
+  // every copy issued was waited for above (batches m >= nmine issue none)
 }
 
 template <typename T, int D, int G, int MODE>
@@ -564,7 +570,19 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
       if (p.cobs_r <= RSC) {
         float4* ring = reinterpret_cast<float4*>(
             sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-        cobs_second_order_ring<G, RSC>(p, lg, nbp, bh, nbv, qf, ring);
+        // fresh ring barriers: the first pass left them at different phases
+        if (tid == 0) {
+#pragma unroll
+          for (int w = 0; w < SEL_NW; ++w)
+#pragma unroll
+            for (int st = 0; st < SEL_STAGES; ++st) {
+              mbar_inval(reinterpret_cast<uint64_t*>(&ms.rbar[w][st]));
+              mbar_init(reinterpret_cast<uint64_t*>(&ms.rbar[w][st]), 1);
+            }
+          fence_mbar_init();
+        }
+        __syncthreads();
+        cobs_second_order_ring<G, RSC>(p, lg, nbp, bh, nbv, qf, ring, reinterpret_cast<uint64_t*>(ms.rbar[warp]));
       } else {
         cobs_second_order<D, G, 1, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qf);
       }
