@@ -1,0 +1,178 @@
+"""Host-side checks of the index arithmetic of the selector and covariance kernels,
+restated from their sources: every row is copied exactly once and inside its buffer,
+every byte count matches the copies it announces, the Jacobi rotation schedule is
+a round-robin tournament, and the covariance kernel's shared-memory carve-up is
+aligned and inside its allocation. No GPU is needed."""
+from __future__ import annotations
+
+import itertools
+
+import pytest
+
+SEL_THREADS = 256
+SEL_NW = SEL_THREADS // 32
+SEL_STAGES = 3
+
+
+def pow2ceil(x):
+    p = 1
+    while p < x:
+        p *= 2
+    return p
+
+
+def ring_rows_per_stage(G):
+    """sel_ring_bytes: rows (512-byte slots) a warp holds per stage."""
+    GP = pow2ceil(G)
+    return 32 // GP if GP >= 4 else 8
+
+
+# ------------------------------------------------------------ Jacobi schedule
+def circle_pairs(m, rnd):
+    """Pairs of one round of the covariance kernel's schedule (thread t < m/2)."""
+    out = []
+    for t in range(m // 2):
+        a, b = t, m - 1 - t
+        p = 0 if a == 0 else 1 + (a - 1 + rnd) % (m - 1)
+        q = 1 + (b - 1 + rnd) % (m - 1)
+        out.append((min(p, q), max(p, q)))
+    return out
+
+
+@pytest.mark.parametrize("m", [2, 4, 6, 16, 32, 64])
+def test_jacobi_round_robin(m):
+    seen = []
+    for rnd in range(m - 1):
+        pairs = circle_pairs(m, rnd)
+        flat = [i for pq in pairs for i in pq]
+        assert sorted(flat) == list(range(m)), f"round {rnd}: pairs not disjoint / not covering"
+        assert all(p != q for p, q in pairs)
+        seen += pairs
+    assert sorted(seen) == sorted(itertools.combinations(range(m), 2)), "a pair missing or repeated in a sweep"
+
+
+# ------------------------------------------------------------ scorer ring
+def scorer_copies(D, G, nbv):
+    """The first-order scorer's bulk copies: (warp, m, slot, first row, rows) and the
+    bytes each (warp, m) announces."""
+    LPR = D // 4
+    RPW = 32 // LPR
+    GP = pow2ceil(G)
+    RS = min(8, max(1, LPR // GP))
+    BATCH = RPW * RS
+    nbt = (nbv + BATCH - 1) // BATCH
+    copies, announced = [], {}
+    for warp in range(SEL_NW):
+        nmine = (nbt - warp + SEL_NW - 1) // SEL_NW if nbt > warp else 0
+        for m in range(nmine):
+            rb = (warp + m * SEL_NW) * BATCH
+            nvalid = min(BATCH, nbv - rb)
+            assert nvalid >= 1
+            announced[(warp, m)] = nvalid * D * 4
+            got = 0
+            for lane in range(RS):
+                r0 = rb + lane * RPW
+                nr = min(RPW, nbv - r0)
+                if nr > 0:
+                    copies.append((warp, m, lane, r0, nr))
+                    got += nr * D * 4
+            assert got == announced[(warp, m)], "expect_tx differs from the bytes copied"
+    return copies, RS
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 7, 8])
+@pytest.mark.parametrize("nbv", [0, 1, 7, 8, 9, 63, 64, 65, 512, 1031])
+def test_scorer_ring_covers_rows_once(D, G, nbv):
+    copies, RS = scorer_copies(D, G, nbv)
+    rows = sorted(r for (_, _, _, r0, nr) in copies for r in range(r0, r0 + nr))
+    assert rows == list(range(nbv))
+    assert RS <= ring_rows_per_stage(G), "stage rows exceed the ring's allocation"
+    for (warp, m, slot, r0, nr) in copies:
+        assert nr * D * 4 <= 512, "a copy larger than its 512-byte slot"
+        f4 = ((m % SEL_STAGES) * RS + slot) * SEL_THREADS + warp * 32  # float4 index of the slot
+        assert f4 + 32 <= SEL_STAGES * ring_rows_per_stage(G) * SEL_THREADS
+
+
+# ------------------------------------------------------------ second-order ring
+def cobs_copies(G, r, nbv):
+    RSC = ring_rows_per_stage(G)
+    assert r <= RSC
+    bpb = RSC // r
+    nbt = (nbv + bpb - 1) // bpb
+    out = []
+    for warp in range(SEL_NW):
+        nmine = (nbt - warp + SEL_NW - 1) // SEL_NW if nbt > warp else 0
+        for m in range(nmine):
+            b0 = (warp + m * SEL_NW) * bpb
+            nrows = min(bpb, nbv - b0) * r
+            assert nrows >= r
+            for lane in range(nrows):
+                row = b0 * r + lane  # factor lane % r of block b0 + lane // r
+                out.append((warp, m, lane, row))
+            assert nrows <= RSC
+    return out, RSC
+
+
+@pytest.mark.parametrize("G", [1, 2, 4, 7, 8])
+@pytest.mark.parametrize("r", [1, 2, 3, 4, 8])
+@pytest.mark.parametrize("nbv", [1, 5, 64, 513])
+def test_cobs_ring_covers_factor_rows_once(G, r, nbv):
+    if r > ring_rows_per_stage(G):
+        pytest.skip("this rank takes the direct-load path")
+    copies, RSC = cobs_copies(G, r, nbv)
+    rows = sorted(row for (_, _, _, row) in copies)
+    assert rows == list(range(nbv * r))
+    for (warp, m, lane, row) in copies:
+        f4 = ((m % SEL_STAGES) * RSC + lane) * SEL_THREADS + warp * 32
+        assert f4 + 32 <= SEL_STAGES * RSC * SEL_THREADS
+
+
+def test_cobs_leaders_sum_whole_blocks():
+    # after the transpose reduction lane c holds value c / SPAN = row * GP + head; a
+    # leader (first row of a block) adds the values r - 1 ... shifts above it, which
+    # must be the same head's later rows of the same block, inside the warp
+    for G in (1, 2, 3, 4, 5, 7, 8):
+        GP = pow2ceil(G)
+        RSC = ring_rows_per_stage(G)
+        NV = RSC * GP
+        SPAN = 32 // NV
+        for r in range(1, RSC + 1):
+            bpb = RSC // r
+            for lane in range(32):
+                vi = lane // SPAN
+                row, g = divmod(vi, GP)
+                if lane % SPAN or g >= G or row % r or row >= bpb * r:
+                    continue
+                for t in range(1, r):
+                    src = lane + t * GP * SPAN
+                    assert src < 32
+                    vs = src // SPAN
+                    assert vs % GP == g and vs // GP == row + t and (row + t) // r == row // r
+
+
+# ------------------------------------------------------------ covariance smem
+def cov_layout(L, D):
+    m = (L + 1) & ~1
+    kx = L * (D + 1) * 4
+    mean = (kx + 15) & ~15
+    A = mean + D * 8
+    V = A + m * (m + 1) * 8
+    rot = V + m * (m + 1) * 8
+    pr = rot + (m // 2) * 16
+    red = pr + (m // 2) * 8
+    sel = red + 32 * 8
+    end = sel + 8 * 4
+    total = ((L * (D + 1) * 4 + 15) & ~15) + D * 8 + 2 * m * (m + 1) * 8 + (m // 2) * 16 + (m // 2) * 8 + 64 * 8
+    return dict(mean=mean, A=A, V=V, rot=rot, pr=pr, red=red, sel=sel, end=end, total=total)
+
+
+@pytest.mark.parametrize("L", [16, 32, 64])
+@pytest.mark.parametrize("D", [64, 128])
+def test_cov_smem_layout(L, D):
+    o = cov_layout(L, D)
+    for k in ("mean", "A", "V", "red"):
+        assert o[k] % 8 == 0, k
+    assert o["rot"] % 16 == 0, "double2 rotations need 16-byte alignment"
+    assert o["end"] <= o["total"], "carve-up runs past the allocation"
+    assert o["total"] <= 227 * 1024
