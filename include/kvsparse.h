@@ -140,6 +140,44 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale,
                            kv_stream_t stream);
 
 /*
+ * kv_build_block_key_means -- the block mean keys at bf16 precision, the block
+ * summary COBS stores for first-order scoring. Source: "COBS: Cumulant Order
+ * Block Sparse Attention", the quantisation paragraph (the block mean is kept at
+ * bf16 precision) and the mean-pool score after Equation (8).
+ *
+ *   k_sum   device [B][Hkv][NBcap][D] fp32 key sums (kv_build_block_summaries)
+ *   counts  device [B][NBcap] int32 token counts (same call)
+ *   k_mean  device out [B][Hkv][NBcap][D] bf16, 16-byte aligned: the correctly
+ *           rounded fp32 quotient k_sum / n_b rounded to the nearest bf16 (ties
+ *           to even); zeros where n_b = 0.
+ * Half the bytes of the fp32 sums for the scorer to stream. Run once after
+ * prefill (after kv_build_block_summaries, on the same stream).
+ */
+kv_status kv_build_block_key_means(const kv_shape* shape, const float* k_sum, const int32_t* counts,
+                                   void* k_mean, kv_stream_t stream);
+
+/*
+ * kv_select_blocks_mean16 -- kv_select_blocks (summary mode) scoring from the
+ * bf16 block means instead of the fp32 sums. Source: "COBS: Cumulant Order Block
+ * Sparse Attention", text after Equation (8), Equation (5), the quantisation
+ * paragraph:
+ *
+ *   s[g,b] = scale * q_g . k_mean_b + ln n_b        (k_mean_b the bf16 mean)
+ *   S[b]   = sum_{g in group} exp(s[g,b] - ln sum_b' exp(s[g,b']))  over valid b'
+ *
+ * Reads NBcap * (2 D + 4) bytes per (sequence, KV head) instead of
+ * NBcap * (4 D + 4). The rounding of the mean moves each logit by at most
+ * scale * sum_d |q_d| |mean_d| 2^-8, so the kept set can differ from the
+ * fp32-sum ranking where two candidates score that close. Forcing, ranking,
+ * kmax, block_idx, n_kept and scores are as in kv_select_blocks. bf16 caches only
+ * (KV_ERR_UNSUPPORTED otherwise).
+ */
+kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float scale, const void* k_mean,
+                                  const int32_t* counts, int k_top, int force_first, int force_last,
+                                  int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
+                                  kv_stream_t stream);
+
+/*
  * kv_build_block_bounds -- per-block, per-channel key minimum and maximum (the
  * axis-aligned bounding box of each block's keys). Source: "COBS: Cumulant Order
  * Block Sparse Attention", the Quest paragraph (a block is scored by the largest
@@ -325,8 +363,9 @@ kv_status kv_workspace_status(const void* workspace, uint32_t* status_out, kv_st
  * the scratch comes from a fixed 16 MiB array inside the library (held on every
  * GPU that loads it, until exit). Shapes whose kv_workspace_bytes exceeds 16 MiB
  * are rejected with KV_ERR_INVALID_ARG. The first call on a device looks up the
- * array's device address (make it before any stream capture). Each call clears
- * the array's counters with an async memset on `stream`; calls share the array,
+ * array's device address (make it before any stream capture). Each call checks
+ * every argument first (a rejected call enqueues nothing), then clears the
+ * array's counters with an async memset on `stream`; calls share the array,
  * so calls that overlap on the GPU race -- order them on one stream or with
  * events. Nothing is allocated. Device-check status bits are not reported.
  */
@@ -338,6 +377,27 @@ kv_status kv_sparse_decode_attn_noalloc(const kv_shape* shape, const void* q, fl
                                         const float* v_tot, int use_tail_proxy,
                                         const int32_t* tok_idx, const float* w, int m,
                                         float* out, float* lse, kv_stream_t stream);
+
+/*
+ * kv_selftest_wait_timeout -- checks the kernels' failure detection on the
+ * device without a fault. The pages have no counterpart: every wait of the
+ * kernels on a copy is bounded, and one that runs out sets KV_DEV_WAIT_TIMEOUT
+ * in the status word and returns instead of hanging; this call runs that same
+ * bounded wait in a one-warp kernel.
+ *
+ *   status     device uint32, 4-byte aligned: KV_DEV_WAIT_TIMEOUT is OR-ed in
+ *              when the wait gives up (other bits untouched).
+ *   waited_ok  device uint32, 4-byte aligned: set to 1 if the wait completed,
+ *              0 if it gave up.
+ *   limit_ns   the wait's limit, 0 < limit_ns <= 2e9 (wall time, %globaltimer).
+ *   arrive     nonzero: the barrier's phase completes (an arrival with no bytes
+ *              expected) and the wait succeeds; zero: the phase expects 16 bytes
+ *              that no copy delivers (none is issued), so the wait runs out.
+ *
+ * Asynchronous on `stream`; KV_ERR_INVALID_ARG for bad pointers or limits.
+ */
+kv_status kv_selftest_wait_timeout(uint32_t* status, uint32_t* waited_ok, uint64_t limit_ns, int arrive,
+                                   kv_stream_t stream);
 
 /* Message of the last failed call on this host thread ("" if none). */
 const char* kv_last_error(void);

@@ -55,6 +55,9 @@ notes of the repository):
       sigma q.mean + (sigma^2 / 2) q^T Sigma_r q + ln n_b, with Sigma_r = sum of the
       top r xi_i xi_i^T, is the block logit in the Equation 5 group score. The
       full-space factors are used (no query subspace, no FP4 quantisation).
+  R13 bf16 block means: the mean key is rounded to the nearest bfloat16 value
+      (ties to even) and used in place of the exact mean in the first-order
+      score; everything else as in R1 to R6.
 """
 from __future__ import annotations
 
@@ -199,6 +202,53 @@ def summary_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, sigma:
         if nb <= 0:
             continue
         mean_key = k_sum[b] / nb
+        out[:, b] = sigma * (qg @ mean_key) + math.log(nb)
+    return out
+
+
+def round_bf16(x) -> np.ndarray:
+    """Nearest bfloat16 value of each float64 (8 significant bits, ties to even):
+    the precision at which COBS keeps the block mean [COBS, the quantisation
+    paragraph: one fp32 scale per eigenvector and the block mean at bf16].
+
+    Written from the definition: with |x| in [2^e, 2^(e+1)) the bf16 grid has
+    spacing 2^(e-7) (2^-133 below 2^-126, the subnormal range); x / spacing is
+    rounded to the nearest integer, ties to even, and scaled back (both scalings
+    by a power of two are exact in float64). Values past the largest finite bf16
+    become +-inf.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    out = np.array(x, dtype=np.float64, copy=True)
+    fin = np.isfinite(x) & (x != 0)
+    if np.any(fin):
+        _, E = np.frexp(x[fin])                  # |x| = m 2^E, m in [0.5, 1)
+        e = np.maximum(E - 1, -126)              # binade exponent, subnormals share -126
+        spacing = np.ldexp(1.0, e - 7)
+        r = np.rint(x[fin] / spacing) * spacing  # np.rint: round half to even
+        r[np.abs(r) > BF16_MAX] = np.inf * np.sign(r[np.abs(r) > BF16_MAX])
+        out[fin] = r
+    return out
+
+
+BF16_MAX = float((2.0 - 2.0 ** -7) * 2.0 ** 127)
+
+
+def summary_mean16_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, sigma: float):
+    """The first-order mean-pool estimate with the block mean stored at bf16
+    precision [COBS, text after Equation (8) and the quantisation paragraph]:
+
+        s_hat[g, b] = sigma * q_g . bf16(k_sum_b / n_b) + ln n_b
+
+    Blocks with n_b = 0 get -inf.
+    """
+    G = qg.shape[0]
+    NB = k_sum.shape[0]
+    out = np.full((G, NB), -math.inf)
+    for b in range(NB):
+        nb = int(counts[b])
+        if nb <= 0:
+            continue
+        mean_key = round_bf16(k_sum[b] / nb)
         out[:, b] = sigma * (qg @ mean_key) + math.log(nb)
     return out
 
@@ -374,12 +424,13 @@ def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
         n = int(seq_lens[b])
         nb = (n + L - 1) // L
         qg = q[b, h * G:(h + 1) * G]
-        if mode == "summary":
+        if mode in ("summary", "summary_mean16"):
             if k_sum is None:
                 ks, _, c, _, _ = block_summaries_one(K[b, h], K[b, h], n, L, NBcap)
             else:
                 ks, c = k_sum[b, h], counts[b]
-            shat = summary_logits(qg, ks[:nb], c[:nb], sigma)
+            fn = summary_logits if mode == "summary" else summary_mean16_logits
+            shat = fn(qg, ks[:nb], c[:nb], sigma)
         elif mode == "exact_mass":
             shat = exact_log_mass(qg, K[b, h], n, L, nb, sigma)
         elif mode == "quest":

@@ -51,9 +51,28 @@ def check_out(got_out, got_lse, ref_out, ref_lse, rows=None, tol=OUT_TOL, what="
     return err
 
 
+# Near ties seen by the selection checks of this session: (label, pairs checked,
+# pairs the oracle flags as a near tie, pairs whose kept set differs there). The
+# session summary (tests/conftest.py) prints them.
+NEAR_TIES = []
+
+
+def record_near_ties(what, n_pairs, n_flagged, n_mismatch):
+    NEAR_TIES.append((what, int(n_pairs), int(n_flagged), int(n_mismatch)))
+
+
+# Other figures a test reports rather than asserts (printed in the session summary).
+NOTES = []
+
+
+def record_note(text):
+    NOTES.append(str(text))
+
+
 def selection_matches(gpu_idx, gpu_nk, sel_ref, pairs, what=""):
     """Kept sets must be bit-exact unless the oracle flags a near tie at the k / k+1
-    boundary; returns the number of near-tie pairs where they differ."""
+    boundary; returns the number of near-tie pairs where they differ (also
+    recorded for the session's near-tie report)."""
     gi = gpu_idx.cpu().numpy()
     gn = gpu_nk.cpu().numpy()
     ties = 0
@@ -64,6 +83,7 @@ def selection_matches(gpu_idx, gpu_nk, sel_ref, pairs, what=""):
         if got != ref["kept"]:
             assert ref["near_tie"], f"{what}: kept {got} != oracle {ref['kept']} at {(b, h)} (no near tie)"
             ties += 1
+    record_near_ties(what, len(pairs), sum(1 for p in pairs if sel_ref[p]["near_tie"]), ties)
     return ties
 
 
@@ -84,6 +104,11 @@ def run_pipeline(wl, *, want_scores=True, use_proxy=True, kmax=None):
         idx, nk, scores = kv.kv_select_blocks_cobs(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_sum"],
                                                    summ["counts"], summ["k_xi"], wl.k_top, wl.force_first,
                                                    wl.force_last, kmax=kmax, want_scores=want_scores)
+    elif wl.score_mode == "summary_mean16":
+        summ["k_mean"] = kv.kv_build_block_key_means(wl.K, sl, wl.block_size, summ["k_sum"], summ["counts"])
+        idx, nk, scores = kv.kv_select_blocks_mean16(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_mean"],
+                                                     summ["counts"], wl.k_top, wl.force_first, wl.force_last,
+                                                     kmax=kmax, want_scores=want_scores)
     elif wl.score_mode == "quest":
         summ["k_bounds"] = kv.kv_build_block_bounds(wl.K, sl, wl.block_size)
         idx, nk, scores = kv.kv_select_blocks_quest(wl.q, wl.K, sl, wl.block_size, wl.scale, summ["k_bounds"],

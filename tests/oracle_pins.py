@@ -528,6 +528,84 @@ def pin_cobs_eigen_structure(seed=20):
             _close(float(np.sum(X[:, a] * X[:, b2])), ca, 1e-11, what="sum of xi xi^T = covariance")
 
 
+def _bf16_bits(x: float) -> int:
+    """Upper 16 bits of the float32 encoding of x (x must be a float32 value)."""
+    import struct
+    return struct.unpack("<I", struct.pack("<f", x))[0] >> 16
+
+
+def _bf16_value(bits: int) -> float:
+    import struct
+    return struct.unpack("<f", struct.pack("<I", (bits & 0xffff) << 16))[0]
+
+
+def pin_round_bf16_nearest_even(seed=21):
+    """round_bf16 against a brute-force search over the bf16 grid: the result is a
+    bf16 value, no bf16 value is nearer, and of two equally near ones the even
+    encoding wins."""
+    r = _rng(seed)
+    xs = list(r.normal(size=300) * np.exp(r.uniform(-30, 30, size=300)))
+    # exact midpoints between neighbouring bf16 values (ties), both parities
+    for bits in (0x3f80, 0x3f81, 0x4049, 0x404a, 0xbf80, 0xc0a3, 0x0001, 0x0080):
+        lo, hi = _bf16_value(bits), _bf16_value(bits + 1)
+        xs.append((lo + hi) / 2)
+    xs += [0.0, 1.0, -2.5, 3.0e38, 1e-40]
+    got = O.round_bf16(np.array(xs))
+    for x, g in zip(xs, got):
+        if x == 0.0:
+            assert g == 0.0
+            continue
+        if abs(x) > O.BF16_MAX * (1 + 2.0 ** -9):
+            assert math.isinf(g)
+            continue
+        g32 = float(np.float32(g))
+        assert g32 == g, f"{x!r}: {g!r} is not a float32 value"
+        b = _bf16_bits(g32)
+        assert _bf16_value(b) == g, f"{x!r}: {g!r} is not a bf16 value"
+        # neighbours on the grid (same sign): none nearer, ties to the even code
+        for nb in (b - 1, b + 1):
+            if (nb & 0x7fff) in (0x7f80,) or nb < 0 or nb > 0xffff or (nb ^ b) & 0x8000:
+                continue
+            v = _bf16_value(nb)
+            if math.isinf(v):
+                continue
+            dg, dv = abs(g - x), abs(v - x)
+            assert dg <= dv, f"{x!r}: {g!r} is not the nearest bf16 value ({v!r} is nearer)"
+            if dg == dv:
+                assert b % 2 == 0, f"{x!r}: tie not broken to the even code"
+
+
+def pin_mean16_score(seed=22):
+    """The bf16-mean score equals the exact-mean score when every block mean is a
+    bf16 value, and otherwise differs by at most sigma * sum_j |q_j| |mean_j| 2^-8
+    (the relative rounding bound of an 8-bit significand)."""
+    r = _rng(seed)
+    G, D, L, NB = 3, 16, 4, 9
+    # keys on a coarse dyadic grid whose block sums divide exactly: means are bf16
+    K = np.round(r.normal(size=(NB * L, D)) * 4) / 4
+    counts = np.full(NB, L)
+    k_sum = K.reshape(NB, L, D).sum(axis=1)
+    means = k_sum / L
+    assert np.array_equal(O.round_bf16(means), means), "test means must be bf16 values"
+    qg = r.normal(size=(G, D))
+    _close(O.summary_mean16_logits(qg, k_sum, counts, 0.3), O.summary_logits(qg, k_sum, counts, 0.3),
+           1e-14, what="bf16-representable means")
+    # general keys: the bound, and the bound is not loose by orders of magnitude
+    K = r.normal(size=(NB * L, D)) * np.exp(r.normal(size=D))
+    counts = np.array([L] * (NB - 1) + [3])
+    k_sum = np.zeros((NB, D))
+    for b in range(NB):
+        k_sum[b] = K[b * L:b * L + counts[b]].sum(axis=0)
+    a = O.summary_mean16_logits(qg, k_sum, counts, 0.3)
+    e = O.summary_logits(qg, k_sum, counts, 0.3)
+    for b in range(NB):
+        mean = k_sum[b] / counts[b]
+        for g in range(G):
+            bound = 0.3 * float(np.sum(np.abs(qg[g]) * np.abs(mean))) * 2.0 ** -8
+            assert abs(a[g, b] - e[g, b]) <= bound * (1 + 1e-12), (b, g)
+    assert np.max(np.abs(a - e)) > 0, "rounding must change some score"
+
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -536,5 +614,5 @@ ALL_PINS = [
     pin_topk_bruteforce, pin_near_tie_flag, pin_worked_example, pin_empty_inputs,
     pin_summary_equals_exact_for_constant_blocks, pin_quest_box_corners, pin_quest_upper_bound,
     pin_cobs_full_rank_is_exact_quadratic, pin_cobs_rank_one_block, pin_cobs_two_point_closed_form,
-    pin_cobs_error_order, pin_cobs_eigen_structure,
+    pin_cobs_error_order, pin_cobs_eigen_structure, pin_round_bf16_nearest_even, pin_mean16_score,
 ]

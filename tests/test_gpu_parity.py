@@ -331,75 +331,3 @@ def test_deterministic_repeat():
     b = run_pipeline(wl)
     assert torch.equal(a["idx"], b["idx"]) and torch.equal(a["out"], b["out"])
     assert torch.equal(a["summ"]["k_tot"], b["summ"]["k_tot"])
-
-
-# ------------------------------------------------------ full-size, sampled
-FULL = [
-    ("llama", dict(budget=0.01)),
-    ("llama", dict(budget=0.05)),
-    ("qwen_long", dict(budget=0.01)),
-    ("llama_osa", dict()),
-]
-
-
-@pytest.mark.parametrize("name,kw", FULL)
-def test_full_size_sampled(name, kw):
-    wl = W.make(name, DEV, **kw)
-    r = run_pipeline(wl)
-    gen = np.random.default_rng(7)
-    pairs = sorted({(int(gen.integers(wl.B)), int(gen.integers(wl.Hkv))) for _ in range(3)}
-                   | {(0, 0), (wl.B - 1, wl.Hkv - 1)})
-    q = to64(wl.q)
-    K = {}
-    res_sel, res_out = {}, {}
-    for (b, h) in pairs:
-        Kb = to64(wl.K[b:b + 1, h:h + 1])
-        Vb = to64(wl.V[b:b + 1, h:h + 1])
-        qb = q[b:b + 1, h * wl.G:(h + 1) * wl.G]
-        sel = O.select_batch(qb, Kb, [wl.seq_lens[b]], wl.block_size, wl.scale, wl.k_top,
-                             True, True, wl.score_mode)
-        res_sel[(b, h)] = sel[(0, 0)]
-        gi = r["idx"][b, h, :int(r["nk"][b, h])].cpu().tolist()
-        o, l, _ = O.sparse_attend_one(qb[0], Kb[0, 0], Vb[0, 0], wl.seq_lens[b], wl.block_size,
-                                      gi, wl.scale, True)
-        res_out[(b, h)] = (o, l)
-    selection_matches(r["idx"], r["nk"], res_sel, pairs, f"full {name} select")
-    go = r["out"].cpu().numpy().astype(np.float64)
-    gl = r["lse"].cpu().numpy().astype(np.float64)
-    for (b, h), (o, l) in res_out.items():
-        sl_ = slice(h * wl.G, (h + 1) * wl.G)
-        err = row_rel_err(go[b, sl_], o)
-        assert err <= OUT_TOL, f"full {name} {(b, h)}: {err:.3e}"
-        assert np.max(np.abs(gl[b, sl_] - l)) <= OUT_TOL * max(1.0, float(np.max(np.abs(l))))
-
-
-def test_full_size_weighted_sampled():
-    wl = W.make("llama_coreset", DEV)
-    sl = wl.seq_lens_tensor(DEV)
-    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
-    out, lse = kv.kv_sparse_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws,
-                                        tok_idx=wl.tok_idx, w=wl.w)
-    torch.cuda.synchronize()
-    assert kv.kv_workspace_status(ws.tensor) == 0
-    q = to64(wl.q)
-    for (b, h) in [(0, 0), (13, 5), (31, 7)]:
-        qb = q[b, h * wl.G:(h + 1) * wl.G]
-        o, l = O.weighted_attend_one(qb, to64(wl.K[b, h]), to64(wl.V[b, h]), wl.seq_lens[b],
-                                     wl.tok_idx[b, h].cpu().numpy(),
-                                     wl.w[b, h].cpu().numpy().astype(np.float64), wl.scale)
-        err = row_rel_err(out[b, h * wl.G:(h + 1) * wl.G].cpu().numpy().astype(np.float64), o)
-        assert err <= OUT_TOL, err
-
-
-def test_full_size_dense_sampled():
-    wl = W.make("llama", DEV)
-    sl = wl.seq_lens_tensor(DEV)
-    ws = kv.Workspace(kv.make_shape(wl.q, wl.K, sl, wl.block_size), DEV)
-    out, lse = kv.kv_dense_decode_attn(wl.q, wl.K, wl.V, sl, wl.block_size, wl.scale, ws)
-    torch.cuda.synchronize()
-    q = to64(wl.q)
-    for (b, h) in [(0, 0), (17, 3), (31, 7)]:
-        qb = q[b, h * wl.G:(h + 1) * wl.G]
-        o, l = O.dense_attend_one(qb, to64(wl.K[b, h]), to64(wl.V[b, h]), wl.seq_lens[b], wl.scale)
-        err = row_rel_err(out[b, h * wl.G:(h + 1) * wl.G].cpu().numpy().astype(np.float64), o)
-        assert err <= OUT_TOL, err

@@ -38,6 +38,30 @@ def _mut_summary_sum_not_mean(orig):
     return f
 
 
+def _mut_round_bf16_truncate(orig):
+    def f(x):
+        x = np.asarray(x, dtype=np.float64)
+        out = np.array(x, copy=True)
+        fin = np.isfinite(x) & (x != 0)
+        _, E = np.frexp(x[fin])
+        sp = np.ldexp(1.0, np.maximum(E - 1, -126) - 7)
+        out[fin] = np.trunc(x[fin] / sp) * sp
+        return out
+    return f
+
+
+def _mut_round_bf16_ties_up(orig):
+    def f(x):
+        x = np.asarray(x, dtype=np.float64)
+        out = np.array(x, copy=True)
+        fin = np.isfinite(x) & (x != 0)
+        _, E = np.frexp(x[fin])
+        sp = np.ldexp(1.0, np.maximum(E - 1, -126) - 7)
+        out[fin] = np.floor(x[fin] / sp + 0.5) * sp
+        return out
+    return f
+
+
 def _mut_group_score_logits(orig):
     def f(shat):
         return np.where(np.isfinite(shat), shat, 0.0).sum(axis=0)
@@ -154,6 +178,10 @@ MUTANTS = {
     "tail_proxy/sum not mean": ("tail_proxy", _mut_proxy_sum_value),
     "summary_logits/no ln n_b": ("summary_logits", _mut_summary_no_log),
     "summary_logits/sum not mean": ("summary_logits", _mut_summary_sum_not_mean),
+    "mean16/no ln n_b": ("summary_mean16_logits", _mut_summary_no_log),
+    "mean16/sum not mean": ("summary_mean16_logits", _mut_summary_sum_not_mean),
+    "round_bf16/truncates": ("round_bf16", _mut_round_bf16_truncate),
+    "round_bf16/ties up": ("round_bf16", _mut_round_bf16_ties_up),
     "group_score/sums logits": ("group_score", _mut_group_score_logits),
     "select_blocks/high-index ties": ("select_blocks", _mut_select_high_index),
     "exact_log_mass/max not lse": ("exact_log_mass", _mut_exact_mass_max),

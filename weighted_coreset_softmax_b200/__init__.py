@@ -27,9 +27,10 @@ __all__ = [
     "KV_BF16", "KV_F32", "KV_SCORE_SUMMARY", "KV_SCORE_EXACT_MASS", "KV_STEP_AUTO", "KV_STEP_TWO_KERNELS",
     "KV_STEP_FUSED", "KVShape", "KVError",
     "lib", "library_path", "header_path", "make_shape", "kv_build_block_summaries",
-    "kv_select_blocks", "kv_build_block_bounds", "kv_select_blocks_quest",
+    "kv_select_blocks", "kv_build_block_bounds", "kv_select_blocks_quest", "kv_build_block_key_means",
+    "kv_select_blocks_mean16",
     "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
-    "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace",
+    "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace", "kv_selftest_wait_timeout",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
@@ -83,6 +84,8 @@ def lib():
         "kv_build_block_summaries": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P],
         "kv_select_blocks": [_SHP, _P, _F, _I, _P, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_build_block_bounds": [_SHP, _P, _P, _P],
+        "kv_build_block_key_means": [_SHP, _P, _P, _P, _P],
+        "kv_select_blocks_mean16": [_SHP, _P, _F, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_select_blocks_quest": [_SHP, _P, _F, _P, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_build_block_cov_factors": [_SHP, _P, _I, _P, _P],
         "kv_select_blocks_cobs": [_SHP, _P, _F, _P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P],
@@ -93,6 +96,7 @@ def lib():
                            _P, _S, _I, _P],
         "kv_workspace_init": [_P, _S, _P],
         "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
+        "kv_selftest_wait_timeout": [_P, _P, ctypes.c_uint64, _I, _P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -249,6 +253,52 @@ def kv_select_blocks(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, b
                                   _ptr(counts), _ptr(K) if mode == KV_SCORE_EXACT_MASS else None,
                                   int(k_top), int(bool(force_first)), int(bool(force_last)), int(kmax),
                                   _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
+    return block_idx, n_kept, scores
+
+
+def kv_build_block_key_means(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int, k_sum: torch.Tensor,
+                             counts: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block mean keys at bf16 precision [B][Hkv][NB][D] from the fp32 key sums and
+    counts of kv_build_block_summaries (K gives the shape only)."""
+    _need(K, "K", torch.bfloat16)
+    _need(k_sum, "k_sum", torch.float32)
+    _need(counts, "counts", torch.int32)
+    B, Hkv, Ncap, D = K.shape
+    NB = (Ncap + block_size - 1) // block_size
+    if out is None:
+        out = torch.empty(B, Hkv, NB, D, dtype=torch.bfloat16, device=K.device)
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, block_size, KV_BF16, seq_lens.data_ptr())
+    _check(lib().kv_build_block_key_means(ctypes.byref(shape), _ptr(k_sum), _ptr(counts), _ptr(out),
+                                          _stream(K.device)))
+    return out
+
+
+def kv_select_blocks_mean16(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                            scale: float, k_mean: torch.Tensor, counts: torch.Tensor, k_top: int,
+                            force_first: bool = False, force_last: bool = False, kmax: Optional[int] = None,
+                            block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                            scores: Optional[torch.Tensor] = None, want_scores: bool = False):
+    """Kept blocks per KV head scored from the bf16 block means (summary score
+    with the mean at bf16). K is not read. Returns (block_idx [B][Hkv][kmax],
+    n_kept [B][Hkv], scores or None)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_mean, "k_mean", torch.bfloat16)
+    _need(counts, "counts", torch.int32)
+    shape = make_shape(q, K, seq_lens, block_size)
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    dev = q.device
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if scores is None and want_scores:
+        scores = torch.empty(shape.B, shape.Hkv, NB, dtype=torch.float32, device=dev)
+    _check(lib().kv_select_blocks_mean16(ctypes.byref(shape), _ptr(q), float(scale), _ptr(k_mean), _ptr(counts),
+                                         int(k_top), int(bool(force_first)), int(bool(force_last)), int(kmax),
+                                         _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
     return block_idx, n_kept, scores
 
 
@@ -434,3 +484,16 @@ def kv_dense_decode_attn(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_
                                       _ptr(out), _ptr(lse), workspace.ptr(), workspace.nbytes,
                                       _stream(dev)))
     return out, lse
+
+
+def kv_selftest_wait_timeout(status: torch.Tensor, limit_ns: int, arrive: bool) -> torch.Tensor:
+    """Runs the kernels' bounded copy wait once in a one-warp kernel: with
+    arrive=False it waits for bytes no copy delivers and must give up after
+    limit_ns, OR-ing KV_DEV_WAIT_TIMEOUT into status (a 1-element int32 device
+    tensor); with arrive=True the wait completes. Returns a 1-element device
+    tensor: 1 if the wait completed, 0 if it gave up."""
+    _need(status, "status", torch.int32)
+    ok = torch.full((1,), 7, dtype=torch.int32, device=status.device)
+    _check(lib().kv_selftest_wait_timeout(_ptr(status), _ptr(ok), ctypes.c_uint64(int(limit_ns)), 1 if arrive else 0,
+                                          _stream(status.device)))
+    return ok

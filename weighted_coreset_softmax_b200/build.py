@@ -45,12 +45,30 @@ def build(force: bool = False, verbose: bool = False, ptxas_info: bool = False) 
     nvcc = _nvcc()
     hdr_time = _newest(headers) if headers else 0.0
 
+    def deps_of(obj):
+        """Headers the object was built from (nvcc's -MD file), or None."""
+        dep = obj[:-2] + ".d"
+        if not os.path.exists(dep):
+            return None
+        with open(dep) as f:
+            text = f.read().replace("\\\n", " ")
+        parts = text.split(":", 1)
+        if len(parts) != 2:
+            return None
+        # the repository's own headers only (system headers belong to the image)
+        return [t for t in parts[1].split() if t.endswith((".h", ".cuh")) and (
+            os.path.realpath(t).startswith(os.path.realpath(CSRC)) or
+            os.path.realpath(t).startswith(os.path.realpath(INCLUDE)))]
+
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
-        if (not force and os.path.exists(obj)
-                and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_time)):
-            return obj, ""
-        cmd = [nvcc, *ARCH, *FLAGS, "-c", src, "-o", obj]
+        if not force and os.path.exists(obj):
+            deps = deps_of(obj)
+            newest = max([os.path.getmtime(src)] + ([os.path.getmtime(d) for d in deps if os.path.exists(d)]
+                                                    if deps is not None else [hdr_time]))
+            if os.path.getmtime(obj) >= newest:
+                return obj, ""
+        cmd = [nvcc, *ARCH, *FLAGS, "-MD", "-MF", obj[:-2] + ".d", "-c", src, "-o", obj]
         if ptxas_info:
             cmd[1:1] = ["-Xptxas", "-v"]
         r = subprocess.run(cmd, capture_output=True, text=True)

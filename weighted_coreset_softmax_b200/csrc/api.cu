@@ -212,6 +212,19 @@ bool attention_uses_tensor_cores() {
   return v;
 }
 
+// Block-mode attention over a bf16 cache with block size >= 32 runs the
+// warp-specialised kernel (one CTA per SM, a producer warp streaming the kept
+// chunks far ahead of eight tensor-core consumer warps) when the environment
+// variable KVSPARSE_ATTN=v2 asks for it (read once per process); otherwise, and
+// for other modes and shapes, the per-worker-ring kernel runs.
+bool attention_uses_gather() {
+  static const bool v = [] {
+    const char* e = std::getenv("KVSPARSE_ATTN");
+    return e && std::strcmp(e, "v2") == 0;
+  }();
+  return v;
+}
+
 // Tiled 2-D tensor map over a [rows][D] bf16 cache: boxes of box_rows rows x 64
 // elements (128 bytes; 32 rows for block copies, 1 row for gather4), 128-byte
 // swizzle, zero fill past the last row. Encoded
@@ -293,7 +306,8 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
                         const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
                         const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
                         int use_proxy, const int32_t* tok_idx, const float* w, int m, int mode, float* out,
-                        float* lse, void* ws, size_t ws_bytes, kv_stream_t stream, const FusedSel* fs = nullptr) {
+                        float* lse, void* ws, size_t ws_bytes, kv_stream_t stream, const FusedSel* fs = nullptr,
+                        bool check_only = false) {
   const int G = s->Hq / s->Hkv;
   const int NBH = s->B * s->Hkv;
   const int NBcap = (s->Ncap + s->block_size - 1) / s->block_size;
@@ -341,6 +355,10 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   if (fs && !use_mma) return fail(KV_ERR_UNSUPPORTED, "the fused decode step needs the tensor-core path");
   const int cps = kvs::attn_ctas_per_sm(s->dtype, s->D, G, use_mma, dev);
   if (cps <= 0) return fail(KV_ERR_CUDA, "attention kernel does not fit on an SM");
+  if (use_mma && static_cast<uint64_t>(NBH) * s->Ncap > 0x7fffffffull)
+    return fail(KV_ERR_UNSUPPORTED, "B * Hkv * Ncap = %llu rows is too many",
+                static_cast<unsigned long long>(static_cast<uint64_t>(NBH) * s->Ncap));
+  if (check_only) return KV_OK;
   kvs::AttnParams p{};
   p.q = q;
   p.K = K;
@@ -402,14 +420,36 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
     KV_TRY(encode_kv_map(K, rows, s->D, box_rows, &tk));
     KV_TRY(encode_kv_map(V, rows, s->D, box_rows, &tv));
   }
-  cudaError_t e = fs ? kvs::launch_fused(s->dtype, s->D, G, p, tk, tv, NBH, reinterpret_cast<cudaStream_t>(stream))
-                     : kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),
-                                        reinterpret_cast<cudaStream_t>(stream));
+  const bool gather = !fs && use_mma && mode == kvs::ATTN_BLOCKS && s->block_size >= 32 && attention_uses_gather();
+  cudaError_t e;
+  if (gather) {
+    const long long T = static_cast<long long>(NBH) * (kmax > 0 ? kmax : 1) * (s->block_size / 32);
+    const int grid = static_cast<int>(std::min<long long>(sms, T));
+    e = kvs::launch_gather(s->D, G, p, tk, tv, grid, reinterpret_cast<cudaStream_t>(stream));
+  } else {
+    e = fs ? kvs::launch_fused(s->dtype, s->D, G, p, tk, tv, NBH, reinterpret_cast<cudaStream_t>(stream))
+           : kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),
+                              reinterpret_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) return cuda_fail(e, fs ? "fused decode step launch" : "attention launch");
   return KV_OK;
 }
 
 }  // namespace
+
+namespace kvs {
+// Every argument check of kv_sparse_decode_attn, with nothing enqueued.
+kv_status sparse_attn_check(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                            const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
+                            const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
+                            int use_tail_proxy, const int32_t* tok_idx, const float* w, int m, float* out, float* lse,
+                            void* workspace, size_t ws_bytes) {
+  KV_TRY(check_shape(shape));
+  const int mode = tok_idx ? kvs::ATTN_WEIGHTED : kvs::ATTN_BLOCKS;
+  return run_attention(shape, q, scale, K, V, block_idx, n_kept, kmax, k_sum, v_sum, counts, k_tot, v_tot,
+                       use_tail_proxy, tok_idx, w, m, mode, out, lse, workspace, ws_bytes, nullptr, nullptr, true);
+}
+}  // namespace kvs
 
 extern "C" {
 
@@ -430,6 +470,28 @@ kv_status kv_build_block_summaries(const kv_shape* shape, const void* K, const v
                                    NBH, shape->Hkv, shape->Ncap, shape->block_size, NBcap,
                                    reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "summary launch");
+  return KV_OK;
+}
+
+kv_status kv_build_block_key_means(const kv_shape* shape, const float* k_sum, const int32_t* counts, void* k_mean,
+                                   kv_stream_t stream) {
+  KV_TRY(check_shape(shape));
+  KV_TRY(need(k_sum, "k_sum"));
+  KV_TRY(need(counts, "counts", 4));
+  KV_TRY(need(k_mean, "k_mean"));
+  const int NBH = shape->B * shape->Hkv;
+  const int NBcap = (shape->Ncap + shape->block_size - 1) / shape->block_size;
+  if (NBH == 0 || NBcap == 0) return KV_OK;
+  const int64_t rows = static_cast<int64_t>(NBH) * NBcap;
+  const int64_t work = rows * (shape->D / 8);
+  const int sms = num_sms_current();
+  if (sms <= 0) return fail(KV_ERR_CUDA, "no CUDA device available");
+  const int64_t want = (work + 255) / 256;
+  const int grid = static_cast<int>(std::min<int64_t>(want, static_cast<int64_t>(sms) * 8));
+  kvs::block_mean16_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      k_sum, counts, static_cast<__nv_bfloat16*>(k_mean), rows, shape->Hkv, NBcap, shape->D);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "key-mean launch");
   return KV_OK;
 }
 
@@ -474,7 +536,7 @@ namespace {
 kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_mode, const float* k_sum,
                      const void* k_bounds, const int32_t* counts, const void* K, int k_top, int force_first,
                      int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
-                     kv_stream_t stream, const float* k_xi = nullptr, int rank = 0) {
+                     kv_stream_t stream, const float* k_xi = nullptr, int rank = 0, const void* k_mean16 = nullptr) {
   KV_TRY(check_shape(shape));
   if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
   KV_TRY(need(q, "q"));
@@ -488,6 +550,10 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
     }
   } else if (sel_mode == kvs::SEL_EXACT) {
     KV_TRY(need(K, "K"));
+  } else if (sel_mode == kvs::SEL_MEAN16) {
+    if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "bf16-mean scoring is built for bf16 caches only");
+    KV_TRY(need(k_mean16, "k_mean"));
+    KV_TRY(need(counts, "counts", 4));
   } else {
     if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "Quest scoring reads bf16 bounds (bf16 caches only)");
     KV_TRY(need(k_bounds, "k_bounds"));
@@ -507,6 +573,7 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
   p.q = q;
   p.k_sum = k_sum;
   p.k_bounds = k_bounds;
+  p.k_mean16 = k_mean16;
   p.k_xi = k_xi;
   p.cobs_r = rank;
   p.counts = counts;
@@ -543,6 +610,13 @@ kv_status kv_select_blocks(const kv_shape* shape, const void* q, float scale, kv
     return fail(KV_ERR_INVALID_ARG, "unknown score mode %d", (int)mode);
   return select_any(shape, q, scale, mode == KV_SCORE_SUMMARY ? kvs::SEL_SUMMARY : kvs::SEL_EXACT, k_sum, nullptr,
                     counts, K, k_top, force_first, force_last, kmax, block_idx, n_kept, scores, stream);
+}
+
+kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float scale, const void* k_mean,
+                                  const int32_t* counts, int k_top, int force_first, int force_last, int kmax,
+                                  int32_t* block_idx, int32_t* n_kept, float* scores, kv_stream_t stream) {
+  return select_any(shape, q, scale, kvs::SEL_MEAN16, nullptr, nullptr, counts, nullptr, k_top, force_first,
+                    force_last, kmax, block_idx, n_kept, scores, stream, nullptr, 0, k_mean);
 }
 
 kv_status kv_select_blocks_cobs(const kv_shape* shape, const void* q, float scale, const float* k_sum,

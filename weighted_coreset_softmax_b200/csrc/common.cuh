@@ -73,16 +73,20 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 // Bounded wait for the phase with the given parity. Returns false (and sets the
-// timeout bit in *status) once WAIT_LIMIT_NS of wall time has passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+// timeout bit in *status) once limit_ns of wall time has passed.
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, uint32_t* status, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > WAIT_LIMIT_NS) break;
+    if (global_ns() - t0 > limit_ns) break;
   }
   if (status) atomicOr(status, KV_DEV_WAIT_TIMEOUT);
   return false;
+}
+// The kernels' wait on a copy: gives up after WAIT_LIMIT_NS.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t* status) {
+  return mbar_wait_for(bar, parity, status, WAIT_LIMIT_NS);
 }
 
 // ------------------------------------------------ programmatic dependent launch
@@ -99,6 +103,11 @@ __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol
 __device__ __forceinline__ uint64_t l2_evict_first_policy() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 // Global -> this CTA's shared memory, completion counted in bytes on `bar`.

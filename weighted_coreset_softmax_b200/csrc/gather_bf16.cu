@@ -1,0 +1,60 @@
+// Launchers of the warp-specialised block-mode attention kernel (bf16 caches,
+// D in {64, 128}, G in 1..8).
+#include <cuda_runtime.h>
+
+#include <atomic>
+
+#include "gather_attn.cuh"
+
+namespace kvs {
+
+template <int D, int G>
+static cudaError_t gather_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                                     cudaStream_t st) {
+  using C = GaCfg<D, G>;
+  static std::atomic<int> configured{0};  // one bit per device: smem limit raised
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (!(configured.load() & (1 << (dev & 31)))) {
+    const cudaError_t e =
+        cudaFuncSetAttribute(gather_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    configured.fetch_or(1 << (dev & 31));
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(GA_THREADS);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, gather_attn_kernel<D, G>, p, tk, tv);
+  if (le != cudaSuccess) return le;
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t gather_launch_d(int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                                   cudaStream_t st) {
+  switch (G) {
+    case 1: return gather_launch_one<D, 1>(p, tk, tv, grid, st);
+    case 2: return gather_launch_one<D, 2>(p, tk, tv, grid, st);
+    case 3: return gather_launch_one<D, 3>(p, tk, tv, grid, st);
+    case 4: return gather_launch_one<D, 4>(p, tk, tv, grid, st);
+    case 5: return gather_launch_one<D, 5>(p, tk, tv, grid, st);
+    case 6: return gather_launch_one<D, 6>(p, tk, tv, grid, st);
+    case 7: return gather_launch_one<D, 7>(p, tk, tv, grid, st);
+    case 8: return gather_launch_one<D, 8>(p, tk, tv, grid, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_gather(int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                          cudaStream_t st) {
+  return D == 64 ? gather_launch_d<64>(G, p, tk, tv, grid, st) : gather_launch_d<128>(G, p, tk, tv, grid, st);
+}
+
+}  // namespace kvs

@@ -153,7 +153,8 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
   static std::atomic<int> configured{0};  // one bit per device: smem limit raised
   int dev = 0;
   cudaGetDevice(&dev);
-  if constexpr (MODE == SEL_QUEST && sizeof(T) != 2) return cudaErrorInvalidValue;  // bf16 bounds only
+  if constexpr ((MODE == SEL_QUEST || MODE == SEL_MEAN16) && sizeof(T) != 2)
+    return cudaErrorInvalidValue;  // bf16 bounds and bf16 means: bf16 caches only
   const size_t smem = MODE != SEL_EXACT ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
   if (!(configured.load() & (1 << (dev & 31)))) {
     size_t most = MODE != SEL_EXACT ? sel_summary_smem_bytes(G, SEL_MAXNB) : sel_smem_bytes(G, SEL_MAXNB);
@@ -173,6 +174,10 @@ template <typename T, int D, int G>
 cudaError_t select_launch_one(int mode, const SelParams& p, int grid, cudaStream_t st) {
   if (mode == SEL_QUEST) {
     if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_QUEST>(p, grid, st);
+    return cudaErrorInvalidValue;
+  }
+  if (mode == SEL_MEAN16) {
+    if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_MEAN16>(p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (mode == SEL_COBS) return select_launch_mode<T, D, G, SEL_COBS>(p, grid, st);

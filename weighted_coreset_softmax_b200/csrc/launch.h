@@ -22,6 +22,10 @@ int attn_ctas_per_sm(int dtype, int D, int G, bool use_mma, int dev);
 bool fused_fits(int dtype, int D, int G, int NBcap);
 cudaError_t launch_fused(int dtype, int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                          int grid, cudaStream_t st);
+// Warp-specialised block-mode attention (bf16, tensor cores, block size >= 32):
+// one CTA per SM, grid <= number of SMs.
+cudaError_t launch_gather(int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
+                          cudaStream_t st);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,

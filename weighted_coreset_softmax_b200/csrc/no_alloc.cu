@@ -15,9 +15,9 @@
 // on each device looks the address up with cudaGetSymbolAddress (with that
 // device current) and caches it; make that first call before capturing any
 // stream into a CUDA graph. All calls on a device share the array and it keeps
-// the previous call's contents: each call clears the parts that must start at
-// zero (status word and arrival counters) with an async memset on the caller's
-// stream. Two calls whose kernels overlap on the GPU (different streams without
+// the previous call's contents: each call, once its arguments have passed every
+// check, clears the parts that must start at zero (status word and arrival
+// counters) with an async memset on the caller's stream. Two calls whose kernels overlap on the GPU (different streams without
 // ordering) race on the shared array and give wrong results; order them.
 // Device-side index checks still skip bad entries, but their status bits are
 // cleared by the next call and are not reported here.
@@ -30,6 +30,11 @@
 
 namespace kvs {
 void set_last_error(const char* msg);
+kv_status sparse_attn_check(const kv_shape* shape, const void* q, float scale, const void* K, const void* V,
+                            const int32_t* block_idx, const int32_t* n_kept, int kmax, const float* k_sum,
+                            const float* v_sum, const int32_t* counts, const float* k_tot, const float* v_tot,
+                            int use_tail_proxy, const int32_t* tok_idx, const float* w, int m, float* out, float* lse,
+                            void* workspace, size_t ws_bytes);
 }
 
 namespace {
@@ -88,6 +93,11 @@ extern "C" kv_status kv_sparse_decode_attn_noalloc(
   }
   void* scratch = nullptr;
   kv_status st = scratch_address(&scratch);
+  if (st != KV_OK) return st;
+  // every argument check first: a call that is rejected enqueues nothing (not
+  // even the clearing memset below, which would disturb a call still in flight)
+  st = kvs::sparse_attn_check(shape, q, scale, K, V, block_idx, n_kept, kmax, k_sum, v_sum, counts, k_tot, v_tot,
+                              use_tail_proxy, tok_idx, w, m, out, lse, scratch, KV_NOALLOC_SCRATCH_BYTES);
   if (st != KV_OK) return st;
   if (need > 0 && shape->B > 0 && shape->Hkv > 0) {
     // status word and arrival counters must start at zero

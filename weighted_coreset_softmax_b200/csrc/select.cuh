@@ -32,12 +32,16 @@ constexpr int SEL_THREADS = 256;
 constexpr int SEL_NW = SEL_THREADS / 32;
 constexpr int SEL_MAXNB = 4096;  // NBcap limit
 
-enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2, SEL_COBS = 3 };
+enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2, SEL_COBS = 3, SEL_MEAN16 = 4 };
+// Row kinds of the summary-style scorer: fp32 key sums, Quest (min, max) bf16
+// pairs (both four bytes a channel), bf16 block means (two bytes a channel).
+enum SelRow { ROW_SUM32 = 0, ROW_QUEST = 1, ROW_MEAN16 = 2 };
 
 struct SelParams {
   const void* q;
   const float* k_sum;
   const void* k_bounds;  // Quest mode: [B][Hkv][NBcap][D][2] bf16 (min, max)
+  const void* k_mean16;  // bf16-mean mode: [B][Hkv][NBcap][D] bf16 block mean keys
   const float* k_xi;     // second-order mode: [B][Hkv][NBcap][cobs_r][D] fp32 scaled eigenvectors
   int cobs_r;
   const int32_t* counts;
@@ -119,27 +123,38 @@ __host__ __device__ inline size_t sel_summary_smem_bytes(int G, int NBcap) {
          sel_ring_bytes(G);
 }
 
-// QUEST: the rows are the Quest bounds -- per channel a (min, max) bf16 pair, also
-// four bytes per channel -- and a lane's logit part is sum_j max(q_j min_j,
+// ROW_QUEST: the rows are the Quest bounds -- per channel a (min, max) bf16 pair,
+// also four bytes per channel -- and a lane's logit part is sum_j max(q_j min_j,
 // q_j max_j) over its four channels, with no count term ("COBS: Cumulant Order
 // Block Sparse Attention", the Quest paragraph: the largest inner product any
 // point of the block's bounding box can reach).
-template <typename T, int D, int G, bool QUEST = false>
+// ROW_MEAN16: the rows are the block mean keys at bf16 precision (the same
+// page's quantisation paragraph keeps the block mean at bf16), two bytes a
+// channel: a lane covers eight channels with one 16-byte piece, a 512-byte ring
+// slot holds two rows at D = 128, and the logit is the dot plus log2 n_b (no
+// division: the row is already the mean).
+template <typename T, int D, int G, int ROWK = ROW_SUM32>
 __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, int nbv, float4* ring, int* cnt,
                               SelMisc& ms) {
-  constexpr int LPR = D / 4;  // fp32 rows, float4 per lane
+  constexpr bool QUEST = ROWK == ROW_QUEST;
+  constexpr bool M16 = ROWK == ROW_MEAN16;
+  constexpr int CPL = M16 ? 8 : 4;        // channels per lane (one 16-byte piece)
+  constexpr int RB = D * (M16 ? 2 : 4);   // bytes per row
+  constexpr int LPR = D / CPL;            // lanes per row
   constexpr int RPW = 32 / LPR;
   constexpr int GP = pow2ceil(G);
-  constexpr int RS0 = LPR / GP;
-  constexpr int RS = RS0 < 1 ? 1 : (RS0 > 8 ? 8 : RS0);  // rows per lane per batch
+  constexpr int RS0 = (D / 4) / GP;       // ring bytes as for fp32 rows (sel_ring_bytes)
+  constexpr int RS = RS0 < 1 ? 1 : (RS0 > 8 ? 8 : RS0);  // row slots per lane per batch
   constexpr int NV = RS * GP;
   constexpr int BATCH = RPW * RS;                         // rows per warp per batch
   using HV = HeldValues<NV, LPR, GP>;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rg = lane / LPR, c = lane % LPR;
   const int b = bh / p.Hkv, h = bh % p.Hkv;
-  // four bytes per channel in either layout: fp32 sums, or (min, max) bf16 pairs
-  const float* krows = (QUEST ? static_cast<const float*>(p.k_bounds) : p.k_sum) + static_cast<size_t>(bh) * p.NBcap * D;
+  // RB bytes a row: fp32 sums, (min, max) bf16 pairs, or bf16 means
+  const unsigned char* krows =
+      static_cast<const unsigned char*>(QUEST ? p.k_bounds : (M16 ? p.k_mean16 : static_cast<const void*>(p.k_sum))) +
+      static_cast<size_t>(bh) * p.NBcap * RB;
   const int nbt = (nbv + BATCH - 1) / BATCH;               // batches of the bh
   const int nmine = nbt > warp ? (nbt - warp + SEL_NW - 1) / SEL_NW : 0;  // batches of this warp
   // The ring is filled by bulk copies with an L2 evict-first policy (the rows are
@@ -155,14 +170,14 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     const int st = m % SEL_STAGES;
     const int rb = (warp + m * SEL_NW) * BATCH;
     const int nvalid = min(BATCH, nbv - rb);  // >= 1: batch rb starts below nbv
-    if (lane == 0) mbar_arrive_expect_tx(rbar + st, static_cast<uint32_t>(nvalid) * D * 4);
+    if (lane == 0) mbar_arrive_expect_tx(rbar + st, static_cast<uint32_t>(nvalid) * RB);
     __syncwarp();
     if (lane < RS) {
       const int r0 = rb + lane * RPW;
       const int nr = min(RPW, nbv - r0);
       if (nr > 0)
-        bulk_g2s(ring + (st * RS + lane) * SEL_THREADS + warp * 32, krows + static_cast<size_t>(r0) * D,
-                 static_cast<uint32_t>(nr) * D * 4, rbar + st, pol);
+        bulk_g2s(ring + (st * RS + lane) * SEL_THREADS + warp * 32, krows + static_cast<size_t>(r0) * RB,
+                 static_cast<uint32_t>(nr) * RB, rbar + st, pol);
     }
   };
 #pragma unroll
@@ -172,12 +187,20 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     const int32_t* cn = p.counts + static_cast<size_t>(b) * p.NBcap;
     for (int i = tid; i < nbv; i += SEL_THREADS) cnt[i] = __ldg(cn + i);
   }
-  const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c * 4;
+  const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D + c * CPL;
   float4 qf[G];
+  float q8[M16 ? G : 1][8];
+  if constexpr (M16) {
 #pragma unroll
-  for (int g = 0; g < G; ++g)
-    qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
-                        load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
+    for (int g = 0; g < G; ++g)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q8[g][e] = load_as_float(qrow + g * D + e) * p.qscale;
+  } else {
+#pragma unroll
+    for (int g = 0; g < G; ++g)
+      qf[g] = make_float4(load_as_float(qrow + g * D) * p.qscale, load_as_float(qrow + g * D + 1) * p.qscale,
+                          load_as_float(qrow + g * D + 2) * p.qscale, load_as_float(qrow + g * D + 3) * p.qscale);
+  }
   // QUEST: max(q min, q max) = max(q, 0) max + min(q, 0) min (max >= min), two FMAs
   float qa[QUEST ? G : 1][4], qb[QUEST ? G : 1][4];
   if constexpr (QUEST) {
@@ -211,7 +234,27 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
     for (int i = 0; i < RS; ++i) {
       const int row = rb + i * RPW + rg;
       const float4 k4 = row < nbv ? ring[(st * RS + i) * SEL_THREADS + tid] : make_float4(0.f, 0.f, 0.f, 0.f);
-      if constexpr (QUEST) {
+      if constexpr (M16) {
+        // bf16 means of channels 8c .. 8c + 7
+        float2 kf[4];
+        Chunk<__nv_bfloat16>::unpack(*reinterpret_cast<const uint4*>(&k4), kf);
+#pragma unroll
+        for (int g = 0; g < GP; ++g) {
+          if (g < G) {
+            float d = q8[g][0] * kf[0].x;
+            d = fmaf(q8[g][1], kf[0].y, d);
+            d = fmaf(q8[g][2], kf[1].x, d);
+            d = fmaf(q8[g][3], kf[1].y, d);
+            d = fmaf(q8[g][4], kf[2].x, d);
+            d = fmaf(q8[g][5], kf[2].y, d);
+            d = fmaf(q8[g][6], kf[3].x, d);
+            d = fmaf(q8[g][7], kf[3].y, d);
+            part[i * GP + g] = d;
+          } else {
+            part[i * GP + g] = 0.f;
+          }
+        }
+      } else if constexpr (QUEST) {
         // (min, max) pairs of channels 4c .. 4c + 3
         const __nv_bfloat162* mm = reinterpret_cast<const __nv_bfloat162*>(&k4);
         float lo[4], hi[4];
@@ -261,6 +304,9 @@ __device__ void score_summary(const SelParams& p, float* lg, int nbp, int bh, in
         float x;
         if constexpr (QUEST) {
           x = part[j];  // the box bound, in the log2 domain through qscale
+        } else if constexpr (M16) {
+          const int nb = cnt[row];
+          x = nb > 0 ? part[j] + log2f(static_cast<float>(nb)) : -INFINITY;
         } else {
           const int nb = cnt[row];
           x = nb > 0 ? part[j] / static_cast<float>(nb) + log2f(static_cast<float>(nb)) : -INFINITY;
@@ -539,7 +585,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
-  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS || MODE == SEL_MEAN16) {
     // the scorer ring's mbarriers (one per warp and stage)
     if (tid == 0) {
 #pragma unroll
@@ -551,7 +597,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
     __syncthreads();
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-    score_summary<T, D, G, MODE == SEL_QUEST>(p, lg, nbp, bh, nbv, ring, cnt, ms);
+    score_summary<T, D, G, MODE == SEL_QUEST ? ROW_QUEST : (MODE == SEL_MEAN16 ? ROW_MEAN16 : ROW_SUM32)>(
+        p, lg, nbp, bh, nbv, ring, cnt, ms);
   }
   else
     score_exact<T, D, G>(p, lg, nbp, bh, nbv, n);
@@ -597,7 +644,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   // per-head normaliser log2 sum_b 2^lg (Equation 5's Z, log2 domain): in summary
   // and Quest modes from the warps' (max, sum) pairs of the scoring pass, else
   // (exact and second-order modes) a pass over lg
-  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_MEAN16) {
     if (warp == 0 && lane < G) {
       float M = -INFINITY;
 #pragma unroll

@@ -159,3 +159,44 @@ __global__ void __launch_bounds__(256) block_totals_kernel(const float* __restri
 }
 
 }  // namespace kvs
+
+namespace kvs {
+
+// Block mean keys at bf16 precision, built once from the fp32 key sums and the
+// counts ("COBS: Cumulant Order Block Sparse Attention", the quantisation
+// paragraph: the block mean is kept at bf16). Each thread converts eight
+// channels: the mean is the correctly rounded fp32 quotient k_sum / n_b, rounded
+// to the nearest bf16 (ties to even); blocks with no token get zeros.
+__global__ void __launch_bounds__(256) block_mean16_kernel(const float* __restrict__ k_sum,
+                                                           const int32_t* __restrict__ counts,
+                                                           __nv_bfloat16* __restrict__ k_mean, int64_t rows, int Hkv,
+                                                           int NBcap, int D) {
+  const int per_row = D / 8;
+  const int64_t total = rows * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / per_row;  // (b, h, blk)
+    const int c = static_cast<int>(i - row * per_row);
+    const int blk = static_cast<int>(row % NBcap);
+    const int64_t bh = row / NBcap;
+    const int b = static_cast<int>(bh / Hkv);
+    const int n = counts[static_cast<int64_t>(b) * NBcap + blk];
+    const float4* src = reinterpret_cast<const float4*>(k_sum + row * D + c * 8);
+    const float4 a = __ldcs(src), bq = __ldcs(src + 1);
+    const float v[8] = {a.x, a.y, a.z, a.w, bq.x, bq.y, bq.z, bq.w};
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float lo = 0.f, hi = 0.f;
+      if (n > 0) {
+        lo = __fdiv_rn(v[2 * e], static_cast<float>(n));
+        hi = __fdiv_rn(v[2 * e + 1], static_cast<float>(n));
+      }
+      const __nv_bfloat16 bl = __float2bfloat16_rn(lo), bhv = __float2bfloat16_rn(hi);
+      w[e] = static_cast<uint32_t>(__bfloat16_as_ushort(bl)) | (static_cast<uint32_t>(__bfloat16_as_ushort(bhv)) << 16);
+    }
+    *reinterpret_cast<uint4*>(k_mean + row * D + c * 8) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+}  // namespace kvs
