@@ -45,8 +45,14 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="llama", choices=["llama", "qwen_long", "llama_osa", "llama_quest", "llama_cobs",
-                                                           "llama_coreset"])
+    ap.add_argument("--workload", default="llama", choices=["llama", "llama_b1", "qwen_long", "llama_osa", "llama_quest",
+                                                           "llama_cobs", "llama_coreset"])
+    ap.add_argument("--scorer", choices=["mean16", "sum32"], default="mean16",
+                    help="summary-mode selection: bf16 block means (default) or fp32 block sums")
+    ap.add_argument("--attn", choices=["v1", "v2"], default=None,
+                    help="attention kernel for block mode (default: the library's choice)")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the 5%% budget line and the read floor")
+    ap.add_argument("--no-selection-check", action="store_true", help="skip the oracle check of the kept blocks")
     ap.add_argument("--budget", type=float, default=0.01)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline work")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -157,11 +163,11 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
 
 
-# DRAM bytes per launch from the committed ncu capture
-# (profiles/attn_kernel_llama_b8_32k_1pct.md: 15.416 MB read, 0 written at B=8,
-# scaled x4 by sequences to the B=32 launch). Keyed by (kernel, workload, budget, B);
-# to be re-taken whenever the kernel changes.
-NCU_TRAFFIC = {("kv_sparse_decode_attn", "llama", 0.01, 32): 4 * 15_415_808}
+# DRAM bytes per launch of the dominant kernel from an ncu capture of the same
+# kernel build, keyed by (kernel, attention variant, workload, budget, B): the
+# capture ran at B = 8 and is scaled x4 by sequences to the B = 32 launch. An entry
+# is removed whenever its kernel changes, and the line then reports null.
+NCU_TRAFFIC = {}
 
 
 def measured_peak_hbm():
@@ -197,15 +203,18 @@ def attention_bytes(wl, n_kept, seq_lens):
     return total
 
 
-def select_bytes(wl, seq_lens):
-    """Algorithmic bytes of one kv_select_blocks launch (summary mode): every valid
-    block's fp32 key sum and count, q, and the kept indices written."""
+def select_bytes(wl, seq_lens, kmax=None):
+    """Algorithmic bytes of one summary-mode selection launch: every valid block's
+    key summary row (fp32 sum, or bf16 mean with the bf16-mean scorer) and count,
+    q, and the kept indices written."""
     L, D, G = wl.block_size, wl.D, wl.G
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    row = D * 2 if wl.score_mode == "summary_mean16" else D * 4
+    kmax = wl.kmax if kmax is None else kmax
     total = 0
     for b in range(wl.B):
         nbv = (seq_lens[b] + L - 1) // L
-        total += wl.Hkv * (nbv * (D * 4 + 4) + G * D * es + wl.kmax * 4 + 4)
+        total += wl.Hkv * (nbv * (row + 4) + G * D * es + kmax * 4 + 4)
     return total
 
 
@@ -243,10 +252,13 @@ def weighted_bytes(wl):
 
 # ----------------------------------------------------------------- CPU oracle
 def _oracle_task(args):
-    """One (sequence, KV head) decode step with the float64 oracle."""
+    """One (sequence, KV head) decode step with the float64 oracle. Returns the
+    kept blocks and near-tie flag (block modes), plus the kept set at the other
+    budgets asked for and, for bf16-mean scoring, the exact-mean kept set."""
     import numpy as np
     from oracle import oracle as O
-    kind, q16, K16, V16, n, L, scale, k_top, ff, fl, extra = args
+    kind, q16, K16, V16, n, L, scale, k_top, ff, fl, extra = args[:11]
+    more_k = args[11] if len(args) > 11 else ()
 
     def f64(a):
         if a.dtype == np.uint16:
@@ -256,11 +268,20 @@ def _oracle_task(args):
     q, K, V = f64(q16)[None], f64(K16)[None, None], f64(V16)[None, None]
     if kind == "weighted":
         O.weighted_batch(q, K, V, [n], extra[0][None, None], extra[1][None, None], scale)
-    elif kind == "dense":
+        return None
+    if kind == "dense":
         O.dense_batch(q, K, V, [n], scale)
-    else:
-        O.decode_step(q, K, V, [n], L, scale, k_top, ff, fl, score_mode=kind, use_proxy=True)
-    return 1
+        return None
+    sel, _, _ = O.decode_step(q, K, V, [n], L, scale, k_top, ff, fl, score_mode=kind, use_proxy=True)
+    s = sel[(0, 0)]
+    nb = (n + L - 1) // L
+    res = {"kept": s["kept"], "near_tie": s["near_tie"],
+           "more": {k: O.select_blocks(s["S"], nb, k, ff, fl) for k in more_k}}
+    res["more"] = {k: {"kept": v["kept"], "near_tie": v["near_tie"]} for k, v in res["more"].items()}
+    if kind == "summary_mean16":
+        ex = O.select_batch(q, K, [n], L, scale, k_top, ff, fl, "summary")[(0, 0)]
+        res["exact_mean_kept"] = ex["kept"]
+    return res
 
 
 def _pool_init():
@@ -269,11 +290,12 @@ def _pool_init():
     os.environ.setdefault("MKL_NUM_THREADS", "1")
 
 
-def oracle_tasks(wl, pairs):
+def oracle_tasks(wl, pairs, more_k=()):
     import numpy as np
     import torch
     tasks = []
-    kind = {"summary": "summary", "exact_mass": "exact_mass", "quest": "quest", "cobs": "cobs"}[wl.score_mode]
+    kind = {"summary": "summary", "summary_mean16": "summary_mean16", "exact_mass": "exact_mass", "quest": "quest",
+            "cobs": "cobs"}[wl.score_mode]
     if wl.attn_mode == "weighted":
         kind = "weighted"
     for (b, h) in pairs:
@@ -287,29 +309,34 @@ def oracle_tasks(wl, pairs):
         if kind == "weighted":
             extra = (wl.tok_idx[b, h].cpu().numpy(), wl.w[b, h].cpu().numpy().astype(np.float64))
         tasks.append((kind, q, K, V, wl.seq_lens[b], wl.block_size, wl.scale, wl.k_top,
-                      bool(wl.force_first), bool(wl.force_last), extra))
+                      bool(wl.force_first), bool(wl.force_last), extra, tuple(more_k)))
     return tasks
 
 
-def time_oracle(wl, n_pairs_target, workers, warm_pairs=1):
-    """Wall time of the oracle over n pairs (sequence, KV head) on a spawn pool."""
+def time_oracle(wl, n_pairs_target, workers, warm_pairs=1, more_k=()):
+    """Wall time of the oracle over n pairs (sequence, KV head) on a spawn pool;
+    also returns each distinct pair's oracle result."""
     pairs_all = [(b, h) for b in range(wl.B) for h in range(wl.Hkv)]
     n = max(1, n_pairs_target)
     pairs = [pairs_all[i % len(pairs_all)] for i in range(n)]
     uniq = sorted(set(pairs))
-    tmap = dict(zip(uniq, oracle_tasks(wl, uniq)))
+    tmap = dict(zip(uniq, oracle_tasks(wl, uniq, more_k)))
     tasks = [tmap[p] for p in pairs]
     ctx = mp.get_context("spawn")
     with ctx.Pool(workers, initializer=_pool_init) as pool:
         pool.map(_oracle_task, tasks[:max(1, min(warm_pairs, len(tasks)))] * 1)
         t0 = time.perf_counter()
-        pool.map(_oracle_task, tasks, chunksize=1)
+        outs = pool.map(_oracle_task, tasks, chunksize=1)
         dt = time.perf_counter() - t0
-    return dt, n
+    results = {}
+    for pr, o in zip(pairs, outs):
+        results.setdefault(pr, o)
+    return dt, n, results
 
 
-def cpu_baseline(wl, seconds, label_sample):
-    """Oracle throughput on the host cores over a bounded sample of the workload."""
+def cpu_baseline(wl, seconds, label_sample, more_k=()):
+    """Oracle throughput on the host cores over a bounded sample of the workload;
+    also returns the oracle's per-pair results (kept blocks) for the sample."""
     workers = max(1, min(os.cpu_count() or 1, 32))
     # calibrate with one pair in-process, single-threaded BLAS
     _pool_init()
@@ -318,18 +345,64 @@ def cpu_baseline(wl, seconds, label_sample):
     t1 = time.perf_counter() - t0
     n = int(max(1, min(wl.B * wl.Hkv * 4, seconds * workers / max(t1, 1e-3))))
     n = max(workers, n) if n >= workers else n
-    dt, n = time_oracle(wl, n, workers)
+    dt, n, results = time_oracle(wl, n, workers, more_k=more_k)
     queries = n / wl.Hkv
     return {"value": queries / dt, "unit": "queries/s", "cores": workers, "kind": "oracle",
             "sample": f"{n} (sequence, KV head) decode steps = {queries:g} queries of {label_sample}; "
                       f"float64 NumPy oracle (select + attend), {workers} spawn workers, 1 BLAS thread each",
-            "seconds": dt}
+            "seconds": dt}, results
+
+
+def selection_check(wl, oracle_res, idx, nk, idx5=None, nk5=None, more_k=()):
+    """Kept blocks of batch 0 on the GPU against the oracle's on the pairs the CPU
+    baseline sample covered: exact matches, mismatches at flagged near ties
+    (allowed, reported) and any other mismatch; for the bf16-mean scorer also how
+    many kept sets differ from the exact-mean (float64) ranking."""
+    gi, gn = idx.cpu().numpy(), nk.cpu().numpy()
+    out = {"pairs": 0, "exact": 0, "near_tie_flagged": 0, "near_tie_mismatch": 0, "other_mismatch": 0}
+    if wl.score_mode == "summary_mean16":
+        out["differ_from_exact_mean_ranking"] = 0
+    out5 = None
+    if idx5 is not None and more_k:
+        g5i, g5n = idx5.cpu().numpy(), nk5.cpu().numpy()
+        out5 = {"pairs": 0, "exact": 0, "near_tie_flagged": 0, "near_tie_mismatch": 0, "other_mismatch": 0}
+    for (b, h), r in sorted(oracle_res.items()):
+        if r is None:
+            continue
+        got = [int(x) for x in gi[b, h, :gn[b, h]]]
+        out["pairs"] += 1
+        out["near_tie_flagged"] += int(r["near_tie"])
+        if got == r["kept"]:
+            out["exact"] += 1
+        elif r["near_tie"]:
+            out["near_tie_mismatch"] += 1
+        else:
+            out["other_mismatch"] += 1
+        if "exact_mean_kept" in r and "differ_from_exact_mean_ranking" in out:
+            out["differ_from_exact_mean_ranking"] += int(got != r["exact_mean_kept"])
+        if out5 is not None and more_k[0] in r["more"]:
+            r5 = r["more"][more_k[0]]
+            got5 = [int(x) for x in g5i[b, h, :g5n[b, h]]]
+            out5["pairs"] += 1
+            out5["near_tie_flagged"] += int(r5["near_tie"])
+            if got5 == r5["kept"]:
+                out5["exact"] += 1
+            elif r5["near_tie"]:
+                out5["near_tie_mismatch"] += 1
+            else:
+                out5["other_mismatch"] += 1
+    out["reference"] = ("float64 oracle, " + ("bf16-mean ranking" if wl.score_mode == "summary_mean16" else
+                                               "exact-mean ranking") + ", pairs of the CPU baseline sample")
+    if out5 is not None:
+        out["budget_5pct"] = out5
+    return out
 
 
 # ----------------------------------------------------------------- our arm
 def workload_label(wl, budget):
     names = {
         "llama": "Llama-3.1-8B-shaped GQA decode",
+        "llama_b1": "Llama-3.1-8B-shaped GQA decode, batch 1 (latency)",
         "qwen_long": "Qwen2.5-7B-shaped long-context GQA decode",
         "llama_osa": "Llama-3.1-8B-shaped GQA decode, OSA exact-mass selection",
         "llama_quest": "Llama-3.1-8B-shaped GQA decode, Quest key-box selection",
@@ -343,6 +416,8 @@ def workload_label(wl, budget):
 
 
 def run_ours(args, dist):
+    if args.attn:
+        os.environ["KVSPARSE_ATTN"] = args.attn  # read once, when the library first runs attention
     import torch
     import weighted_coreset_softmax_b200 as kv
     from weighted_coreset_softmax_b200 import workloads as W
@@ -353,14 +428,19 @@ def run_ours(args, dist):
     kv.lib()
 
     name = args.workload
-    base_seed = (100 if name == "llama" else 3) + shard_seed_offset(dist.rank)
+    base_seed = {"llama": 100, "llama_b1": 1, "qwen_long": 2}.get(name, 3) + shard_seed_offset(dist.rank)
+    score_override = "summary_mean16" if args.scorer == "mean16" else None
     L2_BYTES = 126 << 20
 
     def make_set(j):
         seed = (None if dist.rank == 0 else base_seed) if j == 0 else base_seed + 50000 * j
         w_ = W.make(name, dev, budget=args.budget, B=args.batch, seed=seed)
+        if score_override and w_.score_mode == "summary":
+            w_.score_mode = score_override
         sl_ = w_.seq_lens_tensor(dev)
         su_ = kv.kv_build_block_summaries(w_.K, w_.V, sl_, w_.block_size)
+        if w_.score_mode == "summary_mean16":
+            su_["k_mean"] = kv.kv_build_block_key_means(w_.K, sl_, w_.block_size, su_["k_sum"], su_["counts"])
         if w_.score_mode == "quest":
             su_["k_bounds"] = kv.kv_build_block_bounds(w_.K, sl_, w_.block_size)
         if w_.score_mode == "cobs":
@@ -390,16 +470,27 @@ def run_ours(args, dist):
     wl, sl, summ, idx, nk, out, lse, ws = (s0[k] for k in ("wl", "sl", "summ", "idx", "nk", "out", "lse", "ws"))
     B = wl.B
     quest = wl.score_mode == "quest"
-    mode = kv.KV_SCORE_SUMMARY if wl.score_mode == "summary" else kv.KV_SCORE_EXACT_MASS
+    mode = kv.KV_SCORE_SUMMARY if wl.score_mode in ("summary", "summary_mean16") else kv.KV_SCORE_EXACT_MASS
     kmax = wl.kmax
     weighted = wl.attn_mode == "weighted"
 
-    def select_on(st_, q_=None):
+    def select_on(st_, q_=None, k_top=None, kmax_=None, idx_=None, nk_=None):
         if weighted:
             return
         w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
         q_ = w_.q if q_ is None else q_
-        if wl.score_mode == "cobs":
+        if k_top is not None:
+            kv.kv_select_blocks_mean16(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_mean"], su_["counts"], k_top,
+                                       w_.force_first, w_.force_last, kmax=kmax_, block_idx=idx_, n_kept=nk_) \
+                if wl.score_mode == "summary_mean16" else \
+                kv.kv_select_blocks(q_, w_.K, sl_, w_.block_size, w_.scale, su_["counts"], k_top, w_.force_first,
+                                    w_.force_last, k_sum=su_["k_sum"], kmax=kmax_, block_idx=idx_, n_kept=nk_)
+            return
+        if wl.score_mode == "summary_mean16":
+            kv.kv_select_blocks_mean16(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_mean"], su_["counts"], w_.k_top,
+                                       w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
+                                       n_kept=st_["nk"])
+        elif wl.score_mode == "cobs":
             kv.kv_select_blocks_cobs(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_sum"], su_["counts"], su_["k_xi"],
                                      w_.k_top, w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
                                      n_kept=st_["nk"])
@@ -412,9 +503,13 @@ def run_ours(args, dist):
                                 w_.force_first, w_.force_last, mode=mode, k_sum=su_["k_sum"], kmax=kmax,
                                 block_idx=st_["idx"], n_kept=st_["nk"])
 
-    def attend_on(st_, q_=None):
+    def attend_on(st_, q_=None, idx_=None, nk_=None):
         w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
         q_ = w_.q if q_ is None else q_
+        if idx_ is not None:
+            kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"], block_idx=idx_,
+                                     n_kept=nk_, summaries=su_, use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
+            return
         if weighted:
             kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
                                      tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
@@ -647,6 +742,86 @@ def run_ours(args, dist):
         dense = {"ms": d_ms, "GB_s": dbytes / (d_ms * 1e-3) / 1e9, "bytes": dbytes,
                  "speedup_attn_kernel": d_ms / att_avg, "speedup_step": d_ms / step_ms_local}
 
+    # secondary figures on the same batches: each kernel back to back (a graph of
+    # launches over the rotating batches: a decode loop's steady state), the 5%
+    # read budget, and a plain streaming read of the same byte counts (the time one
+    # launch needs just to move those bytes, launch and ramp included)
+    def graph_avg_ms(fn, n):
+        capst = torch.cuda.Stream(dev)
+        capst.wait_stream(stream)
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_, stream=capst):
+            for i in range(n):
+                fn(i)
+        stream.wait_stream(capst)
+        g_.replay()
+        torch.cuda.synchronize(dev)
+        a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_.record(stream)
+        g_.replay()
+        b_.record(stream)
+        torch.cuda.synchronize(dev)
+        del g_
+        return a_.elapsed_time(b_) / n
+
+    def alone_avg_ms(fn, n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        host_ahead(n)
+        for i in range(n):
+            evs[i][0].record(stream)
+            fn(i)
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        return statistics.fmean(e[0].elapsed_time(e[1]) for e in evs)
+
+    secondary = {}
+    if not args.no_secondary:
+        secondary["kernels_ms_back_to_back"] = {
+            "kv_sparse_decode_attn": graph_avg_ms(lambda i: attend_on(sets[i % ROT]), k_steps)}
+        if not weighted:
+            secondary["kernels_ms_back_to_back"]["kv_select_blocks"] = graph_avg_ms(
+                lambda i: select_on(sets[i % ROT]), k_steps)
+        sink = torch.zeros(1, dtype=torch.int32, device=dev)
+        a_b = attention_bytes(wl, nk, wl.seq_lens) if not weighted else weighted_bytes(wl)
+        floor = {"attn_bytes_alone_ms": alone_avg_ms(
+            lambda i: kv.kv_stream_read(sets[i % ROT]["wl"].K, a_b & ~15, sink), k_steps),
+                 "attn_bytes_back_to_back_ms": graph_avg_ms(
+            lambda i: kv.kv_stream_read(sets[i % ROT]["wl"].K, a_b & ~15, sink), k_steps)}
+        if not weighted:
+            s_b = select_bytes(wl, wl.seq_lens) if wl.score_mode in ("summary", "summary_mean16") else None
+            if s_b:
+                floor["select_bytes_alone_ms"] = alone_avg_ms(
+                    lambda i: kv.kv_stream_read(sets[i % ROT]["wl"].K, s_b & ~15, sink), k_steps)
+        secondary["read_floor"] = floor
+        if not weighted and wl.score_mode in ("summary", "summary_mean16") and abs(args.budget - 0.01) < 1e-9:
+            NBv = wl.NBcap
+            k5 = max(1, int(math.floor(0.05 * NBv)))
+            kmax5 = min(NBv, k5 + int(bool(wl.force_first)) + int(bool(wl.force_last)))
+            for st_ in sets:
+                st_["idx5"] = torch.zeros(st_["wl"].B, st_["wl"].Hkv, kmax5, dtype=torch.int32, device=dev)
+                st_["nk5"] = torch.zeros(st_["wl"].B, st_["wl"].Hkv, dtype=torch.int32, device=dev)
+
+            def step5(i):
+                st_ = sets[i % ROT]
+                select_on(st_, k_top=k5, kmax_=kmax5, idx_=st_["idx5"], nk_=st_["nk5"])
+                attend_on(st_, idx_=st_["idx5"], nk_=st_["nk5"])
+            for i in range(ROT):
+                step5(i)
+            torch.cuda.synchronize(dev)
+            step5_ms = graph_avg_ms(step5, k_steps)
+            att5 = alone_avg_ms(lambda i: attend_on(sets[i % ROT], idx_=sets[i % ROT]["idx5"],
+                                                    nk_=sets[i % ROT]["nk5"]), k_steps)
+            sel5 = alone_avg_ms(lambda i: select_on(sets[i % ROT], k_top=k5, kmax_=kmax5, idx_=sets[i % ROT]["idx5"],
+                                                    nk_=sets[i % ROT]["nk5"]), k_steps)
+            a5 = attention_bytes(wl, s0["nk5"], wl.seq_lens)
+            secondary["budget_5pct"] = {
+                "k_top": k5, "kmax": kmax5, "ms_per_step": step5_ms, "queries_per_s": B / (step5_ms * 1e-3),
+                "kernels_ms": {"kv_select_blocks": sel5, "kv_sparse_decode_attn": att5},
+                "attn_bytes_per_launch": a5, "attn_GB_s": a5 / (att5 * 1e-3) / 1e9,
+                "dense_over_sparse_attn_kernel": (dense["ms"] / att5) if dense else None,
+                "dense_over_sparse_step": (dense["ms"] / step5_ms) if dense else None}
+        check_status("in the secondary measurements")
+
     torch.cuda.synchronize(dev)
     check_status("during timing")
 
@@ -681,12 +856,15 @@ def run_ours(args, dist):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f32",
+        "dtype": "bf16",
         "data": "synthetic (seeded bf16 caches shaped like the pages' workloads)",
         "config": {
             "workload": workload_label(wl, args.budget),
             "B_per_gpu": B, "Hq": wl.Hq, "Hkv": wl.Hkv, "D": wl.D, "ctx": wl.Ncap,
-            "block": wl.block_size, "k_top": wl.k_top, "kmax": kmax, "kv_dtype": "bf16",
+            "block": wl.block_size, "k_top": wl.k_top, "kmax": kmax, "kv_dtype": "bf16", "accumulate": "fp32",
+            "selection": {"summary_mean16": "bf16 block means (kv_select_blocks_mean16)",
+                          "summary": "fp32 block sums (kv_select_blocks)"}.get(wl.score_mode, wl.score_mode),
+            "attention_kernel": os.environ.get("KVSPARSE_ATTN", "library default"),
             "parallelism": f"replicas: batch-sharded, {dist.world} rank(s), no collective",
             "l2": "one batch and no flush (--rot 1, a profiling run: the timed steps may hit L2)" if ROT == 1 else
                   f"inputs larger than L2: {ROT} independent batches (own caches, summaries, queries) rotate, "
@@ -703,7 +881,9 @@ def run_ours(args, dist):
         "bytes_per_launch": {"kv_select_blocks": s_bytes, "kv_sparse_decode_attn": a_bytes},
         "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": NCU_TRAFFIC.get((dom, args.workload, args.budget, B)),
+                     "traffic": NCU_TRAFFIC.get((dom, os.environ.get("KVSPARSE_ATTN", "default"), args.workload,
+                                                 args.budget, B)),
+                     "timing": "event pair around each launch, batches rotating (the kernel alone)",
                      "pct_of_8TBs": 100.0 * achieved / NOMINAL_HBM_GBS},
         "e2e": None if e2e_ms is None else {
             "value": queries / (e2e_ms * 1e-3), "unit": "queries/s", "h2d_bytes_per_step": h2d_bytes,
@@ -715,9 +895,14 @@ def run_ours(args, dist):
         "clocks": clk,
         "dense": dense,
         "builds_once_after_prefill": builds,
+        **secondary,
     }
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(wl, args.cpu_seconds, workload_label(wl, args.budget))
+        more_k = (secondary["budget_5pct"]["k_top"],) if "budget_5pct" in secondary else ()
+        res["cpu_baseline"], oracle_res = cpu_baseline(wl, args.cpu_seconds, workload_label(wl, args.budget), more_k)
+        if not weighted and not args.no_selection_check:
+            res["selection_check"] = selection_check(wl, oracle_res, idx, nk,
+                                                     s0.get("idx5"), s0.get("nk5"), more_k)
     dist.close()
     return res
 
@@ -733,7 +918,10 @@ def run_reference(args, dist):
     name = args.workload
     # a bounded sample of the same workload: the first sequences of the batch
     nseq = 4
-    wl = W.make(name, "cpu", budget=args.budget, B=nseq)
+    wl = W.make(name, "cpu", budget=args.budget, B=min(nseq, W.make(name, "cpu", materialize=False).B))
+    if args.scorer == "mean16" and wl.score_mode == "summary":
+        wl.score_mode = "summary_mean16"
+    nseq = wl.B
     workers = max(1, min(os.cpu_count() or 1, 32))
     steps = args.steps
     # one step = one (sequence, KV head) decode step; capped so the run stays short
@@ -744,7 +932,7 @@ def run_reference(args, dist):
     n = min(steps, cap)
     if args.warmup:
         time_oracle(wl, min(args.warmup, workers), workers)
-    dt, n = time_oracle(wl, n, workers)
+    dt, n, _ = time_oracle(wl, n, workers)
     queries = n / wl.Hkv
     value = queries / dt
     sample = (f"{n} (sequence, KV head) decode steps = {queries:g} queries from the first {nseq} sequences "

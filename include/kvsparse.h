@@ -399,6 +399,20 @@ kv_status kv_sparse_decode_attn_noalloc(const kv_shape* shape, const void* q, fl
 kv_status kv_selftest_wait_timeout(uint32_t* status, uint32_t* waited_ok, uint64_t limit_ns, int arrive,
                                    kv_stream_t stream);
 
+/*
+ * kv_stream_read -- a measurement reference with no counterpart on the pages:
+ * reads `bytes` from src once, as a plain streaming kernel (16-byte loads, four
+ * in flight per thread, eight 256-thread CTAs per SM) and produces nothing. Timed
+ * like the attention kernel, it gives the time one launch needs just to move the
+ * same number of bytes from HBM, launch and ramp included.
+ *
+ *   src    device, 16-byte aligned; bytes a multiple of 16
+ *   sink   device uint32, 4-byte aligned (written only if the folded words hit a
+ *          fixed constant, so the loads cannot be optimised away)
+ * Asynchronous on `stream`; KV_ERR_INVALID_ARG for bad pointers or sizes.
+ */
+kv_status kv_stream_read(const void* src, size_t bytes, uint32_t* sink, kv_stream_t stream);
+
 /* Message of the last failed call on this host thread ("" if none). */
 const char* kv_last_error(void);
 

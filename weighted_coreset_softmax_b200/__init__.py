@@ -31,6 +31,7 @@ __all__ = [
     "kv_select_blocks_mean16",
     "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace", "kv_selftest_wait_timeout",
+    "kv_stream_read",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
@@ -97,6 +98,7 @@ def lib():
         "kv_workspace_init": [_P, _S, _P],
         "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
         "kv_selftest_wait_timeout": [_P, _P, ctypes.c_uint64, _I, _P],
+        "kv_stream_read": [_P, _S, _P, _P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -497,3 +499,12 @@ def kv_selftest_wait_timeout(status: torch.Tensor, limit_ns: int, arrive: bool) 
     _check(lib().kv_selftest_wait_timeout(_ptr(status), _ptr(ok), ctypes.c_uint64(int(limit_ns)), 1 if arrive else 0,
                                           _stream(status.device)))
     return ok
+
+
+def kv_stream_read(src: torch.Tensor, nbytes: int, sink: torch.Tensor) -> None:
+    """Reads the first nbytes of src once with a plain streaming kernel (a
+    measurement reference: the time one launch needs to move that many bytes)."""
+    _need(sink, "sink", torch.int32)
+    if nbytes > src.numel() * src.element_size():
+        raise ValueError("nbytes exceeds the tensor")
+    _check(lib().kv_stream_read(_ptr(src), ctypes.c_size_t(int(nbytes)), _ptr(sink), _stream(src.device)))

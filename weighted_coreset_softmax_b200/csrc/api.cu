@@ -225,12 +225,15 @@ bool attention_uses_gather() {
   return v;
 }
 
-// Tiled 2-D tensor map over a [rows][D] bf16 cache: boxes of box_rows rows x 64
-// elements (128 bytes; 32 rows for block copies, 1 row for gather4), 128-byte
-// swizzle, zero fill past the last row. Encoded
-// through the driver entry point (no link against the driver library); the last
-// few maps are cached, keyed by address and extent.
-kv_status encode_kv_map(const void* base, uint64_t rows, int D, int box_rows, CUtensorMap* out) {
+// Tiled tensor map over a [rows][D] bf16 cache, 128-byte swizzle, zero fill past
+// the last row. whole_rows == 0: 2-D, boxes of box_rows rows x 64 elements (128
+// bytes; 32 rows for block copies, 1 row for gather4). whole_rows != 0 and D =
+// 128: 3-D with the row's two 128-byte halves as the outermost dimension, so one
+// box of {64, box_rows, 2} lands as two swizzled box_rows x 128-byte tiles, the
+// first half then the second. Encoded through the driver entry point (no link
+// against the driver library); the last few maps are cached, keyed by address,
+// extent and shape.
+kv_status encode_kv_map(const void* base, uint64_t rows, int D, int box_rows, CUtensorMap* out, int whole_rows = 0) {
   using Encode = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -239,14 +242,14 @@ kv_status encode_kv_map(const void* base, uint64_t rows, int D, int box_rows, CU
   struct Entry {
     const void* base;
     uint64_t rows;
-    int D, box_rows;
+    int D, box_rows, whole;
     CUtensorMap map;
   };
   static Entry cache[16];
   static int next_slot = 0;
   std::lock_guard<std::mutex> lock(mu);
   for (const Entry& e : cache)
-    if (e.base == base && e.rows == rows && e.D == D && e.box_rows == box_rows) {
+    if (e.base == base && e.rows == rows && e.D == D && e.box_rows == box_rows && e.whole == whole_rows) {
       *out = e.map;
       return KV_OK;
     }
@@ -257,16 +260,27 @@ kv_status encode_kv_map(const void* base, uint64_t rows, int D, int box_rows, CU
       return fail(KV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
     encode = reinterpret_cast<Encode>(fn);
   }
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
-  const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
-  const cuuint32_t estr[2] = {1, 1};
   CUtensorMap m;
-  const CUresult r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r;
+  if (whole_rows && D == 128) {
+    const cuuint64_t dims[3] = {64, rows, 2};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, 128};
+    const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 2};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  } else {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(D), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(D) * 2};
+    const cuuint32_t box[2] = {64, static_cast<cuuint32_t>(box_rows)};
+    const cuuint32_t estr[2] = {1, 1};
+    r = encode(&m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  }
   if (r != CUDA_SUCCESS) return fail(KV_ERR_CUDA, "tensor map encoding failed (CUresult %d)", static_cast<int>(r));
-  cache[next_slot] = Entry{base, rows, D, box_rows, m};
+  cache[next_slot] = Entry{base, rows, D, box_rows, whole_rows, m};
   next_slot = (next_slot + 1) % 16;
   *out = m;
   return KV_OK;
@@ -410,22 +424,28 @@ kv_status run_attention(const kv_shape* s, const void* q, float scale, const voi
   } else {
     p.part = kvs::make_partition(NBH, P, static_cast<int64_t>(sms) * cps * kvs::ATTN_NW);
   }
+  const bool gather = !fs && use_mma && mode == kvs::ATTN_BLOCKS && s->block_size >= 32 && attention_uses_gather();
+  const int ga_rows = s->block_size >= 64 ? 64 : 32;  // rows a chunk of the warp-specialised kernel
   CUtensorMap tk, tv;
   std::memset(&tk, 0, sizeof(tk));
   std::memset(&tv, 0, sizeof(tv));
   if (use_mma) {
     const uint64_t rows = static_cast<uint64_t>(NBH) * s->Ncap;
     if (rows > 0x7fffffffull) return fail(KV_ERR_UNSUPPORTED, "B * Hkv * Ncap = %llu rows is too many", (unsigned long long)rows);
-    const int box_rows = mode == kvs::ATTN_WEIGHTED ? 1 : 32;  // gather4 needs a one-row box
-    KV_TRY(encode_kv_map(K, rows, s->D, box_rows, &tk));
-    KV_TRY(encode_kv_map(V, rows, s->D, box_rows, &tv));
+    if (gather) {
+      KV_TRY(encode_kv_map(K, rows, s->D, ga_rows, &tk, 1));
+      KV_TRY(encode_kv_map(V, rows, s->D, ga_rows, &tv, 1));
+    } else {
+      const int box_rows = mode == kvs::ATTN_WEIGHTED ? 1 : 32;  // gather4 needs a one-row box
+      KV_TRY(encode_kv_map(K, rows, s->D, box_rows, &tk));
+      KV_TRY(encode_kv_map(V, rows, s->D, box_rows, &tv));
+    }
   }
-  const bool gather = !fs && use_mma && mode == kvs::ATTN_BLOCKS && s->block_size >= 32 && attention_uses_gather();
   cudaError_t e;
   if (gather) {
-    const long long T = static_cast<long long>(NBH) * (kmax > 0 ? kmax : 1) * (s->block_size / 32);
+    const long long T = static_cast<long long>(NBH) * (kmax > 0 ? kmax : 1) * (s->block_size / ga_rows);
     const int grid = static_cast<int>(std::min<long long>(sms, T));
-    e = kvs::launch_gather(s->D, G, p, tk, tv, grid, reinterpret_cast<cudaStream_t>(stream));
+    e = kvs::launch_gather(s->D, G, ga_rows, p, tk, tv, grid, reinterpret_cast<cudaStream_t>(stream));
   } else {
     e = fs ? kvs::launch_fused(s->dtype, s->D, G, p, tk, tv, NBH, reinterpret_cast<cudaStream_t>(stream))
            : kvs::launch_attn(s->dtype, s->D, G, use_mma, p, tk, tv, kvs::part_grid(p.part),

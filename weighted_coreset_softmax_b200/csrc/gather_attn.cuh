@@ -9,17 +9,23 @@
 // of "COBS: Cumulant Order Block Sparse Attention".
 //
 // Design (sm_100a, one CTA per SM).
-//  * Work: every (sequence, KV head) pair ("bh") owns kmax * L / 32 chunk slots
-//    of 32 rows on one axis (kept-block slot j, 32-row half); the axis is cut
-//    into one equal contiguous range per CTA, so every SM streams about the same
-//    bytes. A CTA takes the pairs it shares with its neighbours first, so that
-//    their cross-CTA merges finish while its own pairs still stream.
+//  * Work: every (sequence, KV head) pair ("bh") owns kmax * L / ROWS chunk
+//    slots of ROWS = min(L, 64) rows on one axis (kept-block slot j, part of the
+//    block); the axis is cut into one contiguous range per CTA -- whole pairs when
+//    there are at least as many pairs as CTAs, else an even cut that shares pairs
+//    between CTAs (a CTA then takes its shared pairs first, so that their
+//    cross-CTA merges finish while its own pairs still stream).
 //  * Producer warp: loads the chunk metadata (kept count, block index, sequence
 //    length) 32 chunks per memory round trip, skips empty chunks, and keeps a
-//    ring of NS slots full: per chunk two or four tiled tensor copies (K and V,
-//    32 rows x 128 bytes each, 128-byte swizzle) and one bulk copy of the pair's
-//    q, all counted in bytes on the slot's "full" mbarrier, L2 evict-first.
-//    Copies run ahead of the consumers by up to the whole ring (~190 KB per SM).
+//    ring of NS slots full: per chunk one tensor copy of the ROWS x D key tile and
+//    one of the value tile (128-byte swizzle; for D = 128 a three-dimensional
+//    box takes both 128-byte column halves at once) and one bulk copy of the
+//    pair's q, all counted in bytes on the slot's "full" mbarrier, keys and
+//    values L2 evict-first. A single thread issues every copy, and each copy
+//    instruction costs it tens of nanoseconds, so the copies are as few and as
+//    large as the shared memory allows. It publishes the CTA's chunk count as
+//    soon as its last metadata batch is read, which tells each consumer where
+//    its work ends.
 //  * Consumer warps (NC): issue index i goes to consumer i % NC. A consumer keeps
 //    the online-softmax state of its current pair on the tensor cores (q.k:
 //    mma.sync m16n8k16 with the 16 tokens of a tile as M and the G query heads
@@ -30,31 +36,32 @@
 //    each pair's partial records (and the proxy) with the log-sum-exp merge, and
 //    writes out / lse; a pair shared with other CTAs leaves one record in the
 //    workspace and the last arriving CTA merges them.
+//  * Proxy warp: computes the tail proxies of the CTA's pairs ahead of the merge
+//    warp (their dependent memory round trips stay off every other warp's path).
 // Progress: the producer waits only for ring slots, a consumer only for its next
-// chunk and for its record buffer; with NS >= NC the chunk that lets any consumer
-// flush the pair the merge warp waits for is always already issued. Every wait is
-// bounded (1 s of %globaltimer, then KV_DEV_WAIT_TIMEOUT and give up).
+// chunk and for its record buffers; with NS >= NC the chunk that lets any
+// consumer flush the pair the merge warp waits for is always already issued.
+// Every wait is bounded (1 s of %globaltimer, then KV_DEV_WAIT_TIMEOUT).
 #pragma once
 
 #include "attention.cuh"
 
 namespace kvs {
 
-constexpr int GA_NC = 8;                        // consumer warps
+constexpr int GA_NC = 4;                        // consumer warps
 constexpr int GA_PRODUCER = GA_NC;              // warp indices of the other roles
 constexpr int GA_MERGER = GA_NC + 1;
 constexpr int GA_PROXY = GA_NC + 2;
 constexpr int GA_THREADS = (GA_NC + 3) * 32;
-constexpr int GA_ROWS = 32;                     // rows per chunk (one tensor box)
 constexpr int GA_MAX_SLOTS = 32;
 constexpr int GA_RB = 2;                        // record buffers per consumer
 constexpr int GA_PR = 4;                        // proxy ring entries
 
-template <int D, int G>
+template <int D, int G, int ROWS>
 struct GaCfg {
   static constexpr int RB = D * 2;              // bytes per bf16 row
-  static constexpr int KH = RB / 128;           // 128-byte column boxes per row
-  static constexpr int BOX = GA_ROWS * 128;     // one swizzled box
+  static constexpr int KH = RB / 128;           // 128-byte column halves per row
+  static constexpr int BOX = ROWS * 128;        // one swizzled column half of a tile
   static constexpr int KS = D / 16;             // k-steps of q.k, d-tiles of p.v
   static constexpr int QB = G * RB;             // q of one group
   static constexpr int SL_K = 0;
@@ -80,6 +87,7 @@ struct GaCfg {
   static constexpr int O_BAR = O_HDR + HDR_BYTES;
   static_assert(NS >= GA_NC, "progress needs at least as many ring slots as consumers");
   static_assert(G <= 8 && RB % 128 == 0, "tensor-core consumer: G <= 8, rows of 128-byte boxes");
+  static_assert(ROWS == 32 || ROWS == 64, "chunk rows");
   static_assert(SMEM <= 227 * 1024, "shared memory per CTA");
   // byte offset of 16-byte chunk c of row r in a slot's K or V tiles
   // (128-byte swizzle: chunk c of a 128-byte line sits at c ^ (r mod 8))
@@ -91,20 +99,29 @@ struct GaCfg {
 // Slot header written by the producer (generic stores, published by the slot's
 // full-barrier arrival).
 struct GaHdr {
-  int bh;      // pair of the chunk; -1: end of this consumer's work
-  int nvalid;  // rows that take part (a prefix of the 32)
-  int pad0, pad1;
+  int bh;      // pair of the chunk
+  int nvalid;  // rows that take part (a prefix of the chunk's rows)
+  int idx;     // issue index of the chunk now in the slot (-1: none yet)
+  int pad;
 };
 
 // The CTA's chunk range [x0, x1) of the pair-major chunk axis (PC chunks a pair),
 // in processing order: the pair it shares with the CTA before (segment A), the
-// pair it shares with the CTA after (segment B), then the pairs in between.
+// pair it shares with the CTA after (segment B), then the pairs in between. With
+// at least as many pairs as CTAs the ranges hold whole pairs (pair c * NBH / N
+// up to pair (c + 1) * NBH / N): no pair is shared, so every merge stays in
+// shared memory, and an SM holding one pair more than another still finishes in
+// time because HBM, not the SM, bounds the stream. With fewer pairs the chunk
+// axis is cut evenly and pairs are shared.
+__device__ __forceinline__ int64_t ga_x0(int64_t T, int c, int ncta, int PC, int NBH) {
+  return NBH >= ncta ? static_cast<int64_t>(PC) * (static_cast<int64_t>(NBH) * c / ncta) : T * c / ncta;
+}
 struct GaRange {
   int64_t x0, x1, endA, startB;
   int64_t lenA, lenB;
-  __device__ __forceinline__ void init(int64_t T, int cta, int ncta, int PC) {
-    x0 = T * cta / ncta;
-    x1 = T * (cta + 1) / ncta;
+  __device__ __forceinline__ void init(int64_t T, int cta, int ncta, int PC, int NBH) {
+    x0 = ga_x0(T, cta, ncta, PC, NBH);
+    x1 = ga_x0(T, cta + 1, ncta, PC, NBH);
     const int64_t pA = x0 / PC, pB = (x1 - 1) / PC;
     endA = min(x1, (pA + 1) * PC);
     if (pB != pA) {
@@ -124,7 +141,8 @@ struct GaRange {
   }
 };
 
-// CTA whose range holds chunk x: the largest c with floor(T c / N) <= x.
+// CTA whose range holds chunk x (even cut: the largest c with floor(T c / N) <= x;
+// only used when pairs are shared, i.e. with fewer pairs than CTAs).
 __device__ __forceinline__ int ga_cta_of(int64_t x, int64_t T, int ncta) {
   return static_cast<int>((static_cast<int64_t>(ncta) * (x + 1) + T - 1) / T) - 1;
 }
@@ -137,7 +155,8 @@ struct GaChunk {
   int bh, nvalid;
   int64_t row;  // bh * Ncap + first token
 };
-__device__ __forceinline__ GaChunk ga_chunk(const AttnParams& p, int64_t x, int PC, int CPB, bool in, bool report) {
+__device__ __forceinline__ GaChunk ga_chunk(const AttnParams& p, int64_t x, int PC, int CPB, int ROWS, bool in,
+                                            bool report) {
   GaChunk c;
   c.bh = in ? static_cast<int>(x / PC) : -1;
   c.nvalid = 0;
@@ -164,8 +183,8 @@ __device__ __forceinline__ GaChunk ga_chunk(const AttnParams& p, int64_t x, int 
     if (report) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
     return c;
   }
-  const int tok0 = (blk << p.log2L) + half * GA_ROWS;
-  c.nvalid = max(0, min(GA_ROWS, n - tok0));
+  const int tok0 = (blk << p.log2L) + half * ROWS;
+  c.nvalid = max(0, min(ROWS, n - tok0));
   c.row = static_cast<int64_t>(c.bh) * p.Ncap + tok0;
   return c;
 }
@@ -174,9 +193,9 @@ __device__ __forceinline__ GaChunk ga_chunk(const AttnParams& p, int64_t x, int 
 // Online-softmax state of one consumer warp for one pair (tensor-core layout):
 // lane holds heads h0 = 2 (lane & 3) and h0 + 1; acc[4 k + e] is the fragment of
 // O^T rows 16 k + lane / 4 (+ 8) for those heads.
-template <int D, int G>
+template <int D, int G, int ROWS>
 struct GaState {
-  using C = GaCfg<D, G>;
+  using C = GaCfg<D, G, ROWS>;
   float m[2], l[2];
   float acc[C::KS * 4];
   uint32_t qb[C::KS * 2];  // q^T fragments (B operand of q.k)
@@ -197,11 +216,12 @@ struct GaState {
       qb[2 * k + 1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2) : 0u;
     }
   }
-  // One chunk of nvalid (1..32) rows in slot sl: logits in the log2 domain
-  // (qscale = softmax scale * log2 e), rows >= nvalid masked. The V rows past
-  // nvalid (the next block, or cache rows past the sequence) must have been
-  // zeroed: their p is 0, and 0 times a non-finite pattern would reach acc.
-  __device__ __forceinline__ void consume(const unsigned char* sl, int nvalid, float qscale, int lane) {
+  // Rows rb .. rb + 31 of the chunk in slot sl, of which the first nvalid (1..32)
+  // take part: logits in the log2 domain (qscale = softmax scale * log2 e), rows
+  // >= nvalid masked. The V rows past nvalid (the next block, or cache rows past
+  // the sequence) must have been zeroed: their p is 0, and 0 times a non-finite
+  // pattern would reach acc.
+  __device__ __forceinline__ void consume(const unsigned char* sl, int rb, int nvalid, float qscale, int lane) {
     const uint32_t kbase = smem_u32(sl + C::SL_K);
     const uint32_t vbase = smem_u32(sl + C::SL_V);
     float sc4[2][4], sc4o[2][4];
@@ -209,7 +229,7 @@ struct GaState {
     for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc4[mt][e] = sc4o[mt][e] = 0.f;
-      const int row = 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
+      const int row = rb + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int k = 0; k < C::KS; ++k) {
         uint32_t a[4];
@@ -275,7 +295,7 @@ struct GaState {
     l[1] = l[1] * r1 + ls1;
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
-      const int row = 16 * mt + (lane & 7) + (lane >> 4) * 8;
+      const int row = rb + 16 * mt + (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
       for (int k = 0; k < C::KS; ++k) {
         uint32_t a[4];
@@ -321,13 +341,13 @@ struct GaState {
 };
 
 
-// Zeroes the V rows nvalid..31 of a slot (all column boxes); the caller fences
-// the generic writes against the tensor copies that later refill the slot.
-template <int D, int G>
+// Zeroes the V rows nvalid..ROWS-1 of a slot (both column halves); the caller
+// fences the generic writes against the tensor copies that later refill the slot.
+template <int D, int G, int ROWS>
 __device__ __forceinline__ void ga_zero_tail_rows(unsigned char* sl, int nvalid, int lane) {
-  using C = GaCfg<D, G>;
+  using C = GaCfg<D, G, ROWS>;
   unsigned char* vz = sl + C::SL_V;
-  const int per_box = (GA_ROWS - nvalid) * 8;  // 16-byte pieces past the valid rows
+  const int per_box = (ROWS - nvalid) * 8;  // 16-byte pieces past the valid rows
   for (int e = lane; e < per_box * C::KH; e += 32) {
     const int hx = e / per_box, r = e - hx * per_box;
     *reinterpret_cast<uint4*>(vz + hx * C::BOX + nvalid * 128 + r * 16) = make_uint4(0, 0, 0, 0);
@@ -492,11 +512,61 @@ struct GaMerge {
   }
 };
 
-template <int D, int G>
+// Waits until the chunk with issue index i has landed in its slot: 1, or 0 once
+// *total shows that index i will never be issued, or -1 (and the timeout bit)
+// after WAIT_LIMIT_NS. A parity wait is exact only while the barrier has at most
+// one phase to go before the awaited one; consumers take the slots in turns, so
+// a consumer can arrive at a slot while its previous use (another consumer's
+// chunk) is still in flight. The slot header's issue index closes that gap: once
+// it reads i, the producer has issued this use, which it does only after the
+// previous use was consumed, and the parity wait is then exact.
+__device__ __forceinline__ int ga_wait_chunk(uint64_t* bar, uint32_t parity, const volatile int* total,
+                                             const volatile int* slot_idx, int i, uint32_t* status) {
+  const uint64_t t0 = global_ns();
+  while (true) {
+    if (*slot_idx == i) {
+      uint32_t ok;
+      asm volatile(
+          "{\n\t.reg .pred p;\n\t"
+          "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+          "selp.u32 %0, 1, 0, p;\n\t}"
+          : "=r"(ok)
+          : "r"(smem_u32(bar)), "r"(parity), "r"(2000u)
+          : "memory");
+      if (ok) return 1;  // the chunk landed
+    } else if (i >= *total) {
+      return 0;  // no such chunk: this consumer's work is done
+    } else {
+      __nanosleep(64);
+    }
+    if (global_ns() - t0 > WAIT_LIMIT_NS) {
+      atomicOr(status, KV_DEV_WAIT_TIMEOUT);
+      return -1;
+    }
+  }
+}
+
+// One tile (ROWS rows x D) of K or V into its 128-byte-swizzled slot region:
+// D = 128 takes both column halves with one three-dimensional box, D = 64 is one
+// two-dimensional box.
+template <int D>
+__device__ __forceinline__ void ga_load_tile(void* dst, const CUtensorMap* m, int row, uint64_t* bar, uint64_t pol) {
+  if constexpr (D == 128) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(0), "r"(row), "r"(0), "r"(smem_u32(bar)), "l"(pol)
+        : "memory");
+  } else {
+    tma_load_2d(dst, m, 0, row, bar, pol);
+  }
+}
+
+template <int D, int G, int ROWS>
 __global__ void __launch_bounds__(GA_THREADS, 1)
     gather_attn_kernel(const AttnParams p, const __grid_constant__ CUtensorMap tmK,
                        const __grid_constant__ CUtensorMap tmV) {
-  using C = GaCfg<D, G>;
+  using C = GaCfg<D, G, ROWS>;
   constexpr int VEC = D / 32;
   extern __shared__ __align__(1024) unsigned char ga_smem_raw[];
   unsigned char* smem = ga_smem_raw + ((1024u - (smem_u32(ga_smem_raw) & 1023u)) & 1023u);
@@ -512,12 +582,13 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
   };
   auto px_buf = [&](int e) -> float* { return reinterpret_cast<float*>(smem + C::O_PX + e * C::PX_BYTES); };
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int CPB = p.L / GA_ROWS;                     // chunks per kept block
+  const int CPB = p.L / ROWS;                        // chunks per kept block
   const int PC = (p.kmax > 0 ? p.kmax : 1) * CPB;    // chunks per pair
-  const int64_t T = static_cast<int64_t>(p.B) * p.Hkv * PC;
+  const int NBH = p.B * p.Hkv;
+  const int64_t T = static_cast<int64_t>(NBH) * PC;
   const int cta = blockIdx.x, ncta = gridDim.x;
   GaRange rg;
-  rg.init(T, cta, ncta, PC);
+  rg.init(T, cta, ncta, PC, NBH);
   // the CTA's pairs in processing order: pA, then pB (if another pair), then the
   // pairs between them
   const int64_t pA = rg.x0 / PC, pB = (rg.x1 - 1) / PC;
@@ -525,7 +596,8 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
   auto pair_at = [&](int64_t k) -> int64_t { return k == 0 ? pA : (k == 1 ? pB : pA + k - 1); };
   auto owns = [&](int64_t bh) { const int64_t ps = bh * PC; return ps >= rg.x0 && ps < rg.x1; };
   const bool proxy_on = p.use_proxy != 0;
-  __shared__ int prod_issued;  // ring uses the producer armed (for the drain at the end)
+  __shared__ int prod_issued;       // ring uses the producer armed (for the drain at the end)
+  __shared__ volatile int total;    // chunks this CTA issues, once the producer knows it
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::NS; ++s) {
@@ -541,7 +613,9 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
       mbar_init(px_empty + e, 1);
     }
     fence_mbar_init();
+    for (int s = 0; s < GA_MAX_SLOTS; ++s) hdr[s].idx = -1;
     prod_issued = 0;
+    total = INT_MAX;
   }
   __syncthreads();
 
@@ -565,8 +639,15 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
     const int64_t len = rg.len();
     for (int64_t k0 = 0; k0 < len && ok; k0 += 32) {
       const bool in = k0 + lane < len;
-      const GaChunk ch = ga_chunk(p, in ? rg.x_at(k0 + lane) : 0, PC, CPB, in, true);
+      const GaChunk ch = ga_chunk(p, in ? rg.x_at(k0 + lane) : 0, PC, CPB, ROWS, in, true);
       const int cnt = static_cast<int>(min(static_cast<int64_t>(32), len - k0));
+      if (k0 + 32 >= len) {
+        // the last batch: publish how many chunks this CTA issues in all, before
+        // any of them is issued (no consumer has reached its end yet)
+        const int nval = __popc(__ballot_sync(FULL_MASK, ch.nvalid > 0));
+        if (lane == 0) total = issued + nval;
+        __syncwarp();
+      }
       for (int t = 0; t < cnt; ++t) {
         const int nv = __shfl_sync(FULL_MASK, ch.nvalid, t);
         if (nv <= 0) continue;
@@ -577,14 +658,12 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
         if (lane == 0) {
           hdr[s].bh = cbh;
           hdr[s].nvalid = nv;
+          *reinterpret_cast<volatile int*>(&hdr[s].idx) = issued;
           unsigned char* sl = smem + s * C::SLOT;
           mbar_arrive_expect_tx(full + s, C::SLOT_TX);
           const int y = static_cast<int>(row);
-#pragma unroll
-          for (int hx = 0; hx < C::KH; ++hx) {
-            tma_load_2d(sl + C::SL_K + hx * C::BOX, &tmK, hx * 64, y, full + s, pol);
-            tma_load_2d(sl + C::SL_V + hx * C::BOX, &tmV, hx * 64, y, full + s, pol);
-          }
+          ga_load_tile<D>(sl + C::SL_K, &tmK, y, full + s, pol);
+          ga_load_tile<D>(sl + C::SL_V, &tmV, y, full + s, pol);
           const int b = cbh / p.Hkv, h = cbh - b * p.Hkv;
           bulk_g2s(sl + C::SL_Q, Qg + (static_cast<size_t>(b) * p.Hq + h * G) * C::RB, C::QB, full + s, qpol);
         }
@@ -592,23 +671,13 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
         ++issued;
       }
     }
-    // one end marker per consumer (issue indices issued .. issued + NC - 1); after
-    // a timed-out wait none is sent (the consumers' own bounded waits end them)
-    for (int t = 0; t < GA_NC && ok; ++t) {
-      const int s = take_slot(issued);
-      if (!ok) break;
-      if (lane == 0) {
-        hdr[s].bh = -1;
-        hdr[s].nvalid = 0;
-        mbar_arrive(full + s);
-      }
-      __syncwarp();
-      ++issued;
+    if (lane == 0) {
+      prod_issued = issued;
+      total = issued;  // after a timed-out wait: what was issued
     }
-    if (lane == 0) prod_issued = issued;
   } else if (warp < GA_NC) {
     // ================================================================ consumer
-    GaState<D, G> st;
+    GaState<D, G, ROWS> st;
     st.reset();
     int cur = -1;
     int flushes = 0;
@@ -625,8 +694,13 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
     };
     for (int i = warp;; i += GA_NC) {
       const int s = i % C::NS;
-      if (ok && !mbar_wait(full + s, static_cast<uint32_t>(i / C::NS) & 1u, p.status)) ok = false;
-      const int bh = ok ? hdr[s].bh : -1;
+      int got = 0;
+      if (ok) {
+        got = ga_wait_chunk(full + s, static_cast<uint32_t>(i / C::NS) & 1u, &total,
+                            reinterpret_cast<volatile int*>(&hdr[s].idx), i, p.status);
+        if (got < 0) ok = false;
+      }
+      const int bh = got > 0 ? hdr[s].bh : -1;
       const int nv = hdr[s].nvalid;
       unsigned char* sl = smem + s * C::SLOT;
       if (bh != cur) {
@@ -637,12 +711,14 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
           st.load_q(sl + C::SL_Q, lane);
         }
       }
-      if (bh < 0) break;  // end marker (or a timed-out wait)
-      if (nv < GA_ROWS) {
-        ga_zero_tail_rows<D, G>(sl, nv, lane);
+      if (bh < 0) break;  // past this consumer's last chunk (or a timed-out wait)
+      if (nv < ROWS) {
+        ga_zero_tail_rows<D, G, ROWS>(sl, nv, lane);
         __syncwarp();
       }
-      st.consume(sl, nv, p.qscale, lane);
+#pragma unroll
+      for (int r0 = 0; r0 < ROWS; r0 += 32)
+        if (nv > r0) st.consume(sl, r0, min(32, nv - r0), p.qscale, lane);
       // the slot is free: order these reads before the copies that refill it
       __syncwarp();
       fence_proxy_async_smem();
@@ -735,7 +811,7 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
       __threadfence();
       mg.reset();
       for (int c = cf; c <= cl; ++c) {
-        const int64_t cx0 = T * c / ncta;
+        const int64_t cx0 = ga_x0(T, c, ncta, PC, NBH);
         const int cside = (static_cast<int64_t>(bh) == cx0 / PC) ? 0 : 1;
         mg.fold_record(p.recs + static_cast<size_t>(2 * c + cside) * C::RECF, lane, true);
       }
@@ -743,7 +819,7 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
     };
     for (int64_t k0 = 0; k0 < len; k0 += 32) {
       const bool in = k0 + lane < len;
-      const GaChunk ch = ga_chunk(p, in ? rg.x_at(k0 + lane) : 0, PC, CPB, in, false);
+      const GaChunk ch = ga_chunk(p, in ? rg.x_at(k0 + lane) : 0, PC, CPB, ROWS, in, false);
       const int cnt = static_cast<int>(min(static_cast<int64_t>(32), len - k0));
       for (int t = 0; t < cnt; ++t) {
         const int cbh = __shfl_sync(FULL_MASK, ch.bh, t);

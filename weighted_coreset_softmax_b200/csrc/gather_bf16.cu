@@ -1,5 +1,5 @@
 // Launchers of the warp-specialised block-mode attention kernel (bf16 caches,
-// D in {64, 128}, G in 1..8).
+// D in {64, 128}, G in 1..8, chunks of 32 or 64 rows).
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -8,16 +8,16 @@
 
 namespace kvs {
 
-template <int D, int G>
+template <int D, int G, int ROWS>
 static cudaError_t gather_launch_one(const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                                      cudaStream_t st) {
-  using C = GaCfg<D, G>;
+  using C = GaCfg<D, G, ROWS>;
   static std::atomic<int> configured{0};  // one bit per device: smem limit raised
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured.load() & (1 << (dev & 31)))) {
     const cudaError_t e =
-        cudaFuncSetAttribute(gather_attn_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+        cudaFuncSetAttribute(gather_attn_kernel<D, G, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     configured.fetch_or(1 << (dev & 31));
   }
@@ -31,30 +31,32 @@ static cudaError_t gather_launch_one(const AttnParams& p, const CUtensorMap& tk,
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t le = cudaLaunchKernelEx(&cfg, gather_attn_kernel<D, G>, p, tk, tv);
+  const cudaError_t le = cudaLaunchKernelEx(&cfg, gather_attn_kernel<D, G, ROWS>, p, tk, tv);
   if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 
-template <int D>
+template <int D, int ROWS>
 static cudaError_t gather_launch_d(int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
                                    cudaStream_t st) {
   switch (G) {
-    case 1: return gather_launch_one<D, 1>(p, tk, tv, grid, st);
-    case 2: return gather_launch_one<D, 2>(p, tk, tv, grid, st);
-    case 3: return gather_launch_one<D, 3>(p, tk, tv, grid, st);
-    case 4: return gather_launch_one<D, 4>(p, tk, tv, grid, st);
-    case 5: return gather_launch_one<D, 5>(p, tk, tv, grid, st);
-    case 6: return gather_launch_one<D, 6>(p, tk, tv, grid, st);
-    case 7: return gather_launch_one<D, 7>(p, tk, tv, grid, st);
-    case 8: return gather_launch_one<D, 8>(p, tk, tv, grid, st);
+    case 1: return gather_launch_one<D, 1, ROWS>(p, tk, tv, grid, st);
+    case 2: return gather_launch_one<D, 2, ROWS>(p, tk, tv, grid, st);
+    case 3: return gather_launch_one<D, 3, ROWS>(p, tk, tv, grid, st);
+    case 4: return gather_launch_one<D, 4, ROWS>(p, tk, tv, grid, st);
+    case 5: return gather_launch_one<D, 5, ROWS>(p, tk, tv, grid, st);
+    case 6: return gather_launch_one<D, 6, ROWS>(p, tk, tv, grid, st);
+    case 7: return gather_launch_one<D, 7, ROWS>(p, tk, tv, grid, st);
+    case 8: return gather_launch_one<D, 8, ROWS>(p, tk, tv, grid, st);
     default: return cudaErrorInvalidValue;
   }
 }
 
-cudaError_t launch_gather(int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                          cudaStream_t st) {
-  return D == 64 ? gather_launch_d<64>(G, p, tk, tv, grid, st) : gather_launch_d<128>(G, p, tk, tv, grid, st);
+cudaError_t launch_gather(int D, int G, int rows, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                          int grid, cudaStream_t st) {
+  if (rows == 64)
+    return D == 64 ? gather_launch_d<64, 64>(G, p, tk, tv, grid, st) : gather_launch_d<128, 64>(G, p, tk, tv, grid, st);
+  return D == 64 ? gather_launch_d<64, 32>(G, p, tk, tv, grid, st) : gather_launch_d<128, 32>(G, p, tk, tv, grid, st);
 }
 
 }  // namespace kvs

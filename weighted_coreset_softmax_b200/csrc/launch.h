@@ -23,9 +23,10 @@ bool fused_fits(int dtype, int D, int G, int NBcap);
 cudaError_t launch_fused(int dtype, int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                          int grid, cudaStream_t st);
 // Warp-specialised block-mode attention (bf16, tensor cores, block size >= 32):
-// one CTA per SM, grid <= number of SMs.
-cudaError_t launch_gather(int D, int G, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv, int grid,
-                          cudaStream_t st);
+// one CTA per SM, grid <= number of SMs; rows = min(block size, 64) a chunk, with
+// tensor maps whose boxes are one rows x D tile (3-D for D = 128).
+cudaError_t launch_gather(int D, int G, int rows, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                          int grid, cudaStream_t st);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,

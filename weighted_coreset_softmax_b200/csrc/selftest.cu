@@ -59,3 +59,48 @@ extern "C" kv_status kv_selftest_wait_timeout(uint32_t* status, uint32_t* waited
   }
   return KV_OK;
 }
+
+namespace kvs {
+// Streams `n16` 16-byte words from src with four loads in flight per thread and
+// folds them into one word (so the loads cannot be dropped); the word lands in
+// *sink only in the impossible case that it equals a fixed constant.
+__global__ void __launch_bounds__(256) stream_read_kernel(const uint4* __restrict__ src, size_t n16,
+                                                          uint32_t* sink) {
+  size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  uint32_t acc = 0;
+  for (; i + 3 * stride < n16; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldcs(src + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) acc ^= v[u].x ^ v[u].y ^ v[u].z ^ v[u].w;
+  }
+  for (; i < n16; i += stride) {
+    const uint4 v = __ldcs(src + i);
+    acc ^= v.x ^ v.y ^ v.z ^ v.w;
+  }
+  if (acc == 0x9e3779b9u) *sink = acc;
+}
+}  // namespace kvs
+
+extern "C" kv_status kv_stream_read(const void* src, size_t bytes, uint32_t* sink, kv_stream_t stream) {
+  if (!src || !sink || (reinterpret_cast<uintptr_t>(src) & 15u) || (reinterpret_cast<uintptr_t>(sink) & 3u) ||
+      (bytes & 15u)) {
+    kvs::set_last_error("kv_stream_read: src must be 16-byte aligned, sink 4-byte aligned, bytes a multiple of 16");
+    return KV_ERR_INVALID_ARG;
+  }
+  if (bytes == 0) return KV_OK;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    kvs::set_last_error("kv_stream_read: no CUDA device");
+    return KV_ERR_CUDA;
+  }
+  kvs::stream_read_kernel<<<sms * 8, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint4*>(src), bytes / 16, sink);
+  if (cudaGetLastError() != cudaSuccess) {
+    kvs::set_last_error("kv_stream_read: launch failed");
+    return KV_ERR_CUDA;
+  }
+  return KV_OK;
+}
