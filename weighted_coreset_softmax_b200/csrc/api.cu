@@ -214,13 +214,13 @@ bool attention_uses_tensor_cores() {
 
 // Block-mode attention over a bf16 cache with block size >= 32 runs the
 // warp-specialised kernel (one CTA per SM, a producer warp streaming the kept
-// chunks far ahead of eight tensor-core consumer warps) when the environment
-// variable KVSPARSE_ATTN=v2 asks for it (read once per process); otherwise, and
-// for other modes and shapes, the per-worker-ring kernel runs.
+// chunks ahead of the tensor-core consumer warps) unless the environment
+// variable KVSPARSE_ATTN is "v1" (or "fma"), which selects the per-worker-ring
+// kernel (read once per process); other modes and shapes always run the latter.
 bool attention_uses_gather() {
   static const bool v = [] {
     const char* e = std::getenv("KVSPARSE_ATTN");
-    return e && std::strcmp(e, "v2") == 0;
+    return !(e && (std::strcmp(e, "v1") == 0 || std::strcmp(e, "fma") == 0));
   }();
   return v;
 }

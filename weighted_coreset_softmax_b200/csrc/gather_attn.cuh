@@ -26,7 +26,7 @@
 //    large as the shared memory allows. It publishes the CTA's chunk count as
 //    soon as its last metadata batch is read, which tells each consumer where
 //    its work ends.
-//  * Consumer warps (NC): issue index i goes to consumer i % NC. A consumer keeps
+//  * Consumer warps (NC = 3): issue index i goes to consumer i % NC. A consumer keeps
 //    the online-softmax state of its current pair on the tensor cores (q.k:
 //    mma.sync m16n8k16 with the 16 tokens of a tile as M and the G query heads
 //    as N; p.v: P split into a bf16 high part and remainder), and writes one
@@ -48,11 +48,16 @@
 
 namespace kvs {
 
-constexpr int GA_NC = 4;                        // consumer warps
-constexpr int GA_PRODUCER = GA_NC;              // warp indices of the other roles
-constexpr int GA_MERGER = GA_NC + 1;
-constexpr int GA_PROXY = GA_NC + 2;
-constexpr int GA_THREADS = (GA_NC + 3) * 32;
+// Warp roles. Warp w runs on scheduler partition w % 4; the consumers' tensor-core
+// work slows every warp that shares their partition, so the producer and the
+// merge warp get partition 3 to themselves (warps 3 and 7), the consumers are
+// warps 0..2 and the proxy warp (memory round trips, few instructions) shares
+// partition 2. Warps 4 and 5 have no role.
+constexpr int GA_NC = 3;                        // consumer warps (warps 0 .. GA_NC - 1)
+constexpr int GA_PRODUCER = 3;
+constexpr int GA_PROXY = 6;
+constexpr int GA_MERGER = 7;
+constexpr int GA_THREADS = 8 * 32;
 constexpr int GA_MAX_SLOTS = 32;
 constexpr int GA_RB = 2;                        // record buffers per consumer
 constexpr int GA_PR = 4;                        // proxy ring entries
@@ -76,7 +81,9 @@ struct GaCfg {
   static constexpr int HDR_BYTES = GA_MAX_SLOTS * 16;      // per slot: bh, nvalid, tag
   static constexpr int BAR_BYTES = (2 * GA_MAX_SLOTS + 2 * GA_NC * GA_RB + 2 * GA_PR) * 8;
   static constexpr int FIXED = GA_NC * GA_RB * REC_BYTES + GA_PR * PX_BYTES + HDR_BYTES + BAR_BYTES;
-  static constexpr int BUDGET = 227 * 1024 - 1024 - 64;    // minus the alignment slack and static smem
+  // the opt-in per-block limit (227 KB) minus the base-alignment slack, 1 KB of
+  // margin and the static variables
+  static constexpr int BUDGET = 227 * 1024 - 2 * 1024 - 64;
   static constexpr int NS0 = (BUDGET - FIXED) / SLOT;
   static constexpr int NS = NS0 > GA_MAX_SLOTS ? GA_MAX_SLOTS : NS0;
   static constexpr int SMEM = NS * SLOT + FIXED + 1024;
@@ -216,22 +223,29 @@ struct GaState {
       qb[2 * k + 1] = hq < G ? *reinterpret_cast<const uint32_t*>(qrow + (d0 + 8) * 2) : 0u;
     }
   }
-  // Rows rb .. rb + 31 of the chunk in slot sl, of which the first nvalid (1..32)
+  // Rows rb .. rb + 16 MT - 1 of the chunk in slot sl, of which the first nvalid
   // take part: logits in the log2 domain (qscale = softmax scale * log2 e), rows
-  // >= nvalid masked. The V rows past nvalid (the next block, or cache rows past
-  // the sequence) must have been zeroed: their p is 0, and 0 times a non-finite
-  // pattern would reach acc.
+  // >= nvalid masked. The MT tiles of 16 rows go through the tensor cores
+  // together (independent accumulation chains) and share one softmax update. The
+  // V rows past nvalid (the next block, or cache rows past the sequence) must
+  // have been zeroed: their p is 0, and 0 times a non-finite pattern would reach
+  // acc.
+  template <int MT>
   __device__ __forceinline__ void consume(const unsigned char* sl, int rb, int nvalid, float qscale, int lane) {
     const uint32_t kbase = smem_u32(sl + C::SL_K);
     const uint32_t vbase = smem_u32(sl + C::SL_V);
-    float sc4[2][4], sc4o[2][4];
+    // S^T = K q^T: rows t = 16 mt + lane / 4 (+ 8), heads h0, h0 + 1; even and
+    // odd k-steps accumulate separately (shorter dependency chains)
+    float sc4[MT][4], sc4o[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < MT; ++mt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sc4[mt][e] = sc4o[mt][e] = 0.f;
-      const int row = rb + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int k = 0; k < C::KS; ++k) {
+    for (int k = 0; k < C::KS; ++k) {
+#pragma unroll
+      for (int mt = 0; mt < MT; ++mt) {
+        const int row = rb + 16 * mt + (lane & 7) + ((lane >> 3) & 1) * 8;
         uint32_t a[4];
         ldsm_x4(kbase + C::swz(row, 2 * k + (lane >> 4)), a);
         if (k & 1)
@@ -239,19 +253,17 @@ struct GaState {
         else
           mma_bf16(sc4[mt][0], sc4[mt][1], sc4[mt][2], sc4[mt][3], a, qb[2 * k], qb[2 * k + 1]);
       }
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sc4[mt][e] += sc4o[mt][e];
     }
     const int tr = lane >> 2;
-    float x[2][4];
+    float x[MT][4];
     float cm0 = -INFINITY, cm1 = -INFINITY;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
       const bool va = 16 * mt + tr < nvalid, vb = 16 * mt + tr + 8 < nvalid;
-      x[mt][0] = va ? sc4[mt][0] * qscale : -INFINITY;
-      x[mt][1] = va ? sc4[mt][1] * qscale : -INFINITY;
-      x[mt][2] = vb ? sc4[mt][2] * qscale : -INFINITY;
-      x[mt][3] = vb ? sc4[mt][3] * qscale : -INFINITY;
+      x[mt][0] = va ? (sc4[mt][0] + sc4o[mt][0]) * qscale : -INFINITY;
+      x[mt][1] = va ? (sc4[mt][1] + sc4o[mt][1]) * qscale : -INFINITY;
+      x[mt][2] = vb ? (sc4[mt][2] + sc4o[mt][2]) * qscale : -INFINITY;
+      x[mt][3] = vb ? (sc4[mt][3] + sc4o[mt][3]) * qscale : -INFINITY;
       cm0 = fmaxf(cm0, fmaxf(x[mt][0], x[mt][2]));
       cm1 = fmaxf(cm1, fmaxf(x[mt][1], x[mt][3]));
     }
@@ -275,10 +287,11 @@ struct GaState {
         acc[4 * k + 3] *= r1;
       }
     }
+    // P as the B operand of p.v: a bf16 high part and the bf16 remainder
     float ls0 = 0.f, ls1 = 0.f;
-    uint32_t bh_[2][2], bl_[2][2];
+    uint32_t bh_[MT][2], bl_[MT][2];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
+    for (int mt = 0; mt < MT; ++mt) {
       const float p0 = fast_exp2(x[mt][0] - ms0), p1 = fast_exp2(x[mt][1] - ms1);
       const float p2 = fast_exp2(x[mt][2] - ms0), p3 = fast_exp2(x[mt][3] - ms1);
       ls0 += p0 + p2;
@@ -293,11 +306,12 @@ struct GaState {
     }
     l[0] = l[0] * r0 + ls0;
     l[1] = l[1] * r1 + ls1;
+    // O^T += V^T P over the MT token tiles
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt) {
-      const int row = rb + 16 * mt + (lane & 7) + (lane >> 4) * 8;
+    for (int k = 0; k < C::KS; ++k) {
 #pragma unroll
-      for (int k = 0; k < C::KS; ++k) {
+      for (int mt = 0; mt < MT; ++mt) {
+        const int row = rb + 16 * mt + (lane & 7) + (lane >> 4) * 8;
         uint32_t a[4];
         ldsm_x4_trans(vbase + C::swz(row, 2 * k + ((lane >> 3) & 1)), a);
         mma_bf16(acc[4 * k], acc[4 * k + 1], acc[4 * k + 2], acc[4 * k + 3], a, bh_[mt][0], bh_[mt][1]);
@@ -360,32 +374,49 @@ __device__ __forceinline__ void ga_zero_tail_rows(unsigned char* sl, int nvalid,
 // scale * log2(e) * q . (mean unread key) + log2(unread count); -inf when every
 // token is kept. The unread sums are the totals minus the kept blocks' sums.
 // Kept indices are checked (in [0, nbv), ascending); a bad one is left out and
-// flags KV_DEV_BAD_BLOCK_INDEX. Four kept rows of sums are in flight at a time
-// and q is read only after the sums, to keep the merge warp's registers low.
+// flags KV_DEV_BAD_BLOCK_INDEX. Two dependent memory round trips (up to 32 kept
+// blocks): the indices with the totals and q, then the kept blocks' counts and
+// sums, eight rows in flight; under a saturated HBM each round trip costs
+// microseconds, and the merge of the CTA's last pair waits for this value.
 template <int D, int G>
 __device__ void ga_proxy(const AttnParams& p, int bh, int lane, float (&vb)[D / 32], float (&pm)[G]) {
   constexpr int VEC = D / 32;
-  constexpr int UNR = 4;
+  constexpr int UNR = 8;  // kept rows of sums in flight together
   const int b = bh / p.Hkv;
+  const int32_t* idx = p.block_idx + static_cast<size_t>(bh) * p.kmax;
+  // first round trip: everything that does not depend on the kept indices
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nk = max(0, min(p.n_kept[bh], p.kmax));
+  const int first32 = lane < p.kmax ? idx[lane] : INT_MAX;
+  float kt[VEC], vt[VEC], qv[G][VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    kt[v] = p.k_tot[static_cast<size_t>(bh) * D + lane * VEC + v];
+    vt[v] = p.v_tot[static_cast<size_t>(bh) * D + lane * VEC + v];
+  }
+  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.Hq +
+                                                                          (bh - b * p.Hkv) * G) * D + lane * VEC;
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) qv[g][v] = __bfloat162float(qrow[g * D + v]);
   const int nbv = (n + p.L - 1) >> p.log2L;
   float ks[VEC], vs[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) ks[v] = vs[v] = 0.f;
   int cnt = 0;
   int prev = -1;
-  const int32_t* idx = p.block_idx + static_cast<size_t>(bh) * p.kmax;
+  // second round trip (per 32 kept blocks): their counts and sums together
   for (int s0 = 0; s0 < nk; s0 += 32) {
     const bool in_list = s0 + lane < nk;
-    const int mine = in_list ? idx[s0 + lane] : INT_MAX;
+    const int mine = in_list ? (s0 == 0 ? first32 : idx[s0 + lane]) : INT_MAX;
     int before = __shfl_up_sync(FULL_MASK, mine, 1);
     if (lane == 0) before = prev;
     const bool ok = in_list && mine >= 0 && mine < nbv && mine > before;
     if (__any_sync(FULL_MASK, in_list && !ok) && lane == 0) atomicOr(p.status, KV_DEV_BAD_BLOCK_INDEX);
     const unsigned okmask = __ballot_sync(FULL_MASK, ok);
     prev = __shfl_sync(FULL_MASK, mine, 31);
-    cnt += __reduce_add_sync(FULL_MASK, ok ? p.counts[static_cast<size_t>(b) * p.NBcap + mine] : 0);
+    const int c = ok ? p.counts[static_cast<size_t>(b) * p.NBcap + mine] : 0;
     const int lim = min(32, nk - s0);
     for (int j0 = 0; j0 < lim; j0 += UNR) {
       float kr[UNR][VEC], vr[UNR][VEC];
@@ -409,6 +440,7 @@ __device__ void ga_proxy(const AttnParams& p, int bh, int lane, float (&vb)[D / 
           vs[v] += vr[u][v];
         }
     }
+    cnt += __reduce_add_sync(FULL_MASK, c);
   }
   const int nT = n - cnt;
   if (nT <= 0) {
@@ -422,17 +454,15 @@ __device__ void ga_proxy(const AttnParams& p, int bh, int lane, float (&vb)[D / 
   float kb[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) {
-    kb[v] = (p.k_tot[static_cast<size_t>(bh) * D + lane * VEC + v] - ks[v]) * inv;
-    vb[v] = (p.v_tot[static_cast<size_t>(bh) * D + lane * VEC + v] - vs[v]) * inv;
+    kb[v] = (kt[v] - ks[v]) * inv;
+    vb[v] = (vt[v] - vs[v]) * inv;
   }
   const float lc = log2f(static_cast<float>(nT));
-  const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + (static_cast<size_t>(b) * p.Hq +
-                                                                          (bh - b * p.Hkv) * G) * D + lane * VEC;
 #pragma unroll
   for (int g = 0; g < G; ++g) {
     float d = 0.f;
 #pragma unroll
-    for (int v = 0; v < VEC; ++v) d = fmaf(__bfloat162float(qrow[g * D + v]), kb[v], d);
+    for (int v = 0; v < VEC; ++v) d = fmaf(qv[g][v], kb[v], d);
     pm[g] = warp_sum(d) * p.qscale + lc;
   }
 }
@@ -480,6 +510,54 @@ struct GaMerge {
         l = rec[G * D + G + g];
       }
       fold(g, m, l, x);
+    }
+  }
+  // Folds up to N records of shared memory at once (rec[t] for t < n): the
+  // maxima and sums first, then each lane's channels with 16-byte loads.
+  template <int N>
+  __device__ __forceinline__ void fold_records(const float* const (&rec)[N], int n, int lane) {
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      float mt[N], lt[N];
+      float Mn = M[g];
+#pragma unroll
+      for (int t = 0; t < N; ++t) {
+        mt[t] = t < n ? rec[t][G * D + g] : -INFINITY;
+        lt[t] = t < n ? rec[t][G * D + G + g] : 0.f;
+        Mn = fmaxf(Mn, mt[t]);
+      }
+      if (Mn == -INFINITY) continue;
+      const float a = fast_exp2(M[g] - Mn);
+      float wt[N];
+      float Lsum = Ls[g] * a;
+#pragma unroll
+      for (int t = 0; t < N; ++t) {
+        wt[t] = mt[t] == -INFINITY ? 0.f : fast_exp2(mt[t] - Mn);
+        Lsum = fmaf(wt[t], lt[t], Lsum);
+      }
+      float x[VEC];
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) x[v] = acc[g][v] * a;
+#pragma unroll
+      for (int t = 0; t < N; ++t) {
+        if (t < n) {
+          const float* r = rec[t] + g * D + lane * VEC;
+          if constexpr (VEC == 4) {
+            const float4 f = *reinterpret_cast<const float4*>(r);
+            x[0] = fmaf(wt[t], f.x, x[0]);
+            x[1] = fmaf(wt[t], f.y, x[1]);
+            x[2] = fmaf(wt[t], f.z, x[2]);
+            x[3] = fmaf(wt[t], f.w, x[3]);
+          } else {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) x[v] = fmaf(wt[t], r[v], x[v]);
+          }
+        }
+      }
+#pragma unroll
+      for (int v = 0; v < VEC; ++v) acc[g][v] = x[v];
+      Ls[g] = Lsum;
+      M[g] = Mn;
     }
   }
   __device__ __forceinline__ void write_record(float* rec, int lane) const {
@@ -716,9 +794,10 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
         ga_zero_tail_rows<D, G, ROWS>(sl, nv, lane);
         __syncwarp();
       }
-#pragma unroll
-      for (int r0 = 0; r0 < ROWS; r0 += 32)
-        if (nv > r0) st.consume(sl, r0, min(32, nv - r0), p.qscale, lane);
+      if (ROWS == 64 && nv > 32)
+        st.template consume<ROWS / 16>(sl, 0, nv, p.qscale, lane);
+      else
+        st.template consume<2>(sl, 0, nv, p.qscale, lane);
       // the slot is free: order these reads before the copies that refill it
       __syncwarp();
       fence_proxy_async_smem();
@@ -751,7 +830,7 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
         ++e;
       }
     }
-  } else {
+  } else if (warp == GA_MERGER) {
     // ================================================================ merge warp
     grid_dep_wait();
     uint32_t taken = 0;  // records taken per consumer (bits 4w..4w+3, modulo 16)
@@ -765,17 +844,8 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
       const bool shared = ps < rg.x0 || pe > rg.x1;
       GaMerge<D, G> mg;
       mg.reset();
-      const int nrec = min(GA_NC, cnt);
-      for (int t = 0; t < nrec; ++t) {
-        const int w = (first + t) % GA_NC;
-        const int tk = static_cast<int>((taken >> (4 * w)) & 15u);
-        const int k = tk % GA_RB;
-        if (ok && !mbar_wait(rec_full + w * GA_RB + k, static_cast<uint32_t>(tk / GA_RB) & 1u, p.status)) ok = false;
-        mg.fold_record(rec_buf(w, k), lane, false);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(rec_empty + w * GA_RB + k);
-        taken = (taken & ~(15u << (4 * w))) | (static_cast<uint32_t>((tk + 1) & 15) << (4 * w));
-      }
+      // the proxy (computed ahead by the proxy warp), then every record of the
+      // pair; all of them are folded in one pass once they are there
       if (proxy_on && owns(bh)) {
         const int slot = pxe % GA_PR;
         if (ok && !mbar_wait(px_full + slot, static_cast<uint32_t>(pxe / GA_PR) & 1u, p.status)) ok = false;
@@ -788,6 +858,31 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(px_empty + slot);
         ++pxe;
+      }
+      const int nrec = min(GA_NC, cnt);
+      const float* recp[GA_NC];
+#pragma unroll
+      for (int t = 0; t < GA_NC; ++t) {
+        recp[t] = nullptr;
+        if (t < nrec) {
+          const int w = (first + t) % GA_NC;
+          const int tk = static_cast<int>((taken >> (4 * w)) & 15u);
+          const int k = tk % GA_RB;
+          if (ok && !mbar_wait(rec_full + w * GA_RB + k, static_cast<uint32_t>(tk / GA_RB) & 1u, p.status))
+            ok = false;
+          recp[t] = rec_buf(w, k);
+        }
+      }
+      mg.template fold_records<GA_NC>(recp, nrec, lane);
+      __syncwarp();
+#pragma unroll
+      for (int t = 0; t < GA_NC; ++t) {
+        if (t < nrec) {
+          const int w = (first + t) % GA_NC;
+          const int tk = static_cast<int>((taken >> (4 * w)) & 15u);
+          if (lane == 0) mbar_arrive(rec_empty + w * GA_RB + tk % GA_RB);
+          taken = (taken & ~(15u << (4 * w))) | (static_cast<uint32_t>((tk + 1) & 15) << (4 * w));
+        }
       }
       if (!shared) {
         mg.write_out(p, bh, lane);

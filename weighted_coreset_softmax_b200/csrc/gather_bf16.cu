@@ -18,7 +18,10 @@ static cudaError_t gather_launch_one(const AttnParams& p, const CUtensorMap& tk,
   if (!(configured.load() & (1 << (dev & 31)))) {
     const cudaError_t e =
         cudaFuncSetAttribute(gather_attn_kernel<D, G, ROWS>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();  // do not leave the failure for an unrelated later check
+      return e;
+    }
     configured.fetch_or(1 << (dev & 31));
   }
   cudaLaunchConfig_t cfg = {};
@@ -32,7 +35,10 @@ static cudaError_t gather_launch_one(const AttnParams& p, const CUtensorMap& tk,
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t le = cudaLaunchKernelEx(&cfg, gather_attn_kernel<D, G, ROWS>, p, tk, tv);
-  if (le != cudaSuccess) return le;
+  if (le != cudaSuccess) {
+    (void)cudaGetLastError();
+    return le;
+  }
   return cudaGetLastError();
 }
 
