@@ -58,6 +58,13 @@ notes of the repository):
   R13 bf16 block means: the mean key is rounded to the nearest bfloat16 value
       (ties to even) and used in place of the exact mean in the first-order
       score; everything else as in R1 to R6.
+  R14 WildCat coreset (the abstract names randomly pivoted Cholesky and weights
+      that minimise reconstruction error, not the kernel or the error): the kernel
+      is the exponential kernel of attention on the keys, exp(sigma k_i . k_j)
+      (shifted by a constant, which cancels); the error is the kernel (feature
+      space) distance between the sum over all tokens and the weighted coreset,
+      whose minimiser solves A_SS w = A_{S,:} 1; negative weights are clipped to
+      0; the uniforms of the pivot draws are inputs.
 """
 from __future__ import annotations
 
@@ -390,6 +397,63 @@ def weighted_attend_one(qg, K, V, n, tok_idx, w, sigma):
         logits = sigma * (K[idx] @ qg[g]) + np.log(w)
         out[g], lse[g] = softmax_attend(logits, V[idx])
     return out, lse
+
+
+def wildcat_kernel(K: np.ndarray, n: int, sigma: float) -> np.ndarray:
+    """The kernel on the keys the coreset is chosen for [WC, abstract; reading R20]:
+    A[i, j] = exp(sigma k_i . k_j - sigma M) over the first n keys, M = max_i |k_i|^2.
+    The constant shift keeps every entry in (0, 1] (k_i . k_j <= M by Cauchy-Schwarz)
+    and cancels in the pivot choice and in the weights."""
+    Kn = np.asarray(K[:n], dtype=np.float64)
+    if n == 0:
+        return np.zeros((0, 0))
+    M = float(np.max(np.sum(Kn * Kn, axis=1)))
+    return np.exp(sigma * (Kn @ Kn.T) - sigma * M)
+
+
+def rpcholesky(K: np.ndarray, n: int, sigma: float, u, m: int):
+    """Randomly pivoted Cholesky on the key kernel [WC, abstract: the coreset is
+    selected by randomly pivoted Cholesky]. Step t draws the pivot with probability
+    proportional to the residual diagonal d (the kernel's diagonal minus what the
+    factor so far explains): with the uniform u[t] in (0, 1), the pivot is the
+    smallest i with d_0 + ... + d_i >= u[t] (d_0 + ... + d_{n-1}). The new factor
+    column is the pivot's residual kernel column divided by the square root of its
+    pivot entry, and d drops by its square. Stops early when the residual is zero.
+    Returns the pivots (in order) and the factor F [n][t] with F F^T = A on the
+    pivots' rows and columns."""
+    A = wildcat_kernel(K, n, sigma)
+    d = np.diag(A).copy() if n else np.zeros(0)
+    F = np.zeros((n, m))
+    S: List[int] = []
+    for t in range(m):
+        tot = float(np.sum(d))
+        if n == 0 or tot <= 0.0:
+            break
+        c = np.cumsum(d)
+        s = int(np.searchsorted(c, float(u[t]) * tot, side="left"))
+        s = min(s, n - 1)
+        g = A[:, s] - F[:, :t] @ F[s, :t]
+        if g[s] <= 0.0:
+            break
+        F[:, t] = g / math.sqrt(g[s])
+        d = np.maximum(d - F[:, t] ** 2, 0.0)
+        d[s] = 0.0
+        S.append(s)
+    return S, F[:, :len(S)]
+
+
+def wildcat_weights(K: np.ndarray, n: int, sigma: float, S) -> Tuple[np.ndarray, np.ndarray]:
+    """The coreset weights [WC, abstract: "weight the elements optimally to
+    minimise reconstruction error"; reading R20]: the w minimising the kernel
+    distance || sum_{i<n} phi(k_i) - sum_{j in S} w_j phi(k_j) ||^2, i.e. the
+    solution of A_SS w = A_{S,:} 1. Returns (w, w clipped at 0); the attention
+    takes ln w, so a negative weight drops its token."""
+    A = wildcat_kernel(K, n, sigma)
+    S = list(S)
+    if not S:
+        return np.zeros(0), np.zeros(0)
+    w = np.linalg.solve(A[np.ix_(S, S)], A[S, :].sum(axis=1))
+    return w, np.maximum(w, 0.0)
 
 
 def dense_attend_one(qg, K, V, n, sigma):

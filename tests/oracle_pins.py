@@ -606,6 +606,124 @@ def pin_mean16_score(seed=22):
     assert np.max(np.abs(a - e)) > 0, "rounding must change some score"
 
 
+def pin_wildcat_kernel_bruteforce(seed=23):
+    """The key kernel, entry by entry in Python floats."""
+    r = _rng(seed)
+    K = r.normal(size=(9, 5))
+    sigma = 0.4
+    A = O.wildcat_kernel(K, 7, sigma)
+    M = max(sum(float(x) * float(x) for x in K[i]) for i in range(7))
+    for i in range(7):
+        for j in range(7):
+            dot = sum(float(K[i][d]) * float(K[j][d]) for d in range(5))
+            _close(A[i, j], math.exp(sigma * dot - sigma * M), 1e-13, what="kernel entry")
+    assert np.all(A <= 1.0 + 1e-15) and A.shape == (7, 7)
+
+
+def pin_rpcholesky_pivot_rule(seed=24):
+    """Each pivot is the inverse-CDF draw of u over the residual diagonal, which is
+    recomputed here by brute force from the pivots before it (diag(A) minus the
+    squares of the factor columns, each column the residual kernel column over the
+    square root of its pivot entry)."""
+    r = _rng(seed)
+    n, m = 40, 12
+    K = r.normal(size=(n, 6))
+    u = r.uniform(size=m)
+    sigma = 0.3
+    S, F = O.rpcholesky(K, n, sigma, u, m)
+    A = O.wildcat_kernel(K, n, sigma)
+    cols = []
+    for t, s_t in enumerate(S):
+        d = [A[i][i] - sum(c[i] ** 2 for c in cols) for i in range(n)]
+        for j in S[:t]:
+            d[j] = 0.0
+        d = [max(x, 0.0) for x in d]
+        tot = sum(d)
+        acc, want = 0.0, None
+        for i in range(n):
+            acc += d[i]
+            if acc >= u[t] * tot:
+                want = i
+                break
+        assert s_t == want, (t, s_t, want)
+        res = [A[i][s_t] - sum(c[i] * c[s_t] for c in cols) for i in range(n)]
+        cols.append([x / math.sqrt(res[s_t]) for x in res])
+    _close(F, np.array(cols).T, 1e-10, what="factor columns")
+
+
+def pin_rpcholesky_interpolates(seed=25):
+    """F F^T reproduces the kernel on the pivots' rows; the residual diagonal is
+    non-negative and zero on the pivots; the pivots are distinct."""
+    r = _rng(seed)
+    n = 120
+    K = r.normal(size=(n, 8))
+    S, F = O.rpcholesky(K, n, 0.25, r.uniform(size=30), 30)
+    A = O.wildcat_kernel(K, n, 0.25)
+    assert len(set(S)) == len(S) == 30
+    _close((F @ F.T)[S], A[S], 1e-10, what="interpolation on pivot rows")
+    res = np.diag(A) - np.sum(F * F, axis=1)
+    assert np.min(res) > -1e-10 and np.max(np.abs(res[S])) < 1e-10
+
+
+def pin_wildcat_all_points_is_exact(seed=26):
+    """With every token a pivot the optimal weights are all 1, and the weighted
+    coreset attention is dense attention."""
+    r = _rng(seed)
+    n, D = 14, 4
+    K, V = r.normal(size=(n, D)), r.normal(size=(n, D))
+    qg = r.normal(size=(2, D))
+    S, _ = O.rpcholesky(K, n, 0.5, r.uniform(size=n), n)
+    assert sorted(S) == list(range(n))
+    w, wc = O.wildcat_weights(K, n, 0.5, S)
+    _close(w, np.ones(n), 1e-8, what="weights with every token kept")
+    o, l = O.weighted_attend_one(qg, K, V, n, S, wc, 0.5)
+    od, ld = O.dense_attend_one(qg, K, V, n, 0.5)
+    _close(o, od, 1e-8, what="coreset of all tokens = dense")
+    _close(l, ld, 1e-8, what="lse")
+
+
+def pin_wildcat_identical_tokens(seed=27):
+    """n identical tokens: one pivot explains the kernel, its weight is n, and the
+    coreset attention equals dense attention over the n copies."""
+    r = _rng(seed)
+    n, D = 25, 6
+    k, v = r.normal(size=D), r.normal(size=D)
+    K, V = np.tile(k, (n, 1)), np.tile(v, (n, 1))
+    qg = r.normal(size=(3, D))
+    S, _ = O.rpcholesky(K, n, 0.7, r.uniform(size=5), 5)
+    assert len(S) == 1
+    w, wc = O.wildcat_weights(K, n, 0.7, S)
+    _close(w, [float(n)], 1e-10, what="weight of the single pivot")
+    o, l = O.weighted_attend_one(qg, K, V, n, S, wc, 0.7)
+    od, ld = O.dense_attend_one(qg, K, V, n, 0.7)
+    _close(o, od, 1e-10, what="identical tokens")
+    _close(l, ld, 1e-10, what="lse")
+
+
+def pin_wildcat_weights_optimal(seed=28):
+    """The weights minimise the kernel distance: the objective
+    w^T A_SS w - 2 w^T A_{S,:} 1 (written out with Python sums) is not lowered by
+    moving any single weight either way."""
+    r = _rng(seed)
+    n = 30
+    K = r.normal(size=(n, 5))
+    S, _ = O.rpcholesky(K, n, 0.3, r.uniform(size=6), 6)
+    w, _ = O.wildcat_weights(K, n, 0.3, S)
+    A = O.wildcat_kernel(K, n, 0.3)
+
+    def J(x):
+        quad = sum(x[a] * x[b] * A[S[a]][S[b]] for a in range(len(S)) for b in range(len(S)))
+        lin = sum(x[a] * sum(A[S[a]][i] for i in range(n)) for a in range(len(S)))
+        return quad - 2.0 * lin
+
+    base = J(list(w))
+    for a in range(len(S)):
+        for eps in (1e-3, -1e-3):
+            x = list(w)
+            x[a] += eps
+            assert J(x) > base, (a, eps)
+
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -615,4 +733,6 @@ ALL_PINS = [
     pin_summary_equals_exact_for_constant_blocks, pin_quest_box_corners, pin_quest_upper_bound,
     pin_cobs_full_rank_is_exact_quadratic, pin_cobs_rank_one_block, pin_cobs_two_point_closed_form,
     pin_cobs_error_order, pin_cobs_eigen_structure, pin_round_bf16_nearest_even, pin_mean16_score,
+    pin_wildcat_kernel_bruteforce, pin_rpcholesky_pivot_rule, pin_rpcholesky_interpolates,
+    pin_wildcat_all_points_is_exact, pin_wildcat_identical_tokens, pin_wildcat_weights_optimal,
 ]

@@ -62,6 +62,62 @@ def _mut_round_bf16_ties_up(orig):
     return f
 
 
+def _mut_rpchol_greedy(orig):
+    def f(K, n, sigma, u, m):
+        return _greedy(K, n, sigma, m)
+    return f
+
+
+def _greedy(K, n, sigma, m):
+    A = O.wildcat_kernel(K, n, sigma)
+    d = np.diag(A).copy()
+    F = np.zeros((n, m))
+    S = []
+    for t in range(m):
+        if d.sum() <= 0:
+            break
+        s_ = int(np.argmax(d))
+        g = A[:, s_] - F[:, :t] @ F[s_, :t]
+        F[:, t] = g / math.sqrt(g[s_])
+        d = np.maximum(d - F[:, t] ** 2, 0.0)
+        d[s_] = 0.0
+        S.append(s_)
+    return S, F[:, :len(S)]
+
+
+def _mut_rpchol_no_downdate(orig):
+    def f(K, n, sigma, u, m):
+        A = O.wildcat_kernel(K, n, sigma)
+        d = np.diag(A).copy()
+        F = np.zeros((n, m))
+        S = []
+        for t in range(m):
+            tot = d.sum()
+            if tot <= 0:
+                break
+            s_ = min(int(np.searchsorted(np.cumsum(d), u[t] * tot)), n - 1)
+            g = A[:, s_].copy()
+            F[:, t] = g / math.sqrt(g[s_])
+            d = np.maximum(d - F[:, t] ** 2, 0.0)
+            d[s_] = 0.0
+            S.append(s_)
+        return S, F[:, :len(S)]
+    return f
+
+
+def _mut_wildcat_uniform_weights(orig):
+    def f(K, n, sigma, S):
+        w = np.full(len(S), n / max(1, len(S)))
+        return w, w
+    return f
+
+
+def _mut_wildcat_kernel_no_sigma(orig):
+    def f(K, n, sigma):
+        return orig(K, n, 1.0)
+    return f
+
+
 def _mut_group_score_logits(orig):
     def f(shat):
         return np.where(np.isfinite(shat), shat, 0.0).sum(axis=0)
@@ -181,6 +237,10 @@ MUTANTS = {
     "mean16/no ln n_b": ("summary_mean16_logits", _mut_summary_no_log),
     "mean16/sum not mean": ("summary_mean16_logits", _mut_summary_sum_not_mean),
     "round_bf16/truncates": ("round_bf16", _mut_round_bf16_truncate),
+    "rpcholesky/greedy pivots": ("rpcholesky", _mut_rpchol_greedy),
+    "rpcholesky/no downdate": ("rpcholesky", _mut_rpchol_no_downdate),
+    "wildcat/uniform weights": ("wildcat_weights", _mut_wildcat_uniform_weights),
+    "wildcat/kernel without scale": ("wildcat_kernel", _mut_wildcat_kernel_no_sigma),
     "round_bf16/ties up": ("round_bf16", _mut_round_bf16_ties_up),
     "group_score/sums logits": ("group_score", _mut_group_score_logits),
     "select_blocks/high-index ties": ("select_blocks", _mut_select_high_index),
