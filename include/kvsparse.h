@@ -178,6 +178,40 @@ kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float sc
                                   kv_stream_t stream);
 
 /*
+ * kv_build_wildcat_coreset -- a weighted coreset of every (sequence, KV head)'s
+ * keys, for the weighted-coreset mode of kv_sparse_decode_attn. Source:
+ * "WildCat: Near-Linear Attention in Theory and Practice", abstract (the coreset is
+ * selected by randomly pivoted Cholesky and weighted to minimise the
+ * reconstruction error). Readings: the kernel is exp(scale k_i . k_j) on the first
+ * seq_len keys (evaluated shifted by scale * max_i |k_i|^2; the shift cancels);
+ * the weights minimise the kernel distance between the sum over all tokens and the
+ * weighted coreset (A_SS w = A_{S,:} 1); a negative weight is clipped to 0.
+ *
+ *   K        device cache [B][Hkv][Ncap][D] (bf16 or fp32), 16-byte aligned
+ *   scale    the softmax scale, > 0
+ *   m        coreset size per (sequence, KV head), 1 <= m <= min(4096, Ncap)
+ *   u        device [B][Hkv][m] fp32 uniforms in (0, 1): u[.][t] draws pivot t as the
+ *            first token whose running sum of the residual diagonal reaches u times
+ *            its total (randomness is an input, so results are reproducible)
+ *   tok_idx  device out [B][Hkv][m] int32: the pivots in the order drawn
+ *   w        device out [B][Hkv][m] fp32: their weights (>= 0)
+ *   n_sel    device out [B][Hkv] int32 (or NULL): pivots drawn; fewer than m when
+ *            the residual vanishes (entries past it: index 0, weight 0, which the
+ *            attention leaves out)
+ *   workspace  device, kv_wildcat_workspace_bytes(shape, m) bytes, 16-byte aligned
+ *            (the factor, m + 1 rows of Ncap floats per (sequence, KV head))
+ * One CTA per (sequence, KV head) runs the m pivot steps (each a scan of the
+ * residual diagonal and one residual kernel column); run once after prefill.
+ * KV_ERR_INVALID_ARG for bad sizes or pointers, KV_ERR_UNSUPPORTED for D not 64/128.
+ */
+kv_status kv_build_wildcat_coreset(const kv_shape* shape, const void* K, float scale, int m,
+                                   const float* u, int32_t* tok_idx, float* w, int32_t* n_sel,
+                                   void* workspace, size_t ws_bytes, kv_stream_t stream);
+
+/* Workspace bytes kv_build_wildcat_coreset needs for this shape and m (0 if invalid). */
+size_t kv_wildcat_workspace_bytes(const kv_shape* shape, int m);
+
+/*
  * kv_build_block_bounds -- per-block, per-channel key minimum and maximum (the
  * axis-aligned bounding box of each block's keys). Source: "COBS: Cumulant Order
  * Block Sparse Attention", the Quest paragraph (a block is scored by the largest

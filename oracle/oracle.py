@@ -421,17 +421,30 @@ def rpcholesky(K: np.ndarray, n: int, sigma: float, u, m: int):
     pivot entry, and d drops by its square. Stops early when the residual is zero.
     Returns the pivots (in order) and the factor F [n][t] with F F^T = A on the
     pivots' rows and columns."""
+    S, F, _ = rpcholesky_steps(K, n, sigma, u, m)
+    return S, F
+
+
+def rpcholesky_steps(K: np.ndarray, n: int, sigma: float, u, m: int, pivots=None):
+    """The steps of rpcholesky, also returning each step's residual diagonal (before
+    the step's pivot is drawn). With pivots given, those are taken in order instead
+    of the draws (to replay another implementation's choices)."""
     A = wildcat_kernel(K, n, sigma)
     d = np.diag(A).copy() if n else np.zeros(0)
     F = np.zeros((n, m))
     S: List[int] = []
+    resid = []
     for t in range(m):
         tot = float(np.sum(d))
-        if n == 0 or tot <= 0.0:
+        if n == 0 or tot <= 0.0 or (pivots is not None and t >= len(pivots)):
             break
-        c = np.cumsum(d)
-        s = int(np.searchsorted(c, float(u[t]) * tot, side="left"))
-        s = min(s, n - 1)
+        resid.append(d.copy())
+        if pivots is None:
+            c = np.cumsum(d)
+            s = int(np.searchsorted(c, float(u[t]) * tot, side="left"))
+            s = min(s, n - 1)
+        else:
+            s = int(pivots[t])
         g = A[:, s] - F[:, :t] @ F[s, :t]
         if g[s] <= 0.0:
             break
@@ -439,7 +452,7 @@ def rpcholesky(K: np.ndarray, n: int, sigma: float, u, m: int):
         d = np.maximum(d - F[:, t] ** 2, 0.0)
         d[s] = 0.0
         S.append(s)
-    return S, F[:, :len(S)]
+    return S, F[:, :len(S)], resid
 
 
 def wildcat_weights(K: np.ndarray, n: int, sigma: float, S) -> Tuple[np.ndarray, np.ndarray]:

@@ -31,7 +31,7 @@ __all__ = [
     "kv_select_blocks_mean16",
     "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace", "kv_selftest_wait_timeout",
-    "kv_stream_read",
+    "kv_stream_read", "kv_build_wildcat_coreset",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
@@ -99,6 +99,7 @@ def lib():
         "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
         "kv_selftest_wait_timeout": [_P, _P, ctypes.c_uint64, _I, _P],
         "kv_stream_read": [_P, _S, _P, _P],
+        "kv_build_wildcat_coreset": [_SHP, _P, _F, _I, _P, _P, _P, _P, _P, _S, _P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -106,6 +107,8 @@ def lib():
         fn.restype = _I
     L.kv_workspace_bytes.argtypes = [_SHP]
     L.kv_workspace_bytes.restype = _S
+    L.kv_wildcat_workspace_bytes.argtypes = [_SHP, _I]
+    L.kv_wildcat_workspace_bytes.restype = _S
     L.kv_last_error.argtypes = []
     L.kv_last_error.restype = ctypes.c_char_p
     _lib = L
@@ -508,3 +511,25 @@ def kv_stream_read(src: torch.Tensor, nbytes: int, sink: torch.Tensor) -> None:
     if nbytes > src.numel() * src.element_size():
         raise ValueError("nbytes exceeds the tensor")
     _check(lib().kv_stream_read(_ptr(src), ctypes.c_size_t(int(nbytes)), _ptr(sink), _stream(src.device)))
+
+
+def kv_build_wildcat_coreset(K: torch.Tensor, seq_lens: torch.Tensor, scale: float, m: int, u: torch.Tensor,
+                             workspace: Optional[torch.Tensor] = None):
+    """Weighted coreset of every (sequence, KV head)'s keys by randomly pivoted
+    Cholesky with kernel-distance weights. u: [B][Hkv][m] fp32 uniforms in (0, 1)
+    on the device. Returns (tok_idx [B][Hkv][m] int32, w [B][Hkv][m] fp32, n_sel
+    [B][Hkv] int32) for kv_sparse_decode_attn(tok_idx=..., w=...)."""
+    _need(K, "K")
+    _need(u, "u", torch.float32)
+    B, Hkv, Ncap, D = K.shape
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, 64, _dtype_code(K.dtype), seq_lens.data_ptr())
+    need = int(lib().kv_wildcat_workspace_bytes(ctypes.byref(shape), int(m)))
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=K.device)
+    tok_idx = torch.zeros(B, Hkv, m, dtype=torch.int32, device=K.device)
+    w = torch.zeros(B, Hkv, m, dtype=torch.float32, device=K.device)
+    n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=K.device)
+    _check(lib().kv_build_wildcat_coreset(ctypes.byref(shape), _ptr(K), float(scale), int(m), _ptr(u), _ptr(tok_idx),
+                                          _ptr(w), _ptr(n_sel), _ptr(workspace),
+                                          workspace.numel() * workspace.element_size(), _stream(K.device)))
+    return tok_idx, w, n_sel
