@@ -18,6 +18,7 @@ cores instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import datetime
 import json
 import math
@@ -61,6 +62,8 @@ def parse_args(argv=None):
     ap.add_argument("--rot", type=int, default=None,
                     help="independent batches rotated through the steps (default: enough to pass twice "
                          "the L2 capacity between two uses of a batch; 1 for small profiling captures)")
+    ap.add_argument("--wildcat-m", type=int, default=64,
+                    help="coreset size of the timed WildCat build after prefill (0: skip it)")
     ap.add_argument("--batch", type=int, default=None,
                     help="sequences per GPU (default: the workload's own batch; smaller for profiler captures)")
     return ap.parse_args(argv)
@@ -246,6 +249,21 @@ def cobs_select_bytes(wl, seq_lens, rank=4):
 def osa_select_bytes(wl, seq_lens):
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
     return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
+
+
+def wildcat_bytes(wl, seq_lens, n_sel):
+    """Algorithmic bytes of kv_build_wildcat_coreset: per (sequence, KV head) with n
+    tokens and T pivots, one read of the keys for the shift, then per step t the n
+    keys, t factor rows read and one written (n fp32 each) and the residual diagonal
+    read and written."""
+    kb = wl.K.element_size()
+    total = 0
+    ns = n_sel.cpu().tolist()
+    for b, n in enumerate(seq_lens):
+        for h in range(wl.Hkv):
+            T = int(ns[b][h])
+            total += n * wl.D * kb + T * n * (wl.D * kb + 12) + 4 * n * T * (T - 1) // 2
+    return total
 
 
 def weighted_bytes(wl):
@@ -549,6 +567,28 @@ def run_ours(args, dist):
     if wl.score_mode == "cobs":
         builds["kv_build_block_cov_factors_ms"] = time_build(
             lambda: kv.kv_build_block_cov_factors(wl.K, sl, wl.block_size, 4, out=summ["k_xi"]), reps=1)
+
+    if args.wildcat_m > 0:
+        # the WildCat coreset producer on the same cache (randomly pivoted Cholesky
+        # with kernel-distance weights, m pivots per (sequence, KV head))
+        m_wc = min(args.wildcat_m, wl.Ncap)
+        g_wc = torch.Generator(device=dev).manual_seed(4242 + shard_seed_offset(dist.rank))
+        u_wc = torch.rand(wl.B, wl.Hkv, m_wc, generator=g_wc, device=dev).clamp_(1e-6, 1 - 1e-6)
+        shp_wc = kv.KVShape(wl.B, wl.Hkv, wl.Hkv, wl.D, wl.Ncap, wl.block_size, kv._dtype_code(wl.K.dtype), sl.data_ptr())
+        ws_wc = torch.empty(int(kv.lib().kv_wildcat_workspace_bytes(ctypes.byref(shp_wc), m_wc)),
+                            dtype=torch.uint8, device=dev)
+        out_wc = {}
+
+        def wc_build():
+            out_wc["r"] = kv.kv_build_wildcat_coreset(wl.K, sl, wl.scale, m_wc, u_wc, workspace=ws_wc)
+        wc_ms = time_build(wc_build, reps=1)
+        wc_b = wildcat_bytes(wl, wl.seq_lens, out_wc["r"][2])
+        pk, pk_kind = measured_peak_hbm()
+        builds["kv_build_wildcat_coreset"] = {
+            "m": m_wc, "ms": wc_ms, "bytes": wc_b, "GB_s": wc_b / (wc_ms * 1e-3) / 1e9,
+            "frac": wc_b / (wc_ms * 1e-3) / 1e9 / pk, "peak_kind": pk_kind,
+            "pivots_min": int(out_wc["r"][2].min()) if out_wc["r"][2].numel() else 0}
+        del ws_wc, out_wc
 
     def check_status(what):
         for st_ in sets:

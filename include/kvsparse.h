@@ -190,6 +190,9 @@ kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float sc
  *   K        device cache [B][Hkv][Ncap][D] (bf16 or fp32), 16-byte aligned
  *   scale    the softmax scale, > 0
  *   m        coreset size per (sequence, KV head), 1 <= m <= min(4096, Ncap)
+ *   ctas_per_pair  CTAs (a thread-block cluster) per (sequence, KV head), 1..8, or 0
+ *            for min(8, SMs / pairs); the pivots differ between cluster sizes only
+ *            where fp32 rounding of the running sums decides a draw
  *   u        device [B][Hkv][m] fp32 uniforms in (0, 1): u[.][t] draws pivot t as the
  *            first token whose running sum of the residual diagonal reaches u times
  *            its total (randomness is an input, so results are reproducible)
@@ -199,13 +202,16 @@ kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float sc
  *            the residual vanishes (entries past it: index 0, weight 0, which the
  *            attention leaves out)
  *   workspace  device, kv_wildcat_workspace_bytes(shape, m) bytes, 16-byte aligned
- *            (the factor, m + 1 rows of Ncap floats per (sequence, KV head))
- * One CTA per (sequence, KV head) runs the m pivot steps (each a scan of the
- * residual diagonal and one residual kernel column); run once after prefill.
- * KV_ERR_INVALID_ARG for bad sizes or pointers, KV_ERR_UNSUPPORTED for D not 64/128.
+ *            (per (sequence, KV head): the factor and the residual diagonal, m + 1
+ *            rows of Ncap floats, and 8 x m partial column sums)
+ * The cluster of a pair runs the m pivot steps (each a draw from the residual
+ * diagonal and one pass over the keys for a residual kernel column); run once after
+ * prefill. Bytes per pair and step: the n keys plus t + 1 factor rows of n floats.
+ * KV_ERR_INVALID_ARG for bad sizes or pointers, KV_ERR_UNSUPPORTED for D not 64/128
+ * or Ncap above 2^20.
  */
 kv_status kv_build_wildcat_coreset(const kv_shape* shape, const void* K, float scale, int m,
-                                   const float* u, int32_t* tok_idx, float* w, int32_t* n_sel,
+                                   int ctas_per_pair, const float* u, int32_t* tok_idx, float* w, int32_t* n_sel,
                                    void* workspace, size_t ws_bytes, kv_stream_t stream);
 
 /* Workspace bytes kv_build_wildcat_coreset needs for this shape and m (0 if invalid). */

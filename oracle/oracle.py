@@ -425,12 +425,27 @@ def rpcholesky(K: np.ndarray, n: int, sigma: float, u, m: int):
     return S, F
 
 
+def wildcat_kernel_cols(K: np.ndarray, n: int, sigma: float, cols) -> np.ndarray:
+    """Columns `cols` of wildcat_kernel (an n x len(cols) array), evaluated from the
+    same formula without forming the n x n matrix."""
+    Kn = np.asarray(K[:n], dtype=np.float64)
+    M = float(np.max(np.sum(Kn * Kn, axis=1)))
+    return np.exp(sigma * (Kn @ Kn[list(cols)].T) - sigma * M)
+
+
+def wildcat_kernel_diag(K: np.ndarray, n: int, sigma: float) -> np.ndarray:
+    """The diagonal of wildcat_kernel: exp(sigma |k_i|^2 - sigma M)."""
+    Kn = np.asarray(K[:n], dtype=np.float64)
+    sq = np.sum(Kn * Kn, axis=1)
+    return np.exp(sigma * sq - sigma * float(np.max(sq)))
+
+
 def rpcholesky_steps(K: np.ndarray, n: int, sigma: float, u, m: int, pivots=None):
     """The steps of rpcholesky, also returning each step's residual diagonal (before
     the step's pivot is drawn). With pivots given, those are taken in order instead
-    of the draws (to replay another implementation's choices)."""
-    A = wildcat_kernel(K, n, sigma)
-    d = np.diag(A).copy() if n else np.zeros(0)
+    of the draws (to replay another implementation's choices). The kernel is
+    evaluated a column at a time, so long sequences fit in memory."""
+    d = wildcat_kernel_diag(K, n, sigma) if n else np.zeros(0)
     F = np.zeros((n, m))
     S: List[int] = []
     resid = []
@@ -445,7 +460,7 @@ def rpcholesky_steps(K: np.ndarray, n: int, sigma: float, u, m: int, pivots=None
             s = min(s, n - 1)
         else:
             s = int(pivots[t])
-        g = A[:, s] - F[:, :t] @ F[s, :t]
+        g = wildcat_kernel_cols(K, n, sigma, [s])[:, 0] - F[:, :t] @ F[s, :t]
         if g[s] <= 0.0:
             break
         F[:, t] = g / math.sqrt(g[s])
@@ -461,11 +476,11 @@ def wildcat_weights(K: np.ndarray, n: int, sigma: float, S) -> Tuple[np.ndarray,
     distance || sum_{i<n} phi(k_i) - sum_{j in S} w_j phi(k_j) ||^2, i.e. the
     solution of A_SS w = A_{S,:} 1. Returns (w, w clipped at 0); the attention
     takes ln w, so a negative weight drops its token."""
-    A = wildcat_kernel(K, n, sigma)
     S = list(S)
     if not S:
         return np.zeros(0), np.zeros(0)
-    w = np.linalg.solve(A[np.ix_(S, S)], A[S, :].sum(axis=1))
+    AS = wildcat_kernel_cols(K, n, sigma, S)  # A[:, S], n x |S|
+    w = np.linalg.solve(AS[S, :], AS.sum(axis=0))
     return w, np.maximum(w, 0.0)
 
 

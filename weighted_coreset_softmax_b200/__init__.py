@@ -99,7 +99,7 @@ def lib():
         "kv_workspace_status": [_P, ctypes.POINTER(ctypes.c_uint32), _P],
         "kv_selftest_wait_timeout": [_P, _P, ctypes.c_uint64, _I, _P],
         "kv_stream_read": [_P, _S, _P, _P],
-        "kv_build_wildcat_coreset": [_SHP, _P, _F, _I, _P, _P, _P, _P, _P, _S, _P],
+        "kv_build_wildcat_coreset": [_SHP, _P, _F, _I, _I, _P, _P, _P, _P, _P, _S, _P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -514,10 +514,10 @@ def kv_stream_read(src: torch.Tensor, nbytes: int, sink: torch.Tensor) -> None:
 
 
 def kv_build_wildcat_coreset(K: torch.Tensor, seq_lens: torch.Tensor, scale: float, m: int, u: torch.Tensor,
-                             workspace: Optional[torch.Tensor] = None):
+                             workspace: Optional[torch.Tensor] = None, ctas_per_pair: int = 0):
     """Weighted coreset of every (sequence, KV head)'s keys by randomly pivoted
     Cholesky with kernel-distance weights. u: [B][Hkv][m] fp32 uniforms in (0, 1)
-    on the device. Returns (tok_idx [B][Hkv][m] int32, w [B][Hkv][m] fp32, n_sel
+    on the device; ctas_per_pair: CTAs per pair (0: min(8, SMs / pairs)). Returns (tok_idx [B][Hkv][m] int32, w [B][Hkv][m] fp32, n_sel
     [B][Hkv] int32) for kv_sparse_decode_attn(tok_idx=..., w=...)."""
     _need(K, "K")
     _need(u, "u", torch.float32)
@@ -529,7 +529,8 @@ def kv_build_wildcat_coreset(K: torch.Tensor, seq_lens: torch.Tensor, scale: flo
     tok_idx = torch.zeros(B, Hkv, m, dtype=torch.int32, device=K.device)
     w = torch.zeros(B, Hkv, m, dtype=torch.float32, device=K.device)
     n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=K.device)
-    _check(lib().kv_build_wildcat_coreset(ctypes.byref(shape), _ptr(K), float(scale), int(m), _ptr(u), _ptr(tok_idx),
+    _check(lib().kv_build_wildcat_coreset(ctypes.byref(shape), _ptr(K), float(scale), int(m), int(ctas_per_pair),
+                                          _ptr(u), _ptr(tok_idx),
                                           _ptr(w), _ptr(n_sel), _ptr(workspace),
                                           workspace.numel() * workspace.element_size(), _stream(K.device)))
     return tok_idx, w, n_sel
