@@ -180,6 +180,121 @@ def cobs_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, xi: np.nd
     return out
 
 
+def query_basis(Qc: np.ndarray, Hkv: int):
+    """The eigenvectors of each KV head's query second moment [COBS, the subspace
+    paragraph: U_Q holds the top s eigenvectors of E[q q^T]; reading R22]. The
+    second moment of KV head h is the mean of q q^T over the calibration positions
+    and the query heads of its group. Qc: [Nc][Hq][D]. Returns (evals [Hkv][D] in
+    descending order, evecs [Hkv][D][D] whose row j is the unit eigenvector of
+    evals[h][j])."""
+    Nc, Hq, D = Qc.shape
+    G = Hq // Hkv
+    evals = np.zeros((Hkv, D))
+    evecs = np.zeros((Hkv, D, D))
+    for h in range(Hkv):
+        X = np.asarray(Qc[:, h * G:(h + 1) * G, :], dtype=np.float64).reshape(-1, D)
+        C = X.T @ X / X.shape[0]
+        w, U = np.linalg.eigh(C)  # ascending
+        evals[h] = w[::-1]
+        evecs[h] = U[:, ::-1].T
+    return evals, evecs
+
+
+def subspace_rank(evals: np.ndarray, energy: float = 0.9):
+    """The subspace dimension s [COBS, the subspace paragraph: s is set per layer
+    from the rank capturing 90% of the query spectral energy, averaged over heads;
+    reading R22]: per head the smallest s_h whose leading eigenvalues sum to at least
+    `energy` of the trace, then s = ceil(mean over heads of s_h). Returns (s, [s_h])."""
+    sh = []
+    for lam in np.asarray(evals, dtype=np.float64):
+        tot = float(np.sum(lam))
+        acc, pick = 0.0, len(lam)
+        for j, x in enumerate(lam):
+            acc += float(x)
+            if acc >= energy * tot:
+                pick = j + 1
+                break
+        sh.append(pick)
+    return int(math.ceil(sum(sh) / len(sh))), sh
+
+
+def block_cov_factors_ss_one(K: np.ndarray, n: int, L: int, NBcap: int, r: int, U: np.ndarray):
+    """Per block, the top r scaled eigenvectors of the covariance kept within the
+    query subspace [COBS, the subspace paragraph: B_b = U_Q^T Sigma_b U_Q, rank-r
+    spectral decomposition in the projected space; reading R22]. U: [s][D], rows the
+    basis (U_Q^T). Returns xi [NBcap][r][s] (xi_i = sqrt(lambda_i) u_i for the r
+    largest eigenvalues of B_b, descending) and the eigenvalues [NBcap][r]; blocks
+    past the sequence and directions past B_b's rank stay 0."""
+    U = np.asarray(U, dtype=np.float64)
+    s_dim = U.shape[0]
+    xi = np.zeros((NBcap, r, s_dim))
+    lam = np.zeros((NBcap, r))
+    for b, (st, e) in enumerate(blocks_of(n, L)):
+        X = K[st:e] - K[st:e].mean(axis=0)
+        Bm = U @ (X.T @ X / (e - st)) @ U.T
+        w, V = np.linalg.eigh(Bm)  # ascending
+        for i in range(min(r, s_dim)):
+            li = max(float(w[s_dim - 1 - i]), 0.0)
+            lam[b, i] = li
+            xi[b, i] = math.sqrt(li) * V[:, s_dim - 1 - i]
+    return xi, lam
+
+
+E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # magnitudes of codes 0..7
+
+
+def fp4_e2m1_quantize(x):
+    """E2M1 FP4 codes of one vector with one fp32 scale [COBS, the quantisation
+    paragraph: the scaled eigenvectors in E2M1 FP4 with one fp32 scale each;
+    reading R22]. The scale is max|x| / 6 (6 is the largest E2M1 magnitude); each
+    x_j / scale goes to the nearest E2M1 magnitude, a tie to the code with mantissa
+    bit 0 (the even code), with the sign in bit 3 (zero keeps code 0). The scale and
+    the quotients are float32 operations, the precision in which the kernel takes the
+    same decisions. Returns (codes uint8 [len] in 0..15, scale float32)."""
+    x32 = np.asarray(x, dtype=np.float32)
+    codes = np.zeros(x32.shape, dtype=np.uint8)
+    amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0.0)
+    scale = np.float32(amax / np.float32(6.0))
+    if not scale > 0:
+        return codes, np.float32(0.0)
+    for j, v in enumerate(x32):
+        a = abs(float(np.float32(v / scale)))
+        best, bd = 0, None
+        for c, gv in enumerate(E2M1_GRID):
+            dist = abs(a - gv)
+            if bd is None or dist < bd or (dist == bd and c % 2 == 0):
+                best, bd = c, dist
+        codes[j] = best | (8 if (v < 0 and best != 0) else 0)
+    return codes, scale
+
+
+def fp4_e2m1_decode(codes, scale) -> np.ndarray:
+    """The values of E2M1 codes times their scale (float64)."""
+    c = np.asarray(codes, dtype=np.int64)
+    mag = np.array(E2M1_GRID)[c & 7]
+    return np.where(c & 8, -mag, mag) * float(scale)
+
+
+def cobs_subspace_logits(qg: np.ndarray, mean: np.ndarray, counts: np.ndarray, xi: np.ndarray, sigma: float,
+                         U=None):
+    """s_hat[g][b] = sigma q_g . mean_b + (sigma^2 / 2) sum_i (q~_g . xi_bi)^2 + ln n_b
+    with the projected query q~ = U q (U None: the full space, q~ = q) [COBS, the
+    projected quadratic form after (13), exact when the query lies in the subspace].
+    mean: [NB][D] the stored block means; xi: [NB][r][s] the stored factors."""
+    G = qg.shape[0]
+    NB = mean.shape[0]
+    qt = qg if U is None else qg @ np.asarray(U, dtype=np.float64).T
+    out = np.full((G, NB), -math.inf)
+    for b in range(NB):
+        nb = int(counts[b])
+        if nb <= 0:
+            continue
+        for g in range(G):
+            quad = float(np.sum((xi[b] @ qt[g]) ** 2))
+            out[g, b] = sigma * float(qg[g] @ mean[b]) + 0.5 * sigma * sigma * quad + math.log(nb)
+    return out
+
+
 # --------------------------------------------------------------------------- scores
 def logsumexp(x: np.ndarray) -> float:
     """ln sum exp(x) with a max shift; -inf for an empty or all -inf input."""
@@ -498,7 +613,7 @@ def dense_attend_one(qg, K, V, n, sigma):
 
 # --------------------------------------------------------------------------- batched
 def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
-                 k_sum=None, counts=None, bh=None, rank=4):
+                 k_sum=None, counts=None, bh=None, rank=4, stored_xi=None, stored_U=None):
     """Block choice for every (sequence, KV head), or for the listed ones.
 
     q: [B][Hq][D]; K: [B][Hkv][Ncap][D] float64 (needed for exact-mass mode and to
@@ -532,6 +647,20 @@ def select_batch(q, K, seq_lens, L, sigma, k, force_first, force_last, mode,
             ks, _, c, _, _ = block_summaries_one(K[b, h], K[b, h], n, L, NBcap)
             xi, _ = block_cov_factors_one(K[b, h], n, L, NBcap, rank)
             shat = cobs_logits(qg, ks[:nb], c[:nb], xi[:nb], sigma)
+        elif mode == "cobs_stored":
+            # the stored descriptor: bf16 block means and the given factors
+            # (stored_xi[(b, h)]: [NB][r][s], e.g. FP4-decoded) in the subspace of
+            # stored_U[h] ([s][D]; None: the full space)
+            if k_sum is None:
+                ks, _, c, _, _ = block_summaries_one(K[b, h], K[b, h], n, L, NBcap)
+            else:
+                ks, c = k_sum[b, h], counts[b]
+            mean = np.zeros((nb, D))
+            for j in range(nb):
+                if int(c[j]) > 0:
+                    mean[j] = round_bf16(ks[j] / int(c[j]))
+            Uh = None if stored_U is None else stored_U[h]
+            shat = cobs_subspace_logits(qg, mean, c[:nb], stored_xi[(b, h)][:nb], sigma, Uh)
         else:
             raise ValueError(mode)
         S = group_score(shat)

@@ -724,6 +724,144 @@ def pin_wildcat_weights_optimal(seed=28):
             assert J(x) > base, (a, eps)
 
 
+
+def _rotation(r, D):
+    Q, _ = np.linalg.qr(r.normal(size=(D, D)))
+    return Q
+
+
+def pin_query_basis_closed_form(seed=29):
+    """Calibration queries built along the columns of a random rotation R, one row
+    of length sqrt(D lambda_j) per direction, give the second moment R diag(lambda)
+    R^T exactly: the eigenvalues come back sorted and each eigenvector is +-R's
+    column. In a group of two heads the rows of both heads enter the moment."""
+    r = _rng(seed)
+    D, Hkv, G = 6, 2, 2
+    lam = np.array([5.0, 0.5, 3.0, 1.0, 0.25, 2.0])
+    R = _rotation(r, D)
+    rows = [math.sqrt(D * lam[j]) * R[:, j] for j in range(D)]
+    Qc = np.zeros((D // G, Hkv * G, D))
+    for h in range(Hkv):
+        for j in range(D):  # direction j: position j // G, head j % G of the group
+            Qc[j // G, h * G + j % G] = rows[j] * (1 if (j + h) % 2 == 0 else -1)
+    evals, evecs = O.query_basis(Qc, Hkv)
+    order = np.argsort(-lam)
+    for h in range(Hkv):
+        _close(evals[h], lam[order], 1e-12, what="eigenvalues")
+        for k, j in enumerate(order):
+            c = sum(float(evecs[h][k][d]) * float(R[d][j]) for d in range(D))
+            _close(abs(c), 1.0, 1e-10, what="eigenvector direction")
+
+
+def pin_subspace_rank_by_hand():
+    """s: the smallest rank with 90% of the trace per head, the mean over heads
+    rounded up; a cumulative sum equal to 90% counts as reaching it."""
+    ev = np.array([[5.0, 3.0, 1.0, 1.0],    # 5, 8, 9 >= 9: 3
+                   [9.5, 0.3, 0.2, 0.0]])   # 9.5 >= 9: 1
+    s, sh = O.subspace_rank(ev, 0.9)
+    assert sh == [3, 1] and s == 2, (s, sh)
+    ev2 = np.array([[5.0, 3.0, 1.0, 1.0], [4.0, 3.0, 2.0, 1.0], [9.5, 0.5, 0.0, 0.0]])  # 3, 3 (4+3+2=9), 1
+    s2, sh2 = O.subspace_rank(ev2, 0.9)
+    assert sh2 == [3, 3, 1] and s2 == 3, (s2, sh2)  # mean 7/3 rounds up to 3
+    assert O.subspace_rank(np.array([[1.0, 1.0, 1.0, 1.0]]), 0.9)[0] == 4
+
+
+def _py_cov(X):
+    n, D = len(X), len(X[0])
+    mu = [sum(X[k][d] for k in range(n)) / n for d in range(D)]
+    return [[sum((X[k][a] - mu[a]) * (X[k][b] - mu[b]) for k in range(n)) / n for b in range(D)] for a in range(D)]
+
+
+def pin_subspace_factors_exact_in_subspace(seed=30):
+    """With r = s the subspace factors hold B_b whole, so for a query inside the
+    subspace (q = U^T z) the projected quadratic form equals q^T Sigma_b q with the
+    covariance written out as Python sums; with U = I they reproduce the full-space
+    factors' quadratic forms."""
+    r = _rng(seed)
+    D, s_dim, L, n = 7, 3, 5, 12
+    K = r.normal(size=(n, D))
+    U = _rotation(r, D)[:s_dim]  # orthonormal rows
+    xi, lam = O.block_cov_factors_ss_one(K, n, L, 3, s_dim, U)
+    for b, (st, e) in enumerate(O.blocks_of(n, L)):
+        cov = _py_cov(K[st:e].tolist())
+        for _ in range(3):
+            z = r.normal(size=s_dim)
+            q = U.T @ z
+            qt = U @ q
+            got = sum(float(xi[b, i] @ qt) ** 2 for i in range(s_dim))
+            want = sum(q[a] * cov[a][c] * q[c] for a in range(D) for c in range(D))
+            _close(got, want, 1e-10, what="projected quadratic form")
+    xf, lf = O.block_cov_factors_one(K, n, L, 3, 4)
+    xs, ls = O.block_cov_factors_ss_one(K, n, L, 3, 4, np.eye(D))
+    _close(ls, lf, 1e-10, what="identity basis eigenvalues")
+    for b in range(3):
+        for _ in range(3):
+            q = r.normal(size=D)
+            _close(np.sum((xs[b] @ q) ** 2), np.sum((xf[b] @ q) ** 2), 1e-10, what="identity basis forms")
+
+
+def pin_fp4_e2m1_grid_and_ties(seed=31):
+    """E2M1 codes: the grid points times the scale round-trip exactly; every tie
+    between two neighbouring magnitudes goes to the code with mantissa bit 0; the
+    largest magnitude is code 7 (6 x scale); zero keeps code 0; a zero vector has
+    scale 0; each code is the nearest grid point (checked against every point)."""
+    grid = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    for sgn in (1.0, -1.0):
+        x = [sgn * g for g in grid]
+        c, sc = O.fp4_e2m1_quantize(x)
+        assert float(sc) == 1.0
+        _close(O.fp4_e2m1_decode(c, sc), x, 0.0, what="grid round trip")
+        ties = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+        want = [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]  # the even neighbour of each midpoint
+        c, sc = O.fp4_e2m1_quantize([sgn * t for t in ties] + [sgn * 6.0])
+        _close(O.fp4_e2m1_decode(c, sc)[:-1], [sgn * w for w in want], 0.0, what="ties to even")
+        assert int(c[-1]) == (7 if sgn > 0 else 15)
+    c, sc = O.fp4_e2m1_quantize(np.zeros(5))
+    assert float(sc) == 0.0 and not np.any(c)
+    r = _rng(seed)
+    for _ in range(20):
+        x = r.normal(size=33) * math.exp(r.normal())
+        c, sc = O.fp4_e2m1_quantize(x)
+        scale = float(sc)
+        assert abs(scale - float(np.float32(np.max(np.abs(np.float32(x))))) / 6.0) <= 1e-6 * scale
+        dec = O.fp4_e2m1_decode(c, sc)
+        for j in range(len(x)):
+            best = min(abs(abs(float(x[j])) - g * scale) for g in grid)
+            assert abs(abs(dec[j]) - abs(float(x[j]))) <= best + 1e-6 * scale, (j, x[j], dec[j])
+            assert dec[j] == 0.0 or (dec[j] > 0) == (x[j] > 0)
+        assert np.max(np.abs(dec)) == 6.0 * scale
+
+
+def pin_cobs_subspace_logits(seed=32):
+    """The stored-descriptor score: with the full space (U = None), the exact mean
+    and the full-space factors it is the second-order score of cobs_logits; with a
+    query inside the subspace and r = s it is sigma q.mean + (sigma^2 / 2)
+    q^T Sigma_b q + ln n_b written out with Python sums."""
+    r = _rng(seed)
+    D, L, n, sig = 6, 4, 10, 0.4
+    K = r.normal(size=(n, D))
+    NB = 3
+    ks, _, cnt, _, _ = O.block_summaries_one(K, K, n, L, NB)
+    xi, _ = O.block_cov_factors_one(K, n, L, NB, 3)
+    qg = r.normal(size=(2, D))
+    mean = ks / cnt[:, None]
+    _close(O.cobs_subspace_logits(qg, mean, cnt, xi, sig), O.cobs_logits(qg, ks, cnt, xi, sig), 1e-12,
+           what="full space")
+    U = _rotation(r, D)[:2]
+    xs, _ = O.block_cov_factors_ss_one(K, n, L, NB, 2, U)
+    z = r.normal(size=(2, 2))
+    qs = z @ U  # rows inside the subspace
+    got = O.cobs_subspace_logits(qs, mean, cnt, xs, sig, U)
+    for b, (st, e) in enumerate(O.blocks_of(n, L)):
+        cov = _py_cov(K[st:e].tolist())
+        mu = [sum(K[k][d] for k in range(st, e)) / (e - st) for d in range(D)]
+        for g in range(2):
+            q = qs[g]
+            want = (sig * sum(q[d] * mu[d] for d in range(D))
+                    + 0.5 * sig * sig * sum(q[a] * cov[a][c] * q[c] for a in range(D) for c in range(D))
+                    + math.log(e - st))
+            _close(got[g, b], want, 1e-10, what="subspace score")
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -735,4 +873,6 @@ ALL_PINS = [
     pin_cobs_error_order, pin_cobs_eigen_structure, pin_round_bf16_nearest_even, pin_mean16_score,
     pin_wildcat_kernel_bruteforce, pin_rpcholesky_pivot_rule, pin_rpcholesky_interpolates,
     pin_wildcat_all_points_is_exact, pin_wildcat_identical_tokens, pin_wildcat_weights_optimal,
+    pin_query_basis_closed_form, pin_subspace_rank_by_hand, pin_subspace_factors_exact_in_subspace,
+    pin_fp4_e2m1_grid_and_ties, pin_cobs_subspace_logits,
 ]

@@ -229,6 +229,74 @@ def _mut_logsumexp_shift(orig):
     return f
 
 
+
+def _mut_fp4_ties_away(orig):
+    def f(x):
+        x32 = np.asarray(x, dtype=np.float32)
+        codes = np.zeros(x32.shape, dtype=np.uint8)
+        amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0.0)
+        scale = np.float32(amax / np.float32(6.0))
+        if not scale > 0:
+            return codes, np.float32(0.0)
+        for j, v in enumerate(x32):
+            a = abs(float(np.float32(v / scale)))
+            best, bd = 0, None
+            for c, gv in enumerate(O.E2M1_GRID):
+                dist = abs(a - gv)
+                if bd is None or dist <= bd:  # a tie goes to the larger magnitude
+                    best, bd = c, dist
+            codes[j] = best | (8 if (v < 0 and best != 0) else 0)
+        return codes, scale
+    return f
+
+
+def _mut_fp4_scale_by_4(orig):
+    def f(x):
+        x32 = np.asarray(x, dtype=np.float32)
+        amax = np.float32(np.max(np.abs(x32))) if x32.size else np.float32(0.0)
+        scale = np.float32(amax / np.float32(4.0))  # the largest magnitude lands on 4, not 6
+        codes = np.zeros(x32.shape, dtype=np.uint8)
+        if not scale > 0:
+            return codes, np.float32(0.0)
+        for j, v in enumerate(x32):
+            a = abs(float(np.float32(v / scale)))
+            best = min(range(8), key=lambda c: (abs(a - O.E2M1_GRID[c]), c % 2))
+            codes[j] = best | (8 if (v < 0 and best != 0) else 0)
+        return codes, scale
+    return f
+
+
+def _mut_query_basis_first_head(orig):
+    def f(Qc, Hkv):
+        G = Qc.shape[1] // Hkv
+        return orig(Qc[:, ::G, :], Hkv)
+    return f
+
+
+def _mut_subspace_rank_floor(orig):
+    def f(evals, energy=0.9):
+        s, sh = orig(evals, energy)
+        return int(math.floor(sum(sh) / len(sh))), sh
+    return f
+
+
+def _mut_subspace_logits_unprojected(orig):
+    def f(qg, mean, counts, xi, sigma, U=None):
+        if U is None:
+            return orig(qg, mean, counts, xi, sigma, None)
+        # the query's first s coordinates instead of its projection
+        return orig(qg, mean, counts, xi, sigma, np.eye(xi.shape[-1], qg.shape[1]))
+    return f
+
+
+def _mut_ss_factors_full_space_projected(orig):
+    def f(K, n, L, NBcap, r, U):
+        # project the full-space top-r directions instead of decomposing U Sigma U^T
+        xf, lf = O.block_cov_factors_one(K, n, L, NBcap, r)
+        xs = np.einsum("brd,sd->brs", xf, np.asarray(U, dtype=np.float64))
+        return xs, np.sum(xs * xs, axis=2)
+    return f
+
 MUTANTS = {
     "tail_proxy/no ln count": ("tail_proxy", _mut_proxy_no_log_count),
     "tail_proxy/sum not mean": ("tail_proxy", _mut_proxy_sum_value),
@@ -255,6 +323,12 @@ MUTANTS = {
     "cobs/projections not squared": ("cobs_logits", _mut_cobs_unsquared),
     "cobs/sample covariance (n - 1)": ("block_cov_factors_one", _mut_cov_sample),
     "cobs/smallest eigendirections": ("block_cov_factors_one", _mut_cov_smallest),
+    "fp4/ties away from zero": ("fp4_e2m1_quantize", _mut_fp4_ties_away),
+    "fp4/scale max over 4": ("fp4_e2m1_quantize", _mut_fp4_scale_by_4),
+    "query_basis/first head of the group": ("query_basis", _mut_query_basis_first_head),
+    "subspace_rank/mean rounded down": ("subspace_rank", _mut_subspace_rank_floor),
+    "subspace_logits/query not projected": ("cobs_subspace_logits", _mut_subspace_logits_unprojected),
+    "ss_factors/projected full-space directions": ("block_cov_factors_ss_one", _mut_ss_factors_full_space_projected),
 }
 
 
