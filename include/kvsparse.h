@@ -291,6 +291,86 @@ kv_status kv_select_blocks_cobs(const kv_shape* shape, const void* q, float scal
                                 int32_t* n_kept, float* scores, kv_stream_t stream);
 
 /*
+ * The stored second-order descriptor. Source: "COBS: Cumulant Order Block Sparse
+ * Attention" -- the subspace paragraph (keep each block's covariance only within
+ * the span U_Q of the top s eigenvectors of the query second moment E[q q^T], store
+ * the rank-r factors of B_b = U_Q^T Sigma_b U_Q, score with the projected query
+ * U_Q^T q; s set from the rank capturing 90% of the query spectral energy, averaged
+ * over heads) and the quantisation paragraph (the factors in E2M1 FP4 with one fp32
+ * scale per factor, the block mean at bf16).
+ *
+ * kv_build_query_basis -- per KV head h, the eigenvectors of the query second moment
+ * C_h = mean over the Nc calibration positions and the group's Hq / Hkv query heads
+ * of q q^T (float64 accumulation and Jacobi diagonalisation).
+ *   Qc       device [Nc][Hq][D] (bf16 or fp32 per dtype), 16-byte aligned
+ *   evecs    device out [Hkv][D][D] fp32: row j of head h is the unit eigenvector of
+ *            evals[h][j] (sign arbitrary)
+ *   evals    device out [Hkv][D] fp32, descending (ties to the lower index)
+ *   workspace  device, kv_query_basis_workspace_bytes(Hkv, D) bytes (float64 scratch)
+ * D must be 64 or 128 (KV_ERR_UNSUPPORTED); Hq a multiple of Hkv.
+ */
+kv_status kv_build_query_basis(const void* Qc, kv_dtype dtype, int Nc, int Hq, int Hkv, int D, float* evecs,
+                               float* evals, void* workspace, size_t ws_bytes, kv_stream_t stream);
+size_t kv_query_basis_workspace_bytes(int Hkv, int D);
+
+/*
+ * kv_query_subspace_rank -- host function: s = ceil(mean over heads of s_h), s_h the
+ * smallest count of leading eigenvalues of head h whose sum reaches `energy` (0..1]
+ * of the head's total. evals: HOST [Hkv][D] fp32, descending (kv_build_query_basis's,
+ * copied back). Returns s, or -1 for bad arguments.
+ */
+int kv_query_subspace_rank(const float* evals, int Hkv, int D, double energy);
+
+/*
+ * kv_build_block_cov_factors_ss -- per block, the r largest eigenpairs of
+ * B_b = U Sigma_b U^T as scaled eigenvectors xi_i = sqrt(lambda_i) u_i (s values),
+ * Sigma_b the population covariance of the block's keys.
+ *   U      device [Hkv][s][D] fp32: rows the subspace basis (the first s rows of
+ *          kv_build_query_basis's evecs per head)
+ *   s      1..D
+ *   xi_ss  device out [B][Hkv][NBcap][rank][SP] fp32, SP = s rounded up to 32 (values
+ *          past s, directions past B_b's rank, blocks with fewer than two keys and
+ *          blocks past the sequence are zero), 16-byte aligned
+ * block_size <= 64 and D in {64, 128} (KV_ERR_UNSUPPORTED otherwise); rank 1..8.
+ */
+kv_status kv_build_block_cov_factors_ss(const kv_shape* shape, const void* K, const float* U, int s, int rank,
+                                        float* xi_ss, kv_stream_t stream);
+
+/*
+ * kv_quantize_fp4 -- E2M1 FP4 codes of nvec vectors of len fp32 values, one fp32 scale
+ * per vector: scale = max|x| / 6; each x_j / scale (an IEEE fp32 division) goes to
+ * the nearest of the magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6, a tie to the code with
+ * mantissa bit 0, the sign in bit 3 (zero is code 0).
+ *   x       device [nvec][len] fp32, 16-byte aligned; len a multiple of 32, <= 4096
+ *   codes   device out [nvec][len / 2] bytes: element 2j in the low nibble
+ *   scales  device out [nvec] fp32 (0 for an all-zero vector)
+ */
+kv_status kv_quantize_fp4(const float* x, long long nvec, int len, uint8_t* codes, float* scales,
+                          kv_stream_t stream);
+
+/*
+ * kv_select_blocks_cobs_fp4 -- kv_select_blocks with the second-order block logit read
+ * from the stored descriptor:
+ *   s[g,b] = scale * q_g . mean_b + (scale^2 / 2) sum_i (q~_g . xi_bi)^2 + ln n_b,
+ *   q~_g = U q_g (s values; the full space, q~ = q, when U is NULL and s = D),
+ *   xi_bi = code_scales[b][i] * e2m1(codes[b][i]),
+ * and Equation (5) over the group's heads as in kv_select_blocks.
+ *   k_mean       device [B][Hkv][NBcap][D] bf16 block means (kv_build_block_key_means)
+ *   counts       device [B][NBcap] int32 (kv_build_block_summaries)
+ *   U, s         device [Hkv][s][D] fp32 basis, or NULL with s = D
+ *   codes        device [B][Hkv][NBcap][rank][SP / 2] E2M1 codes (kv_quantize_fp4 of
+ *                kv_build_block_cov_factors_ss's output, or of full-space factors),
+ *                SP = s rounded up to 32, 16-byte aligned
+ *   code_scales  device [B][Hkv][NBcap][rank] fp32
+ * bf16 caches only (KV_ERR_UNSUPPORTED otherwise); rank 1..8. Forcing, ranking, kmax,
+ * block_idx, n_kept and scores are as in kv_select_blocks.
+ */
+kv_status kv_select_blocks_cobs_fp4(const kv_shape* shape, const void* q, float scale, const void* k_mean,
+                                    const int32_t* counts, const float* U, int s, const uint8_t* codes,
+                                    const float* code_scales, int rank, int k_top, int force_first, int force_last,
+                                    int kmax, int32_t* block_idx, int32_t* n_kept, float* scores, kv_stream_t stream);
+
+/*
  * kv_sparse_decode_attn -- softmax attention over a reduced KV cache.
  *
  * Block mode (tok_idx == NULL). Source: "OpenAttention reads 1% of the KV cache

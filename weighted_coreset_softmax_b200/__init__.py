@@ -31,7 +31,8 @@ __all__ = [
     "kv_select_blocks_mean16",
     "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace", "kv_selftest_wait_timeout",
-    "kv_stream_read", "kv_build_wildcat_coreset",
+    "kv_stream_read", "kv_build_wildcat_coreset", "kv_build_query_basis", "kv_query_subspace_rank",
+    "kv_build_block_cov_factors_ss", "kv_quantize_fp4", "kv_select_blocks_cobs_fp4",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
@@ -100,6 +101,11 @@ def lib():
         "kv_selftest_wait_timeout": [_P, _P, ctypes.c_uint64, _I, _P],
         "kv_stream_read": [_P, _S, _P, _P],
         "kv_build_wildcat_coreset": [_SHP, _P, _F, _I, _I, _P, _P, _P, _P, _P, _S, _P],
+        "kv_build_query_basis": [_P, _I, _I, _I, _I, _I, _P, _P, _P, _S, _P],
+        "kv_build_block_cov_factors_ss": [_SHP, _P, _P, _I, _I, _P, _P],
+        "kv_quantize_fp4": [_P, ctypes.c_longlong, _I, _P, _P, _P],
+        "kv_select_blocks_cobs_fp4": [_SHP, _P, _F, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P],
+        "kv_query_subspace_rank": [_P, _I, _I, ctypes.c_double],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -109,6 +115,8 @@ def lib():
     L.kv_workspace_bytes.restype = _S
     L.kv_wildcat_workspace_bytes.argtypes = [_SHP, _I]
     L.kv_wildcat_workspace_bytes.restype = _S
+    L.kv_query_basis_workspace_bytes.argtypes = [_I, _I]
+    L.kv_query_basis_workspace_bytes.restype = _S
     L.kv_last_error.argtypes = []
     L.kv_last_error.restype = ctypes.c_char_p
     _lib = L
@@ -534,3 +542,97 @@ def kv_build_wildcat_coreset(K: torch.Tensor, seq_lens: torch.Tensor, scale: flo
                                           _ptr(w), _ptr(n_sel), _ptr(workspace),
                                           workspace.numel() * workspace.element_size(), _stream(K.device)))
     return tok_idx, w, n_sel
+
+
+# ----------------------------------------------------------------- stored second-order descriptor
+def kv_build_query_basis(Qc: torch.Tensor, Hkv: int):
+    """Eigenvectors (rows, [Hkv][D][D] fp32) and descending eigenvalues ([Hkv][D]) of
+    each KV head's query second moment over calibration queries Qc [Nc][Hq][D]."""
+    _need(Qc, "Qc")
+    Nc, Hq, D = Qc.shape
+    dev = Qc.device
+    evecs = torch.empty(Hkv, D, D, dtype=torch.float32, device=dev)
+    evals = torch.empty(Hkv, D, dtype=torch.float32, device=dev)
+    need = int(lib().kv_query_basis_workspace_bytes(int(Hkv), int(D)))
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _check(lib().kv_build_query_basis(_ptr(Qc), _dtype_code(Qc.dtype), int(Nc), int(Hq), int(Hkv), int(D),
+                                      _ptr(evecs), _ptr(evals), _ptr(ws), ws.numel(), _stream(dev)))
+    return evecs, evals
+
+
+def kv_query_subspace_rank(evals: torch.Tensor, energy: float = 0.9) -> int:
+    """s from the basis eigenvalues [Hkv][D] (copied to the host for the library's
+    host function)."""
+    ev = evals.detach().to("cpu", torch.float32).contiguous()
+    Hkv, D = ev.shape
+    s = int(lib().kv_query_subspace_rank(ctypes.c_void_p(ev.data_ptr()), int(Hkv), int(D), float(energy)))
+    if s < 0:
+        raise KVError(KV_ERR_INVALID_ARG, "kv_query_subspace_rank: bad arguments")
+    return s
+
+
+def kv_build_block_cov_factors_ss(K: torch.Tensor, seq_lens: torch.Tensor, block_size: int, U: torch.Tensor,
+                                  rank: int = 4, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Per-block factors of the covariance within the subspace of U [Hkv][s][D]:
+    [B][Hkv][NB][rank][SP] fp32, SP = s rounded up to 32 (zero past s)."""
+    _need(K, "K")
+    _need(seq_lens, "seq_lens", torch.int32)
+    _need(U, "U", torch.float32)
+    B, Hkv, Ncap, D = K.shape
+    s = int(U.shape[1])
+    SP = (s + 31) // 32 * 32
+    NB = (Ncap + block_size - 1) // block_size
+    if out is None:
+        out = torch.empty(B, Hkv, NB, rank, SP, dtype=torch.float32, device=K.device)
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, block_size, _dtype_code(K.dtype), seq_lens.data_ptr())
+    _check(lib().kv_build_block_cov_factors_ss(ctypes.byref(shape), _ptr(K), _ptr(U), s, int(rank), _ptr(out),
+                                               _stream(K.device)))
+    return out
+
+
+def kv_quantize_fp4(x: torch.Tensor):
+    """E2M1 codes of the vectors along x's last axis (a multiple of 32 long) with one
+    fp32 scale each: (codes uint8 [..., len / 2], scales fp32 [...])."""
+    _need(x, "x", torch.float32)
+    length = int(x.shape[-1])
+    nvec = x.numel() // length if length else 0
+    codes = torch.empty(*x.shape[:-1], length // 2, dtype=torch.uint8, device=x.device)
+    scales = torch.empty(*x.shape[:-1], dtype=torch.float32, device=x.device)
+    _check(lib().kv_quantize_fp4(_ptr(x), int(nvec), length, _ptr(codes), _ptr(scales), _stream(x.device)))
+    return codes, scales
+
+
+def kv_select_blocks_cobs_fp4(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, block_size: int,
+                              scale: float, k_mean: torch.Tensor, counts: torch.Tensor, U: Optional[torch.Tensor],
+                              codes: torch.Tensor, code_scales: torch.Tensor, rank: int, k_top: int,
+                              force_first: bool = False, force_last: bool = False, kmax: Optional[int] = None,
+                              block_idx: Optional[torch.Tensor] = None, n_kept: Optional[torch.Tensor] = None,
+                              scores: Optional[torch.Tensor] = None, want_scores: bool = False):
+    """Kept blocks per KV head scored with the stored second-order descriptor (bf16
+    means, E2M1 factors, the query subspace of U or the full space when U is None).
+    Returns (block_idx [B][Hkv][kmax], n_kept [B][Hkv], scores or None)."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_mean, "k_mean", torch.bfloat16)
+    _need(counts, "counts", torch.int32)
+    _need(codes, "codes", torch.uint8)
+    _need(code_scales, "code_scales", torch.float32)
+    if U is not None:
+        _need(U, "U", torch.float32)
+    shape = make_shape(q, K, seq_lens, block_size)
+    s = int(U.shape[1]) if U is not None else shape.D
+    NB = (shape.Ncap + block_size - 1) // block_size
+    forced = int(bool(force_first)) + int(bool(force_last))
+    if kmax is None:
+        kmax = max(1, min(NB, k_top + forced))
+    dev = q.device
+    if block_idx is None:
+        block_idx = torch.zeros(shape.B, shape.Hkv, kmax, dtype=torch.int32, device=dev)
+    if n_kept is None:
+        n_kept = torch.zeros(shape.B, shape.Hkv, dtype=torch.int32, device=dev)
+    if scores is None and want_scores:
+        scores = torch.empty(shape.B, shape.Hkv, NB, dtype=torch.float32, device=dev)
+    _check(lib().kv_select_blocks_cobs_fp4(ctypes.byref(shape), _ptr(q), float(scale), _ptr(k_mean), _ptr(counts),
+                                           _ptr(U), s, _ptr(codes), _ptr(code_scales), int(rank), int(k_top),
+                                           int(bool(force_first)), int(bool(force_last)), int(kmax),
+                                           _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
+    return block_idx, n_kept, scores

@@ -109,14 +109,14 @@ static cudaError_t cov_td(const void* K, const int32_t* seq_lens, float* xi, int
   int dev = 0;
   cudaGetDevice(&dev);
   if (!(configured.load() & (1 << (dev & 31)))) {
-    const cudaError_t e = cudaFuncSetAttribute(cov_factors_kernel<T, D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    const cudaError_t e = cudaFuncSetAttribute(cov_factors_kernel<T, D, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                static_cast<int>(cov_smem_bytes(COV_MAX_ROWS, D)));
     if (e != cudaSuccess) return e;
     configured.fetch_or(1 << (dev & 31));
   }
   const long long grid = static_cast<long long>(NBH) * NBcap;
-  cov_factors_kernel<T, D><<<static_cast<unsigned>(grid), COV_THREADS, smem, st>>>(static_cast<const T*>(K), seq_lens, xi,
-                                                                                  Hkv, Ncap, L, NBcap, r);
+  cov_factors_kernel<T, D, false><<<static_cast<unsigned>(grid), COV_THREADS, smem, st>>>(
+      static_cast<const T*>(K), seq_lens, xi, Hkv, Ncap, L, NBcap, r, nullptr, 0, 0);
   return cudaGetLastError();
 }
 
@@ -556,7 +556,9 @@ namespace {
 kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_mode, const float* k_sum,
                      const void* k_bounds, const int32_t* counts, const void* K, int k_top, int force_first,
                      int force_last, int kmax, int32_t* block_idx, int32_t* n_kept, float* scores,
-                     kv_stream_t stream, const float* k_xi = nullptr, int rank = 0, const void* k_mean16 = nullptr) {
+                     kv_stream_t stream, const float* k_xi = nullptr, int rank = 0, const void* k_mean16 = nullptr,
+                     const uint8_t* xi4 = nullptr, const float* xi4_scale = nullptr, const float* Uq = nullptr,
+                     int s_dim = 0) {
   KV_TRY(check_shape(shape));
   if (!std::isfinite(scale)) return fail(KV_ERR_INVALID_ARG, "scale is not finite");
   KV_TRY(need(q, "q"));
@@ -570,10 +572,19 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
     }
   } else if (sel_mode == kvs::SEL_EXACT) {
     KV_TRY(need(K, "K"));
-  } else if (sel_mode == kvs::SEL_MEAN16) {
+  } else if (sel_mode == kvs::SEL_MEAN16 || sel_mode == kvs::SEL_COBS4) {
     if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "bf16-mean scoring is built for bf16 caches only");
     KV_TRY(need(k_mean16, "k_mean"));
     KV_TRY(need(counts, "counts", 4));
+    if (sel_mode == kvs::SEL_COBS4) {
+      KV_TRY(need(xi4, "codes"));
+      KV_TRY(need(xi4_scale, "code_scales", 4));
+      if (Uq) KV_TRY(need(Uq, "U", 4));
+      if (rank < 1 || rank > kvs::COV_MAX_RANK)
+        return fail(KV_ERR_INVALID_ARG, "rank = %d outside 1..%d", rank, kvs::COV_MAX_RANK);
+      if (Uq ? (s_dim < 1 || s_dim > shape->D) : s_dim != shape->D)
+        return fail(KV_ERR_INVALID_ARG, "s = %d: 1..D with a basis, D without one", s_dim);
+    }
   } else {
     if (shape->dtype != KV_BF16) return fail(KV_ERR_UNSUPPORTED, "Quest scoring reads bf16 bounds (bf16 caches only)");
     KV_TRY(need(k_bounds, "k_bounds"));
@@ -596,6 +607,11 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
   p.k_mean16 = k_mean16;
   p.k_xi = k_xi;
   p.cobs_r = rank;
+  p.xi4 = xi4;
+  p.xi4_scale = xi4_scale;
+  p.Uq = Uq;
+  p.s_dim = s_dim;
+  p.SP = (s_dim + 31) & ~31;
   p.counts = counts;
   p.K = K;
   p.seq_lens = shape->seq_lens;
@@ -645,6 +661,14 @@ kv_status kv_select_blocks_cobs(const kv_shape* shape, const void* q, float scal
                                 kv_stream_t stream) {
   return select_any(shape, q, scale, kvs::SEL_COBS, k_sum, nullptr, counts, nullptr, k_top, force_first, force_last,
                     kmax, block_idx, n_kept, scores, stream, k_xi, rank);
+}
+
+kv_status kv_select_blocks_cobs_fp4(const kv_shape* shape, const void* q, float scale, const void* k_mean,
+                                    const int32_t* counts, const float* U, int s, const uint8_t* codes,
+                                    const float* code_scales, int rank, int k_top, int force_first, int force_last,
+                                    int kmax, int32_t* block_idx, int32_t* n_kept, float* scores, kv_stream_t stream) {
+  return select_any(shape, q, scale, kvs::SEL_COBS4, nullptr, nullptr, counts, nullptr, k_top, force_first, force_last,
+                    kmax, block_idx, n_kept, scores, stream, nullptr, rank, k_mean, codes, code_scales, U, s);
 }
 
 kv_status kv_select_blocks_quest(const kv_shape* shape, const void* q, float scale, const void* k_bounds, int k_top,

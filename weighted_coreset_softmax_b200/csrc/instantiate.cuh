@@ -153,7 +153,7 @@ cudaError_t select_launch_mode(const SelParams& p, int grid, cudaStream_t st) {
   static std::atomic<int> configured{0};  // one bit per device: smem limit raised
   int dev = 0;
   cudaGetDevice(&dev);
-  if constexpr ((MODE == SEL_QUEST || MODE == SEL_MEAN16) && sizeof(T) != 2)
+  if constexpr ((MODE == SEL_QUEST || MODE == SEL_MEAN16 || MODE == SEL_COBS4) && sizeof(T) != 2)
     return cudaErrorInvalidValue;  // bf16 bounds and bf16 means: bf16 caches only
   const size_t smem = MODE != SEL_EXACT ? sel_summary_smem_bytes(G, p.NBcap) : sel_smem_bytes(G, p.NBcap);
   if (!(configured.load() & (1 << (dev & 31)))) {
@@ -178,6 +178,10 @@ cudaError_t select_launch_one(int mode, const SelParams& p, int grid, cudaStream
   }
   if (mode == SEL_MEAN16) {
     if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_MEAN16>(p, grid, st);
+    return cudaErrorInvalidValue;
+  }
+  if (mode == SEL_COBS4) {
+    if constexpr (sizeof(T) == 2) return select_launch_mode<T, D, G, SEL_COBS4>(p, grid, st);
     return cudaErrorInvalidValue;
   }
   if (mode == SEL_COBS) return select_launch_mode<T, D, G, SEL_COBS>(p, grid, st);

@@ -26,13 +26,15 @@
 #include "common.cuh"
 #include "rank.cuh"
 
+#include <cuda_fp4.h>
+
 namespace kvs {
 
 constexpr int SEL_THREADS = 256;
 constexpr int SEL_NW = SEL_THREADS / 32;
 constexpr int SEL_MAXNB = 4096;  // NBcap limit
 
-enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2, SEL_COBS = 3, SEL_MEAN16 = 4 };
+enum SelMode { SEL_SUMMARY = 0, SEL_EXACT = 1, SEL_QUEST = 2, SEL_COBS = 3, SEL_MEAN16 = 4, SEL_COBS4 = 5 };
 // Row kinds of the summary-style scorer: fp32 key sums, Quest (min, max) bf16
 // pairs (both four bytes a channel), bf16 block means (two bytes a channel).
 enum SelRow { ROW_SUM32 = 0, ROW_QUEST = 1, ROW_MEAN16 = 2 };
@@ -44,6 +46,14 @@ struct SelParams {
   const void* k_mean16;  // bf16-mean mode: [B][Hkv][NBcap][D] bf16 block mean keys
   const float* k_xi;     // second-order mode: [B][Hkv][NBcap][cobs_r][D] fp32 scaled eigenvectors
   int cobs_r;
+  // stored-descriptor second-order mode: [B][Hkv][NBcap][cobs_r][SP / 2] E2M1 codes
+  // (element 2j in the low nibble), [B][Hkv][NBcap][cobs_r] fp32 scales, and the
+  // query basis U [Hkv][s_dim][D] (NULL: the full space, s_dim = D); SP = s_dim
+  // rounded up to 32
+  const uint8_t* xi4;
+  const float* xi4_scale;
+  const float* Uq;
+  int s_dim, SP;
   const int32_t* counts;
   const void* K;
   const int32_t* seq_lens;
@@ -570,6 +580,89 @@ __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, i
   // every copy issued was waited for above (batches m >= nmine issue none)
 }
 
+// Second-order term from the stored descriptor ("COBS: Cumulant Order Block Sparse
+// Attention", the subspace and quantisation paragraphs): adds
+// (sigma^2 / 2) sum_i (q~ . xi_i)^2 to lg, q~ = U q the projected query (qt: the
+// log2-domain q~ of the G heads, [G][SP] in shared memory, zero past s) and
+// xi_i = scale_i * e2m1(codes_i). Each half-warp takes one block: lane c of the half
+// holds nibble columns 8c .. 8c+7 of every factor (one 32-bit word a factor),
+// decodes them with the E2M1 -> f16x2 conversion, forms its partial dots for every
+// (head, factor) pair, and a transpose reduction over the half's 16 lanes sums them
+// (NV - 1 shuffles for NV pairs). The squared dots, times scale_i^2, are summed
+// over the factors through a per-warp scratch.
+template <int G, int RMAX>
+__device__ void cobs_fp4_second_order(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float* qt,
+                                      float* scratch) {
+  constexpr int GP = pow2ceil(G);
+  constexpr int NV = GP * RMAX;
+  constexpr int NH = NV >= 16 ? NV / 16 : 1;    // values a lane holds after the reduction
+  constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes holding each value (NV < 16)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int hw = lane >> 4, c = lane & 15;
+  const int r = p.cobs_r, SP = p.SP;
+  const bool active = c < SP / 8;
+  float qv[G][8];
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) qv[g][k] = active ? qt[g * SP + 8 * c + k] : 0.f;
+  float* scr = scratch + (warp * 2 + hw) * NV;
+  const size_t fbytes = static_cast<size_t>(SP) / 2;  // bytes a factor
+  for (int b2 = warp * 2; b2 < nbv; b2 += SEL_NW * 2) {  // warp-uniform
+    const int b = b2 + hw;
+    const bool live = b < nbv;
+    const size_t fb = (static_cast<size_t>(bh) * p.NBcap + b) * r;  // first factor of block b
+    uint32_t w[RMAX];
+#pragma unroll
+    for (int i = 0; i < RMAX; ++i)
+      w[i] = (active && live && i < r) ? __ldg(reinterpret_cast<const uint32_t*>(p.xi4 + (fb + i) * fbytes) + c) : 0u;
+    float part[NV];
+#pragma unroll
+    for (int i = 0; i < RMAX; ++i) {
+      float x[8];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __half2 h2 = __half2(__nv_cvt_fp4x2_to_halfraw2(
+            static_cast<__nv_fp4x2_storage_t>((w[i] >> (8 * k)) & 0xffu), __NV_E2M1));
+        const float2 f2 = __half22float2(h2);
+        x[2 * k] = f2.x;
+        x[2 * k + 1] = f2.y;
+      }
+#pragma unroll
+      for (int g = 0; g < GP; ++g) {
+        float d = 0.f;
+        if (g < G) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) d = fmaf(qv[g][k], x[k], d);
+        }
+        part[g * RMAX + i] = d;
+      }
+    }
+    transpose_reduce<NV, 8>(part, lane);
+    __syncwarp();
+#pragma unroll
+    for (int j = 0; j < NH; ++j) {
+      const int idx = NV >= 16 ? c * NH + j : c / REP;
+      const int g = idx / RMAX, i = idx - (idx / RMAX) * RMAX;
+      if (c % REP == 0) {
+        float v = 0.f;
+        if (live && g < G && i < r) {
+          const float sc = __ldg(p.xi4_scale + fb + i);
+          v = part[j] * part[j] * sc * sc;
+        }
+        scr[idx] = v;
+      }
+    }
+    __syncwarp();
+    if (live && c < G) {
+      float sum = 0.f;
+      for (int i = 0; i < r; ++i) sum += scr[c * RMAX + i];
+      lg[c * nbp + b] += 0.34657359027997264f * sum;  // ln 2 / 2
+    }
+    __syncwarp();
+  }
+}
+
 template <typename T, int D, int G, int MODE>
 __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams p) {
   extern __shared__ __align__(16) unsigned char sel_smem[];
@@ -585,7 +678,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   const int n = max(0, min(p.seq_lens[b], p.Ncap));
   const int nbv = (n + p.L - 1) / p.L;
 
-  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS || MODE == SEL_MEAN16) {
+  if (MODE == SEL_SUMMARY || MODE == SEL_QUEST || MODE == SEL_COBS || MODE == SEL_MEAN16 || MODE == SEL_COBS4) {
     // the scorer ring's mbarriers (one per warp and stage)
     if (tid == 0) {
 #pragma unroll
@@ -597,7 +690,8 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
     __syncthreads();
     int* cnt = reinterpret_cast<int*>(sel_smem + sel_smem_bytes(G, p.NBcap));
     float4* ring = reinterpret_cast<float4*>(sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-    score_summary<T, D, G, MODE == SEL_QUEST ? ROW_QUEST : (MODE == SEL_MEAN16 ? ROW_MEAN16 : ROW_SUM32)>(
+    score_summary<T, D, G,
+                  MODE == SEL_QUEST ? ROW_QUEST : ((MODE == SEL_MEAN16 || MODE == SEL_COBS4) ? ROW_MEAN16 : ROW_SUM32)>(
         p, lg, nbp, bh, nbv, ring, cnt, ms);
   }
   else
@@ -638,6 +732,35 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
     } else {
       cobs_second_order<D, G, 1, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qf);
     }
+    __syncthreads();
+  }
+
+  if constexpr (MODE == SEL_COBS4) {
+    // the first-order (bf16-mean) logits are in lg; the projected queries and the
+    // per-warp scratch go where the scorer's ring was
+    float* qt = reinterpret_cast<float*>(
+        sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
+    float* scratch = qt + G * p.SP;
+    const int h = bh - b * p.Hkv;
+    const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D;
+    for (int e = tid; e < G * p.SP; e += SEL_THREADS) {
+      const int g = e / p.SP, j = e - (e / p.SP) * p.SP;
+      float v = 0.f;
+      if (j < p.s_dim) {
+        if (p.Uq) {
+          const float* u = p.Uq + (static_cast<size_t>(h) * p.s_dim + j) * D;
+          for (int d = 0; d < D; ++d) v = fmaf(__ldg(u + d), load_as_float(qrow + g * D + d), v);
+        } else {
+          v = load_as_float(qrow + g * D + j);
+        }
+      }
+      qt[e] = v * p.qscale;
+    }
+    __syncthreads();
+    if (p.cobs_r <= 4)
+      cobs_fp4_second_order<G, 4>(p, lg, nbp, bh, nbv, qt, scratch);
+    else
+      cobs_fp4_second_order<G, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qt, scratch);
     __syncthreads();
   }
 

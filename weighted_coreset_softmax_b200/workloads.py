@@ -17,7 +17,12 @@ of that suite is reproduced.
 Key distribution: k = s_c * z with z ~ N(0, 1) and a per-(sequence, KV head,
 channel) scale s_c ~ lognormal(0, 0.5); a number of planted heavy-hitter tokens per
 KV head have keys hh_gain * unit(sum of the group's queries) + N(0, 0.1^2).
-Values ~ N(0, 1). Queries ~ N(0, 1).
+Values ~ N(0, 1). Queries ~ N(0, 1), except in the stored-descriptor workload
+(llama_cobs_fp4), whose queries are anisotropic: q = R (sigma * z) with z ~ N(0, I),
+a seeded rotation R and sigma_j^2 proportional to exp(-j / 45) (normalised to
+E|q|^2 = D), so that about 85 of 128 directions carry 90% of the query energy --
+the subspace size the COBS page reports at D = 128 (340 = 4 x 85 floats per block).
+Its calibration queries (calibration_queries) come from the same model.
 
 Draw order per generator: q, channel scales, K, V, planted positions, planted
 noise, then (weighted workloads) coreset indices and weights.
@@ -54,6 +59,7 @@ class Workload:
     V: Optional[torch.Tensor] = None        # [B][Hkv][Ncap][D]
     tok_idx: Optional[torch.Tensor] = None  # [B][Hkv][m] int32
     w: Optional[torch.Tensor] = None        # [B][Hkv][m] fp32
+    q_model: Optional[tuple] = None         # (R [D][D], sigma [D]) of anisotropic queries
 
     @property
     def G(self) -> int:
@@ -73,11 +79,25 @@ class Workload:
         return torch.tensor(self.seq_lens, dtype=torch.int32, device=device)
 
 
+def query_model(D: int, tau: float = 45.0, seed: int = 77):
+    """The anisotropic query distribution: (R, sigma) with R a seeded rotation (QR of
+    a Gaussian matrix, drawn on the CPU so every device sees the same one) and
+    sigma_j = sqrt(lambda_j), lambda_j proportional to exp(-j / tau), sum lambda = D."""
+    g = torch.Generator().manual_seed(seed)
+    R, _ = torch.linalg.qr(torch.randn(D, D, generator=g, dtype=torch.float64))
+    lam = torch.exp(-torch.arange(D, dtype=torch.float64) / tau)
+    lam = lam * (D / lam.sum())
+    return R.to(torch.float32), lam.sqrt().to(torch.float32)
+
+
 def _draw_sequence(gen, device, Hq, Hkv, D, N, n_planted, hh_gain, dtype,
-                   q_scale=1.0, channel_sigma=0.5, plain=False):
+                   q_scale=1.0, channel_sigma=0.5, plain=False, q_model=None):
     """Draws one sequence's query and cache. Returns q [Hq][D], K, V [Hkv][N][D]."""
     G = Hq // Hkv
     q = torch.randn(Hq, D, generator=gen, device=device, dtype=torch.float32) * q_scale
+    if q_model is not None:
+        R, sig = q_model
+        q = (q * sig.to(device)) @ R.to(device).T
     if plain:
         K = torch.randn(Hkv, N, D, generator=gen, device=device, dtype=torch.float32)
         V = torch.randn(Hkv, N, D, generator=gen, device=device, dtype=torch.float32)
@@ -118,7 +138,8 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
     "llama" (batch 32, 32K, seeds 100..131), "qwen_long" (batch 8, 128K, G=7),
     "llama_osa" (exact-mass scoring), "llama_quest" (key-box bound scoring),
     "llama_cobs" (second-order scoring, rank-4 covariance factors),
-    "llama_coreset" (weighted coreset, m=2048).
+    "llama_cobs_fp4" (the stored descriptor: bf16 means, query-subspace E2M1
+    factors; anisotropic queries), "llama_coreset" (weighted coreset, m=2048).
     Keyword overrides shrink a workload for fast tests while keeping its head
     shapes and distributions.
     """
@@ -151,6 +172,10 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=None, ff=1, fl=1, smode="cobs", amode="proxy", planted=32,
                     seeds=[5], per_seq=False, plain=False)
+    elif name == "llama_cobs_fp4":
+        spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
+                    k_top=None, ff=1, fl=1, smode="cobs_fp4", amode="proxy", planted=32,
+                    seeds=[6], per_seq=False, plain=False, aniso=True)
     elif name == "llama_coreset":
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=0, ff=0, fl=0, smode="summary", amode="weighted", planted=32,
@@ -188,6 +213,8 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
     seeds = spec["seeds"]
     if seed is not None:
         seeds = [seed + i for i in range(len(seeds))]
+    qm = query_model(spec["D"]) if spec.get("aniso") else None
+    wl.q_model = qm
     gen = None
     for b in range(Bv):
         if spec["per_seq"] or gen is None:
@@ -195,7 +222,7 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
             gen = torch.Generator(device=dev)
             gen.manual_seed(s)
         qb, Kb, Vb = _draw_sequence(gen, dev, wl.Hq, wl.Hkv, wl.D, N, n_planted, hh_gain,
-                                    wl.dtype, q_scale=q_scale, plain=spec["plain"])
+                                    wl.dtype, q_scale=q_scale, plain=spec["plain"], q_model=qm)
         q[b], K[b], V[b] = qb, Kb, Vb
     wl.q, wl.K, wl.V = q, K, V
     if wl.attn_mode == "weighted":
@@ -222,3 +249,16 @@ def equalize_tail(wl: Workload, kept_blocks) -> None:
                 tail = wl.K[b, h, :n][mask].to(torch.float64)
                 mean = tail.mean(dim=0).to(wl.dtype)
                 wl.K[b, h, :n][mask] = mean
+
+
+def calibration_queries(wl: Workload, Nc: int, seed: int = 9001) -> torch.Tensor:
+    """Nc calibration positions of queries [Nc][Hq][D] (the workload's dtype) from the
+    workload's query distribution (its anisotropic model when it has one)."""
+    dev = wl.q.device if wl.q is not None else torch.device("cpu")
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(seed)
+    z = torch.randn(Nc, wl.Hq, wl.D, generator=gen, device=dev, dtype=torch.float32)
+    if wl.q_model is not None:
+        R, sig = wl.q_model
+        z = (z * sig.to(dev)) @ R.to(dev).T
+    return z.to(wl.dtype)
