@@ -47,7 +47,7 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama", choices=["llama", "llama_b1", "qwen_long", "llama_osa", "llama_quest",
-                                                           "llama_cobs", "llama_coreset"])
+                                                           "llama_cobs", "llama_cobs_fp4", "llama_coreset"])
     ap.add_argument("--scorer", choices=["mean16", "sum32"], default="mean16",
                     help="summary-mode selection: bf16 block means (default) or fp32 block sums")
     ap.add_argument("--attn", choices=["v1", "v2"], default=None,
@@ -176,6 +176,9 @@ NCU_TRAFFIC = {
 }
 
 
+CALIB_POSITIONS = 512  # calibration query positions for the stored descriptor's basis
+
+
 def measured_peak_hbm():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -246,6 +249,20 @@ def cobs_select_bytes(wl, seq_lens, rank=4):
     return total
 
 
+def cobs_fp4_select_bytes(wl, seq_lens, s_dim, rank=4):
+    """Algorithmic bytes of one kv_select_blocks_cobs_fp4 launch: every valid block's
+    bf16 mean, count, rank E2M1 factors of SP / 2 bytes and rank fp32 scales, q, the
+    kept indices, and the query basis (Hkv x s x D fp32, counted once: every
+    sequence's CTA of a KV head reads the same rows)."""
+    L, D, G = wl.block_size, wl.D, wl.G
+    SP = (s_dim + 31) // 32 * 32
+    total = wl.Hkv * s_dim * D * 4
+    for b in range(wl.B):
+        nbv = (seq_lens[b] + L - 1) // L
+        total += wl.Hkv * (nbv * (D * 2 + 4 + rank * (SP // 2) + rank * 4) + G * D * 2 + wl.kmax * 4 + 4)
+    return total
+
+
 def osa_select_bytes(wl, seq_lens):
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
     return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
@@ -293,6 +310,27 @@ def _oracle_task(args):
     if kind == "dense":
         O.dense_batch(q, K, V, [n], scale)
         return None
+    if kind == "cobs_fp4":
+        # the oracle's own stored descriptor of this pair: factors within its basis
+        # (stored at fp32), rounded to fp32 and E2M1-coded with float32 decisions
+        U_pad, s_dim, rank = extra
+        SP = U_pad.shape[0]
+        NBc = (K.shape[2] + L - 1) // L
+        xo, _ = O.block_cov_factors_ss_one(K[0, 0], n, L, NBc, rank, U_pad[:s_dim])
+        dec = np.zeros((NBc, rank, SP))
+        x32 = np.zeros((NBc, rank, SP), dtype=np.float32)
+        x32[:, :, :s_dim] = xo.astype(np.float32)
+        for blk in range(NBc):
+            for i in range(rank):
+                c, sc = O.fp4_e2m1_quantize(x32[blk, i])
+                dec[blk, i] = O.fp4_e2m1_decode(c, sc)
+        sel = O.select_batch(q, K, [n], L, scale, k_top, ff, fl, "cobs_stored", rank=rank, stored_xi={(0, 0): dec},
+                             stored_U=U_pad[None])
+        s = sel[(0, 0)]
+        O.sparse_batch(q, K, V, [n], L, scale, {(0, 0): s["kept"]}, True)
+        nb = (n + L - 1) // L
+        return {"kept": s["kept"], "near_tie": s["near_tie"],
+                "more": {k: O.select_blocks(s["S"], nb, k, ff, fl) for k in more_k}}
     sel, _, _ = O.decode_step(q, K, V, [n], L, scale, k_top, ff, fl, score_mode=kind, use_proxy=True)
     s = sel[(0, 0)]
     nb = (n + L - 1) // L
@@ -314,9 +352,20 @@ def _pool_init():
 def oracle_tasks(wl, pairs, more_k=()):
     import numpy as np
     import torch
+    from weighted_coreset_softmax_b200 import workloads as W
     tasks = []
     kind = {"summary": "summary", "summary_mean16": "summary_mean16", "exact_mass": "exact_mass", "quest": "quest",
-            "cobs": "cobs"}[wl.score_mode]
+            "cobs": "cobs", "cobs_fp4": "cobs_fp4"}[wl.score_mode]
+    if kind == "cobs_fp4" and not hasattr(wl, "oracle_basis"):
+        # the oracle's basis and s from the calibration queries, stored at fp32
+        from oracle import oracle as O
+        Qc = W.calibration_queries(wl, CALIB_POSITIONS).to(torch.float64).cpu().numpy()
+        ev, vec = O.query_basis(Qc, wl.Hkv)
+        s_o, _ = O.subspace_rank(ev, 0.9)
+        SP = (s_o + 31) // 32 * 32
+        U_pad = np.zeros((wl.Hkv, SP, wl.D))
+        U_pad[:, :s_o] = vec[:, :s_o, :].astype(np.float32).astype(np.float64)
+        wl.oracle_basis = (U_pad, s_o)
     if wl.attn_mode == "weighted":
         kind = "weighted"
     for (b, h) in pairs:
@@ -329,6 +378,8 @@ def oracle_tasks(wl, pairs, more_k=()):
         extra = None
         if kind == "weighted":
             extra = (wl.tok_idx[b, h].cpu().numpy(), wl.w[b, h].cpu().numpy().astype(np.float64))
+        if kind == "cobs_fp4":
+            extra = (wl.oracle_basis[0][h], wl.oracle_basis[1], 4)
         tasks.append((kind, q, K, V, wl.seq_lens[b], wl.block_size, wl.scale, wl.k_top,
                       bool(wl.force_first), bool(wl.force_last), extra, tuple(more_k)))
     return tasks
@@ -412,8 +463,10 @@ def selection_check(wl, oracle_res, idx, nk, idx5=None, nk5=None, more_k=()):
                 out5["near_tie_mismatch"] += 1
             else:
                 out5["other_mismatch"] += 1
-    out["reference"] = ("float64 oracle, " + ("bf16-mean ranking" if wl.score_mode == "summary_mean16" else
-                                               "exact-mean ranking") + ", pairs of the CPU baseline sample")
+    ranking = {"summary_mean16": "bf16-mean ranking",
+               "cobs_fp4": "stored-descriptor ranking (the oracle's own basis, factors and E2M1 codes)"}
+    out["reference"] = ("float64 oracle, " + ranking.get(wl.score_mode, "exact-mean ranking")
+                        + ", pairs of the CPU baseline sample")
     if out5 is not None:
         out["budget_5pct"] = out5
     return out
@@ -428,6 +481,8 @@ def workload_label(wl, budget):
         "llama_osa": "Llama-3.1-8B-shaped GQA decode, OSA exact-mass selection",
         "llama_quest": "Llama-3.1-8B-shaped GQA decode, Quest key-box selection",
         "llama_cobs": "Llama-3.1-8B-shaped GQA decode, COBS second-order selection (rank-4 factors)",
+        "llama_cobs_fp4": "Llama-3.1-8B-shaped GQA decode, COBS stored descriptor (bf16 means, rank-4 E2M1 "
+                          "factors in the 90%-energy query subspace)",
         "llama_coreset": "Llama-3.1-8B-shaped GQA decode, weighted coreset m=2048",
     }
     return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, "
@@ -453,6 +508,8 @@ def run_ours(args, dist):
     score_override = "summary_mean16" if args.scorer == "mean16" else None
     L2_BYTES = 126 << 20
 
+    shared_basis = {}
+
     def make_set(j):
         seed = (None if dist.rank == 0 else base_seed) if j == 0 else base_seed + 50000 * j
         w_ = W.make(name, dev, budget=args.budget, B=args.batch, seed=seed)
@@ -466,6 +523,16 @@ def run_ours(args, dist):
             su_["k_bounds"] = kv.kv_build_block_bounds(w_.K, sl_, w_.block_size)
         if w_.score_mode == "cobs":
             su_["k_xi"] = kv.kv_build_block_cov_factors(w_.K, sl_, w_.block_size, 4)
+        if w_.score_mode == "cobs_fp4":
+            if "U" not in shared_basis:  # one basis for the model: every batch draws queries from it
+                Qc = W.calibration_queries(w_, CALIB_POSITIONS)
+                evecs, evals = kv.kv_build_query_basis(Qc, w_.Hkv)
+                s_q = kv.kv_query_subspace_rank(evals, 0.9)
+                shared_basis.update(U=evecs[:, :s_q, :].contiguous(), s=s_q, Qc=Qc)
+            su_["k_mean"] = kv.kv_build_block_key_means(w_.K, sl_, w_.block_size, su_["k_sum"], su_["counts"])
+            xi_ss = kv.kv_build_block_cov_factors_ss(w_.K, sl_, w_.block_size, shared_basis["U"], 4)
+            su_["codes"], su_["code_scales"] = kv.kv_quantize_fp4(xi_ss)
+            del xi_ss
         return dict(wl=w_, sl=sl_, summ=su_,
                     idx=torch.zeros(w_.B, w_.Hkv, w_.kmax, dtype=torch.int32, device=dev),
                     nk=torch.zeros(w_.B, w_.Hkv, dtype=torch.int32, device=dev),
@@ -511,6 +578,11 @@ def run_ours(args, dist):
             kv.kv_select_blocks_mean16(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_mean"], su_["counts"], w_.k_top,
                                        w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
                                        n_kept=st_["nk"])
+        elif wl.score_mode == "cobs_fp4":
+            kv.kv_select_blocks_cobs_fp4(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_mean"], su_["counts"],
+                                         shared_basis["U"], su_["codes"], su_["code_scales"], 4, w_.k_top,
+                                         w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
+                                         n_kept=st_["nk"])
         elif wl.score_mode == "cobs":
             kv.kv_select_blocks_cobs(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_sum"], su_["counts"], su_["k_xi"],
                                      w_.k_top, w_.force_first, w_.force_last, kmax=kmax, block_idx=st_["idx"],
@@ -567,6 +639,17 @@ def run_ours(args, dist):
     if wl.score_mode == "cobs":
         builds["kv_build_block_cov_factors_ms"] = time_build(
             lambda: kv.kv_build_block_cov_factors(wl.K, sl, wl.block_size, 4, out=summ["k_xi"]), reps=1)
+    if wl.score_mode == "cobs_fp4":
+        builds["kv_build_query_basis_ms"] = time_build(
+            lambda: kv.kv_build_query_basis(shared_basis["Qc"], wl.Hkv), reps=1)
+        xi_t = {}
+
+        def ss_build():
+            xi_t["x"] = kv.kv_build_block_cov_factors_ss(wl.K, sl, wl.block_size, shared_basis["U"], 4)
+        builds["kv_build_block_cov_factors_ss_ms"] = time_build(ss_build, reps=1)
+        builds["kv_quantize_fp4_ms"] = time_build(lambda: kv.kv_quantize_fp4(xi_t["x"]), reps=1)
+        builds["subspace_s"] = shared_basis["s"]
+        del xi_t
 
     if args.wildcat_m > 0:
         # the WildCat coreset producer on the same cache (randomly pivoted Cholesky
@@ -875,6 +958,7 @@ def run_ours(args, dist):
         a_bytes = attention_bytes(wl, nk, wl.seq_lens)
         s_bytes = (quest_select_bytes(wl, wl.seq_lens) if quest else
                    cobs_select_bytes(wl, wl.seq_lens) if wl.score_mode == "cobs" else
+                   cobs_fp4_select_bytes(wl, wl.seq_lens, shared_basis["s"]) if wl.score_mode == "cobs_fp4" else
                    select_bytes(wl, wl.seq_lens) if mode == kv.KV_SCORE_SUMMARY else osa_select_bytes(wl, wl.seq_lens))
     peak, peak_kind = measured_peak_hbm()
     # the roofline line is the attention kernel's (the kernel the target names);

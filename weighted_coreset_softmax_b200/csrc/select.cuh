@@ -584,82 +584,116 @@ __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, i
 // Attention", the subspace and quantisation paragraphs): adds
 // (sigma^2 / 2) sum_i (q~ . xi_i)^2 to lg, q~ = U q the projected query (qt: the
 // log2-domain q~ of the G heads, [G][SP] in shared memory, zero past s) and
-// xi_i = scale_i * e2m1(codes_i). Each half-warp takes one block: lane c of the half
-// holds nibble columns 8c .. 8c+7 of every factor (one 32-bit word a factor),
-// decodes them with the E2M1 -> f16x2 conversion, forms its partial dots for every
-// (head, factor) pair, and a transpose reduction over the half's 16 lanes sums them
-// (NV - 1 shuffles for NV pairs). The squared dots, times scale_i^2, are summed
-// over the factors through a per-warp scratch.
-template <int G, int RMAX>
+// xi_i = scale_i * e2m1(codes_i). Each half-warp takes one block at a time: lane c
+// of the half holds nibble columns 8c .. 8c+7 of every factor (one 32-bit word a
+// factor), decodes them with the E2M1 -> f16x2 conversion, forms its partial dots
+// for every (head, factor) pair of a group of FG = 4 factors, and a transpose
+// reduction over the half's 16 lanes sums them (NV - 1 shuffles for NV pairs); the
+// squared dots, times scale_i^2, are summed over the factors through a per-warp
+// scratch (ranks above 4 take a second group). A warp issues the words and scales of
+// NBW block pairs before decoding any of them, so NBW * FG loads a lane are in
+// flight.
+template <int G>
 __device__ void cobs_fp4_second_order(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float* qt,
                                       float* scratch) {
+  constexpr int FG = 4;
   constexpr int GP = pow2ceil(G);
-  constexpr int NV = GP * RMAX;
-  constexpr int NH = NV >= 16 ? NV / 16 : 1;    // values a lane holds after the reduction
+  constexpr int NV = GP * FG;                  // 4 .. 32
+  constexpr int NH = NV >= 16 ? NV / 16 : 1;   // values a lane holds after the reduction
   constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes holding each value (NV < 16)
+  constexpr int NBW = NV <= 16 ? 8 : 4;        // block pairs a warp loads ahead
+  constexpr bool QREG = G <= 4;                // the projected queries in registers (else shared memory)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int hw = lane >> 4, c = lane & 15;
   const int r = p.cobs_r, SP = p.SP;
   const bool active = c < SP / 8;
-  float qv[G][8];
+  float qv[QREG ? G : 1][8];
+  if constexpr (QREG) {
 #pragma unroll
-  for (int g = 0; g < G; ++g)
+    for (int g = 0; g < G; ++g)
 #pragma unroll
-    for (int k = 0; k < 8; ++k) qv[g][k] = active ? qt[g * SP + 8 * c + k] : 0.f;
+      for (int k = 0; k < 8; ++k) qv[g][k] = active ? qt[g * SP + 8 * c + k] : 0.f;
+  }
+  const float* qs = qt + 8 * (active ? c : 0);  // this lane's columns (inactive lanes decode zeros)
   float* scr = scratch + (warp * 2 + hw) * NV;
   const size_t fbytes = static_cast<size_t>(SP) / 2;  // bytes a factor
-  for (int b2 = warp * 2; b2 < nbv; b2 += SEL_NW * 2) {  // warp-uniform
-    const int b = b2 + hw;
-    const bool live = b < nbv;
-    const size_t fb = (static_cast<size_t>(bh) * p.NBcap + b) * r;  // first factor of block b
-    uint32_t w[RMAX];
+  const size_t base = static_cast<size_t>(bh) * p.NBcap * r;
+  for (int f0 = 0; f0 < r; f0 += FG) {
+    for (int b0 = warp * 2 * NBW; b0 < nbv; b0 += SEL_NW * 2 * NBW) {  // warp-uniform
+      uint32_t w[NBW][FG];
+      float sc[NBW][NH];
 #pragma unroll
-    for (int i = 0; i < RMAX; ++i)
-      w[i] = (active && live && i < r) ? __ldg(reinterpret_cast<const uint32_t*>(p.xi4 + (fb + i) * fbytes) + c) : 0u;
-    float part[NV];
+      for (int j = 0; j < NBW; ++j) {
+        const int b = b0 + 2 * j + hw;
+        const bool live = b < nbv;
+        const size_t fb = base + static_cast<size_t>(b) * r + f0;
 #pragma unroll
-    for (int i = 0; i < RMAX; ++i) {
-      float x[8];
+        for (int i = 0; i < FG; ++i)
+          w[j][i] = (active && live && f0 + i < r)
+                        ? __ldg(reinterpret_cast<const uint32_t*>(p.xi4 + (fb + i) * fbytes) + c)
+                        : 0u;
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const __half2 h2 = __half2(__nv_cvt_fp4x2_to_halfraw2(
-            static_cast<__nv_fp4x2_storage_t>((w[i] >> (8 * k)) & 0xffu), __NV_E2M1));
-        const float2 f2 = __half22float2(h2);
-        x[2 * k] = f2.x;
-        x[2 * k + 1] = f2.y;
-      }
-#pragma unroll
-      for (int g = 0; g < GP; ++g) {
-        float d = 0.f;
-        if (g < G) {
-#pragma unroll
-          for (int k = 0; k < 8; ++k) d = fmaf(qv[g][k], x[k], d);
+        for (int t = 0; t < NH; ++t) {
+          const int idx = NV >= 16 ? c * NH + t : c / REP;
+          const int i = idx - (idx / FG) * FG;
+          sc[j][t] = (live && f0 + i < r) ? __ldg(p.xi4_scale + fb + i) : 0.f;
         }
-        part[g * RMAX + i] = d;
       }
-    }
-    transpose_reduce<NV, 8>(part, lane);
-    __syncwarp();
 #pragma unroll
-    for (int j = 0; j < NH; ++j) {
-      const int idx = NV >= 16 ? c * NH + j : c / REP;
-      const int g = idx / RMAX, i = idx - (idx / RMAX) * RMAX;
-      if (c % REP == 0) {
-        float v = 0.f;
-        if (live && g < G && i < r) {
-          const float sc = __ldg(p.xi4_scale + fb + i);
-          v = part[j] * part[j] * sc * sc;
+      for (int j = 0; j < NBW; ++j) {
+        const int b = b0 + 2 * j + hw;
+        float part[NV];
+#pragma unroll
+        for (int i = 0; i < FG; ++i) {
+          float x[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const __half2 h2 = __half2(__nv_cvt_fp4x2_to_halfraw2(
+                static_cast<__nv_fp4x2_storage_t>((w[j][i] >> (8 * k)) & 0xffu), __NV_E2M1));
+            const float2 f2 = __half22float2(h2);
+            x[2 * k] = f2.x;
+            x[2 * k + 1] = f2.y;
+          }
+#pragma unroll
+          for (int g = 0; g < GP; ++g) {
+            float d = 0.f;
+            if (g < G) {
+              if constexpr (QREG) {
+#pragma unroll
+                for (int k = 0; k < 8; ++k) d = fmaf(qv[g][k], x[k], d);
+              } else {
+                const float4 a = *reinterpret_cast<const float4*>(qs + g * SP);
+                const float4 e = *reinterpret_cast<const float4*>(qs + g * SP + 4);
+                d = fmaf(a.x, x[0], d);
+                d = fmaf(a.y, x[1], d);
+                d = fmaf(a.z, x[2], d);
+                d = fmaf(a.w, x[3], d);
+                d = fmaf(e.x, x[4], d);
+                d = fmaf(e.y, x[5], d);
+                d = fmaf(e.z, x[6], d);
+                d = fmaf(e.w, x[7], d);
+              }
+            }
+            part[g * FG + i] = d;
+          }
         }
-        scr[idx] = v;
+        transpose_reduce<NV, 8>(part, lane);
+        if (c % REP == 0) {
+#pragma unroll
+          for (int t = 0; t < NH; ++t) {
+            const int idx = NV >= 16 ? c * NH + t : c / REP;
+            const float sct = sc[j][t];
+            scr[idx] = part[t] * part[t] * sct * sct;  // zero past r, G and the blocks (sc = 0 or part = 0)
+          }
+        }
+        __syncwarp();
+        if (b < nbv && c < G) {
+          const float sum = scr[c * FG] + scr[c * FG + 1] + scr[c * FG + 2] + scr[c * FG + 3];
+          lg[c * nbp + b] += 0.34657359027997264f * sum;  // ln 2 / 2
+        }
+        __syncwarp();
       }
     }
-    __syncwarp();
-    if (live && c < G) {
-      float sum = 0.f;
-      for (int i = 0; i < r; ++i) sum += scr[c * RMAX + i];
-      lg[c * nbp + b] += 0.34657359027997264f * sum;  // ln 2 / 2
-    }
-    __syncwarp();
   }
 }
 
@@ -743,24 +777,37 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
     float* scratch = qt + G * p.SP;
     const int h = bh - b * p.Hkv;
     const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D;
-    for (int e = tid; e < G * p.SP; e += SEL_THREADS) {
-      const int g = e / p.SP, j = e - (e / p.SP) * p.SP;
-      float v = 0.f;
-      if (j < p.s_dim) {
-        if (p.Uq) {
-          const float* u = p.Uq + (static_cast<size_t>(h) * p.s_dim + j) * D;
-          for (int d = 0; d < D; ++d) v = fmaf(__ldg(u + d), load_as_float(qrow + g * D + d), v);
-        } else {
-          v = load_as_float(qrow + g * D + j);
+    if (p.Uq) {
+      // q~[g][j] = U_j . q_g: a warp per basis row j (coalesced), the group's queries
+      // in registers (D / 32 channels a lane)
+      constexpr int CPL = D / 32;
+      float qreg[G][CPL];
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) qreg[g][k] = load_as_float(qrow + g * D + lane * CPL + k);
+      for (int j = warp; j < p.SP; j += SEL_NW) {
+        float u[CPL];
+#pragma unroll
+        for (int k = 0; k < CPL; ++k)
+          u[k] = j < p.s_dim ? __ldg(p.Uq + (static_cast<size_t>(h) * p.s_dim + j) * D + lane * CPL + k) : 0.f;
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+          float v = 0.f;
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) v = fmaf(u[k], qreg[g][k], v);
+          v = warp_sum(v);
+          if (lane == 0) qt[g * p.SP + j] = v * p.qscale;
         }
       }
-      qt[e] = v * p.qscale;
+    } else {
+      for (int e = tid; e < G * p.SP; e += SEL_THREADS) {
+        const int g = e / p.SP, j = e - (e / p.SP) * p.SP;
+        qt[e] = (j < p.s_dim ? load_as_float(qrow + g * D + j) : 0.f) * p.qscale;
+      }
     }
     __syncthreads();
-    if (p.cobs_r <= 4)
-      cobs_fp4_second_order<G, 4>(p, lg, nbp, bh, nbv, qt, scratch);
-    else
-      cobs_fp4_second_order<G, COV_MAX_RANK_SEL>(p, lg, nbp, bh, nbv, qt, scratch);
+    cobs_fp4_second_order<G>(p, lg, nbp, bh, nbv, qt, scratch);
     __syncthreads();
   }
 
