@@ -295,6 +295,203 @@ def cobs_subspace_logits(qg: np.ndarray, mean: np.ndarray, counts: np.ndarray, x
     return out
 
 
+# --------------------------------------------------------------------------- QGC + ErrorGate
+def qgc_project(K: np.ndarray, n: int, P: np.ndarray) -> np.ndarray:
+    """z_i = P k_i, the keys' coordinates on the top eigenvectors of the queries,
+    stored at fp32 [OA, "Three helpers that make the proxy accurate": keys are
+    projected onto the top eigenvectors of the queries; reading R23]. P: [16][D]."""
+    return (np.asarray(K[:n], dtype=np.float64) @ np.asarray(P, dtype=np.float64).T).astype(np.float32)
+
+
+def qgc_kmeans(Z32: np.ndarray, C: int, iters: int):
+    """k-means in the projection [OA, "Three helpers": k-means in 16 dimensions, once
+    after prefill; reading R23], Lloyd's iteration in float64 on the fp32 coordinates:
+    C' = min(C, n) centroids start at the tokens ((2c + 1) n) // (2 C'); each iteration
+    assigns every token to the nearest centroid (squared distance summed over the
+    coordinates in order; ties to the lower cluster) and moves every non-empty
+    cluster's centroid to its members' mean. Returns (labels [n] of the last
+    assignment, centroids [C'][16])."""
+    Z = np.asarray(Z32, dtype=np.float64)
+    n = Z.shape[0]
+    Ce = min(C, n)
+    if Ce == 0:
+        return np.zeros(0, dtype=np.int64), np.zeros((0, Z.shape[1] if Z.ndim == 2 else 16))
+    cent = np.stack([Z[((2 * c + 1) * n) // (2 * Ce)] for c in range(Ce)])
+    labels = np.zeros(n, dtype=np.int64)
+    for _ in range(iters):
+        d = np.zeros((n, Ce))
+        for c in range(Ce):
+            diff = Z - cent[c]
+            acc = np.zeros(n)
+            for j in range(Z.shape[1]):
+                acc = acc + diff[:, j] * diff[:, j]
+            d[:, c] = acc
+        labels = np.argmin(d, axis=1)
+        for c in range(Ce):
+            m = labels == c
+            if m.any():
+                cent[c] = Z[m].mean(axis=0)
+    return labels, cent
+
+
+def qgc_cluster_stats(K: np.ndarray, V: np.ndarray, n: int, labels: np.ndarray, C: int):
+    """The cached tokens of every cluster [OA, "Three helpers": the mean and variance
+    tokens; reading R23]: count [C], key sum [C][D], value sum [C][D] and per-channel
+    key sum of squares [C][D] (mean = sum / count, variance = squares / count - mean^2)."""
+    D = K.shape[1]
+    cnt = np.zeros(C, dtype=np.int64)
+    ks, vs, kq = np.zeros((C, D)), np.zeros((C, D)), np.zeros((C, D))
+    for i in range(n):
+        c = int(labels[i])
+        cnt[c] += 1
+        ks[c] += K[i]
+        vs[c] += V[i]
+        kq[c] += K[i] * K[i]
+    return cnt, ks, vs, kq
+
+
+def errorgate_errors(qg: np.ndarray, cnt, ks, kq, sigma: float) -> np.ndarray:
+    """The estimated weight error each cluster's proxy would leave [OA, "Skipping
+    reviews without losing the verdict": a proxy's unnormalised weight error is its
+    mass times the spread of the weights it hides; "Three helpers": ErrorGate
+    estimates it from the cached mean and variance tokens; reading R23]. With the
+    cluster's logits read as normal with mean mu_gc = sigma q_g . mean_c and variance
+    s2_gc = sigma^2 sum_d q_gd^2 var_cd, the mean-logit proxy's mass n_c e^mu falls
+    short of the cluster's expected mass n_c e^(mu + s2/2) by
+    E_gc = n_c e^mu_gc (e^(s2_gc / 2) - 1); per head it is divided by the estimated
+    total Zhat_g = sum_c n_c e^(mu_gc + s2_gc / 2) and summed over the group's heads.
+    Empty clusters get 0. Returns E [C]."""
+    C = len(cnt)
+    G = qg.shape[0]
+    mu = np.full((G, C), -math.inf)
+    s2 = np.zeros((G, C))
+    for c in range(C):
+        if cnt[c] <= 0:
+            continue
+        mean = ks[c] / cnt[c]
+        var = np.maximum(kq[c] / cnt[c] - mean * mean, 0.0)
+        for g in range(G):
+            mu[g, c] = sigma * float(qg[g] @ mean)
+            s2[g, c] = sigma * sigma * float(np.sum(qg[g] * qg[g] * var))
+    E = np.zeros(C)
+    for g in range(G):
+        live = cnt > 0
+        if not live.any():
+            continue
+        M = float(np.max(mu[g, live] + 0.5 * s2[g, live]))
+        zhat = float(np.sum(cnt[live] * np.exp(mu[g, live] + 0.5 * s2[g, live] - M)))
+        for c in range(C):
+            if cnt[c] > 0:
+                E[c] += cnt[c] * math.exp(mu[g, c] - M) * math.expm1(0.5 * s2[g, c]) / zhat
+    return E
+
+
+def errorgate_split(E: np.ndarray, cnt, R: int):
+    """Exact reads per cluster [OA, "Three helpers": ErrorGate splits the exact-read
+    budget across clusters in proportion to the error each proxy would leave; reading
+    R23]: r_c = min(n_c, floor(R E_c / sum E)); all 0 when sum E = 0. Also returns the
+    near-integer flag: some R E_c / sum E within 1e-4 (relative) of an integer below
+    n_c, where float rounding may decide the floor."""
+    tot = float(np.sum(E))
+    r = np.zeros(len(E), dtype=np.int64)
+    near = False
+    if tot <= 0.0 or R <= 0:
+        return r, near
+    for c in range(len(E)):
+        x = R * float(E[c]) / tot
+        fl = math.floor(x)
+        r[c] = min(int(cnt[c]), fl)
+        if fl < cnt[c] and (x - fl < 1e-4 * max(1.0, x) or fl + 1 - x < 1e-4 * max(1.0, x)):
+            near = True
+    return r, near
+
+
+def qgs_token_scores(qg: np.ndarray, Z16: np.ndarray, P: np.ndarray, sigma: float) -> np.ndarray:
+    """Token scores inside the clusters [OA, "Three helpers": QGS picks the top tokens
+    inside each cluster from low-bit projections; reading R23]: with the projections
+    stored at bf16 (Z16) and the query projected the same way (P q_g),
+    t_i = sum_g exp(sigma (P q_g) . z_i - LSE_g), LSE_g over all tokens (the group
+    combination of Equation 5, per token)."""
+    qt = np.asarray(qg, dtype=np.float64) @ np.asarray(P, dtype=np.float64).T
+    lg = sigma * (np.asarray(Z16, dtype=np.float64) @ qt.T)  # [n][G]
+    t = np.zeros(lg.shape[0])
+    for g in range(lg.shape[1]):
+        t += np.exp(lg[:, g] - logsumexp(lg[:, g]))
+    return t
+
+
+def qgc_select(t: np.ndarray, labels: np.ndarray, r) -> Tuple[List[int], bool]:
+    """The read tokens: in every cluster c the r_c largest scores (ties to the lower
+    index); ascending. Also a near-tie flag: inside some cluster the r_c-th and the
+    next score within 1e-3 (relative)."""
+    out: List[int] = []
+    near = False
+    for c in range(len(r)):
+        mem = [int(i) for i in np.nonzero(labels == c)[0]]
+        if r[c] <= 0 or not mem:
+            continue
+        mem.sort(key=lambda i: (-t[i], i))
+        out += mem[:r[c]]
+        if r[c] < len(mem):
+            a, b = t[mem[r[c] - 1]], t[mem[r[c]]]
+            if a - b <= 1e-3 * abs(a):
+                near = True
+    return sorted(out), near
+
+
+def qgc_attend_one(qg, K, V, n, labels, read, C, sigma):
+    """Softmax over the read tokens and one count-aware proxy per cluster with unread
+    tokens: their mean key and value, logit sigma q . mean + ln count [OA, "Skipping
+    reviews": the proxy is one virtual token with the tail's mean value and mean
+    logit plus the log of its count; "Three helpers": one proxy per cluster]. Built
+    directly from the unread tokens."""
+    G, D = qg.shape[0], V.shape[1]
+    rs = set(int(i) for i in read)
+    out = np.zeros((G, D))
+    lse = np.full(G, -math.inf)
+    for g in range(G):
+        logits, vals = [], []
+        for i in sorted(rs):
+            logits.append(sigma * float(qg[g] @ K[i]))
+            vals.append(V[i])
+        for c in range(C):
+            un = [i for i in range(n) if int(labels[i]) == c and i not in rs]
+            if not un:
+                continue
+            km = K[un].mean(axis=0)
+            vm = V[un].mean(axis=0)
+            logits.append(sigma * float(qg[g] @ km) + math.log(len(un)))
+            vals.append(vm)
+        if logits:
+            out[g], lse[g] = softmax_attend(np.array(logits), np.array(vals))
+    return out, lse
+
+
+def qgc_read_budget(n: int, budget: float, C_live: int) -> int:
+    """Exact rows a query may read: floor(budget n) less the cached mean and variance
+    tokens, 1.5 KV rows a cluster, charged to the read [OA, "Three helpers"]; at least 0."""
+    return max(0, int(math.floor(budget * n)) - int(math.ceil(1.5 * C_live)))
+
+
+def qgc_decode_one(qg, K, V, n, P, C, iters, budget, sigma):
+    """One (sequence, KV head) decode step of QGC + ErrorGate from scratch: the
+    build (projection, k-means, cluster statistics) and the query (errors, split,
+    in-cluster selection, attention with the proxies). Returns a dict with labels,
+    counts, E, r, read, near_tie, out, lse."""
+    Z32 = qgc_project(K, n, P)
+    labels, _ = qgc_kmeans(Z32, C, iters)
+    Ce = min(C, n)
+    cnt, ks, vs, kq = qgc_cluster_stats(K, V, n, labels, Ce)
+    E = errorgate_errors(qg, cnt, ks, kq, sigma)
+    R = qgc_read_budget(n, budget, int(np.sum(cnt > 0)))
+    r, near_split = errorgate_split(E, cnt, R)
+    t = qgs_token_scores(qg, round_bf16(Z32.astype(np.float64)), P, sigma)
+    read, near_sel = qgc_select(t, labels, r)
+    out, lse = qgc_attend_one(qg, K, V, n, labels, read, Ce, sigma)
+    return dict(labels=labels, counts=cnt, E=E, R=R, r=r, read=read, near_tie=near_split or near_sel,
+                out=out, lse=lse, Z32=Z32, t=t)
+
+
 # --------------------------------------------------------------------------- scores
 def logsumexp(x: np.ndarray) -> float:
     """ln sum exp(x) with a max shift; -inf for an empty or all -inf input."""

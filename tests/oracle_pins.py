@@ -862,6 +862,146 @@ def pin_cobs_subspace_logits(seed=32):
                     + math.log(e - st))
             _close(got[g, b], want, 1e-10, what="subspace score")
 
+
+def pin_qgc_kmeans_lloyd_steps(seed=35):
+    """k-means: the start is the tokens ((2c + 1) n) // (2C); one iteration assigns
+    every token to its nearest start centroid (distances and argmin written as
+    Python loops, ties to the lower cluster) and moves each centroid to its members'
+    mean; two iterations assign against those means. Well separated blobs come back
+    as the clusters."""
+    r = _rng(seed)
+    n, C = 23, 4
+    Z = r.normal(size=(n, 16)).astype(np.float32)
+    Zl = Z.astype(np.float64).tolist()
+
+    def assign(cent):
+        lab = []
+        for i in range(n):
+            best, bd = 0, None
+            for c in range(len(cent)):
+                dd = sum((Zl[i][j] - cent[c][j]) ** 2 for j in range(16))
+                if bd is None or dd < bd:
+                    best, bd = c, dd
+            lab.append(best)
+        return lab
+
+    def update(lab, cent):
+        out = []
+        for c in range(len(cent)):
+            mem = [i for i in range(n) if lab[i] == c]
+            out.append([sum(Zl[i][j] for i in mem) / len(mem) for j in range(16)] if mem else cent[c])
+        return out
+
+    start = [Zl[((2 * c + 1) * n) // (2 * C)] for c in range(C)]
+    lab1 = assign(start)
+    cent1 = update(lab1, start)
+    l1, c1 = O.qgc_kmeans(Z, C, 1)
+    assert list(l1) == lab1
+    _close(c1, cent1, 1e-12, what="centroids after one step")
+    lab2 = assign(cent1)
+    assert lab2 != lab1  # (this case still moves at the second step)
+    l2, c2 = O.qgc_kmeans(Z, C, 2)
+    assert list(l2) == lab2
+    _close(c2, update(lab2, cent1), 1e-12, what="centroids after two steps")
+    # blobs 40 apart with unit spread: recovered as the clusters
+    centers = r.normal(size=(3, 16)) * 40.0
+    B = np.concatenate([centers[k] + r.normal(size=(20, 16)) for k in range(3)]).astype(np.float32)
+    lab, _ = O.qgc_kmeans(B, 3, 6)
+    for k in range(3):
+        assert len(set(int(x) for x in lab[20 * k:20 * (k + 1)])) == 1
+    assert len(set(int(x) for x in lab)) == 3
+
+
+def pin_qgc_project_identity(seed=34):
+    """With the identity as the basis (16-dim keys) the coordinates are the keys in fp32."""
+    r = _rng(seed)
+    K = r.normal(size=(9, 16))
+    _close(O.qgc_project(K, 7, np.eye(16)), K[:7].astype(np.float32), 0.0, what="identity projection")
+
+
+def pin_errorgate_closed_form(seed=35):
+    """A cluster of two keys m +- delta e_0: var_0 = delta^2, so for one head
+    s2 = sigma^2 q_0^2 delta^2 and E = 2 e^mu (e^(s2/2) - 1) / (2 e^(mu + s2/2))
+    = 1 - e^(-s2/2); a cluster of identical keys leaves no error; two heads add their
+    normalised errors."""
+    r = _rng(seed)
+    D, sig, dl = 5, 0.7, 0.9
+    m = r.normal(size=D)
+    K = np.stack([m + dl * np.eye(D)[0], m - dl * np.eye(D)[0]])
+    qg = r.normal(size=(2, D))
+    cnt, ks, vs, kq = O.qgc_cluster_stats(K, K, 2, np.array([0, 0]), 1)
+    E = O.errorgate_errors(qg, cnt, ks, kq, sig)
+    want = sum(1.0 - math.exp(-0.5 * (sig * qg[g][0] * dl) ** 2) for g in range(2))
+    _close(E[0], want, 1e-12, what="two-point cluster")
+    K2 = np.concatenate([K, np.tile(m + 3.0, (3, 1))])
+    cnt, ks, vs, kq = O.qgc_cluster_stats(K2, K2, 5, np.array([0, 0, 1, 1, 1]), 2)
+    E2 = O.errorgate_errors(qg[:1], cnt, ks, kq, sig)
+    assert abs(E2[1]) <= 1e-15 and E2[0] > 0
+
+
+def pin_errorgate_split_by_hand():
+    """r_c = min(n_c, floor(R E_c / sum E))."""
+    r, _ = O.errorgate_split(np.array([1.0, 2.0, 3.5]), [50, 50, 50], 10)  # 1.54, 3.08, 5.38
+    assert list(r) == [1, 3, 5]
+    r, _ = O.errorgate_split(np.array([1.0, 2.0, 3.5]), [50, 2, 50], 10)   # the second is capped
+    assert list(r) == [1, 2, 5]
+    r, _ = O.errorgate_split(np.zeros(3), [5, 5, 5], 10)
+    assert list(r) == [0, 0, 0]
+
+
+def pin_qgs_scores(seed=36):
+    """Token scores: each head contributes a softmax over the tokens (so the scores
+    add up to G), written here with Python loops."""
+    r = _rng(seed)
+    n, D, G, sig = 11, 20, 3, 0.3
+    P = _rotation(r, D)[:16]
+    qg = r.normal(size=(G, D))
+    Z = r.normal(size=(n, 16))
+    t = O.qgs_token_scores(qg, Z, P, sig)
+    _close(np.sum(t), float(G), 1e-12, what="scores add up to G")
+    qt = [[sum(P[j][d] * qg[g][d] for d in range(D)) for j in range(16)] for g in range(G)]
+    for i in range(n):
+        want = 0.0
+        for g in range(G):
+            lg = [sig * sum(qt[g][j] * Z[k][j] for j in range(16)) for k in range(n)]
+            mx = max(lg)
+            want += math.exp(lg[i] - mx) / sum(math.exp(x - mx) for x in lg)
+        _close(t[i], want, 1e-12, what="token score")
+
+
+def pin_qgc_single_cluster_no_reads(seed=37):
+    """One cluster and nothing read: the output is the count-aware proxy of all tokens
+    (the value mean, lse = sigma q . mean key + ln n), as the tail proxy of A4."""
+    r = _rng(seed)
+    n, D = 30, 6
+    K, V = r.normal(size=(n, D)), r.normal(size=(n, D))
+    qg = r.normal(size=(2, D))
+    o, l = O.qgc_attend_one(qg, K, V, n, np.zeros(n, dtype=np.int64), [], 1, 0.4)
+    for g in range(2):
+        _close(o[g], V.mean(axis=0), 1e-12, what="proxy value")
+        _close(l[g], 0.4 * float(qg[g] @ K.mean(axis=0)) + math.log(n), 1e-12, what="proxy lse")
+    ot, lt, _ = O.sparse_attend_one(qg, K, V, n, 10, [], 0.4, True)
+    _close(o, ot, 1e-12, what="same as the tail proxy")
+
+
+def pin_qgc_equal_logits_exact(seed=38):
+    """Clusters of identical keys: every proxy hides equal logits, ErrorGate's errors
+    vanish (up to the rounding of sum-of-squares minus squared mean), and whatever
+    it reads, the output is exact dense attention (the proxy is exact when all the
+    weights it hides are equal)."""
+    r = _rng(seed)
+    D, per, C = 16, 12, 3
+    keys = r.normal(size=(C, D)) * 8.0
+    K = np.concatenate([np.tile(keys[c], (per, 1)) for c in range(C)])
+    V = r.normal(size=(C * per, D))
+    n = C * per
+    qg = r.normal(size=(2, D))
+    res = O.qgc_decode_one(qg, K, V, n, np.eye(D), C, 5, 0.25, 0.3)
+    assert np.max(np.abs(res["E"])) <= 1e-12
+    od, ld = O.dense_attend_one(qg, K, V, n, 0.3)
+    _close(res["out"], od, 1e-12, what="equal logits: dense")
+    _close(res["lse"], ld, 1e-12, what="equal logits: lse")
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -875,4 +1015,6 @@ ALL_PINS = [
     pin_wildcat_all_points_is_exact, pin_wildcat_identical_tokens, pin_wildcat_weights_optimal,
     pin_query_basis_closed_form, pin_subspace_rank_by_hand, pin_subspace_factors_exact_in_subspace,
     pin_fp4_e2m1_grid_and_ties, pin_cobs_subspace_logits,
+    pin_qgc_kmeans_lloyd_steps, pin_qgc_project_identity, pin_errorgate_closed_form, pin_errorgate_split_by_hand,
+    pin_qgs_scores, pin_qgc_single_cluster_no_reads, pin_qgc_equal_logits_exact,
 ]

@@ -297,6 +297,72 @@ def _mut_ss_factors_full_space_projected(orig):
         return xs, np.sum(xs * xs, axis=2)
     return f
 
+
+def _mut_kmeans_no_update(orig):
+    def f(Z32, C, iters):
+        return orig(Z32, C, min(iters, 1))  # the centroids stop after one move
+    return f
+
+
+def _mut_kmeans_first_tokens(orig):
+    def f(Z32, C, iters):
+        Z = np.asarray(Z32, dtype=np.float64)
+        n = Z.shape[0]
+        Ce = min(C, n)
+        cent = Z[:Ce].copy()  # starts at the first tokens
+        labels = np.zeros(n, dtype=np.int64)
+        for _ in range(iters):
+            d = ((Z[:, None, :] - cent[None]) ** 2).sum(axis=2)
+            labels = np.argmin(d, axis=1)
+            for c in range(Ce):
+                if (labels == c).any():
+                    cent[c] = Z[labels == c].mean(axis=0)
+        return labels, cent
+    return f
+
+
+def _mut_errorgate_no_minus_one(orig):
+    def f(qg, cnt, ks, kq, sigma):
+        E = orig(qg, cnt, ks, kq, sigma)
+        return E + np.where(np.asarray(cnt) > 0, 1.0, 0.0) * qg.shape[0] / max(1, int(np.sum(np.asarray(cnt) > 0)))
+    return f
+
+
+def _mut_split_uncapped(orig):
+    def f(E, cnt, R):
+        return orig(E, [10 ** 9] * len(cnt), R)
+    return f
+
+
+def _mut_qgs_no_normaliser(orig):
+    def f(qg, Z16, P, sigma):
+        qt = np.asarray(qg, dtype=np.float64) @ np.asarray(P, dtype=np.float64).T
+        lg = sigma * (np.asarray(Z16, dtype=np.float64) @ qt.T)
+        return np.exp(lg).sum(axis=1)
+    return f
+
+
+def _mut_qgc_proxy_no_count(orig):
+    def f(qg, K, V, n, labels, read, C, sigma):
+        G, D = qg.shape[0], V.shape[1]
+        rs = set(int(i) for i in read)
+        out = np.zeros((G, D))
+        lse = np.full(G, -math.inf)
+        for g in range(G):
+            logits, vals = [], []
+            for i in sorted(rs):
+                logits.append(sigma * float(qg[g] @ K[i]))
+                vals.append(V[i])
+            for c in range(C):
+                un = [i for i in range(n) if int(labels[i]) == c and i not in rs]
+                if un:
+                    logits.append(sigma * float(qg[g] @ K[un].mean(axis=0)))  # no ln count
+                    vals.append(V[un].mean(axis=0))
+            if logits:
+                out[g], lse[g] = O.softmax_attend(np.array(logits), np.array(vals))
+        return out, lse
+    return f
+
 MUTANTS = {
     "tail_proxy/no ln count": ("tail_proxy", _mut_proxy_no_log_count),
     "tail_proxy/sum not mean": ("tail_proxy", _mut_proxy_sum_value),
@@ -329,6 +395,12 @@ MUTANTS = {
     "subspace_rank/mean rounded down": ("subspace_rank", _mut_subspace_rank_floor),
     "subspace_logits/query not projected": ("cobs_subspace_logits", _mut_subspace_logits_unprojected),
     "ss_factors/projected full-space directions": ("block_cov_factors_ss_one", _mut_ss_factors_full_space_projected),
+    "kmeans/centroids stop moving": ("qgc_kmeans", _mut_kmeans_no_update),
+    "kmeans/starts at the first tokens": ("qgc_kmeans", _mut_kmeans_first_tokens),
+    "errorgate/mass not the gap": ("errorgate_errors", _mut_errorgate_no_minus_one),
+    "errorgate/split not capped": ("errorgate_split", _mut_split_uncapped),
+    "qgs/no per-head normaliser": ("qgs_token_scores", _mut_qgs_no_normaliser),
+    "qgc/proxy without ln count": ("qgc_attend_one", _mut_qgc_proxy_no_count),
 }
 
 
