@@ -371,6 +371,76 @@ kv_status kv_select_blocks_cobs_fp4(const kv_shape* shape, const void* q, float 
                                     int kmax, int32_t* block_idx, int32_t* n_kept, float* scores, kv_stream_t stream);
 
 /*
+ * Query-guided clusters with one proxy each and an error-gated read budget. Source:
+ * "OpenAttention reads 1% of the KV cache" -- section "Three helpers that make the
+ * proxy accurate" (QGC: keys projected onto the top eigenvectors of the queries and
+ * clustered by k-means in 16 dimensions once after prefill; ErrorGate: the exact-read
+ * budget split across clusters in proportion to the error each proxy would leave,
+ * estimated from cached mean and variance tokens at 1.5 KV rows a cluster, charged
+ * to the read; QGS: the top tokens inside each cluster from low-bit projections) and
+ * section "Skipping reviews without losing the verdict" (the count-aware mean proxy;
+ * a proxy's weight error is its mass times the spread of the weights it hides).
+ * A decode step is kv_select_qgc, kv_sparse_decode_attn in weighted mode over the
+ * read list, then kv_merge_qgc_proxies.
+ *
+ * kv_build_qgc -- once after prefill, per (sequence, KV head):
+ *   P        device [Hkv][16][D] fp32: the projection rows (the 16 leading rows of
+ *            kv_build_query_basis's evecs per head)
+ *   C        clusters, 1..64 (min(C, seq_len) are used); iters: Lloyd iterations, 1..100
+ *   z16      device out [B][Hkv][Ncap][16] bf16: P k per token (fp32, then bf16)
+ *   labels   device out [B][Hkv][Ncap] int32: cluster of each token (-1 past seq_len)
+ *   perm     device out [B][Hkv][Ncap] int32: the tokens grouped by cluster, ascending
+ *            inside a cluster (-1 past seq_len); offs: [B][Hkv][C + 1] int32 starts
+ *   counts   device out [B][Hkv][C] int32
+ *   k_sum, v_sum, k_sq  device out [B][Hkv][C][D] fp32: per cluster the key and value
+ *            sums and the per-channel key sum of squares (the mean and variance tokens)
+ *   workspace  device, kv_qgc_workspace_bytes(shape) bytes (fp32 coordinates)
+ * k-means: float64, starts at tokens ((2c + 1) n) // (2C'), ties to the lower cluster,
+ * the clusters are the last assignment.
+ */
+kv_status kv_build_qgc(const kv_shape* shape, const void* K, const void* V, const float* P, int C, int iters,
+                       void* z16, int32_t* labels, int32_t* perm, int32_t* offs, int32_t* counts, float* k_sum,
+                       float* v_sum, float* k_sq, void* workspace, size_t ws_bytes, kv_stream_t stream);
+size_t kv_qgc_workspace_bytes(const kv_shape* shape);
+
+/*
+ * kv_select_qgc -- per query: per cluster c, from the mean and variance tokens,
+ *   mu_g = scale q_g . mean_c, s2_g = scale^2 sum_d q_gd^2 var_cd,
+ *   E_c = sum_g n_c e^mu_g (e^(s2_g / 2) - 1) / sum_c' n_c' e^(mu_g + s2_g / 2)
+ * (the mean-logit proxy's shortfall against the cluster's expected mass under normal
+ * logits, per head normalised and summed over the group); the exact-read budget
+ * R = floor(budget n) - ceil(1.5 live clusters) split as r_c = min(n_c, floor(R E_c /
+ * sum E)); in every cluster the r_c tokens of largest t_i = sum_g exp(scale (P q_g) .
+ * z16_i - LSE_g) (ties to the lower index).
+ *   budget     read fraction in [0, 1]; max_read >= floor(budget Ncap)
+ *   tok_idx, w device out [B][Hkv][max_read]: the read tokens grouped by cluster with
+ *              weight 1, then index 0 / weight 0 (kv_sparse_decode_attn's weighted mode)
+ *   n_read     device out [B][Hkv] int32
+ *   proxy_k, proxy_v  device out [B][Hkv][C][D] fp32: per cluster the mean key and
+ *              value of its unread tokens (cluster sums minus the read rows)
+ *   proxy_n    device out [B][Hkv][C] int32: unread tokens per cluster (0: no proxy)
+ *   workspace  device, kv_qgc_select_workspace_bytes(shape) bytes (token scores)
+ * q bf16 or fp32 per shape->dtype; G <= 8.
+ */
+kv_status kv_select_qgc(const kv_shape* shape, const void* q, float scale, const float* P, int C, const void* z16,
+                        const int32_t* perm, const int32_t* offs, const int32_t* counts, const float* k_sum,
+                        const float* v_sum, const float* k_sq, const void* K, const void* V, float budget,
+                        int max_read, int32_t* tok_idx, float* w, int32_t* n_read, float* proxy_k, float* proxy_v,
+                        int32_t* proxy_n, void* workspace, size_t ws_bytes, kv_stream_t stream);
+size_t kv_qgc_select_workspace_bytes(const kv_shape* shape);
+
+/*
+ * kv_merge_qgc_proxies -- folds the cluster proxies into the attention over the read
+ * tokens, in place: with the read tokens' out [B][Hq][D] and lse [B][Hq] (from
+ * kv_sparse_decode_attn; lse is required) and proxy logits l_c = scale q . proxy_k_c +
+ * ln proxy_n_c, out <- (e^lse out + sum_c e^l_c proxy_v_c) / (e^lse + sum_c e^l_c) and
+ * lse <- ln(e^lse + sum_c e^l_c), evaluated with a max shift.
+ */
+kv_status kv_merge_qgc_proxies(const kv_shape* shape, const void* q, float scale, int C, const float* proxy_k,
+                               const float* proxy_v, const int32_t* proxy_n, float* out, float* lse,
+                               kv_stream_t stream);
+
+/*
  * kv_sparse_decode_attn -- softmax attention over a reduced KV cache.
  *
  * Block mode (tok_idx == NULL). Source: "OpenAttention reads 1% of the KV cache

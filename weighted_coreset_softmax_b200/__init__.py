@@ -16,6 +16,7 @@ Method (see include/kvsparse.h for the per-call sources):
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import re
 from typing import Optional
@@ -32,7 +33,8 @@ __all__ = [
     "kv_build_block_cov_factors", "kv_select_blocks_cobs", "kv_sparse_decode_attn", "kv_dense_decode_attn", "kv_decode_step", "kv_workspace_bytes",
     "kv_workspace_init", "kv_workspace_status", "kv_last_error", "Workspace", "kv_selftest_wait_timeout",
     "kv_stream_read", "kv_build_wildcat_coreset", "kv_build_query_basis", "kv_query_subspace_rank",
-    "kv_build_block_cov_factors_ss", "kv_quantize_fp4", "kv_select_blocks_cobs_fp4",
+    "kv_build_block_cov_factors_ss", "kv_quantize_fp4", "kv_select_blocks_cobs_fp4", "kv_build_qgc",
+    "kv_select_qgc", "kv_merge_qgc_proxies", "qgc_decode",
 ]
 
 KV_OK, KV_ERR_INVALID_ARG, KV_ERR_UNSUPPORTED, KV_ERR_CUDA, KV_ERR_DEVICE_CHECK = 0, 1, 2, 3, 4
@@ -106,6 +108,10 @@ def lib():
         "kv_quantize_fp4": [_P, ctypes.c_longlong, _I, _P, _P, _P],
         "kv_select_blocks_cobs_fp4": [_SHP, _P, _F, _P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P],
         "kv_query_subspace_rank": [_P, _I, _I, ctypes.c_double],
+        "kv_build_qgc": [_SHP, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P],
+        "kv_select_qgc": [_SHP, _P, _F, _P, _I, _P, _P, _P, _P, _P, _P, _P, _P, _P, _F, _I, _P, _P, _P, _P, _P,
+                          _P, _P, _S, _P],
+        "kv_merge_qgc_proxies": [_SHP, _P, _F, _I, _P, _P, _P, _P, _P, _P],
     }
     for name, args in sigs.items():
         fn = getattr(L, name)
@@ -117,6 +123,9 @@ def lib():
     L.kv_wildcat_workspace_bytes.restype = _S
     L.kv_query_basis_workspace_bytes.argtypes = [_I, _I]
     L.kv_query_basis_workspace_bytes.restype = _S
+    for fn in ("kv_qgc_workspace_bytes", "kv_qgc_select_workspace_bytes"):
+        getattr(L, fn).argtypes = [_SHP]
+        getattr(L, fn).restype = _S
     L.kv_last_error.argtypes = []
     L.kv_last_error.restype = ctypes.c_char_p
     _lib = L
@@ -636,3 +645,85 @@ def kv_select_blocks_cobs_fp4(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.
                                            int(bool(force_first)), int(bool(force_last)), int(kmax),
                                            _ptr(block_idx), _ptr(n_kept), _ptr(scores), _stream(dev)))
     return block_idx, n_kept, scores
+
+
+# ----------------------------------------------------------------- query-guided clusters
+def kv_build_qgc(K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, P: torch.Tensor, C: int = 32,
+                 iters: int = 8) -> dict:
+    """Clusters of every (sequence, KV head)'s keys in the projection P [Hkv][16][D]
+    and their cached mean and variance tokens (once after prefill)."""
+    _need(K, "K")
+    _need(V, "V", K.dtype)
+    _need(P, "P", torch.float32)
+    B, Hkv, Ncap, D = K.shape
+    dev = K.device
+    shape = KVShape(B, Hkv, Hkv, D, Ncap, 64, _dtype_code(K.dtype), seq_lens.data_ptr())
+    out = dict(
+        C=int(C),
+        z16=torch.empty(B, Hkv, Ncap, 16, dtype=torch.bfloat16, device=dev),
+        labels=torch.empty(B, Hkv, Ncap, dtype=torch.int32, device=dev),
+        perm=torch.empty(B, Hkv, Ncap, dtype=torch.int32, device=dev),
+        offs=torch.empty(B, Hkv, C + 1, dtype=torch.int32, device=dev),
+        counts=torch.empty(B, Hkv, C, dtype=torch.int32, device=dev),
+        k_sum=torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev),
+        v_sum=torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev),
+        k_sq=torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev),
+    )
+    ws = torch.empty(max(16, int(lib().kv_qgc_workspace_bytes(ctypes.byref(shape)))), dtype=torch.uint8, device=dev)
+    _check(lib().kv_build_qgc(ctypes.byref(shape), _ptr(K), _ptr(V), _ptr(P), int(C), int(iters), _ptr(out["z16"]),
+                              _ptr(out["labels"]), _ptr(out["perm"]), _ptr(out["offs"]), _ptr(out["counts"]),
+                              _ptr(out["k_sum"]), _ptr(out["v_sum"]), _ptr(out["k_sq"]), _ptr(ws), ws.numel(),
+                              _stream(dev)))
+    return out
+
+
+def kv_select_qgc(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+                  P: torch.Tensor, qgc: dict, budget: float, max_read: Optional[int] = None,
+                  workspace: Optional[torch.Tensor] = None):
+    """Error-gated read list and cluster proxies for one decode step. Returns
+    (tok_idx, w, n_read, proxy_k, proxy_v, proxy_n)."""
+    _need(q, "q", K.dtype)
+    B, Hkv, Ncap, D = K.shape
+    Hq = q.shape[1]
+    C = qgc["C"]
+    dev = q.device
+    if max_read is None:
+        max_read = max(1, int(math.floor(budget * Ncap)))
+    shape = KVShape(B, Hq, Hkv, D, Ncap, 64, _dtype_code(K.dtype), seq_lens.data_ptr())
+    tok_idx = torch.empty(B, Hkv, max_read, dtype=torch.int32, device=dev)
+    w = torch.empty(B, Hkv, max_read, dtype=torch.float32, device=dev)
+    n_read = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    pk = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
+    pv = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
+    pn = torch.empty(B, Hkv, C, dtype=torch.int32, device=dev)
+    need = int(lib().kv_qgc_select_workspace_bytes(ctypes.byref(shape)))
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
+    _check(lib().kv_select_qgc(ctypes.byref(shape), _ptr(q), float(scale), _ptr(P), int(C), _ptr(qgc["z16"]),
+                               _ptr(qgc["perm"]), _ptr(qgc["offs"]), _ptr(qgc["counts"]), _ptr(qgc["k_sum"]),
+                               _ptr(qgc["v_sum"]), _ptr(qgc["k_sq"]), _ptr(K), _ptr(V), float(budget), int(max_read),
+                               _ptr(tok_idx), _ptr(w), _ptr(n_read), _ptr(pk), _ptr(pv), _ptr(pn), _ptr(workspace),
+                               workspace.numel() * workspace.element_size(), _stream(dev)))
+    return tok_idx, w, n_read, pk, pv, pn
+
+
+def kv_merge_qgc_proxies(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tensor, scale: float, C: int,
+                         proxy_k: torch.Tensor, proxy_v: torch.Tensor, proxy_n: torch.Tensor, out: torch.Tensor,
+                         lse: torch.Tensor) -> None:
+    """Folds the cluster proxies into out / lse in place."""
+    B, Hkv, Ncap, D = K.shape
+    shape = KVShape(B, q.shape[1], Hkv, D, Ncap, 64, _dtype_code(K.dtype), seq_lens.data_ptr())
+    _check(lib().kv_merge_qgc_proxies(ctypes.byref(shape), _ptr(q), float(scale), int(C), _ptr(proxy_k),
+                                      _ptr(proxy_v), _ptr(proxy_n), _ptr(out), _ptr(lse), _stream(q.device)))
+
+
+def qgc_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+               P: torch.Tensor, qgc: dict, budget: float, ws: "Workspace", out: Optional[torch.Tensor] = None,
+               lse: Optional[torch.Tensor] = None, sel_workspace: Optional[torch.Tensor] = None):
+    """One decode step: the error-gated read list, attention over it (weighted mode,
+    weights 1) and the proxies folded in. Returns (out, lse, selection tuple)."""
+    sel = kv_select_qgc(q, K, V, seq_lens, scale, P, qgc, budget, workspace=sel_workspace)
+    tok_idx, w = sel[0], sel[1]
+    out, lse = kv_sparse_decode_attn(q, K, V, seq_lens, 64, scale, ws, tok_idx=tok_idx, w=w, out=out, lse=lse)
+    kv_merge_qgc_proxies(q, K, seq_lens, scale, qgc["C"], sel[3], sel[4], sel[5], out, lse)
+    return out, lse, sel
