@@ -47,7 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="llama", choices=["llama", "llama_b1", "qwen_long", "llama_osa", "llama_quest",
-                                                           "llama_cobs", "llama_cobs_fp4", "llama_coreset"])
+                                                           "llama_cobs", "llama_cobs_fp4", "llama_qgc",
+                                                           "llama_coreset"])
     ap.add_argument("--scorer", choices=["mean16", "sum32"], default="mean16",
                     help="summary-mode selection: bf16 block means (default) or fp32 block sums")
     ap.add_argument("--attn", choices=["v1", "v2"], default=None,
@@ -263,6 +264,32 @@ def cobs_fp4_select_bytes(wl, seq_lens, s_dim, rank=4):
     return total
 
 
+QGC_C, QGC_ITERS = 32, 8  # clusters per (sequence, KV head), Lloyd iterations
+
+
+def qgc_step_bytes(wl, n_read, budget):
+    """Algorithmic bytes of one QGC decode step, (selection, attention + merge): the
+    selection scans every token's bf16 projection (32 B) and member index, writes and
+    reads back its score, reads the cluster mean and variance tokens and the read rows
+    (keys and values, for the proxies), and writes the read list and the proxies; the
+    attention reads the read rows, q, and writes out / lse; the merge reads the proxies
+    and q and rewrites out / lse."""
+    D, G, C = wl.D, wl.G, QGC_C
+    es = 2 if str(wl.dtype).endswith("bfloat16") else 4
+    nr = n_read.cpu().tolist()
+    max_read = max(1, int(math.floor(budget * wl.Ncap)))
+    sel = att = 0
+    for b in range(wl.B):
+        n = wl.seq_lens[b]
+        for h in range(wl.Hkv):
+            r = int(nr[b][h])
+            sel += n * (32 + 4 + 8) + C * (3 * D * 4 + 8) + r * D * es * 2 + C * (2 * D * 4 + 4) + max_read * 8 \
+                + G * D * es + 4
+            att += r * (D * es * 2 + 8) + G * D * es + G * (D + 1) * 4 \
+                + C * (2 * D * 4 + 4) + G * D * es + 2 * G * (D + 1) * 4
+    return sel, att
+
+
 def osa_select_bytes(wl, seq_lens):
     es = 2 if str(wl.dtype).endswith("bfloat16") else 4
     return sum(wl.Hkv * (seq_lens[b] * wl.D * es + wl.G * wl.D * es) for b in range(wl.B))
@@ -310,6 +337,10 @@ def _oracle_task(args):
     if kind == "dense":
         O.dense_batch(q, K, V, [n], scale)
         return None
+    if kind == "qgc":
+        P_o, C_o, it_o, budget_o = extra
+        r = O.qgc_decode_one(q[0], K[0, 0], V[0, 0], n, P_o, C_o, it_o, budget_o, scale)
+        return {"kept": r["read"], "near_tie": r["near_tie"], "more": {}}
     if kind == "cobs_fp4":
         # the oracle's own stored descriptor of this pair: factors within its basis
         # (stored at fp32), rounded to fp32 and E2M1-coded with float32 decisions
@@ -355,7 +386,13 @@ def oracle_tasks(wl, pairs, more_k=()):
     from weighted_coreset_softmax_b200 import workloads as W
     tasks = []
     kind = {"summary": "summary", "summary_mean16": "summary_mean16", "exact_mass": "exact_mass", "quest": "quest",
-            "cobs": "cobs", "cobs_fp4": "cobs_fp4"}[wl.score_mode]
+            "cobs": "cobs", "cobs_fp4": "cobs_fp4", "qgc": "qgc"}[wl.score_mode]
+    if kind == "qgc" and not hasattr(wl, "oracle_qgc_basis"):
+        # the oracle's projection rows: its own top-16 query eigenvectors, stored at fp32
+        from oracle import oracle as O
+        Qc = W.calibration_queries(wl, CALIB_POSITIONS).to(torch.float64).cpu().numpy()
+        _, vec = O.query_basis(Qc, wl.Hkv)
+        wl.oracle_qgc_basis = vec[:, :16, :].astype(np.float32).astype(np.float64)
     if kind == "cobs_fp4" and not hasattr(wl, "oracle_basis"):
         # the oracle's basis and s from the calibration queries, stored at fp32
         from oracle import oracle as O
@@ -380,6 +417,8 @@ def oracle_tasks(wl, pairs, more_k=()):
             extra = (wl.tok_idx[b, h].cpu().numpy(), wl.w[b, h].cpu().numpy().astype(np.float64))
         if kind == "cobs_fp4":
             extra = (wl.oracle_basis[0][h], wl.oracle_basis[1], 4)
+        if kind == "qgc":
+            extra = (wl.oracle_qgc_basis[h], QGC_C, QGC_ITERS, wl.qgc_budget)
         tasks.append((kind, q, K, V, wl.seq_lens[b], wl.block_size, wl.scale, wl.k_top,
                       bool(wl.force_first), bool(wl.force_last), extra, tuple(more_k)))
     return tasks
@@ -464,7 +503,8 @@ def selection_check(wl, oracle_res, idx, nk, idx5=None, nk5=None, more_k=()):
             else:
                 out5["other_mismatch"] += 1
     ranking = {"summary_mean16": "bf16-mean ranking",
-               "cobs_fp4": "stored-descriptor ranking (the oracle's own basis, factors and E2M1 codes)"}
+               "cobs_fp4": "stored-descriptor ranking (the oracle's own basis, factors and E2M1 codes)",
+               "qgc": "read tokens of the oracle's own clusters, error split and in-cluster scores"}
     out["reference"] = ("float64 oracle, " + ranking.get(wl.score_mode, "exact-mean ranking")
                         + ", pairs of the CPU baseline sample")
     if out5 is not None:
@@ -484,7 +524,11 @@ def workload_label(wl, budget):
         "llama_cobs_fp4": "Llama-3.1-8B-shaped GQA decode, COBS stored descriptor (bf16 means, rank-4 E2M1 "
                           "factors in the 90%-energy query subspace)",
         "llama_coreset": "Llama-3.1-8B-shaped GQA decode, weighted coreset m=2048",
+        "llama_qgc": f"Llama-3.1-8B-shaped GQA decode, query-guided clusters (C={QGC_C}) with error-gated reads",
     }
+    if wl.attn_mode == "qgc":
+        return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, ctx={wl.Ncap}, "
+                f"read budget {budget:g} (exact tokens plus 1.5 rows a cluster, one proxy a cluster)")
     return (f"{names[wl.name]}: B={wl.B}, {wl.Hq} q heads / {wl.Hkv} KV heads, d={wl.D}, "
             f"ctx={wl.Ncap}, block={wl.block_size}, read budget {budget:g} "
             f"(top-{wl.k_top} + first + last + tail proxy)" if wl.attn_mode != "weighted" else
@@ -523,6 +567,21 @@ def run_ours(args, dist):
             su_["k_bounds"] = kv.kv_build_block_bounds(w_.K, sl_, w_.block_size)
         if w_.score_mode == "cobs":
             su_["k_xi"] = kv.kv_build_block_cov_factors(w_.K, sl_, w_.block_size, 4)
+        if w_.score_mode == "qgc":
+            if "P" not in shared_basis:  # the model's projection rows, from calibration queries
+                Qc = W.calibration_queries(w_, CALIB_POSITIONS)
+                evecs, _ = kv.kv_build_query_basis(Qc, w_.Hkv)
+                shared_basis.update(P=evecs[:, :16, :].contiguous(), Qc=Qc)
+            su_["qgc"] = kv.kv_build_qgc(w_.K, w_.V, sl_, shared_basis["P"], QGC_C, QGC_ITERS)
+            mr = max(1, int(math.floor(args.budget * w_.Ncap)))
+            su_["qsel"] = (torch.zeros(w_.B, w_.Hkv, mr, dtype=torch.int32, device=dev),
+                           torch.zeros(w_.B, w_.Hkv, mr, dtype=torch.float32, device=dev),
+                           torch.zeros(w_.B, w_.Hkv, dtype=torch.int32, device=dev),
+                           torch.zeros(w_.B, w_.Hkv, QGC_C, w_.D, dtype=torch.float32, device=dev),
+                           torch.zeros(w_.B, w_.Hkv, QGC_C, w_.D, dtype=torch.float32, device=dev),
+                           torch.zeros(w_.B, w_.Hkv, QGC_C, dtype=torch.int32, device=dev))
+            su_["qws"] = torch.empty(w_.B * w_.Hkv * w_.Ncap * 4, dtype=torch.uint8, device=dev)
+            w_.qgc_budget = args.budget
         if w_.score_mode == "cobs_fp4":
             if "U" not in shared_basis:  # one basis for the model: every batch draws queries from it
                 Qc = W.calibration_queries(w_, CALIB_POSITIONS)
@@ -561,12 +620,20 @@ def run_ours(args, dist):
     mode = kv.KV_SCORE_SUMMARY if wl.score_mode in ("summary", "summary_mean16") else kv.KV_SCORE_EXACT_MASS
     kmax = wl.kmax
     weighted = wl.attn_mode == "weighted"
+    qgc = wl.attn_mode == "qgc"
+
+    def su0_qsel():
+        return s0["summ"]["qsel"]
 
     def select_on(st_, q_=None, k_top=None, kmax_=None, idx_=None, nk_=None):
         if weighted:
             return
         w_, sl_, su_ = st_["wl"], st_["sl"], st_["summ"]
         q_ = w_.q if q_ is None else q_
+        if qgc:
+            kv.kv_select_qgc(q_, w_.K, w_.V, sl_, w_.scale, shared_basis["P"], su_["qgc"], args.budget,
+                             workspace=su_["qws"], out=su_["qsel"])
+            return
         if k_top is not None:
             kv.kv_select_blocks_mean16(q_, w_.K, sl_, w_.block_size, w_.scale, su_["k_mean"], su_["counts"], k_top,
                                        w_.force_first, w_.force_last, kmax=kmax_, block_idx=idx_, n_kept=nk_) \
@@ -603,7 +670,12 @@ def run_ours(args, dist):
             kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"], block_idx=idx_,
                                      n_kept=nk_, summaries=su_, use_tail_proxy=True, out=st_["out"], lse=st_["lse"])
             return
-        if weighted:
+        if qgc:
+            qs = su_["qsel"]
+            kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
+                                     tok_idx=qs[0], w=qs[1], out=st_["out"], lse=st_["lse"])
+            kv.kv_merge_qgc_proxies(q_, w_.K, sl_, w_.scale, QGC_C, qs[3], qs[4], qs[5], st_["out"], st_["lse"])
+        elif weighted:
             kv.kv_sparse_decode_attn(q_, w_.K, w_.V, sl_, w_.block_size, w_.scale, st_["ws"],
                                      tok_idx=w_.tok_idx, w=w_.w, out=st_["out"], lse=st_["lse"])
         else:
@@ -639,6 +711,10 @@ def run_ours(args, dist):
     if wl.score_mode == "cobs":
         builds["kv_build_block_cov_factors_ms"] = time_build(
             lambda: kv.kv_build_block_cov_factors(wl.K, sl, wl.block_size, 4, out=summ["k_xi"]), reps=1)
+    if qgc:
+        builds["kv_build_qgc_ms"] = time_build(
+            lambda: kv.kv_build_qgc(wl.K, wl.V, sl, shared_basis["P"], QGC_C, QGC_ITERS), reps=1)
+        builds["qgc"] = {"clusters": QGC_C, "lloyd_iterations": QGC_ITERS}
     if wl.score_mode == "cobs_fp4":
         builds["kv_build_query_basis_ms"] = time_build(
             lambda: kv.kv_build_query_basis(shared_basis["Qc"], wl.Hkv), reps=1)
@@ -908,7 +984,8 @@ def run_ours(args, dist):
             secondary["kernels_ms_back_to_back"]["kv_select_blocks"] = graph_avg_ms(
                 lambda i: select_on(sets[i % ROT]), k_steps)
         sink = torch.zeros(1, dtype=torch.int32, device=dev)
-        a_b = attention_bytes(wl, nk, wl.seq_lens) if not weighted else weighted_bytes(wl)
+        a_b = (qgc_step_bytes(wl, su0_qsel()[2], args.budget)[1] if qgc else
+               attention_bytes(wl, nk, wl.seq_lens) if not weighted else weighted_bytes(wl))
         floor = {"attn_bytes_alone_ms": alone_avg_ms(
             lambda i: kv.kv_stream_read(sets[i % ROT]["wl"].K, a_b & ~15, sink), k_steps),
                  "attn_bytes_back_to_back_ms": graph_avg_ms(
@@ -954,6 +1031,8 @@ def run_ours(args, dist):
     # algorithmic bytes and the roofline of the dominant kernel
     if weighted:
         a_bytes, s_bytes = weighted_bytes(wl), 0
+    elif qgc:
+        s_bytes, a_bytes = qgc_step_bytes(wl, su0_qsel()[2], args.budget)
     else:
         a_bytes = attention_bytes(wl, nk, wl.seq_lens)
         s_bytes = (quest_select_bytes(wl, wl.seq_lens) if quest else
@@ -1004,7 +1083,9 @@ def run_ours(args, dist):
                   f"ms_per_step: K steps back to back (one CUDA graph) in one event pair; ms_per_step_isolated: an event "
                   f"pair around each step; ms_per_step_l2_flushed: the step on one batch after a 512 MiB "
                   f"L2-flushing write",
-            "step": "kv_select_blocks + kv_sparse_decode_attn" if not weighted else "kv_sparse_decode_attn",
+            "step": ("kv_select_qgc + kv_sparse_decode_attn (weighted, the read tokens) + kv_merge_qgc_proxies "
+                     "(kernels_ms.kv_sparse_decode_attn covers the last two)") if qgc else
+                    "kv_select_blocks + kv_sparse_decode_attn" if not weighted else "kv_sparse_decode_attn",
         },
         "achieved_step_GB_s": step_gbs,
         "achieved_step_pct_of_8TBs": 100.0 * step_gbs / NOMINAL_HBM_GBS,
@@ -1023,7 +1104,7 @@ def run_ours(args, dist):
             "how": "q in from pinned host memory and out/lse back every step, on two copy streams "
                    f"overlapping the neighbouring steps' kernels; {ROT} independent batches rotate "
                    "(inputs never L2-resident); 24 steps per CUDA graph replay"},
-        "gpu_launches": (1 if weighted else 2) * K_steps,  # our kernels in the timed steps
+        "gpu_launches": (1 if weighted else 3 if qgc else 2) * K_steps,  # our kernels in the timed steps
         "clocks": clk,
         "dense": dense,
         "builds_once_after_prefill": builds,
@@ -1032,7 +1113,12 @@ def run_ours(args, dist):
     if dist.rank == 0 and dist.world == 1 and not args.no_cpu_baseline:
         more_k = (secondary["budget_5pct"]["k_top"],) if "budget_5pct" in secondary else ()
         res["cpu_baseline"], oracle_res = cpu_baseline(wl, args.cpu_seconds, workload_label(wl, args.budget), more_k)
-        if not weighted and not args.no_selection_check:
+        if qgc and not args.no_selection_check:
+            qs = su0_qsel()
+            big = torch.iinfo(torch.int32).max
+            srt = torch.sort(torch.where(qs[1] > 0, qs[0], torch.full_like(qs[0], big)), dim=-1).values
+            res["selection_check"] = selection_check(wl, oracle_res, srt, qs[2])
+        elif not weighted and not args.no_selection_check:
             res["selection_check"] = selection_check(wl, oracle_res, idx, nk,
                                                      s0.get("idx5"), s0.get("nk5"), more_k)
     dist.close()

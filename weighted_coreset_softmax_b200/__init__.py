@@ -679,9 +679,9 @@ def kv_build_qgc(K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, P: to
 
 def kv_select_qgc(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, scale: float,
                   P: torch.Tensor, qgc: dict, budget: float, max_read: Optional[int] = None,
-                  workspace: Optional[torch.Tensor] = None):
+                  workspace: Optional[torch.Tensor] = None, out: Optional[tuple] = None):
     """Error-gated read list and cluster proxies for one decode step. Returns
-    (tok_idx, w, n_read, proxy_k, proxy_v, proxy_n)."""
+    (tok_idx, w, n_read, proxy_k, proxy_v, proxy_n) (written into `out` when given)."""
     _need(q, "q", K.dtype)
     B, Hkv, Ncap, D = K.shape
     Hq = q.shape[1]
@@ -690,12 +690,16 @@ def kv_select_qgc(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: t
     if max_read is None:
         max_read = max(1, int(math.floor(budget * Ncap)))
     shape = KVShape(B, Hq, Hkv, D, Ncap, 64, _dtype_code(K.dtype), seq_lens.data_ptr())
-    tok_idx = torch.empty(B, Hkv, max_read, dtype=torch.int32, device=dev)
-    w = torch.empty(B, Hkv, max_read, dtype=torch.float32, device=dev)
-    n_read = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
-    pk = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
-    pv = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
-    pn = torch.empty(B, Hkv, C, dtype=torch.int32, device=dev)
+    if out is not None:
+        tok_idx, w, n_read, pk, pv, pn = out
+        max_read = int(tok_idx.shape[-1])
+    else:
+        tok_idx = torch.empty(B, Hkv, max_read, dtype=torch.int32, device=dev)
+        w = torch.empty(B, Hkv, max_read, dtype=torch.float32, device=dev)
+        n_read = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+        pk = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
+        pv = torch.empty(B, Hkv, C, D, dtype=torch.float32, device=dev)
+        pn = torch.empty(B, Hkv, C, dtype=torch.int32, device=dev)
     need = int(lib().kv_qgc_select_workspace_bytes(ctypes.byref(shape)))
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(16, need), dtype=torch.uint8, device=dev)
@@ -719,10 +723,11 @@ def kv_merge_qgc_proxies(q: torch.Tensor, K: torch.Tensor, seq_lens: torch.Tenso
 
 def qgc_decode(q: torch.Tensor, K: torch.Tensor, V: torch.Tensor, seq_lens: torch.Tensor, scale: float,
                P: torch.Tensor, qgc: dict, budget: float, ws: "Workspace", out: Optional[torch.Tensor] = None,
-               lse: Optional[torch.Tensor] = None, sel_workspace: Optional[torch.Tensor] = None):
+               lse: Optional[torch.Tensor] = None, sel_workspace: Optional[torch.Tensor] = None,
+               sel_out: Optional[tuple] = None):
     """One decode step: the error-gated read list, attention over it (weighted mode,
     weights 1) and the proxies folded in. Returns (out, lse, selection tuple)."""
-    sel = kv_select_qgc(q, K, V, seq_lens, scale, P, qgc, budget, workspace=sel_workspace)
+    sel = kv_select_qgc(q, K, V, seq_lens, scale, P, qgc, budget, workspace=sel_workspace, out=sel_out)
     tok_idx, w = sel[0], sel[1]
     out, lse = kv_sparse_decode_attn(q, K, V, seq_lens, 64, scale, ws, tok_idx=tok_idx, w=w, out=out, lse=lse)
     kv_merge_qgc_proxies(q, K, seq_lens, scale, qgc["C"], sel[3], sel[4], sel[5], out, lse)

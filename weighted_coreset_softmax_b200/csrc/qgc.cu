@@ -47,6 +47,7 @@ constexpr int QG_THREADS = 512;
 constexpr int QG_NW = QG_THREADS / 32;
 constexpr int QG_DIM = 16;     // projection dimension
 constexpr int QG_MAX_C = 64;   // clusters per (sequence, KV head)
+constexpr int QG_TCAP = 49152;  // token scores kept in shared memory (longer sequences use the scratch)
 
 __host__ __device__ inline size_t qgc_build_smem_bytes(int D, int C) {
   return static_cast<size_t>(QG_DIM) * D * 4 +                 // P rows
@@ -251,6 +252,45 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_build_kernel(const T* __restri
   }
 }
 
+__device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    const unsigned long long y = __shfl_xor_sync(FULL_MASK, x, o);
+    x = y > x ? y : x;
+  }
+  return x;
+}
+
+// A lane's CPL consecutive channels of a row, as fp32 (one vector load).
+template <typename T, int CPL>
+__device__ __forceinline__ void qg_slice(const T* row, int lane, float (&x)[CPL]) {
+  if constexpr (sizeof(T) == 2) {
+    if constexpr (CPL == 4) {
+      const uint2 r = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+      x[0] = __uint_as_float(r.x << 16);
+      x[1] = __uint_as_float(r.x & 0xffff0000u);
+      x[2] = __uint_as_float(r.y << 16);
+      x[3] = __uint_as_float(r.y & 0xffff0000u);
+    } else {
+      const uint32_t r = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
+      x[0] = __uint_as_float(r << 16);
+      x[1] = __uint_as_float(r & 0xffff0000u);
+    }
+  } else {
+    if constexpr (CPL == 4) {
+      const float4 r = __ldg(reinterpret_cast<const float4*>(row) + lane);
+      x[0] = r.x;
+      x[1] = r.y;
+      x[2] = r.z;
+      x[3] = r.w;
+    } else {
+      const float2 r = __ldg(reinterpret_cast<const float2*>(row) + lane);
+      x[0] = r.x;
+      x[1] = r.y;
+    }
+  }
+}
+
 struct QgcSel {
   const void* q;
   const void* K;
@@ -287,6 +327,7 @@ struct QgcSelShared {
 template <typename T, int D, int G>
 __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) {
   __shared__ QgcSelShared sh;
+  extern __shared__ __align__(16) float qg_ts[];  // token scores, when n <= QG_TCAP
   constexpr int CPL = D / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x, b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
@@ -298,7 +339,7 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
   const int32_t* pm = p.perm + static_cast<size_t>(bh) * p.Ncap;
   const T* Kb = static_cast<const T*>(p.K) + static_cast<size_t>(bh) * p.Ncap * D;
   const T* Vb = static_cast<const T*>(p.V) + static_cast<size_t>(bh) * p.Ncap * D;
-  float* t = p.tws + static_cast<size_t>(bh) * p.Ncap;
+  float* t = p.Ncap <= QG_TCAP ? qg_ts : p.tws + static_cast<size_t>(bh) * p.Ncap;
 
   // the group's queries, a lane CPL channels of each
   float qf[G][CPL];
@@ -398,37 +439,64 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
   }
   __syncthreads();
 
-  // ---- token scores: LSE per head over the tokens, then t_i (two passes)
+  // ---- token scores: LSE per head over the tokens, then t_i (two passes; the next
+  // token's coordinates are loaded before the current one's arithmetic)
   {
+    const uint4* zbase = reinterpret_cast<const uint4*>(p.z16 + static_cast<size_t>(bh) * p.Ncap * QG_DIM);
+    auto logits = [&](uint4 a, uint4 bq, float (&sg)[G]) {
+      float z[QG_DIM];
+      float2 f[4];
+      Chunk<__nv_bfloat16>::unpack(a, f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        z[2 * e] = f[e].x;
+        z[2 * e + 1] = f[e].y;
+      }
+      Chunk<__nv_bfloat16>::unpack(bq, f);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        z[8 + 2 * e] = f[e].x;
+        z[8 + 2 * e + 1] = f[e].y;
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float a2 = 0.f;
+#pragma unroll
+        for (int j = 0; j < QG_DIM; ++j) a2 = fmaf(sh.qt[g][j], z[j], a2);
+        sg[g] = a2 * p.sigma;
+      }
+    };
     float m[G], l[G];
 #pragma unroll
     for (int g = 0; g < G; ++g) {
       m[g] = -INFINITY;
       l[g] = 0.f;
     }
+    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
+    if (tid < n) {
+      c0 = __ldg(zbase + 2 * tid);
+      c1 = __ldg(zbase + 2 * tid + 1);
+    }
     for (int i = tid; i < n; i += QG_THREADS) {
-      const uint4* zr = reinterpret_cast<const uint4*>(p.z16 + (static_cast<size_t>(bh) * p.Ncap + i) * QG_DIM);
-      float z[QG_DIM];
-      float2 f[4];
-      Chunk<__nv_bfloat16>::unpack(__ldg(zr), f);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) { z[2 * e] = f[e].x; z[2 * e + 1] = f[e].y; }
-      Chunk<__nv_bfloat16>::unpack(__ldg(zr + 1), f);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) { z[8 + 2 * e] = f[e].x; z[8 + 2 * e + 1] = f[e].y; }
+      const int inx = i + QG_THREADS;
+      uint4 n0 = c0, n1 = c1;
+      if (inx < n) {
+        n0 = __ldg(zbase + 2 * inx);
+        n1 = __ldg(zbase + 2 * inx + 1);
+      }
+      float sg[G];
+      logits(c0, c1, sg);
 #pragma unroll
       for (int g = 0; g < G; ++g) {
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < QG_DIM; ++j) s = fmaf(sh.qt[g][j], z[j], s);
-        s *= p.sigma;
-        if (s > m[g]) {
-          l[g] = l[g] * __expf(m[g] - s) + 1.f;
-          m[g] = s;
+        if (sg[g] > m[g]) {
+          l[g] = l[g] * __expf(m[g] - sg[g]) + 1.f;
+          m[g] = sg[g];
         } else {
-          l[g] += __expf(s - m[g]);
+          l[g] += __expf(sg[g] - m[g]);
         }
       }
+      c0 = n0;
+      c1 = n1;
     }
 #pragma unroll
     for (int g = 0; g < G; ++g) {
@@ -451,50 +519,65 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
       sh.lse[tid] = M == -INFINITY ? -INFINITY : M + __logf(L);
     }
     __syncthreads();
+    if (tid < n) {
+      c0 = __ldg(zbase + 2 * tid);
+      c1 = __ldg(zbase + 2 * tid + 1);
+    }
     for (int i = tid; i < n; i += QG_THREADS) {
-      const uint4* zr = reinterpret_cast<const uint4*>(p.z16 + (static_cast<size_t>(bh) * p.Ncap + i) * QG_DIM);
-      float z[QG_DIM];
-      float2 f[4];
-      Chunk<__nv_bfloat16>::unpack(__ldg(zr), f);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) { z[2 * e] = f[e].x; z[2 * e + 1] = f[e].y; }
-      Chunk<__nv_bfloat16>::unpack(__ldg(zr + 1), f);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) { z[8 + 2 * e] = f[e].x; z[8 + 2 * e + 1] = f[e].y; }
+      const int inx = i + QG_THREADS;
+      uint4 n0 = c0, n1 = c1;
+      if (inx < n) {
+        n0 = __ldg(zbase + 2 * inx);
+        n1 = __ldg(zbase + 2 * inx + 1);
+      }
+      float sg[G];
+      logits(c0, c1, sg);
       float tv = 0.f;
 #pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float s = 0.f;
-#pragma unroll
-        for (int j = 0; j < QG_DIM; ++j) s = fmaf(sh.qt[g][j], z[j], s);
-        tv += __expf(p.sigma * s - sh.lse[g]);
-      }
+      for (int g = 0; g < G; ++g) tv += __expf(sg[g] - sh.lse[g]);
       t[i] = tv;
+      c0 = n0;
+      c1 = n1;
     }
   }
   __syncthreads();
 
   // ---- per cluster: the r_c largest keys (t's bits, inverted index), the read list,
-  // the read rows' sums and the proxy of the unread tokens (a warp per cluster)
+  // the read rows' sums and the proxy of the unread tokens (a warp per cluster); the
+  // scores are read through the member list (shared memory for sequences up to
+  // QG_TCAP tokens)
+  auto key_of = [&](int i) {
+    return (static_cast<unsigned long long>(__float_as_uint(t[i])) << 32) |
+           static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(i));
+  };
   for (int c = warp; c < C; c += QG_NW) {
     const int nc = cnt[c], rc = sh.r[c];
     const int m0 = off[c], m1 = off[c + 1];
     unsigned long long thr = 0ull;  // keys >= thr are read
     if (rc > 0 && rc < nc) {
-      unsigned long long prefix = 0ull;
-      for (int bit = 63; bit >= 0; --bit) {
-        const unsigned long long cand = prefix | (1ull << bit);
-        int k = 0;
-        for (int m = m0 + lane; m < m1; m += 32) {
-          const int i = pm[m];
-          const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(t[i])) << 32) |
-                                         static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(i));
-          k += key >= cand;
+      if (rc <= 32) {
+        // rc rounds of "largest key below the previous one" (keys are distinct)
+        unsigned long long prev = ~0ull;
+        for (int k = 0; k < rc; ++k) {
+          unsigned long long best = 0ull;
+          for (int m = m0 + lane; m < m1; m += 32) {
+            const unsigned long long x = key_of(pm[m]);
+            if (x < prev && x > best) best = x;
+          }
+          prev = warp_max_u64(best);
         }
-        k = __reduce_add_sync(FULL_MASK, k);
-        if (k >= rc) prefix = cand;
+        thr = prev;
+      } else {
+        unsigned long long prefix = 0ull;
+        for (int bit = 63; bit >= 0; --bit) {
+          const unsigned long long cand = prefix | (1ull << bit);
+          int k = 0;
+          for (int m = m0 + lane; m < m1; m += 32) k += key_of(pm[m]) >= cand;
+          k = __reduce_add_sync(FULL_MASK, k);
+          if (k >= rc) prefix = cand;
+        }
+        thr = prefix;
       }
-      thr = prefix;
     }
     float rk[CPL], rv[CPL];
 #pragma unroll
@@ -507,9 +590,7 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
         bool take = false;
         if (mi < m1) {
           i = pm[mi];
-          const unsigned long long key = (static_cast<unsigned long long>(__float_as_uint(t[i])) << 32) |
-                                         static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(i));
-          take = rc >= nc || key >= thr;
+          take = rc >= nc || key_of(i) >= thr;
         }
         const unsigned bal = __ballot_sync(FULL_MASK, take);
         if (take) {
@@ -520,15 +601,31 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
           }
         }
         pos += __popc(bal);
-        for (unsigned bb = bal; bb; bb &= bb - 1) {  // the read rows of this chunk
-          const int src = __ffs(bb) - 1;
-          const int ti = __shfl_sync(FULL_MASK, i, src);
+      }
+      // the read rows' key and value sums, eight rows' loads in flight
+      __syncwarp();  // the list entries written above are visible to every lane
+      const int32_t* lst = p.tok_idx + static_cast<size_t>(bh) * p.max_read + sh.roff[c];
+      const int nl = min(rc, p.max_read - sh.roff[c]);
+      for (int j0 = 0; j0 < nl; j0 += 8) {
+        float kx[8][CPL], vx[8][CPL];
 #pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            rk[k] += load_as_float(Kb + static_cast<size_t>(ti) * D + lane * CPL + k);
-            rv[k] += load_as_float(Vb + static_cast<size_t>(ti) * D + lane * CPL + k);
+        for (int u = 0; u < 8; ++u) {
+          if (j0 + u < nl) {
+            const int ti = lst[j0 + u];
+            qg_slice<T, CPL>(Kb + static_cast<size_t>(ti) * D, lane, kx[u]);
+            qg_slice<T, CPL>(Vb + static_cast<size_t>(ti) * D, lane, vx[u]);
+          } else {
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) kx[u][k] = vx[u][k] = 0.f;
           }
         }
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+#pragma unroll
+          for (int k = 0; k < CPL; ++k) {
+            rk[k] += kx[u][k];
+            rv[k] += vx[u][k];
+          }
       }
     }
     const int un = nc - rc;  // unread tokens of the cluster
@@ -641,11 +738,26 @@ cudaError_t qgc_build_td(const kv_shape* s, const void* K, const void* V, const 
   return cudaGetLastError();
 }
 
+constexpr int QG_KEY_SMEM = kvs::QG_TCAP * 4;
+
 template <typename T, int D>
 cudaError_t qgc_select_td(int G, const kvs::QgcSel& p, int grid, cudaStream_t st) {
   switch (G) {
-#define QG_CASE(GG) \
-  case GG: kvs::qgc_select_kernel<T, D, GG><<<grid, kvs::QG_THREADS, 0, st>>>(p); break;
+#define QG_CASE(GG)                                                                                     \
+  case GG: {                                                                                             \
+    static std::atomic<int> cfg_##GG{0};                                                                 \
+    int dev = 0;                                                                                         \
+    cudaGetDevice(&dev);                                                                                 \
+    if (!(cfg_##GG.load() & (1 << (dev & 31)))) {                                                        \
+      const cudaError_t e = cudaFuncSetAttribute(kvs::qgc_select_kernel<T, D, GG>,                       \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, QG_KEY_SMEM); \
+      if (e != cudaSuccess) return e;                                                                    \
+      cfg_##GG.fetch_or(1 << (dev & 31));                                                                \
+    }                                                                                                    \
+    kvs::qgc_select_kernel<T, D, GG><<<grid, kvs::QG_THREADS,                                           \
+                                       p.Ncap <= kvs::QG_TCAP ? p.Ncap * 4 : 0, st>>>(p);                \
+    break;                                                                                               \
+  }
     QG_CASE(1) QG_CASE(2) QG_CASE(3) QG_CASE(4) QG_CASE(5) QG_CASE(6) QG_CASE(7) QG_CASE(8)
 #undef QG_CASE
     default: return cudaErrorInvalidValue;

@@ -139,7 +139,8 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
     "llama_osa" (exact-mass scoring), "llama_quest" (key-box bound scoring),
     "llama_cobs" (second-order scoring, rank-4 covariance factors),
     "llama_cobs_fp4" (the stored descriptor: bf16 means, query-subspace E2M1
-    factors; anisotropic queries), "llama_coreset" (weighted coreset, m=2048).
+    factors; anisotropic queries), "llama_qgc" (query-guided clusters with an
+    error-gated read; anisotropic queries), "llama_coreset" (weighted coreset, m=2048).
     Keyword overrides shrink a workload for fast tests while keeping its head
     shapes and distributions.
     """
@@ -176,6 +177,10 @@ def make(name: str, device="cpu", *, B=None, Ncap=None, seq_lens=None, budget=0.
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=None, ff=1, fl=1, smode="cobs_fp4", amode="proxy", planted=32,
                     seeds=[6], per_seq=False, plain=False, aniso=True)
+    elif name == "llama_qgc":
+        spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
+                    k_top=0, ff=0, fl=0, smode="qgc", amode="qgc", planted=32,
+                    seeds=[7], per_seq=False, plain=False, aniso=True)
     elif name == "llama_coreset":
         spec = dict(B=32, Hq=32, Hkv=8, D=128, Ncap=32768, L=64, dtype=torch.bfloat16,
                     k_top=0, ff=0, fl=0, smode="summary", amode="weighted", planted=32,
