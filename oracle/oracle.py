@@ -65,6 +65,25 @@ notes of the repository):
       space) distance between the sum over all tokens and the weighted coreset,
       whose minimiser solves A_SS w = A_{S,:} 1; negative weights are clipped to
       0; the uniforms of the pivot draws are inputs.
+  R15 COBS stored descriptor (the subspace and quantisation paragraphs): U_Q is
+      the top-s eigenvectors of each KV head's query second moment, the mean of
+      q q^T over calibration positions and the group's query heads, stored at
+      fp32; s = ceil(mean over heads of the smallest rank reaching 90% of the
+      head's trace); the factors are the scaled top-r eigenvectors of
+      U_Q^T Sigma_b U_Q; E2M1 codes take one scale per factor, max|x| / 6, the
+      nearest magnitude with ties to the even code, decided in float32; the
+      block mean is the bf16 mean of R13.
+  R16 QGC + ErrorGate (OpenAttention, "Three helpers"): the projection is the
+      top-16 query eigenvectors of R15, stored at fp32; k-means is Lloyd's
+      iteration in float64 from evenly spaced tokens, the clusters being the
+      last assignment; the mean and variance tokens are per cluster the key and
+      value means and the per-channel key variance; a proxy's error is the
+      lognormal gap n e^mu (e^(s2/2) - 1) between its cluster's expected mass and
+      the mean-logit proxy's mass, normalised per head and summed over the group;
+      the read budget floor(budget n) less 1.5 rows a cluster is split as
+      floor(R E_c / sum E) capped at the cluster size; inside a cluster the top
+      tokens by the Equation 5 combination of per-head softmax scores from the bf16
+      projections; one count-aware proxy per cluster of its unread tokens.
 """
 from __future__ import annotations
 
@@ -182,7 +201,7 @@ def cobs_logits(qg: np.ndarray, k_sum: np.ndarray, counts: np.ndarray, xi: np.nd
 
 def query_basis(Qc: np.ndarray, Hkv: int):
     """The eigenvectors of each KV head's query second moment [COBS, the subspace
-    paragraph: U_Q holds the top s eigenvectors of E[q q^T]; reading R22]. The
+    paragraph: U_Q holds the top s eigenvectors of E[q q^T]; reading R15]. The
     second moment of KV head h is the mean of q q^T over the calibration positions
     and the query heads of its group. Qc: [Nc][Hq][D]. Returns (evals [Hkv][D] in
     descending order, evecs [Hkv][D][D] whose row j is the unit eigenvector of
@@ -203,7 +222,7 @@ def query_basis(Qc: np.ndarray, Hkv: int):
 def subspace_rank(evals: np.ndarray, energy: float = 0.9):
     """The subspace dimension s [COBS, the subspace paragraph: s is set per layer
     from the rank capturing 90% of the query spectral energy, averaged over heads;
-    reading R22]: per head the smallest s_h whose leading eigenvalues sum to at least
+    reading R15]: per head the smallest s_h whose leading eigenvalues sum to at least
     `energy` of the trace, then s = ceil(mean over heads of s_h). Returns (s, [s_h])."""
     sh = []
     for lam in np.asarray(evals, dtype=np.float64):
@@ -221,7 +240,7 @@ def subspace_rank(evals: np.ndarray, energy: float = 0.9):
 def block_cov_factors_ss_one(K: np.ndarray, n: int, L: int, NBcap: int, r: int, U: np.ndarray):
     """Per block, the top r scaled eigenvectors of the covariance kept within the
     query subspace [COBS, the subspace paragraph: B_b = U_Q^T Sigma_b U_Q, rank-r
-    spectral decomposition in the projected space; reading R22]. U: [s][D], rows the
+    spectral decomposition in the projected space; reading R15]. U: [s][D], rows the
     basis (U_Q^T). Returns xi [NBcap][r][s] (xi_i = sqrt(lambda_i) u_i for the r
     largest eigenvalues of B_b, descending) and the eigenvalues [NBcap][r]; blocks
     past the sequence and directions past B_b's rank stay 0."""
@@ -246,7 +265,7 @@ E2M1_GRID = (0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0)  # magnitudes of codes 0..7
 def fp4_e2m1_quantize(x):
     """E2M1 FP4 codes of one vector with one fp32 scale [COBS, the quantisation
     paragraph: the scaled eigenvectors in E2M1 FP4 with one fp32 scale each;
-    reading R22]. The scale is max|x| / 6 (6 is the largest E2M1 magnitude); each
+    reading R15]. The scale is max|x| / 6 (6 is the largest E2M1 magnitude); each
     x_j / scale goes to the nearest E2M1 magnitude, a tie to the code with mantissa
     bit 0 (the even code), with the sign in bit 3 (zero keeps code 0). The scale and
     the quotients are float32 operations, the precision in which the kernel takes the
@@ -299,13 +318,13 @@ def cobs_subspace_logits(qg: np.ndarray, mean: np.ndarray, counts: np.ndarray, x
 def qgc_project(K: np.ndarray, n: int, P: np.ndarray) -> np.ndarray:
     """z_i = P k_i, the keys' coordinates on the top eigenvectors of the queries,
     stored at fp32 [OA, "Three helpers that make the proxy accurate": keys are
-    projected onto the top eigenvectors of the queries; reading R23]. P: [16][D]."""
+    projected onto the top eigenvectors of the queries; reading R16]. P: [16][D]."""
     return (np.asarray(K[:n], dtype=np.float64) @ np.asarray(P, dtype=np.float64).T).astype(np.float32)
 
 
 def qgc_kmeans(Z32: np.ndarray, C: int, iters: int):
     """k-means in the projection [OA, "Three helpers": k-means in 16 dimensions, once
-    after prefill; reading R23], Lloyd's iteration in float64 on the fp32 coordinates:
+    after prefill; reading R16], Lloyd's iteration in float64 on the fp32 coordinates:
     C' = min(C, n) centroids start at the tokens ((2c + 1) n) // (2 C'); each iteration
     assigns every token to the nearest centroid (squared distance summed over the
     coordinates in order; ties to the lower cluster) and moves every non-empty
@@ -336,7 +355,7 @@ def qgc_kmeans(Z32: np.ndarray, C: int, iters: int):
 
 def qgc_cluster_stats(K: np.ndarray, V: np.ndarray, n: int, labels: np.ndarray, C: int):
     """The cached tokens of every cluster [OA, "Three helpers": the mean and variance
-    tokens; reading R23]: count [C], key sum [C][D], value sum [C][D] and per-channel
+    tokens; reading R16]: count [C], key sum [C][D], value sum [C][D] and per-channel
     key sum of squares [C][D] (mean = sum / count, variance = squares / count - mean^2)."""
     D = K.shape[1]
     cnt = np.zeros(C, dtype=np.int64)
@@ -354,7 +373,7 @@ def errorgate_errors(qg: np.ndarray, cnt, ks, kq, sigma: float) -> np.ndarray:
     """The estimated weight error each cluster's proxy would leave [OA, "Skipping
     reviews without losing the verdict": a proxy's unnormalised weight error is its
     mass times the spread of the weights it hides; "Three helpers": ErrorGate
-    estimates it from the cached mean and variance tokens; reading R23]. With the
+    estimates it from the cached mean and variance tokens; reading R16]. With the
     cluster's logits read as normal with mean mu_gc = sigma q_g . mean_c and variance
     s2_gc = sigma^2 sum_d q_gd^2 var_cd, the mean-logit proxy's mass n_c e^mu falls
     short of the cluster's expected mass n_c e^(mu + s2/2) by
@@ -408,7 +427,7 @@ def errorgate_split(E: np.ndarray, cnt, R: int):
 
 def qgs_token_scores(qg: np.ndarray, Z16: np.ndarray, P: np.ndarray, sigma: float) -> np.ndarray:
     """Token scores inside the clusters [OA, "Three helpers": QGS picks the top tokens
-    inside each cluster from low-bit projections; reading R23]: with the projections
+    inside each cluster from low-bit projections; reading R16]: with the projections
     stored at bf16 (Z16) and the query projected the same way (P q_g),
     t_i = sum_g exp(sigma (P q_g) . z_i - LSE_g), LSE_g over all tokens (the group
     combination of Equation 5, per token)."""
@@ -712,7 +731,7 @@ def weighted_attend_one(qg, K, V, n, tok_idx, w, sigma):
 
 
 def wildcat_kernel(K: np.ndarray, n: int, sigma: float) -> np.ndarray:
-    """The kernel on the keys the coreset is chosen for [WC, abstract; reading R20]:
+    """The kernel on the keys the coreset is chosen for [WC, abstract; reading R14]:
     A[i, j] = exp(sigma k_i . k_j - sigma M) over the first n keys, M = max_i |k_i|^2.
     The constant shift keeps every entry in (0, 1] (k_i . k_j <= M by Cauchy-Schwarz)
     and cancels in the pivot choice and in the weights."""
@@ -784,7 +803,7 @@ def rpcholesky_steps(K: np.ndarray, n: int, sigma: float, u, m: int, pivots=None
 
 def wildcat_weights(K: np.ndarray, n: int, sigma: float, S) -> Tuple[np.ndarray, np.ndarray]:
     """The coreset weights [WC, abstract: "weight the elements optimally to
-    minimise reconstruction error"; reading R20]: the w minimising the kernel
+    minimise reconstruction error"; reading R14]: the w minimising the kernel
     distance || sum_{i<n} phi(k_i) - sum_{j in S} w_j phi(k_j) ||^2, i.e. the
     solution of A_SS w = A_{S,:} 1. Returns (w, w clipped at 0); the attention
     takes ln w, so a negative weight drops its token."""

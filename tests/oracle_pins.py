@@ -1002,6 +1002,30 @@ def pin_qgc_equal_logits_exact(seed=38):
     _close(res["out"], od, 1e-12, what="equal logits: dense")
     _close(res["lse"], ld, 1e-12, what="equal logits: lse")
 
+
+def pin_qgc_select_and_budget(seed=39):
+    """In-cluster choice by brute force: in every cluster the r_c tokens of largest
+    score, ties to the lower index (written as a sort over (score, index) pairs per
+    cluster), ascending; the near-tie flag on a constructed tie; the read budget by
+    hand (1% of 32768 less 1.5 rows for each of 32 clusters: 327 - 48 = 279)."""
+    r = _rng(seed)
+    n, C = 40, 4
+    t = r.uniform(size=n)
+    labels = r.integers(0, C, size=n)
+    rc = [3, 0, 5, 100]
+    got, near = O.qgc_select(t, labels, rc)
+    want = []
+    for c in range(C):
+        mem = [(-float(t[i]), i) for i in range(n) if labels[i] == c]
+        mem.sort()
+        want += [i for _, i in mem[:rc[c]]]
+    assert got == sorted(want) and not near
+    t2 = np.array([0.5, 0.5, 0.1, 0.9])
+    got2, near2 = O.qgc_select(t2, np.zeros(4, dtype=np.int64), [2])
+    assert got2 == [0, 3] and near2  # 0.5 at index 0 wins the tie; flagged
+    assert O.qgc_read_budget(32768, 0.01, 32) == 279
+    assert O.qgc_read_budget(100, 0.01, 4) == 0
+
 ALL_PINS = [
     pin_dense_bruteforce, pin_summaries_closed_form, pin_exact_mass_bruteforce,
     pin_block_decomposition, pin_discard_error_identity, pin_all_kept_equals_dense,
@@ -1016,5 +1040,5 @@ ALL_PINS = [
     pin_query_basis_closed_form, pin_subspace_rank_by_hand, pin_subspace_factors_exact_in_subspace,
     pin_fp4_e2m1_grid_and_ties, pin_cobs_subspace_logits,
     pin_qgc_kmeans_lloyd_steps, pin_qgc_project_identity, pin_errorgate_closed_form, pin_errorgate_split_by_hand,
-    pin_qgs_scores, pin_qgc_single_cluster_no_reads, pin_qgc_equal_logits_exact,
+    pin_qgs_scores, pin_qgc_single_cluster_no_reads, pin_qgc_equal_logits_exact, pin_qgc_select_and_budget,
 ]
