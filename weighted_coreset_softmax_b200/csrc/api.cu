@@ -551,6 +551,21 @@ kv_status kv_build_block_cov_factors(const kv_shape* shape, const void* K, int r
 }  // extern "C"
 
 namespace {
+// CTAs per pair for the few-pairs selector (0: the one-CTA kernel): the summary and
+// bf16-mean scorers with k_top <= 16, when at least two CTAs per pair fit on the SMs.
+// KVSPARSE_SELECT_SPLIT=0 in the environment (read once) keeps the one-CTA kernel.
+int split_select_ctas(int sel_mode, int k_top, int NBH) {
+  static const bool disabled = [] {
+    const char* v = std::getenv("KVSPARSE_SELECT_SPLIT");
+    return v && v[0] == '0';
+  }();
+  if (disabled || (sel_mode != kvs::SEL_SUMMARY && sel_mode != kvs::SEL_MEAN16) || k_top > kvs::SEL_TOPK || NBH < 1)
+    return 0;
+  const int sms = num_sms_current();
+  const int S = std::min(8, sms / NBH);
+  return S >= 2 ? S : 0;
+}
+
 // Shared by the summary, exact-mass and Quest selections: argument checks and the
 // launch. sel_mode is a kvs::SelMode.
 kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_mode, const float* k_sum,
@@ -630,7 +645,12 @@ kv_status select_any(const kv_shape* shape, const void* q, float scale, int sel_
   p.kmax = kmax;
   p.qscale = scale * 1.4426950408889634f;
   const int G = shape->Hq / shape->Hkv;
-  cudaError_t e = kvs::launch_select(shape->dtype, shape->D, G, sel_mode, p, NBH, reinterpret_cast<cudaStream_t>(stream));
+  // few pairs: split each pair's blocks over a cluster of CTAs
+  const int S = split_select_ctas(sel_mode, k_top, NBH);
+  cudaError_t e = S >= 2 ? kvs::launch_select_split(shape->dtype, shape->D, G, sel_mode, p, NBH, S,
+                                                    reinterpret_cast<cudaStream_t>(stream))
+                         : kvs::launch_select(shape->dtype, shape->D, G, sel_mode, p, NBH,
+                                              reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "select launch");
   return KV_OK;
 }

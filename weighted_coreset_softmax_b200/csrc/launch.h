@@ -28,6 +28,10 @@ cudaError_t launch_fused(int dtype, int D, int G, const AttnParams& p, const CUt
 cudaError_t launch_gather(int D, int G, int rows, const AttnParams& p, const CUtensorMap& tk, const CUtensorMap& tv,
                           int grid, cudaStream_t st);
 cudaError_t launch_select(int dtype, int D, int G, int mode, const SelParams& p, int grid, cudaStream_t st);
+// Few pairs: each pair's blocks over a cluster of S CTAs (summary and bf16-mean modes,
+// k_top <= 16); cudaErrorInvalidValue when the shape is not covered.
+cudaError_t launch_select_split(int dtype, int D, int G, int mode, const SelParams& p, int NBH, int S,
+                                cudaStream_t st);
 cudaError_t launch_sums(int dtype, int D, const void* K, const void* V, const int32_t* seq_lens, float* k_sum,
                         float* v_sum, int32_t* counts, float* k_tot, float* v_tot, int NBH, int Hkv, int Ncap,
                         int L, int NBcap, cudaStream_t st);
