@@ -1095,6 +1095,9 @@ def run_ours(args, dist):
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": NCU_TRAFFIC.get((dom, os.environ.get("KVSPARSE_ATTN", "default"), args.workload,
                                                  args.budget, B)),
+                     "traffic_how": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the current "
+                                    "kernel on a B = 8 capture of this workload, scaled x4 by the pairs processed "
+                                    "(null for shapes without a capture)",
                      "timing": "event pair around each launch, batches rotating (the kernel alone)",
                      "pct_of_8TBs": 100.0 * achieved / NOMINAL_HBM_GBS},
         "roofline_select": sel_roof,
