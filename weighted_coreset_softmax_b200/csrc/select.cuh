@@ -26,6 +26,7 @@
 #include "common.cuh"
 #include "rank.cuh"
 
+#include <cuda_fp16.h>
 #include <cuda_fp4.h>
 
 namespace kvs {
@@ -581,117 +582,179 @@ __device__ void cobs_second_order_ring(const SelParams& p, float* lg, int nbp, i
 }
 
 // Second-order term from the stored descriptor ("COBS: Cumulant Order Block Sparse
-// Attention", the subspace and quantisation paragraphs): adds
-// (sigma^2 / 2) sum_i (q~ . xi_i)^2 to lg, q~ = U q the projected query (qt: the
-// log2-domain q~ of the G heads, [G][SP] in shared memory, zero past s) and
-// xi_i = scale_i * e2m1(codes_i). Each half-warp takes one block at a time: lane c
-// of the half holds nibble columns 8c .. 8c+7 of every factor (one 32-bit word a
-// factor), decodes them with the E2M1 -> f16x2 conversion, forms its partial dots
-// for every (head, factor) pair of a group of FG = 4 factors, and a transpose
-// reduction over the half's 16 lanes sums them (NV - 1 shuffles for NV pairs); the
-// squared dots, times scale_i^2, are summed over the factors through a per-warp
-// scratch (ranks above 4 take a second group). A warp issues the words and scales of
-// NBW block pairs before decoding any of them, so NBW * FG loads a lane are in
-// flight.
+// Attention", the subspace and quantisation paragraphs): adds (sigma^2 / 2)
+// sum_i (q~ . xi_i)^2 to lg, q~ = U q the projected query (qt: the log2-domain q~ of
+// the G heads, [G][SP] in shared memory, zero past s) and xi_i = scale_i *
+// e2m1(codes_i), on the tensor cores (mma.sync m16n8k16, f16 inputs, fp32
+// accumulation). A warp takes 4 blocks at a time: the 16 rows of A are (block j,
+// factor i) = row 4j + i, the K dimension the SP subspace columns (SP / 16 steps); the
+// 8 columns of B are the projected queries split into f16 high and low parts (heads
+// 0..3 high, then low; for G > 4 two column tiles, all high then all low). A thread of
+// the mma layout needs byte tig of every 32-bit word of its two rows (E2M1 codes, 2j in
+// the low nibble): the E2M1 -> f16x2 conversion of that byte is exactly its A register
+// for columns (2 tig, 2 tig + 1), or (+8, +9) for the odd words. E2M1 values are exact
+// in f16, and high + low carries the query to about 22 bits. Epilogue: the high and low
+// columns added (xor 2), squared, times scale^2, summed over the 4 factor rows (xor 4,
+// 8), and (ln 2 / 2) times that added to the block's logits.
+__device__ __forceinline__ void mma_f16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  const __half2_raw h = __nv_cvt_fp4x2_to_halfraw2(static_cast<__nv_fp4x2_storage_t>(byte), __NV_E2M1);
+  return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+__device__ __forceinline__ uint32_t pack_f16x2(float lo_k, float hi_k) {
+  const __half a = __float2half_rn(lo_k), b = __float2half_rn(hi_k);
+  return static_cast<uint32_t>(__half_as_ushort(a)) | (static_cast<uint32_t>(__half_as_ushort(b)) << 16);
+}
+
 template <int G>
-__device__ void cobs_fp4_second_order(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float* qt,
-                                      float* scratch) {
-  constexpr int FG = 4;
-  constexpr int GP = pow2ceil(G);
-  constexpr int NV = GP * FG;                  // 4 .. 32
-  constexpr int NH = NV >= 16 ? NV / 16 : 1;   // values a lane holds after the reduction
-  constexpr int REP = NV >= 16 ? 1 : 16 / NV;  // lanes holding each value (NV < 16)
-  constexpr int NBW = NV <= 16 ? 8 : 4;        // block pairs a warp loads ahead
-  constexpr bool QREG = G <= 4;                // the projected queries in registers (else shared memory)
+__device__ void cobs_fp4_second_order_tc(const SelParams& p, float* lg, int nbp, int bh, int nbv, const float* qt) {
+  constexpr int NT = G <= 4 ? 1 : 2;  // column tiles of B
+  constexpr int KMAX = 8;             // SP <= 128
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int hw = lane >> 4, c = lane & 15;
-  const int r = p.cobs_r, SP = p.SP;
-  const bool active = c < SP / 8;
-  float qv[QREG ? G : 1][8];
-  if constexpr (QREG) {
+  const int grp = lane >> 2, tig = lane & 3;
+  const int r = p.cobs_r, SP = p.SP, KS = SP / 16, WPR = SP / 8;  // k steps, words a row
+  // B fragments: column n = grp of each tile; rows k = 16 ks + 2 tig (+1) and (+8, +9)
+  uint32_t bq[NT][KMAX][2];
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+  for (int t = 0; t < NT; ++t) {
+    // tile t, column grp: head and part
+    int g, part;
+    if constexpr (NT == 1) {
+      g = grp & 3;
+      part = grp >> 2;  // 0 high, 1 low
+    } else {
+      g = grp;
+      part = t;
+    }
 #pragma unroll
-      for (int k = 0; k < 8; ++k) qv[g][k] = active ? qt[g * SP + 8 * c + k] : 0.f;
+    for (int ks = 0; ks < KMAX; ++ks) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        float v[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int k = ks * 16 + tig * 2 + hh * 8 + e;
+          const float x = (ks < KS && g < G) ? qt[g * SP + k] : 0.f;
+          const float hi = __half2float(__float2half_rn(x));
+          v[e] = part == 0 ? hi : x - hi;
+        }
+        bq[t][ks][hh] = pack_f16x2(v[0], v[1]);
+      }
+    }
   }
-  const float* qs = qt + 8 * (active ? c : 0);  // this lane's columns (inactive lanes decode zeros)
-  float* scr = scratch + (warp * 2 + hw) * NV;
-  const size_t fbytes = static_cast<size_t>(SP) / 2;  // bytes a factor
+  const size_t fbytes = static_cast<size_t>(SP) / 2;
   const size_t base = static_cast<size_t>(bh) * p.NBcap * r;
-  for (int f0 = 0; f0 < r; f0 += FG) {
-    for (int b0 = warp * 2 * NBW; b0 < nbv; b0 += SEL_NW * 2 * NBW) {  // warp-uniform
-      uint32_t w[NBW][FG];
-      float sc[NBW][NH];
+  constexpr int U = 2;  // block quads a warp loads before converting any
+  for (int f0 = 0; f0 < r; f0 += 4) {
+    for (int bq0 = warp * 4; bq0 < nbv; bq0 += SEL_NW * 4 * U) {  // warp-uniform
+      // per quad u: this thread's rows grp -> (block + grp / 4, factor f0 + grp % 4),
+      // grp + 8 -> block + 2; whole rows (every thread of a quad loads them, keeping
+      // different bytes)
+      uint32_t w[U][2][12];
+      float sc[U][2];
 #pragma unroll
-      for (int j = 0; j < NBW; ++j) {
-        const int b = b0 + 2 * j + hw;
-        const bool live = b < nbv;
-        const size_t fb = base + static_cast<size_t>(b) * r + f0;
+      for (int u = 0; u < U; ++u) {
+        const int b0 = bq0 + u * SEL_NW * 4;
 #pragma unroll
-        for (int i = 0; i < FG; ++i)
-          w[j][i] = (active && live && f0 + i < r)
-                        ? __ldg(reinterpret_cast<const uint32_t*>(p.xi4 + (fb + i) * fbytes) + c)
-                        : 0u;
+        for (int h2 = 0; h2 < 2; ++h2) {
+          const int rb = b0 + (grp >> 2) + 2 * h2, rf = f0 + (grp & 3);
+          const bool live = rb < nbv && rf < r;
+          const size_t row = base + static_cast<size_t>(rb) * r + rf;
+          const uint4* src = reinterpret_cast<const uint4*>(p.xi4 + row * fbytes);
 #pragma unroll
-        for (int t = 0; t < NH; ++t) {
-          const int idx = NV >= 16 ? c * NH + t : c / REP;
-          const int i = idx - (idx / FG) * FG;
-          sc[j][t] = (live && f0 + i < r) ? __ldg(p.xi4_scale + fb + i) : 0.f;
+          for (int q4 = 0; q4 < 3; ++q4) {
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (live && q4 < WPR / 4) v = __ldg(src + q4);
+            w[u][h2][4 * q4] = v.x;
+            w[u][h2][4 * q4 + 1] = v.y;
+            w[u][h2][4 * q4 + 2] = v.z;
+            w[u][h2][4 * q4 + 3] = v.w;
+          }
+          sc[u][h2] = live ? __ldg(p.xi4_scale + row) : 0.f;
         }
       }
 #pragma unroll
-      for (int j = 0; j < NBW; ++j) {
-        const int b = b0 + 2 * j + hw;
-        float part[NV];
+      for (int u = 0; u < U; ++u) {
+        const int b0 = bq0 + u * SEL_NW * 4;
+        if (b0 >= nbv) break;  // warp-uniform
+        float acc[NT][4];
 #pragma unroll
-        for (int i = 0; i < FG; ++i) {
-          float x[8];
+        for (int t = 0; t < NT; ++t)
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const __half2 h2 = __half2(__nv_cvt_fp4x2_to_halfraw2(
-                static_cast<__nv_fp4x2_storage_t>((w[j][i] >> (8 * k)) & 0xffu), __NV_E2M1));
-            const float2 f2 = __half22float2(h2);
-            x[2 * k] = f2.x;
-            x[2 * k + 1] = f2.y;
+          for (int e = 0; e < 4; ++e) acc[t][e] = 0.f;
+#pragma unroll
+        for (int ks = 0; ks < 6; ++ks) {
+          if (ks < KS) {
+            uint32_t a[4];
+            a[0] = e2m1x2_to_f16x2((w[u][0][2 * ks] >> (8 * tig)) & 0xffu);
+            a[1] = e2m1x2_to_f16x2((w[u][1][2 * ks] >> (8 * tig)) & 0xffu);
+            a[2] = e2m1x2_to_f16x2((w[u][0][2 * ks + 1] >> (8 * tig)) & 0xffu);
+            a[3] = e2m1x2_to_f16x2((w[u][1][2 * ks + 1] >> (8 * tig)) & 0xffu);
+#pragma unroll
+            for (int t = 0; t < NT; ++t) mma_f16_16816(acc[t], a, bq[t][ks][0], bq[t][ks][1]);
+          }
+        }
+        if (KS > 6) {  // SP = 112 or 128: the last words, loaded here
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int rb = b0 + (grp >> 2) + 2 * h2, rf = f0 + (grp & 3);
+            const bool live = rb < nbv && rf < r;
+            const uint4* src =
+                reinterpret_cast<const uint4*>(p.xi4 + (base + static_cast<size_t>(rb) * r + rf) * fbytes);
+            const uint4 v = (live && WPR > 12) ? __ldg(src + 3) : make_uint4(0u, 0u, 0u, 0u);
+            w[u][h2][0] = v.x;
+            w[u][h2][1] = v.y;
+            w[u][h2][2] = v.z;
+            w[u][h2][3] = v.w;
           }
 #pragma unroll
-          for (int g = 0; g < GP; ++g) {
-            float d = 0.f;
-            if (g < G) {
-              if constexpr (QREG) {
+          for (int ks = 6; ks < KMAX; ++ks) {
+            if (ks < KS) {
+              uint32_t a[4];
+              a[0] = e2m1x2_to_f16x2((w[u][0][2 * (ks - 6)] >> (8 * tig)) & 0xffu);
+              a[1] = e2m1x2_to_f16x2((w[u][1][2 * (ks - 6)] >> (8 * tig)) & 0xffu);
+              a[2] = e2m1x2_to_f16x2((w[u][0][2 * (ks - 6) + 1] >> (8 * tig)) & 0xffu);
+              a[3] = e2m1x2_to_f16x2((w[u][1][2 * (ks - 6) + 1] >> (8 * tig)) & 0xffu);
 #pragma unroll
-                for (int k = 0; k < 8; ++k) d = fmaf(qv[g][k], x[k], d);
-              } else {
-                const float4 a = *reinterpret_cast<const float4*>(qs + g * SP);
-                const float4 e = *reinterpret_cast<const float4*>(qs + g * SP + 4);
-                d = fmaf(a.x, x[0], d);
-                d = fmaf(a.y, x[1], d);
-                d = fmaf(a.z, x[2], d);
-                d = fmaf(a.w, x[3], d);
-                d = fmaf(e.x, x[4], d);
-                d = fmaf(e.y, x[5], d);
-                d = fmaf(e.z, x[6], d);
-                d = fmaf(e.w, x[7], d);
-              }
+              for (int t = 0; t < NT; ++t) mma_f16_16816(acc[t], a, bq[t][ks][0], bq[t][ks][1]);
             }
-            part[g * FG + i] = d;
           }
         }
-        transpose_reduce<NV, 8>(part, lane);
-        if (c % REP == 0) {
+        // dots: acc[t][e] is row grp (e < 2) or grp + 8 (e >= 2), column 2 tig + (e & 1)
+        float dot[4];
+        if constexpr (NT == 1) {
 #pragma unroll
-          for (int t = 0; t < NH; ++t) {
-            const int idx = NV >= 16 ? c * NH + t : c / REP;
-            const float sct = sc[j][t];
-            scr[idx] = part[t] * part[t] * sct * sct;  // zero past r, G and the blocks (sc = 0 or part = 0)
+          for (int e = 0; e < 4; ++e) dot[e] = acc[0][e] + __shfl_xor_sync(FULL_MASK, acc[0][e], 2);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dot[e] = acc[0][e] + acc[1][e];
+        }
+        // squares times scale^2, summed over the 4 factor rows (lane bits 2, 3)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float s2 = sc[u][e >> 1] * sc[u][e >> 1];
+          float v = dot[e] * dot[e] * s2;
+          v += __shfl_xor_sync(FULL_MASK, v, 4);
+          v += __shfl_xor_sync(FULL_MASK, v, 8);
+          dot[e] = v;
+        }
+        // lanes with grp % 4 == 0 hold blocks b0 + grp / 4 (e < 2) and + 2 (e >= 2)
+        if ((grp & 3) == 0 && (NT == 2 || tig < 2)) {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int g = 2 * tig + (e & 1);
+            const int blk = b0 + (grp >> 2) + 2 * (e >> 1);
+            if (g < G && blk < nbv) lg[g * nbp + blk] += 0.34657359027997264f * dot[e];  // ln 2 / 2
           }
         }
-        __syncwarp();
-        if (b < nbv && c < G) {
-          const float sum = scr[c * FG] + scr[c * FG + 1] + scr[c * FG + 2] + scr[c * FG + 3];
-          lg[c * nbp + b] += 0.34657359027997264f * sum;  // ln 2 / 2
-        }
-        __syncwarp();
       }
     }
   }
@@ -770,11 +833,10 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
   }
 
   if constexpr (MODE == SEL_COBS4) {
-    // the first-order (bf16-mean) logits are in lg; the projected queries and the
-    // per-warp scratch go where the scorer's ring was
+    // the first-order (bf16-mean) logits are in lg; the projected queries go where the
+    // scorer's ring was
     float* qt = reinterpret_cast<float*>(
         sel_smem + ((sel_smem_bytes(G, p.NBcap) + static_cast<size_t>(nbp) * 4 + 15) & ~static_cast<size_t>(15)));
-    float* scratch = qt + G * p.SP;
     const int h = bh - b * p.Hkv;
     const T* qrow = static_cast<const T*>(p.q) + (static_cast<size_t>(b) * p.Hq + h * G) * D;
     if (p.Uq) {
@@ -786,18 +848,30 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
       for (int g = 0; g < G; ++g)
 #pragma unroll
         for (int k = 0; k < CPL; ++k) qreg[g][k] = load_as_float(qrow + g * D + lane * CPL + k);
-      for (int j = warp; j < p.SP; j += SEL_NW) {
-        float u[CPL];
+      // the warp's basis rows, eight at a time, all eight loaded before the first
+      // reduction, so their latencies overlap
+      constexpr int RB8 = 8;
+      for (int j0 = warp; j0 < p.SP; j0 += RB8 * SEL_NW) {  // warp-uniform
+        float u[RB8][CPL];
 #pragma unroll
-        for (int k = 0; k < CPL; ++k)
-          u[k] = j < p.s_dim ? __ldg(p.Uq + (static_cast<size_t>(h) * p.s_dim + j) * D + lane * CPL + k) : 0.f;
+        for (int jj = 0; jj < RB8; ++jj) {
+          const int j = j0 + jj * SEL_NW;
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
-          float v = 0.f;
+          for (int k = 0; k < CPL; ++k)
+            u[jj][k] = j < p.s_dim ? __ldg(p.Uq + (static_cast<size_t>(h) * p.s_dim + j) * D + lane * CPL + k) : 0.f;
+        }
 #pragma unroll
-          for (int k = 0; k < CPL; ++k) v = fmaf(u[k], qreg[g][k], v);
-          v = warp_sum(v);
-          if (lane == 0) qt[g * p.SP + j] = v * p.qscale;
+        for (int jj = 0; jj < RB8; ++jj) {
+          const int j = j0 + jj * SEL_NW;
+          if (j >= p.SP) break;  // warp-uniform
+#pragma unroll
+          for (int g = 0; g < G; ++g) {
+            float v = 0.f;
+#pragma unroll
+            for (int k = 0; k < CPL; ++k) v = fmaf(u[jj][k], qreg[g][k], v);
+            v = warp_sum(v);
+            if (lane == 0) qt[g * p.SP + j] = v * p.qscale;
+          }
         }
       }
     } else {
@@ -807,7 +881,7 @@ __global__ void __launch_bounds__(SEL_THREADS, 2) select_kernel(const SelParams 
       }
     }
     __syncthreads();
-    cobs_fp4_second_order<G>(p, lg, nbp, bh, nbv, qt, scratch);
+    cobs_fp4_second_order_tc<G>(p, lg, nbp, bh, nbv, qt);  // SP <= D <= 128
     __syncthreads();
   }
 
