@@ -512,6 +512,33 @@ struct GaMerge {
       fold(g, m, l, x);
     }
   }
+  // Folds records of other CTAs (global memory, read through L2), NB at a time: every
+  // record's loads of a batch are issued before the first fold, so their latencies
+  // overlap.
+  template <int NB>
+  __device__ __forceinline__ void fold_records_global(const float* const (&rec)[NB], int n, int lane) {
+    float x[NB][G][VEC], m[NB][G], l[NB][G];
+#pragma unroll
+    for (int t = 0; t < NB; ++t) {
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        if (t < n) {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) x[t][g][v] = __ldcg(rec[t] + g * D + lane * VEC + v);
+          m[t][g] = __ldcg(rec[t] + G * D + g);
+          l[t][g] = __ldcg(rec[t] + G * D + G + g);
+        } else {
+          m[t][g] = -INFINITY;
+          l[t][g] = 0.f;
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < NB; ++t)
+#pragma unroll
+      for (int g = 0; g < G; ++g)
+        if (t < n) fold(g, m[t][g], l[t][g], x[t][g]);
+  }
   // Folds up to N records of shared memory at once (rec[t] for t < n): the
   // maxima and sums first, then each lane's channels with 16-byte loads.
   template <int N>
@@ -905,10 +932,17 @@ __global__ void __launch_bounds__(GA_THREADS, 1)
       if (!last) return;
       __threadfence();
       mg.reset();
-      for (int c = cf; c <= cl; ++c) {
-        const int64_t cx0 = ga_x0(T, c, ncta, PC, NBH);
-        const int cside = (static_cast<int64_t>(bh) == cx0 / PC) ? 0 : 1;
-        mg.fold_record(p.recs + static_cast<size_t>(2 * c + cside) * C::RECF, lane, true);
+      constexpr int NBR = G <= 4 ? 4 : 2;  // records whose loads are in flight together
+      for (int c0 = cf; c0 <= cl; c0 += NBR) {
+        const float* recs[NBR];
+#pragma unroll
+        for (int t = 0; t < NBR; ++t) {
+          const int c = min(c0 + t, cl);
+          const int64_t cx0 = ga_x0(T, c, ncta, PC, NBH);
+          const int cside = (static_cast<int64_t>(bh) == cx0 / PC) ? 0 : 1;
+          recs[t] = p.recs + static_cast<size_t>(2 * c + cside) * C::RECF;
+        }
+        mg.template fold_records_global<NBR>(recs, min(NBR, cl - c0 + 1), lane);
       }
       mg.write_out(p, bh, lane);
     };
