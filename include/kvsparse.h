@@ -203,7 +203,8 @@ kv_status kv_select_blocks_mean16(const kv_shape* shape, const void* q, float sc
  *            attention leaves out)
  *   workspace  device, kv_wildcat_workspace_bytes(shape, m) bytes, 16-byte aligned
  *            (per (sequence, KV head): the factor and the residual diagonal, m + 1
- *            rows of Ncap floats, and 8 x m partial column sums)
+ *            rows of Ncap floats with Ncap rounded up to a multiple of 32, and 8 x m
+ *            partial column sums)
  * The cluster of a pair runs the m pivot steps (each a draw from the residual
  * diagonal and one pass over the keys for a residual kernel column); run once after
  * prefill. Bytes per pair and step: the n keys plus t + 1 factor rows of n floats.

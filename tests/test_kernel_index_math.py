@@ -176,3 +176,65 @@ def test_cov_smem_layout(L, D):
     assert o["rot"] % 16 == 0, "double2 rotations need 16-byte alignment"
     assert o["end"] <= o["total"], "carve-up runs past the allocation"
     assert o["total"] <= 227 * 1024
+
+
+# ------------------------------------------------------------ WildCat producer
+def wc_fidx(j, i, m):
+    """Tiled factor index: F[j][i] at (i / 32) * 32 m + 32 j + i % 32."""
+    return (i >> 5) * (32 * m) + 32 * j + (i & 31)
+
+
+@pytest.mark.parametrize("Ncap,m", [(1, 1), (31, 3), (32, 4), (33, 5), (100, 7), (1000, 64)])
+def test_wildcat_factor_tiles_bijective(Ncap, m):
+    # every (row j < m, token i < Ncap rounded up to 32) has its own slot inside the
+    # m rows of the factor, ahead of the residual diagonal and the column sums
+    n32 = (Ncap + 31) & ~31
+    idx = {wc_fidx(j, i, m) for j in range(m) for i in range(n32)}
+    assert len(idx) == m * n32 and min(idx) == 0 and max(idx) == m * n32 - 1
+    # a batch's t rows are one contiguous run of 32 t floats
+    for t in (1, m):
+        run = sorted(wc_fidx(j, 32 + lane, m) for j in range(t) for lane in range(32)) if n32 > 32 else []
+        if run:
+            assert run == list(range(run[0], run[0] + 32 * t))
+    # per-pair stride and the workspace bytes of the C entry
+    per_pair = (m + 1) * n32 + 8 * m
+    assert m * n32 + n32 + 8 * m == per_pair
+
+
+def transpose_reduce(vals, N, MASK):
+    """Restatement of transpose_reduce<N, MASK> over 32 lanes (vals[lane][k])."""
+    v = [list(x) for x in vals]
+    while MASK >= 1:
+        if N > 1:
+            nv = []
+            for lane in range(32):
+                up = (lane & MASK) != 0
+                other = lane ^ MASK
+                row = []
+                for j in range(N // 2):
+                    keep = v[lane][j + N // 2] if up else v[lane][j]
+                    up_o = (other & MASK) != 0
+                    send_o = v[other][j] if up_o else v[other][j + N // 2]
+                    row.append(keep + send_o)
+                nv.append(row)
+            v, N = nv, N // 2
+        else:
+            v = [[v[lane][0] + v[lane ^ MASK][0]] for lane in range(32)]
+        MASK //= 2
+    return [x[0] for x in v]
+
+
+@pytest.mark.parametrize("esize,D", [(2, 128), (2, 64), (4, 128), (4, 64)])
+def test_wildcat_lane_layout_covers_rows(esize, D):
+    che = 16 // esize
+    cpl = D // che // 8
+    assert cpl * che * 8 == D
+    # the 8 lanes of a group read the 16-byte chunks c + 8 kk of a row: each once
+    chunks = sorted(c + 8 * kk for c in range(8) for kk in range(cpl))
+    assert chunks == list(range(D // che))
+    # lane l's partial for row 8 (l / 8) + k is v[k]; after the 8-value transpose
+    # reduction lane l holds the sum over its group of v[l % 8]: row l's dot product
+    part = [[1000.0 * (8 * (lane >> 3) + k) + (lane & 7) for k in range(8)] for lane in range(32)]
+    out = transpose_reduce(part, 8, 4)
+    for lane in range(32):
+        assert out[lane] == 8 * 1000.0 * lane + sum(range(8))

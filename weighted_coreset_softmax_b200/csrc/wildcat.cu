@@ -25,11 +25,12 @@
 //      g_i = exp(scale k_i.k_s - shift) - sum_{j<t} F[j][i] F[j][s], the factor
 //      column F[t][i] = g_i / sqrt(g_s), d_i -= F[t][i]^2 (0 at the pivot), the new
 //      group sums of d for the next draw, and the column's sum.
-// The key dot products are warp-cooperative: every lane holds D/32 of the pivot's
-// key, a warp loads one whole row per instruction (coalesced) for 32 rows, and a
-// transpose reduction leaves row r's dot product in lane r, which owns token r for
-// the coalesced factor, d and output traffic. The factor lives in the workspace as
-// F[t][i] (token index fastest). With the pivots' rows F_S (lower triangular in
+// The key dot products are warp-cooperative: 8 lanes share a row, each holding 1/8 of
+// the pivot's key in 16-byte chunks, a warp load covers 4 rows, and a transpose
+// reduction over the 8 lanes leaves row r's dot product in lane r, which owns token r
+// for the coalesced factor, d and output traffic. The factor lives in the workspace
+// as F[t][i] in tiles of 32 tokens (each batch's factor rows contiguous). With the
+// pivots' rows F_S (lower triangular in
 // pivot order), A_SS = F_S F_S^T and A_{S,:} = F_S F^T exactly, so
 // w = F_S^-T (F^T 1): CTA 0 adds the C partial column sums in rank order and runs
 // one back substitution. Bytes per pair and step: the n keys, t factor rows read
@@ -55,82 +56,76 @@ constexpr int WC_MAX_M = 4096;
 constexpr int WC_MAX_C = 8;
 constexpr int WC_MAX_NCAP = 1 << 20;
 
-// A lane's slice of a key row (D/32 elements) as loaded, and its fp32 values.
-template <typename T, int E>
-struct WcRaw;
-template <>
-struct WcRaw<__nv_bfloat16, 2> {
-  using type = unsigned int;
-  __device__ __forceinline__ static void unpack(type r, float (&x)[2]) {
-    x[0] = __uint_as_float(r << 16);
-    x[1] = __uint_as_float(r & 0xffff0000u);
-  }
-};
-template <>
-struct WcRaw<__nv_bfloat16, 4> {
-  using type = uint2;
-  __device__ __forceinline__ static void unpack(type r, float (&x)[4]) {
-    x[0] = __uint_as_float(r.x << 16);
-    x[1] = __uint_as_float(r.x & 0xffff0000u);
-    x[2] = __uint_as_float(r.y << 16);
-    x[3] = __uint_as_float(r.y & 0xffff0000u);
-  }
-};
-template <>
-struct WcRaw<float, 2> {
-  using type = float2;
-  __device__ __forceinline__ static void unpack(type r, float (&x)[2]) {
-    x[0] = r.x;
-    x[1] = r.y;
-  }
-};
-template <>
-struct WcRaw<float, 4> {
-  using type = float4;
-  __device__ __forceinline__ static void unpack(type r, float (&x)[4]) {
-    x[0] = r.x;
-    x[1] = r.y;
-    x[2] = r.z;
-    x[3] = r.w;
-  }
-};
+// The factor matrix is stored in tiles of 32 tokens: F[j][i] at
+// (i / 32) * 32 m + 32 j + i % 32, so that the t factor rows a warp reads for one
+// batch of 32 tokens are one contiguous t * 128-byte run and the factor column it
+// writes is one 128-byte piece.
+__device__ __forceinline__ size_t wc_fidx(int j, int i, int m) {
+  return static_cast<size_t>(i >> 5) * (32 * static_cast<size_t>(m)) + 32 * j + (i & 31);
+}
 
+// Lane layout of the key-row dot products: 8 lanes a row, lane c (= lane % 8) of a
+// group holding the 16-byte chunks c, c + 8, ... of the row (so a warp load reads 4
+// rows as 4 contiguous 128-byte pieces); group gq (= lane / 8) takes the rows
+// i0 + 8 gq + k, k < 8, so that an 8-value transpose reduction over the group leaves
+// row i0 + lane's dot product in lane `lane`.
 template <typename T, int D>
-struct WcRow {
-  static constexpr int E = D / 32;
-  using R = WcRaw<T, E>;
-  using raw = typename R::type;
-  // rows whose slices are loaded before any is used (64 registers of loads)
-  static constexpr int RB = sizeof(raw) >= 16 ? 16 : 32;
-  __device__ __forceinline__ static raw load(const T* row, int lane) {
-    return __ldcs(reinterpret_cast<const raw*>(row) + lane);  // keys stream: evict first
-  }
+struct WcLay {
+  static constexpr int CHE = 16 / static_cast<int>(sizeof(T));  // elements a chunk
+  static constexpr int CPL = D / CHE / 8;                        // chunks a lane (1, 2 or 4)
+  static constexpr int EPL = CPL * CHE;                          // elements a lane (8 or 16)
+  static constexpr int RBK = CPL * 4 * 8 > 64 ? 4 : 8;          // rows loaded at once (64 registers)
+  static constexpr bool R64 = CPL == 2 && CHE == 8;              // factor rounds of 64 rows fit (16-bit, D = 128)
 };
 
-// Dot products of the 32 key rows i0 .. i0+31 with the lane-split vector ks
-// (SELF: each row with itself); lane j returns row i0+j's. Rows at or past n
-// read row n-1 (in bounds) and their results are ignored by the caller.
+// This lane's elements of one row (the pivot's key), as fp32 pairs.
+template <typename T, int D>
+__device__ __forceinline__ void wc_slice2(const T* row, int lane, float2 (&x)[WcLay<T, D>::EPL / 2]) {
+  using Ly = WcLay<T, D>;
+  const int c = lane & 7;
+#pragma unroll
+  for (int kk = 0; kk < Ly::CPL; ++kk) {
+    const uint4 r = __ldg(reinterpret_cast<const uint4*>(row) + c + 8 * kk);
+    float2 f[Ly::CHE / 2];
+    Chunk<T>::unpack(r, f);
+#pragma unroll
+    for (int e = 0; e < Ly::CHE / 2; ++e) x[kk * (Ly::CHE / 2) + e] = f[e];
+  }
+}
+
+// Dot products of the 32 key rows i0 .. i0+31 with the lane-split vector ks (SELF:
+// each row with itself); lane j returns row i0+j's. Rows at or past n read row n-1
+// (in bounds) and their results are ignored by the caller.
 template <typename T, int D, bool SELF>
-__device__ __forceinline__ float wc_dots(const T* Kb, int i0, int n, const float (&ks)[D / 32], int lane) {
-  using W = WcRow<T, D>;
-  constexpr int E = W::E, RB = W::RB;
-  float v[32];
+__device__ __forceinline__ float wc_dots(const T* Kb, int i0, int n, const float2 (&ks)[WcLay<T, D>::EPL / 2],
+                                         int lane) {
+  using Ly = WcLay<T, D>;
+  const int gq = lane >> 3, c = lane & 7;
+  float v[8];
 #pragma unroll
-  for (int r0 = 0; r0 < 32; r0 += RB) {
-    typename W::raw raw[RB];
+  for (int k0 = 0; k0 < 8; k0 += Ly::RBK) {
+    uint4 raw[Ly::RBK][Ly::CPL];
 #pragma unroll
-    for (int r = 0; r < RB; ++r) raw[r] = W::load(Kb + static_cast<size_t>(min(i0 + r0 + r, n - 1)) * D, lane);
+    for (int k = 0; k < Ly::RBK; ++k) {
+      const int row = min(i0 + 8 * gq + k0 + k, n - 1);
 #pragma unroll
-    for (int r = 0; r < RB; ++r) {
-      float x[E];
-      W::R::unpack(raw[r], x);
-      float a = 0.f;
+      for (int kk = 0; kk < Ly::CPL; ++kk)
+        raw[k][kk] = __ldcs(reinterpret_cast<const uint4*>(Kb + static_cast<size_t>(row) * D) + c + 8 * kk);
+    }
 #pragma unroll
-      for (int e = 0; e < E; ++e) a = fmaf(x[e], SELF ? x[e] : ks[e], a);
-      v[r0 + r] = a;
+    for (int k = 0; k < Ly::RBK; ++k) {
+      float2 a = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int kk = 0; kk < Ly::CPL; ++kk) {
+        float2 f[Ly::CHE / 2];
+        Chunk<T>::unpack(raw[k][kk], f);
+#pragma unroll
+        for (int e = 0; e < Ly::CHE / 2; ++e) a = ffma2(f[e], SELF ? f[e] : ks[kk * (Ly::CHE / 2) + e], a);
+      }
+      v[k0 + k] = a.x + a.y;
     }
   }
-  transpose_reduce<32, 16>(v, lane);
+  transpose_reduce<8, 4>(v, lane);
   return v[0];
 }
 
@@ -138,23 +133,64 @@ __device__ __forceinline__ float wc_dots(const T* Kb, int i0, int n, const float
 // factor rows so far times fs (fs[j] = F[j][s]). The factor is read through L2
 // (it is written by every CTA of the cluster).
 template <typename T, int D>
-__device__ __forceinline__ float wc_column(const T* Kb, int i0, int n, const float (&ks)[D / 32], const float* F,
-                                           int Ncap, const float* fs, int t, float scale, float sM, int lane) {
+__device__ __forceinline__ float wc_column(const T* Kb, int i0, int n, const float2 (&ks)[WcLay<T, D>::EPL / 2],
+                                           const float* F, int m, const float* fs, int t, float scale, float sM,
+                                           int lane) {
+  // the first FP factor rows are requested before the key rows, so that both
+  // round trips overlap (none where the key rows already take 64 registers at 4
+  // rows a batch). The rest go in unpredicated rounds of 64 rows (16-bit keys,
+  // D = 128) or 32 (the key rows' registers are free by then), all loads of a round
+  // issued before the first use, and a predicated tail of fewer than 32 rows (rows
+  // past t load nothing and add nothing). The sum runs in row order whatever the
+  // rounds.
+  constexpr int FP = WcLay<T, D>::RBK == 4 ? 0 : 16;
+  const int i = i0 + lane;
+  const float* Fi = F + wc_fidx(0, min(i, n - 1), m);
+  float f0[FP > 0 ? FP : 1];
+#pragma unroll
+  for (int k = 0; k < FP; ++k) f0[k] = k < t ? __ldcg(Fi + 32 * k) : 0.f;
   const float dot = wc_dots<T, D, false>(Kb, i0, n, ks, lane);
   float g = __expf(scale * dot - sM);
-  const int i = i0 + lane;
-  if (i < n) {
-    // 32 factor rows per batch, all loads issued before the first use (one
-    // round trip per 32 rows); rows past t load nothing and add nothing
-    const float* Fi = F + i;
-    for (int j0 = 0; j0 < t; j0 += 32) {
-      float f[32];
 #pragma unroll
-      for (int k = 0; k < 32; ++k) f[k] = j0 + k < t ? __ldcg(Fi + static_cast<size_t>(j0 + k) * Ncap) : 0.f;
+  for (int k = 0; k < FP; ++k)
+    if (k < t) g = fmaf(-f0[k], fs[k], g);
+  int j = FP;  // a multiple of 4: fs + j is 16-byte aligned
+  for (; WcLay<T, D>::R64 && j + 64 <= t; j += 64) {
+    const float* Fj = Fi + 32 * j;
+    float f[64];
 #pragma unroll
-      for (int k = 0; k < 32; ++k)
-        if (j0 + k < t) g = fmaf(-f[k], fs[j0 + k], g);
+    for (int k = 0; k < 64; ++k) f[k] = __ldcg(Fj + 32 * k);
+#pragma unroll
+    for (int k = 0; k < 64; k += 4) {
+      const float4 c = *reinterpret_cast<const float4*>(fs + j + k);
+      g = fmaf(-f[k], c.x, g);
+      g = fmaf(-f[k + 1], c.y, g);
+      g = fmaf(-f[k + 2], c.z, g);
+      g = fmaf(-f[k + 3], c.w, g);
     }
+  }
+  for (; j + 32 <= t; j += 32) {
+    const float* Fj = Fi + 32 * j;
+    float f[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) f[k] = __ldcg(Fj + 32 * k);
+#pragma unroll
+    for (int k = 0; k < 32; k += 4) {
+      const float4 c = *reinterpret_cast<const float4*>(fs + j + k);
+      g = fmaf(-f[k], c.x, g);
+      g = fmaf(-f[k + 1], c.y, g);
+      g = fmaf(-f[k + 2], c.z, g);
+      g = fmaf(-f[k + 3], c.w, g);
+    }
+  }
+  if (j < t) {
+    const float* Fj = Fi + 32 * j;
+    float f[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) f[k] = j + k < t ? __ldcg(Fj + 32 * k) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k)
+      if (j + k < t) g = fmaf(-f[k], fs[j + k], g);
   }
   return g;
 }
@@ -191,7 +227,7 @@ __device__ __forceinline__ float wc_sum(float v, float* wsum) {
   return total;
 }
 
-struct WcShared {
+struct alignas(16) WcShared {
   float fs[WC_MAX_M];     // F[j][s] of the current pivot, j < t; at the end the weights
   int piv_list[WC_MAX_M];  // the pivots in the order drawn
   float wsum[WC_NW];
@@ -206,7 +242,7 @@ template <typename T, int D>
 __global__ void __launch_bounds__(WC_THREADS, 1)
     wildcat_kernel(const T* __restrict__ K, const int32_t* seq_lens, int Hkv, int Ncap, int m, float scale,
                    const float* __restrict__ u, int32_t* tok_idx, float* w, int32_t* n_sel, float* ws) {
-  constexpr int E = D / 32;
+  constexpr int E2 = WcLay<T, D>::EPL / 2;
   __shared__ WcShared sh;
   extern __shared__ float gsum[];  // this CTA's group sums of d
   cg::cluster_group cluster = cg::this_cluster();
@@ -216,16 +252,17 @@ __global__ void __launch_bounds__(WC_THREADS, 1)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int n = max(0, min(seq_lens[b], Ncap));
   const T* Kb = K + static_cast<size_t>(bh) * Ncap * D;
-  const size_t stride = (static_cast<size_t>(m) + 1) * Ncap + static_cast<size_t>(WC_MAX_C) * m;
-  float* F = ws + static_cast<size_t>(bh) * stride;  // F[t][i], t < m
-  float* d = F + static_cast<size_t>(m) * Ncap;      // residual diagonal
-  float* cs = d + Ncap;                              // column sums [C][m]
+  const size_t n32 = static_cast<size_t>((Ncap + 31) & ~31);
+  const size_t stride = (static_cast<size_t>(m) + 1) * n32 + static_cast<size_t>(WC_MAX_C) * m;
+  float* F = ws + static_cast<size_t>(bh) * stride;  // F[t][i], t < m, tiled by wc_fidx
+  float* d = F + static_cast<size_t>(m) * n32;       // residual diagonal
+  float* cs = d + n32;                               // column sums [C][m]
   const float* ub = u + static_cast<size_t>(bh) * m;
   const int ngrp = (n + 31) / 32;
   const int g_beg = static_cast<int>(static_cast<long long>(ngrp) * rank / C);
   const int g_end = static_cast<int>(static_cast<long long>(ngrp) * (rank + 1) / C);
   const int ng = g_end - g_beg;
-  const float no_vec[E] = {};
+  const float2 no_vec[E2] = {};
 
   // ---- the shift M = max_i |k_i|^2 over the pair; d_i = exp(scale |k_i|^2 - scale M)
   float mx = 0.f;
@@ -355,14 +392,14 @@ __global__ void __launch_bounds__(WC_THREADS, 1)
     if (s < 0 || s >= n) break;  // (no positive entry in the drawn group: not reached for finite keys)
 
     // ---- 2. the pivot's key slice, its factor row, and the residual at the pivot
-    float ks[E];
-    WcRow<T, D>::R::unpack(WcRow<T, D>::load(Kb + static_cast<size_t>(s) * D, lane), ks);
-    for (int j = tid; j < t; j += WC_THREADS) sh.fs[j] = __ldcg(F + static_cast<size_t>(j) * Ncap + s);
+    float2 ks[E2];
+    wc_slice2<T, D>(Kb + static_cast<size_t>(s) * D, lane, ks);
+    for (int j = tid; j < t; j += WC_THREADS) sh.fs[j] = __ldcg(F + wc_fidx(j, s, m));
     if (tid == 0) sh.piv_list[t] = s;
     __syncthreads();
     if (warp == 0) {
       // the same computation as the pivot's lane in the column pass, so bit-identical
-      const float g = wc_column<T, D>(Kb, s & ~31, n, ks, F, Ncap, sh.fs, t, scale, sM, lane);
+      const float g = wc_column<T, D>(Kb, s & ~31, n, ks, F, m, sh.fs, t, scale, sM, lane);
       const float gs = __shfl_sync(FULL_MASK, g, s & 31);
       if (lane == 0) sh.gpiv = gs;
     }
@@ -373,15 +410,14 @@ __global__ void __launch_bounds__(WC_THREADS, 1)
 
     // ---- 3. the fused pass: factor column t, the downdate of d, group sums, column sum
     float csum = 0.f;
-    float* Ft = F + static_cast<size_t>(t) * Ncap;
     for (int g = g_beg + warp; g < g_end; g += WC_NW) {
       const int i = g * 32 + lane;
       const float di = i < n ? d[i] : 0.f;  // issued ahead of the column's loads
-      const float gi = wc_column<T, D>(Kb, g * 32, n, ks, F, Ncap, sh.fs, t, scale, sM, lane);
+      const float gi = wc_column<T, D>(Kb, g * 32, n, ks, F, m, sh.fs, t, scale, sM, lane);
       float dn = 0.f;
       if (i < n) {
         const float f = gi * inv;
-        Ft[i] = f;
+        F[wc_fidx(t, i, m)] = f;
         dn = i == s ? 0.f : fmaxf(di - f * f, 0.f);
         d[i] = dn;
         csum += f;
@@ -411,11 +447,10 @@ __global__ void __launch_bounds__(WC_THREADS, 1)
   if (warp == 0) {
     for (int c = taken - 1; c >= 0; --c) {
       // w_c = (rhs_c - sum_{r > c} F_S[r][c] w_r) / F_S[c][c]
-      const float* Fc = F + static_cast<size_t>(c) * Ncap;
       float acc = 0.f;
-      for (int r = c + 1 + lane; r < taken; r += 32) acc = fmaf(__ldcg(Fc + sh.piv_list[r]), sh.fs[r], acc);
+      for (int r = c + 1 + lane; r < taken; r += 32) acc = fmaf(__ldcg(F + wc_fidx(c, sh.piv_list[r], m)), sh.fs[r], acc);
       acc = warp_sum(acc);
-      if (lane == 0) sh.fs[c] = (sh.fs[c] - acc) / __ldcg(Fc + sh.piv_list[c]);
+      if (lane == 0) sh.fs[c] = (sh.fs[c] - acc) / __ldcg(F + wc_fidx(c, sh.piv_list[c], m));
       __syncwarp();
     }
   }
@@ -459,7 +494,8 @@ static cudaError_t wildcat_launch(const kv_shape* s, const void* K, float scale,
 
 extern "C" size_t kv_wildcat_workspace_bytes(const kv_shape* shape, int m) {
   if (!shape || m < 1 || shape->B < 0 || shape->Hkv < 1 || shape->Ncap < 1) return 0;
-  const size_t per_pair = (static_cast<size_t>(m) + 1) * shape->Ncap + static_cast<size_t>(kvs::WC_MAX_C) * m;
+  const size_t n32 = static_cast<size_t>((shape->Ncap + 31) & ~31);
+  const size_t per_pair = (static_cast<size_t>(m) + 1) * n32 + static_cast<size_t>(kvs::WC_MAX_C) * m;
   return static_cast<size_t>(shape->B) * shape->Hkv * per_pair * sizeof(float);
 }
 
