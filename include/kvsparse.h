@@ -388,7 +388,9 @@ kv_status kv_select_blocks_cobs_fp4(const kv_shape* shape, const void* q, float 
  *   P        device [Hkv][16][D] fp32: the projection rows (the 16 leading rows of
  *            kv_build_query_basis's evecs per head)
  *   C        clusters, 1..64 (min(C, seq_len) are used); iters: Lloyd iterations, 1..100
- *   z16      device out [B][Hkv][Ncap][16] bf16: P k per token (fp32, then bf16)
+ *   z16      device out [B][Hkv][Ncap][16] bf16: P k (fp32, then bf16) in member
+ *            order: entry m is the projection of token perm[m] (zero past seq_len),
+ *            so every cluster's projections are one contiguous run
  *   labels   device out [B][Hkv][Ncap] int32: cluster of each token (-1 past seq_len)
  *   perm     device out [B][Hkv][Ncap] int32: the tokens grouped by cluster, ascending
  *            inside a cluster (-1 past seq_len); offs: [B][Hkv][C + 1] int32 starts

@@ -43,7 +43,8 @@ def _check_build(wl, g, P, pairs, C, iters, what):
         n = wl.seq_lens[b]
         Z32 = O.qgc_project(K64[b, h], n, P64)
         zo = O.round_bf16(Z32.astype(np.float64))
-        bad = int(np.sum(z16[b, h, :n] != zo))
+        # z16 is in member order: entry m is token perm[m]'s projection
+        bad = int(np.sum(z16[b, h, :n] != zo[perm[b, h, :n]]))
         assert bad <= max(1, n * 16 // 10000), f"{what}: {bad} bf16 coordinates differ at {(b, h)}"
         assert not np.any(z16[b, h, n:])
         lo, cent = O.qgc_kmeans(Z32, C, iters)

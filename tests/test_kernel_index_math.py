@@ -238,3 +238,72 @@ def test_wildcat_lane_layout_covers_rows(esize, D):
     out = transpose_reduce(part, 8, 4)
     for lane in range(32):
         assert out[lane] == 8 * 1000.0 * lane + sum(range(8))
+
+
+# ------------------------------------------------------------ QGC radix selection
+def kth_largest_radix(keys, rc):
+    """Restatement of qg_kth_largest: radix selection on 8-bit digits below the bits
+    all keys share, then a direct ranking of at most 32 candidates."""
+    M = (1 << 64) - 1
+    a, o = M, 0
+    for x in keys:
+        a &= x
+        o |= x
+    hb = (a ^ o).bit_length() - 1
+    assert hb >= 0
+    pmask = 0 if hb == 63 else (~((2 << hb) - 1)) & M
+    prefix = a & pmask
+    need = rc
+    top = hb
+    while True:
+        lo = top - 7
+        dmask = (255 << lo) if lo >= 0 else (255 >> (-lo))
+        hist = [0] * 256
+        for x in keys:
+            if x & pmask == prefix:
+                hist[((x >> lo) if lo >= 0 else (x << (-lo))) & 255] += 1
+        # lanes hold bins 255 - 8 L - j: a descending walk over the digits
+        acc = 0
+        for dig in range(255, -1, -1):
+            if acc + hist[dig] >= need:
+                above, cdig = acc, hist[dig]
+                break
+            acc += hist[dig]
+        need -= above
+        prefix |= (dig << lo) if lo >= 0 else (dig >> (-lo))
+        pmask |= dmask
+        if cdig <= 32:
+            break
+        top -= 8
+    cand = [x for x in keys if x & pmask == prefix]
+    assert len(cand) <= 32
+    win = [x for x in cand if sum(y > x for y in cand) == need - 1]
+    assert len(win) == 1
+    return win[0]
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_qgc_radix_selection_matches_sort(seed):
+    import random
+    import struct
+    rng = random.Random(seed)
+    for trial in range(16):
+        nc = rng.choice([2, 3, 17, 33, 100, 1000, 3000])
+        kind = trial % 4
+        m0 = rng.randrange(0, 1 << 20)
+        keys = []
+        for m in range(m0, m0 + nc):
+            if kind == 0:
+                t = rng.random() * 1e-3
+            elif kind == 1:
+                t = 0.0 if rng.random() < 0.7 else rng.random()  # many equal scores
+            elif kind == 2:
+                t = 10 ** rng.uniform(-30, 0)
+            else:
+                t = 0.25  # all equal: order by member position alone
+            tb = struct.unpack("<I", struct.pack("<f", t))[0]
+            keys.append((tb << 32) | (0xFFFFFFFF - m))
+        for rc in {1, 2, nc // 2 or 1, nc - 1, min(28, nc - 1)}:
+            if not 1 <= rc < nc:
+                continue
+            assert kth_largest_radix(keys, rc) == sorted(keys, reverse=True)[rc - 1]

@@ -9,22 +9,24 @@
 // the weights it hides).
 //
 // kv_build_qgc (once after prefill, one CTA per (sequence, KV head)):
-//   z = P k for every token (float64 dot products, stored at fp32 in the scratch and
-//   at bf16 for the per-query scan); Lloyd k-means on z in float64 (starts at the
+//   z = P k for every token (float64 dot products, stored at fp32 in the scratch);
+//   Lloyd k-means on z in float64 (starts at the
 //   tokens ((2c + 1) n) // (2C'), C' = min(C, n); distance summed over the 16
 //   coordinates in order as separately rounded products and sums; ties to the lower
 //   cluster; the labels of the last assignment are the clusters; centroid sums per
 //   warp over contiguous token ranges, added in warp order); the members of every
 //   cluster in ascending token order (a stable counting sort: ranks inside 32-token
 //   chunks from match-any masks); per cluster the count, key sum, value sum and
-//   per-channel key sum of squares, accumulated in float64 in member order.
+//   per-channel key sum of squares, accumulated in float64 in member order; z at
+//   bf16 in member order for the per-query scan (each cluster one contiguous run).
 // kv_select_qgc (per query, one CTA per pair):
 //   per cluster mu_g = sigma q_g . mean, s2_g = sigma^2 sum_d q_gd^2 var_d, the error
 //   E_c = sum_g n_c e^(mu - M_g) expm1(s2 / 2) / Zhat_g, Zhat_g = sum_c n_c e^(mu + s2/2 - M_g);
 //   the read budget R = floor(budget n) - ceil(1.5 C_live) and r_c = min(n_c,
 //   floor(R E_c / sum E)); token scores t_i = sum_g exp(sigma (P q_g) . z16_i - LSE_g)
-//   in two passes; in every cluster the r_c tokens of largest (t, then lower index)
-//   found by bisection on the 64-bit key (t's bits, inverted index); the read list
+//   in two passes over the members on the tensor cores; in every cluster the r_c
+//   tokens of largest (t, then lower index), from its contiguous run of scores, by
+//   repeated maxima or bisection on the 64-bit key (t's bits, inverted position); the read list
 //   with weight 1 (padding weight 0) for kv_sparse_decode_attn's weighted mode; and
 //   per cluster the proxy of its unread tokens (cluster sums minus the read rows,
 //   over their count).
@@ -36,6 +38,7 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <type_traits>
 
 #include "common.cuh"
 #include "kvsparse.h"
@@ -47,7 +50,14 @@ constexpr int QG_THREADS = 512;
 constexpr int QG_NW = QG_THREADS / 32;
 constexpr int QG_DIM = 16;     // projection dimension
 constexpr int QG_MAX_C = 64;   // clusters per (sequence, KV head)
-constexpr int QG_TCAP = 49152;  // token scores kept in shared memory (longer sequences use the scratch)
+constexpr int QG_STAGES = 3;          // ring stages a warp
+constexpr int QG_CHUNK = 4096;        // ring stage bytes: 128 tokens' bf16 projections
+constexpr int QG_CHUNK_TOK = QG_CHUNK / (QG_DIM * 2);
+// The per-query selection runs 256 threads a CTA, two CTAs an SM: while one CTA of an
+// SM streams its projections, the other can run its cluster phase.
+constexpr int QS_THREADS = 256;
+constexpr int QS_NW = QS_THREADS / 32;
+constexpr int QG_RING = QS_NW * QG_STAGES * QG_CHUNK;  // dynamic shared memory of the selection (96 KB)
 
 __host__ __device__ inline size_t qgc_build_smem_bytes(int D, int C) {
   return static_cast<size_t>(QG_DIM) * D * 4 +                 // P rows
@@ -87,10 +97,9 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_build_kernel(const T* __restri
   for (int e = tid; e < QG_DIM * D; e += QG_THREADS) Ps[e] = P[static_cast<size_t>(h) * QG_DIM * D + e];
   __syncthreads();
 
-  // ---- 1. projection z = P k (float64), stored at fp32 (scratch) and bf16 (output)
+  // ---- 1. projection z = P k (float64), stored at fp32 (scratch)
   constexpr int CH = 16 / sizeof(T);
   for (int i = tid; i < Ncap; i += QG_THREADS) {
-    __nv_bfloat16* zo = z16 + (tok0 + i) * QG_DIM;
     if (i < n) {
       double a[QG_DIM];
 #pragma unroll
@@ -111,14 +120,8 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_build_kernel(const T* __restri
         }
       }
 #pragma unroll
-      for (int j = 0; j < QG_DIM; ++j) {
-        const float zf = static_cast<float>(a[j]);
-        Z[static_cast<size_t>(i) * QG_DIM + j] = zf;
-        zo[j] = __float2bfloat16_rn(zf);
-      }
+      for (int j = 0; j < QG_DIM; ++j) Z[static_cast<size_t>(i) * QG_DIM + j] = static_cast<float>(a[j]);
     } else {
-#pragma unroll
-      for (int j = 0; j < QG_DIM; ++j) zo[j] = __float2bfloat16_rn(0.f);
       lab[i] = -1;
       pm[i] = -1;
     }
@@ -225,6 +228,24 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_build_kernel(const T* __restri
   for (int c = tid; c <= C; c += QG_THREADS) offs[static_cast<size_t>(bh) * (C + 1) + c] = cstart[c];
   for (int c = tid; c < C; c += QG_THREADS) counts[static_cast<size_t>(bh) * C + c] = cstart[c + 1] - cstart[c];
 
+  // ---- 3b. the bf16 projections in member order (entry m: token pm[m]; zero past n),
+  // so that the per-query scan reads every cluster's tokens as one contiguous run
+  for (int e = tid; e < Ncap * 2; e += QG_THREADS) {
+    const int m = e >> 1, hf = e & 1;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    if (m < n) {
+      const float* zr = Z + static_cast<size_t>(pm[m]) * QG_DIM + 8 * hf;
+      uint32_t w[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const __nv_bfloat162 v = __floats2bfloat162_rn(zr[2 * k], zr[2 * k + 1]);
+        w[k] = *reinterpret_cast<const uint32_t*>(&v);
+      }
+      o = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    reinterpret_cast<uint4*>(z16 + (tok0 + m) * QG_DIM)[hf] = o;
+  }
+
   // ---- 4. cluster statistics, a warp per cluster, lanes over the channels
   constexpr int CPL = D / 32;
   for (int c = warp; c < C; c += QG_NW) {
@@ -261,34 +282,132 @@ __device__ __forceinline__ unsigned long long warp_max_u64(unsigned long long x)
   return x;
 }
 
-// A lane's CPL consecutive channels of a row, as fp32 (one vector load).
-template <typename T, int CPL>
-__device__ __forceinline__ void qg_slice(const T* row, int lane, float (&x)[CPL]) {
+// A lane's CPL consecutive channels of a row as loaded (one vector) -> fp32.
+template <typename T, int CPL, typename R>
+__device__ __forceinline__ void qg_unpack(const R& r, float (&x)[CPL]) {
   if constexpr (sizeof(T) == 2) {
     if constexpr (CPL == 4) {
-      const uint2 r = __ldg(reinterpret_cast<const uint2*>(row) + lane);
       x[0] = __uint_as_float(r.x << 16);
       x[1] = __uint_as_float(r.x & 0xffff0000u);
       x[2] = __uint_as_float(r.y << 16);
       x[3] = __uint_as_float(r.y & 0xffff0000u);
     } else {
-      const uint32_t r = __ldg(reinterpret_cast<const uint32_t*>(row) + lane);
       x[0] = __uint_as_float(r << 16);
       x[1] = __uint_as_float(r & 0xffff0000u);
     }
   } else {
     if constexpr (CPL == 4) {
-      const float4 r = __ldg(reinterpret_cast<const float4*>(row) + lane);
       x[0] = r.x;
       x[1] = r.y;
       x[2] = r.z;
       x[3] = r.w;
     } else {
-      const float2 r = __ldg(reinterpret_cast<const float2*>(row) + lane);
       x[0] = r.x;
       x[1] = r.y;
     }
   }
+}
+
+// D += A B, m16n8k16, bf16 inputs, fp32 accumulation (a: the four A words in
+// fragment order, b0 / b1: the two B words)
+__device__ __forceinline__ void qg_mma_bf16(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// The rc-th largest of the keys of members m0 .. m1 - 1 (distinct 64-bit keys,
+// 1 <= rc < m1 - m0), by one warp: radix selection on 8-bit digits from the highest
+// bit where the keys differ (a histogram of the digit among the keys that match the
+// digits chosen so far; the digit whose range holds the rc-th key is kept), until at
+// most 32 keys match; those are ranked directly. hist: 256 counters, cand: 32 keys,
+// both the warp's own.
+template <typename KeyOf>
+__device__ unsigned long long qg_kth_largest(KeyOf key_of, int m0, int m1, int rc, unsigned* hist,
+                                             unsigned long long* cand, int lane) {
+  unsigned long long a = ~0ull, o = 0ull;
+  for (int m = m0 + lane; m < m1; m += 32) {
+    const unsigned long long x = key_of(m);
+    a &= x;
+    o |= x;
+  }
+  a = (static_cast<unsigned long long>(__reduce_and_sync(FULL_MASK, static_cast<unsigned>(a >> 32))) << 32) |
+      __reduce_and_sync(FULL_MASK, static_cast<unsigned>(a));
+  o = (static_cast<unsigned long long>(__reduce_or_sync(FULL_MASK, static_cast<unsigned>(o >> 32))) << 32) |
+      __reduce_or_sync(FULL_MASK, static_cast<unsigned>(o));
+  const int hb = 63 - __clzll(static_cast<long long>(a ^ o));  // >= 0: at least two distinct keys
+  unsigned long long pmask = hb == 63 ? 0ull : ~((2ull << hb) - 1ull);  // bits above hb: shared
+  unsigned long long prefix = a & pmask;
+  unsigned need = static_cast<unsigned>(rc);  // rank of the threshold among the keys matching prefix
+  for (int top = hb;; top -= 8) {
+    const int lo = top - 7;  // the digit is bits max(lo, 0) .. top
+    const unsigned long long dmask = lo >= 0 ? (255ull << lo) : (255ull >> (-lo));
+    for (int bn = lane; bn < 256; bn += 32) hist[bn] = 0u;
+    __syncwarp();
+    for (int m = m0 + lane; m < m1; m += 32) {
+      const unsigned long long x = key_of(m);
+      if ((x & pmask) == prefix)
+        atomicAdd(hist + static_cast<int>(lo >= 0 ? (x >> lo) & 255ull : (x << (-lo)) & 255ull), 1u);
+    }
+    __syncwarp();
+    // lane L holds bins 255 - 8L - j (j < 8), so lower lanes hold higher digits
+    unsigned cb[8], sum = 0u;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      cb[j] = hist[255 - 8 * lane - j];
+      sum += cb[j];
+    }
+    unsigned incl = sum;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const unsigned v = __shfl_up_sync(FULL_MASK, incl, d);
+      if (lane >= d) incl += v;
+    }
+    const unsigned excl = incl - sum;  // keys in higher digits than this lane's
+    const bool mine = excl < need && need <= incl;
+    const int src = __ffs(__ballot_sync(FULL_MASK, mine)) - 1;
+    unsigned dig = 0u, above = 0u, cdig = 0u;
+    if (mine) {
+      unsigned acc = excl;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (cdig == 0u && acc + cb[j] >= need) {
+          dig = static_cast<unsigned>(255 - 8 * lane - j);
+          above = acc;
+          cdig = cb[j];
+        }
+        acc += cb[j];
+      }
+    }
+    dig = __shfl_sync(FULL_MASK, dig, src);
+    above = __shfl_sync(FULL_MASK, above, src);
+    cdig = __shfl_sync(FULL_MASK, cdig, src);
+    need -= above;
+    prefix |= lo >= 0 ? (static_cast<unsigned long long>(dig) << lo) : (static_cast<unsigned long long>(dig) >> (-lo));
+    pmask |= dmask;
+    if (cdig <= 32u) break;  // always by the last digit: the keys are distinct
+  }
+  // the (at most 32) keys matching prefix, compacted, then ranked
+  int base = 0;
+  for (int m = m0; m < m1; m += 32) {
+    const int mi = m + lane;
+    const unsigned long long x = mi < m1 ? key_of(mi) : 0ull;
+    const bool match = mi < m1 && (x & pmask) == prefix;
+    const unsigned bal = __ballot_sync(FULL_MASK, match);
+    const int slot = base + __popc(bal & ((1u << lane) - 1u));
+    if (match && slot < 32) cand[slot] = x;  // (never more than 32: the keys are distinct)
+    base += __popc(bal);
+  }
+  __syncwarp();
+  base = min(base, 32);
+  const unsigned long long kj = lane < base ? cand[lane] : 0ull;
+  unsigned rank = 0u;
+  for (int i = 0; i < base; ++i) rank += cand[i] > kj;
+  const int win = max(__ffs(__ballot_sync(FULL_MASK, lane < base && rank == need - 1u)) - 1, 0);
+  __syncwarp();  // cand and hist are free again
+  return __shfl_sync(FULL_MASK, kj, win);
 }
 
 struct QgcSel {
@@ -321,13 +440,16 @@ struct QgcSelShared {
   int r[QG_MAX_C], roff[QG_MAX_C + 1];
   float qt[8][QG_DIM];
   float lse[8];
-  float pmx[QG_NW][8], psm[QG_NW][8];
+  float pmx[QS_NW][8], psm[QS_NW][8];
+  alignas(8) unsigned long long rbar[QS_NW][QG_STAGES];
+  unsigned long long cand[QS_NW][32];  // the radix selection's last candidates, per warp
+  unsigned hist[QS_NW][256];           // its digit histogram, per warp
 };
 
 template <typename T, int D, int G>
-__global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) {
+__global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel p) {
   __shared__ QgcSelShared sh;
-  extern __shared__ __align__(16) float qg_ts[];  // token scores, when n <= QG_TCAP
+  extern __shared__ __align__(128) unsigned char qg_ring[];  // the warps' rings, then their score runs
   constexpr int CPL = D / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int bh = blockIdx.x, b = bh / p.Hkv, h = bh - (bh / p.Hkv) * p.Hkv;
@@ -339,7 +461,39 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
   const int32_t* pm = p.perm + static_cast<size_t>(bh) * p.Ncap;
   const T* Kb = static_cast<const T*>(p.K) + static_cast<size_t>(bh) * p.Ncap * D;
   const T* Vb = static_cast<const T*>(p.V) + static_cast<size_t>(bh) * p.Ncap * D;
-  float* t = p.Ncap <= QG_TCAP ? qg_ts : p.tws + static_cast<size_t>(bh) * p.Ncap;
+  float* t = p.tws + static_cast<size_t>(bh) * p.Ncap;  // token scores in member order
+  unsigned char* ring = qg_ring + static_cast<size_t>(warp) * QG_STAGES * QG_CHUNK;
+  uint64_t* rbar = reinterpret_cast<uint64_t*>(sh.rbar[warp]);
+  if (lane == 0) {
+#pragma unroll
+    for (int k = 0; k < QG_STAGES; ++k) mbar_init(rbar + k, 1);
+    fence_mbar_init();
+  }
+  __syncwarp();
+  // The projections stream through the warp's ring: chunk j of warp w is tokens
+  // 128 (w + QS_NW j) .. + 127 in member order, one bulk copy into stage j % QG_STAGES;
+  // both passes take the same chunk sequence (copy u < nmine of pass 1, u - nmine of
+  // pass 2), L2 evict-last in pass 1 (pass 2 reads the bytes again) and evict-first
+  // in pass 2. A lane reads its A words from the stage: token row r at r * 32 bytes,
+  // coordinates 4tq .. 4tq + 3 at + 8 tq (8 rows x 32 bytes a warp load, no conflicts).
+  const unsigned char* zsrc = reinterpret_cast<const unsigned char*>(p.z16) + static_cast<size_t>(bh) * p.Ncap * QG_DIM * 2;
+  const int nck = (n + QG_CHUNK_TOK - 1) / QG_CHUNK_TOK;
+  const int nmine = nck > warp ? (nck - warp + QS_NW - 1) / QS_NW : 0;
+  const uint64_t pol_keep = l2_evict_last_policy(), pol_drop = l2_evict_first_policy();
+  auto issue = [&](int u) {
+    if (u >= 2 * nmine) return;  // warp-uniform
+    const int ck = warp + QS_NW * (u < nmine ? u : u - nmine);
+    const int rows = min(QG_CHUNK_TOK, n - ck * QG_CHUNK_TOK);  // >= 1
+    if (lane == 0) {
+      uint64_t* bar = rbar + u % QG_STAGES;
+      mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * QG_DIM * 2);
+      bulk_g2s(ring + (u % QG_STAGES) * QG_CHUNK, zsrc + static_cast<size_t>(ck) * QG_CHUNK,
+               static_cast<uint32_t>(rows) * QG_DIM * 2, bar, u < nmine ? pol_keep : pol_drop);
+    }
+  };
+  // the first copies go out before the cluster statistics, so their latency overlaps them
+#pragma unroll
+  for (int u = 0; u < QG_STAGES; ++u) issue(u);
 
   // the group's queries, a lane CPL channels of each
   float qf[G][CPL];
@@ -349,7 +503,7 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
     for (int k = 0; k < CPL; ++k) qf[g][k] = load_as_float(qrow + g * D + lane * CPL + k);
 
   // ---- projected queries q~_g = P q_g (warp j: row j of P)
-  for (int j = warp; j < QG_DIM; j += QG_NW) {
+  for (int j = warp; j < QG_DIM; j += QS_NW) {
     float u[CPL];
 #pragma unroll
     for (int k = 0; k < CPL; ++k) u[k] = __ldg(p.P + (static_cast<size_t>(h) * QG_DIM + j) * D + lane * CPL + k);
@@ -364,7 +518,7 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
   }
 
   // ---- per cluster mean logit and logit variance (a warp per cluster)
-  for (int c = warp; c < C; c += QG_NW) {
+  for (int c = warp; c < C; c += QS_NW) {
     const int nc = cnt[c];
     const size_t o = (static_cast<size_t>(bh) * C + c) * D + lane * CPL;
     float mean[CPL], var[CPL];
@@ -439,206 +593,259 @@ __global__ void __launch_bounds__(QG_THREADS) qgc_select_kernel(const QgcSel p) 
   }
   __syncthreads();
 
-  // ---- token scores: LSE per head over the tokens, then t_i (two passes; the next
-  // token's coordinates are loaded before the current one's arithmetic)
+  // ---- token scores in member order: LSE per head over the tokens, then t_m (two
+  // passes over the bf16 projections on the tensor cores). mma.sync m16n8k16: the 16
+  // tokens of a step as M, the 16 coordinates as K, the G <= 8 heads as N. The bf16
+  // projections are exact operands; sigma q~ is split into a bf16 high part and a
+  // bf16 remainder (two products into one fp32 accumulator, about 16 significant
+  // bits of sigma q~). K is taken in the order the A words load: MMA k = 2tq + e is
+  // coordinate 4tq + e and k = 2tq + 8 + e is 4tq + 2 + e (tq = lane % 4), so a lane
+  // reads coordinates 4tq .. 4tq + 3 of its two rows as one 8-byte word pair each.
   {
-    const uint4* zbase = reinterpret_cast<const uint4*>(p.z16 + static_cast<size_t>(bh) * p.Ncap * QG_DIM);
-    auto logits = [&](uint4 a, uint4 bq, float (&sg)[G]) {
-      float z[QG_DIM];
-      float2 f[4];
-      Chunk<__nv_bfloat16>::unpack(a, f);
+    const int gq = lane >> 2, tq = lane & 3;
+    uint32_t bhi[2], blo[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        z[2 * e] = f[e].x;
-        z[2 * e + 1] = f[e].y;
-      }
-      Chunk<__nv_bfloat16>::unpack(bq, f);
+    for (int k = 0; k < 2; ++k) {
+      float v[2];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        z[8 + 2 * e] = f[e].x;
-        z[8 + 2 * e + 1] = f[e].y;
-      }
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float a2 = 0.f;
-#pragma unroll
-        for (int j = 0; j < QG_DIM; ++j) a2 = fmaf(sh.qt[g][j], z[j], a2);
-        sg[g] = a2 * p.sigma;
-      }
+      for (int e = 0; e < 2; ++e) v[e] = gq < G ? p.sigma * sh.qt[gq < G ? gq : 0][4 * tq + 2 * k + e] : 0.f;
+      const __nv_bfloat162 hv = __floats2bfloat162_rn(v[0], v[1]);
+      const float2 hf = __bfloat1622float2(hv);
+      const __nv_bfloat162 lv = __floats2bfloat162_rn(v[0] - hf.x, v[1] - hf.y);
+      bhi[k] = *reinterpret_cast<const uint32_t*>(&hv);
+      blo[k] = *reinterpret_cast<const uint32_t*>(&lv);
+    }
+    // waits for copy u and returns its stage (a bounded wait: a copy that never lands
+    // leaves stale words, never a hang)
+    auto stage_of = [&](int u) {
+      const int k = u % QG_STAGES;
+      if (!mbar_wait(rbar + k, static_cast<uint32_t>((u / QG_STAGES) & 1), nullptr))
+        mbar_wait(rbar + k, static_cast<uint32_t>((u / QG_STAGES) & 1), nullptr);
+      return ring + k * QG_CHUNK;
     };
-    float m[G], l[G];
+    // after the warp's last read of copy u's stage: the copy that refills it
+    auto release = [&](int u) {
+      __syncwarp();
+      fence_proxy_async_smem();
+      issue(u + QG_STAGES);
+    };
+    // the logits of a 16-token step at row offset r16 of a stage: c[0..1] the heads
+    // 2tq, 2tq + 1 of token row r16 + gq, c[2..3] those of row r16 + gq + 8
+    auto step_logits = [&](const unsigned char* stg, int r16, float (&c)[4]) {
+      const uint2 ra = *reinterpret_cast<const uint2*>(stg + (r16 + gq) * 32 + 8 * tq);
+      const uint2 rb = *reinterpret_cast<const uint2*>(stg + (r16 + gq + 8) * 32 + 8 * tq);
+      const uint32_t a[4] = {ra.x, rb.x, ra.y, rb.y};
+      c[0] = c[1] = c[2] = c[3] = 0.f;
+      qg_mma_bf16(c, a, bhi[0], bhi[1]);
+      qg_mma_bf16(c, a, blo[0], blo[1]);
+    };
+    const bool h0 = 2 * tq < G, h1 = 2 * tq + 1 < G;
+    float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
+    for (int j = 0; j < nmine; ++j) {
+      const unsigned char* stg = stage_of(j);
+      const int tok0 = (warp + QS_NW * j) * QG_CHUNK_TOK;
+      const int nst = min(QG_CHUNK_TOK, n - tok0 + 15) >> 4;  // steps with a live row
+#pragma unroll 2
+      for (int k = 0; k < nst; ++k) {
+        const int r0 = tok0 + 16 * k + gq;
+        float c[4];
+        step_logits(stg, 16 * k, c);
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      m[g] = -INFINITY;
-      l[g] = 0.f;
-    }
-    uint4 c0 = make_uint4(0, 0, 0, 0), c1 = c0;
-    if (tid < n) {
-      c0 = __ldg(zbase + 2 * tid);
-      c1 = __ldg(zbase + 2 * tid + 1);
-    }
-    for (int i = tid; i < n; i += QG_THREADS) {
-      const int inx = i + QG_THREADS;
-      uint4 n0 = c0, n1 = c1;
-      if (inx < n) {
-        n0 = __ldg(zbase + 2 * inx);
-        n1 = __ldg(zbase + 2 * inx + 1);
-      }
-      float sg[G];
-      logits(c0, c1, sg);
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        if (sg[g] > m[g]) {
-          l[g] = l[g] * __expf(m[g] - sg[g]) + 1.f;
-          m[g] = sg[g];
-        } else {
-          l[g] += __expf(sg[g] - m[g]);
+        for (int e = 0; e < 2; ++e) {
+          const float va = r0 < n ? c[e] : -INFINITY, vb = r0 + 8 < n ? c[2 + e] : -INFINITY;
+          const float mn = fmaxf(mx[e], fmaxf(va, vb));
+          if (mn != -INFINITY) {
+            sm[e] = sm[e] * __expf(mx[e] - mn) + __expf(va - mn) + __expf(vb - mn);
+            mx[e] = mn;
+          }
         }
       }
-      c0 = n0;
-      c1 = n1;
+      release(j);
     }
+    // combine over the 8 lanes of a head column, then over the warps
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float M = warp_max(m[g]);
-      float L = (m[g] == -INFINITY) ? 0.f : l[g] * __expf(m[g] - M);
-      L = warp_sum(L);
-      if (lane == 0) {
-        sh.pmx[warp][g] = M;
-        sh.psm[warp][g] = L;
+    for (int e = 0; e < 2; ++e) {
+#pragma unroll
+      for (int o = 4; o <= 16; o <<= 1) {
+        const float m2 = __shfl_xor_sync(FULL_MASK, mx[e], o), s2 = __shfl_xor_sync(FULL_MASK, sm[e], o);
+        const float M = fmaxf(mx[e], m2);
+        if (M != -INFINITY) {
+          sm[e] = (mx[e] == -INFINITY ? 0.f : sm[e] * __expf(mx[e] - M)) + (m2 == -INFINITY ? 0.f : s2 * __expf(m2 - M));
+          mx[e] = M;
+        }
+      }
+    }
+    if (gq == 0) {
+      if (h0) {
+        sh.pmx[warp][2 * tq] = mx[0];
+        sh.psm[warp][2 * tq] = sm[0];
+      }
+      if (h1) {
+        sh.pmx[warp][2 * tq + 1] = mx[1];
+        sh.psm[warp][2 * tq + 1] = sm[1];
       }
     }
     __syncthreads();
     if (tid < G) {
       float M = -INFINITY;
-      for (int w = 0; w < QG_NW; ++w) M = fmaxf(M, sh.pmx[w][tid]);
+      for (int w = 0; w < QS_NW; ++w) M = fmaxf(M, sh.pmx[w][tid]);
       float L = 0.f;
       if (M != -INFINITY)
-        for (int w = 0; w < QG_NW; ++w)
+        for (int w = 0; w < QS_NW; ++w)
           if (sh.pmx[w][tid] != -INFINITY) L += sh.psm[w][tid] * __expf(sh.pmx[w][tid] - M);
       sh.lse[tid] = M == -INFINITY ? -INFINITY : M + __logf(L);
     }
     __syncthreads();
-    if (tid < n) {
-      c0 = __ldg(zbase + 2 * tid);
-      c1 = __ldg(zbase + 2 * tid + 1);
-    }
-    for (int i = tid; i < n; i += QG_THREADS) {
-      const int inx = i + QG_THREADS;
-      uint4 n0 = c0, n1 = c1;
-      if (inx < n) {
-        n0 = __ldg(zbase + 2 * inx);
-        n1 = __ldg(zbase + 2 * inx + 1);
+    const float le0 = h0 ? sh.lse[2 * tq] : 0.f, le1 = h1 ? sh.lse[2 * tq + 1] : 0.f;
+    for (int j = 0; j < nmine; ++j) {
+      const unsigned char* stg = stage_of(nmine + j);
+      const int tok0 = (warp + QS_NW * j) * QG_CHUNK_TOK;
+      const int nst = min(QG_CHUNK_TOK, n - tok0 + 15) >> 4;
+#pragma unroll 2
+      for (int k = 0; k < nst; ++k) {
+        const int r0 = tok0 + 16 * k + gq;
+        float c[4];
+        step_logits(stg, 16 * k, c);
+        float ta = (h0 ? __expf(c[0] - le0) : 0.f) + (h1 ? __expf(c[1] - le1) : 0.f);
+        float tb = (h0 ? __expf(c[2] - le0) : 0.f) + (h1 ? __expf(c[3] - le1) : 0.f);
+        ta += __shfl_xor_sync(FULL_MASK, ta, 1);
+        tb += __shfl_xor_sync(FULL_MASK, tb, 1);
+        ta += __shfl_xor_sync(FULL_MASK, ta, 2);
+        tb += __shfl_xor_sync(FULL_MASK, tb, 2);
+        if (tq == 0) {
+          if (r0 < n) t[r0] = ta;
+          if (r0 + 8 < n) t[r0 + 8] = tb;
+        }
       }
-      float sg[G];
-      logits(c0, c1, sg);
-      float tv = 0.f;
-#pragma unroll
-      for (int g = 0; g < G; ++g) tv += __expf(sg[g] - sh.lse[g]);
-      t[i] = tv;
-      c0 = n0;
-      c1 = n1;
+      release(nmine + j);
     }
   }
-  __syncthreads();
+  __syncthreads();  // every score is written; the rings are idle (no copy in flight)
 
-  // ---- per cluster: the r_c largest keys (t's bits, inverted index), the read list,
-  // the read rows' sums and the proxy of the unread tokens (a warp per cluster); the
-  // scores are read through the member list (shared memory for sequences up to
-  // QG_TCAP tokens)
-  auto key_of = [&](int i) {
-    return (static_cast<unsigned long long>(__float_as_uint(t[i])) << 32) |
-           static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(i));
-  };
-  for (int c = warp; c < C; c += QG_NW) {
+  // ---- per cluster: the r_c largest keys (t's bits, inverted member position), the
+  // read list, the read rows' sums and the proxy of the unread tokens (a warp per
+  // cluster). Members are in ascending token order inside a cluster, so the inverted
+  // member position orders ties as the inverted token index does. A cluster's scores
+  // are one contiguous run of the scratch, first copied into the warp's idle ring (up
+  // to QG_RUN scores; longer runs are read from the scratch).
+  constexpr int QG_RUN = QG_STAGES * QG_CHUNK / 4;
+  float* run = reinterpret_cast<float*>(ring);
+  for (int c = warp; c < C; c += QS_NW) {
     const int nc = cnt[c], rc = sh.r[c];
     const int m0 = off[c], m1 = off[c + 1];
-    unsigned long long thr = 0ull;  // keys >= thr are read
-    if (rc > 0 && rc < nc) {
-      if (rc <= 32) {
-        // rc rounds of "largest key below the previous one" (keys are distinct)
-        unsigned long long prev = ~0ull;
-        for (int k = 0; k < rc; ++k) {
-          unsigned long long best = 0ull;
-          for (int m = m0 + lane; m < m1; m += 32) {
-            const unsigned long long x = key_of(pm[m]);
-            if (x < prev && x > best) best = x;
-          }
-          prev = warp_max_u64(best);
-        }
-        thr = prev;
-      } else {
-        unsigned long long prefix = 0ull;
-        for (int bit = 63; bit >= 0; --bit) {
-          const unsigned long long cand = prefix | (1ull << bit);
-          int k = 0;
-          for (int m = m0 + lane; m < m1; m += 32) k += key_of(pm[m]) >= cand;
-          k = __reduce_add_sync(FULL_MASK, k);
-          if (k >= rc) prefix = cand;
-        }
-        thr = prefix;
-      }
+    const float* tc = t + m0;
+    __syncwarp();  // the previous cluster's reads of the run are done
+    // the proxy's cluster sums, needed at the end, requested now
+    const size_t o = (static_cast<size_t>(bh) * C + c) * D + lane * CPL;
+    float ksum[CPL], vsum[CPL];
+#pragma unroll
+    for (int k = 0; k < CPL; ++k) {
+      ksum[k] = __ldg(p.k_sum + o + k);
+      vsum[k] = __ldg(p.v_sum + o + k);
     }
+    if (rc > 0 && rc < nc && nc <= QG_RUN) {
+      // 16 loads a lane in flight per round
+      for (int m = lane; m < nc; m += 32 * 16) {
+        float v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) v[k] = m + 32 * k < nc ? __ldcg(tc + m + 32 * k) : 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+          if (m + 32 * k < nc) run[m + 32 * k] = v[k];
+      }
+      __syncwarp();
+      tc = run;
+    }
+    auto key_of = [&](int m) {
+      return (static_cast<unsigned long long>(__float_as_uint(tc[m - m0])) << 32) |
+             static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(m));
+    };
+    unsigned long long thr = 0ull;  // keys >= thr are read
+    if (rc > 0 && rc < nc) thr = qg_kth_largest(key_of, m0, m1, rc, sh.hist[warp], sh.cand[warp], lane);
     float rk[CPL], rv[CPL];
 #pragma unroll
     for (int k = 0; k < CPL; ++k) rk[k] = rv[k] = 0.f;
-    int pos = sh.roff[c];
+    // the read list of the cluster: the takers' member positions are collected in
+    // the warp's shared list (up to 256 a round; hist is free after the selection),
+    // then turned into token indices with all their loads in flight, then written
+    int* li = reinterpret_cast<int*>(sh.hist[warp]);
+    const int nl = rc > 0 ? min(rc, p.max_read - sh.roff[c]) : 0;
     if (rc > 0) {
-      for (int m = m0; m < m1; m += 32) {
-        const int mi = m + lane;
-        int i = -1;
-        bool take = false;
-        if (mi < m1) {
-          i = pm[mi];
-          take = rc >= nc || key_of(i) >= thr;
+      int32_t* lo_idx = p.tok_idx + static_cast<size_t>(bh) * p.max_read + sh.roff[c];
+      float* lo_w = p.w + static_cast<size_t>(bh) * p.max_read + sh.roff[c];
+      int mb = m0, done = 0;  // members scanned up to mb; list entries written: done
+      while (done < nl) {
+        int cnt_r = 0;  // entries of this round, at most 256
+        for (; mb < m1 && cnt_r < 256 - 32; mb += 32) {
+          const int mi = mb + lane;
+          const bool take = mi < m1 && (rc >= nc || key_of(mi) >= thr);
+          const unsigned bal = __ballot_sync(FULL_MASK, take);
+          if (take) li[cnt_r + __popc(bal & ((1u << lane) - 1u))] = mi;
+          cnt_r += __popc(bal);
         }
-        const unsigned bal = __ballot_sync(FULL_MASK, take);
-        if (take) {
-          const int q = pos + __popc(bal & ((1u << lane) - 1u));
-          if (q < p.max_read) {
-            p.tok_idx[static_cast<size_t>(bh) * p.max_read + q] = i;
-            p.w[static_cast<size_t>(bh) * p.max_read + q] = 1.f;
+        __syncwarp();
+        const int nr = min(cnt_r, nl - done);
+        for (int j0 = 0; j0 < nr; j0 += 32 * 8) {
+          int tk[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + 32 * u + lane;
+            tk[u] = j < nr ? __ldg(pm + li[j]) : 0;
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = j0 + 32 * u + lane;
+            if (j < nr) {
+              li[j] = tk[u];
+              lo_idx[done + j] = tk[u];
+              lo_w[done + j] = 1.f;
+            }
           }
         }
-        pos += __popc(bal);
-      }
-      // the read rows' key and value sums, eight rows' loads in flight
-      __syncwarp();  // the list entries written above are visible to every lane
-      const int32_t* lst = p.tok_idx + static_cast<size_t>(bh) * p.max_read + sh.roff[c];
-      const int nl = min(rc, p.max_read - sh.roff[c]);
-      for (int j0 = 0; j0 < nl; j0 += 8) {
-        float kx[8][CPL], vx[8][CPL];
+        __syncwarp();
+        // the read rows' key and value sums of this round, RW rows' loads in flight
+        using Raw = typename std::conditional<sizeof(T) == 2, typename std::conditional<CPL == 4, uint2, uint32_t>::type,
+                                              typename std::conditional<CPL == 4, float4, float2>::type>::type;
+        constexpr int RW = sizeof(Raw) >= 16 ? 6 : 12;  // 48 registers of rows at most
+        for (int j0 = 0; j0 < nr; j0 += RW) {
+          Raw kr[RW], vr[RW];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          if (j0 + u < nl) {
-            const int ti = lst[j0 + u];
-            qg_slice<T, CPL>(Kb + static_cast<size_t>(ti) * D, lane, kx[u]);
-            qg_slice<T, CPL>(Vb + static_cast<size_t>(ti) * D, lane, vx[u]);
-          } else {
+          for (int u = 0; u < RW; ++u) {
+            if (j0 + u < nr) {
+              const int ti = li[j0 + u];
+              kr[u] = __ldg(reinterpret_cast<const Raw*>(Kb + static_cast<size_t>(ti) * D) + lane);
+              vr[u] = __ldg(reinterpret_cast<const Raw*>(Vb + static_cast<size_t>(ti) * D) + lane);
+            }
+          }
 #pragma unroll
-            for (int k = 0; k < CPL; ++k) kx[u][k] = vx[u][k] = 0.f;
+          for (int u = 0; u < RW; ++u) {
+            if (j0 + u < nr) {
+              float kx[CPL], vx[CPL];
+              qg_unpack<T, CPL>(kr[u], kx);
+              qg_unpack<T, CPL>(vr[u], vx);
+#pragma unroll
+              for (int k = 0; k < CPL; ++k) {
+                rk[k] += kx[k];
+                rv[k] += vx[k];
+              }
+            }
           }
         }
-#pragma unroll
-        for (int u = 0; u < 8; ++u)
-#pragma unroll
-          for (int k = 0; k < CPL; ++k) {
-            rk[k] += kx[u][k];
-            rv[k] += vx[u][k];
-          }
+        __syncwarp();  // li is refilled by the next round
+        done += nr;
+        if (mb >= m1) break;
       }
     }
     const int un = nc - rc;  // unread tokens of the cluster
-    const size_t o = (static_cast<size_t>(bh) * C + c) * D + lane * CPL;
 #pragma unroll
     for (int k = 0; k < CPL; ++k) {
-      p.pk[o + k] = un > 0 ? __fdiv_rn(p.k_sum[o + k] - rk[k], static_cast<float>(un)) : 0.f;
-      p.pv[o + k] = un > 0 ? __fdiv_rn(p.v_sum[o + k] - rv[k], static_cast<float>(un)) : 0.f;
+      p.pk[o + k] = un > 0 ? __fdiv_rn(ksum[k] - rk[k], static_cast<float>(un)) : 0.f;
+      p.pv[o + k] = un > 0 ? __fdiv_rn(vsum[k] - rv[k], static_cast<float>(un)) : 0.f;
     }
     if (lane == 0) p.pn[static_cast<size_t>(bh) * C + c] = max(un, 0);
   }
   // padding of the read list
-  for (int q = sh.roff[C] + tid; q < p.max_read; q += QG_THREADS) {
+  for (int q = sh.roff[C] + tid; q < p.max_read; q += QS_THREADS) {
     p.tok_idx[static_cast<size_t>(bh) * p.max_read + q] = 0;
     p.w[static_cast<size_t>(bh) * p.max_read + q] = 0.f;
   }
@@ -738,8 +945,6 @@ cudaError_t qgc_build_td(const kv_shape* s, const void* K, const void* V, const 
   return cudaGetLastError();
 }
 
-constexpr int QG_KEY_SMEM = kvs::QG_TCAP * 4;
-
 template <typename T, int D>
 cudaError_t qgc_select_td(int G, const kvs::QgcSel& p, int grid, cudaStream_t st) {
   switch (G) {
@@ -750,12 +955,11 @@ cudaError_t qgc_select_td(int G, const kvs::QgcSel& p, int grid, cudaStream_t st
     cudaGetDevice(&dev);                                                                                 \
     if (!(cfg_##GG.load() & (1 << (dev & 31)))) {                                                        \
       const cudaError_t e = cudaFuncSetAttribute(kvs::qgc_select_kernel<T, D, GG>,                       \
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, QG_KEY_SMEM); \
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, kvs::QG_RING); \
       if (e != cudaSuccess) return e;                                                                    \
       cfg_##GG.fetch_or(1 << (dev & 31));                                                                \
     }                                                                                                    \
-    kvs::qgc_select_kernel<T, D, GG><<<grid, kvs::QG_THREADS,                                           \
-                                       p.Ncap <= kvs::QG_TCAP ? p.Ncap * 4 : 0, st>>>(p);                \
+    kvs::qgc_select_kernel<T, D, GG><<<grid, kvs::QS_THREADS, kvs::QG_RING, st>>>(p);                    \
     break;                                                                                               \
   }
     QG_CASE(1) QG_CASE(2) QG_CASE(3) QG_CASE(4) QG_CASE(5) QG_CASE(6) QG_CASE(7) QG_CASE(8)
