@@ -473,13 +473,14 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
   // The projections stream through the warp's ring: chunk j of warp w is tokens
   // 128 (w + QS_NW j) .. + 127 in member order, one bulk copy into stage j % QG_STAGES;
   // both passes take the same chunk sequence (copy u < nmine of pass 1, u - nmine of
-  // pass 2), L2 evict-last in pass 1 (pass 2 reads the bytes again) and evict-first
-  // in pass 2. A lane reads its A words from the stage: token row r at r * 32 bytes,
+  // pass 2). A lane reads its A words from the stage: token row r at r * 32 bytes,
   // coordinates 4tq .. 4tq + 3 at + 8 tq (8 rows x 32 bytes a warp load, no conflicts).
   const unsigned char* zsrc = reinterpret_cast<const unsigned char*>(p.z16) + static_cast<size_t>(bh) * p.Ncap * QG_DIM * 2;
   const int nck = (n + QG_CHUNK_TOK - 1) / QG_CHUNK_TOK;
   const int nmine = nck > warp ? (nck - warp + QS_NW - 1) / QS_NW : 0;
-  const uint64_t pol_keep = l2_evict_last_policy(), pol_drop = l2_evict_first_policy();
+  // evict-first in both passes: keeping a share of pass 1 in L2 for pass 2 (evict-last)
+  // measured no faster
+  const uint64_t pol = l2_evict_first_policy();
   auto issue = [&](int u) {
     if (u >= 2 * nmine) return;  // warp-uniform
     const int ck = warp + QS_NW * (u < nmine ? u : u - nmine);
@@ -488,7 +489,7 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
       uint64_t* bar = rbar + u % QG_STAGES;
       mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * QG_DIM * 2);
       bulk_g2s(ring + (u % QG_STAGES) * QG_CHUNK, zsrc + static_cast<size_t>(ck) * QG_CHUNK,
-               static_cast<uint32_t>(rows) * QG_DIM * 2, bar, u < nmine ? pol_keep : pol_drop);
+               static_cast<uint32_t>(rows) * QG_DIM * 2, bar, pol);
     }
   };
   // the first copies go out before the cluster statistics, so their latency overlaps them
