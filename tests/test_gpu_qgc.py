@@ -137,6 +137,23 @@ def test_qgc_small(D, dtype, G):
     _decode_check(wl, P, qgc, 0.05, pairs, f"qgc decode D={D}")
 
 
+def test_qgc_large_clusters():
+    # two clusters over 9,000 tokens: clusters above the 3,072 scores a warp's idle
+    # ring holds, so the selection reads their scores from the scratch; a ragged
+    # length below a whole 128-token chunk and a 16-token step
+    wl = W.make("llama_cobs_fp4", DEV, B=1, Ncap=9000, seq_lens=[8999])
+    P = _proj(wl)
+    C, iters = 2, 8
+    sl = wl.seq_lens_tensor(DEV)
+    qgc = kv.kv_build_qgc(wl.K, wl.V, sl, P, C, iters)
+    torch.cuda.synchronize()
+    pairs = [(0, h) for h in range(wl.Hkv)]
+    cnt = qgc["counts"].cpu().numpy()
+    assert cnt.max() > 3072
+    _check_build(wl, qgc, P, pairs, C, iters, "qgc build large clusters")
+    _decode_check(wl, P, qgc, 0.05, pairs, "qgc decode large clusters")
+
+
 def test_qgc_edges():
     # an empty sequence, one shorter than the cluster count, a zero budget (proxies
     # only) and one cluster
