@@ -307,3 +307,22 @@ def test_qgc_radix_selection_matches_sort(seed):
             if not 1 <= rc < nc:
                 continue
             assert kth_largest_radix(keys, rc) == sorted(keys, reverse=True)[rc - 1]
+
+
+def test_qgc_inverted_position_and_or_closed_form():
+    # AND and OR of 2^32 - 1 - m over m0 <= m < m1, as the selection forms them
+    import random
+    rng = random.Random(5)
+    M = 0xFFFFFFFF
+    for _ in range(300):
+        m0 = rng.randrange(0, 1 << 20)
+        m1 = m0 + rng.choice([2, 3, 31, 32, 33, 1000, rng.randrange(2, 5000)])
+        lo_v, hi_v = M - (m1 - 1), M - m0
+        dv = lo_v ^ hi_v
+        lmask = 0 if dv == 0 else (M >> (32 - dv.bit_length()))
+        a = o = None
+        for m in range(m0, m1):
+            v = M - m
+            a = v if a is None else a & v
+            o = v if o is None else o | v
+        assert (lo_v & ~lmask & M) == a and (lo_v | lmask) == o

@@ -322,21 +322,12 @@ __device__ __forceinline__ void qg_mma_bf16(float (&d)[4], const uint32_t (&a)[4
 // 1 <= rc < m1 - m0), by one warp: radix selection on 8-bit digits from the highest
 // bit where the keys differ (a histogram of the digit among the keys that match the
 // digits chosen so far; the digit whose range holds the rc-th key is kept), until at
-// most 32 keys match; those are ranked directly. hist: 256 counters, cand: 32 keys,
-// both the warp's own.
+// most 32 keys match; those are ranked directly. a, o: the AND and the OR of all the
+// keys (the same in every lane). hist: 256 counters, cand: 32 keys, both the warp's own.
 template <typename KeyOf>
-__device__ unsigned long long qg_kth_largest(KeyOf key_of, int m0, int m1, int rc, unsigned* hist,
-                                             unsigned long long* cand, int lane) {
-  unsigned long long a = ~0ull, o = 0ull;
-  for (int m = m0 + lane; m < m1; m += 32) {
-    const unsigned long long x = key_of(m);
-    a &= x;
-    o |= x;
-  }
-  a = (static_cast<unsigned long long>(__reduce_and_sync(FULL_MASK, static_cast<unsigned>(a >> 32))) << 32) |
-      __reduce_and_sync(FULL_MASK, static_cast<unsigned>(a));
-  o = (static_cast<unsigned long long>(__reduce_or_sync(FULL_MASK, static_cast<unsigned>(o >> 32))) << 32) |
-      __reduce_or_sync(FULL_MASK, static_cast<unsigned>(o));
+__device__ unsigned long long qg_kth_largest(KeyOf key_of, int m0, int m1, int rc, unsigned long long a,
+                                             unsigned long long o, unsigned* hist, unsigned long long* cand,
+                                             int lane) {
   const int hb = 63 - __clzll(static_cast<long long>(a ^ o));  // >= 0: at least two distinct keys
   unsigned long long pmask = hb == 63 ? 0ull : ~((2ull << hb) - 1ull);  // bits above hb: shared
   unsigned long long prefix = a & pmask;
@@ -735,6 +726,7 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
     const int nc = cnt[c], rc = sh.r[c];
     const int m0 = off[c], m1 = off[c + 1];
     const float* tc = t + m0;
+    unsigned tand = ~0u, tor = 0u;  // AND and OR of the cluster's score bits
     __syncwarp();  // the previous cluster's reads of the run are done
     // the proxy's cluster sums, needed at the end, requested now
     const size_t o = (static_cast<size_t>(bh) * C + c) * D + lane * CPL;
@@ -745,24 +737,44 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
       vsum[k] = __ldg(p.v_sum + o + k);
     }
     if (rc > 0 && rc < nc && nc <= QG_RUN) {
-      // 16 loads a lane in flight per round
+      // 16 loads a lane in flight per round; the AND and OR of the score bits on the way
       for (int m = lane; m < nc; m += 32 * 16) {
         float v[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) v[k] = m + 32 * k < nc ? __ldcg(tc + m + 32 * k) : 0.f;
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          if (m + 32 * k < nc) run[m + 32 * k] = v[k];
+          if (m + 32 * k < nc) {
+            run[m + 32 * k] = v[k];
+            tand &= __float_as_uint(v[k]);
+            tor |= __float_as_uint(v[k]);
+          }
       }
       __syncwarp();
       tc = run;
+    } else if (rc > 0 && rc < nc) {
+      for (int m = lane; m < nc; m += 32) {
+        tand &= __float_as_uint(tc[m]);
+        tor |= __float_as_uint(tc[m]);
+      }
     }
     auto key_of = [&](int m) {
       return (static_cast<unsigned long long>(__float_as_uint(tc[m - m0])) << 32) |
              static_cast<unsigned long long>(0xffffffffu - static_cast<uint32_t>(m));
     };
     unsigned long long thr = 0ull;  // keys >= thr are read
-    if (rc > 0 && rc < nc) thr = qg_kth_largest(key_of, m0, m1, rc, sh.hist[warp], sh.cand[warp], lane);
+    if (rc > 0 && rc < nc) {
+      // AND and OR of the keys: the score bits' from the lanes; the inverted positions
+      // are the contiguous range [2^32 - m1, 2^32 - 1 - m0], whose AND and OR are its
+      // common high bits followed by zeros and by ones
+      const unsigned ha = __reduce_and_sync(FULL_MASK, tand), ho = __reduce_or_sync(FULL_MASK, tor);
+      const unsigned lo_v = 0xffffffffu - static_cast<uint32_t>(m1 - 1), hi_v = 0xffffffffu - static_cast<uint32_t>(m0);
+      const unsigned dv = lo_v ^ hi_v;
+      const unsigned lmask = dv == 0u ? 0u : (0xffffffffu >> __clz(dv));
+      const unsigned long long ka = (static_cast<unsigned long long>(ha) << 32) | (lo_v & ~lmask);
+      const unsigned long long ko = (static_cast<unsigned long long>(ho) << 32) | (lo_v | lmask);
+      thr = qg_kth_largest(key_of, m0, m1, rc, ka, ko, sh.hist[warp], sh.cand[warp], lane);
+    }
     float rk[CPL], rv[CPL];
 #pragma unroll
     for (int k = 0; k < CPL; ++k) rk[k] = rv[k] = 0.f;
