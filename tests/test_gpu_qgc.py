@@ -111,10 +111,20 @@ def _decode_check(wl, P, qgc, budget, pairs, what):
     return out, lse, sel
 
 
-@pytest.mark.parametrize("D,dtype,G", [(128, torch.bfloat16, 4), (64, torch.float32, 2)])
+@pytest.mark.parametrize("D,dtype,G", [(128, torch.bfloat16, 4), (64, torch.float32, 2), (128, torch.bfloat16, 7)])
 def test_qgc_small(D, dtype, G):
-    if D == 128:
+    if D == 128 and G == 4:
         wl = W.make("llama_cobs_fp4", DEV, B=2, Ncap=3000, seq_lens=[3000, 1234])
+        P = _proj(wl)
+    elif D == 128:
+        # G = 7 (the Qwen-shaped group) on a bf16 cache from the same recipe: the
+        # selection's two-product path for G > 4
+        wl = W.make("llama_cobs_fp4", DEV, B=2, Ncap=2500, seq_lens=[2500, 777])
+        gq = torch.Generator(device=DEV).manual_seed(4)
+        wl.Hkv, wl.Hq = 2, 14
+        wl.K = wl.K[:, :2].contiguous()
+        wl.V = wl.V[:, :2].contiguous()
+        wl.q = (torch.randn(2, 14, 128, generator=gq, device=DEV) * 1.5).to(torch.bfloat16)
         P = _proj(wl)
     else:
         gq = torch.Generator(device=DEV).manual_seed(2)

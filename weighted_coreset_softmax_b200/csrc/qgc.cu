@@ -593,18 +593,24 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
   // bits of sigma q~). K is taken in the order the A words load: MMA k = 2tq + e is
   // coordinate 4tq + e and k = 2tq + 8 + e is 4tq + 2 + e (tq = lane % 4), so a lane
   // reads coordinates 4tq .. 4tq + 3 of its two rows as one 8-byte word pair each.
+  // With G <= 4 one product does both parts: B's columns 0..3 are the heads' high
+  // parts and 4..7 their remainders, so lanes tq and tq + 2 hold the two parts of the
+  // same heads; one exchange adds them, lane tq < 2 keeping row gq and lane tq >= 2 row
+  // gq + 8, and each lane then has one row's logits for heads 2 (tq % 2) and + 1.
   {
+    constexpr bool PK = G <= 4;
     const int gq = lane >> 2, tq = lane & 3;
     uint32_t bhi[2], blo[2];
 #pragma unroll
     for (int k = 0; k < 2; ++k) {
+      const int hd = PK ? (gq & 3) : gq;  // the head of B column gq
       float v[2];
 #pragma unroll
-      for (int e = 0; e < 2; ++e) v[e] = gq < G ? p.sigma * sh.qt[gq < G ? gq : 0][4 * tq + 2 * k + e] : 0.f;
+      for (int e = 0; e < 2; ++e) v[e] = hd < G ? p.sigma * sh.qt[hd < G ? hd : 0][4 * tq + 2 * k + e] : 0.f;
       const __nv_bfloat162 hv = __floats2bfloat162_rn(v[0], v[1]);
       const float2 hf = __bfloat1622float2(hv);
       const __nv_bfloat162 lv = __floats2bfloat162_rn(v[0] - hf.x, v[1] - hf.y);
-      bhi[k] = *reinterpret_cast<const uint32_t*>(&hv);
+      bhi[k] = *reinterpret_cast<const uint32_t*>(PK && gq >= 4 ? &lv : &hv);
       blo[k] = *reinterpret_cast<const uint32_t*>(&lv);
     }
     // waits for copy u and returns its stage (a bounded wait: a copy that never lands
@@ -629,9 +635,20 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
       const uint32_t a[4] = {ra.x, rb.x, ra.y, rb.y};
       c[0] = c[1] = c[2] = c[3] = 0.f;
       qg_mma_bf16(c, a, bhi[0], bhi[1]);
-      qg_mma_bf16(c, a, blo[0], blo[1]);
+      if constexpr (!PK) qg_mma_bf16(c, a, blo[0], blo[1]);
     };
-    const bool h0 = 2 * tq < G, h1 = 2 * tq + 1 < G;
+    // G <= 4: this lane's row (r16 + gq, + 8 when tq >= 2) and its two logits
+    const int prow = tq >= 2 ? gq + 8 : gq;
+    auto step_pair = [&](const unsigned char* stg, int r16, float (&v)[2]) {
+      float c[4];
+      step_logits(stg, r16, c);
+      const float x0 = tq < 2 ? c[2] : c[0], x1 = tq < 2 ? c[3] : c[1];
+      const float y0 = __shfl_xor_sync(FULL_MASK, x0, 2), y1 = __shfl_xor_sync(FULL_MASK, x1, 2);
+      v[0] = tq < 2 ? c[0] + y0 : y0 + c[2];
+      v[1] = tq < 2 ? c[1] + y1 : y1 + c[3];
+    };
+    const int hb = PK ? 2 * (tq & 1) : 2 * tq;  // this lane's heads: hb, hb + 1
+    const bool h0 = hb < G, h1 = hb + 1 < G;
     float mx[2] = {-INFINITY, -INFINITY}, sm[2] = {0.f, 0.f};
     for (int j = 0; j < nmine; ++j) {
       const unsigned char* stg = stage_of(j);
@@ -639,26 +656,46 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
       const int nst = min(QG_CHUNK_TOK, n - tok0 + 15) >> 4;  // steps with a live row
 #pragma unroll 2
       for (int k = 0; k < nst; ++k) {
-        const int r0 = tok0 + 16 * k + gq;
-        float c[4];
-        step_logits(stg, 16 * k, c);
+        if constexpr (PK) {
+          // one value a head: the smaller of (running max, value) minus the larger,
+          // one exponential, and the running sum rescaled when the value is larger
+          const int r = tok0 + 16 * k + prow;
+          float v[2];
+          step_pair(stg, 16 * k, v);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const float va = r0 < n ? c[e] : -INFINITY, vb = r0 + 8 < n ? c[2 + e] : -INFINITY;
-          const float mn = fmaxf(mx[e], fmaxf(va, vb));
-          if (mn != -INFINITY) {
-            sm[e] = sm[e] * __expf(mx[e] - mn) + __expf(va - mn) + __expf(vb - mn);
-            mx[e] = mn;
+          for (int e = 0; e < 2; ++e) {
+            const float x = r < n ? v[e] : -INFINITY;
+            const float mn = fmaxf(mx[e], x);
+            if (mn != -INFINITY) {
+              const float ex = __expf(fminf(mx[e], x) - mn);
+              sm[e] = x > mx[e] ? fmaf(sm[e], ex, 1.f) : sm[e] + ex;
+              mx[e] = mn;
+            }
+          }
+        } else {
+          const int r0 = tok0 + 16 * k + gq;
+          float c[4];
+          step_logits(stg, 16 * k, c);
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float va = r0 < n ? c[e] : -INFINITY, vb = r0 + 8 < n ? c[2 + e] : -INFINITY;
+            const float mn = fmaxf(mx[e], fmaxf(va, vb));
+            if (mn != -INFINITY) {
+              sm[e] = sm[e] * __expf(mx[e] - mn) + __expf(va - mn) + __expf(vb - mn);
+              mx[e] = mn;
+            }
           }
         }
       }
       release(j);
     }
-    // combine over the 8 lanes of a head column, then over the warps
+    // combine over the lanes of a head column (and, with G <= 4, of both row halves),
+    // then over the warps
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
 #pragma unroll
-      for (int o = 4; o <= 16; o <<= 1) {
+      for (int o = PK ? 2 : 4; o <= 16; o <<= 1) {
+        if (o == 2 && !PK) continue;
         const float m2 = __shfl_xor_sync(FULL_MASK, mx[e], o), s2 = __shfl_xor_sync(FULL_MASK, sm[e], o);
         const float M = fmaxf(mx[e], m2);
         if (M != -INFINITY) {
@@ -667,14 +704,14 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
         }
       }
     }
-    if (gq == 0) {
+    if (gq == 0 && (!PK || tq < 2)) {
       if (h0) {
-        sh.pmx[warp][2 * tq] = mx[0];
-        sh.psm[warp][2 * tq] = sm[0];
+        sh.pmx[warp][hb] = mx[0];
+        sh.psm[warp][hb] = sm[0];
       }
       if (h1) {
-        sh.pmx[warp][2 * tq + 1] = mx[1];
-        sh.psm[warp][2 * tq + 1] = sm[1];
+        sh.pmx[warp][hb + 1] = mx[1];
+        sh.psm[warp][hb + 1] = sm[1];
       }
     }
     __syncthreads();
@@ -688,13 +725,23 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
       sh.lse[tid] = M == -INFINITY ? -INFINITY : M + __logf(L);
     }
     __syncthreads();
-    const float le0 = h0 ? sh.lse[2 * tq] : 0.f, le1 = h1 ? sh.lse[2 * tq + 1] : 0.f;
+    const float le0 = h0 ? sh.lse[hb] : 0.f, le1 = h1 ? sh.lse[hb + 1] : 0.f;
     for (int j = 0; j < nmine; ++j) {
       const unsigned char* stg = stage_of(nmine + j);
       const int tok0 = (warp + QS_NW * j) * QG_CHUNK_TOK;
       const int nst = min(QG_CHUNK_TOK, n - tok0 + 15) >> 4;
 #pragma unroll 2
       for (int k = 0; k < nst; ++k) {
+        if constexpr (PK) {
+          // the lanes tq, tq ^ 1 hold the same row's heads 0, 1 and 2, 3
+          const int r = tok0 + 16 * k + prow;
+          float v[2];
+          step_pair(stg, 16 * k, v);
+          float ta = (h0 ? __expf(v[0] - le0) : 0.f) + (h1 ? __expf(v[1] - le1) : 0.f);
+          ta += __shfl_xor_sync(FULL_MASK, ta, 1);
+          if ((tq & 1) == 0 && r < n) t[r] = ta;
+          continue;
+        }
         const int r0 = tok0 + 16 * k + gq;
         float c[4];
         step_logits(stg, 16 * k, c);
