@@ -494,46 +494,71 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
 #pragma unroll
     for (int k = 0; k < CPL; ++k) qf[g][k] = load_as_float(qrow + g * D + lane * CPL + k);
 
-  // ---- projected queries q~_g = P q_g (warp j: row j of P)
-  for (int j = warp; j < QG_DIM; j += QS_NW) {
-    float u[CPL];
+  // ---- projected queries q~_g = P q_g (warp w: rows w, w + QS_NW of P, both loaded
+  // before the first use)
+  static_assert(QG_DIM == 2 * QS_NW, "two projection rows a warp");
+  {
+    float u[2][CPL];
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) u[k] = __ldg(p.P + (static_cast<size_t>(h) * QG_DIM + j) * D + lane * CPL + k);
+    for (int r = 0; r < 2; ++r)
 #pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float v = 0.f;
+      for (int k = 0; k < CPL; ++k)
+        u[r][k] = __ldg(p.P + (static_cast<size_t>(h) * QG_DIM + warp + r * QS_NW) * D + lane * CPL + k);
 #pragma unroll
-      for (int k = 0; k < CPL; ++k) v = fmaf(u[k], qf[g][k], v);
-      v = warp_sum(v);
-      if (lane == 0) sh.qt[g][j] = v;
-    }
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float v = 0.f;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) v = fmaf(u[r][k], qf[g][k], v);
+        v = warp_sum(v);
+        if (lane == 0) sh.qt[g][warp + r * QS_NW] = v;
+      }
   }
 
-  // ---- per cluster mean logit and logit variance (a warp per cluster)
-  for (int c = warp; c < C; c += QS_NW) {
-    const int nc = cnt[c];
-    const size_t o = (static_cast<size_t>(bh) * C + c) * D + lane * CPL;
-    float mean[CPL], var[CPL];
+  // ---- per cluster mean logit and logit variance (a warp per cluster; a warp's
+  // clusters four at a time, their cached tokens all requested before the first use)
+  for (int c0 = warp; c0 < C; c0 += 4 * QS_NW) {
+    float ksr[4][CPL], kqr[4][CPL];
+    int ncr[4];
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) {
-      const float m = nc > 0 ? __fdiv_rn(p.k_sum[o + k], static_cast<float>(nc)) : 0.f;
-      const float sq = nc > 0 ? __fdiv_rn(p.k_sq[o + k], static_cast<float>(nc)) : 0.f;
-      mean[k] = m;
-      var[k] = fmaxf(sq - m * m, 0.f);
-    }
-#pragma unroll
-    for (int g = 0; g < G; ++g) {
-      float a = 0.f, v = 0.f;
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * QS_NW;
+      const size_t o = (static_cast<size_t>(bh) * C + (c < C ? c : 0)) * D + lane * CPL;
+      ncr[u] = c < C ? __ldg(cnt + c) : 0;
 #pragma unroll
       for (int k = 0; k < CPL; ++k) {
-        a = fmaf(qf[g][k], mean[k], a);
-        v = fmaf(qf[g][k] * qf[g][k], var[k], v);
+        ksr[u][k] = c < C ? __ldg(p.k_sum + o + k) : 0.f;
+        kqr[u][k] = c < C ? __ldg(p.k_sq + o + k) : 0.f;
       }
-      a = warp_sum(a);
-      v = warp_sum(v);
-      if (lane == 0) {
-        sh.mu[g][c] = nc > 0 ? p.sigma * a : -INFINITY;
-        sh.s2[g][c] = nc > 0 ? p.sigma * p.sigma * v : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + u * QS_NW;
+      if (c >= C) break;  // warp-uniform
+      const int nc = ncr[u];
+      float mean[CPL], var[CPL];
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) {
+        const float m = nc > 0 ? __fdiv_rn(ksr[u][k], static_cast<float>(nc)) : 0.f;
+        const float sq = nc > 0 ? __fdiv_rn(kqr[u][k], static_cast<float>(nc)) : 0.f;
+        mean[k] = m;
+        var[k] = fmaxf(sq - m * m, 0.f);
+      }
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float a = 0.f, v = 0.f;
+#pragma unroll
+        for (int k = 0; k < CPL; ++k) {
+          a = fmaf(qf[g][k], mean[k], a);
+          v = fmaf(qf[g][k] * qf[g][k], var[k], v);
+        }
+        a = warp_sum(a);
+        v = warp_sum(v);
+        if (lane == 0) {
+          sh.mu[g][c] = nc > 0 ? p.sigma * a : -INFINITY;
+          sh.s2[g][c] = nc > 0 ? p.sigma * p.sigma * v : 0.f;
+        }
       }
     }
   }
@@ -678,11 +703,15 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
           step_logits(stg, 16 * k, c);
 #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const float va = r0 < n ? c[e] : -INFINITY, vb = r0 + 8 < n ? c[2 + e] : -INFINITY;
-            const float mn = fmaxf(mx[e], fmaxf(va, vb));
-            if (mn != -INFINITY) {
-              sm[e] = sm[e] * __expf(mx[e] - mn) + __expf(va - mn) + __expf(vb - mn);
-              mx[e] = mn;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {  // rows r0, r0 + 8: one exponential each
+              const float x = r0 + 8 * hf < n ? c[2 * hf + e] : -INFINITY;
+              const float mn = fmaxf(mx[e], x);
+              if (mn != -INFINITY) {
+                const float ex = __expf(fminf(mx[e], x) - mn);
+                sm[e] = x > mx[e] ? fmaf(sm[e], ex, 1.f) : sm[e] + ex;
+                mx[e] = mn;
+              }
             }
           }
         }
