@@ -960,18 +960,33 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
   float qf[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) qf[k] = load_as_float(q + static_cast<size_t>(row) * D + lane * CPL + k);
+  // proxy logits eight at a time: all eight rows' loads first, then one transpose
+  // reduction leaves proxy c0 + j's dot product in the lanes with (lane >> 2) == j
   float M = lse[row];
-  for (int c = 0; c < C; ++c) {
-    const int nc = pn[bh * C + c];
-    float a = 0.f;
-    if (nc > 0) {
+  for (int c0 = 0; c0 < C; c0 += 8) {
+    float part[8];
+    int ncs[8];
 #pragma unroll
-      for (int k = 0; k < CPL; ++k) a = fmaf(qf[k], pk[(bh * C + c) * D + lane * CPL + k], a);
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + j;
+      ncs[j] = c < C ? pn[bh * C + c] : 0;
+      float kv[CPL];
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) kv[k] = c < C ? pk[(bh * C + c) * D + lane * CPL + k] : 0.f;
+      float a = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) a = fmaf(qf[k], kv[k], a);
+      part[j] = a;
     }
-    a = warp_sum(a);
-    const float lc = nc > 0 ? sigma * a + __logf(static_cast<float>(nc)) : -INFINITY;
-    if (lane == 0) lgs[warp][c] = lc;
-    M = fmaxf(M, lc);
+    transpose_reduce<8, 16>(part, lane);
+    const int j = (lane >> 2) & 7;
+    int nc = ncs[0];
+#pragma unroll
+    for (int jj = 1; jj < 8; ++jj)
+      if (jj == j) nc = ncs[jj];
+    const float lc = (c0 + j < C && nc > 0) ? sigma * part[0] + __logf(static_cast<float>(nc)) : -INFINITY;
+    if ((lane & 3) == 0 && c0 + j < C) lgs[warp][c0 + j] = lc;
+    M = fmaxf(M, warp_max(lc));
   }
   __syncwarp();
   if (M == -INFINITY) return;  // nothing read and no proxy (an empty sequence)
@@ -981,13 +996,23 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
   float o[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) o[k] = a0 * out[static_cast<size_t>(row) * D + lane * CPL + k];
-  for (int c = 0; c < C; ++c) {
-    const float lc = lgs[warp][c];
-    if (lc == -INFINITY) continue;
-    const float e = __expf(lc - M);
-    den += e;
+  // the proxies' values eight at a time, all eight rows' loads first
+  for (int c0 = 0; c0 < C; c0 += 8) {
+    float vv[8][CPL], e[8];
 #pragma unroll
-    for (int k = 0; k < CPL; ++k) o[k] = fmaf(e, pv[(bh * C + c) * D + lane * CPL + k], o[k]);
+    for (int j = 0; j < 8; ++j) {
+      const int c = c0 + j;
+      const float lc = c < C ? lgs[warp][c] : -INFINITY;
+      e[j] = lc == -INFINITY ? 0.f : __expf(lc - M);
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) vv[j][k] = lc != -INFINITY ? pv[(bh * C + c) * D + lane * CPL + k] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      den += e[j];
+#pragma unroll
+      for (int k = 0; k < CPL; ++k) o[k] = fmaf(e[j], vv[j][k], o[k]);
+    }
   }
 #pragma unroll
   for (int k = 0; k < CPL; ++k) out[static_cast<size_t>(row) * D + lane * CPL + k] = o[k] / den;
