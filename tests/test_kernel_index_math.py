@@ -329,9 +329,9 @@ def test_qgc_inverted_position_and_or_closed_form():
 
 
 def test_qgc_merge_transpose_lanes():
-    # the proxy merge reduces eight proxies' partial dots with the 8-value transpose
-    # starting at lane mask 16: lane l then holds proxy (l >> 2) % 8's whole dot
-    part = [[1000.0 * k + lane for k in range(8)] for lane in range(32)]
-    out = transpose_reduce(part, 8, 16)
+    # the proxy merge reduces sixteen proxies' partial dots with the 16-value transpose
+    # starting at lane mask 16: lane l then holds proxy (l >> 1) % 16's whole dot
+    part = [[1000.0 * k + lane for k in range(16)] for lane in range(32)]
+    out = transpose_reduce(part, 16, 16)
     for lane in range(32):
-        assert out[lane] == 32 * 1000.0 * ((lane >> 2) & 7) + sum(range(32))
+        assert out[lane] == 32 * 1000.0 * ((lane >> 1) & 15) + sum(range(32))

@@ -941,7 +941,7 @@ __global__ void __launch_bounds__(QS_THREADS, 2) qgc_select_kernel(const QgcSel 
 }
 
 // Folds the proxies into the attention over the read tokens: a warp per query head,
-// lanes over the channels. With the read tokens' (out, lse) and proxy logits
+// lanes over the channels, sixteen proxies at a time. With the read tokens' (out, lse) and proxy logits
 // l_c = sigma q . pk_c + ln pn_c (pn_c > 0): M = max(lse, l_c),
 // out = (e^(lse - M) out + sum_c e^(l_c - M) pv_c) / (e^(lse - M) + sum_c e^(l_c - M)).
 template <typename T, int D>
@@ -960,14 +960,15 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
   float qf[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) qf[k] = load_as_float(q + static_cast<size_t>(row) * D + lane * CPL + k);
-  // proxy logits eight at a time: all eight rows' loads first, then one transpose
-  // reduction leaves proxy c0 + j's dot product in the lanes with (lane >> 2) == j
+  // proxy logits sixteen at a time: all sixteen rows' loads first, then one transpose
+  // reduction leaves proxy c0 + j's dot product in the lanes with (lane >> 1) == j
+  constexpr int PB = 16;
   float M = lse[row];
-  for (int c0 = 0; c0 < C; c0 += 8) {
-    float part[8];
-    int ncs[8];
+  for (int c0 = 0; c0 < C; c0 += PB) {
+    float part[PB];
+    int ncs[PB];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < PB; ++j) {
       const int c = c0 + j;
       ncs[j] = c < C ? pn[bh * C + c] : 0;
       float kv[CPL];
@@ -978,14 +979,14 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
       for (int k = 0; k < CPL; ++k) a = fmaf(qf[k], kv[k], a);
       part[j] = a;
     }
-    transpose_reduce<8, 16>(part, lane);
-    const int j = (lane >> 2) & 7;
+    transpose_reduce<PB, 16>(part, lane);
+    const int j = (lane >> 1) & (PB - 1);
     int nc = ncs[0];
 #pragma unroll
-    for (int jj = 1; jj < 8; ++jj)
+    for (int jj = 1; jj < PB; ++jj)
       if (jj == j) nc = ncs[jj];
     const float lc = (c0 + j < C && nc > 0) ? sigma * part[0] + __logf(static_cast<float>(nc)) : -INFINITY;
-    if ((lane & 3) == 0 && c0 + j < C) lgs[warp][c0 + j] = lc;
+    if ((lane & 1) == 0 && c0 + j < C) lgs[warp][c0 + j] = lc;
     M = fmaxf(M, warp_max(lc));
   }
   __syncwarp();
@@ -996,11 +997,11 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
   float o[CPL];
 #pragma unroll
   for (int k = 0; k < CPL; ++k) o[k] = a0 * out[static_cast<size_t>(row) * D + lane * CPL + k];
-  // the proxies' values eight at a time, all eight rows' loads first
-  for (int c0 = 0; c0 < C; c0 += 8) {
-    float vv[8][CPL], e[8];
+  // the proxies' values sixteen at a time, all sixteen rows' loads first
+  for (int c0 = 0; c0 < C; c0 += PB) {
+    float vv[PB][CPL], e[PB];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < PB; ++j) {
       const int c = c0 + j;
       const float lc = c < C ? lgs[warp][c] : -INFINITY;
       e[j] = lc == -INFINITY ? 0.f : __expf(lc - M);
@@ -1008,7 +1009,7 @@ __global__ void __launch_bounds__(256) qgc_merge_kernel(const T* __restrict__ q,
       for (int k = 0; k < CPL; ++k) vv[j][k] = lc != -INFINITY ? pv[(bh * C + c) * D + lane * CPL + k] : 0.f;
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < PB; ++j) {
       den += e[j];
 #pragma unroll
       for (int k = 0; k < CPL; ++k) o[k] = fmaf(e[j], vv[j][k], o[k]);
