@@ -111,7 +111,8 @@ def _decode_check(wl, P, qgc, budget, pairs, what):
     return out, lse, sel
 
 
-@pytest.mark.parametrize("D,dtype,G", [(128, torch.bfloat16, 4), (64, torch.float32, 2), (128, torch.bfloat16, 7)])
+@pytest.mark.parametrize("D,dtype,G", [(128, torch.bfloat16, 4), (64, torch.float32, 2), (64, torch.bfloat16, 2),
+                                       (128, torch.bfloat16, 7)])
 def test_qgc_small(D, dtype, G):
     if D == 128 and G == 4:
         wl = W.make("llama_cobs_fp4", DEV, B=2, Ncap=3000, seq_lens=[3000, 1234])
@@ -129,12 +130,12 @@ def test_qgc_small(D, dtype, G):
     else:
         gq = torch.Generator(device=DEV).manual_seed(2)
         wl = W.make("llama_cobs_fp4", DEV, B=2, Ncap=2000, seq_lens=[2000, 333])
-        # a D = 64 fp32 cache with G = 2 from the same recipe's shapes
+        # a D = 64 cache (fp32 or bf16) with G = 2 from the same recipe's shapes
         wl.D, wl.Hq, wl.Hkv = 64, 4, 2
-        wl.K = torch.randn(2, 2, 2000, 64, generator=gq, device=DEV) * torch.exp(
-            0.5 * torch.randn(2, 2, 1, 64, generator=gq, device=DEV))
-        wl.V = torch.randn(2, 2, 2000, 64, generator=gq, device=DEV)
-        wl.q = torch.randn(2, 4, 64, generator=gq, device=DEV)
+        wl.K = (torch.randn(2, 2, 2000, 64, generator=gq, device=DEV) * torch.exp(
+            0.5 * torch.randn(2, 2, 1, 64, generator=gq, device=DEV))).to(dtype)
+        wl.V = torch.randn(2, 2, 2000, 64, generator=gq, device=DEV).to(dtype)
+        wl.q = torch.randn(2, 4, 64, generator=gq, device=DEV).to(dtype)
         wl.scale = 1 / math.sqrt(64)
         Rm = torch.linalg.qr(torch.randn(64, 64, generator=torch.Generator().manual_seed(3), dtype=torch.float64))[0]
         P = Rm[:, :16].T.contiguous().float().to(DEV).unsqueeze(0).expand(2, 16, 64).contiguous()
